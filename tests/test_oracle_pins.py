@@ -1,0 +1,377 @@
+"""Pins for the float64 oracle against what the ELSAA paper and plain mathematics fix.
+
+Each test checks the oracle against something other than itself: a library
+routine the special case reduces to, brute force over subsets, the explicit
+kernel-sum definition of RACE, closed-form identities, the hard-hash collision
+limit, a value printed in the paper, and central finite differences.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import elsaa_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def _params(N, d, T, k, r, causal, **kw):
+    return orc.Params(N=N, d=d, block_size=T, topk=k, rank_r=r, causal=causal,
+                      scale=1.0 / math.sqrt(d), **kw)
+
+
+# --- dense attention is the exact special case [ELSAA §3 dense definition] ---
+
+def test_full_support_no_lowrank_is_dense_softmax():
+    N, d = 40, 16
+    q, k, v = _rand((N, d), 1), _rand((N, d), 2), _rand((N, d), 3)
+    p = _params(N, d, 1, N, 0, False, eps=0.0)
+    out = orc.forward_head(q, k, v, np.zeros((0, d, 4)), p)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[None], torch.tensor(k)[None], torch.tensor(v)[None], scale=p.scale)[0].numpy()
+    np.testing.assert_allclose(out["O"], ref, rtol=0, atol=1e-12)
+    assert np.all(out["m"] == 1.0)
+
+
+def test_causal_all_blocks_no_lowrank_is_causal_softmax():
+    N, d, T = 56, 8, 8            # 7 tiles, k >= 7 selects every eligible block
+    q, k, v = _rand((N, d), 4), _rand((N, d), 5), _rand((N, d), 6)
+    p = _params(N, d, T, 7, 0, True, eps=0.0)
+    out = orc.forward_head(q, k, v, np.zeros((0, d, 4)), p)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[None], torch.tensor(k)[None], torch.tensor(v)[None],
+        scale=p.scale, is_causal=True)[0].numpy()
+    np.testing.assert_allclose(out["O"], ref, rtol=0, atol=1e-12)
+
+
+def test_ragged_tail_all_blocks_is_dense_softmax():
+    N, d, T = 45, 8, 8            # last tile/block has 5 rows
+    q, k, v = _rand((N, d), 7), _rand((N, d), 8), _rand((N, d), 9)
+    for causal in (False, True):
+        p = _params(N, d, T, 6, 0, causal, eps=0.0)
+        out = orc.forward_head(q, k, v, np.zeros((0, d, 4)), p)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.tensor(q)[None], torch.tensor(k)[None], torch.tensor(v)[None],
+            scale=p.scale, is_causal=causal)[0].numpy()
+        np.testing.assert_allclose(out["O"], ref, rtol=0, atol=1e-12)
+
+
+# --- selection: brute force over subsets ---
+
+def test_topk_keys_maximise_selected_mass_bruteforce():
+    """Block size 1: the k selected keys maximise sum_j e^{z_ij} over all k-subsets,
+    and O_s is the softmax restricted to the best subset."""
+    N, d = 12, 5
+    q, k, v = _rand((N, d), 10), _rand((N, d), 11), _rand((N, d), 12)
+    for kk in range(1, N + 1):
+        p = _params(N, d, 1, kk, 0, False)
+        out = orc.forward_head(q, k, v, np.zeros((0, d, 4)), p)
+        for i in range(N):
+            z = p.scale * (k @ q[i])
+            best, best_set = -1.0, None
+            for sub in itertools.combinations(range(N), kk):
+                mass = np.exp(z[list(sub)]).sum()
+                if mass > best:
+                    best, best_set = mass, sub
+            assert tuple(out["idx"][i]) == best_set
+            w = np.exp(z[list(best_set)])
+            np.testing.assert_allclose(out["O_s"][i], w @ v[list(best_set)] / w.sum(), atol=1e-12)
+            np.testing.assert_allclose(np.exp(out["logd_s"][i]), w.sum(), rtol=1e-12)
+
+
+def test_causal_topk_keys_bruteforce_on_16_keys():
+    N, d = 16, 4
+    q, k, v = _rand((N, d), 13), _rand((N, d), 14), _rand((N, d), 15)
+    for kk in (1, 3, 6):
+        p = _params(N, d, 1, kk, 0, True)
+        out = orc.forward_head(q, k, v, np.zeros((0, d, 4)), p)
+        for i in range(N):
+            z = p.scale * (k[:i + 1] @ q[i])
+            # the diagonal (key i) is forced; the rest maximise the mass among keys < i
+            best, best_set = -1.0, None
+            for sub in itertools.combinations(range(i), min(kk - 1, i)):
+                mass = np.exp(z[list(sub)]).sum()
+                if mass > best:
+                    best, best_set = mass, sub
+            chosen = sorted(set(best_set) | {i})
+            got = [b for b in out["idx"][i] if b >= 0]
+            assert got == chosen
+            w = np.exp(z[chosen])
+            np.testing.assert_allclose(out["O_s"][i], w @ v[chosen] / w.sum(), atol=1e-12)
+
+
+def test_block_selection_is_best_subset_of_block_scores():
+    """Blocks of 2 on 16 keys: the selected blocks maximise the summed block score
+    (the arg-top-k), found by enumerating every subset of blocks."""
+    N, d, T = 16, 6, 2
+    q, k = _rand((N, d), 16), _rand((N, d), 17)
+    nb = N // T
+    for causal in (False, True):
+        for kk in (1, 2, 3, 5):
+            p = _params(N, d, T, kk, 0, causal)
+            out = orc.forward_head(q, k, _rand((N, d), 18), np.zeros((0, d, 4)), p)
+            qbar = q.reshape(nb, T, d).mean(1)
+            kbar = k.reshape(nb, T, d).mean(1)
+            for t in range(nb):
+                s = [p.scale * qbar[t] @ kbar[b] for b in range(nb)]
+                elig = list(range(t + 1)) if causal else list(range(nb))
+                size = min(kk, len(elig))
+                best, best_set = -np.inf, None
+                for sub in itertools.combinations(elig, size):
+                    if causal and t not in sub:
+                        continue
+                    tot = sum(s[b] for b in sub if not (causal and b == t))
+                    if tot > best:
+                        best, best_set = tot, sub
+                got = [b for b in out["idx"][t] if b >= 0]
+                assert got == sorted(best_set)
+
+
+def test_select_from_scores_ties_and_forced_diagonal():
+    s = np.array([[0.5, 0.5, 0.5, 0.5],
+                  [1.0, 2.0, 2.0, 0.0],
+                  [3.0, 3.0, -9.0, 1.0],
+                  [0.0, 0.0, 0.0, -5.0]])
+    nc = orc.select_from_scores(s, 2, False)
+    assert nc.tolist() == [[0, 1], [1, 2], [0, 1], [0, 1]]
+    c = orc.select_from_scores(s, 2, True)
+    # tile 0: only block 0; tile 2: diagonal 2 forced despite -9, plus best of {0, 1} (tie -> 0)
+    assert c.tolist() == [[0, -1], [0, 1], [0, 2], [0, 3]]
+    c3 = orc.select_from_scores(s, 3, True)
+    assert c3.tolist() == [[0, -1, -1], [0, 1, -1], [0, 1, 2], [0, 1, 3]]
+
+
+# --- RACE: the linear-time summary form equals the kernel-sum definition ---
+
+def _race_definition(q, k, v, W, p):
+    """Brute force: kappa(q_i, k_j) = (1/L) sum_l sum_c P_l(c|q_i) P_l(c|k_j), per pair."""
+    N, d = q.shape
+    Pq, _, _ = orc.race_bucket_probs(q, W, p)
+    Pk, _, _ = orc.race_bucket_probs(k, W, p)
+    L = p.n_tables
+    O = np.zeros((N, d))
+    dl = np.zeros(N)
+    for i in range(N):
+        num = np.zeros(d)
+        den = 0.0
+        for j in range(N):
+            if p.causal and j > i:
+                continue
+            kap = 0.0
+            for l in range(L):
+                for c in range(1 << p.hash_bits):
+                    kap += Pq[i, l, c] * Pk[j, l, c]
+            kap /= L
+            num += kap * v[j]
+            den += kap
+        O[i] = num / den
+        dl[i] = den
+    return O, dl
+
+
+@pytest.mark.parametrize("causal,chunk", [(False, None), (True, 1), (True, 3), (True, 8), (True, 29)])
+def test_race_summary_form_equals_definition(causal, chunk):
+    N, d, r = 29, 6, 32
+    q, k, v = _rand((N, d), 20), _rand((N, d), 21), _rand((N, d), 22)
+    W = _rand((r // 16, d, 4), 23)
+    p = _params(N, d, 4, 1, r, causal, chunk=chunk)
+    O, dl = orc.race_branch(q, k, v, W, p)
+    Oref, dlref = _race_definition(q, k, v, W, p)
+    np.testing.assert_allclose(dl, dlref, rtol=1e-12)
+    np.testing.assert_allclose(O, Oref, atol=1e-12)
+    rows = [0, 5, 28]
+    Or, dr = orc.race_rows(q, k, v, W, p, rows)
+    np.testing.assert_allclose(dr, dlref[rows], rtol=1e-12)
+    np.testing.assert_allclose(Or, Oref[rows], atol=1e-12)
+
+
+def test_bucket_probabilities_sum_to_one_and_factorise():
+    """softmax over corners of <c,h>/tau == prod_b sigmoid(2 c_b h_b / tau)."""
+    d, L, gamma = 7, 3, 4
+    X = _rand((50, d), 24, 3.0)
+    W = _rand((L, d, gamma), 25)
+    for tau in (1.0, 0.3, 2.5):
+        p = orc.Params(N=50, d=d, block_size=1, topk=1, rank_r=L << gamma, causal=False,
+                       scale=1.0, tau=tau)
+        P, u, n = orc.race_bucket_probs(X, W, p)
+        np.testing.assert_allclose(P.sum(axis=2), 1.0, atol=1e-14)
+        np.testing.assert_allclose(np.linalg.norm(u, axis=1), 1.0, atol=1e-14)
+        for l in range(L):
+            h = u @ W[l]
+            for c in range(1 << gamma):
+                sign = np.array([1.0 if (c >> b) & 1 else -1.0 for b in range(gamma)])
+                prod = np.prod(1.0 / (1.0 + np.exp(-2.0 * sign * h / tau)), axis=1)
+                np.testing.assert_allclose(P[:, l, c], prod, rtol=1e-12)
+
+
+def test_hard_hash_limit_is_collision_count():
+    """tau -> 0: kappa(q, k) -> (1/L) #{tables where sign(W_l^T q) == sign(W_l^T k)}."""
+    N, d, L = 30, 8, 5
+    q, k = _rand((N, d), 26), _rand((N, d), 27)
+    W = _rand((L, d, 4), 28)
+    p = orc.Params(N=N, d=d, block_size=1, topk=1, rank_r=L * 16, causal=False, scale=1.0, tau=1e-9)
+    kap = orc.race_features(q, W, p) @ orc.race_features(k, W, p).T
+    count = np.zeros((N, N))
+    for l in range(L):
+        sq = np.sign(q @ W[l])
+        sk = np.sign(k @ W[l])
+        count += np.all(sq[:, None, :] == sk[None, :, :], axis=2)
+    np.testing.assert_allclose(kap * L, count, atol=1e-9)
+    assert set(np.round(kap * L).astype(int).ravel()) <= set(range(L + 1))
+
+
+# --- fusion [Eq. 5, Eq. 4] ---
+
+def _setup(N=48, d=8, T=8, k=2, r=32, causal=True, seed=30, **kw):
+    q, k_, v = _rand((N, d), seed), _rand((N, d), seed + 1), _rand((N, d), seed + 2)
+    W = _rand((r // 16, d, 4), seed + 3)
+    return q, k_, v, W, _params(N, d, T, k, r, causal, **kw)
+
+
+def test_default_gates_give_convex_combination_of_values():
+    """With g_s = 1, g_lr = 1 - m every output row is sum_j w_ij v_j with w >= 0 and
+    sum_j w_ij = 1; the weights are rebuilt entry by entry from the definitions."""
+    for causal in (True, False):
+        q, k, v, W, p = _setup(causal=causal, N=40, T=8, k=2)
+        out = orc.forward_head(q, k, v, W, p)
+        N = p.N
+        Pq, _, _ = orc.race_bucket_probs(q, W, p)
+        Pk, _, _ = orc.race_bucket_probs(k, W, p)
+        sup = orc.support(out["idx"], p)
+        for i in range(N):
+            z = {j: p.scale * q[i] @ k[j] for j in sup[i]}
+            ds = sum(math.exp(x) for x in z.values())
+            J = range(i + 1) if causal else range(N)
+            kap = {j: float((Pq[i] * Pk[j]).sum() / p.n_tables) for j in J}
+            dl = sum(kap.values())
+            m = ds / (ds + p.lam * dl + p.eps)
+            w = np.zeros(N)
+            for j, x in z.items():
+                w[j] += m * math.exp(x) / ds
+            for j, x in kap.items():
+                w[j] += (1 - m) * x / dl
+            assert np.all(w >= 0)
+            assert abs(w.sum() - 1.0) < 1e-12
+            np.testing.assert_allclose(out["O"][i], w @ v, atol=1e-12)
+            assert abs(out["m"][i] - m) < 1e-12
+
+
+def test_fusion_equals_joint_normalisation():
+    """Default gates: O = (d_s O_s + (lam d_lr + eps) O_lr) / (d_s + lam d_lr + eps)."""
+    q, k, v, W, p = _setup(lam=0.7, eps=0.25)
+    out = orc.forward_head(q, k, v, W, p)
+    ds = np.exp(out["logd_s"])
+    c = p.lam * out["d_lr"] + p.eps
+    ref = (ds[:, None] * out["O_s"] + c[:, None] * out["O_lr"]) / (ds + c)[:, None]
+    np.testing.assert_allclose(out["O"], ref, atol=1e-12)
+
+
+def test_branch_switches():
+    q, k, v, W, p = _setup()
+    # k = 0: no sparse support, m = 0, O = O_lr
+    p0 = _params(p.N, p.d, p.block_size, 0, p.rank_r, True)
+    out = orc.forward_head(q, k, v, W, p0)
+    assert np.all(out["m"] == 0) and np.all(np.isneginf(out["logd_s"]))
+    O_lr, _ = orc.race_branch(q, k, v, W, p0)
+    np.testing.assert_allclose(out["O"], O_lr, atol=1e-14)
+    # r = 0, eps = 0: O = O_s exactly
+    p1 = _params(p.N, p.d, p.block_size, 2, 0, True, eps=0.0)
+    out = orc.forward_head(q, k, v, W, p1)
+    np.testing.assert_allclose(out["O"], out["O_s"], atol=1e-14)
+    # lam -> large: m -> 0; explicit gates are used as given
+    p2 = _params(p.N, p.d, p.block_size, 2, p.rank_r, True, lam=1e30)
+    out = orc.forward_head(q, k, v, W, p2)
+    assert np.all(out["m"] < 1e-20)
+    gs, gl = np.full(p.N, 0.3), np.full(p.N, 2.0)
+    o3 = orc.forward_head(q, k, v, W, p, g_s=gs, g_lr=gl)
+    np.testing.assert_allclose(o3["O"], 0.3 * o3["m"][:, None] * o3["O_s"] + 2.0 * o3["O_lr"], atol=1e-12)
+
+
+def test_equivariance_over_batch_and_heads():
+    Bn, Hn, N, d, r = 2, 3, 32, 8, 16
+    rng = np.random.default_rng(40)
+    Q, K, V = (rng.standard_normal((Bn, Hn, N, d)) for _ in range(3))
+    dO = rng.standard_normal((Bn, Hn, N, d))
+    W = rng.standard_normal((1, d, 4))
+    p = _params(N, d, 8, 2, r, True)
+    fw = orc.forward(Q, K, V, W, p)
+    g = orc.backward(Q, K, V, W, dO, fw, p)
+    perm = rng.permutation(Bn * Hn)
+    P = lambda x: x.reshape((Bn * Hn,) + x.shape[2:])[perm].reshape(x.shape)
+    fw2 = orc.forward(P(Q), P(K), P(V), W, p)
+    g2 = orc.backward(P(Q), P(K), P(V), W, P(dO), fw2, p)
+    np.testing.assert_allclose(fw2["O"], P(fw["O"]), atol=1e-13)
+    for a, b in zip(g2, g):
+        np.testing.assert_allclose(a, P(b), atol=1e-12)
+
+
+def test_key_permutation_invariance_noncausal_block1():
+    N, d, r = 24, 6, 16
+    q, k, v = _rand((N, d), 41), _rand((N, d), 42), _rand((N, d), 43)
+    W = _rand((1, d, 4), 44)
+    p = _params(N, d, 1, 5, r, False)
+    out = orc.forward_head(q, k, v, W, p)
+    perm = np.random.default_rng(45).permutation(N)
+    out2 = orc.forward_head(q, k[perm], v[perm], W, p)
+    np.testing.assert_allclose(out2["O"], out["O"], atol=1e-12)
+
+
+# --- backward: central finite differences ---
+
+def _loss(q, k, v, W, p, dO, lam=None, g_s=None, g_lr=None):
+    out = orc.forward_head(q, k, v, W, p, lam, g_s, g_lr)
+    return float((out["O"] * dO).sum()), out["idx"]
+
+
+@pytest.mark.parametrize("causal,gates,r,k,tau", [(True, False, 32, 2, 1.0), (False, False, 16, 2, 0.6),
+                                                  (True, True, 16, 3, 1.7), (True, False, 0, 2, 1.0),
+                                                  (True, False, 32, 0, 0.8)])
+def test_backward_matches_finite_differences(causal, gates, r, k, tau):
+    N, d, T = 24, 6, 4
+    q, k_, v, W, p = _setup(N=N, d=d, T=T, k=k, r=r, causal=causal, seed=50, lam=0.8, tau=tau)
+    if r == 0:
+        W = np.zeros((0, d, 4))
+    dO = _rand((N, d), 60)
+    lam = np.linspace(0.5, 1.5, N)
+    g_s = np.linspace(0.2, 1.0, N) if gates else None
+    g_lr = np.linspace(1.0, 0.1, N) if gates else None
+    fw = orc.forward_head(q, k_, v, W, p, lam, g_s, g_lr)
+    dq, dk, dv = orc.backward_head(q, k_, v, W, dO, fw, p, lam, g_s, g_lr)
+    h = 1e-6
+    skipped = 0
+    for X, G in ((q, dq), (k_, dk), (v, dv)):
+        fd = np.zeros_like(X)
+        for idx in np.ndindex(X.shape):
+            old = X[idx]
+            X[idx] = old + h
+            lp, ip = _loss(q, k_, v, W, p, dO, lam, g_s, g_lr)
+            X[idx] = old - h
+            lm, im = _loss(q, k_, v, W, p, dO, lam, g_s, g_lr)
+            X[idx] = old
+            if not (np.array_equal(ip, fw["idx"]) and np.array_equal(im, fw["idx"])):
+                skipped += 1
+                fd[idx] = G[idx]
+                continue
+            fd[idx] = (lp - lm) / (2 * h)
+        scale = np.abs(G).max()
+        assert np.abs(fd - G).max() <= 1e-6 * max(scale, 1.0)
+        assert np.linalg.norm(fd - G) <= 1e-6 * np.linalg.norm(G) + 1e-9
+    assert skipped <= 3
+
+
+# --- a value printed in the paper ---
+
+def test_interaction_count_matches_paper_example():
+    with open(os.path.join(GOLDEN, "interaction_count.json")) as f:
+        g = json.load(f)
+    a = g["args"]
+    assert orc.interaction_count(a["N"], a["s"], a["L_s"], a["gamma"]) == g["elsaa_interactions"]
+    assert a["N"] ** 2 == g["dense_interactions"]
