@@ -1,0 +1,153 @@
+/*
+ * elsaa.h — C ABI of libelsaa.so: the ELSAA attention operator (sparse top-k
+ * block branch + RACE low-rank branch + denominator-aware fusion), forward and
+ * backward, on one NVIDIA B200 (sm_100a).
+ *
+ * Source of every definition: the paper page "ELSAA: Efficient Low-Rank and
+ * Sparse Attention Approximation for Training Transformers" (arXiv 2607.20214):
+ *   - dense per-head attention and the per-head procedure ........ §3
+ *   - low-rank branch: RACE soft hash-bucket summaries, normalised
+ *     ratio form giving O_lr and d_lr; causal chunked prefix ...... §3.1
+ *   - sparse branch: exact attention over a selected support,
+ *     returning O_sparse and d_sparse .............................. §3.2, §3.3 Practical notes
+ *   - fusion weight m = d_s / (d_s + lambda d_lr + eps) ............ §3.3, Eq. 5
+ *   - output O = g_s m O_s + g_lr O_lr ............................. §1, Eq. 4
+ *   - sketch size S_R = L 2^gamma (so r = L * 2^gamma) ............. §6
+ * Readings this library takes where the page is silent:
+ *   - selector: top-k key blocks per query tile (block size T = queries per
+ *     tile = keys per block), block score = scale * mean(Q_tile) . mean(K_block),
+ *     ties to the lower block index; causal: the diagonal block is always
+ *     selected, then the best k-1 earlier blocks, keys j > i masked;
+ *   - RACE features: u = x / max(|x|, 1e-12), h_l = W_l^T u, bucket
+ *     probabilities p_l(c|x) = softmax over corners c in {-1,1}^gamma of
+ *     <c, h_l> / tau, Phi(x) = [p_l(c|x) / sqrt(L)];
+ *     kappa(q, k) = Phi(q) . Phi(k); O_lr,i = sum_j kappa v_j / d_lr,i over
+ *     all keys (j <= i when causal), d_lr,i = sum_j kappa;
+ *   - default gates g_s = 1, g_lr = 1 - m; gradients flow to Q, K, V only
+ *     (selection, W_hash, lambda and the gates are constants).
+ *
+ * Conventions shared by every entry point:
+ *   - Ownership: the caller owns every buffer and stream.  The library never
+ *     allocates or frees device memory and keeps no state between calls.
+ *   - Pointers: all tensor pointers are DEVICE pointers, 16-byte aligned,
+ *     except where a function says otherwise.
+ *   - Layout: Q, K, V, O, dO, dQ, dK, dV are contiguous row-major [B, H, N, d]
+ *     in the element type given by params->dtype (float32 or bfloat16).
+ *     W_hash is float32 [L, d, gamma] (L = rank_r >> hash_bits), shared by all
+ *     batches and heads.  lambda_vec, g_sparse, g_lr are float32 [B, H, N] or
+ *     NULL (NULL: scalar params->lambda; g_s = 1; g_lr = 1 - m).
+ *   - Streams: calls are asynchronous on `stream` (a cudaStream_t, may be 0).
+ *     They do not synchronise, except elsaa_check_device_flags.
+ *   - Errors: invalid arguments return before any launch with
+ *     ELSAA_ERR_INVALID_ARG / ELSAA_ERR_UNSUPPORTED / ELSAA_ERR_WORKSPACE;
+ *     a failed launch returns ELSAA_ERR_CUDA.  elsaa_last_error_message()
+ *     returns a one-line description of the last failure on this thread.
+ *   - Supported: N >= 1 (a last tile shorter than block_size is allowed);
+ *     d in {64, 128}; hash_bits == 4; rank_r a multiple of 16 with
+ *     0 <= rank_r <= 256; 0 <= topk <= ceil(N / block_size) <= 1024.
+ *     bfloat16: block_size in {64, 128}.  float32: block_size in {1, 64, 128}
+ *     (block_size 1 only with N <= 4096).
+ */
+#ifndef ELSAA_H_
+#define ELSAA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ELSAA_API __attribute__((visibility("default")))
+#else
+#define ELSAA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ELSAA_OK = 0,
+  ELSAA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned buffer */
+  ELSAA_ERR_UNSUPPORTED = 2,   /* valid operator, shape outside the supported set */
+  ELSAA_ERR_WORKSPACE = 3,     /* workspace or saved buffer smaller than required */
+  ELSAA_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+  ELSAA_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up (see elsaa_check_device_flags) */
+} elsaa_status;
+
+typedef enum { ELSAA_DTYPE_F32 = 0, ELSAA_DTYPE_BF16 = 1 } elsaa_dtype;
+
+typedef struct {
+  int32_t B, H, N, d;     /* batch, heads, sequence length, head dimension */
+  int32_t dtype;          /* elsaa_dtype of Q, K, V, O, dO, dQ, dK, dV */
+  int32_t causal;         /* 0 or 1 */
+  int32_t rank_r;         /* r = L * 2^hash_bits RACE features; 0 disables the low-rank branch */
+  int32_t hash_bits;      /* gamma: bits per RACE table (4) */
+  int32_t block_size;     /* T: queries per tile = keys per block */
+  int32_t topk;           /* k: key blocks selected per query tile; 0 disables the sparse branch */
+  float scale;            /* logit scale, normally 1/sqrt(d) */
+  float lambda;           /* Eq. 5 lambda when lambda_vec == NULL */
+  float eps;              /* Eq. 5 epsilon (>= 0) */
+  float tau;              /* RACE soft-assignment temperature (> 0) */
+} elsaa_params;
+
+/* Bytes of the caller-owned `saved` buffer the forward fills and the backward
+ * reads (selection, per-row denominators, the fusion weight, O_sparse, RACE
+ * features and prefix summaries).  Returns 0 when params are invalid. */
+ELSAA_API size_t elsaa_saved_bytes(const elsaa_params* params);
+
+/* Bytes of scratch device memory a forward (for_backward = 0) or backward
+ * (for_backward = 1) call needs.  Returns 0 when params are invalid. */
+ELSAA_API size_t elsaa_workspace_bytes(const elsaa_params* params, int for_backward);
+
+/* Forward: O = g_s m O_s + g_lr O_lr for every (b, h) [Eq. 4, Eq. 5, §3.1, §3.2].
+ *   Q, K, V      in   [B,H,N,d] dtype
+ *   W_hash       in   float32 [L, d, hash_bits]
+ *   lambda_vec, g_sparse, g_lr  in  float32 [B,H,N] or NULL
+ *   O            out  [B,H,N,d] dtype
+ *   saved        out  elsaa_saved_bytes() bytes, consumed by elsaa_backward
+ *   workspace    scratch, elsaa_workspace_bytes(params, 0) bytes */
+ELSAA_API elsaa_status elsaa_forward(const elsaa_params* params,
+                           const void* Q, const void* K, const void* V,
+                           const float* W_hash, const float* lambda_vec,
+                           const float* g_sparse, const float* g_lr,
+                           void* O, void* saved,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward: exact gradients of sum(dO * O) with respect to Q, K and V through
+ * Eq. 4, Eq. 5, the sparse softmax and the RACE features, given the `saved`
+ * buffer of the forward call with the same params and inputs.
+ *   dO           in   [B,H,N,d] dtype
+ *   dQ, dK, dV   out  [B,H,N,d] dtype (overwritten)
+ *   workspace    scratch, elsaa_workspace_bytes(params, 1) bytes */
+ELSAA_API elsaa_status elsaa_backward(const elsaa_params* params,
+                            const void* Q, const void* K, const void* V,
+                            const float* W_hash, const float* lambda_vec,
+                            const float* g_sparse, const float* g_lr,
+                            const void* dO, const void* saved,
+                            void* dQ, void* dK, void* dV,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Selection only: the float32 block scores the selector ranks and the chosen
+ * blocks, for checking the selector against an external implementation.
+ *   scores  out  float32 [B, H, n_t, n_t]  (n_t = ceil(N / block_size)); every
+ *                entry is written, including blocks a causal tile may not select
+ *   idx     out  int32 [B, H, n_t, topk], ascending block order, -1 padding
+ *   workspace    scratch, elsaa_workspace_bytes(params, 0) bytes */
+ELSAA_API elsaa_status elsaa_debug_select(const elsaa_params* params, const void* Q, const void* K,
+                                float* scores, int32_t* idx,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error flag kept at
+ * the start of `workspace`.  Returns ELSAA_ERR_TIMEOUT if a kernel gave up a
+ * bounded wait since the last check, else ELSAA_OK (or ELSAA_ERR_CUDA). */
+ELSAA_API elsaa_status elsaa_check_device_flags(void* workspace, void* stream);
+
+/* Static English name of a status code. */
+ELSAA_API const char* elsaa_status_string(elsaa_status status);
+
+/* One-line description of the last failed call on this thread ("" if none). */
+ELSAA_API const char* elsaa_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ELSAA_H_ */

@@ -440,6 +440,98 @@ def backward(Q, K, V, W, dO, fw, p: Params, lam=None, g_s=None, g_lr=None):
 
 
 # ----------------------------------------------------------------------------
+# Row-sampled forms for large problems: the same definitions evaluated only for
+# chosen query rows (forward, dq) or key rows (dk, dv).
+# ----------------------------------------------------------------------------
+
+def forward_rows_head(q, k, v, W, p: Params, rows, lam=None, g_s=None, g_lr=None, scores=None):
+    """Forward quantities for the query rows ``rows`` only (per-row definitions)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    rows = np.asarray(rows)
+    sc = block_scores(q, k, p) if scores is None else _f64(scores)
+    idx = select_from_scores(sc, p.topk, p.causal)
+    n, d = rows.size, q.shape[1]
+    O_s = np.zeros((n, d))
+    logd = np.full(n, -np.inf)
+    for a, i in enumerate(rows):
+        keys = _tile_keys(idx[i // p.block_size], p)
+        if p.causal:
+            keys = keys[keys <= i]
+        if keys.size == 0:
+            continue
+        z = p.scale * (k[keys] @ q[i])
+        mx = z.max()
+        e = np.exp(z - mx)
+        O_s[a] = e @ v[keys] / e.sum()
+        logd[a] = mx + np.log(e.sum())
+    O_lr, d_lr = race_rows(q, k, v, W, p, rows)
+    sub = lambda x: None if x is None else _f64(x)[rows]
+    O, m = fuse(O_s, logd, O_lr, d_lr, p, sub(lam), sub(g_s), sub(g_lr))
+    return dict(O=O, O_s=O_s, logd_s=logd, O_lr=O_lr, d_lr=d_lr, m=m, idx=idx, scores=sc)
+
+
+def backward_rows_head(q, k, v, W, dO, fw, p: Params, qrows, krows, lam=None, g_s=None, g_lr=None):
+    """dq for query rows ``qrows`` and (dk, dv) for key rows ``krows``.
+
+    ``fw`` is the full forward dict of the head (every row's denominators are
+    needed for dk, dv).  Same chain rule as ``backward_head``, row by row.
+    """
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    N, d = q.shape
+    T = p.block_size
+    dOs, dOlr, dds_ds, ddlr = _fusion_adjoints(dO, fw, p, lam, g_s, g_lr)
+    Delta = (dOs * fw["O_s"]).sum(axis=1) - dds_ds
+    idx = fw["idx"]
+    qrows, krows = np.asarray(qrows), np.asarray(krows)
+    dq = np.zeros((qrows.size, d))
+    dk = np.zeros((krows.size, d))
+    dv = np.zeros((krows.size, d))
+    for a, i in enumerate(qrows):
+        keys = _tile_keys(idx[i // T], p)
+        if p.causal:
+            keys = keys[keys <= i]
+        if keys.size:
+            P = np.exp(p.scale * (k[keys] @ q[i]) - fw["logd_s"][i])
+            dz = P * (v[keys] @ dOs[i] - Delta[i])
+            dq[a] += p.scale * dz @ k[keys]
+    for a, j in enumerate(krows):
+        b = j // T
+        for t in range(p.n_tiles):
+            if b not in idx[t]:
+                continue
+            I = np.arange(t * T, min(N, (t + 1) * T))
+            if p.causal:
+                I = I[I >= j]
+            if I.size == 0:
+                continue
+            P = np.exp(p.scale * (q[I] @ k[j]) - fw["logd_s"][I])
+            dz = P * (dOs[I] @ v[j] - Delta[I])
+            dk[a] += p.scale * dz @ q[I]
+            dv[a] += P @ dOs[I]
+    if p.rank_r:
+        d_lr = fw["d_lr"]
+        dN = dOlr / d_lr[:, None]
+        delta = ddlr - (dOlr * fw["O_lr"]).sum(axis=1) / d_lr
+        PhiQ = race_features(q, W, p)
+        PhiK = race_features(k, W, p)
+        dPhiQ = np.zeros((qrows.size, p.rank_r))
+        for a, i in enumerate(qrows):
+            J = np.arange(i + 1) if p.causal else np.arange(N)
+            dkap = v[J] @ dN[i] + delta[i]
+            dPhiQ[a] = dkap @ PhiK[J]
+        dq += race_features_backward(q[qrows], W, p, dPhiQ)
+        dPhiK = np.zeros((krows.size, p.rank_r))
+        for a, j in enumerate(krows):
+            I = np.arange(j, N) if p.causal else np.arange(N)
+            kap = PhiQ[I] @ PhiK[j]
+            dkap = dN[I] @ v[j] + delta[I]
+            dv[a] += kap @ dN[I]
+            dPhiK[a] = dkap @ PhiQ[I]
+        dk += race_features_backward(k[krows], W, p, dPhiK)
+    return dq, dk, dv
+
+
+# ----------------------------------------------------------------------------
 # Complexity accounting [ELSAA §6 and the appendix interaction-count example]
 # ----------------------------------------------------------------------------
 

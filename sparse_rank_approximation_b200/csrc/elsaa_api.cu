@@ -1,0 +1,362 @@
+// C ABI of libelsaa.so: argument validation, the layout of the caller-owned
+// `saved` and `workspace` buffers, and the launch sequence of the forward and
+// backward passes.  The operator is defined in include/elsaa.h.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/elsaa.h"
+#include "kernels.h"
+
+using namespace elsaa;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+elsaa_status fail(elsaa_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+elsaa_status fail(elsaa_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+// Sequential sub-allocator over a caller buffer (or a null base to measure).
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    off = align_up(off);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
+  *st = ELSAA_OK;
+  if (!p) { *st = fail(ELSAA_ERR_INVALID_ARG, "params is NULL"); return false; }
+  if (p->B < 1 || p->H < 1 || p->N < 1) {
+    *st = fail(ELSAA_ERR_INVALID_ARG, "B, H, N must be >= 1 (got %d, %d, %d)", p->B, p->H, p->N);
+    return false;
+  }
+  if (p->dtype != ELSAA_DTYPE_F32 && p->dtype != ELSAA_DTYPE_BF16) {
+    *st = fail(ELSAA_ERR_INVALID_ARG, "dtype %d is not an elsaa_dtype", p->dtype);
+    return false;
+  }
+  if (p->causal != 0 && p->causal != 1) { *st = fail(ELSAA_ERR_INVALID_ARG, "causal must be 0 or 1"); return false; }
+  if (!(std::isfinite(p->scale) && std::isfinite(p->lambda) && std::isfinite(p->eps) && p->eps >= 0.f &&
+        std::isfinite(p->tau) && p->tau > 0.f)) {
+    *st = fail(ELSAA_ERR_INVALID_ARG, "scale/lambda must be finite, eps >= 0, tau > 0");
+    return false;
+  }
+  if (p->hash_bits != kHashBits) {
+    *st = fail(ELSAA_ERR_UNSUPPORTED, "hash_bits %d unsupported (4 only)", p->hash_bits);
+    return false;
+  }
+  if (p->rank_r < 0 || p->rank_r > 256 || p->rank_r % 16) {
+    *st = fail(ELSAA_ERR_UNSUPPORTED, "rank_r %d unsupported (multiple of 16 in [0, 256])", p->rank_r);
+    return false;
+  }
+  if (p->d != 64 && p->d != 128) { *st = fail(ELSAA_ERR_UNSUPPORTED, "d %d unsupported (64 or 128)", p->d); return false; }
+  const bool bf16 = p->dtype == ELSAA_DTYPE_BF16;
+  const int T = p->block_size;
+  if (bf16 ? (T != 64 && T != 128) : (T != 1 && T != 64 && T != 128)) {
+    *st = fail(ELSAA_ERR_UNSUPPORTED, "block_size %d unsupported for %s", T, bf16 ? "bf16 (64, 128)" : "f32 (1, 64, 128)");
+    return false;
+  }
+  if (T == 1 && p->N > 4096) {
+    *st = fail(ELSAA_ERR_UNSUPPORTED, "block_size 1 needs N <= 4096 (got %d)", p->N);
+    return false;
+  }
+  const int n_t = (p->N + T - 1) / T;
+  if (n_t > 1024) { *st = fail(ELSAA_ERR_UNSUPPORTED, "ceil(N / block_size) = %d > 1024", n_t); return false; }
+  if (p->topk < 0 || p->topk > n_t) {
+    *st = fail(ELSAA_ERR_INVALID_ARG, "topk %d outside [0, %d]", p->topk, n_t);
+    return false;
+  }
+  g->BH = p->B * p->H;
+  g->N = p->N;
+  g->d = p->d;
+  g->T = T;
+  g->n_t = n_t;
+  g->k = p->topk;
+  g->r = p->rank_r;
+  g->L = p->rank_r >> kHashBits;
+  g->C = bf16 ? T : 64;
+  g->n_c = (p->N + g->C - 1) / g->C;
+  long want = ((long)g->BH * g->n_c + 295) / 296;   // about two segments per SM
+  g->seg = (int)std::max(1L, std::min(16L, want));
+  g->n_seg = (g->n_c + g->seg - 1) / g->seg;
+  g->dp = p->d + 8;
+  g->causal = p->causal;
+  g->scale = p->scale;
+  g->lam = p->lambda;
+  g->eps = p->eps;
+  g->tau = p->tau;
+  return true;
+}
+
+struct Saved {
+  int* idx;
+  float *logd, *dlr, *m;
+  void *Os, *Olr;
+  void *phiQ, *phiK;
+  float *hQ, *hK, *nQ, *nK;
+  float *Ast, *Bst;
+};
+
+Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
+  Carver c(base);
+  Saved s;
+  const size_t rows = (size_t)g.BH * g.N;
+  const size_t state = (size_t)g.r * g.dp;
+  s.idx = c.take<int>((size_t)g.BH * g.n_t * std::max(g.k, 1));
+  s.logd = c.take<float>(rows);
+  s.dlr = c.take<float>(rows);
+  s.m = c.take<float>(rows);
+  s.Os = c.take<char>(rows * g.d * esz);
+  s.Olr = c.take<char>(rows * g.d * esz);
+  s.phiQ = c.take<char>(rows * g.r * esz);
+  s.phiK = c.take<char>(rows * g.r * esz);
+  s.hQ = c.take<float>(rows * g.L * kHashBits);
+  s.hK = c.take<float>(rows * g.L * kHashBits);
+  s.nQ = c.take<float>(rows);
+  s.nK = c.take<float>(rows);
+  s.Ast = c.take<float>((size_t)g.BH * (g.n_seg + 1) * state);
+  s.Bst = c.take<float>(g.causal ? (size_t)g.BH * g.n_c * state : 0);
+  *bytes = align_up(c.off);
+  return s;
+}
+
+struct FwdWs {
+  uint32_t* flag;
+  double *qbar, *kbar;
+  float* scores;
+};
+
+FwdWs carve_fwd_ws(void* base, const Geom& g, size_t* bytes) {
+  Carver c(base);
+  FwdWs w;
+  w.flag = c.take<uint32_t>(64);
+  w.qbar = c.take<double>((size_t)g.BH * g.n_t * g.d);
+  w.kbar = c.take<double>((size_t)g.BH * g.n_t * g.d);
+  w.scores = c.take<float>((size_t)g.BH * g.n_t * g.n_t);
+  *bytes = align_up(c.off);
+  return w;
+}
+
+struct BwdWs {
+  uint32_t* flag;
+  RowScalars rs;
+  float *RA, *RB;
+  int *offs, *tiles;
+  float *dQacc, *dKacc, *dVacc;
+};
+
+BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
+  Carver c(base);
+  BwdWs w;
+  const size_t rows = (size_t)g.BH * g.N;
+  const size_t state = (size_t)g.r * g.dp;
+  w.flag = c.take<uint32_t>(64);
+  w.rs.cs = c.take<float>(rows);
+  w.rs.Delta = c.take<float>(rows);
+  w.rs.cl = c.take<float>(rows);
+  w.rs.delta = c.take<float>(rows);
+  w.RA = c.take<float>((size_t)g.BH * (g.n_seg + 1) * state);
+  w.RB = c.take<float>(g.causal ? (size_t)g.BH * g.n_c * state : 0);
+  w.offs = c.take<int>((size_t)g.BH * (g.n_t + 1));
+  w.tiles = c.take<int>((size_t)g.BH * g.n_t * std::max(g.k, 1));
+  const size_t acc = bf16 && g.r > 0 ? rows * g.d : 0;
+  w.dQacc = c.take<float>(acc);
+  w.dKacc = c.take<float>(acc);
+  w.dVacc = c.take<float>(acc);
+  *bytes = align_up(c.off);
+  return w;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+elsaa_status check_ptr(const void* p, const char* name, bool required = true) {
+  if (!p) return required ? fail(ELSAA_ERR_INVALID_ARG, "%s is NULL", name) : ELSAA_OK;
+  if (!aligned16(p)) return fail(ELSAA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return ELSAA_OK;
+}
+
+elsaa_status cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return ELSAA_OK;
+  return fail(ELSAA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define ELSAA_TRY(expr)                   \
+  do {                                    \
+    elsaa_status _s = (expr);             \
+    if (_s != ELSAA_OK) return _s;        \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t elsaa_saved_bytes(const elsaa_params* p) {
+  Geom g;
+  elsaa_status st;
+  if (!make_geom(p, &g, &st)) return 0;
+  size_t bytes = 0;
+  carve_saved(nullptr, g, p->dtype == ELSAA_DTYPE_BF16 ? 2 : 4, &bytes);
+  return bytes;
+}
+
+size_t elsaa_workspace_bytes(const elsaa_params* p, int for_backward) {
+  Geom g;
+  elsaa_status st;
+  if (!make_geom(p, &g, &st)) return 0;
+  size_t bytes = 0;
+  if (for_backward) carve_bwd_ws(nullptr, g, p->dtype == ELSAA_DTYPE_BF16, &bytes);
+  else carve_fwd_ws(nullptr, g, &bytes);
+  return bytes;
+}
+
+elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, const void* V, const float* W,
+                           const float* lam, const float* gs, const float* glr, void* O, void* saved,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  Geom g;
+  elsaa_status st;
+  if (!make_geom(p, &g, &st)) return st;
+  ELSAA_TRY(check_ptr(Q, "Q"));
+  ELSAA_TRY(check_ptr(K, "K"));
+  ELSAA_TRY(check_ptr(V, "V"));
+  ELSAA_TRY(check_ptr(O, "O"));
+  ELSAA_TRY(check_ptr(saved, "saved"));
+  ELSAA_TRY(check_ptr(workspace, "workspace"));
+  ELSAA_TRY(check_ptr(W, "W_hash", g.r > 0));
+  ELSAA_TRY(check_ptr(lam, "lambda_vec", false));
+  ELSAA_TRY(check_ptr(gs, "g_sparse", false));
+  ELSAA_TRY(check_ptr(glr, "g_lr", false));
+  const bool bf16 = p->dtype == ELSAA_DTYPE_BF16;
+  size_t need = 0;
+  FwdWs w = carve_fwd_ws(workspace, g, &need);
+  if (ws_bytes < need) return fail(ELSAA_ERR_WORKSPACE, "workspace %zu bytes < %zu required", ws_bytes, need);
+  size_t sb = 0;
+  Saved s = carve_saved(saved, g, bf16 ? 2 : 4, &sb);
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+
+  ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st_), "flag reset"));
+  ELSAA_TRY(cuda_status(launch_select(Q, K, bf16, w.qbar, w.kbar, w.scores, s.idx, g, st_), "selection"));
+  ELSAA_TRY(cuda_status(launch_race_features(Q, K, W, bf16, s.phiQ, s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, st_),
+                        "race features"));
+  ELSAA_TRY(cuda_status(launch_race_state_fwd(s.phiK, V, bf16, s.Ast, s.Bst, g, st_), "race summaries"));
+  FwdArgs a{Q, K, V, s.idx, s.phiQ, s.phiK, s.Ast, s.Bst, lam, gs, glr, O, s.Os, s.logd, s.dlr, s.m, s.Olr};
+  if (bf16) ELSAA_TRY(cuda_status(launch_attn_fwd_bf16(a, g, st_), "fused forward"));
+  else ELSAA_TRY(cuda_status(launch_attn_fwd_f32(a, g, st_), "fused forward"));
+  return ELSAA_OK;
+}
+
+elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K, const void* V, const float* W,
+                            const float* lam, const float* gs, const float* glr, const void* dO,
+                            const void* saved, void* dQ, void* dK, void* dV, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  g_last_error.clear();
+  Geom g;
+  elsaa_status st;
+  if (!make_geom(p, &g, &st)) return st;
+  ELSAA_TRY(check_ptr(Q, "Q"));
+  ELSAA_TRY(check_ptr(K, "K"));
+  ELSAA_TRY(check_ptr(V, "V"));
+  ELSAA_TRY(check_ptr(dO, "dO"));
+  ELSAA_TRY(check_ptr(saved, "saved"));
+  ELSAA_TRY(check_ptr(dQ, "dQ"));
+  ELSAA_TRY(check_ptr(dK, "dK"));
+  ELSAA_TRY(check_ptr(dV, "dV"));
+  ELSAA_TRY(check_ptr(workspace, "workspace"));
+  ELSAA_TRY(check_ptr(W, "W_hash", g.r > 0));
+  ELSAA_TRY(check_ptr(lam, "lambda_vec", false));
+  ELSAA_TRY(check_ptr(gs, "g_sparse", false));
+  ELSAA_TRY(check_ptr(glr, "g_lr", false));
+  const bool bf16 = p->dtype == ELSAA_DTYPE_BF16;
+  size_t need = 0;
+  BwdWs w = carve_bwd_ws(workspace, g, bf16, &need);
+  if (ws_bytes < need) return fail(ELSAA_ERR_WORKSPACE, "workspace %zu bytes < %zu required", ws_bytes, need);
+  size_t sb = 0;
+  Saved s = carve_saved(const_cast<void*>(saved), g, bf16 ? 2 : 4, &sb);
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  BwdArgs a{};
+  a.Q = Q; a.K = K; a.V = V; a.dO = dO; a.W = W;
+  a.lam = lam; a.gs = gs; a.glr = glr;
+  a.idx = s.idx; a.logd = s.logd; a.dlr = s.dlr; a.m = s.m;
+  a.Os = s.Os; a.Olr = s.Olr; a.phiQ = s.phiQ; a.phiK = s.phiK;
+  a.hQ = s.hQ; a.hK = s.hK; a.nQ = s.nQ; a.nK = s.nK;
+  a.Ast = s.Ast; a.Bst = s.Bst; a.RA = w.RA; a.RB = w.RB;
+  a.offs = w.offs; a.tiles = w.tiles; a.rs = w.rs;
+  a.dQacc = w.dQacc; a.dKacc = w.dKacc; a.dVacc = w.dVacc;
+  a.dQ = dQ; a.dK = dK; a.dV = dV;
+
+  ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st_), "flag reset"));
+  ELSAA_TRY(cuda_status(launch_row_scalars(a, bf16, g, st_), "row scalars"));
+  ELSAA_TRY(cuda_status(launch_race_state_bwd(a, bf16, g, st_), "race suffix summaries"));
+  if (g.k > 0) ELSAA_TRY(cuda_status(launch_invert_selection(s.idx, w.offs, w.tiles, g, st_), "selection inverse"));
+  if (bf16) ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, st_), "backward"));
+  else ELSAA_TRY(cuda_status(launch_bwd_f32(a, g, st_), "backward"));
+  return ELSAA_OK;
+}
+
+elsaa_status elsaa_debug_select(const elsaa_params* p, const void* Q, const void* K, float* scores, int32_t* idx,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  Geom g;
+  elsaa_status st;
+  if (!make_geom(p, &g, &st)) return st;
+  ELSAA_TRY(check_ptr(Q, "Q"));
+  ELSAA_TRY(check_ptr(K, "K"));
+  ELSAA_TRY(check_ptr(scores, "scores"));
+  ELSAA_TRY(check_ptr(idx, "idx", g.k > 0));
+  ELSAA_TRY(check_ptr(workspace, "workspace"));
+  size_t need = 0;
+  FwdWs w = carve_fwd_ws(workspace, g, &need);
+  if (ws_bytes < need) return fail(ELSAA_ERR_WORKSPACE, "workspace %zu bytes < %zu required", ws_bytes, need);
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_select(Q, K, p->dtype == ELSAA_DTYPE_BF16, w.qbar, w.kbar, scores, idx, g, st_),
+                     "selection");
+}
+
+elsaa_status elsaa_check_device_flags(void* workspace, void* stream) {
+  g_last_error.clear();
+  if (!workspace) return fail(ELSAA_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  uint32_t flag = 0;
+  ELSAA_TRY(cuda_status(cudaStreamSynchronize(st_), "stream sync"));
+  ELSAA_TRY(cuda_status(cudaMemcpy(&flag, workspace, 4, cudaMemcpyDeviceToHost), "flag read"));
+  ELSAA_TRY(cuda_status(cudaMemset(workspace, 0, 4), "flag clear"));
+  if (flag) return fail(ELSAA_ERR_TIMEOUT, "a kernel gave up a bounded wait (flag 0x%x)", flag);
+  return ELSAA_OK;
+}
+
+const char* elsaa_status_string(elsaa_status s) {
+  switch (s) {
+    case ELSAA_OK: return "ok";
+    case ELSAA_ERR_INVALID_ARG: return "invalid argument";
+    case ELSAA_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case ELSAA_ERR_WORKSPACE: return "workspace too small";
+    case ELSAA_ERR_CUDA: return "CUDA error";
+    case ELSAA_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* elsaa_last_error_message(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

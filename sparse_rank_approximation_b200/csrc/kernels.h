@@ -1,0 +1,60 @@
+// Internal launch interface between the C ABI (elsaa_api.cu) and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include "common.cuh"
+
+namespace elsaa {
+
+struct FwdArgs {
+  const void *Q, *K, *V;
+  const int* idx;
+  const void *phiQ, *phiK;
+  const float *Ast, *Bst;
+  const float *lam, *gs, *glr;
+  void *O, *Os;
+  float *logd, *dlr, *m;
+  void* Olr;      // O_lr saved for the backward
+};
+
+// Per-row adjoint scalars of the fusion (Eq. 4 / Eq. 5), float32 [BH, N] each.
+struct RowScalars {
+  float* cs;      // g_s m: dO_s = cs dO
+  float* Delta;   // <dO_s, O_s> - dd_s d_s   (sparse softmax delta)
+  float* cl;      // g_lr / d_lr: dN = cl dO
+  float* delta;   // dd_lr - cl <dO, O_lr>      (RACE key-mass adjoint)
+};
+
+struct BwdArgs {
+  const void *Q, *K, *V, *dO;
+  const float* W;
+  const float *lam, *gs, *glr;
+  const int* idx;
+  const float *logd, *dlr, *m;
+  const void *Os, *Olr;
+  const void *phiQ, *phiK;
+  const float *hQ, *hK, *nQ, *nK;
+  const float *Ast, *Bst;        // forward prefix statistics
+  float *RA, *RB;                // backward suffix statistics
+  const int *offs, *tiles;       // key block -> query tiles
+  RowScalars rs;
+  float *dQacc, *dKacc, *dVacc;  // fp32 low-rank gradient parts (bf16 path)
+  void *dQ, *dK, *dV;
+};
+
+cudaError_t launch_select(const void* Q, const void* K, bool bf16, double* qbar, double* kbar, float* scores,
+                          int* idx, const Geom& g, cudaStream_t st);
+cudaError_t launch_invert_selection(const int* idx, int* offs, int* tiles, const Geom& g, cudaStream_t st);
+cudaError_t launch_race_features(const void* Q, const void* K, const float* W, bool bf16, void* phiQ, void* phiK,
+                                 float* hQ, float* hK, float* nQ, float* nK, const Geom& g, cudaStream_t st);
+// Forward prefix statistics (Ast: per-segment exclusive prefix, Bst: in-segment prefix).
+cudaError_t launch_race_state_fwd(const void* phiK, const void* V, bool bf16, float* Ast, float* Bst,
+                                  const Geom& g, cudaStream_t st);
+// Backward suffix statistics of Phi(q_i) [cl_i dO_i ; delta_i]^T.
+cudaError_t launch_race_state_bwd(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st);
+cudaError_t launch_attn_fwd_bf16(const FwdArgs& a, const Geom& g, cudaStream_t st);
+cudaError_t launch_attn_fwd_f32(const FwdArgs& a, const Geom& g, cudaStream_t st);
+cudaError_t launch_row_scalars(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st);
+cudaError_t launch_bwd_bf16(const BwdArgs& a, const Geom& g, cudaStream_t st);
+cudaError_t launch_bwd_f32(const BwdArgs& a, const Geom& g, cudaStream_t st);
+
+}  // namespace elsaa

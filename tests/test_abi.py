@@ -1,0 +1,83 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, sizes its buffers, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_rank_approximation_b200 import binding as bd
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "elsaa.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return set(re.findall(r"ELSAA_API\s+[\w\s\*]+?\b(elsaa_\w+)\s*\(", text))
+
+
+def test_header_declarations_are_all_exported():
+    names = _declared()
+    assert names == set(bd.EXPORTED)
+    L = bd.lib()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_sizes_for_valid_and_invalid_params():
+    L = bd.lib()
+    p = bd.make_params(1, 32, 16384, 128, rank_r=128, block_size=128, topk=16)
+    assert L.elsaa_saved_bytes(ctypes.byref(p)) > 2 * 32 * 16384 * 128 * 2
+    assert L.elsaa_workspace_bytes(ctypes.byref(p), 0) > 0
+    assert L.elsaa_workspace_bytes(ctypes.byref(p), 1) > L.elsaa_workspace_bytes(ctypes.byref(p), 0)
+    bad = [dict(d=96), dict(rank_r=24), dict(rank_r=512), dict(block_size=32), dict(topk=200),
+           dict(hash_bits=3), dict(tau=0.0), dict(eps=-1.0)]
+    for kw in bad:
+        args = dict(B=1, H=2, N=1024, d=64, rank_r=64, block_size=64, topk=4)
+        hb = kw.pop("hash_bits", 4)
+        args.update(kw)
+        q = bd.make_params(args.pop("B"), args.pop("H"), args.pop("N"), args.pop("d"), hash_bits=hb, **args)
+        assert L.elsaa_saved_bytes(ctypes.byref(q)) == 0, kw
+        assert L.elsaa_workspace_bytes(ctypes.byref(q), 1) == 0, kw
+    assert L.elsaa_saved_bytes(None) == 0
+
+
+def test_block_size_one_is_f32_only():
+    L = bd.lib()
+    p = bd.make_params(1, 1, 256, 64, dtype=bd.ELSAA_DTYPE_F32, causal=False, rank_r=16, block_size=1, topk=32)
+    assert L.elsaa_saved_bytes(ctypes.byref(p)) > 0
+    p.dtype = bd.ELSAA_DTYPE_BF16
+    assert L.elsaa_saved_bytes(ctypes.byref(p)) == 0
+    p.dtype = bd.ELSAA_DTYPE_F32
+    p.N = 8192
+    assert L.elsaa_saved_bytes(ctypes.byref(p)) == 0
+
+
+def _fwd(L, p, Q=0x1000, K=0x1000, V=0x1000, W=0x1000, O=0x1000, saved=0x1000, ws=0x1000, wsb=1 << 40):
+    return L.elsaa_forward(ctypes.byref(p), Q, K, V, W, None, None, None, O, saved, ws, wsb, None)
+
+
+def test_argument_errors_return_before_any_launch():
+    L = bd.lib()
+    p = bd.make_params(1, 2, 1024, 64, rank_r=64, block_size=64, topk=4)
+    assert _fwd(L, p, Q=None) == bd.ELSAA_ERR_INVALID_ARG
+    assert b"Q is NULL" in L.elsaa_last_error_message()
+    assert _fwd(L, p, V=0x1008) == bd.ELSAA_ERR_INVALID_ARG
+    assert b"aligned" in L.elsaa_last_error_message()
+    assert _fwd(L, p, W=None) == bd.ELSAA_ERR_INVALID_ARG
+    assert _fwd(L, p, wsb=16) == bd.ELSAA_ERR_WORKSPACE
+    q = bd.make_params(1, 2, 1024, 96, rank_r=64, block_size=64, topk=4)
+    assert _fwd(L, q) == bd.ELSAA_ERR_UNSUPPORTED
+    q = bd.make_params(1, 2, 1024, 64, rank_r=64, block_size=64, topk=17)
+    assert _fwd(L, q) == bd.ELSAA_ERR_INVALID_ARG
+    st = L.elsaa_backward(ctypes.byref(p), 0x1000, 0x1000, 0x1000, 0x1000, None, None, None, None, 0x1000,
+                          0x1000, 0x1000, 0x1000, 0x1000, 1 << 40, None)
+    assert st == bd.ELSAA_ERR_INVALID_ARG and b"dO" in L.elsaa_last_error_message()
+    assert L.elsaa_check_device_flags(None, None) == bd.ELSAA_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    L = bd.lib()
+    for s in range(6):
+        assert L.elsaa_status_string(s)
+    assert L.elsaa_status_string(99) == b"unknown status"

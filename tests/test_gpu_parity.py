@@ -1,0 +1,158 @@
+"""CUDA path vs the float64 oracle, through the C ABI, on seeded inputs.
+
+Small problems span several tiles and a ragged last tile and are compared
+element by element; the named full-size workloads are compared on every
+selected index and on sampled rows of O, dQ, dK and dV.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import elsaa_oracle as orc
+from sparse_rank_approximation_b200.workloads import WORKLOADS, make_inputs, small_workload
+from tests.harness import check, device_inputs, gpu_op, np64, oracle_params
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "bf16_d64_T64_causal_ragged": small_workload(N=64 * 5 + 37, d=64, block_size=64, topk=3, rank_r=32, H=2),
+    "bf16_d128_T128_causal_ragged": small_workload(N=128 * 4 + 5, d=128, block_size=128, topk=2, rank_r=64, H=2),
+    "bf16_d64_T128_noncausal": small_workload(N=128 * 3 + 50, d=64, block_size=128, topk=2, rank_r=16,
+                                              causal=False),
+    "bf16_d128_T64_r256": small_workload(N=64 * 6, d=128, block_size=64, topk=4, rank_r=256, B=2, H=1),
+    "bf16_all_blocks": small_workload(N=64 * 4, d=64, block_size=64, topk=4, rank_r=16, causal=False),
+    "f32_config_tiny": WORKLOADS["tiny_f32"],
+    "f32_T64_causal_ragged": small_workload(N=64 * 3 + 11, d=64, block_size=64, topk=2, rank_r=32, dtype="f32"),
+    "f32_T1_causal": small_workload(N=200, d=128, block_size=1, topk=24, rank_r=48, dtype="f32", kind="iid"),
+    "f32_T128_noncausal": small_workload(N=300, d=128, block_size=128, topk=2, rank_r=16, dtype="f32",
+                                         causal=False),
+}
+
+
+def _run(w, seed=0, lam_vec=False, gates=False, **over):
+    inp = make_inputs(w, seed)
+    dev = device_inputs(w, inp)
+    op = gpu_op(w, **{k: v for k, v in over.items() if k in ("lam", "eps", "tau")})
+    BH = (w.B, w.H, w.N)
+    g = torch.Generator().manual_seed(seed + 100)
+    extra_cpu = {}
+    if lam_vec:
+        extra_cpu["lam"] = torch.rand(BH, generator=g) * 2.0
+    if gates:
+        extra_cpu["g_s"] = torch.rand(BH, generator=g)
+        extra_cpu["g_lr"] = torch.rand(BH, generator=g)
+    extra = {k: v.cuda() for k, v in extra_cpu.items()}
+    O = op.forward(dev["Q"], dev["K"], dev["V"], dev["W"], extra.get("lam"), extra.get("g_s"), extra.get("g_lr"))
+    scores, idx = op.debug_select(dev["Q"], dev["K"])
+    dQ, dK, dV = op.backward(dev["Q"], dev["K"], dev["V"], dev["W"], dev["dO"], extra.get("lam"),
+                             extra.get("g_s"), extra.get("g_lr"))
+    torch.cuda.synchronize()
+    return inp, extra_cpu, O, scores, idx, (dQ, dK, dV)
+
+
+def _oracle_head(w, inp, extra, scores, b, h, **over):
+    p = oracle_params(w, **over)
+    get = lambda n: inp[n][b, h].double().numpy()
+    ex = {k: v[b, h].double().numpy() for k, v in extra.items()}
+    W = inp["W"].double().numpy()
+    fw = orc.forward_head(get("Q"), get("K"), get("V"), W, p, ex.get("lam"), ex.get("g_s"), ex.get("g_lr"),
+                          scores=np64(scores[b, h]))
+    grads = orc.backward_head(get("Q"), get("K"), get("V"), W, get("dO"), fw, p, ex.get("lam"), ex.get("g_s"),
+                              ex.get("g_lr"))
+    return fw, grads
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_backward_small(name):
+    w = SMALL[name]
+    inp, extra, O, scores, idx, grads = _run(w)
+    for b in range(w.B):
+        for h in range(w.H):
+            fw, (dq, dk, dv) = _oracle_head(w, inp, extra, scores, b, h)
+            assert np.array_equal(idx[b, h].cpu().numpy(), fw["idx"]), "selection differs"
+            check(w, f"O[{b},{h}]", np64(O[b, h]), fw["O"])
+            check(w, f"dQ[{b},{h}]", np64(grads[0][b, h]), dq)
+            check(w, f"dK[{b},{h}]", np64(grads[1][b, h]), dk)
+            check(w, f"dV[{b},{h}]", np64(grads[2][b, h]), dv)
+
+
+@pytest.mark.parametrize("case", ["k0", "r0_eps0", "lam_gates", "tau_lam"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_branch_switches_and_options(case, dtype):
+    base = dict(N=64 * 4 + 20, d=64, block_size=64, topk=2, rank_r=32, dtype=dtype, H=2)
+    kw, over, lam_vec, gates = {}, {}, False, False
+    if case == "k0":
+        base["topk"] = 0
+    elif case == "r0_eps0":
+        base["rank_r"] = 0
+        over["eps"] = 0.0
+    elif case == "lam_gates":
+        lam_vec = gates = True
+    elif case == "tau_lam":
+        over.update(tau=0.5, lam=3.0, eps=0.01)
+    w = small_workload(**base)
+    inp, extra, O, scores, idx, grads = _run(w, lam_vec=lam_vec, gates=gates, **over)
+    for h in range(w.H):
+        fw, (dq, dk, dv) = _oracle_head(w, inp, extra, scores, 0, h, **over)
+        check(w, "O", np64(O[0, h]), fw["O"])
+        check(w, "dQ", np64(grads[0][0, h]), dq)
+        check(w, "dK", np64(grads[1][0, h]), dk)
+        check(w, "dV", np64(grads[2][0, h]), dv)
+
+
+@pytest.mark.parametrize("name", ["n2k_d64", "n8k_d64", "n16k_d128", "n64k_d128"])
+def test_selection_full_size(name):
+    """Bit-exact against the oracle fed the GPU's float32 scores; against the
+    oracle's own float64 scores, differences only at near-ties (1e-6 relative)."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w, 0)
+    dev = device_inputs(w, inp)
+    op = gpu_op(w)
+    scores, idx = op.debug_select(dev["Q"], dev["K"])
+    torch.cuda.synchronize()
+    sc, ix = scores.cpu().numpy(), idx.cpu().numpy()
+    p = oracle_params(w)
+    for b in range(w.B):
+        for h in range(w.H):
+            assert np.array_equal(orc.select_from_scores(sc[b, h], w.topk, w.causal), ix[b, h])
+    for b, h in [(0, 0), (w.B - 1, w.H - 1)]:
+        s64 = orc.block_scores(inp["Q"][b, h].double().numpy(), inp["K"][b, h].double().numpy(), p)
+        np.testing.assert_allclose(sc[b, h], s64, rtol=0, atol=2e-6 * max(1.0, np.abs(s64).max()))
+        own = orc.select_from_scores(s64, w.topk, w.causal)
+        for t in np.nonzero(np.any(own != ix[b, h], axis=1))[0]:
+            a = set(own[t]) - set(ix[b, h, t])
+            g = set(ix[b, h, t]) - set(own[t])
+            for x, y in zip(sorted(a), sorted(g)):
+                assert abs(s64[t, x] - s64[t, y]) <= 1e-6 * max(abs(s64[t, x]), abs(s64[t, y])), (t, x, y)
+
+
+@pytest.mark.parametrize("name", ["n2k_d64", "n8k_d64", "n16k_d128", "n64k_d128"])
+def test_forward_backward_full_size_sampled(name):
+    """Full-size workload, launched exactly as the benchmark launches it; outputs
+    compared on sampled rows of two heads."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w, 0)
+    dev = device_inputs(w, inp)
+    op = gpu_op(w)
+    O = op.forward(dev["Q"], dev["K"], dev["V"], dev["W"])
+    scores, _ = op.debug_select(dev["Q"], dev["K"])
+    dQ, dK, dV = op.backward(dev["Q"], dev["K"], dev["V"], dev["W"], dev["dO"])
+    torch.cuda.synchronize()
+    p = oracle_params(w)
+    rng = np.random.default_rng(1)
+    heads = [(0, 0), (w.B - 1, w.H - 1)] if name != "n64k_d128" else [(0, w.H - 1)]
+    for b, h in heads:
+        get = lambda n: inp[n][b, h].double().numpy()
+        q, k, v, dO = get("Q"), get("K"), get("V"), get("dO")
+        W = inp["W"].double().numpy()
+        sc = np64(scores[b, h])
+        rows = np.unique(np.concatenate([[0, w.N - 1, w.block_size - 1, w.block_size],
+                                         rng.integers(0, w.N, 12)]))
+        fr = orc.forward_rows_head(q, k, v, W, p, rows, scores=sc)
+        check(w, "O rows", np64(O[b, h][rows]), fr["O"])
+        fw = orc.forward_head(q, k, v, W, p, scores=sc)
+        krows = np.unique(np.concatenate([[0, w.N - 1], rng.integers(0, w.N, 6)]))
+        dq, dk, dv = orc.backward_rows_head(q, k, v, W, dO, fw, p, rows, krows)
+        check(w, "dQ rows", np64(dQ[b, h][rows]), dq)
+        check(w, "dK rows", np64(dK[b, h][krows]), dk)
+        check(w, "dV rows", np64(dV[b, h][krows]), dv)

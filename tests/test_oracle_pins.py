@@ -375,3 +375,22 @@ def test_interaction_count_matches_paper_example():
     a = g["args"]
     assert orc.interaction_count(a["N"], a["s"], a["L_s"], a["gamma"]) == g["elsaa_interactions"]
     assert a["N"] ** 2 == g["dense_interactions"]
+
+
+# --- the row-sampled forms agree with the whole-head forms pinned above ---
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_row_sampled_forms_match_full(causal):
+    q, k, v, W, p = _setup(N=44, d=8, T=8, k=2, r=32, causal=causal, seed=70)
+    dO = _rand((p.N, p.d), 71)
+    lam = np.linspace(0.5, 1.5, p.N)
+    fw = orc.forward_head(q, k, v, W, p, lam)
+    rows = [0, 7, 8, 30, 43]
+    fr = orc.forward_rows_head(q, k, v, W, p, rows, lam)
+    for key in ("O", "O_s", "logd_s", "O_lr", "d_lr", "m"):
+        np.testing.assert_allclose(fr[key], fw[key][rows], atol=1e-12, rtol=1e-12)
+    dq, dk, dv = orc.backward_head(q, k, v, W, dO, fw, p, lam)
+    sq, sk, sv = orc.backward_rows_head(q, k, v, W, dO, fw, p, rows, rows, lam)
+    np.testing.assert_allclose(sq, dq[rows], atol=1e-11)
+    np.testing.assert_allclose(sk, dk[rows], atol=1e-11)
+    np.testing.assert_allclose(sv, dv[rows], atol=1e-11)
