@@ -9,9 +9,13 @@ from sparse_rank_approximation_b200.workloads import Workload, make_inputs
 
 # Tolerances (relative to the oracle, float64):
 #   float32 path: max |gpu - oracle| / max |oracle| <= 1e-4 per output tensor;
-#   bf16 path:    max |gpu - oracle| <= 2e-2 (unit-variance V and dO).
+#   bf16 path:    |gpu - oracle| <= 2e-2 + 2^-8 |oracle| element-wise (unit-variance
+#                 V and dO): 2e-2 for the arithmetic plus the rounding of the bf16
+#                 output itself, whose half-ulp is up to 2^-8 of the value (an
+#                 output of magnitude 8 is already 0.03 away from its exact value).
 F32_REL_TOL = 1e-4
 BF16_ABS_TOL = 2e-2
+BF16_STORE_REL = 2.0 ** -8
 
 
 def oracle_params(w: Workload, **kw) -> orc.Params:
@@ -49,5 +53,7 @@ def check(w: Workload, name: str, gpu: np.ndarray, ref: np.ndarray):
         rel = err / max(np.abs(ref).max(), 1e-30)
         assert rel <= F32_REL_TOL, f"{name}: max rel err {rel:.3e} > {F32_REL_TOL}"
         return rel
-    assert err <= BF16_ABS_TOL, f"{name}: max abs err {err:.3e} > {BF16_ABS_TOL} (max |ref| {np.abs(ref).max():.3f})"
+    excess = (np.abs(gpu - ref) - BF16_STORE_REL * np.abs(ref)).max()
+    assert excess <= BF16_ABS_TOL, (f"{name}: max abs err {err:.3e}, beyond bf16 storage {excess:.3e} > "
+                                    f"{BF16_ABS_TOL} (max |ref| {np.abs(ref).max():.3f})")
     return err
