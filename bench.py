@@ -1,0 +1,427 @@
+"""Benchmark of the ELSAA attention operator (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl elsaa|reference]
+
+A step is one forward and one backward pass of the whole operator (selection,
+RACE features and summaries, fused sparse + low-rank forward, row scalars,
+suffix summaries, selection inverse, and the four backward kernels) over one
+batch of synthetic input that is resident in HBM.  Default workload: B=1, H=32,
+N=16384, d=128, bf16, causal, r=128, 128-key blocks, top-16 blocks per tile.
+Each rank runs its own batch (independent problems, no collective on the data
+path), so multi-GPU runs scale weakly; rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
+
+from sparse_rank_approximation_b200.workloads import HEADLINE, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "ELSAA fwd+bwd tokens/sec and % of roofline at N=16K, 1×B200"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------
+# Algorithmic work per kernel (the method's own counts, not what a kernel
+# happens to move): used for the roofline numbers.
+# --------------------------------------------------------------------------
+
+def selected_blocks_per_head(w):
+    """sum over tiles of the number of selected key blocks (causal tiles near the
+    start have fewer eligible blocks)."""
+    n_t = w.n_tiles
+    if w.topk == 0:
+        return 0
+    if not w.causal:
+        return n_t * w.topk
+    return sum(min(w.topk, t + 1) for t in range(n_t))
+
+
+def work_model(w):
+    BH, N, d, T, r = w.B * w.H, w.N, w.d, w.block_size, w.rank_r
+    sel = selected_blocks_per_head(w) * BH          # (tile, block) pairs
+    pair_mma = 2 * T * T * d                        # one T x T x d product
+    L = w.n_tables
+    m = {}
+    # sparse branch forward: QK^T and PV per selected (tile, block) pair
+    f_sparse = 2 * pair_mma * sel
+    # RACE read-out in the fused kernel: Phi_Q P (T x r x (d+1)) per tile, plus the
+    # diagonal-chunk kappa (T x T x r) and kappa [V|1] (T x T x (d+1)) when causal
+    tiles = w.n_tiles * BH
+    f_read = tiles * 2 * T * r * (d + 1) + (tiles * 2 * T * T * (r + d + 1) if w.causal else 0)
+    m["attn_fwd"] = dict(flops=f_sparse + f_read,
+                         bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 5)   # gathered K,V + Q, O, O_s, O_lr
+    m["sparse_dq"] = dict(flops=3 * pair_mma * sel, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 3)
+    m["sparse_dkdv"] = dict(flops=4 * pair_mma * sel, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 4)
+    f_state = tiles * 2 * T * r * (d + 8)
+    m["race_state_fwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)
+    m["race_state_bwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)
+    m["race_features"] = dict(flops=2 * 2 * BH * N * d * 4 * L * 2, bytes=2 * BH * N * (d + r) * 2)
+    unique_fwd = 4 * BH * N * d * 2                # Q, K, V read, O written
+    return m, dict(sel_pairs=sel, tiles=tiles, f_sparse_fwd=f_sparse, f_lr_fwd=f_read + f_state,
+                   gathered_fwd=sel * 2 * T * d * 2, unique_fwd=unique_fwd)
+
+
+def north_star_roofline(w, peaks, t_step_ms):
+    """T_roof = max(F / P_bf16, gathered bytes / BW), forward + backward, counted as
+    sparse F_bwd = 2.5 F_fwd, low-rank F_bwd = 2 F_fwd, backward bytes = 2x gathered
+    plus 8 N d bf16 rows per head."""
+    _, tot = work_model(w)
+    F = tot["f_sparse_fwd"] * 3.5 + tot["f_lr_fwd"] * 3.0
+    BH = w.B * w.H
+    bytes_ = tot["gathered_fwd"] * 3 + 8 * BH * w.N * w.d * 2 + tot["unique_fwd"]
+    t_f = F / (peaks["bf16_tflops"] * 1e12)
+    t_b = bytes_ / (peaks["hbm_gbs"] * 1e9)
+    t_roof = max(t_f, t_b)
+    return dict(t_roof_ms=t_roof * 1e3, frac=t_roof * 1e3 / t_step_ms, flops=F, bytes=bytes_,
+                bound="tensor" if t_f >= t_b else "hbm",
+                compute_only_frac=t_f * 1e3 / t_step_ms)
+
+
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi sampling (every 100 ms) while the timed region runs."""
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = ""
+        self.window = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def mark(self, begin: bool):
+        import datetime
+        now = datetime.datetime.now()
+        self.window = (now, None) if begin else (self.window[0], now)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        import datetime
+        rows = []
+        for r in csv.reader(io.StringIO(self.out)):
+            if len(r) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(r[2]), float(r[3]), [x.strip().lower() for x in r[6:10]]))
+            except ValueError:
+                continue
+        inside = [x for x in rows if self.window and self.window[1] and self.window[0] <= x[0] <= self.window[1]]
+        use = inside or rows
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({n for x in use for n, v in zip(self.REASONS, x[3]) if v == "active"})
+        return {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": max(x[2] for x in use),
+                "reasons": reasons, "samples": len(use), "in_window": bool(inside)}
+
+
+def kernel_sources_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_rank_approximation_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if it was
+    taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_sources_hash()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload \
+                and parts[3] == src:
+            return float(parts[2])
+    return None
+
+
+# --------------------------------------------------------------------------
+
+class OracleSample:
+    """The float64 oracle (forward + backward) on a bounded sample of the workload:
+    one head, and of its query tiles an evenly spaced subset (the backward is a
+    sum of per-tile contributions, so a subset is that share of the work)."""
+
+    def __init__(self, w):
+        from oracle import elsaa_oracle as orc
+        self.orc, self.w = orc, w
+        inp = make_inputs(w, 0, heads=range(1))
+        self.p = orc.Params(N=w.N, d=w.d, block_size=w.block_size, topk=w.topk, rank_r=w.rank_r,
+                            causal=w.causal, scale=w.scale)
+        self.W = inp["W"].double().numpy()
+        self.x = {n: inp[n][0, 0].double().numpy() for n in ("Q", "K", "V", "dO")}
+
+    def run(self, n_tiles):
+        """Returns (equivalent tokens of the full batch, seconds)."""
+        w, x = self.w, self.x
+        nt = w.n_tiles
+        n_tiles = max(1, min(nt, n_tiles))
+        tiles = sorted({int(round(i * (nt - 1) / max(1, n_tiles - 1))) for i in range(n_tiles)})
+        t0 = time.perf_counter()
+        fw = self.orc.forward_head(x["Q"], x["K"], x["V"], self.W, self.p, tiles=tiles)
+        self.orc.backward_head(x["Q"], x["K"], x["V"], self.W, x["dO"], fw, self.p, tiles=tiles)
+        dt = time.perf_counter() - t0
+        return w.B * w.N * (len(tiles) / nt) / w.H, dt
+
+    def calibrate(self, seconds):
+        """Number of query tiles whose fwd+bwd takes about `seconds`."""
+        _, t1 = self.run(1)
+        _, t4 = self.run(4)
+        per_tile = max((t4 - t1) / 3, 1e-3)
+        fixed = max(t1 - per_tile, 0.0)
+        return max(1, min(self.w.n_tiles, int((seconds - fixed) / per_tile)))
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    budget = 150.0                      # seconds for the whole warm-up + timed run
+    smp = OracleSample(w)
+    n_tiles = smp.calibrate(budget / (args.steps + args.warmup))
+    for _ in range(args.warmup):
+        smp.run(n_tiles)
+    tokens, secs = 0.0, 0.0
+    for _ in range(args.steps):
+        tk, dt = smp.run(n_tiles)
+        tokens += tk
+        secs += dt
+    value = tokens / secs
+    sample = (f"float64 oracle fwd+bwd, per step {n_tiles} of {w.n_tiles} query tiles of 1 of {w.H} heads, "
+              f"scaled to the full batch")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "shape": w.describe(), "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="elsaa", choices=["elsaa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    from sparse_rank_approximation_b200 import binding as bd
+    peaks, peak_kind = load_peaks()
+    inp = make_inputs(w, seed=rank)
+    key = "16" if w.dtype == "bf16" else ""
+    q, k, v, dO = (inp[n + key].to(dev) for n in ("Q", "K", "V", "dO"))
+    W = inp["W"].to(dev)
+    op = bd.Elsaa(bd.make_params(w.B, w.H, w.N, w.d,
+                                 dtype=bd.ELSAA_DTYPE_BF16 if w.dtype == "bf16" else bd.ELSAA_DTYPE_F32,
+                                 causal=w.causal, rank_r=w.rank_r, block_size=w.block_size, topk=w.topk), dev)
+    O = op._empty_like_io()
+    grads = (op._empty_like_io(), op._empty_like_io(), op._empty_like_io())
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        op.forward(q, k, v, W, out=O)
+        op.backward(q, k, v, W, dO, grads=grads)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        barrier()
+        bd.profile_begin()
+        clk.mark(True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        barrier()
+        clk.mark(False)
+        prof = bd.profile_end()
+    ms_total = ev0.elapsed_time(ev1)
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens_step = w.B * w.N * world
+    value = tokens_step / (ms_step * 1e-3)
+    launches = sum(c for _, c in prof.values())
+
+    # end to end: pinned host inputs in, results (O and the three gradients) out, every step
+    e2e = None
+    if not args.no_e2e:
+        host = {n: inp[n + key].pin_memory() for n in ("Q", "K", "V", "dO")}
+        host_W = inp["W"].pin_memory()
+        outs = [torch.empty(O.shape, dtype=O.dtype).pin_memory() for _ in range(4)]
+        h2d = sum(x.numel() * x.element_size() for x in host.values()) + host_W.numel() * 4
+        d2h = sum(x.numel() * x.element_size() for x in outs)
+
+        def e2e_step():
+            q.copy_(host["Q"], non_blocking=True)
+            k.copy_(host["K"], non_blocking=True)
+            v.copy_(host["V"], non_blocking=True)
+            dO.copy_(host["dO"], non_blocking=True)
+            W.copy_(host_W, non_blocking=True)
+            step()
+            for hsrc, dsrc in zip(outs, (O,) + grads):
+                hsrc.copy_(dsrc, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, args.steps // 4)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        te = torch.tensor([e0.elapsed_time(e1) / n_e2e], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": tokens_step / (float(te.item()) * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": float(te.item())}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    model, _ = work_model(w)
+    dom = max(prof.items(), key=lambda kv: kv[1][0])[0]
+    dom_ms = prof[dom][0] / prof[dom][1]
+    wm = model.get(dom)
+    roof = None
+    if wm is not None:
+        tensor_kernel = dom in ("attn_fwd", "sparse_dq", "sparse_dkdv", "race_state_fwd", "race_state_bwd")
+        if tensor_kernel:
+            ach = wm["flops"] / (dom_ms * 1e-3) / 1e12
+            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+            roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak}
+        else:
+            ach = wm["bytes"] / (dom_ms * 1e-3) / 1e9
+            peak = peaks["hbm_gbs"]
+            roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak}
+        roof.update({"kernel": dom, "ms_per_launch": dom_ms, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"
+                     if peak_kind == "measured" else "fallback",
+                     "traffic": dram_traffic(dom, w.name)})
+    kernels = {n: {"ms_per_launch": ms / c, "launches": c, "share": ms / sum(x for x, _ in prof.values())}
+               for n, (ms, c) in sorted(prof.items(), key=lambda kv: -kv[1][0])}
+    for n, kd in kernels.items():
+        if n in model:
+            kd["tflops"] = model[n]["flops"] / (kd["ms_per_launch"] * 1e-3) / 1e12
+            kd["alg_gbs"] = model[n]["bytes"] / (kd["ms_per_launch"] * 1e-3) / 1e9
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        smp = OracleSample(w)
+        n_tiles = smp.calibrate(15.0)
+        tk, dt = smp.run(n_tiles)
+        cpu = {"value": tk / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"float64 oracle fwd+bwd on {n_tiles} of {w.n_tiles} query tiles of 1 of {w.H} heads "
+                         f"({dt:.1f} s), scaled to the full batch"}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "shape": w.describe(), "global_batch": w.B * world,
+                       "seq_len": w.N, "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (Q, K, V, dO: 4 x %.0f MB)" % (q.numel() * 2 / 1e6)},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clk.summary(),
+            "north_star_roofline": north_star_roofline(w, peaks, ms_step),
+            "kernels": kernels}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -28,7 +28,8 @@
  *
  * Conventions shared by every entry point:
  *   - Ownership: the caller owns every buffer and stream.  The library never
- *     allocates or frees device memory and keeps no state between calls.
+ *     allocates or frees device memory and keeps no state between calls
+ *     (apart from the opt-in profiler below).
  *   - Pointers: all tensor pointers are DEVICE pointers, 16-byte aligned,
  *     except where a function says otherwise.
  *   - Layout: Q, K, V, O, dO, dQ, dK, dV are contiguous row-major [B, H, N, d]
@@ -140,6 +141,17 @@ ELSAA_API elsaa_status elsaa_debug_select(const elsaa_params* params, const void
  * the start of `workspace`.  Returns ELSAA_ERR_TIMEOUT if a kernel gave up a
  * bounded wait since the last check, else ELSAA_OK (or ELSAA_ERR_CUDA). */
 ELSAA_API elsaa_status elsaa_check_device_flags(void* workspace, void* stream);
+
+/* Opt-in kernel timing.  After elsaa_profile_begin() every kernel the library
+ * launches (from any thread, on any stream) is bracketed by two CUDA events
+ * recorded on its launch stream.  elsaa_profile_end() waits for those events,
+ * turns profiling off and reports, per kernel name, the summed device time in
+ * milliseconds and the number of launches; it fills at most max_entries rows of
+ * the caller's arrays (names point to static strings) and returns the number of
+ * rows, or -1 on a CUDA error.  Profiling is the only state the library keeps
+ * between calls; it holds up to 16384 launches per session. */
+ELSAA_API elsaa_status elsaa_profile_begin(void);
+ELSAA_API int elsaa_profile_end(const char** names, double* total_ms, int* launches, int max_entries);
 
 /* Static English name of a status code. */
 ELSAA_API const char* elsaa_status_string(elsaa_status status);

@@ -152,17 +152,18 @@ def _tile_keys(idx_row: np.ndarray, p: Params) -> np.ndarray:
     return np.concatenate(ks) if ks else np.zeros(0, dtype=np.int64)
 
 
-def sparse_branch(q, k, v, idx, p: Params):
+def sparse_branch(q, k, v, idx, p: Params, tiles=None):
     """O_s[i] = sum_j e^{z_ij} v_j / d_s[i], d_s[i] = sum_j e^{z_ij}, j in Omega_i.
 
     z_ij = scale * q_i . k_j.  Returns (O_s, log d_s); an empty support gives
-    O_s = 0 and log d_s = -inf.
+    O_s = 0 and log d_s = -inf.  ``tiles`` restricts the work to those query
+    tiles (other rows are left empty); used only to time a bounded sample.
     """
     N, d = q.shape
     T = p.block_size
     O_s = np.zeros((N, d))
     logd = np.full(N, -np.inf)
-    for t in range(p.n_tiles):
+    for t in (range(p.n_tiles) if tiles is None else tiles):
         rows = np.arange(t * T, min(N, (t + 1) * T))
         keys = _tile_keys(idx[t], p)
         if keys.size == 0:
@@ -291,16 +292,17 @@ def fuse(O_s, logd_s, O_lr, d_lr, p: Params, lam=None, g_s=None, g_lr=None):
 # Whole operator, one head, then [B, H] batches
 # ----------------------------------------------------------------------------
 
-def forward_head(q, k, v, W, p: Params, lam=None, g_s=None, g_lr=None, scores=None):
+def forward_head(q, k, v, W, p: Params, lam=None, g_s=None, g_lr=None, scores=None, tiles=None):
     """One attention head [ELSAA §3: the method is defined per head].
 
     ``scores`` replaces the block scores (used to feed the selector an external
-    score array).  Returns a dict with O, O_s, logd_s, O_lr, d_lr, m, idx, scores.
+    score array).  ``tiles`` limits the sparse branch to those query tiles (a
+    timing sample).  Returns a dict with O, O_s, logd_s, O_lr, d_lr, m, idx, scores.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     sc = block_scores(q, k, p) if scores is None else _f64(scores)
     idx = select_from_scores(sc, p.topk, p.causal)
-    O_s, logd = sparse_branch(q, k, v, idx, p)
+    O_s, logd = sparse_branch(q, k, v, idx, p, tiles)
     O_lr, d_lr = race_branch(q, k, v, W, p)
     O, m = fuse(O_s, logd, O_lr, d_lr, p, lam, g_s, g_lr)
     return dict(O=O, O_s=O_s, logd_s=logd, O_lr=O_lr, d_lr=d_lr, m=m, idx=idx, scores=sc)
@@ -377,8 +379,11 @@ def race_features_backward(X, W, p: Params, dPhi):
     return np.where((nrm > NORM_FLOOR)[:, None], (du - u * proj) / n[:, None], du / n[:, None])
 
 
-def backward_head(q, k, v, W, dO, fw, p: Params, lam=None, g_s=None, g_lr=None):
-    """(dq, dk, dv) for one head, given the forward dict ``fw``."""
+def backward_head(q, k, v, W, dO, fw, p: Params, lam=None, g_s=None, g_lr=None, tiles=None):
+    """(dq, dk, dv) for one head, given the forward dict ``fw``.
+
+    The gradient is a sum of contributions generated by each query tile;
+    ``tiles`` keeps only those tiles' contributions (a timing sample)."""
     q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
     N, d = q.shape
     T = p.block_size
@@ -389,7 +394,8 @@ def backward_head(q, k, v, W, dO, fw, p: Params, lam=None, g_s=None, g_lr=None):
     # sparse branch: P_ij = e^{z_ij}/d_s, dz_ij = P_ij (<dO_s,i, v_j> - Delta_i),
     # Delta_i = <dO_s,i, O_s,i> - dd_s,i d_s,i
     Delta = (dOs * fw["O_s"]).sum(axis=1) - dds_ds
-    for t in range(p.n_tiles):
+    tile_list = list(range(p.n_tiles)) if tiles is None else list(tiles)
+    for t in tile_list:
         rows = np.arange(t * T, min(N, (t + 1) * T))
         keys = _tile_keys(fw["idx"][t], p)
         if keys.size == 0:
@@ -412,7 +418,7 @@ def backward_head(q, k, v, W, dO, fw, p: Params, lam=None, g_s=None, g_lr=None):
         PhiK = race_features(k, W, p)
         dPhiQ = np.zeros_like(PhiQ)
         dPhiK = np.zeros_like(PhiK)
-        for t in range(p.n_tiles):
+        for t in tile_list:
             rows = np.arange(t * T, min(N, (t + 1) * T))
             keys = np.arange(rows[-1] + 1) if p.causal else np.arange(N)
             mask = (keys[None, :] <= rows[:, None]) if p.causal else np.ones((rows.size, keys.size), bool)

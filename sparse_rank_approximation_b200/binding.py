@@ -28,7 +28,7 @@ ELSAA_DTYPE_BF16 = 1
 
 EXPORTED = ("elsaa_saved_bytes", "elsaa_workspace_bytes", "elsaa_forward", "elsaa_backward",
             "elsaa_debug_select", "elsaa_check_device_flags", "elsaa_status_string",
-            "elsaa_last_error_message")
+            "elsaa_last_error_message", "elsaa_profile_begin", "elsaa_profile_end")
 
 
 class Params(ctypes.Structure):
@@ -74,6 +74,11 @@ def lib() -> ctypes.CDLL:
     L.elsaa_status_string.restype = ctypes.c_char_p
     L.elsaa_last_error_message.argtypes = []
     L.elsaa_last_error_message.restype = ctypes.c_char_p
+    L.elsaa_profile_begin.argtypes = []
+    L.elsaa_profile_begin.restype = i32
+    L.elsaa_profile_end.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
+                                    ctypes.POINTER(ctypes.c_int), i32]
+    L.elsaa_profile_end.restype = i32
     _lib = L
     return L
 
@@ -161,6 +166,21 @@ class Elsaa:
 
     def check_device_flags(self, stream=None) -> int:
         return lib().elsaa_check_device_flags(_ptr(self.ws), _stream(stream))
+
+
+def profile_begin() -> None:
+    _check(lib().elsaa_profile_begin(), "elsaa_profile_begin")
+
+
+def profile_end(max_entries: int = 64) -> dict:
+    """{kernel name: (total device ms, launches)} since profile_begin()."""
+    names = (ctypes.c_char_p * max_entries)()
+    ms = (ctypes.c_double * max_entries)()
+    cnt = (ctypes.c_int * max_entries)()
+    n = lib().elsaa_profile_end(names, ms, cnt, max_entries)
+    if n < 0:
+        _check(ELSAA_ERR_CUDA, "elsaa_profile_end")
+    return {names[i].decode(): (ms[i], cnt[i]) for i in range(n)}
 
 
 class ElsaaFunction(torch.autograd.Function):

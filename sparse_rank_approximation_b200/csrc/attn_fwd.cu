@@ -413,6 +413,7 @@ static cudaError_t launch_fwd_t(const FwdArgs& a, const Geom& g, cudaStream_t st
   auto kern = attn_fwd_bf16_kernel<D, T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  ProfScope ps("attn_fwd", st);
   kern<<<dim3(g.n_t, g.BH), 2 * T, smem, st>>>(
       (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K, (const __nv_bfloat16*)a.V, a.idx,
       (const __nv_bfloat16*)a.phiQ, (const __nv_bfloat16*)a.phiK, a.Ast, a.Bst, a.lam, a.gs, a.glr,

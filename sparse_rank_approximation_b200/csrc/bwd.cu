@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(256) row_scalars_kernel(BwdArgs a, Geom g) {
 cudaError_t launch_row_scalars(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st) {
   const int rpb = 256 / (g.d / 8);
   dim3 grid((g.N + rpb - 1) / rpb, g.BH);
+  ProfScope ps("row_scalars", st);
   if (bf16) row_scalars_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a, g);
   else row_scalars_kernel<float><<<grid, 256, 0, st>>>(a, g);
   return cudaGetLastError();
@@ -952,9 +953,11 @@ __global__ void __launch_bounds__(2 * T) sparse_dkdv_bf16_kernel(BwdArgs a, Geom
 }
 
 template <typename KernT>
-static cudaError_t launch2(KernT kern, size_t smem, int T, const BwdArgs& a, const Geom& g, cudaStream_t st) {
+static cudaError_t launch2(const char* name, KernT kern, size_t smem, int T, const BwdArgs& a, const Geom& g,
+                           cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  ProfScope ps(name, st);
   kern<<<dim3(g.n_t, g.BH), 2 * T, smem, st>>>(a, g);
   return cudaGetLastError();
 }
@@ -964,17 +967,17 @@ static cudaError_t bwd_t(const BwdArgs& a0, const Geom& g, cudaStream_t st) {
   BwdArgs a = a0;
   cudaError_t e;
   if (g.r > 0) {
-    e = launch2(race_q_bwd_bf16_kernel<D, T>, RaceBwdSmem<D, T>::bytes, T, a, g, st);
+    e = launch2("race_q_bwd", race_q_bwd_bf16_kernel<D, T>, RaceBwdSmem<D, T>::bytes, T, a, g, st);
     if (e != cudaSuccess) return e;
-    e = launch2(race_k_bwd_bf16_kernel<D, T>, RaceBwdSmem<D, T>::bytes, T, a, g, st);
+    e = launch2("race_k_bwd", race_k_bwd_bf16_kernel<D, T>, RaceBwdSmem<D, T>::bytes, T, a, g, st);
     if (e != cudaSuccess) return e;
   } else {
     a.dQacc = a.dKacc = a.dVacc = nullptr;
   }
   const size_t lds = (size_t)(D + 8) * 2;
-  e = launch2(sparse_dq_bf16_kernel<D, T>, (size_t)6 * T * lds, T, a, g, st);
+  e = launch2("sparse_dq", sparse_dq_bf16_kernel<D, T>, (size_t)6 * T * lds, T, a, g, st);
   if (e != cudaSuccess) return e;
-  return launch2(sparse_dkdv_bf16_kernel<D, T>, (size_t)6 * T * lds + (size_t)6 * T * 4, T, a, g, st);
+  return launch2("sparse_dkdv", sparse_dkdv_bf16_kernel<D, T>, (size_t)6 * T * lds + (size_t)6 * T * 4, T, a, g, st);
 }
 
 cudaError_t launch_bwd_bf16(const BwdArgs& a, const Geom& g, cudaStream_t st) {

@@ -6,7 +6,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/elsaa.h"
 #include "kernels.h"
@@ -207,9 +209,93 @@ elsaa_status cuda_status(cudaError_t e, const char* where) {
     if (_s != ELSAA_OK) return _s;        \
   } while (0)
 
+// ---- opt-in per-kernel profiler ------------------------------------------
+struct ProfRec {
+  const char* name;
+  int slot;
+};
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> ev;    // 2 events per slot, created on first use
+  std::vector<ProfRec> recs;
+  int used = 0;
+};
+Profiler& prof() {
+  static Profiler p;
+  return p;
+}
+constexpr int kMaxProfSlots = 16384;
+
 }  // namespace
 
+namespace elsaa {
+ProfScope::ProfScope(const char* name, cudaStream_t st) : slot(-1), stream(st) {
+  Profiler& p = prof();
+  if (!p.on) return;
+  std::lock_guard<std::mutex> lk(p.mu);
+  if (p.used >= kMaxProfSlots) return;
+  const int s = p.used;
+  while ((int)p.ev.size() < 2 * (s + 1)) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return;
+    p.ev.push_back(e);
+  }
+  p.used++;
+  slot = s;
+  p.recs.push_back({name, s});
+  cudaEventRecord(p.ev[2 * s], st);
+}
+ProfScope::~ProfScope() {
+  if (slot < 0) return;
+  cudaEventRecord(prof().ev[2 * slot + 1], stream);
+}
+}  // namespace elsaa
+
 extern "C" {
+
+elsaa_status elsaa_profile_begin(void) {
+  g_last_error.clear();
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> lk(p.mu);
+  p.recs.clear();
+  p.used = 0;
+  p.on = true;
+  return ELSAA_OK;
+}
+
+int elsaa_profile_end(const char** names, double* total_ms, int* launches, int max_entries) {
+  g_last_error.clear();
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> lk(p.mu);
+  p.on = false;
+  int n = 0;
+  for (const ProfRec& r : p.recs) {
+    if (cudaEventSynchronize(p.ev[2 * r.slot + 1]) != cudaSuccess) {
+      fail(ELSAA_ERR_CUDA, "profile event sync failed");
+      return -1;
+    }
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, p.ev[2 * r.slot], p.ev[2 * r.slot + 1]) != cudaSuccess) {
+      fail(ELSAA_ERR_CUDA, "profile event timing failed");
+      return -1;
+    }
+    int k = 0;
+    while (k < n && strcmp(names[k], r.name) != 0) ++k;
+    if (k == n) {
+      if (n >= max_entries) continue;
+      names[n] = r.name;
+      total_ms[n] = 0.0;
+      launches[n] = 0;
+      ++n;
+    }
+    total_ms[k] += ms;
+    launches[k] += 1;
+  }
+  p.recs.clear();
+  p.used = 0;
+  return n;
+}
 
 size_t elsaa_saved_bytes(const elsaa_params* p) {
   Geom g;

@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(256) attn_fwd_f32_kernel(FwdArgs a, Geom g) {
 }
 
 cudaError_t launch_attn_fwd_f32(const FwdArgs& a, const Geom& g, cudaStream_t st) {
+  ProfScope ps("attn_fwd_f32", st);
   attn_fwd_f32_kernel<<<dim3((g.N + 7) / 8, g.BH), 256, 0, st>>>(a, g);
   return cudaGetLastError();
 }
@@ -448,7 +449,11 @@ __global__ void __launch_bounds__(256) bwd_dkdv_f32_kernel(BwdArgs a, Geom g) {
 
 cudaError_t launch_bwd_f32(const BwdArgs& a, const Geom& g, cudaStream_t st) {
   const dim3 grid((g.N + 7) / 8, g.BH);
-  bwd_dq_f32_kernel<<<grid, 256, 0, st>>>(a, g);
+  {
+    ProfScope ps("bwd_dq_f32", st);
+    bwd_dq_f32_kernel<<<grid, 256, 0, st>>>(a, g);
+  }
+  ProfScope ps("bwd_dkdv_f32", st);
   bwd_dkdv_f32_kernel<<<grid, 256, 0, st>>>(a, g);
   return cudaGetLastError();
 }

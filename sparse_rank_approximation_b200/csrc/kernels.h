@@ -5,6 +5,16 @@
 
 namespace elsaa {
 
+// Opt-in per-kernel timing (elsaa_profile_begin / elsaa_profile_end): when
+// enabled, every kernel launch is bracketed by a pair of CUDA events recorded on
+// the launching stream.  Costs one branch per launch when disabled.
+struct ProfScope {
+  ProfScope(const char* name, cudaStream_t st);
+  ~ProfScope();
+  int slot;
+  cudaStream_t stream;
+};
+
 struct FwdArgs {
   const void *Q, *K, *V;
   const int* idx;

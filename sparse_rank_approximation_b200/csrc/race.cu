@@ -381,6 +381,7 @@ cudaError_t launch_race_features(const void* Q, const void* K, const float* W, b
                                  float* hQ, float* hK, float* nQ, float* nK, const Geom& g, cudaStream_t st) {
   if (g.r == 0) return cudaSuccess;
   if (!bf16) {
+    ProfScope ps("race_features_f32", st);
     race_features_f32_kernel<<<dim3((g.N + 7) / 8, g.BH, 2), 256, 0, st>>>(
         (const float*)Q, (const float*)K, W, (float*)phiQ, (float*)phiK, hQ, hK, nQ, nK, g);
     return cudaGetLastError();
@@ -389,6 +390,7 @@ cudaError_t launch_race_features(const void* Q, const void* K, const float* W, b
   auto run = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    ProfScope ps("race_features", st);
     kern<<<dim3((g.N + 63) / 64, g.BH, 2), 128, smem, st>>>(
         (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, W, (__nv_bfloat16*)phiQ, (__nv_bfloat16*)phiK, hQ, hK,
         nQ, nK, g);
@@ -403,6 +405,7 @@ static cudaError_t run_state(const void* phi, const void* Y, const float* rsc, c
                              float* Atot, float* Bpart, const Geom& g, cudaStream_t st) {
   if (!bf16) {
     const int n = g.r * g.dp;
+    ProfScope ps(BWD ? "race_state_bwd_f32" : "race_state_fwd_f32", st);
     race_state_f32_kernel<BWD><<<dim3(g.n_seg, g.BH, (n + 255) / 256), 256, 0, st>>>(
         (const float*)phi, (const float*)Y, rsc, rex, Atot, Bpart, g);
   } else {
@@ -410,6 +413,7 @@ static cudaError_t run_state(const void* phi, const void* Y, const float* rsc, c
     auto go = [&](auto kern) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
+      ProfScope ps(BWD ? "race_state_bwd" : "race_state_fwd", st);
       kern<<<dim3(g.n_seg, g.BH), 32 * (g.r / 16), smem, st>>>(
           (const __nv_bfloat16*)phi, (const __nv_bfloat16*)Y, rsc, rex, Atot, Bpart, g);
       return cudaGetLastError();
@@ -421,7 +425,10 @@ static cudaError_t run_state(const void* phi, const void* Y, const float* rsc, c
     else e = go(race_state_bf16_kernel<128, 128, BWD>);
     if (e != cudaSuccess) return e;
   }
-  race_scan_kernel<<<dim3((g.r * g.dp + 255) / 256, g.BH), 256, 0, st>>>(Atot, g, BWD ? 1 : 0);
+  {
+    ProfScope ps(BWD ? "race_scan_bwd" : "race_scan_fwd", st);
+    race_scan_kernel<<<dim3((g.r * g.dp + 255) / 256, g.BH), 256, 0, st>>>(Atot, g, BWD ? 1 : 0);
+  }
   return cudaGetLastError();
 }
 

@@ -207,14 +207,24 @@ __global__ void __launch_bounds__(256) invert_selection_kernel(const int* __rest
 
 cudaError_t launch_select(const void* Q, const void* K, bool bf16, double* qbar, double* kbar, float* scores,
                           int* idx, const Geom& g, cudaStream_t st) {
-  if (bf16)
-    pool_means_kernel<__nv_bfloat16><<<dim3(g.n_t, g.BH, 2), 128, 0, st>>>(
-        (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, qbar, kbar, g);
-  else
-    pool_means_kernel<float><<<dim3(g.n_t, g.BH, 2), 128, 0, st>>>((const float*)Q, (const float*)K, qbar, kbar, g);
+  {
+    ProfScope ps("pool_means", st);
+    if (bf16)
+      pool_means_kernel<__nv_bfloat16><<<dim3(g.n_t, g.BH, 2), 128, 0, st>>>(
+          (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, qbar, kbar, g);
+    else
+      pool_means_kernel<float><<<dim3(g.n_t, g.BH, 2), 128, 0, st>>>((const float*)Q, (const float*)K, qbar, kbar,
+                                                                       g);
+  }
   const int nb = (g.n_t + 31) / 32;
-  block_scores_kernel<<<dim3(nb, nb, g.BH), dim3(32, 8), 0, st>>>(qbar, kbar, scores, g);
-  if (g.k > 0) topk_kernel<<<dim3((g.n_t + 7) / 8, g.BH), 256, 0, st>>>(scores, idx, g);
+  {
+    ProfScope ps("block_scores", st);
+    block_scores_kernel<<<dim3(nb, nb, g.BH), dim3(32, 8), 0, st>>>(qbar, kbar, scores, g);
+  }
+  if (g.k > 0) {
+    ProfScope ps("topk", st);
+    topk_kernel<<<dim3((g.n_t + 7) / 8, g.BH), 256, 0, st>>>(scores, idx, g);
+  }
   return cudaGetLastError();
 }
 
@@ -223,6 +233,7 @@ cudaError_t launch_invert_selection(const int* idx, int* offs, int* tiles, const
   cudaError_t e = cudaFuncSetAttribute(invert_selection_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
+  ProfScope ps("invert_selection", st);
   invert_selection_kernel<<<g.BH, 256, smem, st>>>(idx, offs, tiles, g);
   return cudaGetLastError();
 }
