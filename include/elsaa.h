@@ -137,6 +137,27 @@ ELSAA_API elsaa_status elsaa_debug_select(const elsaa_params* params, const void
                                 float* scores, int32_t* idx,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* Selection with no caller scratch and no allocation (the paper has no
+ * counterpart; this is a deployment convenience).  Same result as the idx
+ * output of elsaa_debug_select, for callers that cannot allocate device memory
+ * when they need it: code inside a region being captured into a CUDA graph,
+ * programs whose device memory is reserved up front by a pool or another
+ * framework, and runtimes that forbid allocation after start-up.
+ *   Q, K    in   [B,H,N,d] dtype, device pointers
+ *   idx     out  int32 [B, H, n_t, topk] (device), as elsaa_debug_select
+ * The pooled means and block scores live in one static device array of
+ * 16 MiB compiled into the library, which every GPU that loads the library
+ * holds until the process exits.  A problem needing more,
+ * B*H*n_t*(16*d + 4*n_t) bytes plus alignment (n_t = ceil(N / block_size)),
+ * is rejected with ELSAA_ERR_UNSUPPORTED before any launch.  The first call on
+ * each device resolves the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.  All
+ * calls share the array: calls whose work can overlap on the GPU (other
+ * streams, other host threads on the same device) race and must be
+ * serialised by the caller.  The function allocates and frees nothing. */
+ELSAA_API elsaa_status elsaa_select_noalloc(const elsaa_params* params, const void* Q, const void* K,
+                                           int32_t* idx, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error flag kept at
  * the start of `workspace`.  Returns ELSAA_ERR_TIMEOUT if a kernel gave up a
  * bounded wait since the last check, else ELSAA_OK (or ELSAA_ERR_CUDA). */

@@ -28,7 +28,7 @@ ELSAA_DTYPE_BF16 = 1
 
 EXPORTED = ("elsaa_saved_bytes", "elsaa_workspace_bytes", "elsaa_forward", "elsaa_backward",
             "elsaa_debug_select", "elsaa_check_device_flags", "elsaa_status_string",
-            "elsaa_last_error_message", "elsaa_profile_begin", "elsaa_profile_end")
+            "elsaa_last_error_message", "elsaa_profile_begin", "elsaa_profile_end", "elsaa_select_noalloc")
 
 
 class Params(ctypes.Structure):
@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
     L.elsaa_profile_end.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
                                     ctypes.POINTER(ctypes.c_int), i32]
     L.elsaa_profile_end.restype = i32
+    L.elsaa_select_noalloc.argtypes = [P, vp, vp, vp, vp]
+    L.elsaa_select_noalloc.restype = i32
     _lib = L
     return L
 

@@ -230,6 +230,8 @@ constexpr int kMaxProfSlots = 16384;
 }  // namespace
 
 namespace elsaa {
+void record_error(const char* msg) { g_last_error = msg; }
+
 ProfScope::ProfScope(const char* name, cudaStream_t st) : slot(-1), stream(st) {
   Profiler& p = prof();
   if (!p.on) return;

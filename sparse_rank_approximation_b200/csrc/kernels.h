@@ -51,6 +51,9 @@ struct BwdArgs {
   void *dQ, *dK, *dV;
 };
 
+// Sets the message elsaa_last_error_message() returns on this thread.
+void record_error(const char* msg);
+
 cudaError_t launch_select(const void* Q, const void* K, bool bf16, double* qbar, double* kbar, float* scores,
                           int* idx, const Geom& g, cudaStream_t st);
 cudaError_t launch_invert_selection(const int* idx, int* offs, int* tiles, const Geom& g, cudaStream_t st);
