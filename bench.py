@@ -103,6 +103,24 @@ def north_star_roofline(w, peaks, t_step_ms):
 
 
 # --------------------------------------------------------------------------
+# Multi-rank plumbing: each rank runs its own batch; the only collectives are a
+# barrier around the timed region and the max-reduce of the elapsed time.
+# --------------------------------------------------------------------------
+
+def max_over_ranks(value: float, device=None) -> float:
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of the batch a rank processes (independent problems per rank)."""
+    return rank
+
+
+# --------------------------------------------------------------------------
 
 class ClockSampler:
     """nvidia-smi sampling (every 100 ms) while the timed region runs."""
@@ -289,7 +307,7 @@ def main():
 
     from sparse_rank_approximation_b200 import binding as bd
     peaks, peak_kind = load_peaks()
-    inp = make_inputs(w, seed=rank)
+    inp = make_inputs(w, seed=rank_seed(rank))
     key = "16" if w.dtype == "bf16" else ""
     q, k, v, dO = (inp[n + key].to(dev) for n in ("Q", "K", "V", "dO"))
     W = inp["W"].to(dev)
@@ -325,11 +343,7 @@ def main():
         barrier()
         clk.mark(False)
         prof = bd.profile_end()
-    ms_total = ev0.elapsed_time(ev1)
-    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), dev)
     ms_step = ms_total / args.steps
     tokens_step = w.B * w.N * world
     value = tokens_step / (ms_step * 1e-3)
@@ -364,11 +378,9 @@ def main():
             e2e_step()
         e1.record(stream)
         barrier()
-        te = torch.tensor([e0.elapsed_time(e1) / n_e2e], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": tokens_step / (float(te.item()) * 1e-3), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": float(te.item())}
+        te = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dev)
+        e2e = {"value": tokens_step / (te * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": te}
 
     if world > 1:
         dist.destroy_process_group()
