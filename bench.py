@@ -286,10 +286,15 @@ def main():
     ap.add_argument("--impl", default="elsaa", choices=["elsaa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with this many heads (a smaller case for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
