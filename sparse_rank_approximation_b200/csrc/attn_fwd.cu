@@ -245,19 +245,38 @@ __global__ void __launch_bounds__(2 * T) attn_fwd_bf16_kernel(
       load_feat(sFa, fq, rc, rcw);
       cp_async_commit();
       const int q4 = DP / 4;
-      for (int i = tid; i < rcw * q4; i += NT) {
-        const int r = i / q4, c = (i % q4) * 4;
-        float4 v = *reinterpret_cast<const float4*>(pa + (size_t)(rc + r) * DP + c);
-        if (pb) {
-          const float4 w = *reinterpret_cast<const float4*>(pb + (size_t)(rc + r) * DP + c);
-          v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-        }
-        const float vv[4] = {v.x, v.y, v.z, v.w};
+      const int total = rcw * q4;
+      // loads batched 4 deep per thread before conversion, so their latencies overlap
+#pragma unroll 1
+      for (int i0 = tid; i0 < total; i0 += 4 * NT) {
+        float4 v[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const __nv_bfloat16 hi = __float2bfloat16_rn(vv[j]);
-          sPh[r * LDV1 + c + j] = hi;
-          sPl[r * LDV1 + c + j] = __float2bfloat16_rn(vv[j] - __bfloat162float(hi));
+        for (int k = 0; k < 4; ++k) {
+          const int i = i0 + k * NT;
+          v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (i < total) {
+            const int r = i / q4, c = (i % q4) * 4;
+            v[k] = __ldg(reinterpret_cast<const float4*>(pa + (size_t)(rc + r) * DP + c));
+            if (pb) {
+              const float4 w = __ldg(reinterpret_cast<const float4*>(pb + (size_t)(rc + r) * DP + c));
+              v[k].x += w.x; v[k].y += w.y; v[k].z += w.z; v[k].w += w.w;
+            }
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int i = i0 + k * NT;
+          if (i >= total) break;
+          const int r = i / q4, c = (i % q4) * 4;
+          const float vv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+          __align__(8) __nv_bfloat16 hi[4], lo[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            hi[j] = __float2bfloat16_rn(vv[j]);
+            lo[j] = __float2bfloat16_rn(vv[j] - __bfloat162float(hi[j]));
+          }
+          *reinterpret_cast<uint2*>(sPh + r * LDV1 + c) = *reinterpret_cast<const uint2*>(hi);
+          *reinterpret_cast<uint2*>(sPl + r * LDV1 + c) = *reinterpret_cast<const uint2*>(lo);
         }
       }
       cp_async_wait<0>();

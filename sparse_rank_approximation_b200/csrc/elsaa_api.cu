@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -190,6 +191,12 @@ BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
   return w;
 }
 
+// ELSAA_DISABLE_TCGEN05=1 selects the mma.sync kernels everywhere (for A/B checks).
+bool tcgen05_disabled() {
+  const char* v = getenv("ELSAA_DISABLE_TCGEN05");
+  return v && v[0] == '1';
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 elsaa_status check_ptr(const void* p, const char* name, bool required = true) {
@@ -349,8 +356,14 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
                         "race features"));
   ELSAA_TRY(cuda_status(launch_race_state_fwd(s.phiK, V, bf16, s.Ast, s.Bst, g, st_), "race summaries"));
   FwdArgs a{Q, K, V, s.idx, s.phiQ, s.phiK, s.Ast, s.Bst, lam, gs, glr, O, s.Os, s.logd, s.dlr, s.m, s.Olr};
-  if (bf16) ELSAA_TRY(cuda_status(launch_attn_fwd_bf16(a, g, st_), "fused forward"));
-  else ELSAA_TRY(cuda_status(launch_attn_fwd_f32(a, g, st_), "fused forward"));
+  if (bf16 && attn_fwd_tc_supported(g) && !tcgen05_disabled()) {
+    ELSAA_TRY(cuda_status(launch_race_readout_bf16(a, g, st_), "race read-out"));
+    ELSAA_TRY(cuda_status(launch_attn_fwd_tc(a, g, w.flag, st_), "tcgen05 forward"));
+  } else if (bf16) {
+    ELSAA_TRY(cuda_status(launch_attn_fwd_bf16(a, g, st_), "fused forward"));
+  } else {
+    ELSAA_TRY(cuda_status(launch_attn_fwd_f32(a, g, st_), "fused forward"));
+  }
   return ELSAA_OK;
 }
 

@@ -65,8 +65,15 @@ cudaError_t launch_race_state_fwd(const void* phiK, const void* V, bool bf16, fl
 // Backward suffix statistics of Phi(q_i) [cl_i dO_i ; delta_i]^T.
 cudaError_t launch_race_state_bwd(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st);
 cudaError_t launch_attn_fwd_bf16(const FwdArgs& a, const Geom& g, cudaStream_t st);
+// tcgen05 sparse-branch forward + fusion epilogue (d = 128, block 128); reads the
+// low-rank output written by launch_race_readout_bf16.
+bool attn_fwd_tc_supported(const Geom& g);
+cudaError_t launch_attn_fwd_tc(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
+cudaError_t launch_race_readout_bf16(const FwdArgs& a, const Geom& g, cudaStream_t st);
 cudaError_t launch_attn_fwd_f32(const FwdArgs& a, const Geom& g, cudaStream_t st);
 cudaError_t launch_row_scalars(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st);
+// RACE backward (bf16): low-rank parts of dQ, dK, dV into the fp32 accumulators.
+cudaError_t launch_race_bwd_bf16(const BwdArgs& a, const Geom& g, cudaStream_t st);
 cudaError_t launch_bwd_bf16(const BwdArgs& a, const Geom& g, cudaStream_t st);
 cudaError_t launch_bwd_f32(const BwdArgs& a, const Geom& g, cudaStream_t st);
 

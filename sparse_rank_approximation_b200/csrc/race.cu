@@ -43,8 +43,11 @@ __global__ void __launch_bounds__(128) race_features_bf16_kernel(
   const int side = blockIdx.z;
   const __nv_bfloat16* X = (side == 0 ? Q : K) + (size_t)blockIdx.y * g.N * D;
   __nv_bfloat16* phi = (side == 0 ? phiQ : phiK) + (size_t)blockIdx.y * g.N * g.r;
-  float* hout = (side == 0 ? hQ : hK) + (size_t)blockIdx.y * g.N * NH;
-  float* nout = (side == 0 ? nQ : nK) + (size_t)blockIdx.y * g.N;
+  // h and the norms are only kept when the caller asks (the bf16 backward recomputes them)
+  float* hout = (side == 0 ? hQ : hK);
+  float* nout = (side == 0 ? nQ : nK);
+  if (hout) hout += (size_t)blockIdx.y * g.N * NH;
+  if (nout) nout += (size_t)blockIdx.y * g.N;
   const int row_base = blockIdx.x * 64;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -112,7 +115,7 @@ __global__ void __launch_bounds__(128) race_features_bf16_kernel(
 #pragma unroll
     for (int b = 0; b < kHashBits; ++b) {
       const float h = sH[r * (NW + 1) + l * kHashBits + b] * inv_n;
-      hout[(size_t)row * NH + l * kHashBits + b] = h;
+      if (hout) hout[(size_t)row * NH + l * kHashBits + b] = h;
       const float y = two_over_tau * h;
       sp[b] = 1.f / (1.f + expf(-y));   // P(c_b = +1)
       sm[b] = 1.f / (1.f + expf(y));    // P(c_b = -1)
@@ -128,7 +131,7 @@ __global__ void __launch_bounds__(128) race_features_bf16_kernel(
     uint4* dst = reinterpret_cast<uint4*>(phi + (size_t)row * g.r + l * kCorners);
     dst[0] = reinterpret_cast<const uint4*>(out)[0];
     dst[1] = reinterpret_cast<const uint4*>(out)[1];
-    if (l == 0) nout[row] = sN[r];
+    if (l == 0 && nout) nout[row] = sN[r];
   }
 }
 
@@ -392,8 +395,8 @@ cudaError_t launch_race_features(const void* Q, const void* K, const float* W, b
     if (e != cudaSuccess) return e;
     ProfScope ps("race_features", st);
     kern<<<dim3((g.N + 63) / 64, g.BH, 2), 128, smem, st>>>(
-        (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, W, (__nv_bfloat16*)phiQ, (__nv_bfloat16*)phiK, hQ, hK,
-        nQ, nK, g);
+        (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, W, (__nv_bfloat16*)phiQ, (__nv_bfloat16*)phiK, nullptr,
+        nullptr, nullptr, nullptr, g);
     return cudaGetLastError();
   };
   if (g.d == 64) return run(race_features_bf16_kernel<64>);

@@ -76,10 +76,11 @@ def test_forward_backward_small(name):
             check(w, f"dV[{b},{h}]", np64(grads[2][b, h]), dv)
 
 
-@pytest.mark.parametrize("case", ["k0", "r0_eps0", "lam_gates", "tau_lam"])
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_branch_switches_and_options(case, dtype):
-    base = dict(N=64 * 4 + 20, d=64, block_size=64, topk=2, rank_r=32, dtype=dtype, H=2)
+@pytest.mark.parametrize("case", ["k0", "r0_eps0", "lam_gates", "tau_lam", "noncausal"])
+@pytest.mark.parametrize("geom", ["bf16_d64_T64", "bf16_d128_T128", "f32_d64_T64"])
+def test_branch_switches_and_options(case, geom):
+    dtype, d, T = geom.split("_")[0], int(geom.split("_")[1][1:]), int(geom.split("_")[2][1:])
+    base = dict(N=T * 3 + 20, d=d, block_size=T, topk=2, rank_r=32, dtype=dtype, H=2)
     kw, over, lam_vec, gates = {}, {}, False, False
     if case == "k0":
         base["topk"] = 0
@@ -90,6 +91,8 @@ def test_branch_switches_and_options(case, dtype):
         lam_vec = gates = True
     elif case == "tau_lam":
         over.update(tau=0.5, lam=3.0, eps=0.01)
+    elif case == "noncausal":
+        base["causal"] = False
     w = small_workload(**base)
     inp, extra, O, scores, idx, grads = _run(w, lam_vec=lam_vec, gates=gates, **over)
     for h in range(w.H):
