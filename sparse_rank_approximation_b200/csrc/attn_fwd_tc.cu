@@ -30,16 +30,22 @@ constexpr uint32_t kTile = 2 * kSlab;    // 128 x 128 bf16
 constexpr uint32_t OFF_Q = 0;
 __host__ __device__ constexpr uint32_t off_k(int s) { return kTile * (1 + 2 * s); }   // K stage s
 __host__ __device__ constexpr uint32_t off_v(int s) { return kTile * (2 + 2 * s); }   // V stage s
-constexpr uint32_t OFF_P = 5 * kTile;
-constexpr uint32_t OFF_MISC = 6 * kTile;
+__host__ __device__ constexpr uint32_t off_p(int b) { return kTile * (5 + b); }      // P buffer b
+constexpr uint32_t OFF_MISC = 7 * kTile;
 constexpr size_t kSmemBytes = OFF_MISC + 512 + 1024;     // + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t TM_O = 0;
 __host__ __device__ constexpr uint32_t tm_s(int s) { return 128u + 128u * s; }        // score buffer s
 constexpr float kRescaleThreshold = 8.f;                 // log2 units
 
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
 struct Misc {
-  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, pv_done, drain;
+  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full[2], pv_done[2], drain;
   uint32_t tmem_base;
   int abort_flag;
   int idx[32];
@@ -77,9 +83,9 @@ __global__ void __launch_bounds__(192, 1)
       tc::mbar_init(&ms->kv_empty[s], 1);
       tc::mbar_init(&ms->s_full[s], 1);
       tc::mbar_init(&ms->s_free[s], 128);
+      tc::mbar_init(&ms->p_full[s], 128);
+      tc::mbar_init(&ms->pv_done[s], 1);
     }
-    tc::mbar_init(&ms->p_full, 128);
-    tc::mbar_init(&ms->pv_done, 1);
     tc::mbar_init(&ms->drain, 1);
     ms->abort_flag = 0;
     tc::fence_barrier_init();
@@ -127,17 +133,18 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = wait_or_abort(&ms->q_full, 0, ms, err, 2u);
       int pv_issued = 0;
       auto issue_pv = [&](int jj) -> bool {
-        if (!wait_or_abort(&ms->p_full, jj & 1, ms, err, 4u)) return false;
+        if (!wait_or_abort(&ms->p_full[jj & 1], (jj >> 1) & 1, ms, err, 4u)) return false;
         tc::tc_fence_after();
         const uint32_t vb = sbase + off_v(jj & 1);
+        const uint32_t pb = sbase + off_p(jj & 1);
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk) {
-          const uint64_t ad = tc::sw128_desc(sbase + OFF_P + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
+          const uint64_t ad = tc::sw128_desc(pb + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = tc::sw128_desc(vb + kk * 2048, kSlab, 1024);
           tc::mma_bf16(tmem + TM_O, ad, bd, idPV, (jj > 0 || kk > 0) ? 1u : 0u);
         }
         tc::mma_commit(&ms->kv_empty[jj & 1]);
-        tc::mma_commit(&ms->pv_done);
+        tc::mma_commit(&ms->pv_done[jj & 1]);
         pv_issued = jj + 1;
         return true;
       };
@@ -167,7 +174,7 @@ __global__ void __launch_bounds__(192, 1)
     const int row = 32 * q4 + lane;
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
     const float sl2 = g.scale * kLog2e;
-    float m_used = -INFINITY, l = 0.f;
+    float m_used = -INFINITY, l = 0.f;     // running max (log2 units, scaled) and row sum
     bool ok = true;
     for (int j = 0; j < n_sel; ++j) {
       const int s = j & 1;
@@ -186,16 +193,21 @@ __global__ void __launch_bounds__(192, 1)
       tc::tc_fence_before();
       tc::mbar_arrive(&ms->s_free[s]);
       const int b = ms->idx[j];
-      const bool diag = g.causal && b == t;
       const int kvalid = g.N - b * kT;            // keys of this block inside the sequence
-      float mx = -INFINITY;
+      if ((g.causal && b == t) || kvalid < kT) {  // block-uniform: only the diagonal / ragged block masks
+        const int lim = min(kvalid - 1, (g.causal && b == t) ? row : kT - 1);
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float v = sv[c] * sl2;
-        if ((diag && c > row) || c >= kvalid) v = -INFINITY;
-        sv[c] = v;
-        mx = fmaxf(mx, v);
+        for (int c = 0; c < 128; ++c) sv[c] = c > lim ? -INFINITY : sv[c];
       }
+      float m4[4] = {sv[0], sv[1], sv[2], sv[3]};
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        m4[0] = fmaxf(m4[0], sv[c]);
+        m4[1] = fmaxf(m4[1], sv[c + 1]);
+        m4[2] = fmaxf(m4[2], sv[c + 2]);
+        m4[3] = fmaxf(m4[3], sv[c + 3]);
+      }
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
       // lazy rescaling: move the reference max only when the row max grew by > 2^8
       const float m_new = fmaxf(m_used, mx);
       const bool resc = m_new > m_used + kRescaleThreshold;     // false while both are -inf
@@ -205,51 +217,55 @@ __global__ void __launch_bounds__(192, 1)
         l *= alpha;
         m_used = m_new;
       }
-      // the P buffer and O must be clear of the previous block's PV product
-      if (j > 0) {
-        ok = wait_or_abort(&ms->pv_done, (j - 1) & 1, ms, err, 64u);
+      if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        // O holds the products through block j-1: wait for the last one, rescale (warp-collective)
+        ok = wait_or_abort(&ms->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ms, err, 64u);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc::tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {      // warp-collective O rescale in TMEM
 #pragma unroll
-          for (int c = 0; c < kD / 32; ++c) {
-            float tmp[32];
-            tc::tmem_ld32(tmem + lane_base + TM_O + 32 * c, tmp);
-            tc::tmem_wait_ld();
+        for (int c = 0; c < kD / 32; ++c) {
+          float tmp[32];
+          tc::tmem_ld32(tmem + lane_base + TM_O + 32 * c, tmp);
+          tc::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) tmp[i] *= alpha;
-            tc::tmem_st32(tmem + lane_base + TM_O + 32 * c, tmp);
-          }
-          tc::tmem_wait_st();
+          for (int i = 0; i < 32; ++i) tmp[i] *= alpha;
+          tc::tmem_st32(tmem + lane_base + TM_O + 32 * c, tmp);
         }
+        tc::tmem_wait_st();
+      }
+      // P buffer j&1 is free once the PV product of block j-2 has finished
+      if (j >= 2) {
+        ok = wait_or_abort(&ms->pv_done[s], ((j >> 1) + 1) & 1, ms, err, 256u);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       }
       const float msub = m_used == -INFINITY ? 0.f : m_used;
-      float rs = 0.f;
-      unsigned char* prow = smem + OFF_P + row * 128;
+      float rs0 = 0.f, rs1 = 0.f;
+      unsigned char* prow = smem + off_p(s) + row * 128;
 #pragma unroll
       for (int ch = 0; ch < 16; ++ch) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float p0 = exp2f(sv[8 * ch + 2 * e] - msub);
-          const float p1 = exp2f(sv[8 * ch + 2 * e + 1] - msub);
-          rs += p0 + p1;
+          const float p0 = ex2_approx(fmaf(sv[8 * ch + 2 * e], sl2, -msub));
+          const float p1 = ex2_approx(fmaf(sv[8 * ch + 2 * e + 1], sl2, -msub));
+          rs0 += p0;
+          rs1 += p1;
           w[e] = pack_bf16(p0, p1);
         }
         const int phys = (ch & 7) ^ (row & 7);
         *reinterpret_cast<uint4*>(prow + (ch >> 3) * kSlab + phys * 16) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      l += rs;
+      l += rs0 + rs1;
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
-      tc::mbar_arrive(&ms->p_full);
+      tc::mbar_arrive(&ms->p_full[s]);
     }
-    // ---- epilogue: O_s = O / l, log d_s, fusion (Eq. 5, Eq. 4), stores
+    // ---- epilogue: O_s = O / l, log d_s, fusion (Eq. 5, Eq. 4), coalesced stores via smem
     float o[kD];
 #pragma unroll
     for (int c = 0; c < kD; ++c) o[c] = 0.f;
     if (ok && n_sel > 0) {
-      ok = wait_or_abort(&ms->pv_done, (n_sel - 1) & 1, ms, err, 128u);
+      ok = wait_or_abort(&ms->pv_done[(n_sel - 1) & 1], ((n_sel - 1) >> 1) & 1, ms, err, 128u);
       if (__all_sync(0xffffffffu, ok)) {
         tc::tc_fence_after();
 #pragma unroll
@@ -264,23 +280,38 @@ __global__ void __launch_bounds__(192, 1)
         ok = false;
       }
     }
+    // every PV product is done (or abandoned): K/V stage 0 and both P buffers are free.
+    // Tiles are [128 rows][256 bytes] with 16-byte chunk c of row r stored at chunk c ^ (r & 15).
+    const int tid = threadIdx.x - 64;                      // 0..127 among the softmax warps
+    unsigned char* sLr = smem + off_p(0);
+    unsigned char* sO = smem + off_p(1);
+    unsigned char* sS = smem + off_k(0);
+    const int rows_here = min(kT, g.N - t * kT);
+    const __nv_bfloat16* olr_g = static_cast<const __nv_bfloat16*>(a.Olr) + (head + (size_t)t * kT) * kD;
+#pragma unroll 4
+    for (int i = tid; i < kT * 16; i += 128) {
+      const int r = i >> 4, c = i & 15;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < rows_here) v = *reinterpret_cast<const uint4*>(olr_g + (size_t)r * kD + c * 8);
+      *reinterpret_cast<uint4*>(sLr + r * 256 + ((c ^ (r & 15)) << 4)) = v;
+    }
+    asm volatile("bar.sync 1, 128;\n" ::: "memory");
     const int qrow = t * kT + row;
-    if (ok && qrow < g.N) {
+    float logd = -INFINITY, mf = 0.f;
+    if (qrow < g.N) {
       const size_t ri = head + qrow;
-      const float logd = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+      logd = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const float dl = a.dlr[ri];
       const float lam = a.lam ? a.lam[ri] : g.lam;
-      const float mf = logd == -INFINITY ? 0.f : 1.f / (1.f + (lam * dl + g.eps) * expf(-logd));
+      mf = logd == -INFINITY ? 0.f : 1.f / (1.f + (lam * dl + g.eps) * expf(-logd));
       const float gs = a.gs ? a.gs[ri] : 1.f;
       const float gl = a.glr ? a.glr[ri] : 1.f - mf;
       const float cs = gs * mf;
-      const uint4* olr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.Olr) + ri * kD);
-      uint4* out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + ri * kD);
-      uint4* outs = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.Os) + ri * kD);
 #pragma unroll
       for (int ch = 0; ch < kD / 8; ++ch) {
-        const uint4 lr = olr[ch];
+        const int off = row * 256 + ((ch ^ (row & 15)) << 4);
+        const uint4 lr = *reinterpret_cast<const uint4*>(sLr + off);
         const __nv_bfloat16* lv = reinterpret_cast<const __nv_bfloat16*>(&lr);
         uint32_t wo[4], ws[4];
 #pragma unroll
@@ -289,11 +320,25 @@ __global__ void __launch_bounds__(192, 1)
           ws[e] = pack_bf16(s0, s1);
           wo[e] = pack_bf16(cs * s0 + gl * __bfloat162float(lv[2 * e]), cs * s1 + gl * __bfloat162float(lv[2 * e + 1]));
         }
-        out[ch] = make_uint4(wo[0], wo[1], wo[2], wo[3]);
-        outs[ch] = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+        *reinterpret_cast<uint4*>(sO + off) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
+        *reinterpret_cast<uint4*>(sS + off) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
       }
       a.logd[ri] = logd;
       a.m[ri] = mf;
+    }
+    asm volatile("bar.sync 1, 128;\n" ::: "memory");
+    if (ok) {
+      __nv_bfloat16* o_g = static_cast<__nv_bfloat16*>(a.O) + (head + (size_t)t * kT) * kD;
+      __nv_bfloat16* s_g = static_cast<__nv_bfloat16*>(a.Os) + (head + (size_t)t * kT) * kD;
+#pragma unroll 4
+      for (int i = tid; i < kT * 16; i += 128) {
+        const int r = i >> 4, c = i & 15;
+        if (r < rows_here) {
+          const int off = r * 256 + ((c ^ (r & 15)) << 4);
+          *reinterpret_cast<uint4*>(o_g + (size_t)r * kD + c * 8) = *reinterpret_cast<const uint4*>(sO + off);
+          *reinterpret_cast<uint4*>(s_g + (size_t)r * kD + c * 8) = *reinterpret_cast<const uint4*>(sS + off);
+        }
+      }
     }
   }
   __syncthreads();
