@@ -12,7 +12,8 @@
 //   warps 3-10  softmax: each query row is split over two warps (64 score
 //               columns each) that exchange their partial row max; online
 //               softmax in fp32 with lazy rescaling (O and l are rescaled only
-//               when the running max grows by more than 2^8); P_j goes to one of
+//               when the running max grows by more than 2^16, after P_j is
+//               written and just before it is released); P_j goes to one of
 //               two shared buffers as bf16 in the swizzled K-major layout; the
 //               epilogue normalises O, applies the fusion and writes O and O_s
 //               through shared memory with TMA stores.
@@ -40,7 +41,7 @@ constexpr uint32_t OFF_MISC = 7 * kTile;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t TM_O = 0;
 __host__ __device__ constexpr uint32_t tm_s(int s) { return 128u + 128u * s; }         // score buffer s
-constexpr float kRescaleThreshold = 8.f;                 // log2 units
+constexpr float kRescaleThreshold = 16.f;                // log2 units: P stays below 2^16
 constexpr int kThreads = 352;
 constexpr int kSoftmaxThreads = 256;
 
@@ -279,24 +280,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           lp *= alpha;
           m_used = m_new;
         }
-        if (j > 0 && __any_sync(0xffffffffu, resc)) {
-          // O holds the products through block j-1: wait for the last one, rescale this half
-          alive = __all_sync(0xffffffffu,
-                             wait_or_abort(&ms->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ms, err, 64u));
-          if (alive) {
-            tc::tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              float tmp[32];
-              tc::tmem_ld32(tmem + lane_base + TM_O + 64 * half + 32 * c, tmp);
-              tc::tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) tmp[i] *= alpha;
-              tc::tmem_st32(tmem + lane_base + TM_O + 64 * half + 32 * c, tmp);
-            }
-            tc::tmem_wait_st();
-          }
-        }
         // P buffer j&1 is free once the PV product of block j-2 has finished
         if (alive && j >= 2)
           alive = __all_sync(0xffffffffu, wait_or_abort(&ms->pv_done[s], ((j >> 1) + 1) & 1, ms, err, 256u));
@@ -319,6 +302,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           lp += rs0 + rs1;
           tc::fence_proxy_async_smem();
+        }
+        // O holds the products through block j-1; a moved reference max rescales it (this half
+        // of the columns) once that product is done, before P_j is released to the MMA warp.
+        if (alive && j > 0 && __any_sync(0xffffffffu, resc)) {
+          alive = __all_sync(0xffffffffu,
+                             wait_or_abort(&ms->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ms, err, 64u));
+          if (alive) {
+            tc::tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              float tmp[32];
+              tc::tmem_ld32(tmem + lane_base + TM_O + 64 * half + 32 * c, tmp);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) tmp[i] *= alpha;
+              tc::tmem_st32(tmem + lane_base + TM_O + 64 * half + 32 * c, tmp);
+            }
+            tc::tmem_wait_st();
+          }
+        }
+        if (alive) {
           tc::tc_fence_before();
           tc::mbar_arrive(&ms->p_full[s]);
         }
