@@ -76,6 +76,8 @@ __global__ void __launch_bounds__(256) row_scalars_kernel(BwdArgs a, Geom g) {
   const double ddlr = D > 0.0 ? -dm * lam * ds / (D * D) : 0.0;
   a.rs.cs[i] = (float)cs;
   a.rs.Delta[i] = (float)(cs * A - dm * m * one_m);
+  if (a.rs.packed)
+    a.rs.packed[i] = make_float4((float)(logd * 1.4426950408889634), (float)cs, (float)(cs * A - dm * m * one_m), 0.f);
   a.rs.cl[i] = (float)cl;
   a.rs.delta[i] = (float)(ddlr - cl * Bv);
 }
@@ -433,26 +435,33 @@ static cudaError_t launch2(const char* name, KernT kern, size_t smem, int T, con
 }
 
 template <int D, int T>
-static cudaError_t bwd_t(const BwdArgs& a0, const Geom& g, cudaStream_t st) {
+static cudaError_t bwd_t(const BwdArgs& a0, const Geom& g, int parts, cudaStream_t st) {
   BwdArgs a = a0;
   cudaError_t e;
   if (g.r > 0) {
-    e = launch_race_bwd_bf16(a, g, st);
-    if (e != cudaSuccess) return e;
+    if (parts & 1) {
+      e = launch_race_bwd_bf16(a, g, st);
+      if (e != cudaSuccess) return e;
+    }
   } else {
     a.dQacc = a.dKacc = a.dVacc = nullptr;
   }
   const size_t lds = (size_t)(D + 8) * 2;
-  e = launch2("sparse_dq", sparse_dq_bf16_kernel<D, T>, (size_t)6 * T * lds, T, a, g, st);
-  if (e != cudaSuccess) return e;
-  return launch2("sparse_dkdv", sparse_dkdv_bf16_kernel<D, T>, (size_t)6 * T * lds + (size_t)6 * T * 4, T, a, g, st);
+  if (parts & 2) {
+    e = launch2("sparse_dq", sparse_dq_bf16_kernel<D, T>, (size_t)6 * T * lds, T, a, g, st);
+    if (e != cudaSuccess) return e;
+  }
+  if (parts & 4)
+    return launch2("sparse_dkdv", sparse_dkdv_bf16_kernel<D, T>, (size_t)6 * T * lds + (size_t)6 * T * 4, T, a, g, st);
+  return cudaSuccess;
 }
 
-cudaError_t launch_bwd_bf16(const BwdArgs& a, const Geom& g, cudaStream_t st) {
-  if (g.d == 64 && g.T == 64) return bwd_t<64, 64>(a, g, st);
-  if (g.d == 64 && g.T == 128) return bwd_t<64, 128>(a, g, st);
-  if (g.d == 128 && g.T == 64) return bwd_t<128, 64>(a, g, st);
-  if (g.d == 128 && g.T == 128) return bwd_t<128, 128>(a, g, st);
+// parts: bit 0 RACE backward, bit 1 sparse dQ, bit 2 sparse dK/dV (mma.sync kernels).
+cudaError_t launch_bwd_bf16(const BwdArgs& a, const Geom& g, int parts, cudaStream_t st) {
+  if (g.d == 64 && g.T == 64) return bwd_t<64, 64>(a, g, parts, st);
+  if (g.d == 64 && g.T == 128) return bwd_t<64, 128>(a, g, parts, st);
+  if (g.d == 128 && g.T == 64) return bwd_t<128, 64>(a, g, parts, st);
+  if (g.d == 128 && g.T == 128) return bwd_t<128, 128>(a, g, parts, st);
   return cudaErrorInvalidValue;
 }
 

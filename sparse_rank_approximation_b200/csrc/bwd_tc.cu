@@ -1,0 +1,344 @@
+// Sparse-branch backward on the 5th-generation tensor cores (tcgen05 + TMEM),
+// 128-query tiles, 128-key blocks, head dimension 128 (ELSAA paper §3.2 with the
+// Eq. 5 adjoint folded into the softmax delta):
+//   P_ij  = exp(z_ij - log d_s,i)            (z = scale q.k, j in the selected blocks)
+//   dz_ij = P_ij (cs_i <dO_i, v_j> - Delta_i)
+//   dq_i  = scale sum_j dz_ij k_j,  dk_j = scale sum_i dz_ij q_i,  dv_j = sum_i P_ij cs_i dO_i
+// plus the low-rank gradient parts accumulated in fp32 by the RACE backward.
+//
+// dq kernel: one CTA per (head, query tile); Q and dO stay in shared memory, the
+// selected K/V blocks stream through a 2-stage TMA ring; S = Q K^T and dP = dO V^T
+// land in TMEM, 8 softmax warps form dS (bf16, swizzled K-major) in shared memory,
+// and dQ += dS K accumulates in TMEM.
+// dkdv kernel: one CTA per (head, key block); K and V stay in shared memory, the
+// query tiles that selected the block (ascending, from the selection inverse)
+// stream in halves of 64 queries through a 3-stage ring together with their
+// per-row scalars; S^T = K Q^T and dP^T = V dO^T land in double-buffered TMEM,
+// the softmax warps form (P^T cs) and dS^T, and dV += (P^T cs) dO, dK += dS^T Q
+// accumulate in TMEM.  No atomics: the results are deterministic.
+// Every mbarrier wait is bounded; a timeout sets a bit in the caller's error word,
+// the CTA drains its copies and MMAs, frees TMEM and exits.
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace elsaa {
+
+namespace {
+
+constexpr int kT = 128;
+constexpr int kD = 128;
+constexpr uint32_t kSlab = kT * 128;     // [128 rows][64 bf16], 128-byte swizzle
+constexpr uint32_t kTile = 2 * kSlab;    // [128 rows][128 bf16]
+constexpr int kSoftmaxThreads = 256;
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];\n"
+               :: "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2) : "memory");
+}
+__device__ __forceinline__ void tma_store_wait() {
+  asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+}
+
+// ------------------------------- dq ----------------------------------------
+constexpr uint32_t DQ_Q = 0, DQ_DO = kTile;
+__host__ __device__ constexpr uint32_t dq_k(int s) { return kTile * (2 + 2 * s); }
+__host__ __device__ constexpr uint32_t dq_v(int s) { return kTile * (3 + 2 * s); }
+constexpr uint32_t DQ_DS = 6 * kTile;
+constexpr uint32_t DQ_MISC = 7 * kTile;
+constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256;
+constexpr int kDqThreads = 320;          // producer, MMA, 8 softmax warps
+
+struct DqMisc {
+  uint64_t qd_full, kv_full[2], kv_empty[2], s_full, st_free, ds_full, dq_done, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int idx[32];
+};
+
+template <typename M>
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, M* ms, uint32_t* err, uint32_t code) {
+  if (*(volatile int*)&ms->abort_flag) return false;
+  if (tc::mbar_wait(bar, parity)) return true;
+  *(volatile int*)&ms->abort_flag = 1;
+  if (err) atomicOr(err, code);
+  return false;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kDqThreads, 1)
+    dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                 const __grid_constant__ CUtensorMap tmdQ, BwdArgs a, Geom g, uint32_t* err) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  DqMisc* ms = reinterpret_cast<DqMisc*>(smem + DQ_MISC);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = g.n_t - 1 - blockIdx.x;
+  const int bh = blockIdx.y;
+  const size_t head = (size_t)bh * g.N;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
+    return;
+  }
+  const int* my_idx = a.idx + ((size_t)bh * g.n_t + t) * g.k;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&ms->qd_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&ms->kv_full[s], 1);
+      tc::mbar_init(&ms->kv_empty[s], 1);
+    }
+    tc::mbar_init(&ms->s_full, 1);
+    tc::mbar_init(&ms->st_free, kSoftmaxThreads);
+    tc::mbar_init(&ms->ds_full, kSoftmaxThreads);
+    tc::mbar_init(&ms->dq_done, 1);
+    tc::mbar_init(&ms->drain, 1);
+    ms->abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (threadIdx.x < 32) ms->idx[threadIdx.x] = threadIdx.x < g.k ? my_idx[threadIdx.x] : -1;
+  if (warp == 1) {
+    tc::tmem_alloc(&ms->tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+  int n_sel = 0;
+  while (n_sel < g.k && n_sel < 32 && ms->idx[n_sel] >= 0) ++n_sel;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tc::mbar_arrive_expect_tx(&ms->qd_full, 2 * kTile);
+      tc::tma_load_3d(smem + DQ_Q, &tmQ, &ms->qd_full, 0, t * kT, bh);
+      tc::tma_load_3d(smem + DQ_Q + kSlab, &tmQ, &ms->qd_full, 64, t * kT, bh);
+      tc::tma_load_3d(smem + DQ_DO, &tmdO, &ms->qd_full, 0, t * kT, bh);
+      tc::tma_load_3d(smem + DQ_DO + kSlab, &tmdO, &ms->qd_full, 64, t * kT, bh);
+      int issued = 0;
+      for (int j = 0; j < n_sel; ++j) {
+        const int s = j & 1;
+        if (j >= 2 && !wait_or_abort(&ms->kv_empty[s], ((j >> 1) + 1) & 1, ms, err, 1u)) break;
+        const int b = ms->idx[j];
+        tc::mbar_arrive_expect_tx(&ms->kv_full[s], 2 * kTile);
+        tc::tma_load_3d(smem + dq_k(s), &tmK, &ms->kv_full[s], 0, b * kT, bh);
+        tc::tma_load_3d(smem + dq_k(s) + kSlab, &tmK, &ms->kv_full[s], 64, b * kT, bh);
+        tc::tma_load_3d(smem + dq_v(s), &tmV, &ms->kv_full[s], 0, b * kT, bh);
+        tc::tma_load_3d(smem + dq_v(s) + kSlab, &tmV, &ms->kv_full[s], 64, b * kT, bh);
+        issued = j + 1;
+      }
+      tc::mbar_wait(&ms->qd_full, 0);
+      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) tc::mbar_wait(&ms->kv_full[j & 1], (j >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);   // both operands K-major
+      const uint32_t idNM = tc::idesc_bf16(128, kD, false, true);     // B MN-major
+      const uint32_t sb = smem_u32(smem);
+      bool ok = wait_or_abort(&ms->qd_full, 0, ms, err, 2u);
+      int dq_issued = 0;
+      auto issue_dq = [&](int jj) -> bool {
+        if (!wait_or_abort(&ms->ds_full, jj & 1, ms, err, 4u)) return false;
+        tc::tc_fence_after();
+        const uint32_t kb = sb + dq_k(jj & 1);
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk) {
+          const uint64_t ad = tc::sw128_desc(sb + DQ_DS + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = tc::sw128_desc(kb + kk * 2048, kSlab, 1024);
+          tc::mma_bf16(tmem + TM_DQ, ad, bd, idNM, (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(&ms->kv_empty[jj & 1]);
+        tc::mma_commit(&ms->dq_done);
+        dq_issued = jj + 1;
+        return true;
+      };
+      for (int j = 0; ok && j < n_sel; ++j) {
+        const int s = j & 1;
+        if (!wait_or_abort(&ms->kv_full[s], (j >> 1) & 1, ms, err, 8u)) break;
+        if (j >= 1 && !wait_or_abort(&ms->st_free, (j - 1) & 1, ms, err, 16u)) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+          tc::mma_bf16(tmem + TM_S, tc::sw128_desc(sb + DQ_Q + off, 16, 1024),
+                       tc::sw128_desc(sb + dq_k(s) + off, 16, 1024), idNN, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+          tc::mma_bf16(tmem + TM_DP, tc::sw128_desc(sb + DQ_DO + off, 16, 1024),
+                       tc::sw128_desc(sb + dq_v(s) + off, 16, 1024), idNN, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&ms->s_full);
+        if (j >= 1 && !issue_dq(j - 1)) break;
+      }
+      if (n_sel > 0 && dq_issued == n_sel - 1) issue_dq(n_sel - 1);
+      tc::mma_commit(&ms->drain);
+      tc::mbar_wait(&ms->drain, 0);
+    }
+  } else {
+    // ---------------- softmax: half a query row per thread ----------------
+    const int q4 = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = 32 * q4 + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+    const int qrow = t * kT + row;
+    const bool row_ok = qrow < g.N;
+    const float4 sc = row_ok ? a.rs.packed[head + qrow] : make_float4(INFINITY, 0.f, 0.f, 0.f);
+    const float lg2 = sc.x, cs = sc.y, Dl = sc.z;
+    const float sl2 = g.scale * kLog2e;
+    bool alive = true;
+    for (int j = 0; j < n_sel; ++j) {
+      float sv[64], dp[64];
+      if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full, j & 1, ms, err, 32u));
+      if (alive) {
+        tc::tc_fence_after();
+        float tmp[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tc::tmem_ld32(tmem + lane_base + TM_S + 64 * half + 32 * c, tmp);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sv[32 * c + i] = tmp[i];
+          tc::tmem_ld32(tmem + lane_base + TM_DP + 64 * half + 32 * c, tmp);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dp[32 * c + i] = tmp[i];
+        }
+        tc::tmem_wait_ld();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&ms->st_free);
+        const int b = ms->idx[j];
+        const int kvalid = g.N - b * kT;
+        const bool mask = (g.causal && b == t) || kvalid < kT;
+        const int lim = min(kvalid - 1, (g.causal && b == t) ? row : kT - 1) - 64 * half;
+        uint32_t w[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          float p0 = ex2_approx(fmaf(sv[c], sl2, -lg2));
+          float p1 = ex2_approx(fmaf(sv[c + 1], sl2, -lg2));
+          if (mask) {
+            p0 = c > lim ? 0.f : p0;
+            p1 = c + 1 > lim ? 0.f : p1;
+          }
+          w[c >> 1] = pack_bf16(p0 * (cs * dp[c] - Dl), p1 * (cs * dp[c + 1] - Dl));
+        }
+        // the dS buffer is free once dQ of block j-1 has been accumulated
+        if (j >= 1) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->dq_done, (j - 1) & 1, ms, err, 64u));
+        if (alive) {
+          unsigned char* drow = smem + DQ_DS + half * kSlab + row * 128;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) =
+                make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
+          tc::fence_proxy_async_smem();
+          tc::tc_fence_before();
+          tc::mbar_arrive(&ms->ds_full);
+        }
+      }
+    }
+    // ---------------- epilogue: dQ = scale dQ_sparse + dQ_lowrank, bf16 TMA store ----------------
+    float o[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c) o[c] = 0.f;
+    if (alive && n_sel > 0) {
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->dq_done, (n_sel - 1) & 1, ms, err, 128u));
+      if (alive) {
+        tc::tc_fence_after();
+        float tmp[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tc::tmem_ld32(tmem + lane_base + TM_DQ + 64 * half + 32 * c, tmp);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[32 * c + i] = tmp[i] * g.scale;
+        }
+        tc::tmem_wait_ld();
+      }
+    }
+    if (alive && row_ok && a.dQacc) {
+      const float4* acc = reinterpret_cast<const float4*>(a.dQacc + (head + qrow) * kD + 64 * half);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float4 v = acc[c];
+        o[4 * c] += v.x;
+        o[4 * c + 1] += v.y;
+        o[4 * c + 2] += v.z;
+        o[4 * c + 3] += v.w;
+      }
+    }
+    // the dS buffer is free after the last dQ product: stage the bf16 tile there
+    unsigned char* orow = smem + DQ_DS + half * kSlab + row * 128;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch)
+      *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) =
+          make_uint4(pack_bf16(o[8 * ch], o[8 * ch + 1]), pack_bf16(o[8 * ch + 2], o[8 * ch + 3]),
+                     pack_bf16(o[8 * ch + 4], o[8 * ch + 5]), pack_bf16(o[8 * ch + 6], o[8 * ch + 7]));
+    tc::fence_proxy_async_smem();
+    softmax_bar();
+    if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
+      tma_store_3d(&tmdQ, smem + DQ_DS, 0, t * kT, bh);
+      tma_store_3d(&tmdQ, smem + DQ_DS + kSlab, 64, t * kT, bh);
+      tma_store_wait();
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// [BH][N][128] bf16 as a 3-D tensor (d, row, head), boxes of 64 x rows x 1, 128-byte swizzle.
+static bool map_rows(CUtensorMap* m, const void* base, int N, int BH, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)N * kD * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool bwd_tc_supported(const Geom& g) { return g.d == kD && g.T == kT && g.k <= 32; }
+
+cudaError_t launch_dq_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
+  if (!bwd_tc_supported(g) || !a.rs.packed) return cudaErrorInvalidValue;
+  CUtensorMap mq, mk, mv, mdo, mdq;
+  if (!map_rows(&mq, a.Q, g.N, g.BH, kT) || !map_rows(&mk, a.K, g.N, g.BH, kT) ||
+      !map_rows(&mv, a.V, g.N, g.BH, kT) || !map_rows(&mdo, a.dO, g.N, g.BH, kT) ||
+      !map_rows(&mdq, a.dQ, g.N, g.BH, kT))
+    return cudaErrorInvalidValue;
+  const size_t smem = DQ_MISC + sizeof(DqMisc);
+  cudaError_t e = cudaFuncSetAttribute(dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  ProfScope ps("dq_tc", st);
+  dq_tc_kernel<<<dim3(g.n_t, g.BH), kDqThreads, smem, st>>>(mq, mk, mv, mdo, mdq, a, g, err);
+  return cudaGetLastError();
+}
+
+}  // namespace elsaa

@@ -179,6 +179,7 @@ BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
   w.rs.Delta = c.take<float>(rows);
   w.rs.cl = c.take<float>(rows);
   w.rs.delta = c.take<float>(rows);
+  w.rs.packed = bf16 ? c.take<float4>(rows) : nullptr;
   w.RA = c.take<float>((size_t)g.BH * (g.n_seg + 1) * state);
   w.RB = c.take<float>(g.causal ? (size_t)g.BH * g.n_c * state : 0);
   w.offs = c.take<int>((size_t)g.BH * (g.n_t + 1));
@@ -410,8 +411,15 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   ELSAA_TRY(cuda_status(launch_row_scalars(a, bf16, g, st_), "row scalars"));
   ELSAA_TRY(cuda_status(launch_race_state_bwd(a, bf16, g, st_), "race suffix summaries"));
   if (g.k > 0) ELSAA_TRY(cuda_status(launch_invert_selection(s.idx, w.offs, w.tiles, g, st_), "selection inverse"));
-  if (bf16) ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, st_), "backward"));
-  else ELSAA_TRY(cuda_status(launch_bwd_f32(a, g, st_), "backward"));
+  if (bf16) {
+    const bool tc = bwd_tc_supported(g) && !tcgen05_disabled();
+    BwdArgs at = a;
+    if (g.r == 0) at.dQacc = at.dKacc = at.dVacc = nullptr;
+    ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, tc ? 1 | 4 : 7, st_), "backward"));
+    if (tc) ELSAA_TRY(cuda_status(launch_dq_tc(at, g, w.flag, st_), "tcgen05 dq"));
+  } else {
+    ELSAA_TRY(cuda_status(launch_bwd_f32(a, g, st_), "backward"));
+  }
   return ELSAA_OK;
 }
 

@@ -32,6 +32,7 @@ struct RowScalars {
   float* Delta;   // <dO_s, O_s> - dd_s d_s   (sparse softmax delta)
   float* cl;      // g_lr / d_lr: dN = cl dO
   float* delta;   // dd_lr - cl <dO, O_lr>      (RACE key-mass adjoint)
+  float4* packed; // (log2 d_s, cs, Delta, 0) per row, for the tensor-core backward
 };
 
 struct BwdArgs {
@@ -74,7 +75,13 @@ cudaError_t launch_attn_fwd_f32(const FwdArgs& a, const Geom& g, cudaStream_t st
 cudaError_t launch_row_scalars(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st);
 // RACE backward (bf16): low-rank parts of dQ, dK, dV into the fp32 accumulators.
 cudaError_t launch_race_bwd_bf16(const BwdArgs& a, const Geom& g, cudaStream_t st);
-cudaError_t launch_bwd_bf16(const BwdArgs& a, const Geom& g, cudaStream_t st);
+// tcgen05 sparse-branch backward (d = 128, block 128): dQ (query-major) and dK/dV
+// (key-major through the selection inverse), adding the low-rank accumulators.
+bool bwd_tc_supported(const Geom& g);
+cudaError_t launch_dq_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
+cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
+// parts: bit 0 RACE backward, bit 1 sparse dQ, bit 2 sparse dK/dV (mma.sync kernels).
+cudaError_t launch_bwd_bf16(const BwdArgs& a, const Geom& g, int parts, cudaStream_t st);
 cudaError_t launch_bwd_f32(const BwdArgs& a, const Geom& g, cudaStream_t st);
 
 }  // namespace elsaa
