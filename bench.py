@@ -75,8 +75,12 @@ def work_model(w):
     f_read = tiles * 2 * T * r * (d + 1) + (tiles * 2 * T * T * (r + d + 1) if w.causal else 0)
     m["attn_fwd"] = dict(flops=f_sparse + f_read,
                          bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 5)   # gathered K,V + Q, O, O_s, O_lr
+    m["attn_fwd_tc"] = dict(flops=f_sparse, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 4)
+    m["race_readout"] = dict(flops=f_read, bytes=tiles * T * (r + d) * 2 * 2 + tiles * r * (d + 8) * 4 * 2)
     m["sparse_dq"] = dict(flops=3 * pair_mma * sel, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 3)
+    m["dq_tc"] = m["sparse_dq"]
     m["sparse_dkdv"] = dict(flops=4 * pair_mma * sel, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 4)
+    m["dkdv_tc"] = m["sparse_dkdv"]
     f_state = tiles * 2 * T * r * (d + 8)
     m["race_state_fwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)
     m["race_state_bwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)
@@ -398,7 +402,8 @@ def main():
     wm = model.get(dom)
     roof = None
     if wm is not None:
-        tensor_kernel = dom in ("attn_fwd", "sparse_dq", "sparse_dkdv", "race_state_fwd", "race_state_bwd")
+        tensor_kernel = dom in ("attn_fwd", "attn_fwd_tc", "sparse_dq", "dq_tc", "sparse_dkdv", "dkdv_tc",
+                                "race_readout", "race_state_fwd", "race_state_bwd")
         if tensor_kernel:
             ach = wm["flops"] / (dom_ms * 1e-3) / 1e12
             peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])

@@ -296,6 +296,292 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   }
 }
 
+
+// ------------------------------- dkdv ------------------------------------------
+namespace {
+constexpr uint32_t kHalf = 64 * 128;                       // [64 rows][64 bf16] swizzled slab
+constexpr uint32_t KV_K = 0, KV_V = kTile;
+__host__ __device__ constexpr uint32_t kv_q(int s) { return 2 * kTile + s * 2 * (2 * kHalf); }   // Q half, stage s
+__host__ __device__ constexpr uint32_t kv_do(int s) { return kv_q(s) + 2 * kHalf; }           // dO half, stage s
+constexpr int kStages = 3;
+constexpr uint32_t KV_SC = 2 * kTile + kStages * 4 * kHalf;                   // scalars [3][64] float4
+constexpr uint32_t KV_P = KV_SC + kStages * 64 * 16;                          // (P^T cs) [128 keys][64 q]
+constexpr uint32_t KV_DS = KV_P + kSlab;                                      // dS^T     [128 keys][64 q]
+constexpr uint32_t KV_MISC = KV_DS + kSlab;
+constexpr int kMaxUnits = 2048;
+__host__ __device__ constexpr uint32_t tm_st(int b) { return 64u * b; }       // S^T buffers
+__host__ __device__ constexpr uint32_t tm_dpt(int b) { return 128u + 64u * b; }
+constexpr uint32_t TM_DK = 256, TM_DV = 384;
+constexpr int kKvThreads = 320;
+
+struct KvMisc {
+  uint64_t kv_full, qd_full[kStages], qd_empty[kStages], s_full[2], st_free[2], p_full, pv_done, ds_full, dk_done,
+      drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int n_units;
+  int units[kMaxUnits];     // (tile << 1) | half
+};
+}  // namespace
+
+__global__ void __launch_bounds__(kKvThreads, 1)
+    dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmdOh,
+                   const __grid_constant__ CUtensorMap tmSc, const __grid_constant__ CUtensorMap tmdK,
+                   const __grid_constant__ CUtensorMap tmdV, BwdArgs a, Geom g, uint32_t* err) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  KvMisc* ms = reinterpret_cast<KvMisc*>(smem + KV_MISC);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x;
+  const int bh = blockIdx.y;
+  const size_t head = (size_t)bh * g.N;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&ms->kv_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&ms->qd_full[s], 1);
+      tc::mbar_init(&ms->qd_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&ms->s_full[s], 1);
+      tc::mbar_init(&ms->st_free[s], kSoftmaxThreads);
+    }
+    tc::mbar_init(&ms->p_full, kSoftmaxThreads);
+    tc::mbar_init(&ms->pv_done, 1);
+    tc::mbar_init(&ms->ds_full, kSoftmaxThreads);
+    tc::mbar_init(&ms->dk_done, 1);
+    tc::mbar_init(&ms->drain, 1);
+    ms->abort_flag = 0;
+    // units: each query tile that selected this block, in ascending order, as 64-query halves
+    int n = 0;
+    if (g.k > 0) {
+      const int* of = a.offs + (size_t)bh * (g.n_t + 1);
+      const int* list = a.tiles + (size_t)bh * g.n_t * g.k;
+      for (int e = of[b]; e < of[b + 1] && n + 2 <= kMaxUnits; ++e) {
+        const int t = list[e];
+        ms->units[n++] = t << 1;
+        if (t * kT + 64 < g.N) ms->units[n++] = (t << 1) | 1;
+      }
+    }
+    ms->n_units = n;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&ms->tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+  const int n_u = ms->n_units;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tc::mbar_arrive_expect_tx(&ms->kv_full, 2 * kTile);
+      tc::tma_load_3d(smem + KV_K, &tmK, &ms->kv_full, 0, b * kT, bh);
+      tc::tma_load_3d(smem + KV_K + kSlab, &tmK, &ms->kv_full, 64, b * kT, bh);
+      tc::tma_load_3d(smem + KV_V, &tmV, &ms->kv_full, 0, b * kT, bh);
+      tc::tma_load_3d(smem + KV_V + kSlab, &tmV, &ms->kv_full, 64, b * kT, bh);
+      int issued = 0;
+      for (int u = 0; u < n_u; ++u) {
+        const int s = u % kStages;
+        if (u >= kStages && !wait_or_abort(&ms->qd_empty[s], ((u / kStages) - 1) & 1, ms, err, 1u)) break;
+        const int row0 = (ms->units[u] >> 1) * kT + (ms->units[u] & 1) * 64;
+        tc::mbar_arrive_expect_tx(&ms->qd_full[s], 4 * kHalf + 64 * 16);
+        tc::tma_load_3d(smem + kv_q(s), &tmQh, &ms->qd_full[s], 0, row0, bh);
+        tc::tma_load_3d(smem + kv_q(s) + kHalf, &tmQh, &ms->qd_full[s], 64, row0, bh);
+        tc::tma_load_3d(smem + kv_do(s), &tmdOh, &ms->qd_full[s], 0, row0, bh);
+        tc::tma_load_3d(smem + kv_do(s) + kHalf, &tmdOh, &ms->qd_full[s], 64, row0, bh);
+        tc::tma_load_3d(smem + KV_SC + s * 64 * 16, &tmSc, &ms->qd_full[s], 0, row0, bh);
+        issued = u + 1;
+      }
+      tc::mbar_wait(&ms->kv_full, 0);
+      for (int u = (issued > kStages ? issued - kStages : 0); u < issued; ++u)
+        tc::mbar_wait(&ms->qd_full[u % kStages], (u / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idS = tc::idesc_bf16(128, 64, false, false);     // K (keys x d) x Q (queries x d)
+      const uint32_t idG = tc::idesc_bf16(128, kD, false, true);      // P^T / dS^T x (dO / Q, MN-major)
+      const uint32_t sb = smem_u32(smem);
+      bool ok = wait_or_abort(&ms->kv_full, 0, ms, err, 2u);
+      int g_issued = 0;
+      auto issue_grads = [&](int uu) -> bool {
+        const int s = uu % kStages;
+        if (!wait_or_abort(&ms->p_full, uu & 1, ms, err, 4u)) return false;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_bf16(tmem + TM_DV, tc::sw128_desc(sb + KV_P + kk * 32, 16, 1024),
+                       tc::sw128_desc(sb + kv_do(s) + kk * 2048, kHalf, 1024), idG, (uu > 0 || kk > 0) ? 1u : 0u);
+        tc::mma_commit(&ms->pv_done);
+        if (!wait_or_abort(&ms->ds_full, uu & 1, ms, err, 64u)) return false;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_bf16(tmem + TM_DK, tc::sw128_desc(sb + KV_DS + kk * 32, 16, 1024),
+                       tc::sw128_desc(sb + kv_q(s) + kk * 2048, kHalf, 1024), idG, (uu > 0 || kk > 0) ? 1u : 0u);
+        tc::mma_commit(&ms->qd_empty[s]);
+        tc::mma_commit(&ms->dk_done);
+        g_issued = uu + 1;
+        return true;
+      };
+      for (int u = 0; ok && u < n_u; ++u) {
+        const int s = u % kStages, b2 = u & 1;
+        if (!wait_or_abort(&ms->qd_full[s], (u / kStages) & 1, ms, err, 8u)) break;
+        if (u >= 2 && !wait_or_abort(&ms->st_free[b2], ((u >> 1) + 1) & 1, ms, err, 16u)) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t ka = (kk >> 2) * kSlab + (kk & 3) * 32;
+          const uint32_t kq = (kk >> 2) * kHalf + (kk & 3) * 32;
+          tc::mma_bf16(tmem + tm_st(b2), tc::sw128_desc(sb + KV_K + ka, 16, 1024),
+                       tc::sw128_desc(sb + kv_q(s) + kq, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t ka = (kk >> 2) * kSlab + (kk & 3) * 32;
+          const uint32_t kq = (kk >> 2) * kHalf + (kk & 3) * 32;
+          tc::mma_bf16(tmem + tm_dpt(b2), tc::sw128_desc(sb + KV_V + ka, 16, 1024),
+                       tc::sw128_desc(sb + kv_do(s) + kq, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&ms->s_full[b2]);
+        if (u >= 1 && !issue_grads(u - 1)) break;
+      }
+      if (n_u > 0 && g_issued == n_u - 1) issue_grads(n_u - 1);
+      tc::mma_commit(&ms->drain);
+      tc::mbar_wait(&ms->drain, 0);
+    }
+  } else {
+    // ---------------- softmax: one key row, 32 of the unit's 64 queries per thread ----------------
+    const int q4 = warp & 3;
+    const int hq = (warp - 2) >> 2;
+    const int row = 32 * q4 + lane;                 // key row within the block
+    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+    const bool key_ok = b * kT + row < g.N;
+    const float sl2 = g.scale * kLog2e;
+    bool alive = true;
+    for (int u = 0; u < n_u; ++u) {
+      const int s = u % kStages, b2 = u & 1;
+      const int t = ms->units[u] >> 1, h = ms->units[u] & 1;
+      float sv[32], dp[32];
+      if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full[b2], (u >> 1) & 1, ms, err, 32u));
+      if (!alive) continue;
+      tc::tc_fence_after();
+      tc::tmem_ld32(tmem + lane_base + tm_st(b2) + 32 * hq, sv);
+      tc::tmem_ld32(tmem + lane_base + tm_dpt(b2) + 32 * hq, dp);
+      tc::tmem_wait_ld();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&ms->st_free[b2]);
+      const float4* sc = reinterpret_cast<const float4*>(smem + KV_SC + s * 64 * 16) + 32 * hq;
+      const int q0 = 64 * h + 32 * hq;              // first query (within tile t) of this thread
+      const int qvalid = g.N - t * kT - q0;         // queries of this thread inside the sequence
+      const bool diag = g.causal && t == b;
+      uint32_t wp[16], wd[16];
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        float pv[2], dv[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float4 q = sc[c + e];               // (log2 d_s, cs, Delta)
+          float p = ex2_approx(fmaf(sv[c + e], sl2, -q.x));
+          if (!key_ok || c + e >= qvalid || (diag && row > q0 + c + e)) p = 0.f;
+          pv[e] = p * q.y;
+          dv[e] = p * (q.y * dp[c + e] - q.z);
+        }
+        wp[c >> 1] = pack_bf16(pv[0], pv[1]);
+        wd[c >> 1] = pack_bf16(dv[0], dv[1]);
+      }
+      // (P^T cs): the buffer is free once dV of the previous unit has been accumulated
+      if (u >= 1) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->pv_done, (u - 1) & 1, ms, err, 128u));
+      if (!alive) continue;
+      unsigned char* prow = smem + KV_P + row * 128;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+        *reinterpret_cast<uint4*>(prow + (((4 * hq + cc) ^ (row & 7)) << 4)) =
+            make_uint4(wp[4 * cc], wp[4 * cc + 1], wp[4 * cc + 2], wp[4 * cc + 3]);
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&ms->p_full);
+      // dS^T: free once dK of the previous unit has been accumulated
+      if (u >= 1) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->dk_done, (u - 1) & 1, ms, err, 256u));
+      if (!alive) continue;
+      unsigned char* drow = smem + KV_DS + row * 128;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+        *reinterpret_cast<uint4*>(drow + (((4 * hq + cc) ^ (row & 7)) << 4)) =
+            make_uint4(wd[4 * cc], wd[4 * cc + 1], wd[4 * cc + 2], wd[4 * cc + 3]);
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&ms->ds_full);
+    }
+    // ---------------- epilogue: dK = scale dK_sparse + dK_lowrank, dV likewise; TMA stores ----------------
+    float dk[64], dvv[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c) dk[c] = dvv[c] = 0.f;
+    if (alive && n_u > 0) {
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->dk_done, (n_u - 1) & 1, ms, err, 512u));
+      if (alive) {
+        tc::tc_fence_after();
+        float tmp[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tc::tmem_ld32(tmem + lane_base + TM_DK + 64 * hq + 32 * c, tmp);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dk[32 * c + i] = tmp[i] * g.scale;
+          tc::tmem_ld32(tmem + lane_base + TM_DV + 64 * hq + 32 * c, tmp);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dvv[32 * c + i] = tmp[i];
+        }
+        tc::tmem_wait_ld();
+      }
+    }
+    if (alive && key_ok && a.dKacc) {
+      const float4* ak = reinterpret_cast<const float4*>(a.dKacc + (head + (size_t)b * kT + row) * kD + 64 * hq);
+      const float4* av = reinterpret_cast<const float4*>(a.dVacc + (head + (size_t)b * kT + row) * kD + 64 * hq);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float4 x = ak[c], y = av[c];
+        dk[4 * c] += x.x; dk[4 * c + 1] += x.y; dk[4 * c + 2] += x.z; dk[4 * c + 3] += x.w;
+        dvv[4 * c] += y.x; dvv[4 * c + 1] += y.y; dvv[4 * c + 2] += y.z; dvv[4 * c + 3] += y.w;
+      }
+    }
+    // the Q/dO stages are free after the last product: stage dK there (stage 0) and dV (stage 1)
+    unsigned char* krow = smem + kv_q(0) + hq * kSlab + row * 128;
+    unsigned char* vrow = smem + kv_q(1) + hq * kSlab + row * 128;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      const int sw = (ch ^ (row & 7)) << 4;
+      *reinterpret_cast<uint4*>(krow + sw) =
+          make_uint4(pack_bf16(dk[8 * ch], dk[8 * ch + 1]), pack_bf16(dk[8 * ch + 2], dk[8 * ch + 3]),
+                     pack_bf16(dk[8 * ch + 4], dk[8 * ch + 5]), pack_bf16(dk[8 * ch + 6], dk[8 * ch + 7]));
+      *reinterpret_cast<uint4*>(vrow + sw) =
+          make_uint4(pack_bf16(dvv[8 * ch], dvv[8 * ch + 1]), pack_bf16(dvv[8 * ch + 2], dvv[8 * ch + 3]),
+                     pack_bf16(dvv[8 * ch + 4], dvv[8 * ch + 5]), pack_bf16(dvv[8 * ch + 6], dvv[8 * ch + 7]));
+    }
+    tc::fence_proxy_async_smem();
+    softmax_bar();
+    if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
+      tma_store_3d(&tmdK, smem + kv_q(0), 0, b * kT, bh);
+      tma_store_3d(&tmdK, smem + kv_q(0) + kSlab, 64, b * kT, bh);
+      tma_store_3d(&tmdV, smem + kv_q(1), 0, b * kT, bh);
+      tma_store_3d(&tmdV, smem + kv_q(1) + kSlab, 64, b * kT, bh);
+      tma_store_wait();
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
@@ -338,6 +624,35 @@ cudaError_t launch_dq_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStr
   if (e != cudaSuccess) return e;
   ProfScope ps("dq_tc", st);
   dq_tc_kernel<<<dim3(g.n_t, g.BH), kDqThreads, smem, st>>>(mq, mk, mv, mdo, mdq, a, g, err);
+  return cudaGetLastError();
+}
+
+// Per-row scalars (log2 d_s, cs, Delta, 0) as float32 [BH][N][4]; boxes of 4 x 64 x 1.
+static bool map_scalars(CUtensorMap* m, const void* base, int N, int BH) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {4, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {16, (cuuint64_t)N * 16};
+  cuuint32_t box[3] = {4, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
+  if (!bwd_tc_supported(g) || !a.rs.packed || 2 * g.n_t > kMaxUnits) return cudaErrorInvalidValue;
+  CUtensorMap mk, mv, mq, mdo, msc, mdk, mdv;
+  if (!map_rows(&mk, a.K, g.N, g.BH, kT) || !map_rows(&mv, a.V, g.N, g.BH, kT) ||
+      !map_rows(&mq, a.Q, g.N, g.BH, 64) || !map_rows(&mdo, a.dO, g.N, g.BH, 64) ||
+      !map_scalars(&msc, a.rs.packed, g.N, g.BH) || !map_rows(&mdk, a.dK, g.N, g.BH, kT) ||
+      !map_rows(&mdv, a.dV, g.N, g.BH, kT))
+    return cudaErrorInvalidValue;
+  const size_t smem = KV_MISC + sizeof(KvMisc);
+  cudaError_t e = cudaFuncSetAttribute(dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  ProfScope ps("dkdv_tc", st);
+  dkdv_tc_kernel<<<dim3(g.n_t, g.BH), kKvThreads, smem, st>>>(mk, mv, mq, mdo, msc, mdk, mdv, a, g, err);
   return cudaGetLastError();
 }
 

@@ -415,8 +415,11 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
     const bool tc = bwd_tc_supported(g) && !tcgen05_disabled();
     BwdArgs at = a;
     if (g.r == 0) at.dQacc = at.dKacc = at.dVacc = nullptr;
-    ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, tc ? 1 | 4 : 7, st_), "backward"));
-    if (tc) ELSAA_TRY(cuda_status(launch_dq_tc(at, g, w.flag, st_), "tcgen05 dq"));
+    ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, tc ? 1 : 7, st_), "backward"));
+    if (tc) {
+      ELSAA_TRY(cuda_status(launch_dq_tc(at, g, w.flag, st_), "tcgen05 dq"));
+      ELSAA_TRY(cuda_status(launch_dkdv_tc(at, g, w.flag, st_), "tcgen05 dkdv"));
+    }
   } else {
     ELSAA_TRY(cuda_status(launch_bwd_f32(a, g, st_), "backward"));
   }
