@@ -300,27 +300,29 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 // ------------------------------- dkdv ------------------------------------------
 namespace {
 constexpr uint32_t kHalf = 64 * 128;                       // [64 rows][64 bf16] swizzled slab
+constexpr int kStages = 4;
 constexpr uint32_t KV_K = 0, KV_V = kTile;
-__host__ __device__ constexpr uint32_t kv_q(int s) { return 2 * kTile + s * 2 * (2 * kHalf); }   // Q half, stage s
-__host__ __device__ constexpr uint32_t kv_do(int s) { return kv_q(s) + 2 * kHalf; }           // dO half, stage s
-constexpr int kStages = 3;
-constexpr uint32_t KV_SC = 2 * kTile + kStages * 4 * kHalf;                   // scalars [3][64] float4
-constexpr uint32_t KV_P = KV_SC + kStages * 64 * 16;                          // (P^T cs) [128 keys][64 q]
-constexpr uint32_t KV_DS = KV_P + kSlab;                                      // dS^T     [128 keys][64 q]
-constexpr uint32_t KV_MISC = KV_DS + kSlab;
+__host__ __device__ constexpr uint32_t kv_q(int s) { return 2 * kTile + s * 4 * kHalf; }   // Q half, stage s
+__host__ __device__ constexpr uint32_t kv_do(int s) { return kv_q(s) + 2 * kHalf; }      // dO half, stage s
+constexpr uint32_t KV_SC = 2 * kTile + kStages * 4 * kHalf;                   // scalars [stage][64] float4
 constexpr int kMaxUnits = 2048;
-__host__ __device__ constexpr uint32_t tm_st(int b) { return 64u * b; }       // S^T buffers
+constexpr uint32_t KV_UNITS = KV_SC + kStages * 64 * 16;                      // (tile << 1) | half
+constexpr uint32_t KV_MISC = KV_UNITS + kMaxUnits * 4;
+// TMEM columns: S^T and dP^T of a 64-query unit, double-buffered; after the
+// softmax has read them, (P^T cs) and dS^T (bf16, two per column) overwrite the
+// first 16 columns of each 32-column half and feed the dV / dK products as the
+// tensor-memory A operand.
+__host__ __device__ constexpr uint32_t tm_st(int b) { return 64u * b; }
 __host__ __device__ constexpr uint32_t tm_dpt(int b) { return 128u + 64u * b; }
+// column of the K = 16 step kk (queries 16 kk .. 16 kk + 15) of a packed operand
+__host__ __device__ constexpr uint32_t tm_ka(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
 constexpr uint32_t TM_DK = 256, TM_DV = 384;
 constexpr int kKvThreads = 320;
 
 struct KvMisc {
-  uint64_t kv_full, qd_full[kStages], qd_empty[kStages], s_full[2], st_free[2], p_full, pv_done, ds_full, dk_done,
-      drain;
+  uint64_t kv_full, qd_full[kStages], qd_empty[kStages], s_full[2], p_full[2], done;
   uint32_t tmem_base;
   int abort_flag;
-  int n_units;
-  int units[kMaxUnits];     // (tile << 1) | half
 };
 }  // namespace
 
@@ -331,13 +333,30 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                    const __grid_constant__ CUtensorMap tmdV, BwdArgs a, Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   KvMisc* ms = reinterpret_cast<KvMisc*>(smem + KV_MISC);
+  int* units = reinterpret_cast<int*>(smem + KV_UNITS);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.x;
-  const int bh = blockIdx.y;
+  const int bh = blockIdx.x;
+  // heaviest key blocks of every head first (order from the selection inverse)
+  const int b = a.kv_order ? a.kv_order[(size_t)bh * g.n_t + blockIdx.y] : (int)blockIdx.y;
   const size_t head = (size_t)bh * g.N;
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
     return;
+  }
+  // units: each query tile that selected this block, ascending, as 64-query halves;
+  // only the last tile of the sequence can lack its second half
+  int n_u = 0;
+  if (g.k > 0) {
+    const int* of = a.offs + (size_t)bh * (g.n_t + 1);
+    const int* list = a.tiles + (size_t)bh * g.n_t * g.k;
+    const int e0 = of[b], cnt = min(of[b + 1] - e0, kMaxUnits / 2);
+    for (int i = threadIdx.x; i < cnt; i += kKvThreads) {
+      const int t = list[e0 + i];
+      units[2 * i] = t << 1;
+      units[2 * i + 1] = (t << 1) | 1;
+    }
+    n_u = 2 * cnt;
+    if (cnt > 0 && list[e0 + cnt - 1] * kT + 64 >= g.N) n_u -= 1;
   }
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->kv_full, 1);
@@ -347,26 +366,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&ms->s_full[s], 1);
-      tc::mbar_init(&ms->st_free[s], kSoftmaxThreads);
+      tc::mbar_init(&ms->p_full[s], kSoftmaxThreads);
     }
-    tc::mbar_init(&ms->p_full, kSoftmaxThreads);
-    tc::mbar_init(&ms->pv_done, 1);
-    tc::mbar_init(&ms->ds_full, kSoftmaxThreads);
-    tc::mbar_init(&ms->dk_done, 1);
-    tc::mbar_init(&ms->drain, 1);
+    tc::mbar_init(&ms->done, 1);
     ms->abort_flag = 0;
-    // units: each query tile that selected this block, in ascending order, as 64-query halves
-    int n = 0;
-    if (g.k > 0) {
-      const int* of = a.offs + (size_t)bh * (g.n_t + 1);
-      const int* list = a.tiles + (size_t)bh * g.n_t * g.k;
-      for (int e = of[b]; e < of[b + 1] && n + 2 <= kMaxUnits; ++e) {
-        const int t = list[e];
-        ms->units[n++] = t << 1;
-        if (t * kT + 64 < g.N) ms->units[n++] = (t << 1) | 1;
-      }
-    }
-    ms->n_units = n;
     tc::fence_barrier_init();
   }
   if (warp == 1) {
@@ -377,7 +380,6 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
-  const int n_u = ms->n_units;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       for (int u = 0; u < n_u; ++u) {
         const int s = u % kStages;
         if (u >= kStages && !wait_or_abort(&ms->qd_empty[s], ((u / kStages) - 1) & 1, ms, err, 1u)) break;
-        const int row0 = (ms->units[u] >> 1) * kT + (ms->units[u] & 1) * 64;
+        const int row0 = (units[u] >> 1) * kT + (units[u] & 1) * 64;
         tc::mbar_arrive_expect_tx(&ms->qd_full[s], 4 * kHalf + 64 * 16);
         tc::tma_load_3d(smem + kv_q(s), &tmQh, &ms->qd_full[s], 0, row0, bh);
         tc::tma_load_3d(smem + kv_q(s) + kHalf, &tmQh, &ms->qd_full[s], 64, row0, bh);
@@ -408,34 +410,32 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idS = tc::idesc_bf16(128, 64, false, false);     // K (keys x d) x Q (queries x d)
-      const uint32_t idG = tc::idesc_bf16(128, kD, false, true);      // P^T / dS^T x (dO / Q, MN-major)
+      const uint32_t idG = tc::idesc_bf16(128, kD, false, true);      // P^T / dS^T (TMEM) x (dO / Q, MN-major)
       const uint32_t sb = smem_u32(smem);
       bool ok = wait_or_abort(&ms->kv_full, 0, ms, err, 2u);
       int g_issued = 0;
+      // dV += (P^T cs) dO and dK += dS^T Q for unit uu; both A operands in TMEM.
+      // The next S^T into the same columns is issued after these, and tcgen05
+      // MMAs of one thread run in issue order, so the reuse needs no wait.
       auto issue_grads = [&](int uu) -> bool {
-        const int s = uu % kStages;
-        if (!wait_or_abort(&ms->p_full, uu & 1, ms, err, 4u)) return false;
+        const int s = uu % kStages, bb = uu & 1;
+        if (!wait_or_abort(&ms->p_full[bb], (uu >> 1) & 1, ms, err, 4u)) return false;
         tc::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc::mma_bf16(tmem + TM_DV, tc::sw128_desc(sb + KV_P + kk * 32, 16, 1024),
-                       tc::sw128_desc(sb + kv_do(s) + kk * 2048, kHalf, 1024), idG, (uu > 0 || kk > 0) ? 1u : 0u);
-        tc::mma_commit(&ms->pv_done);
-        if (!wait_or_abort(&ms->ds_full, uu & 1, ms, err, 64u)) return false;
-        tc::tc_fence_after();
+          tc::mma_bf16_ts(tmem + TM_DV, tmem + tm_st(bb) + tm_ka(kk),
+                          tc::sw128_desc(sb + kv_do(s) + kk * 2048, kHalf, 1024), idG, (uu > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc::mma_bf16(tmem + TM_DK, tc::sw128_desc(sb + KV_DS + kk * 32, 16, 1024),
-                       tc::sw128_desc(sb + kv_q(s) + kk * 2048, kHalf, 1024), idG, (uu > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_bf16_ts(tmem + TM_DK, tmem + tm_dpt(bb) + tm_ka(kk),
+                          tc::sw128_desc(sb + kv_q(s) + kk * 2048, kHalf, 1024), idG, (uu > 0 || kk > 0) ? 1u : 0u);
         tc::mma_commit(&ms->qd_empty[s]);
-        tc::mma_commit(&ms->dk_done);
         g_issued = uu + 1;
         return true;
       };
       for (int u = 0; ok && u < n_u; ++u) {
         const int s = u % kStages, b2 = u & 1;
         if (!wait_or_abort(&ms->qd_full[s], (u / kStages) & 1, ms, err, 8u)) break;
-        if (u >= 2 && !wait_or_abort(&ms->st_free[b2], ((u >> 1) + 1) & 1, ms, err, 16u)) break;
         tc::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
@@ -455,8 +455,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         if (u >= 1 && !issue_grads(u - 1)) break;
       }
       if (n_u > 0 && g_issued == n_u - 1) issue_grads(n_u - 1);
-      tc::mma_commit(&ms->drain);
-      tc::mbar_wait(&ms->drain, 0);
+      tc::mma_commit(&ms->done);
+      tc::mbar_wait(&ms->done, 0);
     }
   } else {
     // ---------------- softmax: one key row, 32 of the unit's 64 queries per thread ----------------
@@ -467,103 +467,90 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     const bool key_ok = b * kT + row < g.N;
     const float sl2 = g.scale * kLog2e;
     bool alive = true;
-    for (int u = 0; u < n_u; ++u) {
+    for (int u = 0; u < n_u && alive; ++u) {
       const int s = u % kStages, b2 = u & 1;
-      const int t = ms->units[u] >> 1, h = ms->units[u] & 1;
-      float sv[32], dp[32];
-      if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full[b2], (u >> 1) & 1, ms, err, 32u));
-      if (!alive) continue;
+      const int t = units[u] >> 1, h = units[u] & 1;
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full[b2], (u >> 1) & 1, ms, err, 32u));
+      if (!alive) break;
       tc::tc_fence_after();
-      tc::tmem_ld32(tmem + lane_base + tm_st(b2) + 32 * hq, sv);
-      tc::tmem_ld32(tmem + lane_base + tm_dpt(b2) + 32 * hq, dp);
-      tc::tmem_wait_ld();
-      tc::tc_fence_before();
-      tc::mbar_arrive(&ms->st_free[b2]);
       const float4* sc = reinterpret_cast<const float4*>(smem + KV_SC + s * 64 * 16) + 32 * hq;
       const int q0 = 64 * h + 32 * hq;              // first query (within tile t) of this thread
       const int qvalid = g.N - t * kT - q0;         // queries of this thread inside the sequence
       const bool diag = g.causal && t == b;
-      uint32_t wp[16], wd[16];
+      const bool masked = !key_ok || qvalid < 32 || (diag && row > q0);
+      // valid queries of this thread: c in [lo, hi) (causal diagonal, sequence end, key row)
+      const int lo = diag ? row - q0 : 0;
+      const int hi = key_ok ? qvalid : 0;
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float pv[2], dv[2];
+      for (int c0 = 0; c0 < 32; c0 += 16) {
+        // 16 columns at a time keeps S^T, dP^T and the scalars within the register budget;
+        // the packed results of columns c0.. land in columns c0/2.., which this thread
+        // has already read
+        float sv[16], dp[16];
+        tc::tmem_ld16(tmem + lane_base + tm_st(b2) + 32 * hq + c0, sv);
+        tc::tmem_ld16(tmem + lane_base + tm_dpt(b2) + 32 * hq + c0, dp);
+        tc::tmem_wait_ld();
+        uint32_t wp[8], wd[8];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float4 q = sc[c + e];               // (log2 d_s, cs, Delta)
-          float p = ex2_approx(fmaf(sv[c + e], sl2, -q.x));
-          if (!key_ok || c + e >= qvalid || (diag && row > q0 + c + e)) p = 0.f;
-          pv[e] = p * q.y;
-          dv[e] = p * (q.y * dp[c + e] - q.z);
+        for (int c = 0; c < 16; c += 2) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float4 q = sc[c0 + c + e];          // (log2 d_s, cs, Delta)
+            float p = ex2_approx(fmaf(sv[c + e], sl2, -q.x));
+            if (masked && (c0 + c + e < lo || c0 + c + e >= hi)) p = 0.f;
+            pv[e] = p * q.y;
+            dv[e] = p * (q.y * dp[c + e] - q.z);
+          }
+          wp[c >> 1] = pack_bf16(pv[0], pv[1]);
+          wd[c >> 1] = pack_bf16(dv[0], dv[1]);
         }
-        wp[c >> 1] = pack_bf16(pv[0], pv[1]);
-        wd[c >> 1] = pack_bf16(dv[0], dv[1]);
+        tc::tmem_st8(tmem + lane_base + tm_st(b2) + 32 * hq + c0 / 2, wp);
+        tc::tmem_st8(tmem + lane_base + tm_dpt(b2) + 32 * hq + c0 / 2, wd);
       }
-      // (P^T cs): the buffer is free once dV of the previous unit has been accumulated
-      if (u >= 1) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->pv_done, (u - 1) & 1, ms, err, 128u));
-      if (!alive) continue;
-      unsigned char* prow = smem + KV_P + row * 128;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc)
-        *reinterpret_cast<uint4*>(prow + (((4 * hq + cc) ^ (row & 7)) << 4)) =
-            make_uint4(wp[4 * cc], wp[4 * cc + 1], wp[4 * cc + 2], wp[4 * cc + 3]);
-      tc::fence_proxy_async_smem();
+      tc::tmem_wait_st();
       tc::tc_fence_before();
-      tc::mbar_arrive(&ms->p_full);
-      // dS^T: free once dK of the previous unit has been accumulated
-      if (u >= 1) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->dk_done, (u - 1) & 1, ms, err, 256u));
-      if (!alive) continue;
-      unsigned char* drow = smem + KV_DS + row * 128;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc)
-        *reinterpret_cast<uint4*>(drow + (((4 * hq + cc) ^ (row & 7)) << 4)) =
-            make_uint4(wd[4 * cc], wd[4 * cc + 1], wd[4 * cc + 2], wd[4 * cc + 3]);
-      tc::fence_proxy_async_smem();
-      tc::tc_fence_before();
-      tc::mbar_arrive(&ms->ds_full);
+      tc::mbar_arrive(&ms->p_full[b2]);
     }
     // ---------------- epilogue: dK = scale dK_sparse + dK_lowrank, dV likewise; TMA stores ----------------
-    float dk[64], dvv[64];
-#pragma unroll
-    for (int c = 0; c < 64; ++c) dk[c] = dvv[c] = 0.f;
+    bool have = false;
     if (alive && n_u > 0) {
-      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->dk_done, (n_u - 1) & 1, ms, err, 512u));
-      if (alive) {
-        tc::tc_fence_after();
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->done, 0, ms, err, 512u));
+      have = alive;
+      if (have) tc::tc_fence_after();
+    }
+    // every product has completed: stage dK in the stage-0 Q/dO buffers and dV in stage 1
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      float o[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) o[c] = 0.f;
+      if (have) {
+        const float mul = which == 0 ? g.scale : 1.f;
         float tmp[32];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          tc::tmem_ld32(tmem + lane_base + TM_DK + 64 * hq + 32 * c, tmp);
+          tc::tmem_ld32(tmem + lane_base + (which == 0 ? TM_DK : TM_DV) + 64 * hq + 32 * c, tmp);
+          tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) dk[32 * c + i] = tmp[i] * g.scale;
-          tc::tmem_ld32(tmem + lane_base + TM_DV + 64 * hq + 32 * c, tmp);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) dvv[32 * c + i] = tmp[i];
+          for (int i = 0; i < 32; ++i) o[32 * c + i] = tmp[i] * mul;
         }
-        tc::tmem_wait_ld();
       }
-    }
-    if (alive && key_ok && a.dKacc) {
-      const float4* ak = reinterpret_cast<const float4*>(a.dKacc + (head + (size_t)b * kT + row) * kD + 64 * hq);
-      const float4* av = reinterpret_cast<const float4*>(a.dVacc + (head + (size_t)b * kT + row) * kD + 64 * hq);
+      const float* accp = which == 0 ? a.dKacc : a.dVacc;
+      if (alive && key_ok && accp) {
+        const float4* ak = reinterpret_cast<const float4*>(accp + (head + (size_t)b * kT + row) * kD + 64 * hq);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float4 x = ak[c], y = av[c];
-        dk[4 * c] += x.x; dk[4 * c + 1] += x.y; dk[4 * c + 2] += x.z; dk[4 * c + 3] += x.w;
-        dvv[4 * c] += y.x; dvv[4 * c + 1] += y.y; dvv[4 * c + 2] += y.z; dvv[4 * c + 3] += y.w;
+        for (int c = 0; c < 16; ++c) {
+          const float4 x = ak[c];
+          o[4 * c] += x.x; o[4 * c + 1] += x.y; o[4 * c + 2] += x.z; o[4 * c + 3] += x.w;
+        }
       }
-    }
-    // the Q/dO stages are free after the last product: stage dK there (stage 0) and dV (stage 1)
-    unsigned char* krow = smem + kv_q(0) + hq * kSlab + row * 128;
-    unsigned char* vrow = smem + kv_q(1) + hq * kSlab + row * 128;
+      unsigned char* orow = smem + kv_q(which) + hq * kSlab + row * 128;
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      const int sw = (ch ^ (row & 7)) << 4;
-      *reinterpret_cast<uint4*>(krow + sw) =
-          make_uint4(pack_bf16(dk[8 * ch], dk[8 * ch + 1]), pack_bf16(dk[8 * ch + 2], dk[8 * ch + 3]),
-                     pack_bf16(dk[8 * ch + 4], dk[8 * ch + 5]), pack_bf16(dk[8 * ch + 6], dk[8 * ch + 7]));
-      *reinterpret_cast<uint4*>(vrow + sw) =
-          make_uint4(pack_bf16(dvv[8 * ch], dvv[8 * ch + 1]), pack_bf16(dvv[8 * ch + 2], dvv[8 * ch + 3]),
-                     pack_bf16(dvv[8 * ch + 4], dvv[8 * ch + 5]), pack_bf16(dvv[8 * ch + 6], dvv[8 * ch + 7]));
+      for (int ch = 0; ch < 8; ++ch)
+        *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) =
+            make_uint4(pack_bf16(o[8 * ch], o[8 * ch + 1]), pack_bf16(o[8 * ch + 2], o[8 * ch + 3]),
+                       pack_bf16(o[8 * ch + 4], o[8 * ch + 5]), pack_bf16(o[8 * ch + 6], o[8 * ch + 7]));
     }
     tc::fence_proxy_async_smem();
     softmax_bar();
@@ -652,7 +639,7 @@ cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaS
   cudaError_t e = cudaFuncSetAttribute(dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("dkdv_tc", st);
-  dkdv_tc_kernel<<<dim3(g.n_t, g.BH), kKvThreads, smem, st>>>(mk, mv, mq, mdo, msc, mdk, mdv, a, g, err);
+  dkdv_tc_kernel<<<dim3(g.BH, g.n_t), kKvThreads, smem, st>>>(mk, mv, mq, mdo, msc, mdk, mdv, a, g, err);
   return cudaGetLastError();
 }
 

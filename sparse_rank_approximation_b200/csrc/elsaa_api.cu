@@ -165,7 +165,7 @@ struct BwdWs {
   uint32_t* flag;
   RowScalars rs;
   float *RA, *RB;
-  int *offs, *tiles;
+  int *offs, *tiles, *order;
   float *dQacc, *dKacc, *dVacc;
 };
 
@@ -184,6 +184,7 @@ BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
   w.RB = c.take<float>(g.causal ? (size_t)g.BH * g.n_c * state : 0);
   w.offs = c.take<int>((size_t)g.BH * (g.n_t + 1));
   w.tiles = c.take<int>((size_t)g.BH * g.n_t * std::max(g.k, 1));
+  w.order = c.take<int>((size_t)g.BH * g.n_t);
   const size_t acc = bf16 && g.r > 0 ? rows * g.d : 0;
   w.dQacc = c.take<float>(acc);
   w.dKacc = c.take<float>(acc);
@@ -403,14 +404,14 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   a.Os = s.Os; a.Olr = s.Olr; a.phiQ = s.phiQ; a.phiK = s.phiK;
   a.hQ = s.hQ; a.hK = s.hK; a.nQ = s.nQ; a.nK = s.nK;
   a.Ast = s.Ast; a.Bst = s.Bst; a.RA = w.RA; a.RB = w.RB;
-  a.offs = w.offs; a.tiles = w.tiles; a.rs = w.rs;
+  a.offs = w.offs; a.tiles = w.tiles; a.kv_order = g.k > 0 ? w.order : nullptr; a.rs = w.rs;
   a.dQacc = w.dQacc; a.dKacc = w.dKacc; a.dVacc = w.dVacc;
   a.dQ = dQ; a.dK = dK; a.dV = dV;
 
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st_), "flag reset"));
   ELSAA_TRY(cuda_status(launch_row_scalars(a, bf16, g, st_), "row scalars"));
   ELSAA_TRY(cuda_status(launch_race_state_bwd(a, bf16, g, st_), "race suffix summaries"));
-  if (g.k > 0) ELSAA_TRY(cuda_status(launch_invert_selection(s.idx, w.offs, w.tiles, g, st_), "selection inverse"));
+  if (g.k > 0) ELSAA_TRY(cuda_status(launch_invert_selection(s.idx, w.offs, w.tiles, w.order, g, st_), "selection inverse"));
   if (bf16) {
     const bool tc = bwd_tc_supported(g) && !tcgen05_disabled();
     BwdArgs at = a;

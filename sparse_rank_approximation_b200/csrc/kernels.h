@@ -47,6 +47,7 @@ struct BwdArgs {
   const float *Ast, *Bst;        // forward prefix statistics
   float *RA, *RB;                // backward suffix statistics
   const int *offs, *tiles;       // key block -> query tiles
+  const int* kv_order;           // per head, key blocks by descending tile count (ties: lower block first)
   RowScalars rs;
   float *dQacc, *dKacc, *dVacc;  // fp32 low-rank gradient parts (bf16 path)
   void *dQ, *dK, *dV;
@@ -57,7 +58,8 @@ void record_error(const char* msg);
 
 cudaError_t launch_select(const void* Q, const void* K, bool bf16, double* qbar, double* kbar, float* scores,
                           int* idx, const Geom& g, cudaStream_t st);
-cudaError_t launch_invert_selection(const int* idx, int* offs, int* tiles, const Geom& g, cudaStream_t st);
+cudaError_t launch_invert_selection(const int* idx, int* offs, int* tiles, int* order, const Geom& g,
+                                    cudaStream_t st);
 cudaError_t launch_race_features(const void* Q, const void* K, const float* W, bool bf16, void* phiQ, void* phiK,
                                  float* hQ, float* hK, float* nQ, float* nK, const Geom& g, cudaStream_t st);
 // Forward prefix statistics (Ast: per-segment exclusive prefix, Bst: in-segment prefix).

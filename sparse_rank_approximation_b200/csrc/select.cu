@@ -155,10 +155,12 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
 
 // Inverse of the selection for the key-major backward: for each key block b the
 // ascending list of query tiles that selected it.  grid (BH), block 256.
-// Output per head: offs[n_t + 1] and tiles[n_t * k] (CSR).  Deterministic.
+// Output per head: offs[n_t + 1] and tiles[n_t * k] (CSR), and order[n_t]: the key
+// blocks by descending count, ties by ascending block (a longest-first launch
+// order for the key-major backward).  Deterministic.
 __global__ void __launch_bounds__(256) invert_selection_kernel(const int* __restrict__ idx,
                                                                int* __restrict__ offs, int* __restrict__ tiles,
-                                                               Geom g) {
+                                                               int* __restrict__ order, Geom g) {
   extern __shared__ uint32_t bits[];      // n_t rows x words bitmap: bit (t, b)
   const int bh = blockIdx.x;
   const int words = (g.n_t + 31) >> 5;
@@ -182,6 +184,19 @@ __global__ void __launch_bounds__(256) invert_selection_kernel(const int* __rest
     if (lane == 0) cnt_s[b] = c;
   }
   __syncthreads();
+  if (order) {
+    int* od = order + (size_t)bh * g.n_t;
+    for (int b = threadIdx.x; b < g.n_t; b += blockDim.x) {
+      const int c = cnt_s[b];
+      int rank = 0;
+      for (int b2 = 0; b2 < g.n_t; ++b2) {
+        const int c2 = cnt_s[b2];
+        rank += (c2 > c) || (c2 == c && b2 < b);
+      }
+      od[rank] = b;
+    }
+    __syncthreads();
+  }
   if (threadIdx.x == 0) {
     int acc = 0;
     for (int b = 0; b < g.n_t; ++b) {
@@ -228,13 +243,14 @@ cudaError_t launch_select(const void* Q, const void* K, bool bf16, double* qbar,
   return cudaGetLastError();
 }
 
-cudaError_t launch_invert_selection(const int* idx, int* offs, int* tiles, const Geom& g, cudaStream_t st) {
+cudaError_t launch_invert_selection(const int* idx, int* offs, int* tiles, int* order, const Geom& g,
+                                    cudaStream_t st) {
   const size_t smem = (size_t)g.n_t * ((g.n_t + 31) / 32) * 4;
   cudaError_t e = cudaFuncSetAttribute(invert_selection_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("invert_selection", st);
-  invert_selection_kernel<<<g.BH, 256, smem, st>>>(idx, offs, tiles, g);
+  invert_selection_kernel<<<g.BH, 256, smem, st>>>(idx, offs, tiles, order, g);
   return cudaGetLastError();
 }
 
