@@ -81,6 +81,21 @@ def work_model(w):
     m["dq_tc"] = m["sparse_dq"]
     m["sparse_dkdv"] = dict(flops=4 * pair_mma * sel, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 4)
     m["dkdv_tc"] = m["sparse_dkdv"]
+    # RACE read-out and backward on the tensor cores, per chunk of T rows (C = T):
+    # read-out  Phi_Q Phi_K^T, kappa V, Phi_Q P;
+    # query side  dO V^T, dO P^T, dkappa Phi_K, dh W^T;
+    # key side  Phi_K Phi_Q^T, V dO^T, Phi_K R, V R^T, kappa^T dO, dkappa^T Phi_Q, dh W^T.
+    NH = 4 * L
+    cz = 1 if w.causal else 0
+    state_b = r * (d + 8) * 4 * (2 if w.causal else 1)          # prefix/suffix statistics read per chunk
+    m["race_readout_tc"] = dict(flops=tiles * 2 * T * (cz * T * r + cz * T * d + r * d),
+                                bytes=tiles * (T * r * 2 * (1 + cz) + cz * T * d * 2 + state_b + T * d * 2 + T * 4))
+    m["race_q_bwd_tc"] = dict(flops=tiles * 2 * T * (cz * T * d + d * r + cz * T * r + NH * d),
+                              bytes=tiles * (T * d * 2 * (2 + cz) + cz * T * r * 2 + state_b + T * NH * 4 + T * 12
+                                             + T * d * 4))
+    m["race_k_bwd_tc"] = dict(flops=tiles * 2 * T * (2 * cz * T * r + 2 * cz * T * d + 2 * r * d + NH * d),
+                              bytes=tiles * (T * r * 2 * (1 + cz) + T * d * 2 * (2 + cz) + state_b + T * NH * 4
+                                             + T * 12 + 2 * T * d * 4))
     f_state = tiles * 2 * T * r * (d + 8)
     m["race_state_fwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)
     m["race_state_bwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)

@@ -585,7 +585,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [BH][N][128] bf16 as a 3-D tensor (d, row, head), boxes of 64 x rows x 1, 128-byte swizzle.
-static bool map_rows(CUtensorMap* m, const void* base, int N, int BH, int rows) {
+bool tc::map_rows_bf16(CUtensorMap* m, const void* base, int N, int BH, int rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)N, (cuuint64_t)BH};
@@ -602,9 +602,9 @@ bool bwd_tc_supported(const Geom& g) { return g.d == kD && g.T == kT && g.k <= 3
 cudaError_t launch_dq_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
   if (!bwd_tc_supported(g) || !a.rs.packed) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if (!map_rows(&mq, a.Q, g.N, g.BH, kT) || !map_rows(&mk, a.K, g.N, g.BH, kT) ||
-      !map_rows(&mv, a.V, g.N, g.BH, kT) || !map_rows(&mdo, a.dO, g.N, g.BH, kT) ||
-      !map_rows(&mdq, a.dQ, g.N, g.BH, kT))
+  if (!tc::map_rows_bf16(&mq, a.Q, g.N, g.BH, kT) || !tc::map_rows_bf16(&mk, a.K, g.N, g.BH, kT) ||
+      !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kT) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, kT) ||
+      !tc::map_rows_bf16(&mdq, a.dQ, g.N, g.BH, kT))
     return cudaErrorInvalidValue;
   const size_t smem = DQ_MISC + sizeof(DqMisc);
   cudaError_t e = cudaFuncSetAttribute(dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -630,10 +630,10 @@ static bool map_scalars(CUtensorMap* m, const void* base, int N, int BH) {
 cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
   if (!bwd_tc_supported(g) || !a.rs.packed || 2 * g.n_t > kMaxUnits) return cudaErrorInvalidValue;
   CUtensorMap mk, mv, mq, mdo, msc, mdk, mdv;
-  if (!map_rows(&mk, a.K, g.N, g.BH, kT) || !map_rows(&mv, a.V, g.N, g.BH, kT) ||
-      !map_rows(&mq, a.Q, g.N, g.BH, 64) || !map_rows(&mdo, a.dO, g.N, g.BH, 64) ||
-      !map_scalars(&msc, a.rs.packed, g.N, g.BH) || !map_rows(&mdk, a.dK, g.N, g.BH, kT) ||
-      !map_rows(&mdv, a.dV, g.N, g.BH, kT))
+  if (!tc::map_rows_bf16(&mk, a.K, g.N, g.BH, kT) || !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kT) ||
+      !tc::map_rows_bf16(&mq, a.Q, g.N, g.BH, 64) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, 64) ||
+      !map_scalars(&msc, a.rs.packed, g.N, g.BH) || !tc::map_rows_bf16(&mdk, a.dK, g.N, g.BH, kT) ||
+      !tc::map_rows_bf16(&mdv, a.dV, g.N, g.BH, kT))
     return cudaErrorInvalidValue;
   const size_t smem = KV_MISC + sizeof(KvMisc);
   cudaError_t e = cudaFuncSetAttribute(dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -359,7 +359,10 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
   ELSAA_TRY(cuda_status(launch_race_state_fwd(s.phiK, V, bf16, s.Ast, s.Bst, g, st_), "race summaries"));
   FwdArgs a{Q, K, V, s.idx, s.phiQ, s.phiK, s.Ast, s.Bst, lam, gs, glr, O, s.Os, s.logd, s.dlr, s.m, s.Olr};
   if (bf16 && attn_fwd_tc_supported(g) && !tcgen05_disabled()) {
-    ELSAA_TRY(cuda_status(launch_race_readout_bf16(a, g, st_), "race read-out"));
+    if (g.r > 0 && race_bwd_tc_supported(g))
+      ELSAA_TRY(cuda_status(launch_race_readout_tc(a, g, w.flag, st_), "tcgen05 race read-out"));
+    else
+      ELSAA_TRY(cuda_status(launch_race_readout_bf16(a, g, st_), "race read-out"));
     ELSAA_TRY(cuda_status(launch_attn_fwd_tc(a, g, w.flag, st_), "tcgen05 forward"));
   } else if (bf16) {
     ELSAA_TRY(cuda_status(launch_attn_fwd_bf16(a, g, st_), "fused forward"));
@@ -414,9 +417,11 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   if (g.k > 0) ELSAA_TRY(cuda_status(launch_invert_selection(s.idx, w.offs, w.tiles, w.order, g, st_), "selection inverse"));
   if (bf16) {
     const bool tc = bwd_tc_supported(g) && !tcgen05_disabled();
+    const bool race_tc = tc && g.r > 0 && race_bwd_tc_supported(g);
     BwdArgs at = a;
     if (g.r == 0) at.dQacc = at.dKacc = at.dVacc = nullptr;
-    ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, tc ? 1 : 7, st_), "backward"));
+    if (race_tc) ELSAA_TRY(cuda_status(launch_race_bwd_tc(a, g, w.flag, st_), "tcgen05 race backward"));
+    ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, tc ? (race_tc ? 0 : 1) : 7, st_), "backward"));
     if (tc) {
       ELSAA_TRY(cuda_status(launch_dq_tc(at, g, w.flag, st_), "tcgen05 dq"));
       ELSAA_TRY(cuda_status(launch_dkdv_tc(at, g, w.flag, st_), "tcgen05 dkdv"));

@@ -73,6 +73,8 @@ cudaError_t launch_attn_fwd_bf16(const FwdArgs& a, const Geom& g, cudaStream_t s
 bool attn_fwd_tc_supported(const Geom& g);
 cudaError_t launch_attn_fwd_tc(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
 cudaError_t launch_race_readout_bf16(const FwdArgs& a, const Geom& g, cudaStream_t st);
+// tcgen05 RACE read-out (same shapes as race_bwd_tc_supported): O_lr (bf16) and d_lr.
+cudaError_t launch_race_readout_tc(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
 cudaError_t launch_attn_fwd_f32(const FwdArgs& a, const Geom& g, cudaStream_t st);
 cudaError_t launch_row_scalars(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st);
 // RACE backward (bf16): low-rank parts of dQ, dK, dV into the fp32 accumulators.
@@ -80,6 +82,10 @@ cudaError_t launch_race_bwd_bf16(const BwdArgs& a, const Geom& g, cudaStream_t s
 // tcgen05 sparse-branch backward (d = 128, block 128): dQ (query-major) and dK/dV
 // (key-major through the selection inverse), adding the low-rank accumulators.
 bool bwd_tc_supported(const Geom& g);
+// tcgen05 RACE backward (d = 128, chunk 128, r = 128): low-rank parts of dQ, dK, dV
+// into the fp32 accumulators; needs the saved projections and row norms.
+bool race_bwd_tc_supported(const Geom& g);
+cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
 cudaError_t launch_dq_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
 cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
 // parts: bit 0 RACE backward, bit 1 sparse dQ, bit 2 sparse dK/dV (mma.sync kernels).

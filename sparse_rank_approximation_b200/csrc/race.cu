@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(128) race_features_bf16_kernel(
   const int side = blockIdx.z;
   const __nv_bfloat16* X = (side == 0 ? Q : K) + (size_t)blockIdx.y * g.N * D;
   __nv_bfloat16* phi = (side == 0 ? phiQ : phiK) + (size_t)blockIdx.y * g.N * g.r;
-  // h and the norms are only kept when the caller asks (the bf16 backward recomputes them)
+  // h and the norms are kept for the backward when the caller passes buffers for them
   float* hout = (side == 0 ? hQ : hK);
   float* nout = (side == 0 ? nQ : nK);
   if (hout) hout += (size_t)blockIdx.y * g.N * NH;
@@ -395,8 +395,8 @@ cudaError_t launch_race_features(const void* Q, const void* K, const float* W, b
     if (e != cudaSuccess) return e;
     ProfScope ps("race_features", st);
     kern<<<dim3((g.N + 63) / 64, g.BH, 2), 128, smem, st>>>(
-        (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, W, (__nv_bfloat16*)phiQ, (__nv_bfloat16*)phiK, nullptr,
-        nullptr, nullptr, nullptr, g);
+        (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, W, (__nv_bfloat16*)phiQ, (__nv_bfloat16*)phiK, hQ, hK,
+        nQ, nK, g);
     return cudaGetLastError();
   };
   if (g.d == 64) return run(race_features_bf16_kernel<64>);

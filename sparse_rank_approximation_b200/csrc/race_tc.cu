@@ -1,0 +1,886 @@
+// RACE low-rank branch (ELSAA paper §3.1) read-out and backward on the 5th-generation
+// tensor cores, for d = 128, chunk C = 128 and r = 128 (L = 8 tables of 16 corners).
+// One CTA per (head, chunk of 128 rows); every accumulator lives in tensor memory.
+//
+// Read-out, chunk t (query rows i):
+//   [N_lr,i ; d_lr,i] = Phi(q_i) [P^V ; p1] + sum_{j in t, j <= i} (Phi(q_i).Phi(k_j)) [v_j ; 1],
+//   O_lr,i = N_lr,i / d_lr,i (bf16) and d_lr,i (fp32), with P the prefix statistics.
+//
+// Key side, chunk c (rows j):
+//   kappa^T = Phi(K_c) Phi(Q_c)^T and X = V_c dO_c^T (causal intra-chunk terms),
+//   dv_j    = R^V^T Phi(k_j) + sum_{i in c, i >= j} cl_i kappa_ij dO_i,
+//   dPhi_kj = R^V v_j + r1 + sum_{i in c, i >= j} (cl_i <dO_i, v_j> + delta_i) Phi(q_i),
+// with R the suffix statistics of the later chunks (sum of Phi(q_i) [cl_i dO_i; delta_i]^T).
+// Query side, chunk t (rows i):
+//   dPhi_qi = cl_i P^V dO_i + delta_i p1 + sum_{j in t, j <= i} (cl_i <dO_i, v_j> + delta_i) Phi(k_j),
+// with P the prefix statistics of the earlier chunks.  Both then go through the
+// corner softmax (dh_b = (1/tau) sum_c p_c (dp_c - <dp, p>) c_b, dp = dPhi / sqrt(L)),
+// du = dh W^T and dx = (du - x <x, du> / |x|^2) / |x| into the fp32 accumulators.
+//
+// Work split: warp 0 issues the TMA loads, warp 1 the MMAs, warps 2..9 (256
+// threads, TMEM lane quarter = warp % 4, column half = (warp - 2) / 4) stage the
+// statistics (fp32 prefix + in-segment part -> bf16 hi + lo halves, 128-byte
+// swizzled) and W, then run the element-wise passes.  The masked intra-chunk
+// matrices (bf16) and dh (bf16 hi + lo) are written back into tensor memory over
+// the fp32 values they replace and feed the next products as the A operand.
+// Every mbarrier wait is bounded; a timeout sets a bit in the caller's error word.
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace elsaa {
+
+namespace {
+
+constexpr int kC = 128;
+constexpr int kD = 128;
+constexpr int kR = 128;
+constexpr int kNH = 32;                          // projection columns 4 L
+constexpr uint32_t kSlab = 128 * 128;            // [128 rows][64 bf16], 128-byte swizzle
+constexpr uint32_t kTile = 2 * kSlab;            // [128 rows][128 bf16]
+constexpr uint32_t kWSlab = kNH * 128;           // [32 rows][64 bf16]
+constexpr int kThreads = 320;
+constexpr int kComputeThreads = 256;
+
+// Byte offset of element (row, col) of a [rows][128] bf16 tile kept as two
+// 64-column slabs of `slab` bytes with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw_off(int row, int col, uint32_t slab) {
+  return (uint32_t)(col >> 6) * slab + (uint32_t)row * 128u + (uint32_t)((((col & 63) >> 3) ^ (row & 7)) << 4) +
+         (uint32_t)(col & 7) * 2u;
+}
+__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+
+// K-major operand, K = 16 step kk of a [rows][128] tile.
+__device__ __forceinline__ uint64_t desc_k(uint32_t base, int kk) {
+  return tc::sw128_desc(base + (uint32_t)(kk >> 2) * kSlab + (uint32_t)(kk & 3) * 32u, 16, 1024);
+}
+// MN-major operand: rows are K, 128 columns are N; K = 16 step kk.
+__device__ __forceinline__ uint64_t desc_mn(uint32_t base, int kk, uint32_t slab) {
+  return tc::sw128_desc(base + (uint32_t)kk * 2048u, slab, 1024);
+}
+// TMEM column of the K = 16 step kk of a packed bf16 operand whose K index
+// 64 h + m (h = column half of the thread that wrote it) sits at column 64 h + m / 2.
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
+
+struct Bars {
+  uint64_t in_main, ready, s_full, p_full, acc_full, dh_full, du_full;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Bars* ms, uint32_t* err,
+                                              uint32_t code) {
+  if (*(volatile int*)&ms->abort_flag) return false;
+  if (tc::mbar_wait(bar, parity)) return true;
+  *(volatile int*)&ms->abort_flag = 1;
+  if (err) atomicOr(err, code);
+  return false;
+}
+
+__device__ __forceinline__ void split2(float x, float y, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x - hf.x, y - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Statistics of the value columns, (s0 + s1)[f][0:128) for f < 128 from fp32
+// [r][dp] states, as bf16 hi and lo [128 f][128] swizzled tiles; the key-mass
+// column goes to m1[f].  256 threads; each issues all of its loads (16 rows of
+// each source) before the first conversion, so the staging costs one round trip.
+__device__ void stage_state(const float* __restrict__ s0, const float* __restrict__ s1, int dp, unsigned char* hi,
+                            unsigned char* lo, float* m1, int ct) {
+  const int w8 = ct >> 5, lane = ct & 31;
+  float4 v[16], w[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __ldg(reinterpret_cast<const float4*>(s0 + (size_t)(w8 + 8 * k) * dp) + lane);
+#pragma unroll
+  for (int k = 0; k < 16; ++k)
+    w[k] = s1 ? __ldg(reinterpret_cast<const float4*>(s1 + (size_t)(w8 + 8 * k) * dp) + lane)
+              : make_float4(0.f, 0.f, 0.f, 0.f);
+  const float mass = ct < kR ? s0[(size_t)ct * dp + kD] + (s1 ? s1[(size_t)ct * dp + kD] : 0.f) : 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int f = w8 + 8 * k;
+    uint32_t h0, l0, h1, l1;
+    split2(v[k].x + w[k].x, v[k].y + w[k].y, h0, l0);
+    split2(v[k].z + w[k].z, v[k].w + w[k].w, h1, l1);
+    const uint32_t off = sw_off(f, 4 * lane, kSlab);
+    *reinterpret_cast<uint2*>(hi + off) = make_uint2(h0, h1);
+    *reinterpret_cast<uint2*>(lo + off) = make_uint2(l0, l1);
+  }
+  if (ct < kR) m1[ct] = mass;
+}
+
+// W[l][k][b] (fp32 [L][128][4]) -> Wt[n = 4 l + b][k] as bf16 hi and lo [32][128]
+// swizzled tiles.  256 threads, two 8-element chunks each.
+__device__ void stage_w(const float* __restrict__ W, unsigned char* hi, unsigned char* lo, int ct) {
+#pragma unroll
+  for (int q = ct; q < kNH * 16; q += kComputeThreads) {
+    const int n = q >> 4, k0 = (q & 15) * 8;
+    float w[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) w[e] = __ldg(W + ((size_t)(n >> 2) * kD + k0 + e) * kHashBits + (n & 3));
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) split2(w[2 * e], w[2 * e + 1], h[e], l[e]);
+    const uint32_t off = sw_off(n, k0, kWSlab);
+    *reinterpret_cast<uint4*>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
+  }
+}
+
+// Corner-softmax backward of one table: h (4 normalised projections), dp (16
+// corner adjoints, already divided by sqrt(L)) -> dh (4 values).
+__device__ __forceinline__ void corner_bwd(const float (&h)[4], const float (&dp)[16], float inv_tau,
+                                           float (&dh)[4]) {
+  float sp[4], sm[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const float y = 2.f * h[b] * inv_tau;
+    sp[b] = 1.f / (1.f + expf(-y));
+    sm[b] = 1.f / (1.f + expf(y));
+  }
+  float p[16], s = 0.f;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    float v = 1.f;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) v *= ((c >> b) & 1) ? sp[b] : sm[b];
+    p[c] = v;
+    s = fmaf(v, dp[c], s);
+  }
+#pragma unroll
+  for (int b = 0; b < 4; ++b) dh[b] = 0.f;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const float da = p[c] * (dp[c] - s);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) dh[b] += ((c >> b) & 1) ? da : -da;
+  }
+#pragma unroll
+  for (int b = 0; b < 4; ++b) dh[b] *= inv_tau;
+}
+
+// Corner pass for the 4 tables 4 hc .. 4 hc + 3 of one row: dPhi of those tables
+// (fp32, 64 TMEM columns from `dphi_col`, plus the optional `cl * G + de * m1`
+// terms), projections h (global, fp32), then dh as bf16 hi / lo into TMEM columns
+// 8 hc (hi) and 16 + 8 hc (lo).
+__device__ __forceinline__ void load_h(const float* __restrict__ hrow, int hc, float (&h16)[16]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 v = hrow ? __ldg(reinterpret_cast<const float4*>(hrow + 16 * hc) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+    h16[4 * q] = v.x; h16[4 * q + 1] = v.y; h16[4 * q + 2] = v.z; h16[4 * q + 3] = v.w;
+  }
+}
+__device__ __forceinline__ void load_x(const __nv_bfloat16* __restrict__ xrow, int hc, bool valid, uint4 (&xr)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    xr[q] = valid ? __ldg(reinterpret_cast<const uint4*>(xrow + 64 * hc) + q) : make_uint4(0u, 0u, 0u, 0u);
+}
+
+__device__ __forceinline__ void corner_pass(uint32_t tmem, uint32_t lane_base, int hc, uint32_t dphi_col,
+                                            bool has_dphi, uint32_t g_col, float cl, float de, const float* m1,
+                                            const float (&h16)[16], float inv_sqrt_L, float inv_tau) {
+  float dh16[16];
+#pragma unroll
+  for (int tl = 0; tl < 4; ++tl) {
+    float a[16], gg[16];
+    const uint32_t col = 64u * hc + 16u * tl;
+    if (has_dphi) tc::tmem_ld16(tmem + lane_base + dphi_col + col, a);
+    if (g_col) tc::tmem_ld16(tmem + lane_base + g_col + col, gg);
+    tc::tmem_wait_ld();
+    float dp[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      float v = has_dphi ? a[c] : 0.f;
+      if (g_col) v = fmaf(cl, gg[c], v);
+      v = fmaf(de, m1[col + c], v);
+      dp[c] = v * inv_sqrt_L;
+    }
+    float h[4] = {h16[4 * tl], h16[4 * tl + 1], h16[4 * tl + 2], h16[4 * tl + 3]}, dh[4];
+    corner_bwd(h, dp, inv_tau, dh);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) dh16[4 * tl + b] = dh[b];
+  }
+  uint32_t hi[8], lo[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) split2(dh16[2 * e], dh16[2 * e + 1], hi[e], lo[e]);
+  tc::tmem_st8(tmem + lane_base + 8u * hc, hi);
+  tc::tmem_st8(tmem + lane_base + 16u + 8u * hc, lo);
+}
+
+// du = dh W^T: three products (hi hi, hi lo, lo hi), K = 32 (two steps each).
+__device__ __forceinline__ void issue_du(uint32_t tmem, uint32_t d_col, uint32_t sb, uint32_t w_hi, uint32_t w_lo) {
+  const uint32_t idG = tc::idesc_bf16(128, kD, false, true);
+#pragma unroll
+  for (int part = 0; part < 3; ++part) {
+    const uint32_t a_col = part == 2 ? 16u : 0u;
+    const uint32_t wb = sb + (part == 1 ? w_lo : w_hi);
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk)
+      tc::mma_bf16_ts(tmem + d_col, tmem + a_col + 8u * kk, desc_mn(wb, kk, kWSlab), idG,
+                      (part > 0 || kk > 0) ? 1u : 0u);
+  }
+}
+
+// dx = (du - x <x, du> / n^2) / n for one row, this thread's 64 columns; the two
+// column halves of a row meet through `xch`.  Stores fp32 into out (row pointer).
+// Every compute thread calls this (the exchange barrier); `alive` false skips the
+// tensor-memory reads and the stores.
+__device__ __forceinline__ void chain_pass(uint32_t tmem, uint32_t lane_base, int hc, int row_in_chunk,
+                                           uint32_t du_col, const uint4 (&xr)[8], float n, float* xch,
+                                           float* __restrict__ out, bool valid, bool alive) {
+  float du[64];
+  if (alive) {
+    tc::tc_fence_after();
+    tc::tmem_ld32(tmem + lane_base + du_col + 64u * hc, *reinterpret_cast<float(*)[32]>(du));
+    tc::tmem_ld32(tmem + lane_base + du_col + 64u * hc + 32u, *reinterpret_cast<float(*)[32]>(du + 32));
+  } else {
+#pragma unroll
+    for (int q = 0; q < 64; ++q) du[q] = 0.f;
+  }
+  valid = valid && alive;
+  if (alive) tc::tmem_wait_ld();
+  float xd = 0.f;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&xr[q]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(p[e]);
+      xd = fmaf(x.x, du[8 * q + 2 * e], xd);
+      xd = fmaf(x.y, du[8 * q + 2 * e + 1], xd);
+    }
+  }
+  xch[2 * row_in_chunk + hc] = xd;
+  compute_bar();
+  xd = xch[2 * row_in_chunk] + xch[2 * row_in_chunk + 1];
+  if (!valid) return;
+  const float proj = n <= kNormFloor ? 0.f : xd / (n * n);
+  const float inv = 1.f / n;
+  float4* o = reinterpret_cast<float4*>(out + 64 * hc);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&xr[q]);
+    const float2 x0 = __bfloat1622float2(p[0]), x1 = __bfloat1622float2(p[1]);
+    const float2 x2 = __bfloat1622float2(p[2]), x3 = __bfloat1622float2(p[3]);
+    o[2 * q] = make_float4((du[8 * q] - x0.x * proj) * inv, (du[8 * q + 1] - x0.y * proj) * inv,
+                           (du[8 * q + 2] - x1.x * proj) * inv, (du[8 * q + 3] - x1.y * proj) * inv);
+    o[2 * q + 1] = make_float4((du[8 * q + 4] - x2.x * proj) * inv, (du[8 * q + 5] - x2.y * proj) * inv,
+                               (du[8 * q + 6] - x3.x * proj) * inv, (du[8 * q + 7] - x3.y * proj) * inv);
+  }
+}
+
+// ------------------------------- key side ------------------------------------
+constexpr uint32_t K_PK = 0, K_PQ = kTile, K_V = 2 * kTile, K_DO = 3 * kTile, K_RH = 4 * kTile, K_RL = 5 * kTile;
+constexpr uint32_t K_WH = 6 * kTile, K_WL = K_WH + 2 * kWSlab;
+constexpr uint32_t K_CL = K_WL + 2 * kWSlab;            // cl [128], delta [128], r1 [128], exchange [256]
+constexpr uint32_t K_BARS = K_CL + (3 * 128 + 256) * 4;
+// TMEM columns
+constexpr uint32_t TK_KAP = 0, TK_X = 128, TK_DV = 256, TK_DPHI = 384, TK_DU = 128;
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+    race_k_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmPQ,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                         BwdArgs a, Geom g, uint32_t* err) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  Bars* ms = reinterpret_cast<Bars*>(smem + K_BARS);
+  float* sCl = reinterpret_cast<float*>(smem + K_CL);
+  float* sDl = sCl + 128;
+  float* sR1 = sCl + 256;
+  float* sX = sCl + 384;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const size_t head = (size_t)bh * g.N;
+  const bool causal = g.causal;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&ms->in_main, 1);
+    tc::mbar_init(&ms->ready, kComputeThreads);
+    tc::mbar_init(&ms->s_full, 1);
+    tc::mbar_init(&ms->p_full, kComputeThreads);
+    tc::mbar_init(&ms->acc_full, 1);
+    tc::mbar_init(&ms->dh_full, kComputeThreads);
+    tc::mbar_init(&ms->du_full, 1);
+    ms->abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&ms->tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 4 : 2) * kTile);
+      for (int s = 0; s < 2; ++s) {
+        tc::tma_load_3d(smem + K_PK + s * kSlab, &tmPK, &ms->in_main, 64 * s, c * kC, bh);
+        tc::tma_load_3d(smem + K_V + s * kSlab, &tmV, &ms->in_main, 64 * s, c * kC, bh);
+        if (causal) {
+          tc::tma_load_3d(smem + K_PQ + s * kSlab, &tmPQ, &ms->in_main, 64 * s, c * kC, bh);
+          tc::tma_load_3d(smem + K_DO + s * kSlab, &tmdO, &ms->in_main, 64 * s, c * kC, bh);
+        }
+      }
+      tc::mbar_wait(&ms->in_main, 0);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);
+      const uint32_t idNM = tc::idesc_bf16(128, 128, false, true);
+      const uint32_t sb = smem_u32(smem);
+      bool ok = wait_or_abort(&ms->in_main, 0, ms, err, 0x100u);
+      if (ok && causal) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_bf16(tmem + TK_KAP, desc_k(sb + K_PK, kk), desc_k(sb + K_PQ, kk), idNN, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_bf16(tmem + TK_X, desc_k(sb + K_V, kk), desc_k(sb + K_DO, kk), idNN, kk > 0 ? 1u : 0u);
+        tc::mma_commit(&ms->s_full);
+      }
+      ok = ok && wait_or_abort(&ms->ready, 0, ms, err, 0x200u);
+      if (ok) {
+        tc::tc_fence_after();
+        // inter-chunk parts: dv = Phi_K R^V, dPhi = V R^V^T (R as bf16 hi + lo)
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t rb = sb + (part ? K_RL : K_RH);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_bf16(tmem + TK_DV, desc_k(sb + K_PK, kk), desc_mn(rb, kk, kSlab), idNM,
+                         (part > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_bf16(tmem + TK_DPHI, desc_k(sb + K_V, kk), desc_k(rb, kk), idNN, (part > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      if (ok && causal) {
+        ok = wait_or_abort(&ms->p_full, 0, ms, err, 0x400u);
+        if (ok) {
+          tc::tc_fence_after();
+          // intra-chunk parts, A operands from tensor memory
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_bf16_ts(tmem + TK_DV, tmem + TK_KAP + packed_col(kk), desc_mn(sb + K_DO, kk, kSlab), idNM, 1u);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_bf16_ts(tmem + TK_DPHI, tmem + TK_X + packed_col(kk), desc_mn(sb + K_PQ, kk, kSlab), idNM, 1u);
+        }
+      }
+      tc::mma_commit(&ms->acc_full);
+      ok = ok && wait_or_abort(&ms->dh_full, 0, ms, err, 0x800u);
+      if (ok) {
+        tc::tc_fence_after();
+        issue_du(tmem, TK_DU, sb, K_WH, K_WL);
+      }
+      tc::mma_commit(&ms->du_full);
+      tc::mbar_wait(&ms->du_full, 0);
+    }
+  } else {
+    const int ct = threadIdx.x - 64;
+    const int q4 = warp & 3, hc = (warp - 2) >> 2;
+    const int j = 32 * q4 + lane;                     // row of the chunk (TMEM lane)
+    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+    const int row = c * kC + j;
+    const bool valid = row < g.N;
+    // row data for the corner and chain passes, fetched up front
+    float h16[16];
+    load_h(valid ? a.hK + (head + row) * kNH : nullptr, hc, h16);
+    const float nrm = valid ? a.nK[head + row] : 1.f;
+    // ---- staging: suffix statistics of the later chunks, W, per-row scalars ----
+    {
+      const float* ra = a.RA + ((size_t)bh * (g.n_seg + 1) + (causal ? c / g.seg + 1 : 0)) * g.r * g.dp;
+      const float* rb = causal ? a.RB + ((size_t)bh * g.n_c + c) * g.r * g.dp : nullptr;
+      stage_state(ra, rb, g.dp, smem + K_RH, smem + K_RL, sR1, ct);
+      stage_w(a.W, smem + K_WH, smem + K_WL, ct);
+      if (ct < kC) {
+        const int r = c * kC + ct;
+        sCl[ct] = r < g.N ? a.rs.cl[head + r] : 0.f;
+        sDl[ct] = r < g.N ? a.rs.delta[head + r] : 0.f;
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&ms->ready);
+      compute_bar();
+    }
+    bool alive = true;
+    // ---- intra-chunk element-wise pass: (cl_i kappa_ji) and (cl_i X_ji + delta_i), i >= j ----
+    if (causal) {
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full, 0, ms, err, 0x1000u));
+      if (alive) {
+        tc::tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+          float kv[16], xv[16];
+          tc::tmem_ld16(tmem + lane_base + TK_KAP + 64 * hc + c0, kv);
+          tc::tmem_ld16(tmem + lane_base + TK_X + 64 * hc + c0, xv);
+          tc::tmem_wait_ld();
+          uint32_t wk[8], wx[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float pk[2], px[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int i = 64 * hc + c0 + e + u;
+              const bool on = i >= j;
+              const float cl = sCl[i];
+              pk[u] = on ? cl * kv[e + u] : 0.f;
+              px[u] = on ? fmaf(cl, xv[e + u], sDl[i]) : 0.f;
+            }
+            wk[e >> 1] = pack_bf16(pk[0], pk[1]);
+            wx[e >> 1] = pack_bf16(px[0], px[1]);
+          }
+          tc::tmem_st8(tmem + lane_base + TK_KAP + 64 * hc + c0 / 2, wk);
+          tc::tmem_st8(tmem + lane_base + TK_X + 64 * hc + c0 / 2, wx);
+        }
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&ms->p_full);
+      }
+    }
+    // ---- dv rows; corner softmax backward -> dh ----
+    if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->acc_full, 0, ms, err, 0x2000u));
+    if (alive) {
+      tc::tc_fence_after();
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float v[32];
+        tc::tmem_ld32(tmem + lane_base + TK_DV + 64 * hc + 32 * h2, v);
+        tc::tmem_wait_ld();
+        if (valid) {
+          float4* o = reinterpret_cast<float4*>(a.dVacc + (head + row) * kD + 64 * hc + 32 * h2);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+      }
+      corner_pass(tmem, lane_base, hc, TK_DPHI, true, 0u, 0.f, valid ? 1.f : 0.f, sR1, h16, rsqrtf((float)g.L),
+                  1.f / g.tau);
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&ms->dh_full);
+    }
+    uint4 xr[8];
+    load_x((const __nv_bfloat16*)a.K + (head + row) * kD, hc, valid && alive, xr);
+    if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->du_full, 0, ms, err, 0x4000u));
+    chain_pass(tmem, lane_base, hc, j, TK_DU, xr, nrm, sX, a.dKacc + (head + row) * kD, valid, alive);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------- query side ------------------------------------
+namespace {
+constexpr uint32_t Q_DO = 0, Q_V = kTile, Q_PK = 2 * kTile, Q_PH = 3 * kTile, Q_PL = 4 * kTile;
+constexpr uint32_t Q_WH = 5 * kTile, Q_WL = Q_WH + 2 * kWSlab;
+constexpr uint32_t Q_P1 = Q_WL + 2 * kWSlab;            // p1 [128], exchange [256]
+constexpr uint32_t Q_BARS = Q_P1 + (128 + 256) * 4;
+constexpr uint32_t TQ_X = 0, TQ_INTRA = 128, TQ_G = 256, TQ_DU = 384;
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+    race_q_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmdO, const __grid_constant__ CUtensorMap tmV,
+                         const __grid_constant__ CUtensorMap tmPK, BwdArgs a, Geom g, uint32_t* err) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  Bars* ms = reinterpret_cast<Bars*>(smem + Q_BARS);
+  float* sP1 = reinterpret_cast<float*>(smem + Q_P1);
+  float* sX = sP1 + 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x, bh = blockIdx.y;
+  const size_t head = (size_t)bh * g.N;
+  const bool causal = g.causal;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&ms->in_main, 1);
+    tc::mbar_init(&ms->ready, kComputeThreads);
+    tc::mbar_init(&ms->s_full, 1);
+    tc::mbar_init(&ms->p_full, kComputeThreads);
+    tc::mbar_init(&ms->acc_full, 1);
+    tc::mbar_init(&ms->dh_full, kComputeThreads);
+    tc::mbar_init(&ms->du_full, 1);
+    ms->abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&ms->tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 3 : 1) * kTile);
+      for (int s = 0; s < 2; ++s) {
+        tc::tma_load_3d(smem + Q_DO + s * kSlab, &tmdO, &ms->in_main, 64 * s, t * kC, bh);
+        if (causal) {
+          tc::tma_load_3d(smem + Q_V + s * kSlab, &tmV, &ms->in_main, 64 * s, t * kC, bh);
+          tc::tma_load_3d(smem + Q_PK + s * kSlab, &tmPK, &ms->in_main, 64 * s, t * kC, bh);
+        }
+      }
+      tc::mbar_wait(&ms->in_main, 0);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);
+      const uint32_t idNM = tc::idesc_bf16(128, 128, false, true);
+      const uint32_t sb = smem_u32(smem);
+      bool ok = wait_or_abort(&ms->in_main, 0, ms, err, 0x100u);
+      if (ok && causal) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_bf16(tmem + TQ_X, desc_k(sb + Q_DO, kk), desc_k(sb + Q_V, kk), idNN, kk > 0 ? 1u : 0u);
+        tc::mma_commit(&ms->s_full);
+      }
+      ok = ok && wait_or_abort(&ms->ready, 0, ms, err, 0x200u);
+      if (ok) {
+        tc::tc_fence_after();
+        // inter-chunk part: G = dO P^V^T (P as bf16 hi + lo)
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t pb = sb + (part ? Q_PL : Q_PH);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_bf16(tmem + TQ_G, desc_k(sb + Q_DO, kk), desc_k(pb, kk), idNN, (part > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      if (ok && causal) {
+        ok = wait_or_abort(&ms->p_full, 0, ms, err, 0x400u);
+        if (ok) {
+          tc::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_bf16_ts(tmem + TQ_INTRA, tmem + TQ_X + packed_col(kk), desc_mn(sb + Q_PK, kk, kSlab), idNM,
+                            kk > 0 ? 1u : 0u);
+        }
+      }
+      tc::mma_commit(&ms->acc_full);
+      ok = ok && wait_or_abort(&ms->dh_full, 0, ms, err, 0x800u);
+      if (ok) {
+        tc::tc_fence_after();
+        issue_du(tmem, TQ_DU, sb, Q_WH, Q_WL);
+      }
+      tc::mma_commit(&ms->du_full);
+      tc::mbar_wait(&ms->du_full, 0);
+    }
+  } else {
+    const int ct = threadIdx.x - 64;
+    const int q4 = warp & 3, hc = (warp - 2) >> 2;
+    const int i = 32 * q4 + lane;                     // row of the tile (TMEM lane)
+    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+    const int row = t * kC + i;
+    const bool valid = row < g.N;
+    const float cl = valid ? a.rs.cl[head + row] : 0.f;
+    const float de = valid ? a.rs.delta[head + row] : 0.f;
+    float h16[16];
+    load_h(valid ? a.hQ + (head + row) * kNH : nullptr, hc, h16);
+    const float nrm = valid ? a.nQ[head + row] : 1.f;
+    {
+      const float* pa = a.Ast + ((size_t)bh * (g.n_seg + 1) + (causal ? t / g.seg : g.n_seg)) * g.r * g.dp;
+      const float* pb = causal ? a.Bst + ((size_t)bh * g.n_c + t) * g.r * g.dp : nullptr;
+      stage_state(pa, pb, g.dp, smem + Q_PH, smem + Q_PL, sP1, ct);
+      stage_w(a.W, smem + Q_WH, smem + Q_WL, ct);
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&ms->ready);
+      compute_bar();
+    }
+    bool alive = true;
+    // ---- intra-chunk element-wise pass: dkappa_ij = cl_i X_ij + delta_i, j <= i ----
+    if (causal) {
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full, 0, ms, err, 0x1000u));
+      if (alive) {
+        tc::tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+          float xv[16];
+          tc::tmem_ld16(tmem + lane_base + TQ_X + 64 * hc + c0, xv);
+          tc::tmem_wait_ld();
+          uint32_t wx[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const int jj = 64 * hc + c0 + e;
+            const float p0 = jj <= i ? fmaf(cl, xv[e], de) : 0.f;
+            const float p1 = jj + 1 <= i ? fmaf(cl, xv[e + 1], de) : 0.f;
+            wx[e >> 1] = pack_bf16(p0, p1);
+          }
+          tc::tmem_st8(tmem + lane_base + TQ_X + 64 * hc + c0 / 2, wx);
+        }
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&ms->p_full);
+      }
+    }
+    if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->acc_full, 0, ms, err, 0x2000u));
+    if (alive) {
+      tc::tc_fence_after();
+      corner_pass(tmem, lane_base, hc, TQ_INTRA, causal, TQ_G, cl, de, sP1, h16, rsqrtf((float)g.L),
+                  1.f / g.tau);
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&ms->dh_full);
+    }
+    uint4 xr[8];
+    load_x((const __nv_bfloat16*)a.Q + (head + row) * kD, hc, valid && alive, xr);
+    if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->du_full, 0, ms, err, 0x4000u));
+    chain_pass(tmem, lane_base, hc, i, TQ_DU, xr, nrm, sX, a.dQacc + (head + row) * kD, valid, alive);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------- read-out ------------------------------------
+namespace {
+constexpr uint32_t R_PQ = 0, R_PK = kTile, R_V = 2 * kTile, R_PH = 3 * kTile, R_PL = 4 * kTile;
+constexpr uint32_t R_P1 = 5 * kTile;                    // p1 [128], exchange [256]
+constexpr uint32_t R_BARS = R_P1 + (128 + 256) * 4;
+constexpr uint32_t TR_KAP = 0, TR_N = 128;
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+    race_readout_tc_kernel(const __grid_constant__ CUtensorMap tmPQ, const __grid_constant__ CUtensorMap tmPK,
+                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmOlr,
+                           FwdArgs a, Geom g, uint32_t* err) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  Bars* ms = reinterpret_cast<Bars*>(smem + R_BARS);
+  float* sP1 = reinterpret_cast<float*>(smem + R_P1);
+  float* sX = sP1 + 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = g.n_t - 1 - blockIdx.x, bh = blockIdx.y;
+  const size_t head = (size_t)bh * g.N;
+  const bool causal = g.causal;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&ms->in_main, 1);
+    tc::mbar_init(&ms->ready, kComputeThreads);
+    tc::mbar_init(&ms->s_full, 1);
+    tc::mbar_init(&ms->p_full, kComputeThreads);
+    tc::mbar_init(&ms->acc_full, 1);
+    ms->abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&ms->tmem_base, 256);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 3 : 1) * kTile);
+      for (int s = 0; s < 2; ++s) {
+        tc::tma_load_3d(smem + R_PQ + s * kSlab, &tmPQ, &ms->in_main, 64 * s, t * kC, bh);
+        if (causal) {
+          tc::tma_load_3d(smem + R_PK + s * kSlab, &tmPK, &ms->in_main, 64 * s, t * kC, bh);
+          tc::tma_load_3d(smem + R_V + s * kSlab, &tmV, &ms->in_main, 64 * s, t * kC, bh);
+        }
+      }
+      tc::mbar_wait(&ms->in_main, 0);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);
+      const uint32_t idNM = tc::idesc_bf16(128, 128, false, true);
+      const uint32_t sb = smem_u32(smem);
+      bool ok = wait_or_abort(&ms->in_main, 0, ms, err, 0x100u);
+      if (ok && causal) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_bf16(tmem + TR_KAP, desc_k(sb + R_PQ, kk), desc_k(sb + R_PK, kk), idNN, kk > 0 ? 1u : 0u);
+        tc::mma_commit(&ms->s_full);
+      }
+      ok = ok && wait_or_abort(&ms->ready, 0, ms, err, 0x200u);
+      if (ok) {
+        tc::tc_fence_after();
+        // inter-chunk part: N = Phi_Q P^V (P as bf16 hi + lo)
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t pb = sb + (part ? R_PL : R_PH);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_bf16(tmem + TR_N, desc_k(sb + R_PQ, kk), desc_mn(pb, kk, kSlab), idNM,
+                         (part > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      if (ok && causal) {
+        ok = wait_or_abort(&ms->p_full, 0, ms, err, 0x400u);
+        if (ok) {
+          tc::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_bf16_ts(tmem + TR_N, tmem + TR_KAP + packed_col(kk), desc_mn(sb + R_V, kk, kSlab), idNM, 1u);
+        }
+      }
+      tc::mma_commit(&ms->acc_full);
+      tc::mbar_wait(&ms->acc_full, 0);
+    }
+  } else {
+    const int ct = threadIdx.x - 64;
+    const int q4 = warp & 3, hc = (warp - 2) >> 2;
+    const int i = 32 * q4 + lane;                     // row of the tile (TMEM lane)
+    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+    const int row = t * kC + i;
+    const bool valid = row < g.N;
+    {
+      const float* pa = a.Ast + ((size_t)bh * (g.n_seg + 1) + (causal ? t / g.seg : g.n_seg)) * g.r * g.dp;
+      const float* pb = causal ? a.Bst + ((size_t)bh * g.n_c + t) * g.r * g.dp : nullptr;
+      stage_state(pa, pb, g.dp, smem + R_PH, smem + R_PL, sP1, ct);
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&ms->ready);
+      compute_bar();
+    }
+    bool alive = true;
+    float mass = 0.f;                                  // this thread's share of d_lr
+    // ---- intra-chunk kappa_ij, j <= i: bf16 into tensor memory, its row sum into the mass ----
+    if (causal) {
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full, 0, ms, err, 0x1000u));
+      if (alive) {
+        tc::tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+          float kv[16];
+          tc::tmem_ld16(tmem + lane_base + TR_KAP + 64 * hc + c0, kv);
+          tc::tmem_wait_ld();
+          uint32_t wk[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const int jj = 64 * hc + c0 + e;
+            wk[e >> 1] = pack_bf16(jj <= i ? kv[e] : 0.f, jj + 1 <= i ? kv[e + 1] : 0.f);
+            // the mass uses the same bf16 values the product does
+            const float2 r2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wk[e >> 1]));
+            mass += r2.x + r2.y;
+          }
+          tc::tmem_st8(tmem + lane_base + TR_KAP + 64 * hc + c0 / 2, wk);
+        }
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&ms->p_full);
+      }
+    }
+    // inter-chunk mass: Phi(q_i) . p1 over this thread's 64 features (bf16 row from shared memory)
+    if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->in_main, 0, ms, err, 0x8000u));
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      const uint4 v = *reinterpret_cast<const uint4*>(smem + R_PQ + sw_off(i, 64 * hc + 8 * ch, kSlab));
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(p[e]);
+        mass = fmaf(f.x, sP1[64 * hc + 8 * ch + 2 * e], mass);
+        mass = fmaf(f.y, sP1[64 * hc + 8 * ch + 2 * e + 1], mass);
+      }
+    }
+    sX[2 * i + hc] = mass;
+    if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->acc_full, 0, ms, err, 0x2000u));
+    compute_bar();
+    const float dl = sX[2 * i] + sX[2 * i + 1];
+    const float il = dl > 0.f ? 1.f / dl : 0.f;
+    if (alive) {
+      tc::tc_fence_after();
+      // O_lr = N / d_lr as bf16, staged (swizzled) over the Phi(K) tile, then one TMA store
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float v[32];
+        tc::tmem_ld32(tmem + lane_base + TR_N + 64 * hc + 32 * h2, v);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int col = 64 * hc + 32 * h2 + 8 * ch;
+          *reinterpret_cast<uint4*>(smem + R_PK + sw_off(i, col, kSlab)) =
+              make_uint4(pack_bf16(v[8 * ch] * il, v[8 * ch + 1] * il), pack_bf16(v[8 * ch + 2] * il, v[8 * ch + 3] * il),
+                         pack_bf16(v[8 * ch + 4] * il, v[8 * ch + 5] * il), pack_bf16(v[8 * ch + 6] * il, v[8 * ch + 7] * il));
+        }
+      }
+      if (hc == 0 && valid) a.dlr[head + row] = dl;
+    }
+    tc::fence_proxy_async_smem();
+    compute_bar();
+    if (ct == 0 && !*(volatile int*)&ms->abort_flag) {
+      asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];\n"
+                   :: "l"(reinterpret_cast<uint64_t>(&tmOlr)), "r"(smem_u32(smem + R_PK)), "r"(0), "r"(t * kC),
+                      "r"(bh) : "memory");
+      asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];\n"
+                   :: "l"(reinterpret_cast<uint64_t>(&tmOlr)), "r"(smem_u32(smem + R_PK + kSlab)), "r"(64),
+                      "r"(t * kC), "r"(bh) : "memory");
+      asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+      asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+cudaError_t launch_race_readout_tc(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
+  if (!race_bwd_tc_supported(g)) return cudaErrorInvalidValue;
+  CUtensorMap mpq, mpk, mv, mo;
+  if (!tc::map_rows_bf16(&mpq, a.phiQ, g.N, g.BH, kC) || !tc::map_rows_bf16(&mpk, a.phiK, g.N, g.BH, kC) ||
+      !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kC) || !tc::map_rows_bf16(&mo, a.Olr, g.N, g.BH, kC))
+    return cudaErrorInvalidValue;
+  const size_t smem = R_BARS + sizeof(Bars);
+  cudaError_t e = cudaFuncSetAttribute(race_readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  ProfScope ps("race_readout_tc", st);
+  race_readout_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mpq, mpk, mv, mo, a, g, err);
+  return cudaGetLastError();
+}
+
+bool race_bwd_tc_supported(const Geom& g) {
+  return g.d == kD && g.T == kC && g.C == kC && g.r == kR && g.dp == kD + 8;
+}
+
+cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
+  if (!race_bwd_tc_supported(g) || !a.hQ || !a.hK || !a.nQ || !a.nK) return cudaErrorInvalidValue;
+  CUtensorMap mpk, mpq, mv, mdo;
+  if (!tc::map_rows_bf16(&mpk, a.phiK, g.N, g.BH, kC) || !tc::map_rows_bf16(&mpq, a.phiQ, g.N, g.BH, kC) ||
+      !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kC) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, kC))
+    return cudaErrorInvalidValue;
+  {
+    const size_t smem = Q_BARS + sizeof(Bars);
+    cudaError_t e = cudaFuncSetAttribute(race_q_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    ProfScope ps("race_q_bwd_tc", st);
+    race_q_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mdo, mv, mpk, a, g, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const size_t smem = K_BARS + sizeof(Bars);
+  cudaError_t e = cudaFuncSetAttribute(race_k_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  ProfScope ps("race_k_bwd_tc", st);
+  race_k_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mpk, mpq, mv, mdo, a, g, err);
+  return cudaGetLastError();
+}
+
+}  // namespace elsaa

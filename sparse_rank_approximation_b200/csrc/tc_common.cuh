@@ -177,5 +177,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Host: tensor map of a [BH][N][128] bf16 array as (column, row, head) with boxes
+// of 64 columns x `rows` rows, 128-byte swizzle (one 64-column slab per load).
+bool map_rows_bf16(CUtensorMap* m, const void* base, int N, int BH, int rows);
+
 }  // namespace tc
 }  // namespace elsaa

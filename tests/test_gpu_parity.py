@@ -19,6 +19,10 @@ SMALL = {
     "bf16_d128_T128_causal_ragged": small_workload(N=128 * 4 + 5, d=128, block_size=128, topk=2, rank_r=64, H=2),
     "bf16_d64_T128_noncausal": small_workload(N=128 * 3 + 50, d=64, block_size=128, topk=2, rank_r=16,
                                               causal=False),
+    "bf16_d128_T128_r128_causal_ragged": small_workload(N=128 * 6 + 5, d=128, block_size=128, topk=3, rank_r=128,
+                                                        H=2),
+    "bf16_d128_T128_r128_noncausal": small_workload(N=128 * 3 + 50, d=128, block_size=128, topk=2, rank_r=128,
+                                                    causal=False),
     "bf16_d128_T64_r256": small_workload(N=64 * 6, d=128, block_size=64, topk=4, rank_r=256, B=2, H=1),
     "bf16_all_blocks": small_workload(N=64 * 4, d=64, block_size=64, topk=4, rank_r=16, causal=False),
     "f32_config_tiny": WORKLOADS["tiny_f32"],
@@ -77,10 +81,12 @@ def test_forward_backward_small(name):
 
 
 @pytest.mark.parametrize("case", ["k0", "r0_eps0", "lam_gates", "tau_lam", "noncausal"])
-@pytest.mark.parametrize("geom", ["bf16_d64_T64", "bf16_d128_T128", "f32_d64_T64"])
+@pytest.mark.parametrize("geom", ["bf16_d64_T64", "bf16_d128_T128", "bf16_d128_T128_r128", "f32_d64_T64"])
 def test_branch_switches_and_options(case, geom):
-    dtype, d, T = geom.split("_")[0], int(geom.split("_")[1][1:]), int(geom.split("_")[2][1:])
-    base = dict(N=T * 3 + 20, d=d, block_size=T, topk=2, rank_r=32, dtype=dtype, H=2)
+    parts = geom.split("_")
+    dtype, d, T = parts[0], int(parts[1][1:]), int(parts[2][1:])
+    r = int(parts[3][1:]) if len(parts) > 3 else 32
+    base = dict(N=T * 3 + 20, d=d, block_size=T, topk=2, rank_r=r, dtype=dtype, H=2)
     kw, over, lam_vec, gates = {}, {}, False, False
     if case == "k0":
         base["topk"] = 0
