@@ -73,6 +73,23 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, M*
   return false;
 }
 
+// dS = P (cs dP - Delta) for one thread's 64 keys of a query row, as bf16 pairs;
+// MASK: keys after column `lim` get P = 0.
+template <bool MASK>
+__device__ __forceinline__ void dq_softmax_cols(const float (&sv)[64], const float (&dp)[64], float sl2, float lg2,
+                                                float cs, float Dl, int lim, uint32_t (&w)[32]) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    float p0 = ex2_approx(fmaf(sv[c], sl2, -lg2));
+    float p1 = ex2_approx(fmaf(sv[c + 1], sl2, -lg2));
+    if (MASK) {
+      p0 = c > lim ? 0.f : p0;
+      p1 = c + 1 > lim ? 0.f : p1;
+    }
+    w[c >> 1] = pack_bf16(p0 * fmaf(cs, dp[c], -Dl), p1 * fmaf(cs, dp[c + 1], -Dl));
+  }
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kDqThreads, 1)
@@ -221,16 +238,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const bool mask = (g.causal && b == t) || kvalid < kT;
         const int lim = min(kvalid - 1, (g.causal && b == t) ? row : kT - 1) - 64 * half;
         uint32_t w[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float p0 = ex2_approx(fmaf(sv[c], sl2, -lg2));
-          float p1 = ex2_approx(fmaf(sv[c + 1], sl2, -lg2));
-          if (mask) {
-            p0 = c > lim ? 0.f : p0;
-            p1 = c + 1 > lim ? 0.f : p1;
-          }
-          w[c >> 1] = pack_bf16(p0 * (cs * dp[c] - Dl), p1 * (cs * dp[c + 1] - Dl));
-        }
+        // block-uniform: only the diagonal block and a ragged last block need the mask
+        if (mask)
+          dq_softmax_cols<true>(sv, dp, sl2, lg2, cs, Dl, lim, w);
+        else
+          dq_softmax_cols<false>(sv, dp, sl2, lg2, cs, Dl, lim, w);
         // the dS buffer is free once dQ of block j-1 has been accumulated
         if (j >= 1) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->dq_done, (j - 1) & 1, ms, err, 64u));
         if (alive) {
@@ -325,6 +337,38 @@ struct KvMisc {
   int abort_flag;
 };
 }  // namespace
+
+// One thread's 32 queries of a unit: S^T and dP^T (fp32, TMEM) -> (P^T cs) and dS^T
+// (bf16 pairs) written back over the columns already read, 16 columns at a time.
+// MASK: queries outside [lo, hi) get P = 0.
+template <bool MASK>
+__device__ __forceinline__ void dkdv_softmax_cols(uint32_t tmem, uint32_t st_col, uint32_t dp_col, const float4* sc,
+                                                  float sl2, int lo, int hi) {
+#pragma unroll
+  for (int c0 = 0; c0 < 32; c0 += 16) {
+    float sv[16], dp[16];
+    tc::tmem_ld16(tmem + st_col + c0, sv);
+    tc::tmem_ld16(tmem + dp_col + c0, dp);
+    tc::tmem_wait_ld();
+    uint32_t wp[8], wd[8];
+#pragma unroll
+    for (int c = 0; c < 16; c += 2) {
+      float pv[2], dv[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float4 q = sc[c0 + c + e];          // (log2 d_s, cs, Delta)
+        float p = ex2_approx(fmaf(sv[c + e], sl2, -q.x));
+        if (MASK && (c0 + c + e < lo || c0 + c + e >= hi)) p = 0.f;
+        pv[e] = p * q.y;
+        dv[e] = p * fmaf(q.y, dp[c + e], -q.z);
+      }
+      wp[c >> 1] = pack_bf16(pv[0], pv[1]);
+      wd[c >> 1] = pack_bf16(dv[0], dv[1]);
+    }
+    tc::tmem_st8(tmem + st_col + c0 / 2, wp);
+    tc::tmem_st8(tmem + dp_col + c0 / 2, wd);
+  }
+}
 
 __global__ void __launch_bounds__(kKvThreads, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -481,33 +525,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       // valid queries of this thread: c in [lo, hi) (causal diagonal, sequence end, key row)
       const int lo = diag ? row - q0 : 0;
       const int hi = key_ok ? qvalid : 0;
-#pragma unroll
-      for (int c0 = 0; c0 < 32; c0 += 16) {
-        // 16 columns at a time keeps S^T, dP^T and the scalars within the register budget;
-        // the packed results of columns c0.. land in columns c0/2.., which this thread
-        // has already read
-        float sv[16], dp[16];
-        tc::tmem_ld16(tmem + lane_base + tm_st(b2) + 32 * hq + c0, sv);
-        tc::tmem_ld16(tmem + lane_base + tm_dpt(b2) + 32 * hq + c0, dp);
-        tc::tmem_wait_ld();
-        uint32_t wp[8], wd[8];
-#pragma unroll
-        for (int c = 0; c < 16; c += 2) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float4 q = sc[c0 + c + e];          // (log2 d_s, cs, Delta)
-            float p = ex2_approx(fmaf(sv[c + e], sl2, -q.x));
-            if (masked && (c0 + c + e < lo || c0 + c + e >= hi)) p = 0.f;
-            pv[e] = p * q.y;
-            dv[e] = p * (q.y * dp[c + e] - q.z);
-          }
-          wp[c >> 1] = pack_bf16(pv[0], pv[1]);
-          wd[c >> 1] = pack_bf16(dv[0], dv[1]);
-        }
-        tc::tmem_st8(tmem + lane_base + tm_st(b2) + 32 * hq + c0 / 2, wp);
-        tc::tmem_st8(tmem + lane_base + tm_dpt(b2) + 32 * hq + c0 / 2, wd);
-      }
+      // masking is needed only on the causal diagonal, at the end of the sequence and
+      // for padding keys: a warp-uniform branch keeps it out of the common path
+      if (__any_sync(0xffffffffu, masked))
+        dkdv_softmax_cols<true>(tmem, lane_base + tm_st(b2) + 32 * hq, lane_base + tm_dpt(b2) + 32 * hq, sc, sl2, lo, hi);
+      else
+        dkdv_softmax_cols<false>(tmem, lane_base + tm_st(b2) + 32 * hq, lane_base + tm_dpt(b2) + 32 * hq, sc, sl2, lo,
+                                 hi);
       tc::tmem_wait_st();
       tc::tc_fence_before();
       tc::mbar_arrive(&ms->p_full[b2]);
