@@ -50,15 +50,17 @@ __device__ __forceinline__ void tma_store_wait() {
 
 // ------------------------------- dq ----------------------------------------
 constexpr uint32_t DQ_Q = 0, DQ_DO = kTile;
-__host__ __device__ constexpr uint32_t dq_k(int s) { return kTile * (2 + 2 * s); }
-__host__ __device__ constexpr uint32_t dq_v(int s) { return kTile * (3 + 2 * s); }
-constexpr uint32_t DQ_DS = 6 * kTile;
-constexpr uint32_t DQ_MISC = 7 * kTile;
-constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256;
-constexpr int kDqThreads = 320;          // producer, MMA, 8 softmax warps
+constexpr int kDqKStages = 3, kDqVStages = 2;
+__host__ __device__ constexpr uint32_t dq_k(int s) { return kTile * (2 + s); }                 // K ring
+__host__ __device__ constexpr uint32_t dq_v(int s) { return kTile * (2 + kDqKStages + s); }    // V ring
+constexpr uint32_t DQ_MISC = kTile * (2 + kDqKStages + kDqVStages);
+// TMEM: S and dP (fp32), the dQ accumulator, dS (bf16 pairs) double-buffered
+constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256, TM_DS = 384;
+constexpr int kDqThreads = 352;          // Q/dO + K producer, MMA, 8 softmax warps, V producer
 
 struct DqMisc {
-  uint64_t qd_full, kv_full[2], kv_empty[2], s_full, st_free, ds_full, dq_done, drain;
+  uint64_t qd_full, k_full[kDqKStages], k_empty[kDqKStages], v_full[kDqVStages], v_empty[kDqVStages], s_full,
+      st_free, ds_full[2], done;
   uint32_t tmem_base;
   int abort_flag;
   int idx[32];
@@ -109,15 +111,19 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   const int* my_idx = a.idx + ((size_t)bh * g.n_t + t) * g.k;
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->qd_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&ms->kv_full[s], 1);
-      tc::mbar_init(&ms->kv_empty[s], 1);
+    for (int s = 0; s < kDqKStages; ++s) {
+      tc::mbar_init(&ms->k_full[s], 1);
+      tc::mbar_init(&ms->k_empty[s], 1);
+    }
+    for (int s = 0; s < kDqVStages; ++s) {
+      tc::mbar_init(&ms->v_full[s], 1);
+      tc::mbar_init(&ms->v_empty[s], 1);
     }
     tc::mbar_init(&ms->s_full, 1);
     tc::mbar_init(&ms->st_free, kSoftmaxThreads);
-    tc::mbar_init(&ms->ds_full, kSoftmaxThreads);
-    tc::mbar_init(&ms->dq_done, 1);
-    tc::mbar_init(&ms->drain, 1);
+    tc::mbar_init(&ms->ds_full[0], kSoftmaxThreads);
+    tc::mbar_init(&ms->ds_full[1], kSoftmaxThreads);
+    tc::mbar_init(&ms->done, 1);
     ms->abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -133,28 +139,33 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   int n_sel = 0;
   while (n_sel < g.k && n_sel < 32 && ms->idx[n_sel] >= 0) ++n_sel;
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
+  if (warp == 0 || warp == 10) {
+    // ---------------- TMA producers: warp 0 Q, dO and the K ring; warp 10 the V ring ----------------
     if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&ms->qd_full, 2 * kTile);
-      tc::tma_load_3d(smem + DQ_Q, &tmQ, &ms->qd_full, 0, t * kT, bh);
-      tc::tma_load_3d(smem + DQ_Q + kSlab, &tmQ, &ms->qd_full, 64, t * kT, bh);
-      tc::tma_load_3d(smem + DQ_DO, &tmdO, &ms->qd_full, 0, t * kT, bh);
-      tc::tma_load_3d(smem + DQ_DO + kSlab, &tmdO, &ms->qd_full, 64, t * kT, bh);
+      const bool kside = warp == 0;
+      const int NS = kside ? kDqKStages : kDqVStages;
+      uint64_t* full = kside ? ms->k_full : ms->v_full;
+      uint64_t* empty = kside ? ms->k_empty : ms->v_empty;
+      if (kside) {
+        tc::mbar_arrive_expect_tx(&ms->qd_full, 2 * kTile);
+        tc::tma_load_3d(smem + DQ_Q, &tmQ, &ms->qd_full, 0, t * kT, bh);
+        tc::tma_load_3d(smem + DQ_Q + kSlab, &tmQ, &ms->qd_full, 64, t * kT, bh);
+        tc::tma_load_3d(smem + DQ_DO, &tmdO, &ms->qd_full, 0, t * kT, bh);
+        tc::tma_load_3d(smem + DQ_DO + kSlab, &tmdO, &ms->qd_full, 64, t * kT, bh);
+      }
       int issued = 0;
       for (int j = 0; j < n_sel; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !wait_or_abort(&ms->kv_empty[s], ((j >> 1) + 1) & 1, ms, err, 1u)) break;
+        const int s = j % NS;
+        if (j >= NS && !wait_or_abort(&empty[s], ((j / NS) - 1) & 1, ms, err, kside ? 1u : 2u)) break;
         const int b = ms->idx[j];
-        tc::mbar_arrive_expect_tx(&ms->kv_full[s], 2 * kTile);
-        tc::tma_load_3d(smem + dq_k(s), &tmK, &ms->kv_full[s], 0, b * kT, bh);
-        tc::tma_load_3d(smem + dq_k(s) + kSlab, &tmK, &ms->kv_full[s], 64, b * kT, bh);
-        tc::tma_load_3d(smem + dq_v(s), &tmV, &ms->kv_full[s], 0, b * kT, bh);
-        tc::tma_load_3d(smem + dq_v(s) + kSlab, &tmV, &ms->kv_full[s], 64, b * kT, bh);
+        unsigned char* dst = smem + (kside ? dq_k(s) : dq_v(s));
+        tc::mbar_arrive_expect_tx(&full[s], kTile);
+        tc::tma_load_3d(dst, kside ? &tmK : &tmV, &full[s], 0, b * kT, bh);
+        tc::tma_load_3d(dst + kSlab, kside ? &tmK : &tmV, &full[s], 64, b * kT, bh);
         issued = j + 1;
       }
-      tc::mbar_wait(&ms->qd_full, 0);
-      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) tc::mbar_wait(&ms->kv_full[j & 1], (j >> 1) & 1);
+      if (kside) tc::mbar_wait(&ms->qd_full, 0);
+      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j) tc::mbar_wait(&full[j % NS], (j / NS) & 1);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -162,46 +173,47 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);   // both operands K-major
       const uint32_t idNM = tc::idesc_bf16(128, kD, false, true);     // B MN-major
       const uint32_t sb = smem_u32(smem);
-      bool ok = wait_or_abort(&ms->qd_full, 0, ms, err, 2u);
+      bool ok = wait_or_abort(&ms->qd_full, 0, ms, err, 4u);
       int dq_issued = 0;
+      // dQ += dS K: dS (bf16 pairs, TMEM buffer jj & 1) is the A operand
       auto issue_dq = [&](int jj) -> bool {
-        if (!wait_or_abort(&ms->ds_full, jj & 1, ms, err, 4u)) return false;
+        if (!wait_or_abort(&ms->ds_full[jj & 1], (jj >> 1) & 1, ms, err, 8u)) return false;
         tc::tc_fence_after();
-        const uint32_t kb = sb + dq_k(jj & 1);
+        const uint32_t kb = sb + dq_k(jj % kDqKStages);
 #pragma unroll
-        for (int kk = 0; kk < kT / 16; ++kk) {
-          const uint64_t ad = tc::sw128_desc(sb + DQ_DS + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::sw128_desc(kb + kk * 2048, kSlab, 1024);
-          tc::mma_bf16(tmem + TM_DQ, ad, bd, idNM, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc::mma_commit(&ms->kv_empty[jj & 1]);
-        tc::mma_commit(&ms->dq_done);
+        for (int kk = 0; kk < kT / 16; ++kk)
+          tc::mma_bf16_ts(tmem + TM_DQ, tmem + TM_DS + 64u * (jj & 1) + 8u * kk,
+                          tc::sw128_desc(kb + kk * 2048, kSlab, 1024), idNM, (jj > 0 || kk > 0) ? 1u : 0u);
+        tc::mma_commit(&ms->k_empty[jj % kDqKStages]);
         dq_issued = jj + 1;
         return true;
       };
       for (int j = 0; ok && j < n_sel; ++j) {
-        const int s = j & 1;
-        if (!wait_or_abort(&ms->kv_full[s], (j >> 1) & 1, ms, err, 8u)) break;
-        if (j >= 1 && !wait_or_abort(&ms->st_free, (j - 1) & 1, ms, err, 16u)) break;
+        const int sv = j % kDqVStages, sk = j % kDqKStages;
+        if (!wait_or_abort(&ms->v_full[sv], (j / kDqVStages) & 1, ms, err, 16u)) break;
+        if (j >= 1 && !wait_or_abort(&ms->st_free, (j - 1) & 1, ms, err, 32u)) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+          tc::mma_bf16(tmem + TM_DP, tc::sw128_desc(sb + DQ_DO + off, 16, 1024),
+                       tc::sw128_desc(sb + dq_v(sv) + off, 16, 1024), idNN, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&ms->v_empty[sv]);              // V slot free once dP is done
+        if (!wait_or_abort(&ms->k_full[sk], (j / kDqKStages) & 1, ms, err, 64u)) break;
         tc::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
           tc::mma_bf16(tmem + TM_S, tc::sw128_desc(sb + DQ_Q + off, 16, 1024),
-                       tc::sw128_desc(sb + dq_k(s) + off, 16, 1024), idNN, kk > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
-          tc::mma_bf16(tmem + TM_DP, tc::sw128_desc(sb + DQ_DO + off, 16, 1024),
-                       tc::sw128_desc(sb + dq_v(s) + off, 16, 1024), idNN, kk > 0 ? 1u : 0u);
+                       tc::sw128_desc(sb + dq_k(sk) + off, 16, 1024), idNN, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(&ms->s_full);
         if (j >= 1 && !issue_dq(j - 1)) break;
       }
       if (n_sel > 0 && dq_issued == n_sel - 1) issue_dq(n_sel - 1);
-      tc::mma_commit(&ms->drain);
-      tc::mbar_wait(&ms->drain, 0);
+      tc::mma_commit(&ms->done);
+      tc::mbar_wait(&ms->done, 0);
     }
   } else {
     // ---------------- softmax: half a query row per thread ----------------
@@ -215,64 +227,58 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const float lg2 = sc.x, cs = sc.y, Dl = sc.z;
     const float sl2 = g.scale * kLog2e;
     bool alive = true;
-    for (int j = 0; j < n_sel; ++j) {
+    for (int j = 0; j < n_sel && alive; ++j) {
       float sv[64], dp[64];
-      if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full, j & 1, ms, err, 32u));
-      if (alive) {
-        tc::tc_fence_after();
-        float tmp[32];
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full, j & 1, ms, err, 128u));
+      if (!alive) break;
+      tc::tc_fence_after();
+      tc::tmem_ld32(tmem + lane_base + TM_S + 64 * half, *reinterpret_cast<float(*)[32]>(sv));
+      tc::tmem_ld32(tmem + lane_base + TM_S + 64 * half + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
+      tc::tmem_ld32(tmem + lane_base + TM_DP + 64 * half, *reinterpret_cast<float(*)[32]>(dp));
+      tc::tmem_ld32(tmem + lane_base + TM_DP + 64 * half + 32, *reinterpret_cast<float(*)[32]>(dp + 32));
+      tc::tmem_wait_ld();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&ms->st_free);
+      const int b = ms->idx[j];
+      const int kvalid = g.N - b * kT;
+      const bool mask = (g.causal && b == t) || kvalid < kT;
+      const int lim = min(kvalid - 1, (g.causal && b == t) ? row : kT - 1) - 64 * half;
+      uint32_t w[32];
+      // block-uniform: only the diagonal block and a ragged last block need the mask
+      if (mask)
+        dq_softmax_cols<true>(sv, dp, sl2, lg2, cs, Dl, lim, w);
+      else
+        dq_softmax_cols<false>(sv, dp, sl2, lg2, cs, Dl, lim, w);
+      // dS (keys 64 half .. 64 half + 63 of this row) into TMEM buffer j & 1; the product that
+      // read this buffer (block j - 2) finished before S_j was computed
+      const uint32_t dcol = TM_DS + 64u * (j & 1) + 32u * half;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tc::tmem_ld32(tmem + lane_base + TM_S + 64 * half + 32 * c, tmp);
+      for (int q = 0; q < 4; ++q) {
+        uint32_t w8[8];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sv[32 * c + i] = tmp[i];
-          tc::tmem_ld32(tmem + lane_base + TM_DP + 64 * half + 32 * c, tmp);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) dp[32 * c + i] = tmp[i];
-        }
-        tc::tmem_wait_ld();
-        tc::tc_fence_before();
-        tc::mbar_arrive(&ms->st_free);
-        const int b = ms->idx[j];
-        const int kvalid = g.N - b * kT;
-        const bool mask = (g.causal && b == t) || kvalid < kT;
-        const int lim = min(kvalid - 1, (g.causal && b == t) ? row : kT - 1) - 64 * half;
-        uint32_t w[32];
-        // block-uniform: only the diagonal block and a ragged last block need the mask
-        if (mask)
-          dq_softmax_cols<true>(sv, dp, sl2, lg2, cs, Dl, lim, w);
-        else
-          dq_softmax_cols<false>(sv, dp, sl2, lg2, cs, Dl, lim, w);
-        // the dS buffer is free once dQ of block j-1 has been accumulated
-        if (j >= 1) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->dq_done, (j - 1) & 1, ms, err, 64u));
-        if (alive) {
-          unsigned char* drow = smem + DQ_DS + half * kSlab + row * 128;
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
-            *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) =
-                make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
-          tc::fence_proxy_async_smem();
-          tc::tc_fence_before();
-          tc::mbar_arrive(&ms->ds_full);
-        }
+        for (int e = 0; e < 8; ++e) w8[e] = w[8 * q + e];
+        tc::tmem_st8(tmem + lane_base + dcol + 8 * q, w8);
       }
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&ms->ds_full[j & 1]);
     }
     // ---------------- epilogue: dQ = scale dQ_sparse + dQ_lowrank, bf16 TMA store ----------------
     float o[64];
 #pragma unroll
     for (int c = 0; c < 64; ++c) o[c] = 0.f;
     if (alive && n_sel > 0) {
-      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->dq_done, (n_sel - 1) & 1, ms, err, 128u));
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->done, 0, ms, err, 256u));
       if (alive) {
         tc::tc_fence_after();
         float tmp[32];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           tc::tmem_ld32(tmem + lane_base + TM_DQ + 64 * half + 32 * c, tmp);
+          tc::tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[32 * c + i] = tmp[i] * g.scale;
         }
-        tc::tmem_wait_ld();
       }
     }
     if (alive && row_ok && a.dQacc) {
@@ -286,8 +292,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         o[4 * c + 3] += v.w;
       }
     }
-    // the dS buffer is free after the last dQ product: stage the bf16 tile there
-    unsigned char* orow = smem + DQ_DS + half * kSlab + row * 128;
+    // every product has completed: stage the bf16 tile in the Q buffer
+    unsigned char* orow = smem + DQ_Q + half * kSlab + row * 128;
 #pragma unroll
     for (int ch = 0; ch < 8; ++ch)
       *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) =
@@ -296,8 +302,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     tc::fence_proxy_async_smem();
     softmax_bar();
     if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
-      tma_store_3d(&tmdQ, smem + DQ_DS, 0, t * kT, bh);
-      tma_store_3d(&tmdQ, smem + DQ_DS + kSlab, 64, t * kT, bh);
+      tma_store_3d(&tmdQ, smem + DQ_Q, 0, t * kT, bh);
+      tma_store_3d(&tmdQ, smem + DQ_Q + kSlab, 64, t * kT, bh);
       tma_store_wait();
     }
   }
