@@ -3,20 +3,21 @@
 // denominator-aware fusion epilogue (ELSAA paper §3.2, §3.3 Eq. 5, §1 Eq. 4).
 //
 // One CTA per (head, query tile), 11 warps:
-//   warp 0      TMA producer of Q and of the K ring (2 stages); once the last
+//   warp 0      TMA producer of Q and of the K ring (3 stages); once the last
 //               score MMA is done it prefetches the tile's low-rank output O_lr
 //               into a K stage for the epilogue;
 //   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of two TMEM
-//               score buffers, then O += P_{j-1} V_{j-1} into the TMEM output;
-//   warp 2      TMA producer of the V ring (2 stages);
+//               score buffers, then O += P_{j-1} V_{j-1} into the TMEM output
+//               with P_{j-1} read from tensor memory;
+//   warp 2      TMA producer of the V ring (3 stages);
 //   warps 3-10  softmax: each query row is split over two warps (64 score
 //               columns each) that exchange their partial row max; online
 //               softmax in fp32 with lazy rescaling (O and l are rescaled only
 //               when the running max grows by more than 2^16, after P_j is
-//               written and just before it is released); P_j goes to one of
-//               two shared buffers as bf16 in the swizzled K-major layout; the
-//               epilogue normalises O, applies the fusion and writes O and O_s
-//               through shared memory with TMA stores.
+//               written and just before it is released); P_j (bf16 pairs)
+//               overwrites the score columns it came from and is the A operand
+//               of the PV product; the epilogue normalises O, applies the
+//               fusion and writes O and O_s through shared memory with TMA stores.
 // Operand tiles are 64-column slabs with 128-byte swizzle, as TMA writes them.
 // Every mbarrier wait is bounded; a timeout sets a bit in the caller's error
 // word, the CTA drains its copies and MMAs, frees TMEM and exits.
@@ -34,10 +35,12 @@ constexpr int kD = 128;                  // head dimension
 constexpr uint32_t kSlab = kT * 128;     // one [128 rows][64 bf16] swizzled slab
 constexpr uint32_t kTile = 2 * kSlab;    // 128 x 128 bf16
 constexpr uint32_t OFF_Q = 0;
-__host__ __device__ constexpr uint32_t off_k(int s) { return kTile * (1 + 2 * s); }   // K stage s
-__host__ __device__ constexpr uint32_t off_v(int s) { return kTile * (2 + 2 * s); }   // V stage s
-__host__ __device__ constexpr uint32_t off_p(int b) { return kTile * (5 + b); }       // P buffer b
-constexpr uint32_t OFF_MISC = 7 * kTile;
+constexpr int kStages = 3;                 // K and V ring depth
+__host__ __device__ constexpr uint32_t off_k(int s) { return kTile * (1 + s); }              // K stage s
+__host__ __device__ constexpr uint32_t off_v(int s) { return kTile * (1 + kStages + s); }    // V stage s
+constexpr uint32_t OFF_MISC = (1 + 2 * kStages) * kTile;
+// column of the K = 16 step kk of P (key 64 h + m of a row sits at column 64 h + m / 2)
+__host__ __device__ constexpr uint32_t p_col(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t TM_O = 0;
 __host__ __device__ constexpr uint32_t tm_s(int s) { return 128u + 128u * s; }         // score buffer s
@@ -46,7 +49,8 @@ constexpr int kThreads = 352;
 constexpr int kSoftmaxThreads = 256;
 
 struct Misc {
-  uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full[2], p_full[2],
+      pv_done[2];
   uint64_t olr_full, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -99,13 +103,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int* my_idx = a.idx + ((size_t)bh * g.n_t + t) * g.k;
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&ms->k_full[s], 1);
       tc::mbar_init(&ms->k_empty[s], 1);
       tc::mbar_init(&ms->v_full[s], 1);
       tc::mbar_init(&ms->v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&ms->s_full[s], 1);
-      tc::mbar_init(&ms->s_free[s], kSoftmaxThreads);
       tc::mbar_init(&ms->p_full[s], kSoftmaxThreads);
       tc::mbar_init(&ms->pv_done[s], 1);
     }
@@ -141,8 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       bool alive = true;
       for (int j = 0; j < n_sel; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !wait_or_abort(&empty[s], ((j >> 1) + 1) & 1, ms, err, is_k ? 1u : 512u)) {
+        const int s = j % kStages;
+        if (j >= kStages && !wait_or_abort(&empty[s], ((j / kStages) - 1) & 1, ms, err, is_k ? 1u : 512u)) {
           alive = false;
           break;
         }
@@ -156,8 +161,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool lr_issued = false;
       if (is_k && alive) {
         // the low-rank output goes into K stage 0 once every score MMA has read its K tile
-        for (int j = (n_sel > 2 ? n_sel - 2 : 0); alive && j < n_sel; ++j)
-          alive = wait_or_abort(&ms->k_empty[j & 1], (j >> 1) & 1, ms, err, 2048u);
+        for (int j = (n_sel > kStages ? n_sel - kStages : 0); alive && j < n_sel; ++j)
+          alive = wait_or_abort(&ms->k_empty[j % kStages], (j / kStages) & 1, ms, err, 2048u);
         if (alive) {
           tc::mbar_arrive_expect_tx(&ms->olr_full, kTile);
           tc::tma_load_3d(smem + off_k(0), &tmLr, &ms->olr_full, 0, t * kT, bh);
@@ -168,39 +173,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       // drain: every copy this thread started has landed before the CTA may exit
       if (is_k) tc::mbar_wait(&ms->q_full, 0);
       if (lr_issued) tc::mbar_wait(&ms->olr_full, 0);
-      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) tc::mbar_wait(&full[j & 1], (j >> 1) & 1);
+      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+        tc::mbar_wait(&full[j % kStages], (j / kStages) & 1);
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
     if (lane == 0) {
       const uint32_t idS = tc::idesc_bf16(128, 128, false, false);   // Q (K-major) x K (K-major)
-      const uint32_t idPV = tc::idesc_bf16(128, kD, false, true);    // P (K-major) x V (MN-major)
+      const uint32_t idPV = tc::idesc_bf16(128, kD, false, true);    // P (TMEM) x V (MN-major)
       const uint32_t sbase = smem_u32(smem);
       bool ok = wait_or_abort(&ms->q_full, 0, ms, err, 2u);
       int pv_issued = 0;
       auto issue_pv = [&](int jj) -> bool {
         if (!wait_or_abort(&ms->p_full[jj & 1], (jj >> 1) & 1, ms, err, 4u)) return false;
-        if (!wait_or_abort(&ms->v_full[jj & 1], (jj >> 1) & 1, ms, err, 1024u)) return false;
+        if (!wait_or_abort(&ms->v_full[jj % kStages], (jj / kStages) & 1, ms, err, 1024u)) return false;
         tc::tc_fence_after();
-        const uint32_t vb = sbase + off_v(jj & 1);
-        const uint32_t pb = sbase + off_p(jj & 1);
+        const uint32_t vb = sbase + off_v(jj % kStages);
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk) {
-          const uint64_t ad = tc::sw128_desc(pb + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = tc::sw128_desc(vb + kk * 2048, kSlab, 1024);
-          tc::mma_bf16(tmem + TM_O, ad, bd, idPV, (jj > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_bf16_ts(tmem + TM_O, tmem + tm_s(jj & 1) + p_col(kk), bd, idPV, (jj > 0 || kk > 0) ? 1u : 0u);
         }
-        tc::mma_commit(&ms->v_empty[jj & 1]);
+        tc::mma_commit(&ms->v_empty[jj % kStages]);
         tc::mma_commit(&ms->pv_done[jj & 1]);
         pv_issued = jj + 1;
         return true;
       };
+      // S_j reuses the TMEM columns of P_{j-2}: the PV product that reads them was issued
+      // earlier, and tcgen05 MMAs of one thread run in issue order
       for (int j = 0; ok && j < n_sel; ++j) {
-        const int s = j & 1;
-        if (!wait_or_abort(&ms->k_full[s], (j >> 1) & 1, ms, err, 8u)) break;
-        if (j >= 2 && !wait_or_abort(&ms->s_free[s], ((j >> 1) + 1) & 1, ms, err, 16u)) break;
+        const int s = j & 1, sk = j % kStages;
+        if (!wait_or_abort(&ms->k_full[sk], (j / kStages) & 1, ms, err, 8u)) break;
         tc::tc_fence_after();
-        const uint32_t kb = sbase + off_k(s);
+        const uint32_t kb = sbase + off_k(sk);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t ad = tc::sw128_desc(sbase + OFF_Q + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
@@ -208,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mma_bf16(tmem + tm_s(s), ad, bd, idS, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(&ms->s_full[s]);
-        tc::mma_commit(&ms->k_empty[s]);
+        tc::mma_commit(&ms->k_empty[sk]);
         if (j >= 1 && !issue_pv(j - 1)) break;
       }
       if (n_sel > 0 && pv_issued == n_sel - 1) issue_pv(n_sel - 1);
@@ -249,8 +254,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) sv[32 + i] = tmp[i];
         tc::tmem_wait_ld();
-        tc::tc_fence_before();
-        tc::mbar_arrive(&ms->s_free[s]);
         const int b = ms->idx[j];
         const int kvalid = g.N - b * kT;
         if ((g.causal && b == t) || kvalid < kT) {   // block-uniform: only the diagonal / ragged block masks
@@ -280,28 +283,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           lp *= alpha;
           m_used = m_new;
         }
-        // P buffer j&1 is free once the PV product of block j-2 has finished
-        if (alive && j >= 2)
-          alive = __all_sync(0xffffffffu, wait_or_abort(&ms->pv_done[s], ((j >> 1) + 1) & 1, ms, err, 256u));
+        // P_j (bf16 pairs) over the first half of this thread's score columns: the
+        // PV product of block j-2 read that buffer before S_j was written into it
         if (alive) {
           const float msub = m_used == -INFINITY ? 0.f : m_used;
           float rs0 = 0.f, rs1 = 0.f;
-          unsigned char* prow = smem + off_p(s) + half * kSlab + row * 128;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            uint32_t w[4];
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t w[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float p0 = ex2_approx(fmaf(sv[8 * ch + 2 * e], sl2, -msub));
-              const float p1 = ex2_approx(fmaf(sv[8 * ch + 2 * e + 1], sl2, -msub));
+            for (int e = 0; e < 8; ++e) {
+              const float p0 = ex2_approx(fmaf(sv[16 * ch + 2 * e], sl2, -msub));
+              const float p1 = ex2_approx(fmaf(sv[16 * ch + 2 * e + 1], sl2, -msub));
               rs0 += p0;
               rs1 += p1;
               w[e] = pack_bf16(p0, p1);
             }
-            *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            tc::tmem_st8(tmem + lane_base + tm_s(s) + 64 * half + 8 * ch, w);
           }
           lp += rs0 + rs1;
-          tc::fence_proxy_async_smem();
+          tc::tmem_wait_st();
         }
         // O holds the products through block j-1; a moved reference max rescales it (this half
         // of the columns) once that product is done, before P_j is released to the MMA warp.
@@ -352,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->olr_full, 0, ms, err, 4096u));
     softmax_bar();
     const float l = ms->red[rb][row] + ms->red[rb][128 + row];
-    // every PV product is done: both P buffers hold the outgoing O (buffer 1) and O_s (buffer 0)
+    // every PV product is done: V stages 0 and 1 hold the outgoing O and O_s
     if (alive) {
       const float logd = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
@@ -360,8 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float gl = a.glr ? glr_in : 1.f - mf;
       const float cs = gs * mf;
       const unsigned char* lrow = smem + off_k(0) + half * kSlab + row * 128;
-      unsigned char* orow = smem + off_p(1) + half * kSlab + row * 128;
-      unsigned char* srow = smem + off_p(0) + half * kSlab + row * 128;
+      unsigned char* orow = smem + off_v(0) + half * kSlab + row * 128;
+      unsigned char* srow = smem + off_v(1) + half * kSlab + row * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         const int sw = (ch ^ (row & 7)) << 4;
@@ -385,10 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_proxy_async_smem();
     softmax_bar();
     if (threadIdx.x == 96 && !*(volatile int*)&ms->abort_flag) {
-      tma_store_3d(&tmO, smem + off_p(1), 0, t * kT, bh);
-      tma_store_3d(&tmO, smem + off_p(1) + kSlab, 64, t * kT, bh);
-      tma_store_3d(&tmS, smem + off_p(0), 0, t * kT, bh);
-      tma_store_3d(&tmS, smem + off_p(0) + kSlab, 64, t * kT, bh);
+      tma_store_3d(&tmO, smem + off_v(0), 0, t * kT, bh);
+      tma_store_3d(&tmO, smem + off_v(0) + kSlab, 64, t * kT, bh);
+      tma_store_3d(&tmS, smem + off_v(1), 0, t * kT, bh);
+      tma_store_3d(&tmS, smem + off_v(1) + kSlab, 64, t * kT, bh);
       asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
       asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
     }
