@@ -317,36 +317,28 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 
 // ------------------------------- dkdv ------------------------------------------
 namespace {
-constexpr uint32_t kHalf = 64 * 128;                       // [64 rows][64 bf16] swizzled slab
-constexpr int kStages = 4;
+constexpr int kStages = 2;
 constexpr uint32_t KV_K = 0, KV_V = kTile;
-__host__ __device__ constexpr uint32_t kv_q(int s) { return 2 * kTile + s * 4 * kHalf; }   // Q half, stage s
-__host__ __device__ constexpr uint32_t kv_do(int s) { return kv_q(s) + 2 * kHalf; }      // dO half, stage s
-constexpr uint32_t KV_SC = 2 * kTile + kStages * 4 * kHalf;                   // scalars [stage][64] float4
-constexpr int kMaxUnits = 2048;
-constexpr uint32_t KV_UNITS = KV_SC + kStages * 64 * 16;                      // (tile << 1) | half
+__host__ __device__ constexpr uint32_t kv_q(int s) { return 2 * kTile + s * 2 * kTile; }   // Q tile, stage s
+__host__ __device__ constexpr uint32_t kv_do(int s) { return kv_q(s) + kTile; }            // dO tile, stage s
+constexpr uint32_t KV_SC = 2 * kTile + kStages * 2 * kTile;                   // scalars [stage][128] float4
+constexpr int kMaxUnits = 1024;
+constexpr uint32_t KV_UNITS = KV_SC + kStages * 128 * 16;                     // query tiles of this block
 constexpr uint32_t KV_MISC = KV_UNITS + kMaxUnits * 4;
-// TMEM columns: S^T and dP^T of a 64-query unit, double-buffered; after the
-// softmax has read them, (P^T cs) and dS^T (bf16, two per column) overwrite the
-// first 16 columns of each 32-column half and feed the dV / dK products as the
-// tensor-memory A operand.
-__host__ __device__ constexpr uint32_t tm_st(int b) { return 64u * b; }
-__host__ __device__ constexpr uint32_t tm_dpt(int b) { return 128u + 64u * b; }
-// column of the K = 16 step kk (queries 16 kk .. 16 kk + 15) of a packed operand
-__host__ __device__ constexpr uint32_t tm_ka(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
-constexpr uint32_t TM_DK = 256, TM_DV = 384;
+// TMEM columns: S^T [keys][queries] and dP^T (fp32); once read, (P^T cs) and dS^T (bf16 pairs)
+// overwrite the first 8 of every 16 columns and feed dV / dK as the tensor-memory A operand.
+constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_DV = 256, TM_DK = 384;
 constexpr int kKvThreads = 320;
 
 struct KvMisc {
-  uint64_t kv_full, qd_full[kStages], qd_empty[kStages], s_full[2], p_full[2], done;
+  uint64_t kv_full, qd_full[kStages], qd_empty[kStages], s_full, p_half[2], done;
   uint32_t tmem_base;
   int abort_flag;
 };
-}  // namespace
 
-// One thread's 32 queries of a unit: S^T and dP^T (fp32, TMEM) -> (P^T cs) and dS^T
-// (bf16 pairs) written back over the columns already read, 16 columns at a time.
-// MASK: queries outside [lo, hi) get P = 0.
+// One thread's 32 queries (columns q0 .. q0 + 31 of the unit) for its key row: S^T and dP^T
+// (fp32, TMEM) -> (P^T cs) and dS^T as bf16 pairs in the first 8 of each 16 columns read.
+// MASK: queries outside [lo, hi) (relative to q0) get P = 0.
 template <bool MASK>
 __device__ __forceinline__ void dkdv_softmax_cols(uint32_t tmem, uint32_t st_col, uint32_t dp_col, const float4* sc,
                                                   float sl2, int lo, int hi) {
@@ -371,14 +363,21 @@ __device__ __forceinline__ void dkdv_softmax_cols(uint32_t tmem, uint32_t st_col
       wp[c >> 1] = pack_bf16(pv[0], pv[1]);
       wd[c >> 1] = pack_bf16(dv[0], dv[1]);
     }
-    tc::tmem_st8(tmem + st_col + c0 / 2, wp);
-    tc::tmem_st8(tmem + dp_col + c0 / 2, wd);
+    tc::tmem_st8(tmem + st_col + c0, wp);
+    tc::tmem_st8(tmem + dp_col + c0, wd);
   }
 }
+}  // namespace
 
+// One CTA per (head, key block b): K_b and V_b stay in shared memory; the query tiles that
+// selected b (ascending, from the selection inverse) stream through a 2-stage ring with
+// their per-row scalars.  Per tile: S^T = K Q^T and dP^T = V dO^T (N = 128) into TMEM; the
+// softmax warps turn them into (P^T cs) and dS^T in two passes of 64 queries; after each
+// pass dV += (P^T cs) dO and dK += dS^T Q over those 64 queries run on the tensor cores
+// while the other pass is computed.
 __global__ void __launch_bounds__(kKvThreads, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                   const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmdOh,
+                   const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                    const __grid_constant__ CUtensorMap tmSc, const __grid_constant__ CUtensorMap tmdK,
                    const __grid_constant__ CUtensorMap tmdV, BwdArgs a, Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -393,20 +392,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
     return;
   }
-  // units: each query tile that selected this block, ascending, as 64-query halves;
-  // only the last tile of the sequence can lack its second half
   int n_u = 0;
   if (g.k > 0) {
     const int* of = a.offs + (size_t)bh * (g.n_t + 1);
     const int* list = a.tiles + (size_t)bh * g.n_t * g.k;
-    const int e0 = of[b], cnt = min(of[b + 1] - e0, kMaxUnits / 2);
-    for (int i = threadIdx.x; i < cnt; i += kKvThreads) {
-      const int t = list[e0 + i];
-      units[2 * i] = t << 1;
-      units[2 * i + 1] = (t << 1) | 1;
-    }
-    n_u = 2 * cnt;
-    if (cnt > 0 && list[e0 + cnt - 1] * kT + 64 >= g.N) n_u -= 1;
+    const int e0 = of[b];
+    n_u = min(of[b + 1] - e0, kMaxUnits);
+    for (int i = threadIdx.x; i < n_u; i += kKvThreads) units[i] = list[e0 + i];
   }
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->kv_full, 1);
@@ -414,10 +406,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       tc::mbar_init(&ms->qd_full[s], 1);
       tc::mbar_init(&ms->qd_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&ms->s_full[s], 1);
-      tc::mbar_init(&ms->p_full[s], kSoftmaxThreads);
-    }
+    tc::mbar_init(&ms->s_full, 1);
+    tc::mbar_init(&ms->p_half[0], kSoftmaxThreads);
+    tc::mbar_init(&ms->p_half[1], kSoftmaxThreads);
     tc::mbar_init(&ms->done, 1);
     ms->abort_flag = 0;
     tc::fence_barrier_init();
@@ -443,13 +434,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       for (int u = 0; u < n_u; ++u) {
         const int s = u % kStages;
         if (u >= kStages && !wait_or_abort(&ms->qd_empty[s], ((u / kStages) - 1) & 1, ms, err, 1u)) break;
-        const int row0 = (units[u] >> 1) * kT + (units[u] & 1) * 64;
-        tc::mbar_arrive_expect_tx(&ms->qd_full[s], 4 * kHalf + 64 * 16);
-        tc::tma_load_3d(smem + kv_q(s), &tmQh, &ms->qd_full[s], 0, row0, bh);
-        tc::tma_load_3d(smem + kv_q(s) + kHalf, &tmQh, &ms->qd_full[s], 64, row0, bh);
-        tc::tma_load_3d(smem + kv_do(s), &tmdOh, &ms->qd_full[s], 0, row0, bh);
-        tc::tma_load_3d(smem + kv_do(s) + kHalf, &tmdOh, &ms->qd_full[s], 64, row0, bh);
-        tc::tma_load_3d(smem + KV_SC + s * 64 * 16, &tmSc, &ms->qd_full[s], 0, row0, bh);
+        const int row0 = units[u] * kT;
+        tc::mbar_arrive_expect_tx(&ms->qd_full[s], 2 * kTile + 128 * 16);
+        tc::tma_load_3d(smem + kv_q(s), &tmQ, &ms->qd_full[s], 0, row0, bh);
+        tc::tma_load_3d(smem + kv_q(s) + kSlab, &tmQ, &ms->qd_full[s], 64, row0, bh);
+        tc::tma_load_3d(smem + kv_do(s), &tmdO, &ms->qd_full[s], 0, row0, bh);
+        tc::tma_load_3d(smem + kv_do(s) + kSlab, &tmdO, &ms->qd_full[s], 64, row0, bh);
+        tc::tma_load_3d(smem + KV_SC + s * 128 * 16, &tmSc, &ms->qd_full[s], 0, row0, bh);
         issued = u + 1;
       }
       tc::mbar_wait(&ms->kv_full, 0);
@@ -459,97 +450,95 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t idS = tc::idesc_bf16(128, 64, false, false);     // K (keys x d) x Q (queries x d)
+      const uint32_t idS = tc::idesc_bf16(128, 128, false, false);    // K (keys x d) x Q (queries x d)
       const uint32_t idG = tc::idesc_bf16(128, kD, false, true);      // P^T / dS^T (TMEM) x (dO / Q, MN-major)
       const uint32_t sb = smem_u32(smem);
       bool ok = wait_or_abort(&ms->kv_full, 0, ms, err, 2u);
-      int g_issued = 0;
-      // dV += (P^T cs) dO and dK += dS^T Q for unit uu; both A operands in TMEM.
-      // The next S^T into the same columns is issued after these, and tcgen05
-      // MMAs of one thread run in issue order, so the reuse needs no wait.
-      auto issue_grads = [&](int uu) -> bool {
-        const int s = uu % kStages, bb = uu & 1;
-        if (!wait_or_abort(&ms->p_full[bb], (uu >> 1) & 1, ms, err, 4u)) return false;
-        tc::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc::mma_bf16_ts(tmem + TM_DV, tmem + tm_st(bb) + tm_ka(kk),
-                          tc::sw128_desc(sb + kv_do(s) + kk * 2048, kHalf, 1024), idG, (uu > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc::mma_bf16_ts(tmem + TM_DK, tmem + tm_dpt(bb) + tm_ka(kk),
-                          tc::sw128_desc(sb + kv_q(s) + kk * 2048, kHalf, 1024), idG, (uu > 0 || kk > 0) ? 1u : 0u);
-        tc::mma_commit(&ms->qd_empty[s]);
-        g_issued = uu + 1;
-        return true;
-      };
       for (int u = 0; ok && u < n_u; ++u) {
-        const int s = u % kStages, b2 = u & 1;
+        const int s = u % kStages;
         if (!wait_or_abort(&ms->qd_full[s], (u / kStages) & 1, ms, err, 8u)) break;
         tc::tc_fence_after();
+        // S^T and dP^T overwrite the columns that held the previous unit's P^T / dS^T:
+        // the products that read those were issued earlier and tcgen05 MMAs run in order
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t ka = (kk >> 2) * kSlab + (kk & 3) * 32;
-          const uint32_t kq = (kk >> 2) * kHalf + (kk & 3) * 32;
-          tc::mma_bf16(tmem + tm_st(b2), tc::sw128_desc(sb + KV_K + ka, 16, 1024),
-                       tc::sw128_desc(sb + kv_q(s) + kq, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+          tc::mma_bf16(tmem + TM_ST, tc::sw128_desc(sb + KV_K + off, 16, 1024),
+                       tc::sw128_desc(sb + kv_q(s) + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t ka = (kk >> 2) * kSlab + (kk & 3) * 32;
-          const uint32_t kq = (kk >> 2) * kHalf + (kk & 3) * 32;
-          tc::mma_bf16(tmem + tm_dpt(b2), tc::sw128_desc(sb + KV_V + ka, 16, 1024),
-                       tc::sw128_desc(sb + kv_do(s) + kq, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+          tc::mma_bf16(tmem + TM_DPT, tc::sw128_desc(sb + KV_V + off, 16, 1024),
+                       tc::sw128_desc(sb + kv_do(s) + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
-        tc::mma_commit(&ms->s_full[b2]);
-        if (u >= 1 && !issue_grads(u - 1)) break;
+        tc::mma_commit(&ms->s_full);
+        // gradient products over each pass of 64 queries as soon as it is written
+        for (int h = 0; ok && h < 2; ++h) {
+          ok = wait_or_abort(&ms->p_half[h], u & 1, ms, err, 4u);
+          if (!ok) break;
+          tc::tc_fence_after();
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kk = 4 * h + k4;               // queries 16 kk .. 16 kk + 15
+            tc::mma_bf16_ts(tmem + TM_DV, tmem + TM_ST + 16 * kk, tc::sw128_desc(sb + kv_do(s) + kk * 2048, kSlab, 1024),
+                            idG, (u > 0 || kk > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kk = 4 * h + k4;
+            tc::mma_bf16_ts(tmem + TM_DK, tmem + TM_DPT + 16 * kk, tc::sw128_desc(sb + kv_q(s) + kk * 2048, kSlab, 1024),
+                            idG, (u > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        if (ok) tc::mma_commit(&ms->qd_empty[s]);
       }
-      if (n_u > 0 && g_issued == n_u - 1) issue_grads(n_u - 1);
       tc::mma_commit(&ms->done);
       tc::mbar_wait(&ms->done, 0);
     }
   } else {
-    // ---------------- softmax: one key row, 32 of the unit's 64 queries per thread ----------------
+    // ---------------- softmax: one key row; two passes of 32 queries per thread ----------------
     const int q4 = warp & 3;
-    const int hq = (warp - 2) >> 2;
+    const int grp = (warp - 2) >> 2;                // queries 32 grp + 64 pass .. + 31
     const int row = 32 * q4 + lane;                 // key row within the block
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
     const bool key_ok = b * kT + row < g.N;
     const float sl2 = g.scale * kLog2e;
     bool alive = true;
     for (int u = 0; u < n_u && alive; ++u) {
-      const int s = u % kStages, b2 = u & 1;
-      const int t = units[u] >> 1, h = units[u] & 1;
-      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full[b2], (u >> 1) & 1, ms, err, 32u));
+      const int s = u % kStages;
+      const int t = units[u];
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full, u & 1, ms, err, 32u));
       if (!alive) break;
       tc::tc_fence_after();
-      const float4* sc = reinterpret_cast<const float4*>(smem + KV_SC + s * 64 * 16) + 32 * hq;
-      const int q0 = 64 * h + 32 * hq;              // first query (within tile t) of this thread
-      const int qvalid = g.N - t * kT - q0;         // queries of this thread inside the sequence
       const bool diag = g.causal && t == b;
-      const bool masked = !key_ok || qvalid < 32 || (diag && row > q0);
-      // valid queries of this thread: c in [lo, hi) (causal diagonal, sequence end, key row)
-      const int lo = diag ? row - q0 : 0;
-      const int hi = key_ok ? qvalid : 0;
-      // masking is needed only on the causal diagonal, at the end of the sequence and
-      // for padding keys: a warp-uniform branch keeps it out of the common path
-      if (__any_sync(0xffffffffu, masked))
-        dkdv_softmax_cols<true>(tmem, lane_base + tm_st(b2) + 32 * hq, lane_base + tm_dpt(b2) + 32 * hq, sc, sl2, lo, hi);
-      else
-        dkdv_softmax_cols<false>(tmem, lane_base + tm_st(b2) + 32 * hq, lane_base + tm_dpt(b2) + 32 * hq, sc, sl2, lo,
-                                 hi);
-      tc::tmem_wait_st();
-      tc::tc_fence_before();
-      tc::mbar_arrive(&ms->p_full[b2]);
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        const int q0 = 64 * pass + 32 * grp;        // first query (within tile t) of this thread
+        const int qvalid = g.N - t * kT - q0;       // queries of this thread inside the sequence
+        const bool masked = !key_ok || qvalid < 32 || (diag && row > q0);
+        const int lo = diag ? row - q0 : 0;
+        const int hi = key_ok ? qvalid : 0;
+        const float4* sc = reinterpret_cast<const float4*>(smem + KV_SC + s * 128 * 16) + q0;
+        // masking only on the causal diagonal, at the end of the sequence and for padding keys
+        if (__any_sync(0xffffffffu, masked))
+          dkdv_softmax_cols<true>(tmem, lane_base + TM_ST + q0, lane_base + TM_DPT + q0, sc, sl2, lo, hi);
+        else
+          dkdv_softmax_cols<false>(tmem, lane_base + TM_ST + q0, lane_base + TM_DPT + q0, sc, sl2, lo, hi);
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&ms->p_half[pass]);
+      }
     }
     // ---------------- epilogue: dK = scale dK_sparse + dK_lowrank, dV likewise; TMA stores ----------------
+    const int hq = grp;
     bool have = false;
     if (alive && n_u > 0) {
       alive = __all_sync(0xffffffffu, wait_or_abort(&ms->done, 0, ms, err, 512u));
       have = alive;
       if (have) tc::tc_fence_after();
     }
-    // every product has completed: stage dK in the stage-0 Q/dO buffers and dV in stage 1
+    // every product has completed: stage dK in the stage-0 Q buffer and dV in the stage-0 dO buffer
 #pragma unroll 1
     for (int which = 0; which < 2; ++which) {
       float o[64];
@@ -575,7 +564,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           o[4 * c] += x.x; o[4 * c + 1] += x.y; o[4 * c + 2] += x.z; o[4 * c + 3] += x.w;
         }
       }
-      unsigned char* orow = smem + kv_q(which) + hq * kSlab + row * 128;
+      unsigned char* orow = smem + (which == 0 ? kv_q(0) : kv_do(0)) + hq * kSlab + row * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch)
         *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) =
@@ -587,8 +576,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
       tma_store_3d(&tmdK, smem + kv_q(0), 0, b * kT, bh);
       tma_store_3d(&tmdK, smem + kv_q(0) + kSlab, 64, b * kT, bh);
-      tma_store_3d(&tmdV, smem + kv_q(1), 0, b * kT, bh);
-      tma_store_3d(&tmdV, smem + kv_q(1) + kSlab, 64, b * kT, bh);
+      tma_store_3d(&tmdV, smem + kv_do(0), 0, b * kT, bh);
+      tma_store_3d(&tmdV, smem + kv_do(0) + kSlab, 64, b * kT, bh);
       tma_store_wait();
     }
   }
@@ -644,13 +633,13 @@ cudaError_t launch_dq_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStr
   return cudaGetLastError();
 }
 
-// Per-row scalars (log2 d_s, cs, Delta, 0) as float32 [BH][N][4]; boxes of 4 x 64 x 1.
+// Per-row scalars (log2 d_s, cs, Delta, 0) as float32 [BH][N][4]; boxes of 4 x 128 x 1.
 static bool map_scalars(CUtensorMap* m, const void* base, int N, int BH) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {4, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {16, (cuuint64_t)N * 16};
-  cuuint32_t box[3] = {4, 64, 1};
+  cuuint32_t box[3] = {4, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
@@ -658,10 +647,10 @@ static bool map_scalars(CUtensorMap* m, const void* base, int N, int BH) {
 }
 
 cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
-  if (!bwd_tc_supported(g) || !a.rs.packed || 2 * g.n_t > kMaxUnits) return cudaErrorInvalidValue;
+  if (!bwd_tc_supported(g) || !a.rs.packed || g.n_t > kMaxUnits) return cudaErrorInvalidValue;
   CUtensorMap mk, mv, mq, mdo, msc, mdk, mdv;
   if (!tc::map_rows_bf16(&mk, a.K, g.N, g.BH, kT) || !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kT) ||
-      !tc::map_rows_bf16(&mq, a.Q, g.N, g.BH, 64) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, 64) ||
+      !tc::map_rows_bf16(&mq, a.Q, g.N, g.BH, kT) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, kT) ||
       !map_scalars(&msc, a.rs.packed, g.N, g.BH) || !tc::map_rows_bf16(&mdk, a.dK, g.N, g.BH, kT) ||
       !tc::map_rows_bf16(&mdv, a.dV, g.N, g.BH, kT))
     return cudaErrorInvalidValue;
