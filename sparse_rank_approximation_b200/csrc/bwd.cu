@@ -60,6 +60,28 @@ __global__ void __launch_bounds__(256) row_scalars_kernel(BwdArgs a, Geom g) {
     A += __shfl_xor_sync(0xffffffffu, A, o);
     Bv += __shfl_xor_sync(0xffffffffu, Bv, o);
   }
+  // cl = g_lr / d_lr, broadcast from the row's first lane: the rows cl dO (bf16) feed the
+  // RACE suffix statistics
+  if (a.dOcl) {
+    double cl_row = 0.0;
+    if (sub == 0 && row < g.N) {
+      const double logd0 = a.logd[i], dl0 = a.dlr[i];
+      const double lam0 = a.lam ? a.lam[i] : g.lam;
+      const double c0 = lam0 * dl0 + (double)g.eps;
+      const double D0 = exp(logd0) + c0;
+      const double gl0 = a.glr ? (double)a.glr[i] : (D0 > 0.0 ? c0 / D0 : 1.0);
+      cl_row = dl0 > 0.0 ? gl0 / dl0 : 0.0;
+    }
+    const float clf = __shfl_sync(0xffffffffu, (float)cl_row, (threadIdx.x & 31) - sub);
+    if (row < g.N) {
+      uint4 w;
+      w.x = pack_bf16(clf * dO[0], clf * dO[1]);
+      w.y = pack_bf16(clf * dO[2], clf * dO[3]);
+      w.z = pack_bf16(clf * dO[4], clf * dO[5]);
+      w.w = pack_bf16(clf * dO[6], clf * dO[7]);
+      *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dOcl) + i * g.d + sub * 8) = w;
+    }
+  }
   if (sub != 0 || row >= g.N) return;
   const double logd = a.logd[i], dl = a.dlr[i];
   const double lam = a.lam ? a.lam[i] : g.lam;

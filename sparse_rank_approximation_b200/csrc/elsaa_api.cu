@@ -148,6 +148,7 @@ struct FwdWs {
   uint32_t* flag;
   double *qbar, *kbar;
   float* scores;
+  void* wsplit;
 };
 
 FwdWs carve_fwd_ws(void* base, const Geom& g, size_t* bytes) {
@@ -157,6 +158,7 @@ FwdWs carve_fwd_ws(void* base, const Geom& g, size_t* bytes) {
   w.qbar = c.take<double>((size_t)g.BH * g.n_t * g.d);
   w.kbar = c.take<double>((size_t)g.BH * g.n_t * g.d);
   w.scores = c.take<float>((size_t)g.BH * g.n_t * g.n_t);
+  w.wsplit = c.take<char>((size_t)2 * ((g.L * kHashBits + 15) & ~15) * g.d * 2);
   *bytes = align_up(c.off);
   return w;
 }
@@ -167,6 +169,7 @@ struct BwdWs {
   float *RA, *RB;
   int *offs, *tiles, *order;
   float *dQacc, *dKacc, *dVacc;
+  void* dOcl;
 };
 
 BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
@@ -189,6 +192,7 @@ BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
   w.dQacc = c.take<float>(acc);
   w.dKacc = c.take<float>(acc);
   w.dVacc = c.take<float>(acc);
+  w.dOcl = c.take<char>(bf16 && g.r > 0 ? rows * g.d * 2 : 0);
   *bytes = align_up(c.off);
   return w;
 }
@@ -354,7 +358,7 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
 
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st_), "flag reset"));
   ELSAA_TRY(cuda_status(launch_select(Q, K, bf16, w.qbar, w.kbar, w.scores, s.idx, g, st_), "selection"));
-  ELSAA_TRY(cuda_status(launch_race_features(Q, K, W, bf16, s.phiQ, s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, st_),
+  ELSAA_TRY(cuda_status(launch_race_features(Q, K, W, w.wsplit, bf16, s.phiQ, s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, st_),
                         "race features"));
   ELSAA_TRY(cuda_status(launch_race_state_fwd(s.phiK, V, bf16, s.Ast, s.Bst, g, st_), "race summaries"));
   FwdArgs a{Q, K, V, s.idx, s.phiQ, s.phiK, s.Ast, s.Bst, lam, gs, glr, O, s.Os, s.logd, s.dlr, s.m, s.Olr};
@@ -409,6 +413,7 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   a.Ast = s.Ast; a.Bst = s.Bst; a.RA = w.RA; a.RB = w.RB;
   a.offs = w.offs; a.tiles = w.tiles; a.kv_order = g.k > 0 ? w.order : nullptr; a.rs = w.rs;
   a.dQacc = w.dQacc; a.dKacc = w.dKacc; a.dVacc = w.dVacc;
+  a.dOcl = bf16 && g.r > 0 ? w.dOcl : nullptr;
   a.dQ = dQ; a.dK = dK; a.dV = dV;
 
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st_), "flag reset"));

@@ -50,6 +50,7 @@ struct BwdArgs {
   const int* kv_order;           // per head, key blocks by descending tile count (ties: lower block first)
   RowScalars rs;
   float *dQacc, *dKacc, *dVacc;  // fp32 low-rank gradient parts (bf16 path)
+  void* dOcl;                    // cl dO rows (bf16 path), written by the row scalars
   void *dQ, *dK, *dV;
 };
 
@@ -60,8 +61,10 @@ cudaError_t launch_select(const void* Q, const void* K, bool bf16, double* qbar,
                           int* idx, const Geom& g, cudaStream_t st);
 cudaError_t launch_invert_selection(const int* idx, int* offs, int* tiles, int* order, const Geom& g,
                                     cudaStream_t st);
-cudaError_t launch_race_features(const void* Q, const void* K, const float* W, bool bf16, void* phiQ, void* phiK,
-                                 float* hQ, float* hK, float* nQ, float* nK, const Geom& g, cudaStream_t st);
+// wsplit: scratch bf16 [2][NW][d] (NW = 4L rounded up to 16) that receives W split into hi and lo halves.
+cudaError_t launch_race_features(const void* Q, const void* K, const float* W, void* wsplit, bool bf16, void* phiQ,
+                                 void* phiK, float* hQ, float* hK, float* nQ, float* nK, const Geom& g,
+                                 cudaStream_t st);
 // Forward prefix statistics (Ast: per-segment exclusive prefix, Bst: in-segment prefix).
 cudaError_t launch_race_state_fwd(const void* phiK, const void* V, bool bf16, float* Ast, float* Bst,
                                   const Geom& g, cudaStream_t st);

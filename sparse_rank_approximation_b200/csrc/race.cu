@@ -25,9 +25,22 @@ namespace elsaa {
 // Writes Phi (bf16 [BH,N,r]), the normalised projections h (fp32 [BH,N,4L]) and
 // the row norms n (fp32 [BH,N]).
 // ---------------------------------------------------------------------------
+// W[l][k][b] (fp32) -> rows n = 4 l + b of bf16 hi and lo [NW][D] (zero rows beyond 4 L).
+__global__ void race_w_split_kernel(const float* __restrict__ W, __nv_bfloat16* __restrict__ out, int D, int NH,
+                                    int NW) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < NW * D; i += gridDim.x * blockDim.x) {
+    const int n = i / D, k = i % D;
+    const float w = n < NH ? W[((size_t)(n >> 2) * D + k) * kHashBits + (n & 3)] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    out[i] = hi;
+    out[(size_t)NW * D + i] = __float2bfloat16_rn(w - __bfloat162float(hi));
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(128) race_features_bf16_kernel(
-    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K, const float* __restrict__ W,
+    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
+    const __nv_bfloat16* __restrict__ Wsplit,
     __nv_bfloat16* __restrict__ phiQ, __nv_bfloat16* __restrict__ phiK, float* __restrict__ hQ,
     float* __restrict__ hK, float* __restrict__ nQ, float* __restrict__ nK, Geom g) {
   constexpr int LDX = D + 8;
@@ -56,16 +69,12 @@ __global__ void __launch_bounds__(128) race_features_bf16_kernel(
     const int row = row_base + r;
     cp_async16(sX + r * LDX + c, X + (size_t)min(row, g.N - 1) * D + c, row < g.N);
   }
-  cp_async_commit();
-  // W[l][k][b] -> column n = l*4 + b, stored [n][k] as hi + lo bf16 halves
-  for (int i = tid; i < NW * D; i += 128) {
-    const int n = i / D, kk = i % D;
-    float w = 0.f;
-    if (n < NH) w = W[((size_t)(n >> 2) * D + kk) * kHashBits + (n & 3)];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-    sWh[n * LDX + kk] = hi;
-    sWl[n * LDX + kk] = __float2bfloat16_rn(w - __bfloat162float(hi));
+  // W already split into bf16 hi + lo rows n = 4 l + b (race_w_split_kernel), [NW][D] each
+  for (int i = tid; i < 2 * NW * (D / 8); i += 128) {
+    const int half = i / (NW * (D / 8)), r = (i / (D / 8)) % NW, c = (i % (D / 8)) * 8;
+    cp_async16((half ? sWl : sWh) + r * LDX + c, Wsplit + ((size_t)half * NW + r) * D + c, true);
   }
+  cp_async_commit();
   cp_async_wait<0>();
   __syncthreads();
 
@@ -167,7 +176,7 @@ __global__ void __launch_bounds__(512) race_state_bf16_kernel(const __nv_bfloat1
   const int nthr = blockDim.x;
   const __nv_bfloat16* pk = phi + (size_t)bh * g.N * g.r;
   const __nv_bfloat16* vv = Y + (size_t)bh * g.N * D;
-  const float* rsc = BWD ? rscale + (size_t)bh * g.N : nullptr;
+  const float* rsc = BWD && rscale ? rscale + (size_t)bh * g.N : nullptr;
   const float* rex = BWD ? rextra + (size_t)bh * g.N : nullptr;
 
   auto load = [&](int buf, int c) {
@@ -179,7 +188,8 @@ __global__ void __launch_bounds__(512) race_state_bf16_kernel(const __nv_bfloat1
       const int row = c * C + r;
       cp_async16(dP + r * LDP + cc, pk + (size_t)min(row, g.N - 1) * g.r + cc, row < g.N);
     }
-    if (!BWD) {
+    if (!BWD || !rsc) {
+      // forward rows, or backward rows already scaled by cl
       for (int i = tid; i < C * (D / 8); i += nthr) {
         const int r = i / (D / 8), cc = (i % (D / 8)) * 8;
         const int row = c * C + r;
@@ -273,18 +283,32 @@ __global__ void race_scan_kernel(float* __restrict__ A, Geom g, int reverse) {
   const int n = g.r * g.dp;
   if (e >= n) return;
   float* a = A + (size_t)blockIdx.y * (g.n_seg + 1) * n + e;
+  constexpr int kB = 8;          // loads in flight per thread
   float acc = 0.f;
   if (!reverse) {
     a[0] = 0.f;
-    for (int s = 1; s <= g.n_seg; ++s) {
-      acc += a[(size_t)s * n];
-      a[(size_t)s * n] = acc;
+    for (int s0 = 1; s0 <= g.n_seg; s0 += kB) {
+      float v[kB];
+#pragma unroll
+      for (int q = 0; q < kB; ++q) v[q] = s0 + q <= g.n_seg ? a[(size_t)(s0 + q) * n] : 0.f;
+#pragma unroll
+      for (int q = 0; q < kB; ++q)
+        if (s0 + q <= g.n_seg) {
+          acc += v[q];
+          a[(size_t)(s0 + q) * n] = acc;
+        }
     }
   } else {
-    for (int s = g.n_seg - 1; s >= 0; --s) {
-      const float tot = a[(size_t)(s + 1) * n];
-      a[(size_t)(s + 1) * n] = acc;
-      acc += tot;
+    for (int s0 = g.n_seg - 1; s0 >= 0; s0 -= kB) {
+      float v[kB];
+#pragma unroll
+      for (int q = 0; q < kB; ++q) v[q] = s0 - q >= 0 ? a[(size_t)(s0 - q + 1) * n] : 0.f;
+#pragma unroll
+      for (int q = 0; q < kB; ++q)
+        if (s0 - q >= 0) {
+          a[(size_t)(s0 - q + 1) * n] = acc;
+          acc += v[q];
+        }
     }
     a[0] = acc;
   }
@@ -380,8 +404,9 @@ static size_t features_smem(const Geom& g) {
   return (size_t)(64 + 2 * NW) * (g.d + 8) * 2 + (size_t)64 * (NW + 1) * 4 + 64 * 4;
 }
 
-cudaError_t launch_race_features(const void* Q, const void* K, const float* W, bool bf16, void* phiQ, void* phiK,
-                                 float* hQ, float* hK, float* nQ, float* nK, const Geom& g, cudaStream_t st) {
+cudaError_t launch_race_features(const void* Q, const void* K, const float* W, void* wsplit, bool bf16, void* phiQ,
+                                 void* phiK, float* hQ, float* hK, float* nQ, float* nK, const Geom& g,
+                                 cudaStream_t st) {
   if (g.r == 0) return cudaSuccess;
   if (!bf16) {
     ProfScope ps("race_features_f32", st);
@@ -390,13 +415,15 @@ cudaError_t launch_race_features(const void* Q, const void* K, const float* W, b
     return cudaGetLastError();
   }
   const size_t smem = features_smem(g);
+  const int NW = (g.L * kHashBits + 15) & ~15;
+  race_w_split_kernel<<<(NW * g.d + 255) / 256, 256, 0, st>>>(W, (__nv_bfloat16*)wsplit, g.d, g.L * kHashBits, NW);
   auto run = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     ProfScope ps("race_features", st);
     kern<<<dim3((g.N + 63) / 64, g.BH, 2), 128, smem, st>>>(
-        (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, W, (__nv_bfloat16*)phiQ, (__nv_bfloat16*)phiK, hQ, hK,
-        nQ, nK, g);
+        (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)wsplit, (__nv_bfloat16*)phiQ,
+        (__nv_bfloat16*)phiK, hQ, hK, nQ, nK, g);
     return cudaGetLastError();
   };
   if (g.d == 64) return run(race_features_bf16_kernel<64>);
@@ -443,6 +470,8 @@ cudaError_t launch_race_state_fwd(const void* phiK, const void* V, bool bf16, fl
 
 cudaError_t launch_race_state_bwd(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st) {
   if (g.r == 0) return cudaSuccess;
+  // bf16: the row scalars already wrote cl dO, so the rows stream in with cp.async
+  if (bf16 && a.dOcl) return run_state<true>(a.phiQ, a.dOcl, nullptr, a.rs.delta, bf16, a.RA, a.RB, g, st);
   return run_state<true>(a.phiQ, a.dO, a.rs.cl, a.rs.delta, bf16, a.RA, a.RB, g, st);
 }
 
