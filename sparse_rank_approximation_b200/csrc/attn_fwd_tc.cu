@@ -58,6 +58,7 @@ struct Misc {
   float red[2][256];      // partial row maxima / sums exchanged by the two halves of a row
 };
 constexpr size_t kSmemBytes = OFF_MISC + sizeof(Misc);
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -626,6 +626,7 @@ cudaError_t launch_dq_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStr
       !tc::map_rows_bf16(&mdq, a.dQ, g.N, g.BH, kT))
     return cudaErrorInvalidValue;
   const size_t smem = DQ_MISC + sizeof(DqMisc);
+  static_assert(DQ_MISC + sizeof(DqMisc) <= 232448, "shared memory per CTA");
   cudaError_t e = cudaFuncSetAttribute(dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("dq_tc", st);
@@ -655,6 +656,7 @@ cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaS
       !tc::map_rows_bf16(&mdv, a.dV, g.N, g.BH, kT))
     return cudaErrorInvalidValue;
   const size_t smem = KV_MISC + sizeof(KvMisc);
+  static_assert(KV_MISC + sizeof(KvMisc) <= 232448, "shared memory per CTA");
   cudaError_t e = cudaFuncSetAttribute(dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("dkdv_tc", st);

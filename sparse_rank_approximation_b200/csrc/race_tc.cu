@@ -849,6 +849,7 @@ cudaError_t launch_race_readout_tc(const FwdArgs& a, const Geom& g, uint32_t* er
       !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kC) || !tc::map_rows_bf16(&mo, a.Olr, g.N, g.BH, kC))
     return cudaErrorInvalidValue;
   const size_t smem = R_BARS + sizeof(Bars);
+  static_assert(R_BARS + sizeof(Bars) <= 232448, "shared memory per CTA");
   cudaError_t e = cudaFuncSetAttribute(race_readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("race_readout_tc", st);
@@ -868,6 +869,7 @@ cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, c
     return cudaErrorInvalidValue;
   {
     const size_t smem = Q_BARS + sizeof(Bars);
+  static_assert(Q_BARS + sizeof(Bars) <= 232448, "shared memory per CTA");
     cudaError_t e = cudaFuncSetAttribute(race_q_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     ProfScope ps("race_q_bwd_tc", st);
@@ -876,6 +878,7 @@ cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, c
     if (e != cudaSuccess) return e;
   }
   const size_t smem = K_BARS + sizeof(Bars);
+  static_assert(K_BARS + sizeof(Bars) <= 232448, "shared memory per CTA");
   cudaError_t e = cudaFuncSetAttribute(race_k_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("race_k_bwd_tc", st);
