@@ -87,7 +87,10 @@ def work_model(w):
     # key side  Phi_K Phi_Q^T, V dO^T, Phi_K R, V R^T, kappa^T dO, dkappa^T Phi_Q, dh W^T.
     NH = 4 * L
     cz = 1 if w.causal else 0
-    state_b = r * (d + 8) * 4 * (2 if w.causal else 1)          # prefix/suffix statistics read per chunk
+    state_b = r * d * 2 * 2 + r * 4                            # per-chunk statistics (bf16 hi + lo, key mass)
+    split_b = r * (d + 8) * 4 * (2 if w.causal else 1) + state_b   # split kernel: fp32 parts in, bf16 out
+    m["race_split_fwd"] = dict(flops=0, bytes=tiles * split_b)
+    m["race_split_bwd"] = dict(flops=0, bytes=tiles * split_b)
     m["race_readout_tc"] = dict(flops=tiles * 2 * T * (cz * T * r + cz * T * d + r * d),
                                 bytes=tiles * (T * r * 2 * (1 + cz) + cz * T * d * 2 + state_b + T * d * 2 + T * 4))
     m["race_q_bwd_tc"] = dict(flops=tiles * 2 * T * (cz * T * d + d * r + cz * T * r + NH * d),

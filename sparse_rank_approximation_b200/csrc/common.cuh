@@ -72,6 +72,30 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// sigma(y) and sigma(-y) = 1 - sigma(y) without cancellation: with e = exp(-|y|),
+// 1 / (1 + e) is the larger and e / (1 + e) the smaller of the two.
+__device__ __forceinline__ void sigmoid_pair(float y, float& sp, float& sm) {
+  const float e = __expf(-fabsf(y));
+  const float r = __fdividef(1.f, 1.f + e);
+  const float t = e * r;
+  sp = y >= 0.f ? r : t;
+  sm = y >= 0.f ? t : r;
+}
+
+// The 16 corner probabilities of one table, p_c = prod_b (bit b of c ? sp_b : sm_b) * scale,
+// as a two-level product (pairs of bits, then the cross product).
+__device__ __forceinline__ void corner_probs(const float (&sp)[4], const float (&sm)[4], float scale,
+                                             float (&p)[16]) {
+  float lo[4], hi[4];
+#pragma unroll
+  for (int c2 = 0; c2 < 4; ++c2) {
+    lo[c2] = ((c2 & 1) ? sp[0] : sm[0]) * ((c2 & 2) ? sp[1] : sm[1]) * scale;
+    hi[c2] = ((c2 & 1) ? sp[2] : sm[2]) * ((c2 & 2) ? sp[3] : sm[3]);
+  }
+#pragma unroll
+  for (int c = 0; c < 16; ++c) p[c] = lo[c & 3] * hi[c >> 2];
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -119,6 +119,8 @@ struct Saved {
   void *phiQ, *phiK;
   float *hQ, *hK, *nQ, *nK;
   float *Ast, *Bst;
+  void* Psplit;
+  float* Pmass;
 };
 
 Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
@@ -140,6 +142,9 @@ Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
   s.nK = c.take<float>(rows);
   s.Ast = c.take<float>((size_t)g.BH * (g.n_seg + 1) * state);
   s.Bst = c.take<float>(g.causal ? (size_t)g.BH * g.n_c * state : 0);
+  const bool split = esz == 2 && g.r > 0 && race_bwd_tc_supported(g);
+  s.Psplit = split ? c.take<char>((size_t)g.BH * g.n_c * 2 * g.r * g.d * 2) : nullptr;
+  s.Pmass = split ? c.take<float>((size_t)g.BH * g.n_c * g.r) : nullptr;
   *bytes = align_up(c.off);
   return s;
 }
@@ -170,6 +175,8 @@ struct BwdWs {
   int *offs, *tiles, *order;
   float *dQacc, *dKacc, *dVacc;
   void* dOcl;
+  void *Rsplit, *Wsplit;
+  float* Rmass;
 };
 
 BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
@@ -193,6 +200,10 @@ BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
   w.dKacc = c.take<float>(acc);
   w.dVacc = c.take<float>(acc);
   w.dOcl = c.take<char>(bf16 && g.r > 0 ? rows * g.d * 2 : 0);
+  const bool split = bf16 && g.r > 0 && race_bwd_tc_supported(g);
+  w.Rsplit = split ? c.take<char>((size_t)g.BH * g.n_c * 2 * g.r * g.d * 2) : nullptr;
+  w.Rmass = split ? c.take<float>((size_t)g.BH * g.n_c * g.r) : nullptr;
+  w.Wsplit = split ? c.take<char>((size_t)2 * ((g.L * kHashBits + 15) & ~15) * g.d * 2) : nullptr;
   *bytes = align_up(c.off);
   return w;
 }
@@ -361,10 +372,14 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
   ELSAA_TRY(cuda_status(launch_race_features(Q, K, W, w.wsplit, bf16, s.phiQ, s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, st_),
                         "race features"));
   ELSAA_TRY(cuda_status(launch_race_state_fwd(s.phiK, V, bf16, s.Ast, s.Bst, g, st_), "race summaries"));
-  FwdArgs a{Q, K, V, s.idx, s.phiQ, s.phiK, s.Ast, s.Bst, lam, gs, glr, O, s.Os, s.logd, s.dlr, s.m, s.Olr};
+  // per-chunk bf16 hi/lo statistics for the tensor-core read-out and query-side backward
+  if (s.Psplit)
+    ELSAA_TRY(cuda_status(launch_race_state_split(s.Ast, s.Bst, false, s.Psplit, s.Pmass, g, st_),
+                          "race statistics split"));
+  FwdArgs a{Q, K, V, s.idx, s.phiQ, s.phiK, s.Ast, s.Bst, lam, gs, glr, O, s.Os, s.logd, s.dlr, s.m, s.Olr,
+            s.Psplit, s.Pmass};
   if (bf16 && attn_fwd_tc_supported(g) && !tcgen05_disabled()) {
-    if (g.r > 0 && race_bwd_tc_supported(g))
-      ELSAA_TRY(cuda_status(launch_race_readout_tc(a, g, w.flag, st_), "tcgen05 race read-out"));
+    if (s.Psplit) ELSAA_TRY(cuda_status(launch_race_readout_tc(a, g, w.flag, st_), "tcgen05 race read-out"));
     else
       ELSAA_TRY(cuda_status(launch_race_readout_bf16(a, g, st_), "race read-out"));
     ELSAA_TRY(cuda_status(launch_attn_fwd_tc(a, g, w.flag, st_), "tcgen05 forward"));
@@ -414,6 +429,7 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   a.offs = w.offs; a.tiles = w.tiles; a.kv_order = g.k > 0 ? w.order : nullptr; a.rs = w.rs;
   a.dQacc = w.dQacc; a.dKacc = w.dKacc; a.dVacc = w.dVacc;
   a.dOcl = bf16 && g.r > 0 ? w.dOcl : nullptr;
+  a.Psplit = s.Psplit; a.Pmass = s.Pmass; a.Rsplit = w.Rsplit; a.Rmass = w.Rmass; a.Wsplit = w.Wsplit;
   a.dQ = dQ; a.dK = dK; a.dV = dV;
 
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st_), "flag reset"));
@@ -425,7 +441,12 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
     const bool race_tc = tc && g.r > 0 && race_bwd_tc_supported(g);
     BwdArgs at = a;
     if (g.r == 0) at.dQacc = at.dKacc = at.dVacc = nullptr;
-    if (race_tc) ELSAA_TRY(cuda_status(launch_race_bwd_tc(a, g, w.flag, st_), "tcgen05 race backward"));
+    if (race_tc) {
+      ELSAA_TRY(cuda_status(launch_race_state_split(w.RA, w.RB, true, w.Rsplit, w.Rmass, g, st_),
+                            "race statistics split"));
+      ELSAA_TRY(cuda_status(launch_race_w_split(W, w.Wsplit, g, st_), "W split"));
+      ELSAA_TRY(cuda_status(launch_race_bwd_tc(a, g, w.flag, st_), "tcgen05 race backward"));
+    }
     ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, tc ? (race_tc ? 0 : 1) : 7, st_), "backward"));
     if (tc) {
       ELSAA_TRY(cuda_status(launch_dq_tc(at, g, w.flag, st_), "tcgen05 dq"));

@@ -24,6 +24,8 @@ struct FwdArgs {
   void *O, *Os;
   float *logd, *dlr, *m;
   void* Olr;      // O_lr saved for the backward
+  const void* Psplit;  // prefix statistics per chunk as bf16 hi/lo [BH][n_c][2][r][d] (tensor-core RACE path)
+  const float* Pmass;  // their key-mass column [BH][n_c][r]
 };
 
 // Per-row adjoint scalars of the fusion (Eq. 4 / Eq. 5), float32 [BH, N] each.
@@ -51,6 +53,11 @@ struct BwdArgs {
   RowScalars rs;
   float *dQacc, *dKacc, *dVacc;  // fp32 low-rank gradient parts (bf16 path)
   void* dOcl;                    // cl dO rows (bf16 path), written by the row scalars
+  const void* Psplit;            // prefix statistics per chunk, bf16 hi/lo [BH][n_c][2][r][d] (tensor-core RACE)
+  const float* Pmass;            //   key-mass column [BH][n_c][r]
+  const void* Rsplit;            // suffix statistics per chunk, same layout
+  const float* Rmass;
+  const void* Wsplit;            // W as bf16 hi/lo rows n = 4 l + b, [2][NW][d]
   void *dQ, *dK, *dV;
 };
 
@@ -68,6 +75,12 @@ cudaError_t launch_race_features(const void* Q, const void* K, const float* W, v
 // Forward prefix statistics (Ast: per-segment exclusive prefix, Bst: in-segment prefix).
 cudaError_t launch_race_state_fwd(const void* phiK, const void* V, bool bf16, float* Ast, float* Bst,
                                   const Geom& g, cudaStream_t st);
+// Per-chunk statistics A[slot] + B[c] as bf16 hi/lo [BH][n_c][2][r][d] plus the key-mass column
+// [BH][n_c][r] (forward prefix when !bwd, backward suffix when bwd).
+cudaError_t launch_race_state_split(const float* A, const float* B, bool bwd, void* out, float* mass, const Geom& g,
+                                    cudaStream_t st);
+// W[l][d][4] -> bf16 hi/lo rows n = 4 l + b, [2][NW][d] with NW = 4L rounded up to 16.
+cudaError_t launch_race_w_split(const float* W, void* out, const Geom& g, cudaStream_t st);
 // Backward suffix statistics of Phi(q_i) [cl_i dO_i ; delta_i]^T.
 cudaError_t launch_race_state_bwd(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st);
 cudaError_t launch_attn_fwd_bf16(const FwdArgs& a, const Geom& g, cudaStream_t st);

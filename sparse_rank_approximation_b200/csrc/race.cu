@@ -120,23 +120,18 @@ __global__ void __launch_bounds__(128) race_features_bf16_kernel(
     const int row = row_base + r;
     if (row >= g.N) continue;
     const float inv_n = 1.f / sN[r];
-    float sp[kHashBits], sm[kHashBits];
+    float sp[kHashBits], sm[kHashBits], hv[kHashBits];
 #pragma unroll
     for (int b = 0; b < kHashBits; ++b) {
-      const float h = sH[r * (NW + 1) + l * kHashBits + b] * inv_n;
-      if (hout) hout[(size_t)row * NH + l * kHashBits + b] = h;
-      const float y = two_over_tau * h;
-      sp[b] = 1.f / (1.f + expf(-y));   // P(c_b = +1)
-      sm[b] = 1.f / (1.f + expf(y));    // P(c_b = -1)
+      hv[b] = sH[r * (NW + 1) + l * kHashBits + b] * inv_n;
+      sigmoid_pair(two_over_tau * hv[b], sp[b], sm[b]);   // P(c_b = +1), P(c_b = -1)
     }
+    if (hout) *reinterpret_cast<float4*>(hout + (size_t)row * NH + l * kHashBits) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+    float pc[kCorners];
+    corner_probs(sp, sm, inv_sqrt_L, pc);
     __align__(16) __nv_bfloat16 out[kCorners];
 #pragma unroll
-    for (int c = 0; c < kCorners; ++c) {
-      float p = inv_sqrt_L;
-#pragma unroll
-      for (int b = 0; b < kHashBits; ++b) p *= ((c >> b) & 1) ? sp[b] : sm[b];
-      out[c] = __float2bfloat16_rn(p);
-    }
+    for (int c = 0; c < kCorners; ++c) out[c] = __float2bfloat16_rn(pc[c]);
     uint4* dst = reinterpret_cast<uint4*>(phi + (size_t)row * g.r + l * kCorners);
     dst[0] = reinterpret_cast<const uint4*>(out)[0];
     dst[1] = reinterpret_cast<const uint4*>(out)[1];
@@ -397,6 +392,57 @@ __global__ void __launch_bounds__(256) race_state_f32_kernel(const float* __rest
     }
   }
   Atot[((size_t)bh * (g.n_seg + 1) + seg + 1) * n + e] = acc;
+}
+
+// Statistics of chunk c for the tensor-core RACE kernels: S = A[slot] + B[c] (fp32 [r][dp])
+// as bf16 hi and lo halves, row-major [r][d] each, stored [BH][n_c][2][r][d], and the
+// key-mass column [BH][n_c][r] in fp32.  Forward: slot = the segment's exclusive prefix;
+// backward: the exclusive suffix of the later segments.  grid (n_c, BH), block 256.
+__global__ void __launch_bounds__(256) race_state_split_kernel(const float* __restrict__ A,
+                                                               const float* __restrict__ B, int bwd,
+                                                               __nv_bfloat16* __restrict__ out,
+                                                               float* __restrict__ mass, Geom g) {
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const size_t state = (size_t)g.r * g.dp;
+  const int slot = bwd ? (g.causal ? c / g.seg + 1 : 0) : (g.causal ? c / g.seg : g.n_seg);
+  const float* a = A + ((size_t)bh * (g.n_seg + 1) + slot) * state;
+  const float* b = g.causal ? B + ((size_t)bh * g.n_c + c) * state : nullptr;
+  __nv_bfloat16* hi = out + ((size_t)bh * g.n_c + c) * 2 * g.r * g.d;
+  __nv_bfloat16* lo = hi + (size_t)g.r * g.d;
+  const int q4 = g.d / 4;
+#pragma unroll 4
+  for (int i = threadIdx.x; i < g.r * q4; i += blockDim.x) {
+    const int f = i / q4, e = (i % q4) * 4;
+    float4 v = *reinterpret_cast<const float4*>(a + (size_t)f * g.dp + e);
+    if (b) {
+      const float4 w = *reinterpret_cast<const float4*>(b + (size_t)f * g.dp + e);
+      v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+    }
+    __nv_bfloat16 h[4], l[4];
+    const float x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      h[k] = __float2bfloat16_rn(x[k]);
+      l[k] = __float2bfloat16_rn(x[k] - __bfloat162float(h[k]));
+    }
+    *reinterpret_cast<uint2*>(hi + (size_t)f * g.d + e) = *reinterpret_cast<const uint2*>(h);
+    *reinterpret_cast<uint2*>(lo + (size_t)f * g.d + e) = *reinterpret_cast<const uint2*>(l);
+  }
+  for (int f = threadIdx.x; f < g.r; f += blockDim.x)
+    mass[((size_t)bh * g.n_c + c) * g.r + f] = a[(size_t)f * g.dp + g.d] + (b ? b[(size_t)f * g.dp + g.d] : 0.f);
+}
+
+cudaError_t launch_race_state_split(const float* A, const float* B, bool bwd, void* out, float* mass, const Geom& g,
+                                    cudaStream_t st) {
+  ProfScope ps(bwd ? "race_split_bwd" : "race_split_fwd", st);
+  race_state_split_kernel<<<dim3(g.n_c, g.BH), 256, 0, st>>>(A, B, bwd ? 1 : 0, (__nv_bfloat16*)out, mass, g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_race_w_split(const float* W, void* out, const Geom& g, cudaStream_t st) {
+  const int NW = (g.L * kHashBits + 15) & ~15;
+  race_w_split_kernel<<<(NW * g.d + 255) / 256, 256, 0, st>>>(W, (__nv_bfloat16*)out, g.d, g.L * kHashBits, NW);
+  return cudaGetLastError();
 }
 
 static size_t features_smem(const Geom& g) {

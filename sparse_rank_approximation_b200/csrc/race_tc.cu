@@ -17,10 +17,10 @@
 // corner softmax (dh_b = (1/tau) sum_c p_c (dp_c - <dp, p>) c_b, dp = dPhi / sqrt(L)),
 // du = dh W^T and dx = (du - x <x, du> / |x|^2) / |x| into the fp32 accumulators.
 //
-// Work split: warp 0 issues the TMA loads, warp 1 the MMAs, warps 2..9 (256
-// threads, TMEM lane quarter = warp % 4, column half = (warp - 2) / 4) stage the
-// statistics (fp32 prefix + in-segment part -> bf16 hi + lo halves, 128-byte
-// swizzled) and W, then run the element-wise passes.  The masked intra-chunk
+// Work split: warp 0 issues the TMA loads (the chunk's tiles, its statistics as
+// bf16 hi + lo halves written per chunk by the split kernel, and W as bf16 hi + lo),
+// warp 1 the MMAs, warps 2..9 (256 threads, TMEM lane quarter = warp % 4, column
+// half = (warp - 2) / 4) load the per-row scalars and run the element-wise passes.  The masked intra-chunk
 // matrices (bf16) and dh (bf16 hi + lo) are written back into tensor memory over
 // the fp32 values they replace and feed the next products as the A operand.
 // Every mbarrier wait is bounded; a timeout sets a bit in the caller's error word.
@@ -64,7 +64,7 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t base, int kk, uint32_t slab
 __device__ __forceinline__ uint32_t packed_col(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
 
 struct Bars {
-  uint64_t in_main, ready, s_full, p_full, acc_full, dh_full, du_full;
+  uint64_t in_main, s_full, p_full, acc_full, dh_full, du_full;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -86,72 +86,17 @@ __device__ __forceinline__ void split2(float x, float y, uint32_t& hi, uint32_t&
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-// Statistics of the value columns, (s0 + s1)[f][0:128) for f < 128 from fp32
-// [r][dp] states, as bf16 hi and lo [128 f][128] swizzled tiles; the key-mass
-// column goes to m1[f].  256 threads; each issues all of its loads (16 rows of
-// each source) before the first conversion, so the staging costs one round trip.
-__device__ void stage_state(const float* __restrict__ s0, const float* __restrict__ s1, int dp, unsigned char* hi,
-                            unsigned char* lo, float* m1, int ct) {
-  const int w8 = ct >> 5, lane = ct & 31;
-  float4 v[16], w[16];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) v[k] = __ldg(reinterpret_cast<const float4*>(s0 + (size_t)(w8 + 8 * k) * dp) + lane);
-#pragma unroll
-  for (int k = 0; k < 16; ++k)
-    w[k] = s1 ? __ldg(reinterpret_cast<const float4*>(s1 + (size_t)(w8 + 8 * k) * dp) + lane)
-              : make_float4(0.f, 0.f, 0.f, 0.f);
-  const float mass = ct < kR ? s0[(size_t)ct * dp + kD] + (s1 ? s1[(size_t)ct * dp + kD] : 0.f) : 0.f;
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const int f = w8 + 8 * k;
-    uint32_t h0, l0, h1, l1;
-    split2(v[k].x + w[k].x, v[k].y + w[k].y, h0, l0);
-    split2(v[k].z + w[k].z, v[k].w + w[k].w, h1, l1);
-    const uint32_t off = sw_off(f, 4 * lane, kSlab);
-    *reinterpret_cast<uint2*>(hi + off) = make_uint2(h0, h1);
-    *reinterpret_cast<uint2*>(lo + off) = make_uint2(l0, l1);
-  }
-  if (ct < kR) m1[ct] = mass;
-}
-
-// W[l][k][b] (fp32 [L][128][4]) -> Wt[n = 4 l + b][k] as bf16 hi and lo [32][128]
-// swizzled tiles.  256 threads, two 8-element chunks each.
-__device__ void stage_w(const float* __restrict__ W, unsigned char* hi, unsigned char* lo, int ct) {
-#pragma unroll
-  for (int q = ct; q < kNH * 16; q += kComputeThreads) {
-    const int n = q >> 4, k0 = (q & 15) * 8;
-    float w[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) w[e] = __ldg(W + ((size_t)(n >> 2) * kD + k0 + e) * kHashBits + (n & 3));
-    uint32_t h[4], l[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) split2(w[2 * e], w[2 * e + 1], h[e], l[e]);
-    const uint32_t off = sw_off(n, k0, kWSlab);
-    *reinterpret_cast<uint4*>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
-    *reinterpret_cast<uint4*>(lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
-  }
-}
-
 // Corner-softmax backward of one table: h (4 normalised projections), dp (16
 // corner adjoints, already divided by sqrt(L)) -> dh (4 values).
 __device__ __forceinline__ void corner_bwd(const float (&h)[4], const float (&dp)[16], float inv_tau,
                                            float (&dh)[4]) {
   float sp[4], sm[4];
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    const float y = 2.f * h[b] * inv_tau;
-    sp[b] = 1.f / (1.f + expf(-y));
-    sm[b] = 1.f / (1.f + expf(y));
-  }
+  for (int b = 0; b < 4; ++b) sigmoid_pair(2.f * h[b] * inv_tau, sp[b], sm[b]);
   float p[16], s = 0.f;
+  corner_probs(sp, sm, 1.f, p);
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    float v = 1.f;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) v *= ((c >> b) & 1) ? sp[b] : sm[b];
-    p[c] = v;
-    s = fmaf(v, dp[c], s);
-  }
+  for (int c = 0; c < 16; ++c) s = fmaf(p[c], dp[c], s);
 #pragma unroll
   for (int b = 0; b < 4; ++b) dh[b] = 0.f;
 #pragma unroll
@@ -287,6 +232,7 @@ constexpr uint32_t TK_KAP = 0, TK_X = 128, TK_DV = 256, TK_DPHI = 384, TK_DU = 1
 __global__ void __launch_bounds__(kThreads, 1)
     race_k_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmPQ,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                         const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmW,
                          BwdArgs a, Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   Bars* ms = reinterpret_cast<Bars*>(smem + K_BARS);
@@ -304,7 +250,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->in_main, 1);
-    tc::mbar_init(&ms->ready, kComputeThreads);
     tc::mbar_init(&ms->s_full, 1);
     tc::mbar_init(&ms->p_full, kComputeThreads);
     tc::mbar_init(&ms->acc_full, 1);
@@ -324,7 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 4 : 2) * kTile);
+      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 6 : 4) * kTile + 4 * kWSlab);
+      const int z = (bh * g.n_c + c) * 2;
       for (int s = 0; s < 2; ++s) {
         tc::tma_load_3d(smem + K_PK + s * kSlab, &tmPK, &ms->in_main, 64 * s, c * kC, bh);
         tc::tma_load_3d(smem + K_V + s * kSlab, &tmV, &ms->in_main, 64 * s, c * kC, bh);
@@ -332,6 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tma_load_3d(smem + K_PQ + s * kSlab, &tmPQ, &ms->in_main, 64 * s, c * kC, bh);
           tc::tma_load_3d(smem + K_DO + s * kSlab, &tmdO, &ms->in_main, 64 * s, c * kC, bh);
         }
+        tc::tma_load_3d(smem + K_RH + s * kSlab, &tmR, &ms->in_main, 64 * s, 0, z);
+        tc::tma_load_3d(smem + K_RL + s * kSlab, &tmR, &ms->in_main, 64 * s, 0, z + 1);
+        tc::tma_load_3d(smem + K_WH + s * kWSlab, &tmW, &ms->in_main, 64 * s, 0, 0);
+        tc::tma_load_3d(smem + K_WL + s * kWSlab, &tmW, &ms->in_main, 64 * s, 0, 1);
       }
       tc::mbar_wait(&ms->in_main, 0);
     }
@@ -350,9 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mma_bf16(tmem + TK_X, desc_k(sb + K_V, kk), desc_k(sb + K_DO, kk), idNN, kk > 0 ? 1u : 0u);
         tc::mma_commit(&ms->s_full);
       }
-      ok = ok && wait_or_abort(&ms->ready, 0, ms, err, 0x200u);
       if (ok) {
-        tc::tc_fence_after();
         // inter-chunk parts: dv = Phi_K R^V, dPhi = V R^V^T (R as bf16 hi + lo)
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
@@ -399,21 +347,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     float h16[16];
     load_h(valid ? a.hK + (head + row) * kNH : nullptr, hc, h16);
     const float nrm = valid ? a.nK[head + row] : 1.f;
-    // ---- staging: suffix statistics of the later chunks, W, per-row scalars ----
-    {
-      const float* ra = a.RA + ((size_t)bh * (g.n_seg + 1) + (causal ? c / g.seg + 1 : 0)) * g.r * g.dp;
-      const float* rb = causal ? a.RB + ((size_t)bh * g.n_c + c) * g.r * g.dp : nullptr;
-      stage_state(ra, rb, g.dp, smem + K_RH, smem + K_RL, sR1, ct);
-      stage_w(a.W, smem + K_WH, smem + K_WL, ct);
-      if (ct < kC) {
-        const int r = c * kC + ct;
-        sCl[ct] = r < g.N ? a.rs.cl[head + r] : 0.f;
-        sDl[ct] = r < g.N ? a.rs.delta[head + r] : 0.f;
-      }
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&ms->ready);
-      compute_bar();
+    // ---- per-row scalars of the chunk and the key-mass column of the suffix statistics ----
+    if (ct < kC) {
+      const int r = c * kC + ct;
+      sCl[ct] = r < g.N ? a.rs.cl[head + r] : 0.f;
+      sDl[ct] = r < g.N ? a.rs.delta[head + r] : 0.f;
+      sR1[ct] = a.Rmass[((size_t)bh * g.n_c + c) * kR + ct];
     }
+    compute_bar();
     bool alive = true;
     // ---- intra-chunk element-wise pass: (cl_i kappa_ji) and (cl_i X_ji + delta_i), i >= j ----
     if (causal) {
@@ -493,7 +434,8 @@ constexpr uint32_t TQ_X = 0, TQ_INTRA = 128, TQ_G = 256, TQ_DU = 384;
 
 __global__ void __launch_bounds__(kThreads, 1)
     race_q_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmdO, const __grid_constant__ CUtensorMap tmV,
-                         const __grid_constant__ CUtensorMap tmPK, BwdArgs a, Geom g, uint32_t* err) {
+                         const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmP,
+                         const __grid_constant__ CUtensorMap tmW, BwdArgs a, Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   Bars* ms = reinterpret_cast<Bars*>(smem + Q_BARS);
   float* sP1 = reinterpret_cast<float*>(smem + Q_P1);
@@ -508,7 +450,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->in_main, 1);
-    tc::mbar_init(&ms->ready, kComputeThreads);
     tc::mbar_init(&ms->s_full, 1);
     tc::mbar_init(&ms->p_full, kComputeThreads);
     tc::mbar_init(&ms->acc_full, 1);
@@ -528,13 +469,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 3 : 1) * kTile);
+      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 5 : 3) * kTile + 4 * kWSlab);
+      const int z = (bh * g.n_c + t) * 2;
       for (int s = 0; s < 2; ++s) {
         tc::tma_load_3d(smem + Q_DO + s * kSlab, &tmdO, &ms->in_main, 64 * s, t * kC, bh);
         if (causal) {
           tc::tma_load_3d(smem + Q_V + s * kSlab, &tmV, &ms->in_main, 64 * s, t * kC, bh);
           tc::tma_load_3d(smem + Q_PK + s * kSlab, &tmPK, &ms->in_main, 64 * s, t * kC, bh);
         }
+        tc::tma_load_3d(smem + Q_PH + s * kSlab, &tmP, &ms->in_main, 64 * s, 0, z);
+        tc::tma_load_3d(smem + Q_PL + s * kSlab, &tmP, &ms->in_main, 64 * s, 0, z + 1);
+        tc::tma_load_3d(smem + Q_WH + s * kWSlab, &tmW, &ms->in_main, 64 * s, 0, 0);
+        tc::tma_load_3d(smem + Q_WL + s * kWSlab, &tmW, &ms->in_main, 64 * s, 0, 1);
       }
       tc::mbar_wait(&ms->in_main, 0);
     }
@@ -550,9 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mma_bf16(tmem + TQ_X, desc_k(sb + Q_DO, kk), desc_k(sb + Q_V, kk), idNN, kk > 0 ? 1u : 0u);
         tc::mma_commit(&ms->s_full);
       }
-      ok = ok && wait_or_abort(&ms->ready, 0, ms, err, 0x200u);
       if (ok) {
-        tc::tc_fence_after();
         // inter-chunk part: G = dO P^V^T (P as bf16 hi + lo)
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
@@ -593,15 +537,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float h16[16];
     load_h(valid ? a.hQ + (head + row) * kNH : nullptr, hc, h16);
     const float nrm = valid ? a.nQ[head + row] : 1.f;
-    {
-      const float* pa = a.Ast + ((size_t)bh * (g.n_seg + 1) + (causal ? t / g.seg : g.n_seg)) * g.r * g.dp;
-      const float* pb = causal ? a.Bst + ((size_t)bh * g.n_c + t) * g.r * g.dp : nullptr;
-      stage_state(pa, pb, g.dp, smem + Q_PH, smem + Q_PL, sP1, ct);
-      stage_w(a.W, smem + Q_WH, smem + Q_WL, ct);
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&ms->ready);
-      compute_bar();
-    }
+    if (ct < kR) sP1[ct] = a.Pmass[((size_t)bh * g.n_c + t) * kR + ct];
+    compute_bar();
     bool alive = true;
     // ---- intra-chunk element-wise pass: dkappa_ij = cl_i X_ij + delta_i, j <= i ----
     if (causal) {
@@ -660,7 +597,7 @@ constexpr uint32_t TR_KAP = 0, TR_N = 128;
 __global__ void __launch_bounds__(kThreads, 1)
     race_readout_tc_kernel(const __grid_constant__ CUtensorMap tmPQ, const __grid_constant__ CUtensorMap tmPK,
                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmOlr,
-                           FwdArgs a, Geom g, uint32_t* err) {
+                           const __grid_constant__ CUtensorMap tmP, FwdArgs a, Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   Bars* ms = reinterpret_cast<Bars*>(smem + R_BARS);
   float* sP1 = reinterpret_cast<float*>(smem + R_P1);
@@ -675,7 +612,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->in_main, 1);
-    tc::mbar_init(&ms->ready, kComputeThreads);
     tc::mbar_init(&ms->s_full, 1);
     tc::mbar_init(&ms->p_full, kComputeThreads);
     tc::mbar_init(&ms->acc_full, 1);
@@ -693,13 +629,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 3 : 1) * kTile);
+      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 5 : 3) * kTile);
+      const int z = (bh * g.n_c + t) * 2;
       for (int s = 0; s < 2; ++s) {
         tc::tma_load_3d(smem + R_PQ + s * kSlab, &tmPQ, &ms->in_main, 64 * s, t * kC, bh);
         if (causal) {
           tc::tma_load_3d(smem + R_PK + s * kSlab, &tmPK, &ms->in_main, 64 * s, t * kC, bh);
           tc::tma_load_3d(smem + R_V + s * kSlab, &tmV, &ms->in_main, 64 * s, t * kC, bh);
         }
+        tc::tma_load_3d(smem + R_PH + s * kSlab, &tmP, &ms->in_main, 64 * s, 0, z);
+        tc::tma_load_3d(smem + R_PL + s * kSlab, &tmP, &ms->in_main, 64 * s, 0, z + 1);
       }
       tc::mbar_wait(&ms->in_main, 0);
     }
@@ -715,9 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mma_bf16(tmem + TR_KAP, desc_k(sb + R_PQ, kk), desc_k(sb + R_PK, kk), idNN, kk > 0 ? 1u : 0u);
         tc::mma_commit(&ms->s_full);
       }
-      ok = ok && wait_or_abort(&ms->ready, 0, ms, err, 0x200u);
       if (ok) {
-        tc::tc_fence_after();
         // inter-chunk part: N = Phi_Q P^V (P as bf16 hi + lo)
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
@@ -747,14 +684,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
     const int row = t * kC + i;
     const bool valid = row < g.N;
-    {
-      const float* pa = a.Ast + ((size_t)bh * (g.n_seg + 1) + (causal ? t / g.seg : g.n_seg)) * g.r * g.dp;
-      const float* pb = causal ? a.Bst + ((size_t)bh * g.n_c + t) * g.r * g.dp : nullptr;
-      stage_state(pa, pb, g.dp, smem + R_PH, smem + R_PL, sP1, ct);
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&ms->ready);
-      compute_bar();
-    }
+    if (ct < kR) sP1[ct] = a.Pmass[((size_t)bh * g.n_c + t) * kR + ct];
+    compute_bar();
     bool alive = true;
     float mass = 0.f;                                  // this thread's share of d_lr
     // ---- intra-chunk kappa_ij, j <= i: bf16 into tensor memory, its row sum into the mass ----
@@ -843,17 +774,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Host side
 // ---------------------------------------------------------------------------
 cudaError_t launch_race_readout_tc(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
-  if (!race_bwd_tc_supported(g)) return cudaErrorInvalidValue;
-  CUtensorMap mpq, mpk, mv, mo;
+  if (!race_bwd_tc_supported(g) || !a.Psplit || !a.Pmass) return cudaErrorInvalidValue;
+  CUtensorMap mpq, mpk, mv, mo, mp;
   if (!tc::map_rows_bf16(&mpq, a.phiQ, g.N, g.BH, kC) || !tc::map_rows_bf16(&mpk, a.phiK, g.N, g.BH, kC) ||
-      !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kC) || !tc::map_rows_bf16(&mo, a.Olr, g.N, g.BH, kC))
+      !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kC) || !tc::map_rows_bf16(&mo, a.Olr, g.N, g.BH, kC) ||
+      !tc::map_rows_bf16(&mp, a.Psplit, kR, g.BH * g.n_c * 2, kR))
     return cudaErrorInvalidValue;
   const size_t smem = R_BARS + sizeof(Bars);
   static_assert(R_BARS + sizeof(Bars) <= 232448, "shared memory per CTA");
   cudaError_t e = cudaFuncSetAttribute(race_readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("race_readout_tc", st);
-  race_readout_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mpq, mpk, mv, mo, a, g, err);
+  race_readout_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mpq, mpk, mv, mo, mp, a, g, err);
   return cudaGetLastError();
 }
 
@@ -862,10 +794,14 @@ bool race_bwd_tc_supported(const Geom& g) {
 }
 
 cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
-  if (!race_bwd_tc_supported(g) || !a.hQ || !a.hK || !a.nQ || !a.nK) return cudaErrorInvalidValue;
-  CUtensorMap mpk, mpq, mv, mdo;
+  if (!race_bwd_tc_supported(g) || !a.hQ || !a.hK || !a.nQ || !a.nK || !a.Psplit || !a.Pmass || !a.Rsplit ||
+      !a.Rmass || !a.Wsplit)
+    return cudaErrorInvalidValue;
+  CUtensorMap mpk, mpq, mv, mdo, mp, mr, mw;
   if (!tc::map_rows_bf16(&mpk, a.phiK, g.N, g.BH, kC) || !tc::map_rows_bf16(&mpq, a.phiQ, g.N, g.BH, kC) ||
-      !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kC) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, kC))
+      !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kC) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, kC) ||
+      !tc::map_rows_bf16(&mp, a.Psplit, kR, g.BH * g.n_c * 2, kR) ||
+      !tc::map_rows_bf16(&mr, a.Rsplit, kR, g.BH * g.n_c * 2, kR) || !tc::map_rows_bf16(&mw, a.Wsplit, kNH, 2, kNH))
     return cudaErrorInvalidValue;
   {
     const size_t smem = Q_BARS + sizeof(Bars);
@@ -873,7 +809,7 @@ cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, c
     cudaError_t e = cudaFuncSetAttribute(race_q_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     ProfScope ps("race_q_bwd_tc", st);
-    race_q_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mdo, mv, mpk, a, g, err);
+    race_q_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mdo, mv, mpk, mp, mw, a, g, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -882,7 +818,7 @@ cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, c
   cudaError_t e = cudaFuncSetAttribute(race_k_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("race_k_bwd_tc", st);
-  race_k_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mpk, mpq, mv, mdo, a, g, err);
+  race_k_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mpk, mpq, mv, mdo, mr, mw, a, g, err);
   return cudaGetLastError();
 }
 
