@@ -88,6 +88,9 @@ typedef struct {
   float lambda;           /* Eq. 5 lambda when lambda_vec == NULL */
   float eps;              /* Eq. 5 epsilon (>= 0) */
   float tau;              /* RACE soft-assignment temperature (> 0) */
+  int32_t fixed_m;        /* 0: denominator-aware fusion (Eq. 5).  1: the paper's ablation without it
+                             (Sort_Lsh_RACE, §6 "Attention variants"): m = 1 and g_lr defaults to 1,
+                             so O = g_s O_s + g_lr O_lr.  Must match between forward and backward. */
 } elsaa_params;
 
 /* Bytes of the caller-owned `saved` buffer the forward fills and the backward
@@ -126,6 +129,23 @@ ELSAA_API elsaa_status elsaa_backward(const elsaa_params* params,
                             const void* dO, const void* saved,
                             void* dQ, void* dK, void* dV,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Per-row gradients of sum(dO * O) with respect to the fusion parameters of Eq. 5 /
+ * Eq. 4 (the paper's optional learnable lambda, §1 contribution 3, and the two gates):
+ *   dlambda[i] = -dm_i d_s,i d_lr,i / D_i^2     (0 when fixed_m = 1)
+ *   dg_sparse[i] = m_i <dO_i, O_s,i>,  dg_lr[i] = <dO_i, O_lr,i>
+ * with dm_i = g_s,i <dO_i, O_s,i> - [g_lr == NULL] <dO_i, O_lr,i> and D_i = d_s,i + lambda_i d_lr,i + eps.
+ * A gate passed as NULL gets the derivative at its default value.  For a scalar lambda
+ * (lambda_vec == NULL) its gradient is the sum of dlambda over all rows.
+ *   lambda_vec, g_sparse, g_lr  in   float32 [B,H,N] or NULL, as given to the forward
+ *   dO                          in   [B,H,N,d] dtype
+ *   saved                       in   the forward's `saved` buffer
+ *   dlambda, dg_sparse, dg_lr   out  float32 [B,H,N]; any may be NULL (not written)
+ * Asynchronous on `stream`; allocates nothing and needs no workspace. */
+ELSAA_API elsaa_status elsaa_fusion_grads(const elsaa_params* params, const float* lambda_vec,
+                                          const float* g_sparse, const float* g_lr, const void* dO,
+                                          const void* saved, float* dlambda, float* dg_sparse, float* dg_lr,
+                                          void* stream);
 
 /* Selection only: the float32 block scores the selector ranks and the chosen
  * blocks, for checking the selector against an external implementation.

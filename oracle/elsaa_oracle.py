@@ -56,6 +56,7 @@ class Params:
     eps: float = 1e-6
     tau: float = 1.0
     chunk: Optional[int] = None   # RACE causal chunk size; defaults to block_size
+    fixed_m: bool = False    # ablation without denominator-aware fusion: m = 1, default g_lr = 1
 
     @property
     def n_tables(self) -> int:
@@ -275,15 +276,21 @@ def race_rows(q, k, v, W, p: Params, rows) -> tuple:
 # ----------------------------------------------------------------------------
 
 def fuse(O_s, logd_s, O_lr, d_lr, p: Params, lam=None, g_s=None, g_lr=None):
-    """m = d_s / (d_s + lam d_lr + eps);  O = g_s m O_s + g_lr O_lr.
+    """m = d_s / (d_s + lam d_lr + eps);  O = g_s m O_s + g_lr O_lr  [ELSAA §3.3 Eq. 5, §1 Eq. 4].
 
-    Default gates: g_s = 1, g_lr = 1 - m.  Returns (O, m).
+    Default gates: g_s = 1, g_lr = 1 - m.  With ``p.fixed_m`` (the paper's
+    Sort_Lsh_RACE ablation, §6 "Attention variants": m_sparse = 1, no
+    denominator-aware rescaling) m = 1 and the default g_lr is 1, so the two
+    branch outputs are added.  Returns (O, m).
     """
     d_s = np.exp(logd_s)
     lam = p.lam if lam is None else _f64(lam)
-    m = d_s / (d_s + lam * d_lr + p.eps)
+    if p.fixed_m:
+        m = np.ones_like(d_s * d_lr)
+    else:
+        m = d_s / (d_s + lam * d_lr + p.eps)
     gs = 1.0 if g_s is None else _f64(g_s)
-    gl = (1.0 - m) if g_lr is None else _f64(g_lr)
+    gl = (1.0 if p.fixed_m else 1.0 - m) if g_lr is None else _f64(g_lr)
     O = (gs * m)[..., None] * O_s + np.broadcast_to(gl, m.shape)[..., None] * O_lr
     return O, m
 
@@ -347,16 +354,42 @@ def _fusion_adjoints(dO, fw, p: Params, lam, g_s, g_lr):
     d_lr = fw["d_lr"]
     lam = p.lam if lam is None else _f64(lam)
     gs = np.ones_like(m) if g_s is None else _f64(g_s)
-    gl = (1.0 - m) if g_lr is None else _f64(g_lr)
+    gl = (np.ones_like(m) if p.fixed_m else 1.0 - m) if g_lr is None else _f64(g_lr)
     a = (dO * fw["O_s"]).sum(axis=1)
     b = (dO * fw["O_lr"]).sum(axis=1)
-    dm = gs * a - (b if g_lr is None else 0.0)
+    # with m held at 1 nothing flows back through m
+    dm = np.zeros_like(m) if p.fixed_m else gs * a - (b if g_lr is None else 0.0)
     D = d_s + lam * d_lr + p.eps
     dds_ds = dm * (lam * d_lr + p.eps) * d_s / D ** 2
     ddlr = -dm * lam * d_s / D ** 2
     dOs = (gs * m)[:, None] * dO
     dOlr = gl[:, None] * dO
     return dOs, dOlr, dds_ds, ddlr
+
+
+def fusion_param_grads(dO, fw, p: Params, lam=None, g_s=None, g_lr=None):
+    """Per-row gradients of the loss <dO, O> with respect to the fusion parameters
+    lambda_i, g_s,i and g_lr,i of Eq. 5 / Eq. 4 (the paper's optional learnable lambda).
+
+      dlambda = dm * dm/dlambda = -dm d_s d_lr / D^2     (0 when m is held at 1)
+      dg_s    = m <dO, O_s>,   dg_lr = <dO, O_lr>
+    with dm = g_s <dO, O_s> - [g_lr defaulted to 1 - m] <dO, O_lr>.  A gate left at
+    its default still gets the derivative at that value.  Returns (dlam, dgs, dglr)."""
+    dO = _f64(dO)
+    m = fw["m"]
+    d_s = np.exp(fw["logd_s"])
+    d_lr = fw["d_lr"]
+    lam = p.lam if lam is None else _f64(lam)
+    gs = np.ones_like(m) if g_s is None else _f64(g_s)
+    a = (dO * fw["O_s"]).sum(axis=1)
+    b = (dO * fw["O_lr"]).sum(axis=1)
+    if p.fixed_m:
+        dlam = np.zeros_like(m)
+    else:
+        dm = gs * a - (b if g_lr is None else 0.0)
+        D = d_s + lam * d_lr + p.eps
+        dlam = -dm * d_s * d_lr / D ** 2
+    return dlam, m * a, b
 
 
 def race_features_backward(X, W, p: Params, dPhi):

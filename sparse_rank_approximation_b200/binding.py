@@ -28,7 +28,8 @@ ELSAA_DTYPE_BF16 = 1
 
 EXPORTED = ("elsaa_saved_bytes", "elsaa_workspace_bytes", "elsaa_forward", "elsaa_backward",
             "elsaa_debug_select", "elsaa_check_device_flags", "elsaa_status_string",
-            "elsaa_last_error_message", "elsaa_profile_begin", "elsaa_profile_end", "elsaa_select_noalloc")
+            "elsaa_last_error_message", "elsaa_profile_begin", "elsaa_profile_end", "elsaa_select_noalloc",
+            "elsaa_fusion_grads")
 
 
 class Params(ctypes.Structure):
@@ -36,7 +37,7 @@ class Params(ctypes.Structure):
                 ("dtype", ctypes.c_int32), ("causal", ctypes.c_int32), ("rank_r", ctypes.c_int32),
                 ("hash_bits", ctypes.c_int32), ("block_size", ctypes.c_int32), ("topk", ctypes.c_int32),
                 ("scale", ctypes.c_float), ("lam", ctypes.c_float), ("eps", ctypes.c_float),
-                ("tau", ctypes.c_float)]
+                ("tau", ctypes.c_float), ("fixed_m", ctypes.c_int32)]
 
 
 class ElsaaError(RuntimeError):
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
     L.elsaa_profile_end.restype = i32
     L.elsaa_select_noalloc.argtypes = [P, vp, vp, vp, vp]
     L.elsaa_select_noalloc.restype = i32
+    L.elsaa_fusion_grads.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.elsaa_fusion_grads.restype = i32
     _lib = L
     return L
 
@@ -93,9 +96,10 @@ def _check(status: int, where: str) -> None:
 
 
 def make_params(B, H, N, d, *, dtype=ELSAA_DTYPE_BF16, causal=True, rank_r=128, block_size=128, topk=16,
-                scale=None, lam=1.0, eps=1e-6, tau=1.0, hash_bits=4) -> Params:
+                scale=None, lam=1.0, eps=1e-6, tau=1.0, hash_bits=4, fixed_m=False) -> Params:
     return Params(B, H, N, d, dtype, int(bool(causal)), rank_r, hash_bits, block_size, topk,
-                  float(1.0 / math.sqrt(d) if scale is None else scale), float(lam), float(eps), float(tau))
+                  float(1.0 / math.sqrt(d) if scale is None else scale), float(lam), float(eps), float(tau),
+                  int(bool(fixed_m)))
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -157,6 +161,16 @@ class Elsaa:
         _check(st, "elsaa_backward")
         return dQ, dK, dV
 
+    def fusion_grads(self, dO, lam_vec=None, g_s=None, g_lr=None, stream=None):
+        """Per-row gradients (dlambda, dg_sparse, dg_lr), float32 [B, H, N], of sum(dO * O)
+        for the last forward call."""
+        shape = (self.p.B, self.p.H, self.p.N)
+        out = [torch.empty(shape, dtype=torch.float32, device=self.device) for _ in range(3)]
+        st = lib().elsaa_fusion_grads(ctypes.byref(self.p), _ptr(lam_vec), _ptr(g_s), _ptr(g_lr), _ptr(dO),
+                                      _ptr(self.saved), _ptr(out[0]), _ptr(out[1]), _ptr(out[2]), _stream(stream))
+        _check(st, "elsaa_fusion_grads")
+        return tuple(out)
+
     def debug_select(self, q, k, stream=None):
         n_t = -(-self.p.N // self.p.block_size)
         scores = torch.empty(self.p.B, self.p.H, n_t, n_t, dtype=torch.float32, device=self.device)
@@ -199,5 +213,12 @@ class ElsaaFunction(torch.autograd.Function):
     @staticmethod
     def backward(ctx, dO):
         q, k, v, W = ctx.saved_tensors
-        dQ, dK, dV = ctx.op.backward(q, k, v, W, dO.contiguous(), *ctx.extra)
-        return dQ, dK, dV, None, None, None, None, None
+        dO = dO.contiguous()
+        dQ, dK, dV = ctx.op.backward(q, k, v, W, dO, *ctx.extra)
+        lam_vec, g_s, g_lr = ctx.extra
+        need = [t is not None and t.requires_grad for t in (lam_vec, g_s, g_lr)]
+        dl = dgs = dgl = None
+        if any(need):
+            dl, dgs, dgl = ctx.op.fusion_grads(dO, lam_vec, g_s, g_lr)
+        return (dQ, dK, dV, None, None, dl if need[0] else None, dgs if need[1] else None,
+                dgl if need[2] else None)

@@ -378,9 +378,9 @@ __global__ void __launch_bounds__(2 * T) attn_fwd_bf16_kernel(
     const int qc = min(qi, g.N - 1);
     const float lam = lam_vec ? lam_vec[head + qc] : g.lam;
     const float c = lam * dl[h] + g.eps;
-    mfac[h] = logd[h] == -INFINITY ? 0.f : 1.f / (1.f + c * expf(-logd[h]));
+    mfac[h] = g.fixed_m ? 1.f : logd[h] == -INFINITY ? 0.f : 1.f / (1.f + c * expf(-logd[h]));
     const float gs = gs_vec ? gs_vec[head + qc] : 1.f;
-    const float gl = glr_vec ? glr_vec[head + qc] : 1.f - mfac[h];
+    const float gl = glr_vec ? glr_vec[head + qc] : g.fixed_m ? 1.f : 1.f - mfac[h];
     cs[h] = gs * mfac[h];
     cl[h] = dl[h] > 0.f ? gl / dl[h] : 0.f;
   }

@@ -358,8 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (alive) {
       const float logd = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      const float mf = logd == -INFINITY ? 0.f : 1.f / (1.f + (lam * dl + g.eps) * expf(-logd));
-      const float gl = a.glr ? glr_in : 1.f - mf;
+      const float mf = g.fixed_m ? 1.f : logd == -INFINITY ? 0.f : 1.f / (1.f + (lam * dl + g.eps) * expf(-logd));
+      const float gl = a.glr ? glr_in : g.fixed_m ? 1.f : 1.f - mf;
       const float cs = gs * mf;
       const unsigned char* lrow = smem + off_k(0) + half * kSlab + row * 128;
       unsigned char* orow = smem + off_v(0) + half * kSlab + row * 128;

@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(256) row_scalars_kernel(BwdArgs a, Geom g) {
       const double lam0 = a.lam ? a.lam[i] : g.lam;
       const double c0 = lam0 * dl0 + (double)g.eps;
       const double D0 = exp(logd0) + c0;
-      const double gl0 = a.glr ? (double)a.glr[i] : (D0 > 0.0 ? c0 / D0 : 1.0);
+      const double gl0 = a.glr ? (double)a.glr[i] : g.fixed_m ? 1.0 : (D0 > 0.0 ? c0 / D0 : 1.0);
       cl_row = dl0 > 0.0 ? gl0 / dl0 : 0.0;
     }
     const float clf = __shfl_sync(0xffffffffu, (float)cl_row, (threadIdx.x & 31) - sub);
@@ -89,10 +89,11 @@ __global__ void __launch_bounds__(256) row_scalars_kernel(BwdArgs a, Geom g) {
   const double ds = exp(logd);
   const double c = lam * dl + (double)g.eps;
   const double D = ds + c;
-  const double m = D > 0.0 ? ds / D : 0.0;
-  const double one_m = D > 0.0 ? c / D : 1.0;
-  const double gl = a.glr ? (double)a.glr[i] : one_m;
-  const double dm = gs * A - (a.glr ? 0.0 : (double)Bv);
+  // fixed_m: the ablation without denominator-aware fusion (m = 1, default g_lr = 1, no dm)
+  const double m = g.fixed_m ? 1.0 : D > 0.0 ? ds / D : 0.0;
+  const double one_m = g.fixed_m ? 0.0 : D > 0.0 ? c / D : 1.0;
+  const double gl = a.glr ? (double)a.glr[i] : g.fixed_m ? 1.0 : one_m;
+  const double dm = g.fixed_m ? 0.0 : gs * A - (a.glr ? 0.0 : (double)Bv);
   const double cs = gs * m;
   const double cl = dl > 0.0 ? gl / dl : 0.0;
   const double ddlr = D > 0.0 ? -dm * lam * ds / (D * D) : 0.0;
@@ -102,6 +103,62 @@ __global__ void __launch_bounds__(256) row_scalars_kernel(BwdArgs a, Geom g) {
     a.rs.packed[i] = make_float4((float)(logd * 1.4426950408889634), (float)cs, (float)(cs * A - dm * m * one_m), 0.f);
   a.rs.cl[i] = (float)cl;
   a.rs.delta[i] = (float)(ddlr - cl * Bv);
+}
+
+// Per-row gradients of sum(dO * O) with respect to lambda, g_s and g_lr (Eq. 5 / Eq. 4):
+// dlambda = -dm d_s d_lr / D^2 (0 when m is held at 1), dg_s = m <dO, O_s>, dg_lr = <dO, O_lr>,
+// dm = g_s <dO, O_s> - [g_lr defaulted] <dO, O_lr>.  Same row layout as the row scalars.
+template <typename E>
+__global__ void __launch_bounds__(256) fusion_grads_kernel(const E* __restrict__ dO_, const E* __restrict__ Os_,
+                                                           const E* __restrict__ Olr_, const float* __restrict__ logd_,
+                                                           const float* __restrict__ dlr_, const float* lamv,
+                                                           const float* gsv, const float* glrv, float* dlam,
+                                                           float* dgs, float* dglr, Geom g) {
+  const int tpr = g.d / 8;
+  const int rpb = 256 / tpr;
+  const int sub = threadIdx.x % tpr;
+  const int row = blockIdx.x * rpb + threadIdx.x / tpr;
+  const size_t i = (size_t)blockIdx.y * g.N + min(row, g.N - 1);
+  float dO[8], os[8], ol[8];
+  load8<E>(dO_ + i * g.d + sub * 8, dO);
+  load8<E>(Os_ + i * g.d + sub * 8, os);
+  load8<E>(Olr_ + i * g.d + sub * 8, ol);
+  float A = 0.f, Bv = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    A += dO[j] * os[j];
+    Bv += dO[j] * ol[j];
+  }
+  for (int o = 1; o < tpr; o <<= 1) {
+    A += __shfl_xor_sync(0xffffffffu, A, o);
+    Bv += __shfl_xor_sync(0xffffffffu, Bv, o);
+  }
+  if (sub != 0 || row >= g.N) return;
+  const double dl = dlr_[i], ds = exp((double)logd_[i]);
+  const double lam = lamv ? lamv[i] : g.lam;
+  const double gs = gsv ? gsv[i] : 1.0;
+  const double D = ds + lam * dl + (double)g.eps;
+  const double m = g.fixed_m ? 1.0 : D > 0.0 ? ds / D : 0.0;
+  const double dm = g.fixed_m ? 0.0 : gs * A - (glrv ? 0.0 : (double)Bv);
+  if (dlam) dlam[i] = (g.fixed_m || !(D > 0.0)) ? 0.f : (float)(-dm * ds * dl / (D * D));
+  if (dgs) dgs[i] = (float)(m * A);
+  if (dglr) dglr[i] = Bv;
+}
+
+cudaError_t launch_fusion_grads(const void* dO, const void* Os, const void* Olr, const float* logd, const float* dlr,
+                                const float* lam, const float* gs, const float* glr, float* dlam, float* dgs,
+                                float* dglr, bool bf16, const Geom& g, cudaStream_t st) {
+  const int rpb = 256 / (g.d / 8);
+  dim3 grid((g.N + rpb - 1) / rpb, g.BH);
+  ProfScope ps("fusion_grads", st);
+  if (bf16)
+    fusion_grads_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)dO, (const __nv_bfloat16*)Os,
+                                                             (const __nv_bfloat16*)Olr, logd, dlr, lam, gs, glr,
+                                                             dlam, dgs, dglr, g);
+  else
+    fusion_grads_kernel<float><<<grid, 256, 0, st>>>((const float*)dO, (const float*)Os, (const float*)Olr, logd, dlr,
+                                                     lam, gs, glr, dlam, dgs, dglr, g);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_row_scalars(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st) {

@@ -28,6 +28,7 @@ struct Geom {
   int n_seg;      // segments = ceil(n_c / seg)
   int dp;         // state columns: d value columns + 8 (column d holds the key mass)
   int causal;
+  int fixed_m;    // fusion without the denominator-aware weight: m = 1, default g_lr = 1
   float scale, lam, eps, tau;
 };
 

@@ -105,6 +105,7 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
   g->n_seg = (g->n_c + g->seg - 1) / g->seg;
   g->dp = p->d + 8;
   g->causal = p->causal;
+  g->fixed_m = p->fixed_m != 0;
   g->scale = p->scale;
   g->lam = p->lambda;
   g->eps = p->eps;
@@ -456,6 +457,30 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
     ELSAA_TRY(cuda_status(launch_bwd_f32(a, g, st_), "backward"));
   }
   return ELSAA_OK;
+}
+
+elsaa_status elsaa_fusion_grads(const elsaa_params* p, const float* lam, const float* gs, const float* glr,
+                                const void* dO, const void* saved, float* dlam, float* dgs, float* dglr,
+                                void* stream) {
+  g_last_error.clear();
+  Geom g;
+  elsaa_status st;
+  if (!make_geom(p, &g, &st)) return st;
+  ELSAA_TRY(check_ptr(dO, "dO"));
+  ELSAA_TRY(check_ptr(saved, "saved"));
+  ELSAA_TRY(check_ptr(lam, "lambda_vec", false));
+  ELSAA_TRY(check_ptr(gs, "g_sparse", false));
+  ELSAA_TRY(check_ptr(glr, "g_lr", false));
+  ELSAA_TRY(check_ptr(dlam, "dlambda", false));
+  ELSAA_TRY(check_ptr(dgs, "dg_sparse", false));
+  ELSAA_TRY(check_ptr(dglr, "dg_lr", false));
+  const bool bf16 = p->dtype == ELSAA_DTYPE_BF16;
+  size_t sb = 0;
+  Saved s = carve_saved(const_cast<void*>(saved), g, bf16 ? 2 : 4, &sb);
+  if (!dlam && !dgs && !dglr) return ELSAA_OK;
+  return cuda_status(launch_fusion_grads(dO, s.Os, s.Olr, s.logd, s.dlr, lam, gs, glr, dlam, dgs, dglr, bf16, g,
+                                         static_cast<cudaStream_t>(stream)),
+                     "fusion gradients");
 }
 
 elsaa_status elsaa_debug_select(const elsaa_params* p, const void* Q, const void* K, float* scores, int32_t* idx,

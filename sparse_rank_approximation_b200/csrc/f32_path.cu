@@ -103,9 +103,9 @@ __global__ void __launch_bounds__(256) attn_fwd_f32_kernel(FwdArgs a, Geom g) {
   const float dl = __shfl_sync(0xffffffffu, acc[g.d / 32], g.d % 32);
   const float lam = a.lam ? a.lam[head + qi] : g.lam;
   const float cc = lam * dl + g.eps;
-  const float mf = logd == -INFINITY ? 0.f : 1.f / (1.f + cc * expf(-logd));
+  const float mf = g.fixed_m ? 1.f : logd == -INFINITY ? 0.f : 1.f / (1.f + cc * expf(-logd));
   const float gs = a.gs ? a.gs[head + qi] : 1.f;
-  const float gl = a.glr ? a.glr[head + qi] : 1.f - mf;
+  const float gl = a.glr ? a.glr[head + qi] : g.fixed_m ? 1.f : 1.f - mf;
   const float cs = gs * mf, cl = dl > 0.f ? gl / dl : 0.f;
   float* O = (float*)a.O + (head + qi) * g.d;
   float* Os = (float*)a.Os + (head + qi) * g.d;

@@ -93,6 +93,10 @@ cudaError_t launch_race_readout_bf16(const FwdArgs& a, const Geom& g, cudaStream
 cudaError_t launch_race_readout_tc(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
 cudaError_t launch_attn_fwd_f32(const FwdArgs& a, const Geom& g, cudaStream_t st);
 cudaError_t launch_row_scalars(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st);
+// Per-row gradients of the fusion parameters lambda, g_s, g_lr (any output may be null).
+cudaError_t launch_fusion_grads(const void* dO, const void* Os, const void* Olr, const float* logd, const float* dlr,
+                                const float* lam, const float* gs, const float* glr, float* dlam, float* dgs,
+                                float* dglr, bool bf16, const Geom& g, cudaStream_t st);
 // RACE backward (bf16): low-rank parts of dQ, dK, dV into the fp32 accumulators.
 cudaError_t launch_race_bwd_bf16(const BwdArgs& a, const Geom& g, cudaStream_t st);
 // tcgen05 sparse-branch backward (d = 128, block 128): dQ (query-major) and dK/dV

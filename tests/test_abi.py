@@ -74,6 +74,10 @@ def test_argument_errors_return_before_any_launch():
                           0x1000, 0x1000, 0x1000, 0x1000, 1 << 40, None)
     assert st == bd.ELSAA_ERR_INVALID_ARG and b"dO" in L.elsaa_last_error_message()
     assert L.elsaa_check_device_flags(None, None) == bd.ELSAA_ERR_INVALID_ARG
+    st = L.elsaa_fusion_grads(ctypes.byref(p), None, None, None, None, 0x1000, 0x1000, None, None, None)
+    assert st == bd.ELSAA_ERR_INVALID_ARG and b"dO" in L.elsaa_last_error_message()
+    # nothing requested: returns before any launch
+    assert L.elsaa_fusion_grads(ctypes.byref(p), None, None, None, 0x1000, 0x1000, None, None, None, None) == 0
 
 
 def test_status_strings():

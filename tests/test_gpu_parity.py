@@ -10,7 +10,7 @@ import torch
 
 from oracle import elsaa_oracle as orc
 from sparse_rank_approximation_b200.workloads import WORKLOADS, make_inputs, small_workload
-from tests.harness import check, device_inputs, gpu_op, np64, oracle_params
+from tests.harness import BF16_ABS_TOL, check, device_inputs, gpu_op, np64, oracle_params
 
 pytestmark = pytest.mark.gpu
 
@@ -36,7 +36,7 @@ SMALL = {
 def _run(w, seed=0, lam_vec=False, gates=False, **over):
     inp = make_inputs(w, seed)
     dev = device_inputs(w, inp)
-    op = gpu_op(w, **{k: v for k, v in over.items() if k in ("lam", "eps", "tau")})
+    op = gpu_op(w, **{k: v for k, v in over.items() if k in ("lam", "eps", "tau", "fixed_m")})
     BH = (w.B, w.H, w.N)
     g = torch.Generator().manual_seed(seed + 100)
     extra_cpu = {}
@@ -51,6 +51,7 @@ def _run(w, seed=0, lam_vec=False, gates=False, **over):
     dQ, dK, dV = op.backward(dev["Q"], dev["K"], dev["V"], dev["W"], dev["dO"], extra.get("lam"),
                              extra.get("g_s"), extra.get("g_lr"))
     torch.cuda.synchronize()
+    _run.last = (op, dev, extra)
     return inp, extra_cpu, O, scores, idx, (dQ, dK, dV)
 
 
@@ -80,7 +81,7 @@ def test_forward_backward_small(name):
             check(w, f"dV[{b},{h}]", np64(grads[2][b, h]), dv)
 
 
-@pytest.mark.parametrize("case", ["k0", "r0_eps0", "lam_gates", "tau_lam", "noncausal"])
+@pytest.mark.parametrize("case", ["k0", "r0_eps0", "lam_gates", "tau_lam", "noncausal", "fixed_m", "fixed_m_gates"])
 @pytest.mark.parametrize("geom", ["bf16_d64_T64", "bf16_d128_T128", "bf16_d128_T128_r128", "f32_d64_T64"])
 def test_branch_switches_and_options(case, geom):
     parts = geom.split("_")
@@ -99,6 +100,11 @@ def test_branch_switches_and_options(case, geom):
         over.update(tau=0.5, lam=3.0, eps=0.01)
     elif case == "noncausal":
         base["causal"] = False
+    elif case == "fixed_m":
+        over["fixed_m"] = True
+    elif case == "fixed_m_gates":
+        over["fixed_m"] = True
+        lam_vec = gates = True
     w = small_workload(**base)
     inp, extra, O, scores, idx, grads = _run(w, lam_vec=lam_vec, gates=gates, **over)
     for h in range(w.H):
@@ -107,6 +113,46 @@ def test_branch_switches_and_options(case, geom):
         check(w, "dQ", np64(grads[0][0, h]), dq)
         check(w, "dK", np64(grads[1][0, h]), dk)
         check(w, "dV", np64(grads[2][0, h]), dv)
+
+
+@pytest.mark.parametrize("gates", [False, True])
+@pytest.mark.parametrize("fixed_m", [False, True])
+@pytest.mark.parametrize("geom", ["bf16_d128_T128_r128", "bf16_d64_T64", "f32_d64_T64"])
+def test_fusion_parameter_gradients(geom, fixed_m, gates):
+    """elsaa_fusion_grads (per-row d/dlambda, d/dg_s, d/dg_lr) against the oracle's."""
+    parts = geom.split("_")
+    dtype, d, T = parts[0], int(parts[1][1:]), int(parts[2][1:])
+    r = int(parts[3][1:]) if len(parts) > 3 else 32
+    w = small_workload(N=T * 3 + 20, d=d, block_size=T, topk=2, rank_r=r, dtype=dtype, H=2)
+    over = {"fixed_m": fixed_m}
+    inp, extra, O, scores, idx, grads = _run(w, lam_vec=True, gates=gates, **over)
+    op, dev, extra_dev = _run.last
+    dl, dgs, dgl = op.fusion_grads(dev["dO"], extra_dev.get("lam"), extra_dev.get("g_s"), extra_dev.get("g_lr"))
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        p = oracle_params(w, **over)
+        fw, _ = _oracle_head(w, inp, extra, scores, 0, h, **over)
+        ex = {k: v[0, h].double().numpy() for k, v in extra.items()}
+        dO_h = inp["dO"][0, h].double().numpy()
+        ref = orc.fusion_param_grads(dO_h, fw, p, ex.get("lam"), ex.get("g_s"), ex.get("g_lr"))
+        if w.dtype == "f32":
+            for name, got, want in zip(("dlambda", "dg_s", "dg_lr"), (dl, dgs, dgl), ref):
+                check(w, f"{name}[{h}]", np64(got[0, h]), want)
+            continue
+        # bf16: the GPU reduces over the saved bf16 O_s and O_lr, each element within half an
+        # ulp (2^-9 relative) of the exact value, so row i's dot product is off by at most
+        # 2^-9 sum_k |dO_ik O_ik|; the bound below doubles that and adds the usual 2e-2.
+        sa = np.abs(dO_h * fw["O_s"]).sum(axis=1)
+        sb = np.abs(dO_h * fw["O_lr"]).sum(axis=1)
+        gs = ex.get("g_s", np.ones(w.N))
+        ds = np.exp(fw["logd_s"])
+        lam = ex["lam"]
+        D = ds + lam * fw["d_lr"] + p.eps
+        dm_bound = gs * sa + (0.0 if "g_lr" in ex else sb)
+        bounds = (np.where(fixed_m, 0.0, ds * fw["d_lr"] / D ** 2 * dm_bound), fw["m"] * sa, sb)
+        for name, got, want, bnd in zip(("dlambda", "dg_s", "dg_lr"), (dl, dgs, dgl), ref, bounds):
+            err = np.abs(np64(got[0, h]) - want)
+            assert np.all(err <= BF16_ABS_TOL + 2.0 ** -8 * bnd), f"{name}[{h}]: max err {err.max():.3e}"
 
 
 @pytest.mark.parametrize("name", ["n2k_d64", "n8k_d64", "n16k_d128", "n64k_d128"])

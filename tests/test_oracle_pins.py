@@ -331,12 +331,16 @@ def _loss(q, k, v, W, p, dO, lam=None, g_s=None, g_lr=None):
     return float((out["O"] * dO).sum()), out["idx"]
 
 
-@pytest.mark.parametrize("causal,gates,r,k,tau", [(True, False, 32, 2, 1.0), (False, False, 16, 2, 0.6),
-                                                  (True, True, 16, 3, 1.7), (True, False, 0, 2, 1.0),
-                                                  (True, False, 32, 0, 0.8)])
-def test_backward_matches_finite_differences(causal, gates, r, k, tau):
+@pytest.mark.parametrize("causal,gates,r,k,tau,fixed_m", [(True, False, 32, 2, 1.0, False),
+                                                          (False, False, 16, 2, 0.6, False),
+                                                          (True, True, 16, 3, 1.7, False),
+                                                          (True, False, 0, 2, 1.0, False),
+                                                          (True, False, 32, 0, 0.8, False),
+                                                          (True, False, 16, 2, 1.0, True),
+                                                          (False, True, 16, 2, 1.3, True)])
+def test_backward_matches_finite_differences(causal, gates, r, k, tau, fixed_m):
     N, d, T = 24, 6, 4
-    q, k_, v, W, p = _setup(N=N, d=d, T=T, k=k, r=r, causal=causal, seed=50, lam=0.8, tau=tau)
+    q, k_, v, W, p = _setup(N=N, d=d, T=T, k=k, r=r, causal=causal, seed=50, lam=0.8, tau=tau, fixed_m=fixed_m)
     if r == 0:
         W = np.zeros((0, d, 4))
     dO = _rand((N, d), 60)
@@ -365,6 +369,49 @@ def test_backward_matches_finite_differences(causal, gates, r, k, tau):
         assert np.abs(fd - G).max() <= 1e-6 * max(scale, 1.0)
         assert np.linalg.norm(fd - G) <= 1e-6 * np.linalg.norm(G) + 1e-9
     assert skipped <= 3
+
+
+@pytest.mark.parametrize("fixed_m", [False, True])
+def test_fusion_parameter_gradients_match_finite_differences(fixed_m):
+    """d<dO, O>/d lambda_i, d/d g_s,i and d/d g_lr,i, one row at a time; gates left at
+    their default are differentiated at that value (passed explicitly to the FD runs)."""
+    N, d, T = 20, 6, 4
+    q, k, v, W, p = _setup(N=N, d=d, T=T, k=2, r=16, causal=True, seed=70, fixed_m=fixed_m)
+    dO = _rand((N, d), 71)
+    lam = np.linspace(0.4, 1.6, N)
+    fw = orc.forward_head(q, k, v, W, p, lam)
+    dlam, dgs, dglr = orc.fusion_param_grads(dO, fw, p, lam)
+    gs0 = np.ones(N)
+    gl0 = np.ones(N) if fixed_m else 1.0 - fw["m"]
+    h = 1e-6
+
+    def loss(lam_, g_s=None, g_lr=None):
+        return float((orc.forward_head(q, k, v, W, p, lam_, g_s, g_lr)["O"] * dO).sum())
+
+    for i in range(N):
+        e = np.zeros(N)
+        e[i] = h
+        fd_lam = (loss(lam + e) - loss(lam - e)) / (2 * h)
+        assert abs(fd_lam - dlam[i]) <= 1e-6 * max(1.0, abs(dlam[i]))
+        fd_gs = (loss(lam, gs0 + e) - loss(lam, gs0 - e)) / (2 * h)
+        assert abs(fd_gs - dgs[i]) <= 1e-6 * max(1.0, abs(dgs[i]))
+        fd_gl = (loss(lam, gs0, gl0 + e) - loss(lam, gs0, gl0 - e)) / (2 * h)
+        assert abs(fd_gl - dglr[i]) <= 1e-6 * max(1.0, abs(dglr[i]))
+    if fixed_m:
+        assert np.all(dlam == 0.0)
+
+
+def test_fixed_m_adds_the_two_branch_outputs():
+    """The ablation without denominator-aware fusion (m = 1, default g_lr = 1) is the
+    sum of the sparse-only output (r = 0) and the low-rank-only output (k = 0)."""
+    q, k, v, W, p = _setup(N=40, T=8, k=2, r=32, causal=True, seed=80, fixed_m=True)
+    both = orc.forward_head(q, k, v, W, p)
+    p_s = _params(p.N, p.d, p.block_size, p.topk, 0, True, fixed_m=True)
+    p_l = _params(p.N, p.d, p.block_size, 0, p.rank_r, True, fixed_m=True)
+    sparse_only = orc.forward_head(q, k, v, np.zeros((0, p.d, 4)), p_s)["O"]
+    lowrank_only = orc.forward_head(q, k, v, W, p_l)["O"]
+    np.testing.assert_allclose(both["O"], sparse_only + lowrank_only, rtol=0, atol=1e-12)
+    assert np.all(both["m"] == 1.0)
 
 
 # --- a value printed in the paper ---
