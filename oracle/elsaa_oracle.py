@@ -574,6 +574,50 @@ def backward_rows_head(q, k, v, W, dO, fw, p: Params, qrows, krows, lam=None, g_
 # Complexity accounting [ELSAA §6 and the appendix interaction-count example]
 # ----------------------------------------------------------------------------
 
+# ----------------------------------------------------------------------------
+# Rank view of sparse + low-rank attention [ELSAA §4]
+# ----------------------------------------------------------------------------
+
+def max_matching(mask: np.ndarray) -> int:
+    """Maximum matching size nu(Omega) of the bipartite graph with an edge (i, j) for
+    every True entry of ``mask`` (rows on one side, columns on the other); Kuhn's
+    augmenting paths, written out."""
+    n_r, n_c = mask.shape
+    adj = [np.flatnonzero(mask[i]) for i in range(n_r)]
+    match_col = -np.ones(n_c, dtype=np.int64)
+
+    def augment(i, seen):
+        for j in adj[i]:
+            if seen[j]:
+                continue
+            seen[j] = True
+            if match_col[j] < 0 or augment(match_col[j], seen):
+                match_col[j] = i
+                return True
+        return False
+
+    return sum(1 for i in range(n_r) if augment(i, np.zeros(n_c, dtype=bool)))
+
+
+def rank_diagnostic(q, k, idx, p: Params, r: int, seed: int = 0) -> dict:
+    """rank(S_Omega + B A) against min(n, nu(Omega) + r) [ELSAA §4 Theorem].
+
+    S_Omega = Omega * M*, M*_ij = exp(scale q_i . k_j), on the support the selector
+    realised (``idx``; causal rows keep j <= i); B [n, r] and A [r, n] are drawn from a
+    standard normal with ``seed`` (the theorem's absolutely continuous factors).  The
+    rank is numpy's SVD rank.  Returns n, nu, r, the rank and the predicted rank."""
+    q, k = _f64(q), _f64(k)
+    n = q.shape[0]
+    mask = np.zeros((n, n), dtype=bool)
+    for i, keys in enumerate(support(idx, p)):
+        mask[i, keys] = True
+    S = np.where(mask, np.exp(p.scale * (q @ k.T)), 0.0)
+    rng = np.random.default_rng(seed)
+    M = S + rng.standard_normal((n, r)) @ rng.standard_normal((r, n)) if r > 0 else S
+    nu = max_matching(mask)
+    return dict(n=n, nu=nu, r=r, rank=int(np.linalg.matrix_rank(M)), predicted=min(n, nu + r))
+
+
 def interaction_count(N: int, s: int, L_s: int, gamma: int) -> int:
     """Query-key interactions of ELSAA: N (s + L_s 2^gamma) [ELSAA §6]."""
     return N * (s + L_s * (1 << gamma))

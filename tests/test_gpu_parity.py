@@ -155,6 +155,23 @@ def test_fusion_parameter_gradients(geom, fixed_m, gates):
             assert np.all(err <= BF16_ABS_TOL + 2.0 ** -8 * bnd), f"{name}[{h}]: max err {err.max():.3e}"
 
 
+@pytest.mark.parametrize("causal,k,r", [(False, 1, 0), (False, 1, 24), (False, 2, 0), (True, 2, 16)])
+def test_rank_of_sparse_plus_low_rank_on_gpu_selection(causal, k, r):
+    """[ELSAA §4] rank(S_Omega + B A) = min(n, nu(Omega) + r) on the support the GPU selector
+    realised (elsaa_debug_select), evaluated in float64."""
+    w = small_workload(N=256, d=64, block_size=64, topk=k, rank_r=16, causal=causal, H=2)
+    inp = make_inputs(w, 3)
+    dev = device_inputs(w, inp)
+    op = gpu_op(w)
+    _, idx = op.debug_select(dev["Q"], dev["K"])
+    torch.cuda.synchronize()
+    p = oracle_params(w)
+    for h in range(w.H):
+        out = orc.rank_diagnostic(np64(inp["Q"][0, h]), np64(inp["K"][0, h]), idx[0, h].cpu().numpy(), p, r,
+                                  seed=h)
+        assert out["rank"] == out["predicted"], out
+
+
 @pytest.mark.parametrize("name", ["n2k_d64", "n8k_d64", "n16k_d128", "n64k_d128"])
 def test_selection_full_size(name):
     """Bit-exact against the oracle fed the GPU's float32 scores; against the

@@ -414,6 +414,41 @@ def test_fixed_m_adds_the_two_branch_outputs():
     assert np.all(both["m"] == 1.0)
 
 
+# --- rank view [ELSAA §4]: rank(S_Omega + B A) = min(n, nu(Omega) + r) ---
+
+def test_max_matching_against_brute_force():
+    """nu(Omega) equals the largest k for which some k rows can be matched to k
+    distinct columns, found by trying every injective assignment (n <= 6)."""
+    rng = np.random.default_rng(90)
+    for trial in range(60):
+        n_r, n_c = int(rng.integers(1, 6)), int(rng.integers(1, 6))
+        mask = rng.random((n_r, n_c)) < rng.uniform(0.1, 0.7)
+        exact = 0
+        for size in range(min(n_r, n_c), 0, -1):
+            if any(all(mask[i, j] for i, j in zip(rows, perm))
+                   for rows in itertools.combinations(range(n_r), size)
+                   for perm in itertools.permutations(range(n_c), size)):
+                exact = size
+                break
+        assert orc.max_matching(mask) == exact
+
+
+@pytest.mark.parametrize("causal,T,k,r", [(True, 4, 2, 0), (True, 4, 2, 8), (False, 8, 1, 16), (True, 8, 3, 32),
+                                          (False, 4, 16, 0)])
+def test_rank_of_sparse_plus_low_rank_matches_theorem(causal, T, k, r):
+    """On the supports the top-k block selector realises, rank(S_Omega + B A) equals
+    min(n, nu(Omega) + r); r = 0 gives the structural rank nu(Omega) itself, and a full
+    support (k = n_t, non-causal) gives n."""
+    n, d = 64, 16
+    q, kk = _rand((n, d), 91, 0.7), _rand((n, d), 92, 0.7)
+    p = _params(n, d, T, k, 16, causal)
+    idx = orc.select_from_scores(orc.block_scores(q, kk, p), p.topk, p.causal)
+    out = orc.rank_diagnostic(q, kk, idx, p, r, seed=93)
+    assert out["rank"] == out["predicted"], out
+    if not causal and k * T >= n:
+        assert out["nu"] == n
+
+
 # --- a value printed in the paper ---
 
 def test_interaction_count_matches_paper_example():
