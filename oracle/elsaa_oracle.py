@@ -57,6 +57,8 @@ class Params:
     tau: float = 1.0
     chunk: Optional[int] = None   # RACE causal chunk size; defaults to block_size
     fixed_m: bool = False    # ablation without denominator-aware fusion: m = 1, default g_lr = 1
+    selector: str = "topk"   # "topk" (blocks by pooled score) or "sortlsh" (non-causal, §3.2)
+    lsh_planes: Optional[np.ndarray] = None   # sortLSH hyperplanes [d, bits] (selector "sortlsh")
 
     @property
     def n_tables(self) -> int:
@@ -140,6 +142,68 @@ def support(idx: np.ndarray, p: Params) -> list:
                     keys.append(j)
         out.append(np.array(sorted(keys), dtype=np.int64))
     return out
+
+
+# ----------------------------------------------------------------------------
+# sortLSH selector [ELSAA §3.2]: queries and keys are hashed, sorted by hash value
+# and grouped into equal-size blocks; query block t attends exactly key block t.
+# Reading (the page has no pseudocode): angular LSH with the caller's hyperplanes
+# R [d, b], bit c of a row's code set when x . R_c > 0; rows are ordered by the
+# position of their code in the reflected Gray sequence (neighbouring buckets
+# differ in one bit), ties by row index.  Non-causal only.
+# ----------------------------------------------------------------------------
+
+def simhash_codes(X, R) -> np.ndarray:
+    """b-bit angular hash code of every row: bit c is [x . R_c > 0]."""
+    bits = (_f64(X) @ _f64(R)) > 0
+    return (bits.astype(np.int64) << np.arange(bits.shape[1])[None, :]).sum(axis=1)
+
+
+def gray_rank(code: np.ndarray) -> np.ndarray:
+    """Position of ``code`` in the reflected Gray sequence g(n) = n ^ (n >> 1): the
+    inverse map, n = code ^ (code >> 1) ^ (code >> 2) ^ ..."""
+    code = np.asarray(code, dtype=np.int64)
+    n = code.copy()
+    shift = code >> 1
+    while np.any(shift):
+        n ^= shift
+        shift >>= 1
+    return n
+
+
+def sortlsh_order(X, R) -> np.ndarray:
+    """Row indices in sorted order: by Gray position of the code, then by index."""
+    return np.argsort(gray_rank(simhash_codes(X, R)), kind="stable")
+
+
+def sortlsh_support(q, k, p: Params) -> list:
+    """Per query row i, the sorted key indices of the key block that shares its
+    position with i's query block in the two sorted orders."""
+    assert not p.causal, "the sortLSH selector here is the non-causal one"
+    T, N = p.block_size, p.N
+    oq, ok = sortlsh_order(q, p.lsh_planes), sortlsh_order(k, p.lsh_planes)
+    out = [None] * N
+    for t in range(p.n_tiles):
+        keys = np.sort(ok[t * T:(t + 1) * T])
+        for i in oq[t * T:(t + 1) * T]:
+            out[i] = keys
+    return out
+
+
+def sparse_from_support(q, k, v, sup, p: Params):
+    """O_s and log d_s row by row over an explicit support (list of key arrays)."""
+    N, d = q.shape
+    O_s = np.zeros((N, d))
+    logd = np.full(N, -np.inf)
+    for i, keys in enumerate(sup):
+        if keys.size == 0:
+            continue
+        z = p.scale * (k[keys] @ q[i])
+        mx = z.max()
+        e = np.exp(z - mx)
+        O_s[i] = e @ v[keys] / e.sum()
+        logd[i] = mx + np.log(e.sum())
+    return O_s, logd
 
 
 # ----------------------------------------------------------------------------
@@ -307,9 +371,13 @@ def forward_head(q, k, v, W, p: Params, lam=None, g_s=None, g_lr=None, scores=No
     timing sample).  Returns a dict with O, O_s, logd_s, O_lr, d_lr, m, idx, scores.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
-    sc = block_scores(q, k, p) if scores is None else _f64(scores)
-    idx = select_from_scores(sc, p.topk, p.causal)
-    O_s, logd = sparse_branch(q, k, v, idx, p, tiles)
+    if p.selector == "sortlsh":
+        sc = idx = None
+        O_s, logd = sparse_from_support(q, k, v, sortlsh_support(q, k, p), p)
+    else:
+        sc = block_scores(q, k, p) if scores is None else _f64(scores)
+        idx = select_from_scores(sc, p.topk, p.causal)
+        O_s, logd = sparse_branch(q, k, v, idx, p, tiles)
     O_lr, d_lr = race_branch(q, k, v, W, p)
     O, m = fuse(O_s, logd, O_lr, d_lr, p, lam, g_s, g_lr)
     return dict(O=O, O_s=O_s, logd_s=logd, O_lr=O_lr, d_lr=d_lr, m=m, idx=idx, scores=sc)
@@ -428,7 +496,15 @@ def backward_head(q, k, v, W, dO, fw, p: Params, lam=None, g_s=None, g_lr=None, 
     # Delta_i = <dO_s,i, O_s,i> - dd_s,i d_s,i
     Delta = (dOs * fw["O_s"]).sum(axis=1) - dds_ds
     tile_list = list(range(p.n_tiles)) if tiles is None else list(tiles)
-    for t in tile_list:
+    if p.selector == "sortlsh":
+        # the same chain rule row by row over each row's support
+        for i, keys in enumerate(sortlsh_support(q, k, p)):
+            P = np.exp(p.scale * (k[keys] @ q[i]) - fw["logd_s"][i])
+            dz = P * (v[keys] @ dOs[i] - Delta[i])
+            dq[i] += p.scale * dz @ k[keys]
+            dk[keys] += p.scale * np.outer(dz, q[i])
+            dv[keys] += np.outer(P, dOs[i])
+    for t in ([] if p.selector == "sortlsh" else tile_list):
         rows = np.arange(t * T, min(N, (t + 1) * T))
         keys = _tile_keys(fw["idx"][t], p)
         if keys.size == 0:

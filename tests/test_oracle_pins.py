@@ -326,9 +326,16 @@ def test_key_permutation_invariance_noncausal_block1():
 
 # --- backward: central finite differences ---
 
+def _selection(q, k, p, out):
+    """What the selector chose: the block indices, or both sortLSH orders."""
+    if p.selector == "sortlsh":
+        return np.concatenate([orc.sortlsh_order(q, p.lsh_planes), orc.sortlsh_order(k, p.lsh_planes)])
+    return out["idx"]
+
+
 def _loss(q, k, v, W, p, dO, lam=None, g_s=None, g_lr=None):
     out = orc.forward_head(q, k, v, W, p, lam, g_s, g_lr)
-    return float((out["O"] * dO).sum()), out["idx"]
+    return float((out["O"] * dO).sum()), _selection(q, k, p, out)
 
 
 @pytest.mark.parametrize("causal,gates,r,k,tau,fixed_m", [(True, False, 32, 2, 1.0, False),
@@ -337,10 +344,17 @@ def _loss(q, k, v, W, p, dO, lam=None, g_s=None, g_lr=None):
                                                           (True, False, 0, 2, 1.0, False),
                                                           (True, False, 32, 0, 0.8, False),
                                                           (True, False, 16, 2, 1.0, True),
-                                                          (False, True, 16, 2, 1.3, True)])
+                                                          (False, True, 16, 2, 1.3, True),
+                                                          (False, False, 16, "sortlsh", 1.0, False),
+                                                          (False, True, 0, "sortlsh", 0.9, False)])
 def test_backward_matches_finite_differences(causal, gates, r, k, tau, fixed_m):
     N, d, T = 24, 6, 4
-    q, k_, v, W, p = _setup(N=N, d=d, T=T, k=k, r=r, causal=causal, seed=50, lam=0.8, tau=tau, fixed_m=fixed_m)
+    lsh = k == "sortlsh"
+    q, k_, v, W, p = _setup(N=N, d=d, T=T, k=1 if lsh else k, r=r, causal=causal, seed=50, lam=0.8, tau=tau,
+                            fixed_m=fixed_m)
+    if lsh:
+        p.selector = "sortlsh"
+        p.lsh_planes = _rand((d, 3), 55)
     if r == 0:
         W = np.zeros((0, d, 4))
     dO = _rand((N, d), 60)
@@ -348,6 +362,7 @@ def test_backward_matches_finite_differences(causal, gates, r, k, tau, fixed_m):
     g_s = np.linspace(0.2, 1.0, N) if gates else None
     g_lr = np.linspace(1.0, 0.1, N) if gates else None
     fw = orc.forward_head(q, k_, v, W, p, lam, g_s, g_lr)
+    sel0 = _selection(q, k_, p, fw)
     dq, dk, dv = orc.backward_head(q, k_, v, W, dO, fw, p, lam, g_s, g_lr)
     h = 1e-6
     skipped = 0
@@ -360,7 +375,7 @@ def test_backward_matches_finite_differences(causal, gates, r, k, tau, fixed_m):
             X[idx] = old - h
             lm, im = _loss(q, k_, v, W, p, dO, lam, g_s, g_lr)
             X[idx] = old
-            if not (np.array_equal(ip, fw["idx"]) and np.array_equal(im, fw["idx"])):
+            if not (np.array_equal(ip, sel0) and np.array_equal(im, sel0)):
                 skipped += 1
                 fd[idx] = G[idx]
                 continue
@@ -412,6 +427,88 @@ def test_fixed_m_adds_the_two_branch_outputs():
     lowrank_only = orc.forward_head(q, k, v, W, p_l)["O"]
     np.testing.assert_allclose(both["O"], sparse_only + lowrank_only, rtol=0, atol=1e-12)
     assert np.all(both["m"] == 1.0)
+
+
+# --- sortLSH selector [ELSAA §3.2] ---
+
+def test_gray_rank_inverts_the_reflected_gray_code():
+    """gray_rank(n ^ (n >> 1)) = n for every n < 2^b, so neighbouring positions hold
+    codes one bit apart."""
+    for b in (1, 3, 8, 12):
+        n = np.arange(1 << b)
+        g = n ^ (n >> 1)
+        assert np.array_equal(orc.gray_rank(g), n)
+        flips = g[1:] ^ g[:-1]
+        assert np.all((flips & (flips - 1)) == 0) and np.all(flips > 0)
+
+
+def test_simhash_bit_agreement_is_one_minus_angle_over_pi():
+    """Per hyperplane, two rows hash alike with probability 1 - theta/pi (the angular
+    collision probability rho_ij of ELSAA §4), checked over 60000 Gaussian planes."""
+    rng = np.random.default_rng(95)
+    d = 16
+    for trial in range(4):
+        x, y = rng.standard_normal(d), rng.standard_normal(d)
+        R = rng.standard_normal((d, 60000))
+        agree = np.mean(((x @ R) > 0) == ((y @ R) > 0))
+        theta = math.acos(np.dot(x, y) / np.linalg.norm(x) / np.linalg.norm(y))
+        expect = 1 - theta / math.pi
+        assert abs(agree - expect) <= 4 * math.sqrt(expect * (1 - expect) / 60000) + 1e-9
+
+
+def _sortlsh_params(N, d, T, bits, seed, **kw):
+    p = _params(N, d, T, 1, 0, False, eps=0.0, **kw)
+    p.selector = "sortlsh"
+    p.lsh_planes = _rand((d, bits), seed)
+    return p
+
+
+def test_sortlsh_one_block_is_dense_softmax():
+    N, d = 40, 8
+    q, k, v = _rand((N, d), 96), _rand((N, d), 97), _rand((N, d), 98)
+    p = _sortlsh_params(N, d, N, 6, 99)
+    out = orc.forward_head(q, k, v, np.zeros((0, d, 4)), p)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[None], torch.tensor(k)[None], torch.tensor(v)[None], scale=p.scale)[0].numpy()
+    np.testing.assert_allclose(out["O"], ref, rtol=0, atol=1e-12)
+
+
+def test_sortlsh_with_equal_codes_is_block_diagonal_softmax():
+    """Zero hyperplanes give every row the same code, so both orders are the identity
+    and query block t attends key block t of the original order."""
+    N, d, T = 44, 8, 8
+    q, k, v = _rand((N, d), 100), _rand((N, d), 101), _rand((N, d), 102)
+    p = _sortlsh_params(N, d, T, 5, 103)
+    p.lsh_planes = np.zeros((d, 5))
+    out = orc.forward_head(q, k, v, np.zeros((0, d, 4)), p)
+    blk = np.arange(N) // T
+    mask = torch.tensor(blk[:, None] == blk[None, :])
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[None], torch.tensor(k)[None], torch.tensor(v)[None], attn_mask=mask[None],
+        scale=p.scale)[0].numpy()
+    np.testing.assert_allclose(out["O"], ref, rtol=0, atol=1e-12)
+
+
+def test_sortlsh_groups_rows_into_equal_blocks_of_similar_codes():
+    """Each key lands in exactly one block; each block (except a ragged last one) has T
+    queries and T keys; within the sorted order Gray positions never decrease and equal
+    codes keep their index order."""
+    N, d, T = 70, 8, 8
+    q, k = _rand((N, d), 104), _rand((N, d), 105)
+    p = _sortlsh_params(N, d, T, 4, 106)
+    sup = orc.sortlsh_support(q, k, p)
+    seen = np.zeros(N, dtype=int)
+    for t in range(p.n_tiles):
+        keys = sup[orc.sortlsh_order(q, p.lsh_planes)[t * T]]
+        seen[keys] += 1
+        assert keys.size == min(T, N - t * T)
+    assert np.all(seen == 1)
+    for X in (q, k):
+        order = orc.sortlsh_order(X, p.lsh_planes)
+        pos = orc.gray_rank(orc.simhash_codes(X, p.lsh_planes))[order]
+        assert np.all(np.diff(pos) >= 0)
+        same = np.diff(pos) == 0
+        assert np.all(np.diff(order)[same] > 0)
 
 
 # --- rank view [ELSAA §4]: rank(S_Omega + B A) = min(n, nu(Omega) + r) ---
