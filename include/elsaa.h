@@ -76,6 +76,15 @@ typedef enum {
 
 typedef enum { ELSAA_DTYPE_F32 = 0, ELSAA_DTYPE_BF16 = 1 } elsaa_dtype;
 
+/* Sparse-branch selector.  TOPK_BLOCKS: per query tile the top-k key blocks by
+ * mean-pooled logit (§3.3 Practical notes allow any important-key selector).
+ * SORTLSH: the paper's sortLSH (§3.2), non-causal: rows hashed with angular LSH
+ * (lsh_bits hyperplanes, bit c set when x . R_c > 0), sorted by the code's position
+ * in the reflected Gray sequence and then by row, grouped into blocks of block_size;
+ * query block t attends key block t exactly (topk is not used).  Needs causal = 0,
+ * N <= 16384 and block_size 64 or 128. */
+typedef enum { ELSAA_SEL_TOPK_BLOCKS = 0, ELSAA_SEL_SORTLSH = 1 } elsaa_selector;
+
 typedef struct {
   int32_t B, H, N, d;     /* batch, heads, sequence length, head dimension */
   int32_t dtype;          /* elsaa_dtype of Q, K, V, O, dO, dQ, dK, dV */
@@ -91,6 +100,9 @@ typedef struct {
   int32_t fixed_m;        /* 0: denominator-aware fusion (Eq. 5).  1: the paper's ablation without it
                              (Sort_Lsh_RACE, §6 "Attention variants"): m = 1 and g_lr defaults to 1,
                              so O = g_s O_s + g_lr O_lr.  Must match between forward and backward. */
+  int32_t selector;       /* elsaa_selector */
+  int32_t lsh_bits;       /* SORTLSH: hash bits b, 1..16 */
+  const float* lsh_planes;/* SORTLSH: device float32 [d, lsh_bits] hyperplanes R, caller-owned */
 } elsaa_params;
 
 /* Bytes of the caller-owned `saved` buffer the forward fills and the backward
@@ -146,6 +158,13 @@ ELSAA_API elsaa_status elsaa_fusion_grads(const elsaa_params* params, const floa
                                           const float* g_sparse, const float* g_lr, const void* dO,
                                           const void* saved, float* dlambda, float* dg_sparse, float* dg_lr,
                                           void* stream);
+
+/* sortLSH selector only: the hash code of every row and the two sorted orders, for
+ * inspection.  codes and order are int32 [B,H,2,N] (index 0: queries, 1: keys): codes
+ * hold the lsh_bits-bit hash, order[.., s, p] the row at sorted position p.  Needs no
+ * workspace; asynchronous on `stream`. */
+ELSAA_API elsaa_status elsaa_debug_sortlsh(const elsaa_params* params, const void* Q, const void* K,
+                                           int32_t* codes, int32_t* order, void* stream);
 
 /* Selection only: the float32 block scores the selector ranks and the chosen
  * blocks, for checking the selector against an external implementation.

@@ -59,6 +59,7 @@ class Params:
     fixed_m: bool = False    # ablation without denominator-aware fusion: m = 1, default g_lr = 1
     selector: str = "topk"   # "topk" (blocks by pooled score) or "sortlsh" (non-causal, §3.2)
     lsh_planes: Optional[np.ndarray] = None   # sortLSH hyperplanes [d, bits] (selector "sortlsh")
+    lsh_orders: Optional[tuple] = None        # sortLSH: externally decided (query, key) orders
 
     @property
     def n_tables(self) -> int:
@@ -181,7 +182,10 @@ def sortlsh_support(q, k, p: Params) -> list:
     position with i's query block in the two sorted orders."""
     assert not p.causal, "the sortLSH selector here is the non-causal one"
     T, N = p.block_size, p.N
-    oq, ok = sortlsh_order(q, p.lsh_planes), sortlsh_order(k, p.lsh_planes)
+    if p.lsh_orders is not None:      # orders decided elsewhere (the hash signs of another precision)
+        oq, ok = (np.asarray(o) for o in p.lsh_orders)
+    else:
+        oq, ok = sortlsh_order(q, p.lsh_planes), sortlsh_order(k, p.lsh_planes)
     out = [None] * N
     for t in range(p.n_tiles):
         keys = np.sort(ok[t * T:(t + 1) * T])

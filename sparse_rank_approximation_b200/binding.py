@@ -25,11 +25,13 @@ ELSAA_ERR_CUDA = 4
 ELSAA_ERR_TIMEOUT = 5
 ELSAA_DTYPE_F32 = 0
 ELSAA_DTYPE_BF16 = 1
+ELSAA_SEL_TOPK_BLOCKS = 0
+ELSAA_SEL_SORTLSH = 1
 
 EXPORTED = ("elsaa_saved_bytes", "elsaa_workspace_bytes", "elsaa_forward", "elsaa_backward",
             "elsaa_debug_select", "elsaa_check_device_flags", "elsaa_status_string",
             "elsaa_last_error_message", "elsaa_profile_begin", "elsaa_profile_end", "elsaa_select_noalloc",
-            "elsaa_fusion_grads")
+            "elsaa_fusion_grads", "elsaa_debug_sortlsh")
 
 
 class Params(ctypes.Structure):
@@ -37,7 +39,8 @@ class Params(ctypes.Structure):
                 ("dtype", ctypes.c_int32), ("causal", ctypes.c_int32), ("rank_r", ctypes.c_int32),
                 ("hash_bits", ctypes.c_int32), ("block_size", ctypes.c_int32), ("topk", ctypes.c_int32),
                 ("scale", ctypes.c_float), ("lam", ctypes.c_float), ("eps", ctypes.c_float),
-                ("tau", ctypes.c_float), ("fixed_m", ctypes.c_int32)]
+                ("tau", ctypes.c_float), ("fixed_m", ctypes.c_int32), ("selector", ctypes.c_int32),
+                ("lsh_bits", ctypes.c_int32), ("lsh_planes", ctypes.c_void_p)]
 
 
 class ElsaaError(RuntimeError):
@@ -84,6 +87,8 @@ def lib() -> ctypes.CDLL:
     L.elsaa_select_noalloc.restype = i32
     L.elsaa_fusion_grads.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.elsaa_fusion_grads.restype = i32
+    L.elsaa_debug_sortlsh.argtypes = [P, vp, vp, vp, vp, vp]
+    L.elsaa_debug_sortlsh.restype = i32
     _lib = L
     return L
 
@@ -96,10 +101,13 @@ def _check(status: int, where: str) -> None:
 
 
 def make_params(B, H, N, d, *, dtype=ELSAA_DTYPE_BF16, causal=True, rank_r=128, block_size=128, topk=16,
-                scale=None, lam=1.0, eps=1e-6, tau=1.0, hash_bits=4, fixed_m=False) -> Params:
+                scale=None, lam=1.0, eps=1e-6, tau=1.0, hash_bits=4, fixed_m=False, selector=ELSAA_SEL_TOPK_BLOCKS,
+                lsh_bits=0) -> Params:
+    """The plain-data parameter block.  For the sortLSH selector the hyperplanes are
+    attached by ``Elsaa(..., lsh_planes=...)``, which keeps them alive."""
     return Params(B, H, N, d, dtype, int(bool(causal)), rank_r, hash_bits, block_size, topk,
                   float(1.0 / math.sqrt(d) if scale is None else scale), float(lam), float(eps), float(tau),
-                  int(bool(fixed_m)))
+                  int(bool(fixed_m)), int(selector), int(lsh_bits), None)
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -125,9 +133,14 @@ class Elsaa:
     configured dtype (W: float32 [L, d, 4]; lam_vec/g_s/g_lr: float32 [B, H, N]).
     """
 
-    def __init__(self, params: Params, device: Optional[torch.device] = None):
+    def __init__(self, params: Params, device: Optional[torch.device] = None,
+                 lsh_planes: Optional[torch.Tensor] = None):
         self.p = params
         self.device = device or torch.device("cuda", torch.cuda.current_device())
+        # sortLSH hyperplanes: float32 [d, lsh_bits] on the device, kept alive with the op
+        self.lsh_planes = lsh_planes
+        if lsh_planes is not None:
+            self.p.lsh_planes = _ptr(lsh_planes)
         L = lib()
         self.saved_bytes = L.elsaa_saved_bytes(ctypes.byref(self.p))
         self.ws_fwd_bytes = L.elsaa_workspace_bytes(ctypes.byref(self.p), 0)
@@ -170,6 +183,16 @@ class Elsaa:
                                       _ptr(self.saved), _ptr(out[0]), _ptr(out[1]), _ptr(out[2]), _stream(stream))
         _check(st, "elsaa_fusion_grads")
         return tuple(out)
+
+    def debug_sortlsh(self, q, k, stream=None):
+        """sortLSH codes and sorted orders, int32 [B, H, 2, N] each (0: queries, 1: keys)."""
+        shape = (self.p.B, self.p.H, 2, self.p.N)
+        codes = torch.empty(shape, dtype=torch.int32, device=self.device)
+        order = torch.empty(shape, dtype=torch.int32, device=self.device)
+        st = lib().elsaa_debug_sortlsh(ctypes.byref(self.p), _ptr(q), _ptr(k), _ptr(codes), _ptr(order),
+                                       _stream(stream))
+        _check(st, "elsaa_debug_sortlsh")
+        return codes, order
 
     def debug_select(self, q, k, stream=None):
         n_t = -(-self.p.N // self.p.block_size)

@@ -113,14 +113,17 @@ __global__ void __launch_bounds__(256) fusion_grads_kernel(const E* __restrict__
                                                            const E* __restrict__ Olr_, const float* __restrict__ logd_,
                                                            const float* __restrict__ dlr_, const float* lamv,
                                                            const float* gsv, const float* glrv, float* dlam,
-                                                           float* dgs, float* dglr, Geom g) {
+                                                           float* dgs, float* dglr, const int* perm,
+                                                           int perm_stride, Geom g) {
   const int tpr = g.d / 8;
   const int rpb = 256 / tpr;
   const int sub = threadIdx.x % tpr;
   const int row = blockIdx.x * rpb + threadIdx.x / tpr;
-  const size_t i = (size_t)blockIdx.y * g.N + min(row, g.N - 1);
+  const size_t i = (size_t)blockIdx.y * g.N + min(row, g.N - 1);    // row of the saved state
+  // the caller's row: the same, or where the sortLSH order put this one
+  const size_t io = perm ? (size_t)blockIdx.y * g.N + perm[(size_t)blockIdx.y * perm_stride + min(row, g.N - 1)] : i;
   float dO[8], os[8], ol[8];
-  load8<E>(dO_ + i * g.d + sub * 8, dO);
+  load8<E>(dO_ + io * g.d + sub * 8, dO);
   load8<E>(Os_ + i * g.d + sub * 8, os);
   load8<E>(Olr_ + i * g.d + sub * 8, ol);
   float A = 0.f, Bv = 0.f;
@@ -135,29 +138,30 @@ __global__ void __launch_bounds__(256) fusion_grads_kernel(const E* __restrict__
   }
   if (sub != 0 || row >= g.N) return;
   const double dl = dlr_[i], ds = exp((double)logd_[i]);
-  const double lam = lamv ? lamv[i] : g.lam;
-  const double gs = gsv ? gsv[i] : 1.0;
+  const double lam = lamv ? lamv[io] : g.lam;
+  const double gs = gsv ? gsv[io] : 1.0;
   const double D = ds + lam * dl + (double)g.eps;
   const double m = g.fixed_m ? 1.0 : D > 0.0 ? ds / D : 0.0;
   const double dm = g.fixed_m ? 0.0 : gs * A - (glrv ? 0.0 : (double)Bv);
-  if (dlam) dlam[i] = (g.fixed_m || !(D > 0.0)) ? 0.f : (float)(-dm * ds * dl / (D * D));
-  if (dgs) dgs[i] = (float)(m * A);
-  if (dglr) dglr[i] = Bv;
+  if (dlam) dlam[io] = (g.fixed_m || !(D > 0.0)) ? 0.f : (float)(-dm * ds * dl / (D * D));
+  if (dgs) dgs[io] = (float)(m * A);
+  if (dglr) dglr[io] = Bv;
 }
 
 cudaError_t launch_fusion_grads(const void* dO, const void* Os, const void* Olr, const float* logd, const float* dlr,
                                 const float* lam, const float* gs, const float* glr, float* dlam, float* dgs,
-                                float* dglr, bool bf16, const Geom& g, cudaStream_t st) {
+                                float* dglr, const int* perm, int perm_stride, bool bf16, const Geom& g,
+                                cudaStream_t st) {
   const int rpb = 256 / (g.d / 8);
   dim3 grid((g.N + rpb - 1) / rpb, g.BH);
   ProfScope ps("fusion_grads", st);
   if (bf16)
     fusion_grads_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)dO, (const __nv_bfloat16*)Os,
                                                              (const __nv_bfloat16*)Olr, logd, dlr, lam, gs, glr,
-                                                             dlam, dgs, dglr, g);
+                                                             dlam, dgs, dglr, perm, perm_stride, g);
   else
     fusion_grads_kernel<float><<<grid, 256, 0, st>>>((const float*)dO, (const float*)Os, (const float*)Olr, logd, dlr,
-                                                     lam, gs, glr, dlam, dgs, dglr, g);
+                                                     lam, gs, glr, dlam, dgs, dglr, perm, perm_stride, g);
   return cudaGetLastError();
 }
 

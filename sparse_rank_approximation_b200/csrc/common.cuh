@@ -29,6 +29,8 @@ struct Geom {
   int dp;         // state columns: d value columns + 8 (column d holds the key mass)
   int causal;
   int fixed_m;    // fusion without the denominator-aware weight: m = 1, default g_lr = 1
+  int selector;   // 0: top-k key blocks; 1: sortLSH (the operator runs on row-permuted copies)
+  int lsh_bits;
   float scale, lam, eps, tau;
 };
 

@@ -86,7 +86,24 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
   }
   const int n_t = (p->N + T - 1) / T;
   if (n_t > 1024) { *st = fail(ELSAA_ERR_UNSUPPORTED, "ceil(N / block_size) = %d > 1024", n_t); return false; }
-  if (p->topk < 0 || p->topk > n_t) {
+  if (p->selector != ELSAA_SEL_TOPK_BLOCKS && p->selector != ELSAA_SEL_SORTLSH) {
+    *st = fail(ELSAA_ERR_INVALID_ARG, "selector %d is not an elsaa_selector", p->selector);
+    return false;
+  }
+  const bool lsh = p->selector == ELSAA_SEL_SORTLSH;
+  if (lsh) {
+    if (p->causal) {
+      *st = fail(ELSAA_ERR_UNSUPPORTED, "the sortLSH selector is non-causal (the causal recursion is not built)");
+      return false;
+    }
+    if (T == 1) { *st = fail(ELSAA_ERR_UNSUPPORTED, "sortLSH needs block_size 64 or 128"); return false; }
+    if (p->lsh_bits < 1 || p->lsh_bits > 16) {
+      *st = fail(ELSAA_ERR_INVALID_ARG, "lsh_bits %d outside [1, 16]", p->lsh_bits);
+      return false;
+    }
+    if (p->N > 16384) { *st = fail(ELSAA_ERR_UNSUPPORTED, "sortLSH sorts in shared memory: N <= 16384"); return false; }
+  }
+  if (!lsh && (p->topk < 0 || p->topk > n_t)) {
     *st = fail(ELSAA_ERR_INVALID_ARG, "topk %d outside [0, %d]", p->topk, n_t);
     return false;
   }
@@ -95,7 +112,7 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
   g->d = p->d;
   g->T = T;
   g->n_t = n_t;
-  g->k = p->topk;
+  g->k = lsh ? 1 : p->topk;     // sortLSH: tile t selects block t of the sorted orders
   g->r = p->rank_r;
   g->L = p->rank_r >> kHashBits;
   g->C = bf16 ? T : 64;
@@ -106,6 +123,8 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
   g->dp = p->d + 8;
   g->causal = p->causal;
   g->fixed_m = p->fixed_m != 0;
+  g->selector = p->selector;
+  g->lsh_bits = lsh ? p->lsh_bits : 0;
   g->scale = p->scale;
   g->lam = p->lambda;
   g->eps = p->eps;
@@ -122,6 +141,7 @@ struct Saved {
   float *Ast, *Bst;
   void* Psplit;
   float* Pmass;
+  int* lsh_order;          // sortLSH: sorted query and key orders [BH][2][N]
 };
 
 Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
@@ -146,8 +166,34 @@ Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
   const bool split = esz == 2 && g.r > 0 && race_bwd_tc_supported(g);
   s.Psplit = split ? c.take<char>((size_t)g.BH * g.n_c * 2 * g.r * g.d * 2) : nullptr;
   s.Pmass = split ? c.take<float>((size_t)g.BH * g.n_c * g.r) : nullptr;
+  s.lsh_order = g.selector == ELSAA_SEL_SORTLSH ? c.take<int>((size_t)g.BH * 2 * g.N) : nullptr;
   *bytes = align_up(c.off);
   return s;
+}
+
+// sortLSH: row-permuted copies of the inputs and outputs (the operator runs on them).
+struct PermBufs {
+  void *Q, *K, *V, *X, *dQ, *dK, *dV;     // X: O (forward) or dO (backward)
+  float *lam, *gs, *glr;
+};
+
+PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
+  PermBufs b{};
+  if (g.selector != ELSAA_SEL_SORTLSH) return b;
+  const size_t rows = (size_t)g.BH * g.N, mat = rows * g.d * esz;
+  b.Q = c.take<char>(mat);
+  b.K = c.take<char>(mat);
+  b.V = c.take<char>(mat);
+  b.X = c.take<char>(mat);
+  if (backward) {
+    b.dQ = c.take<char>(mat);
+    b.dK = c.take<char>(mat);
+    b.dV = c.take<char>(mat);
+  }
+  b.lam = c.take<float>(rows);
+  b.gs = c.take<float>(rows);
+  b.glr = c.take<float>(rows);
+  return b;
 }
 
 struct FwdWs {
@@ -155,9 +201,10 @@ struct FwdWs {
   double *qbar, *kbar;
   float* scores;
   void* wsplit;
+  PermBufs pm;
 };
 
-FwdWs carve_fwd_ws(void* base, const Geom& g, size_t* bytes) {
+FwdWs carve_fwd_ws(void* base, const Geom& g, size_t esz, size_t* bytes) {
   Carver c(base);
   FwdWs w;
   w.flag = c.take<uint32_t>(64);
@@ -165,6 +212,7 @@ FwdWs carve_fwd_ws(void* base, const Geom& g, size_t* bytes) {
   w.kbar = c.take<double>((size_t)g.BH * g.n_t * g.d);
   w.scores = c.take<float>((size_t)g.BH * g.n_t * g.n_t);
   w.wsplit = c.take<char>((size_t)2 * ((g.L * kHashBits + 15) & ~15) * g.d * 2);
+  w.pm = carve_perm(c, g, esz, false);
   *bytes = align_up(c.off);
   return w;
 }
@@ -178,6 +226,7 @@ struct BwdWs {
   void* dOcl;
   void *Rsplit, *Wsplit;
   float* Rmass;
+  PermBufs pm;
 };
 
 BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
@@ -205,6 +254,7 @@ BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
   w.Rsplit = split ? c.take<char>((size_t)g.BH * g.n_c * 2 * g.r * g.d * 2) : nullptr;
   w.Rmass = split ? c.take<float>((size_t)g.BH * g.n_c * g.r) : nullptr;
   w.Wsplit = split ? c.take<char>((size_t)2 * ((g.L * kHashBits + 15) & ~15) * g.d * 2) : nullptr;
+  w.pm = carve_perm(c, g, bf16 ? 2 : 4, true);
   *bytes = align_up(c.off);
   return w;
 }
@@ -279,6 +329,27 @@ ProfScope::~ProfScope() {
 }
 }  // namespace elsaa
 
+// sortLSH: sort the rows, then gather the inputs into the sorted orders (queries by the
+// query order, keys and values by the key order, per-row vectors by the query order).
+elsaa_status lsh_gather(const elsaa_params* p, const Geom& g, bool bf16, const int* order, bool sort_first,
+                        const void* Q, const void* K, const void* V, const void* X, const float* lam,
+                        const float* gs, const float* glr, const PermBufs& b, cudaStream_t st) {
+  const int row_bytes = g.d * (bf16 ? 2 : 4), stride = 2 * g.N;
+  const int* oq = order;
+  const int* ok = order + g.N;
+  if (sort_first)
+    ELSAA_TRY(cuda_status(launch_sortlsh_order(Q, K, bf16, p->lsh_planes, p->lsh_bits, const_cast<int*>(order),
+                                               nullptr, g, st), "sortLSH order"));
+  ELSAA_TRY(cuda_status(launch_permute_rows(Q, b.Q, oq, row_bytes, g, stride, false, st), "sortLSH gather Q"));
+  ELSAA_TRY(cuda_status(launch_permute_rows(K, b.K, ok, row_bytes, g, stride, false, st), "sortLSH gather K"));
+  ELSAA_TRY(cuda_status(launch_permute_rows(V, b.V, ok, row_bytes, g, stride, false, st), "sortLSH gather V"));
+  if (X) ELSAA_TRY(cuda_status(launch_permute_rows(X, b.X, oq, row_bytes, g, stride, false, st), "sortLSH gather dO"));
+  if (lam) ELSAA_TRY(cuda_status(launch_gather_vec(lam, b.lam, oq, g, stride, st), "sortLSH gather lambda"));
+  if (gs) ELSAA_TRY(cuda_status(launch_gather_vec(gs, b.gs, oq, g, stride, st), "sortLSH gather g_sparse"));
+  if (glr) ELSAA_TRY(cuda_status(launch_gather_vec(glr, b.glr, oq, g, stride, st), "sortLSH gather g_lr"));
+  return ELSAA_OK;
+}
+
 extern "C" {
 
 elsaa_status elsaa_profile_begin(void) {
@@ -339,7 +410,7 @@ size_t elsaa_workspace_bytes(const elsaa_params* p, int for_backward) {
   if (!make_geom(p, &g, &st)) return 0;
   size_t bytes = 0;
   if (for_backward) carve_bwd_ws(nullptr, g, p->dtype == ELSAA_DTYPE_BF16, &bytes);
-  else carve_fwd_ws(nullptr, g, &bytes);
+  else carve_fwd_ws(nullptr, g, p->dtype == ELSAA_DTYPE_BF16 ? 2 : 4, &bytes);
   return bytes;
 }
 
@@ -362,14 +433,29 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
   ELSAA_TRY(check_ptr(glr, "g_lr", false));
   const bool bf16 = p->dtype == ELSAA_DTYPE_BF16;
   size_t need = 0;
-  FwdWs w = carve_fwd_ws(workspace, g, &need);
+  FwdWs w = carve_fwd_ws(workspace, g, bf16 ? 2 : 4, &need);
   if (ws_bytes < need) return fail(ELSAA_ERR_WORKSPACE, "workspace %zu bytes < %zu required", ws_bytes, need);
   size_t sb = 0;
   Saved s = carve_saved(saved, g, bf16 ? 2 : 4, &sb);
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  const bool lsh = g.selector == ELSAA_SEL_SORTLSH;
+  void* O_out = O;
+  if (lsh) {
+    // the operator runs on the sorted rows (non-causal RACE, the fusion and diagonal-block
+    // attention commute with row permutations); O is scattered back at the end
+    ELSAA_TRY(check_ptr(p->lsh_planes, "lsh_planes"));
+    ELSAA_TRY(lsh_gather(p, g, bf16, s.lsh_order, true, Q, K, V, nullptr, lam, gs, glr, w.pm, st_));
+    Q = w.pm.Q; K = w.pm.K; V = w.pm.V; O = w.pm.X;
+    if (lam) lam = w.pm.lam;
+    if (gs) gs = w.pm.gs;
+    if (glr) glr = w.pm.glr;
+  }
 
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st_), "flag reset"));
-  ELSAA_TRY(cuda_status(launch_select(Q, K, bf16, w.qbar, w.kbar, w.scores, s.idx, g, st_), "selection"));
+  if (lsh)
+    ELSAA_TRY(cuda_status(launch_diag_select(s.idx, g, st_), "selection"));
+  else
+    ELSAA_TRY(cuda_status(launch_select(Q, K, bf16, w.qbar, w.kbar, w.scores, s.idx, g, st_), "selection"));
   ELSAA_TRY(cuda_status(launch_race_features(Q, K, W, w.wsplit, bf16, s.phiQ, s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, st_),
                         "race features"));
   ELSAA_TRY(cuda_status(launch_race_state_fwd(s.phiK, V, bf16, s.Ast, s.Bst, g, st_), "race summaries"));
@@ -389,6 +475,9 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
   } else {
     ELSAA_TRY(cuda_status(launch_attn_fwd_f32(a, g, st_), "fused forward"));
   }
+  if (lsh)
+    ELSAA_TRY(cuda_status(launch_permute_rows(O, O_out, s.lsh_order, g.d * (bf16 ? 2 : 4), g, 2 * g.N, true, st_),
+                          "sortLSH scatter O"));
   return ELSAA_OK;
 }
 
@@ -420,6 +509,18 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   size_t sb = 0;
   Saved s = carve_saved(const_cast<void*>(saved), g, bf16 ? 2 : 4, &sb);
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  const bool lsh = g.selector == ELSAA_SEL_SORTLSH;
+  void *dQ_out = dQ, *dK_out = dK, *dV_out = dV;
+  if (lsh) {
+    // the forward ran on the sorted rows and saved its state in that order; so does this,
+    // and the gradients are scattered back at the end
+    ELSAA_TRY(lsh_gather(p, g, bf16, s.lsh_order, false, Q, K, V, dO, lam, gs, glr, w.pm, st_));
+    Q = w.pm.Q; K = w.pm.K; V = w.pm.V; dO = w.pm.X;
+    dQ = w.pm.dQ; dK = w.pm.dK; dV = w.pm.dV;
+    if (lam) lam = w.pm.lam;
+    if (gs) gs = w.pm.gs;
+    if (glr) glr = w.pm.glr;
+  }
   BwdArgs a{};
   a.Q = Q; a.K = K; a.V = V; a.dO = dO; a.W = W;
   a.lam = lam; a.gs = gs; a.glr = glr;
@@ -456,6 +557,14 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   } else {
     ELSAA_TRY(cuda_status(launch_bwd_f32(a, g, st_), "backward"));
   }
+  if (lsh) {
+    const int rb = g.d * (bf16 ? 2 : 4);
+    ELSAA_TRY(cuda_status(launch_permute_rows(dQ, dQ_out, s.lsh_order, rb, g, 2 * g.N, true, st_), "sortLSH dQ"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(dK, dK_out, s.lsh_order + g.N, rb, g, 2 * g.N, true, st_),
+                          "sortLSH dK"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(dV, dV_out, s.lsh_order + g.N, rb, g, 2 * g.N, true, st_),
+                          "sortLSH dV"));
+  }
   return ELSAA_OK;
 }
 
@@ -478,8 +587,9 @@ elsaa_status elsaa_fusion_grads(const elsaa_params* p, const float* lam, const f
   size_t sb = 0;
   Saved s = carve_saved(const_cast<void*>(saved), g, bf16 ? 2 : 4, &sb);
   if (!dlam && !dgs && !dglr) return ELSAA_OK;
-  return cuda_status(launch_fusion_grads(dO, s.Os, s.Olr, s.logd, s.dlr, lam, gs, glr, dlam, dgs, dglr, bf16, g,
-                                         static_cast<cudaStream_t>(stream)),
+  // sortLSH: the saved state is in the sorted query order; each row maps back through it
+  return cuda_status(launch_fusion_grads(dO, s.Os, s.Olr, s.logd, s.dlr, lam, gs, glr, dlam, dgs, dglr, s.lsh_order,
+                                         2 * g.N, bf16, g, static_cast<cudaStream_t>(stream)),
                      "fusion gradients");
 }
 
@@ -489,17 +599,36 @@ elsaa_status elsaa_debug_select(const elsaa_params* p, const void* Q, const void
   Geom g;
   elsaa_status st;
   if (!make_geom(p, &g, &st)) return st;
+  if (g.selector != ELSAA_SEL_TOPK_BLOCKS)
+    return fail(ELSAA_ERR_UNSUPPORTED, "elsaa_debug_select is for the top-k selector (see elsaa_debug_sortlsh)");
   ELSAA_TRY(check_ptr(Q, "Q"));
   ELSAA_TRY(check_ptr(K, "K"));
   ELSAA_TRY(check_ptr(scores, "scores"));
   ELSAA_TRY(check_ptr(idx, "idx", g.k > 0));
   ELSAA_TRY(check_ptr(workspace, "workspace"));
   size_t need = 0;
-  FwdWs w = carve_fwd_ws(workspace, g, &need);
+  FwdWs w = carve_fwd_ws(workspace, g, p->dtype == ELSAA_DTYPE_BF16 ? 2 : 4, &need);
   if (ws_bytes < need) return fail(ELSAA_ERR_WORKSPACE, "workspace %zu bytes < %zu required", ws_bytes, need);
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
   return cuda_status(launch_select(Q, K, p->dtype == ELSAA_DTYPE_BF16, w.qbar, w.kbar, scores, idx, g, st_),
                      "selection");
+}
+
+elsaa_status elsaa_debug_sortlsh(const elsaa_params* p, const void* Q, const void* K, int32_t* codes,
+                                 int32_t* order, void* stream) {
+  g_last_error.clear();
+  Geom g;
+  elsaa_status st;
+  if (!make_geom(p, &g, &st)) return st;
+  if (g.selector != ELSAA_SEL_SORTLSH) return fail(ELSAA_ERR_INVALID_ARG, "params.selector is not ELSAA_SEL_SORTLSH");
+  ELSAA_TRY(check_ptr(Q, "Q"));
+  ELSAA_TRY(check_ptr(K, "K"));
+  ELSAA_TRY(check_ptr(p->lsh_planes, "lsh_planes"));
+  ELSAA_TRY(check_ptr(order, "order"));
+  ELSAA_TRY(check_ptr(codes, "codes", false));
+  return cuda_status(launch_sortlsh_order(Q, K, p->dtype == ELSAA_DTYPE_BF16, p->lsh_planes, p->lsh_bits, order,
+                                          codes, g, static_cast<cudaStream_t>(stream)),
+                     "sortLSH order");
 }
 
 elsaa_status elsaa_check_device_flags(void* workspace, void* stream) {

@@ -61,6 +61,20 @@ struct BwdArgs {
   void *dQ, *dK, *dV;
 };
 
+// sortLSH selector: per head the sorted query and key orders, int32 [BH][2][N]
+// (codes, if not null, receive the hash codes in the same layout).
+cudaError_t launch_sortlsh_order(const void* Q, const void* K, bool bf16, const float* planes, int bits,
+                                 int* order, int* codes, const Geom& g, cudaStream_t st);
+size_t sortlsh_smem_bytes(const Geom& g, int bits);
+// Row permutation of [BH][N] rows of row_bytes (a multiple of 16): gather dst[r] = src[perm[r]]
+// or scatter dst[perm[r]] = src[r]; perm advances by perm_stride per head.
+cudaError_t launch_permute_rows(const void* src, void* dst, const int* perm, int row_bytes, const Geom& g,
+                                int perm_stride, bool scatter, cudaStream_t st);
+cudaError_t launch_gather_vec(const float* src, float* dst, const int* perm, const Geom& g, int perm_stride,
+                              cudaStream_t st);
+// idx[t] = {t, -1, ...}: tile t selects block t.
+cudaError_t launch_diag_select(int* idx, const Geom& g, cudaStream_t st);
+
 // Sets the message elsaa_last_error_message() returns on this thread.
 void record_error(const char* msg);
 
@@ -94,9 +108,12 @@ cudaError_t launch_race_readout_tc(const FwdArgs& a, const Geom& g, uint32_t* er
 cudaError_t launch_attn_fwd_f32(const FwdArgs& a, const Geom& g, cudaStream_t st);
 cudaError_t launch_row_scalars(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st);
 // Per-row gradients of the fusion parameters lambda, g_s, g_lr (any output may be null).
+// With perm (sortLSH), row r of the saved state belongs to input row perm[r] (stride
+// perm_stride per head): dO, lambda and the gates are read there and the results written there.
 cudaError_t launch_fusion_grads(const void* dO, const void* Os, const void* Olr, const float* logd, const float* dlr,
                                 const float* lam, const float* gs, const float* glr, float* dlam, float* dgs,
-                                float* dglr, bool bf16, const Geom& g, cudaStream_t st);
+                                float* dglr, const int* perm, int perm_stride, bool bf16, const Geom& g,
+                                cudaStream_t st);
 // RACE backward (bf16): low-rank parts of dQ, dK, dV into the fp32 accumulators.
 cudaError_t launch_race_bwd_bf16(const BwdArgs& a, const Geom& g, cudaStream_t st);
 // tcgen05 sparse-branch backward (d = 128, block 128): dQ (query-major) and dK/dV

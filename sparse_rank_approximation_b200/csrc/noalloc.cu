@@ -48,6 +48,8 @@ elsaa_status elsaa_select_noalloc(const elsaa_params* p, const void* Q, const vo
   // The size query validates the parameters without touching the GPU.
   if (elsaa_workspace_bytes(p, 0) == 0)
     return noalloc_fail(ELSAA_ERR_INVALID_ARG, std::string("invalid params: ") + elsaa_last_error_message());
+  if (p->selector != ELSAA_SEL_TOPK_BLOCKS)
+    return noalloc_fail(ELSAA_ERR_UNSUPPORTED, "elsaa_select_noalloc is the top-k block selection");
   if (!Q || !K || (p->topk > 0 && !idx)) return noalloc_fail(ELSAA_ERR_INVALID_ARG, "Q, K or idx is NULL");
   if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(idx)) & 15u)
     return noalloc_fail(ELSAA_ERR_INVALID_ARG, "Q, K and idx must be 16-byte aligned");

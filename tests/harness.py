@@ -57,3 +57,28 @@ def check(w: Workload, name: str, gpu: np.ndarray, ref: np.ndarray):
     assert excess <= BF16_ABS_TOL, (f"{name}: max abs err {err:.3e}, beyond bf16 storage {excess:.3e} > "
                                     f"{BF16_ABS_TOL} (max |ref| {np.abs(ref).max():.3f})")
     return err
+
+
+def check_fusion_grads(w: Workload, h: int, p: orc.Params, fw: dict, ex: dict, dO_h: np.ndarray, got, ref):
+    """elsaa_fusion_grads outputs (dlambda, dg_s, dg_lr) of head h against the oracle's.
+
+    float32: the usual relative bound.  bf16: the GPU reduces over the saved bf16 O_s and
+    O_lr, each element within half an ulp (2^-9 relative) of the exact value, so row i's
+    dot product is off by at most 2^-9 sum_k |dO_ik O_ik|; the bound doubles that, carries
+    it through d m / d lambda, and adds the usual 2e-2.
+    """
+    if w.dtype == "f32":
+        for name, g, want in zip(("dlambda", "dg_s", "dg_lr"), got, ref):
+            check(w, f"{name}[{h}]", np64(g[0, h]), want)
+        return
+    sa = np.abs(dO_h * fw["O_s"]).sum(axis=1)
+    sb = np.abs(dO_h * fw["O_lr"]).sum(axis=1)
+    gs = ex.get("g_s", np.ones(w.N))
+    ds = np.exp(fw["logd_s"])
+    lam = ex.get("lam", np.full(w.N, p.lam))
+    D = ds + lam * fw["d_lr"] + p.eps
+    dm_bound = gs * sa + (0.0 if "g_lr" in ex else sb)
+    bounds = (np.where(p.fixed_m, 0.0, ds * fw["d_lr"] / D ** 2 * dm_bound), fw["m"] * sa, sb)
+    for name, g, want, bnd in zip(("dlambda", "dg_s", "dg_lr"), got, ref, bounds):
+        err = np.abs(np64(g[0, h]) - want)
+        assert np.all(err <= BF16_ABS_TOL + 2.0 ** -8 * bnd), f"{name}[{h}]: max err {err.max():.3e}"

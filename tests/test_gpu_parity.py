@@ -10,7 +10,7 @@ import torch
 
 from oracle import elsaa_oracle as orc
 from sparse_rank_approximation_b200.workloads import WORKLOADS, make_inputs, small_workload
-from tests.harness import BF16_ABS_TOL, check, device_inputs, gpu_op, np64, oracle_params
+from tests.harness import check, check_fusion_grads, device_inputs, gpu_op, np64, oracle_params
 
 pytestmark = pytest.mark.gpu
 
@@ -135,24 +135,7 @@ def test_fusion_parameter_gradients(geom, fixed_m, gates):
         ex = {k: v[0, h].double().numpy() for k, v in extra.items()}
         dO_h = inp["dO"][0, h].double().numpy()
         ref = orc.fusion_param_grads(dO_h, fw, p, ex.get("lam"), ex.get("g_s"), ex.get("g_lr"))
-        if w.dtype == "f32":
-            for name, got, want in zip(("dlambda", "dg_s", "dg_lr"), (dl, dgs, dgl), ref):
-                check(w, f"{name}[{h}]", np64(got[0, h]), want)
-            continue
-        # bf16: the GPU reduces over the saved bf16 O_s and O_lr, each element within half an
-        # ulp (2^-9 relative) of the exact value, so row i's dot product is off by at most
-        # 2^-9 sum_k |dO_ik O_ik|; the bound below doubles that and adds the usual 2e-2.
-        sa = np.abs(dO_h * fw["O_s"]).sum(axis=1)
-        sb = np.abs(dO_h * fw["O_lr"]).sum(axis=1)
-        gs = ex.get("g_s", np.ones(w.N))
-        ds = np.exp(fw["logd_s"])
-        lam = ex["lam"]
-        D = ds + lam * fw["d_lr"] + p.eps
-        dm_bound = gs * sa + (0.0 if "g_lr" in ex else sb)
-        bounds = (np.where(fixed_m, 0.0, ds * fw["d_lr"] / D ** 2 * dm_bound), fw["m"] * sa, sb)
-        for name, got, want, bnd in zip(("dlambda", "dg_s", "dg_lr"), (dl, dgs, dgl), ref, bounds):
-            err = np.abs(np64(got[0, h]) - want)
-            assert np.all(err <= BF16_ABS_TOL + 2.0 ** -8 * bnd), f"{name}[{h}]: max err {err.max():.3e}"
+        check_fusion_grads(w, h, p, fw, ex, dO_h, (dl, dgs, dgl), ref)
 
 
 @pytest.mark.parametrize("causal,k,r", [(False, 1, 0), (False, 1, 24), (False, 2, 0), (True, 2, 16)])

@@ -1,0 +1,113 @@
+"""sortLSH selector [ELSAA §3.2] through the C ABI against the float64 oracle.
+
+The hash codes are compared bit for bit (a mismatch is allowed only where a projection
+is within float32 rounding of zero); the outputs and gradients are compared with the
+oracle run on the same sorted orders, for the tensor-core, mma.sync and float32 paths.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import elsaa_oracle as orc
+from sparse_rank_approximation_b200 import binding as bd
+from sparse_rank_approximation_b200.workloads import make_inputs, small_workload
+from tests.harness import check, check_fusion_grads, device_inputs, np64, oracle_params
+
+pytestmark = pytest.mark.gpu
+
+GEOMS = {
+    "bf16_d128_T128_r128": dict(N=128 * 4 + 44, d=128, block_size=128, rank_r=128, dtype="bf16"),
+    "bf16_d64_T64_r32": dict(N=64 * 5 + 11, d=64, block_size=64, rank_r=32, dtype="bf16"),
+    "f32_d64_T64_r16": dict(N=64 * 3 + 20, d=64, block_size=64, rank_r=16, dtype="f32"),
+}
+
+
+def _setup(geom, bits, seed=0, fixed_m=False):
+    w = small_workload(topk=1, causal=False, H=2, **GEOMS[geom])
+    inp = make_inputs(w, seed)
+    dev = device_inputs(w, inp)
+    g = torch.Generator().manual_seed(seed + 7)
+    R = torch.randn(w.d, bits, generator=g)
+    p = bd.make_params(w.B, w.H, w.N, w.d, dtype=bd.ELSAA_DTYPE_BF16 if w.dtype == "bf16" else bd.ELSAA_DTYPE_F32,
+                       causal=False, rank_r=w.rank_r, block_size=w.block_size, topk=1, scale=w.scale,
+                       fixed_m=fixed_m, selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=bits)
+    op = bd.Elsaa(p, torch.device("cuda", 0), lsh_planes=R.cuda())
+    return w, inp, dev, R, op
+
+
+def _oracle_params(w, R, orders, fixed_m=False):
+    p = oracle_params(w, fixed_m=fixed_m)
+    p.selector = "sortlsh"
+    p.lsh_planes = R.double().numpy()
+    p.lsh_orders = orders
+    return p
+
+
+@pytest.mark.parametrize("geom", list(GEOMS))
+@pytest.mark.parametrize("bits", [4, 9])
+def test_codes_and_orders(geom, bits):
+    w, inp, dev, R, op = _setup(geom, bits)
+    codes, order = op.debug_sortlsh(dev["Q"], dev["K"])
+    torch.cuda.synchronize()
+    Rn = R.double().numpy()
+    for h in range(w.H):
+        for side, name in ((0, "Q"), (1, "K")):
+            X = inp[name][0, h].double().numpy()
+            ref = orc.simhash_codes(X, Rn)
+            got = codes[0, h, side].cpu().numpy()
+            proj = X @ Rn
+            near = np.abs(proj) <= 1e-5 * np.linalg.norm(X, axis=1)[:, None] * np.linalg.norm(Rn, axis=0)[None, :]
+            diff = (got ^ ref)[:, None] >> np.arange(bits)[None, :] & 1
+            assert not np.any(diff.astype(bool) & ~near), f"{name}[{h}]: code bits differ away from zero"
+            if np.array_equal(got, ref):
+                assert np.array_equal(order[0, h, side].cpu().numpy(), orc.sortlsh_order(X, Rn))
+            # the order is a permutation sorted by Gray position of the GPU's own codes, ties by row
+            o = order[0, h, side].cpu().numpy()
+            assert np.array_equal(np.sort(o), np.arange(w.N))
+            pos = orc.gray_rank(got)[o]
+            assert np.all(np.diff(pos) >= 0) and np.all(np.diff(o)[np.diff(pos) == 0] > 0)
+
+
+@pytest.mark.parametrize("geom", list(GEOMS))
+@pytest.mark.parametrize("gates,fixed_m", [(False, False), (True, False), (True, True)])
+def test_forward_backward(geom, gates, fixed_m):
+    w, inp, dev, R, op = _setup(geom, 6, seed=1, fixed_m=fixed_m)
+    BH = (w.B, w.H, w.N)
+    g = torch.Generator().manual_seed(11)
+    extra = {}
+    if gates:
+        extra = {"lam": torch.rand(BH, generator=g) * 2.0, "g_s": torch.rand(BH, generator=g),
+                 "g_lr": torch.rand(BH, generator=g)}
+    ex_dev = {k: v.cuda() for k, v in extra.items()}
+    O = op.forward(dev["Q"], dev["K"], dev["V"], dev["W"], ex_dev.get("lam"), ex_dev.get("g_s"), ex_dev.get("g_lr"))
+    dQ, dK, dV = op.backward(dev["Q"], dev["K"], dev["V"], dev["W"], dev["dO"], ex_dev.get("lam"),
+                             ex_dev.get("g_s"), ex_dev.get("g_lr"))
+    dl, dgs, dgl = op.fusion_grads(dev["dO"], ex_dev.get("lam"), ex_dev.get("g_s"), ex_dev.get("g_lr"))
+    _, order = op.debug_sortlsh(dev["Q"], dev["K"])
+    torch.cuda.synchronize()
+    W = inp["W"].double().numpy()
+    for h in range(w.H):
+        orders = (order[0, h, 0].cpu().numpy(), order[0, h, 1].cpu().numpy())
+        p = _oracle_params(w, R, orders, fixed_m)
+        get = lambda n: inp[n][0, h].double().numpy()
+        ex = {k: v[0, h].double().numpy() for k, v in extra.items()}
+        fw = orc.forward_head(get("Q"), get("K"), get("V"), W, p, ex.get("lam"), ex.get("g_s"), ex.get("g_lr"))
+        dq, dk, dv = orc.backward_head(get("Q"), get("K"), get("V"), W, get("dO"), fw, p, ex.get("lam"),
+                                       ex.get("g_s"), ex.get("g_lr"))
+        check(w, f"O[{h}]", np64(O[0, h]), fw["O"])
+        check(w, f"dQ[{h}]", np64(dQ[0, h]), dq)
+        check(w, f"dK[{h}]", np64(dK[0, h]), dk)
+        check(w, f"dV[{h}]", np64(dV[0, h]), dv)
+        ref = orc.fusion_param_grads(get("dO"), fw, p, ex.get("lam"), ex.get("g_s"), ex.get("g_lr"))
+        check_fusion_grads(w, h, p, fw, ex, get("dO"), (dl, dgs, dgl), ref)
+
+
+def test_rejects_causal_and_oversize():
+    L = bd.lib()
+    import ctypes
+    p = bd.make_params(1, 1, 512, 64, block_size=64, topk=1, rank_r=16, causal=True,
+                       selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=8)
+    assert L.elsaa_saved_bytes(ctypes.byref(p)) == 0
+    p = bd.make_params(1, 1, 32768, 64, block_size=64, topk=1, rank_r=16, causal=False,
+                       selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=8)
+    assert L.elsaa_saved_bytes(ctypes.byref(p)) == 0
