@@ -103,6 +103,12 @@ def work_model(w):
     m["race_state_fwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)
     m["race_state_bwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)
     m["race_features"] = dict(flops=2 * 2 * BH * N * d * 4 * L * 2, bytes=2 * BH * N * (d + r) * 2)
+    if w.selector == "sortlsh":
+        esz = 2 if w.dtype == "bf16" else 4
+        mat = BH * N * d * esz
+        m["sortlsh_order"] = dict(flops=0, bytes=2 * mat + 2 * BH * N * 4)   # Q, K read; orders written
+        m["sortlsh_gather"] = dict(flops=0, bytes=2 * mat)                   # per launch: one matrix in, one out
+        m["sortlsh_scatter"] = dict(flops=0, bytes=2 * mat)
     unique_fwd = 4 * BH * N * d * 2                # Q, K, V read, O written
     return m, dict(sel_pairs=sel, tiles=tiles, f_sparse_fwd=f_sparse, f_lr_fwd=f_read + f_state,
                    gathered_fwd=sel * 2 * T * d * 2, unique_fwd=unique_fwd)
@@ -237,6 +243,9 @@ class OracleSample:
         inp = make_inputs(w, 0, heads=range(1))
         self.p = orc.Params(N=w.N, d=w.d, block_size=w.block_size, topk=w.topk, rank_r=w.rank_r,
                             causal=w.causal, scale=w.scale)
+        if w.selector == "sortlsh":
+            self.p.selector = "sortlsh"
+            self.p.lsh_planes = inp["R"].double().numpy()
         self.W = inp["W"].double().numpy()
         self.x = {n: inp[n][0, 0].double().numpy() for n in ("Q", "K", "V", "dO")}
 
@@ -338,9 +347,13 @@ def main():
     key = "16" if w.dtype == "bf16" else ""
     q, k, v, dO = (inp[n + key].to(dev) for n in ("Q", "K", "V", "dO"))
     W = inp["W"].to(dev)
+    lsh = w.selector == "sortlsh"
+    R = inp["R"].to(dev) if lsh else None
     op = bd.Elsaa(bd.make_params(w.B, w.H, w.N, w.d,
                                  dtype=bd.ELSAA_DTYPE_BF16 if w.dtype == "bf16" else bd.ELSAA_DTYPE_F32,
-                                 causal=w.causal, rank_r=w.rank_r, block_size=w.block_size, topk=w.topk), dev)
+                                 causal=w.causal, rank_r=w.rank_r, block_size=w.block_size, topk=w.topk,
+                                 selector=bd.ELSAA_SEL_SORTLSH if lsh else bd.ELSAA_SEL_TOPK_BLOCKS,
+                                 lsh_bits=w.lsh_bits), dev, lsh_planes=R)
     O = op._empty_like_io()
     grads = (op._empty_like_io(), op._empty_like_io(), op._empty_like_io())
     stream = torch.cuda.current_stream(dev)
@@ -381,8 +394,10 @@ def main():
     if not args.no_e2e:
         host = {n: inp[n + key].pin_memory() for n in ("Q", "K", "V", "dO")}
         host_W = inp["W"].pin_memory()
+        host_R = inp["R"].pin_memory() if lsh else None
         outs = [torch.empty(O.shape, dtype=O.dtype).pin_memory() for _ in range(4)]
-        h2d = sum(x.numel() * x.element_size() for x in host.values()) + host_W.numel() * 4
+        h2d = (sum(x.numel() * x.element_size() for x in host.values()) + host_W.numel() * 4
+               + (host_R.numel() * 4 if lsh else 0))
         d2h = sum(x.numel() * x.element_size() for x in outs)
 
         def e2e_step():
@@ -391,6 +406,8 @@ def main():
             v.copy_(host["V"], non_blocking=True)
             dO.copy_(host["dO"], non_blocking=True)
             W.copy_(host_W, non_blocking=True)
+            if lsh:
+                R.copy_(host_R, non_blocking=True)
             step()
             for hsrc, dsrc in zip(outs, (O,) + grads):
                 hsrc.copy_(dsrc, non_blocking=True)
@@ -420,8 +437,9 @@ def main():
     wm = model.get(dom)
     roof = None
     if wm is not None:
-        tensor_kernel = dom in ("attn_fwd", "attn_fwd_tc", "sparse_dq", "dq_tc", "sparse_dkdv", "dkdv_tc",
-                                "race_readout", "race_state_fwd", "race_state_bwd")
+        # the bound is whichever of the kernel's flops and algorithmic bytes takes longer at peak
+        peak_f = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        tensor_kernel = wm["flops"] / (peak_f * 1e12) >= wm["bytes"] / (peaks["hbm_gbs"] * 1e9)
         if tensor_kernel:
             ach = wm["flops"] / (dom_ms * 1e-3) / 1e12
             peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])

@@ -177,17 +177,18 @@ def sortlsh_order(X, R) -> np.ndarray:
     return np.argsort(gray_rank(simhash_codes(X, R)), kind="stable")
 
 
-def sortlsh_support(q, k, p: Params) -> list:
+def sortlsh_support(q, k, p: Params, tiles=None) -> list:
     """Per query row i, the sorted key indices of the key block that shares its
-    position with i's query block in the two sorted orders."""
+    position with i's query block in the two sorted orders.  ``tiles`` keeps only
+    those sorted query blocks (a timing sample); other rows get an empty support."""
     assert not p.causal, "the sortLSH selector here is the non-causal one"
     T, N = p.block_size, p.N
     if p.lsh_orders is not None:      # orders decided elsewhere (the hash signs of another precision)
         oq, ok = (np.asarray(o) for o in p.lsh_orders)
     else:
         oq, ok = sortlsh_order(q, p.lsh_planes), sortlsh_order(k, p.lsh_planes)
-    out = [None] * N
-    for t in range(p.n_tiles):
+    out = [np.zeros(0, dtype=np.int64)] * N
+    for t in (range(p.n_tiles) if tiles is None else tiles):
         keys = np.sort(ok[t * T:(t + 1) * T])
         for i in oq[t * T:(t + 1) * T]:
             out[i] = keys
@@ -377,7 +378,7 @@ def forward_head(q, k, v, W, p: Params, lam=None, g_s=None, g_lr=None, scores=No
     q, k, v = _f64(q), _f64(k), _f64(v)
     if p.selector == "sortlsh":
         sc = idx = None
-        O_s, logd = sparse_from_support(q, k, v, sortlsh_support(q, k, p), p)
+        O_s, logd = sparse_from_support(q, k, v, sortlsh_support(q, k, p, tiles), p)
     else:
         sc = block_scores(q, k, p) if scores is None else _f64(scores)
         idx = select_from_scores(sc, p.topk, p.causal)
@@ -502,7 +503,9 @@ def backward_head(q, k, v, W, dO, fw, p: Params, lam=None, g_s=None, g_lr=None, 
     tile_list = list(range(p.n_tiles)) if tiles is None else list(tiles)
     if p.selector == "sortlsh":
         # the same chain rule row by row over each row's support
-        for i, keys in enumerate(sortlsh_support(q, k, p)):
+        for i, keys in enumerate(sortlsh_support(q, k, p, tiles)):
+            if keys.size == 0:
+                continue
             P = np.exp(p.scale * (k[keys] @ q[i]) - fw["logd_s"][i])
             dz = P * (v[keys] @ dOs[i] - Delta[i])
             dq[i] += p.scale * dz @ k[keys]

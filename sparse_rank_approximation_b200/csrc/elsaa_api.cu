@@ -102,6 +102,7 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
       return false;
     }
     if (p->N > 16384) { *st = fail(ELSAA_ERR_UNSUPPORTED, "sortLSH sorts in shared memory: N <= 16384"); return false; }
+    if ((long)p->B * p->H > 32767) { *st = fail(ELSAA_ERR_UNSUPPORTED, "sortLSH: B * H <= 32767"); return false; }
   }
   if (!lsh && (p->topk < 0 || p->topk > n_t)) {
     *st = fail(ELSAA_ERR_INVALID_ARG, "topk %d outside [0, %d]", p->topk, n_t);

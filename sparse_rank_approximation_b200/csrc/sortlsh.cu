@@ -24,81 +24,177 @@ __device__ __forceinline__ uint32_t gray_position(uint32_t code) {
   return n;
 }
 
-template <typename E>
-__device__ __forceinline__ float to_f(E x);
-template <>
-__device__ __forceinline__ float to_f<float>(float x) { return x; }
-template <>
-__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
-
 }  // namespace
 
-// grid (BH, 2: queries then keys), block 1024.  Shared memory: the planes [bits][d]
-// (fp32) and one 64-bit key (Gray position << 32 | row) per row, padded to a power of
-// two; a bitonic network sorts the keys, which are unique, so the order is stable.
-template <typename E>
-__global__ void __launch_bounds__(kSortThreads) sortlsh_order_kernel(const E* __restrict__ Q,
-                                                                     const E* __restrict__ K,
-                                                                     const float* __restrict__ planes, int bits,
-                                                                     int npow2, int* __restrict__ order,
-                                                                     int* __restrict__ codes, Geom g) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem);
-  float* sR = reinterpret_cast<float*>(keys + npow2);          // [bits][d]
-  const int side = blockIdx.y, bh = blockIdx.x;
-  const E* X = (side == 0 ? Q : K) + (size_t)bh * g.N * g.d;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < bits * g.d; i += kSortThreads) {
-    const int c = i / g.d, k = i % g.d;
-    sR[i] = planes[(size_t)k * bits + c];                        // planes are [d][bits]
+// Hashing: eight lanes per row, each a d/8-element slice (one or two 16-byte loads), and
+// each lane hashes four rows (16 rows per warp), so every plane value read from shared
+// memory serves four rows.  The planes sit there as [bits][d/8][8], so the eight slices
+// of one element index fall in eight banks.  Each row's Gray position goes to `pos` (the
+// sort's input) and, if asked, its code to `codes`; both [BH][2][N].
+constexpr int kHashRows = 4;
+
+template <typename E, int EPL>
+__global__ void __launch_bounds__(256) sortlsh_hash_kernel(const E* __restrict__ Q, const E* __restrict__ K,
+                                                           const float* __restrict__ planes, int bits,
+                                                           int* __restrict__ pos, int* __restrict__ codes, Geom g) {
+  extern __shared__ __align__(16) float sR[];                   // [bits][d/8][8]
+  constexpr int epl = EPL;                                      // elements per lane: d / 8
+  for (int i = threadIdx.x; i < bits * g.d; i += blockDim.x) {
+    const int c = i / g.d, k = i % g.d;                         // plane c, element k = sub * epl + e
+    const int sub = k / epl, e = k % epl;
+    sR[(c * epl + e) * 8 + sub] = planes[(size_t)k * bits + c];   // planes are [d][bits]
   }
   __syncthreads();
-  // one warp per row: lanes split the row, then reduce each plane's projection
-  for (int row = warp; row < g.N; row += kSortThreads / 32) {
-    float x[4];
+  // blockIdx.y: the (head, side) segment; the blocks of a segment stride over its rows
+  const int lane = threadIdx.x & 31, sub = lane & 7;
+  const int seg = blockIdx.y, bh = seg >> 1, side = seg & 1;
+  const E* base = (side ? K : Q) + (size_t)bh * g.N * g.d + sub * epl;
+  const int groups = (g.N + 4 * kHashRows - 1) / (4 * kHashRows);
+  for (int grp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; grp < groups; grp += (gridDim.x * blockDim.x) >> 5) {
+    int row[kHashRows];
+    float v[kHashRows][epl];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int k = lane + 32 * e;
-      x[e] = k < g.d ? to_f<E>(X[(size_t)row * g.d + k]) : 0.f;
-    }
-    uint32_t code = 0;
-    for (int c = 0; c < bits; ++c) {
-      float s = 0.f;
+    for (int m = 0; m < kHashRows; ++m) {
+      row[m] = grp * 4 * kHashRows + 4 * m + (lane >> 3);
+      const E* x = base + (size_t)min(row[m], g.N - 1) * g.d;
+      if constexpr (sizeof(E) == 2) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int k = lane + 32 * e;
-        if (k < g.d) s = fmaf(x[e], sR[c * g.d + k], s);
-      }
+        for (int u = 0; u < epl / 8; ++u) {
+          const uint4 w = *reinterpret_cast<const uint4*>(x + 8 * u);
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
 #pragma unroll
-      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      code |= (s > 0.f ? 1u : 0u) << c;
-    }
-    if (lane == 0) {
-      keys[row] = ((unsigned long long)gray_position(code) << 32) | (unsigned)row;
-      if (codes) codes[((size_t)bh * 2 + side) * g.N + row] = (int)code;
-    }
-  }
-  for (int i = g.N + tid; i < npow2; i += kSortThreads) keys[i] = ~0ull;
-  __syncthreads();
-  // bitonic sort, ascending
-  for (int k = 2; k <= npow2; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < npow2; i += kSortThreads) {
-        const int l = i ^ j;
-        if (l > i) {
-          const unsigned long long a = keys[i], b = keys[l];
-          const bool up = (i & k) == 0;
-          if ((a > b) == up) {
-            keys[i] = b;
-            keys[l] = a;
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(h[j]);
+            v[m][8 * u + 2 * j] = f.x;
+            v[m][8 * u + 2 * j + 1] = f.y;
           }
         }
+      } else {
+#pragma unroll
+        for (int u = 0; u < epl / 4; ++u) {
+          const float4 w = *reinterpret_cast<const float4*>(x + 4 * u);
+          v[m][4 * u] = w.x; v[m][4 * u + 1] = w.y; v[m][4 * u + 2] = w.z; v[m][4 * u + 3] = w.w;
+        }
       }
-      __syncthreads();
+    }
+    uint32_t code[kHashRows] = {};
+    for (int c = 0; c < bits; ++c) {
+      const float* pc = sR + c * epl * 8 + sub;
+      float acc[kHashRows] = {};
+#pragma unroll
+      for (int e = 0; e < epl; ++e) {
+        const float w = pc[e * 8];
+#pragma unroll
+        for (int m = 0; m < kHashRows; ++m) acc[m] = fmaf(v[m][e], w, acc[m]);
+      }
+#pragma unroll
+      for (int m = 0; m < kHashRows; ++m) {
+        float t = acc[m];
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        t += __shfl_xor_sync(0xffffffffu, t, 2);
+        t += __shfl_xor_sync(0xffffffffu, t, 4);
+        code[m] |= (t > 0.f ? 1u : 0u) << c;
+      }
+    }
+    if (sub == 0) {
+#pragma unroll
+      for (int m = 0; m < kHashRows; ++m) {
+        if (row[m] >= g.N) continue;
+        pos[(size_t)seg * g.N + row[m]] = (int)gray_position(code[m]);
+        if (codes) codes[(size_t)seg * g.N + row[m]] = (int)code[m];
+      }
     }
   }
-  int* out = order + ((size_t)bh * 2 + side) * g.N;
-  for (int i = tid; i < g.N; i += kSortThreads) out[i] = (int)(keys[i] & 0xffffffffu);
+}
+
+// Stable sort of one (head, side) by Gray position, in shared memory: least-significant
+// digit first, 8 bits per pass, each pass a counting sort.  Items are packed
+// (position << 14 | row), so rows need N <= 16384.  Warp w owns the rows of the w-th
+// contiguous slice; counts are kept per (digit, warp) and scanned digit-major, warp-minor,
+// and within a warp equal digits are ranked by lane (match_any), which keeps every pass
+// stable.  Reads its `order` segment (the positions) whole before writing the sorted rows
+// over it.
+__global__ void __launch_bounds__(kSortThreads) sortlsh_sort_kernel(int* __restrict__ order, int bits, Geom g) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  int* cnt = reinterpret_cast<int*>(smem);                          // [256 digits][32 warps]
+  uint32_t* bufA = reinterpret_cast<uint32_t*>(cnt + 256 * 32);
+  uint32_t* bufB = bufA + g.N;
+  __shared__ int wsum[32];
+  int* seg = order + ((size_t)blockIdx.x * 2 + blockIdx.y) * g.N;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < g.N; i += kSortThreads) bufA[i] = ((uint32_t)seg[i] << 14) | (uint32_t)i;
+  const int slice = (g.N + 31) / 32;
+  const int r0 = warp * slice, r1 = min(g.N, r0 + slice);
+  uint32_t* src = bufA;
+  uint32_t* dst = bufB;
+  for (int shift = 0; shift < bits; shift += 8) {
+    for (int i = tid; i < 256 * 32; i += kSortThreads) cnt[i] = 0;
+    __syncthreads();
+    // 1: per-warp digit counts
+    for (int base = r0; base < r1; base += 32) {
+      const int i = base + lane;
+      const bool live = i < r1;
+      const uint32_t dig = live ? (src[i] >> (14 + shift)) & 255u : 256u + lane;
+      const unsigned peers = __match_any_sync(0xffffffffu, dig);
+      if (live && lane == __ffs(peers) - 1) cnt[dig * 32 + warp] += __popc(peers);
+      __syncwarp();
+    }
+    __syncthreads();
+    // 2: exclusive scan over (digit, warp); thread t owns entries 8t .. 8t + 7
+    {
+      int loc[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        loc[j] = cnt[8 * tid + j];
+        sum += loc[j];
+      }
+      int inc = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += t;
+      }
+      if (lane == 31) wsum[warp] = inc;
+      __syncthreads();
+      if (warp == 0) {
+        int w = wsum[lane], wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, wi, o);
+          if (lane >= o) wi += t;
+        }
+        wsum[lane] = wi - w;
+      }
+      __syncthreads();
+      int run = wsum[warp] + inc - sum;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[8 * tid + j] = run;
+        run += loc[j];
+      }
+    }
+    __syncthreads();
+    // 3: stable scatter, each warp through its slice in row order
+    for (int base = r0; base < r1; base += 32) {
+      const int i = base + lane;
+      const bool live = i < r1;
+      const uint32_t item = live ? src[i] : 0u;
+      const uint32_t dig = live ? (item >> (14 + shift)) & 255u : 256u + lane;
+      const unsigned peers = __match_any_sync(0xffffffffu, dig);
+      if (live) {
+        const int at = cnt[dig * 32 + warp] + __popc(peers & ((1u << lane) - 1u));
+        dst[at] = item;
+      }
+      __syncwarp();
+      if (live && lane == __ffs(peers) - 1) cnt[dig * 32 + warp] += __popc(peers);
+      __syncwarp();
+    }
+    __syncthreads();
+    uint32_t* t = src;
+    src = dst;
+    dst = t;
+  }
+  for (int i = tid; i < g.N; i += kSortThreads) seg[i] = (int)(src[i] & 0x3fffu);
 }
 
 // Rows of 16-byte units: dst[r] = src[perm[r]] (gather) or dst[perm[r]] = src[r]
@@ -140,26 +236,39 @@ __global__ void diag_select_kernel(int* __restrict__ idx, Geom g) {
 }
 
 size_t sortlsh_smem_bytes(const Geom& g, int bits) {
-  int npow2 = 1;
-  while (npow2 < g.N) npow2 <<= 1;
-  return (size_t)npow2 * 8 + (size_t)bits * g.d * 4;
+  (void)bits;
+  return (size_t)256 * 32 * 4 + (size_t)2 * g.N * 4;
 }
 
 cudaError_t launch_sortlsh_order(const void* Q, const void* K, bool bf16, const float* planes, int bits,
                                  int* order, int* codes, const Geom& g, cudaStream_t st) {
-  int npow2 = 1;
-  while (npow2 < g.N) npow2 <<= 1;
-  const size_t smem = sortlsh_smem_bytes(g, bits);
-  auto run = [&](auto kern, const auto* q, const auto* k) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t hsmem = (size_t)bits * g.d * 4;
+  // about eight blocks of 256 threads per SM over all segments
+  const int per_seg_max = (g.N + 8 * 4 * kHashRows - 1) / (8 * 4 * kHashRows);   // one iteration each
+  const int per_seg = std::max(1, std::min(per_seg_max, (148 * 8 + 2 * g.BH - 1) / (2 * g.BH)));
+  const dim3 hgrid(per_seg, 2 * g.BH);
+  {
+    ProfScope ps("sortlsh_hash", st);
+    auto run = [&](auto kern, const auto* q, const auto* k) {
+      kern<<<hgrid, 256, hsmem, st>>>(q, k, planes, bits, order, codes, g);
+    };
+    const auto* q16 = (const __nv_bfloat16*)Q;
+    const auto* k16 = (const __nv_bfloat16*)K;
+    const auto* q32 = (const float*)Q;
+    const auto* k32 = (const float*)K;
+    if (bf16 && g.d == 128) run(sortlsh_hash_kernel<__nv_bfloat16, 16>, q16, k16);
+    else if (bf16) run(sortlsh_hash_kernel<__nv_bfloat16, 8>, q16, k16);
+    else if (g.d == 128) run(sortlsh_hash_kernel<float, 16>, q32, k32);
+    else run(sortlsh_hash_kernel<float, 8>, q32, k32);
+    const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    ProfScope ps("sortlsh_order", st);
-    kern<<<dim3(g.BH, 2), kSortThreads, smem, st>>>(q, k, planes, bits, npow2, order, codes, g);
-    return cudaGetLastError();
-  };
-  if (bf16)
-    return run(sortlsh_order_kernel<__nv_bfloat16>, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K);
-  return run(sortlsh_order_kernel<float>, (const float*)Q, (const float*)K);
+  }
+  const size_t smem = sortlsh_smem_bytes(g, bits);
+  cudaError_t e = cudaFuncSetAttribute(sortlsh_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  ProfScope ps("sortlsh_sort", st);
+  sortlsh_sort_kernel<<<dim3(g.BH, 2), kSortThreads, smem, st>>>(order, bits, g);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_permute_rows(const void* src, void* dst, const int* perm, int row_bytes, const Geom& g,

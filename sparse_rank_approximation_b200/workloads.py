@@ -46,6 +46,8 @@ class Workload:
     sigma: float = 0.3
     backward: bool = True
     hash_bits: int = HASH_BITS
+    selector: str = "topk"    # "topk" (top-k blocks by pooled score) or "sortlsh"
+    lsh_bits: int = 0         # sortLSH: bits of the angular hash code
 
     @property
     def n_tables(self) -> int:
@@ -62,7 +64,8 @@ class Workload:
     def describe(self) -> str:
         return (f"B{self.B} H{self.H} N{self.N} d{self.d} {self.dtype} "
                 f"{'causal' if self.causal else 'non-causal'} r{self.rank_r} "
-                f"block{self.block_size} top{self.topk}")
+                + (f"block{self.block_size} sortLSH{self.lsh_bits}" if self.selector == "sortlsh"
+                   else f"block{self.block_size} top{self.topk}"))
 
 
 WORKLOADS = {
@@ -74,6 +77,10 @@ WORKLOADS = {
                         n_centroids=128, sigma=0.3),
     "n16k_d128": Workload("n16k_d128", 1, 32, 16384, 128, "bf16", True, 128, 128, 16,
                           n_centroids=256, sigma=0.5),
+    # the headline shape, non-causal, with the sortLSH selector: 2^7 hash buckets for the
+    # 128 blocks of 128 rows
+    "n16k_d128_sortlsh": Workload("n16k_d128_sortlsh", 1, 32, 16384, 128, "bf16", False, 128, 128, 1,
+                                  n_centroids=256, sigma=0.5, selector="sortlsh", lsh_bits=7),
     "n64k_d128": Workload("n64k_d128", 1, 8, 65536, 128, "bf16", True, 256, 128, 32,
                           n_centroids=512, sigma=0.3),
 }
@@ -119,6 +126,8 @@ def make_inputs(w: Workload, seed: int = 0, heads: Optional[range] = None) -> di
             t = t16.float()
         out[name] = t.contiguous()
     out["W"] = W.contiguous()
+    if w.selector == "sortlsh":   # hyperplanes of the angular hash, drawn after everything else
+        out["R"] = torch.randn(d, w.lsh_bits, generator=g).contiguous()
     return out
 
 

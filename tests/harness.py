@@ -26,12 +26,12 @@ def oracle_params(w: Workload, **kw) -> orc.Params:
     return p
 
 
-def gpu_op(w: Workload, **kw) -> bd.Elsaa:
+def gpu_op(w: Workload, lsh_planes=None, **kw) -> bd.Elsaa:
     p = bd.make_params(w.B, w.H, w.N, w.d,
                        dtype=bd.ELSAA_DTYPE_BF16 if w.dtype == "bf16" else bd.ELSAA_DTYPE_F32,
                        causal=w.causal, rank_r=w.rank_r, block_size=w.block_size, topk=w.topk,
                        scale=w.scale, **kw)
-    return bd.Elsaa(p, torch.device("cuda", 0))
+    return bd.Elsaa(p, torch.device("cuda", 0), lsh_planes=lsh_planes)
 
 
 def device_inputs(w: Workload, inp: dict) -> dict:

@@ -10,8 +10,8 @@ import torch
 
 from oracle import elsaa_oracle as orc
 from sparse_rank_approximation_b200 import binding as bd
-from sparse_rank_approximation_b200.workloads import make_inputs, small_workload
-from tests.harness import check, check_fusion_grads, device_inputs, np64, oracle_params
+from sparse_rank_approximation_b200.workloads import WORKLOADS, make_inputs, small_workload
+from tests.harness import BF16_ABS_TOL, BF16_STORE_REL, check, check_fusion_grads, device_inputs, gpu_op, np64, oracle_params
 
 pytestmark = pytest.mark.gpu
 
@@ -111,3 +111,51 @@ def test_rejects_causal_and_oversize():
     p = bd.make_params(1, 1, 32768, 64, block_size=64, topk=1, rank_r=16, causal=False,
                        selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=8)
     assert L.elsaa_saved_bytes(ctypes.byref(p)) == 0
+
+
+def _sparse_rounding_scales(q, k, v, dO, fw, p):
+    """Per-element scales of the bf16 rounding inside the sparse backward, from the oracle's
+    own quantities: dS is rounded before dS K and dS^T Q, P before P^T dO_s, and Delta is a
+    row sum over the bf16-saved O_s, so it is off by up to 2^-9 sum_c |dO_s,ic O_s,ic|, which
+    every dS_ij = P_ij (dP_ij - Delta_i) inherits times P_ij.  When one key dominates a row,
+    dP_ij and Delta_i nearly cancel and that last term is the whole of dS_ij's error."""
+    dOs, _, dds_ds, _ = orc._fusion_adjoints(dO, fw, p, None, None, None)
+    Delta = (dOs * fw["O_s"]).sum(axis=1) - dds_ds
+    eD = (np.abs(dOs) * np.abs(fw["O_s"])).sum(axis=1)
+    Bq, Bk, Bv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for i, keys in enumerate(orc.sortlsh_support(q, k, p)):
+        P = np.exp(p.scale * (k[keys] @ q[i]) - fw["logd_s"][i])
+        dz = np.abs(P * (v[keys] @ dOs[i] - Delta[i])) + P * eD[i]
+        Bq[i] += p.scale * dz @ np.abs(k[keys])
+        Bk[keys] += p.scale * np.outer(dz, np.abs(q[i]))
+        Bv[keys] += np.outer(P, np.abs(dOs[i]))
+    return Bq, Bk, Bv
+
+
+def test_full_size():
+    """The full-length sortLSH workload (B1 H32 N16384 d128, 7-bit codes), launched as the
+    benchmark launches it; every row of two heads against the oracle on the GPU's orders."""
+    w = WORKLOADS["n16k_d128_sortlsh"]
+    inp = make_inputs(w, 0)
+    dev = device_inputs(w, inp)
+    R = inp["R"]
+    op = gpu_op(w, selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=w.lsh_bits, lsh_planes=R.cuda())
+    O = op.forward(dev["Q"], dev["K"], dev["V"], dev["W"])
+    dQ, dK, dV = op.backward(dev["Q"], dev["K"], dev["V"], dev["W"], dev["dO"])
+    _, order = op.debug_sortlsh(dev["Q"], dev["K"])
+    torch.cuda.synchronize()
+    W = inp["W"].double().numpy()
+    for h in (0, w.H - 1):
+        get = lambda n: inp[n][0, h].double().numpy()
+        p = _oracle_params(w, R, (order[0, h, 0].cpu().numpy(), order[0, h, 1].cpu().numpy()))
+        fw = orc.forward_head(get("Q"), get("K"), get("V"), W, p)
+        dq, dk, dv = orc.backward_head(get("Q"), get("K"), get("V"), W, get("dO"), fw, p)
+        check(w, f"O[{h}]", np64(O[0, h]), fw["O"])
+        # the gradients: the usual bf16 bound plus the rounding inside the sparse backward
+        # (twice its half-ulp scale); at this length sorted blocks put most of a row's
+        # mass on a few keys, where the Delta term dominates
+        scales = _sparse_rounding_scales(get("Q"), get("K"), get("V"), get("dO"), fw, p)
+        for name, got, ref, B in zip(("dQ", "dK", "dV"), (dQ, dK, dV), (dq, dk, dv), scales):
+            err = np.abs(np64(got[0, h]) - ref)
+            excess = (err - BF16_STORE_REL * np.abs(ref) - 2.0 ** -8 * B).max()
+            assert excess <= BF16_ABS_TOL, f"{name}[{h}]: max err {err.max():.3e}, beyond the bound {excess:.3e}"
