@@ -57,9 +57,10 @@ class Params:
     tau: float = 1.0
     chunk: Optional[int] = None   # RACE causal chunk size; defaults to block_size
     fixed_m: bool = False    # ablation without denominator-aware fusion: m = 1, default g_lr = 1
-    selector: str = "topk"   # "topk" (blocks by pooled score) or "sortlsh" (non-causal, §3.2)
+    selector: str = "topk"   # "topk" (blocks by pooled score) or "sortlsh" (§3.2; causal: the recursion)
     lsh_planes: Optional[np.ndarray] = None   # sortLSH hyperplanes [d, bits] (selector "sortlsh")
-    lsh_orders: Optional[tuple] = None        # sortLSH: externally decided (query, key) orders
+    lsh_orders: Optional[tuple] = None        # non-causal sortLSH: externally decided (query, key) orders
+    lsh_codes: Optional[tuple] = None         # causal sortLSH: externally decided (query, key) hash codes
 
     @property
     def n_tables(self) -> int:
@@ -151,7 +152,8 @@ def support(idx: np.ndarray, p: Params) -> list:
 # Reading (the page has no pseudocode): angular LSH with the caller's hyperplanes
 # R [d, b], bit c of a row's code set when x . R_c > 0; rows are ordered by the
 # position of their code in the reflected Gray sequence (neighbouring buckets
-# differ in one bit), ties by row index.  Non-causal only.
+# differ in one bit), ties by row index.  The causal selector is the recursion
+# further down.
 # ----------------------------------------------------------------------------
 
 def simhash_codes(X, R) -> np.ndarray:
@@ -193,6 +195,116 @@ def sortlsh_support(q, k, p: Params, tiles=None) -> list:
         for i in oq[t * T:(t + 1) * T]:
             out[i] = keys
     return out
+
+
+# ----------------------------------------------------------------------------
+# Causal sortLSH [ELSAA §3.2, "For the causal setting"]: divide and conquer.  A
+# segment is split into a past and a future half; each half recurses (its own
+# causal problem); the future queries against the past keys are a non-causal
+# sortLSH problem (every such key precedes every such query); the future half's
+# two results are merged by log-sum-exp, which keeps the softmax exact over the
+# union of the two supports.
+# Readings (Algorithm 5 is not on the page): the split is on block boundaries
+# with the extra block of an odd count going to the past half, so the past half
+# has at least as many sorted key blocks as the future half has query blocks; a
+# single block is the leaf, attended exactly under the mask j <= i; every level
+# hashes with the same planes, and the off-diagonal problem is the non-causal
+# selector above restricted to the two halves.
+# ----------------------------------------------------------------------------
+
+def _lsh_codes(q, k, p: Params):
+    if p.lsh_codes is not None:       # codes decided elsewhere (the hash signs of another precision)
+        return tuple(np.asarray(c, dtype=np.int64) for c in p.lsh_codes)
+    return simhash_codes(q, p.lsh_planes), simhash_codes(k, p.lsh_planes)
+
+
+def _split(a: int, b: int, T: int):
+    """Past/future boundary of the row segment [a, b), or None for a leaf."""
+    nb = -(-(b - a) // T)
+    return None if nb <= 1 else a + -(-nb // 2) * T
+
+
+def _sorted_rows(codes, a: int, b: int) -> np.ndarray:
+    """Rows a..b-1 by Gray position of their code, ties by row."""
+    return a + np.argsort(gray_rank(codes[a:b]), kind="stable")
+
+
+def causal_sortlsh(q, k, v, p: Params):
+    """Sparse branch (O_s, log d_s) of the causal recursion, taken in its own steps:
+    recurse on both halves, attend the future queries' sorted blocks to the past
+    keys' sorted blocks, merge the future half by log-sum-exp."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    N, d = q.shape
+    T = p.block_size
+    cq, ck = _lsh_codes(q, k, p)
+
+    def rec(a, b):
+        mid = _split(a, b, T)
+        if mid is None:                                   # leaf: one block, exact under j <= i
+            O = np.zeros((b - a, d))
+            logd = np.zeros(b - a)
+            for i in range(a, b):
+                z = p.scale * (k[a:i + 1] @ q[i])
+                mx = z.max()
+                e = np.exp(z - mx)
+                O[i - a] = e @ v[a:i + 1] / e.sum()
+                logd[i - a] = mx + np.log(e.sum())
+            return O, logd
+        O_past, l_past = rec(a, mid)
+        O_ff, l_ff = rec(mid, b)
+        # future queries x past keys: non-causal sortLSH on the two halves
+        oq, ok = _sorted_rows(cq, mid, b), _sorted_rows(ck, a, mid)
+        O_fp = np.zeros((b - mid, d))
+        l_fp = np.full(b - mid, -np.inf)
+        for t in range(-(-(b - mid) // T)):
+            rows, keys = oq[t * T:(t + 1) * T], ok[t * T:(t + 1) * T]
+            if keys.size == 0:
+                continue
+            z = p.scale * (q[rows] @ k[keys].T)
+            mx = z.max(axis=1, keepdims=True)
+            e = np.exp(z - mx)
+            O_fp[rows - mid] = e @ v[keys] / e.sum(axis=1, keepdims=True)
+            l_fp[rows - mid] = mx[:, 0] + np.log(e.sum(axis=1))
+        # log-sum-exp merge of the future half's two contributions
+        l_f = np.logaddexp(l_ff, l_fp)
+        O_f = np.exp(l_ff - l_f)[:, None] * O_ff + np.exp(l_fp - l_f)[:, None] * O_fp
+        return np.concatenate([O_past, O_f]), np.concatenate([l_past, l_f])
+
+    return rec(0, N)
+
+
+def causal_sortlsh_support(q, k, p: Params, tiles=None) -> list:
+    """Per query row i, its keys under the causal recursion: the union over the
+    levels of the sorted key block its sorted query block meets, plus its own
+    block's keys j <= i.  ``tiles`` keeps only the rows of those query tiles (a
+    timing sample); other rows get an empty support."""
+    N, T = p.N, p.block_size
+    cq, ck = _lsh_codes(q, k, p)
+    parts = [[] for _ in range(N)]
+
+    def rec(a, b):
+        mid = _split(a, b, T)
+        if mid is None:
+            for i in range(a, b):
+                parts[i].append(np.arange(a, i + 1))
+            return
+        rec(a, mid)
+        rec(mid, b)
+        oq, ok = _sorted_rows(cq, mid, b), _sorted_rows(ck, a, mid)
+        for t in range(-(-(b - mid) // T)):
+            keys = ok[t * T:(t + 1) * T]
+            for i in oq[t * T:(t + 1) * T]:
+                parts[i].append(keys)
+
+    rec(0, N)
+    keep = None if tiles is None else {i for t in tiles for i in range(t * T, min(N, (t + 1) * T))}
+    return [np.sort(np.concatenate(parts[i])) if keep is None or i in keep else np.zeros(0, dtype=np.int64)
+            for i in range(N)]
+
+
+def lsh_support(q, k, p: Params, tiles=None) -> list:
+    """Per-row support of the sortLSH selector (the recursion when causal)."""
+    return causal_sortlsh_support(q, k, p, tiles) if p.causal else sortlsh_support(q, k, p, tiles)
 
 
 def sparse_from_support(q, k, v, sup, p: Params):
@@ -378,7 +490,10 @@ def forward_head(q, k, v, W, p: Params, lam=None, g_s=None, g_lr=None, scores=No
     q, k, v = _f64(q), _f64(k), _f64(v)
     if p.selector == "sortlsh":
         sc = idx = None
-        O_s, logd = sparse_from_support(q, k, v, sortlsh_support(q, k, p, tiles), p)
+        if p.causal:
+            O_s, logd = causal_sortlsh(q, k, v, p)
+        else:
+            O_s, logd = sparse_from_support(q, k, v, sortlsh_support(q, k, p, tiles), p)
     else:
         sc = block_scores(q, k, p) if scores is None else _f64(scores)
         idx = select_from_scores(sc, p.topk, p.causal)
@@ -503,7 +618,7 @@ def backward_head(q, k, v, W, dO, fw, p: Params, lam=None, g_s=None, g_lr=None, 
     tile_list = list(range(p.n_tiles)) if tiles is None else list(tiles)
     if p.selector == "sortlsh":
         # the same chain rule row by row over each row's support
-        for i, keys in enumerate(sortlsh_support(q, k, p, tiles)):
+        for i, keys in enumerate(lsh_support(q, k, p, tiles)):
             if keys.size == 0:
                 continue
             P = np.exp(p.scale * (k[keys] @ q[i]) - fw["logd_s"][i])

@@ -328,8 +328,8 @@ def test_key_permutation_invariance_noncausal_block1():
 
 def _selection(q, k, p, out):
     """What the selector chose: the block indices, or both sortLSH orders."""
-    if p.selector == "sortlsh":
-        return np.concatenate([orc.sortlsh_order(q, p.lsh_planes), orc.sortlsh_order(k, p.lsh_planes)])
+    if p.selector == "sortlsh":      # the codes decide every sorted order, at every level
+        return np.concatenate([orc.simhash_codes(q, p.lsh_planes), orc.simhash_codes(k, p.lsh_planes)])
     return out["idx"]
 
 
@@ -346,7 +346,9 @@ def _loss(q, k, v, W, p, dO, lam=None, g_s=None, g_lr=None):
                                                           (True, False, 16, 2, 1.0, True),
                                                           (False, True, 16, 2, 1.3, True),
                                                           (False, False, 16, "sortlsh", 1.0, False),
-                                                          (False, True, 0, "sortlsh", 0.9, False)])
+                                                          (False, True, 0, "sortlsh", 0.9, False),
+                                                          (True, False, 16, "sortlsh", 1.0, False),
+                                                          (True, True, 0, "sortlsh", 1.2, True)])
 def test_backward_matches_finite_differences(causal, gates, r, k, tau, fixed_m):
     N, d, T = 24, 6, 4
     lsh = k == "sortlsh"
@@ -509,6 +511,78 @@ def test_sortlsh_groups_rows_into_equal_blocks_of_similar_codes():
         assert np.all(np.diff(pos) >= 0)
         same = np.diff(pos) == 0
         assert np.all(np.diff(order)[same] > 0)
+
+
+# --- causal sortLSH: the recursion of §3.2 ---
+
+def _causal_lsh_params(N, d, T, bits, seed, **kw):
+    p = _sortlsh_params(N, d, T, bits, seed, **kw)
+    p.causal = True
+    return p
+
+
+@pytest.mark.parametrize("N,T", [(8, 8), (5, 8), (16, 8), (13, 8)])
+def test_causal_sortlsh_up_to_two_blocks_is_dense_causal_softmax(N, T):
+    """One block is the leaf (exact under j <= i); with two, the future block's single
+    sorted query block meets the past half's single key block, i.e. every earlier key."""
+    d = 6
+    q, k, v = _rand((N, d), 120), _rand((N, d), 121), _rand((N, d), 122)
+    p = _causal_lsh_params(N, d, T, 5, 123)
+    out = orc.forward_head(q, k, v, np.zeros((0, d, 4)), p)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[None], torch.tensor(k)[None], torch.tensor(v)[None], is_causal=True,
+        scale=p.scale)[0].numpy()
+    np.testing.assert_allclose(out["O"], ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("N,T,bits", [(64, 8, 3), (70, 8, 4), (96, 4, 2)])
+def test_causal_sortlsh_recursion_is_softmax_over_the_union_of_its_supports(N, T, bits):
+    """The recursion's log-sum-exp merges give the exact softmax over the union of the
+    key sets it visits (computed row by row from the support)."""
+    d = 6
+    q, k, v = _rand((N, d), 124), _rand((N, d), 125), _rand((N, d), 126)
+    p = _causal_lsh_params(N, d, T, bits, 127)
+    O, logd = orc.causal_sortlsh(q, k, v, p)
+    O2, logd2 = orc.sparse_from_support(q, k, v, orc.causal_sortlsh_support(q, k, p), p)
+    np.testing.assert_allclose(O, O2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(logd, logd2, rtol=0, atol=1e-12)
+
+
+def test_causal_sortlsh_support_sizes_follow_the_block_index_bits():
+    """With 2^L blocks every split is exact: row i in block t is in the future half at
+    one level per set bit of t, gaining T keys there, plus its own block's keys j <= i;
+    all keys precede i and no key repeats."""
+    N, d, T = 128, 6, 8
+    q, k = _rand((N, d), 128), _rand((N, d), 129)
+    p = _causal_lsh_params(N, d, T, 4, 130)
+    for i, keys in enumerate(orc.causal_sortlsh_support(q, k, p)):
+        t = i // T
+        assert keys.size == (i % T) + 1 + T * bin(t).count("1")
+        assert np.all(np.diff(keys) > 0) and keys[-1] == i
+        assert np.all(keys[keys >= t * T] == np.arange(t * T, i + 1))
+
+
+def test_causal_sortlsh_with_equal_codes_attends_blocks_t_minus_powers_of_two():
+    """Zero hyperplanes give every row the same code, so each sorted order is the row
+    order: the future block with offset u in a half of 2^j blocks meets the past block
+    with offset u, i.e. block t attends t and t - 2^j for every set bit j of t."""
+    N, d, T = 64, 6, 4
+    q, k, v = _rand((N, d), 131), _rand((N, d), 132), _rand((N, d), 133)
+    p = _causal_lsh_params(N, d, T, 3, 134)
+    p.lsh_planes = np.zeros((d, 3))
+    mask = np.zeros((N, N), dtype=bool)
+    for i in range(N):
+        t = i // T
+        mask[i, t * T:i + 1] = True
+        for j in range(t.bit_length()):
+            if t >> j & 1:
+                b = t - (1 << j)
+                mask[i, b * T:(b + 1) * T] = True
+    out = orc.forward_head(q, k, v, np.zeros((0, d, 4)), p)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[None], torch.tensor(k)[None], torch.tensor(v)[None], attn_mask=torch.tensor(mask)[None],
+        scale=p.scale)[0].numpy()
+    np.testing.assert_allclose(out["O"], ref, rtol=0, atol=1e-12)
 
 
 # --- rank view [ELSAA §4]: rank(S_Omega + B A) = min(n, nu(Omega) + r) ---
