@@ -31,6 +31,8 @@ struct Geom {
   int fixed_m;    // fusion without the denominator-aware weight: m = 1, default g_lr = 1
   int selector;   // 0: top-k key blocks; 1: sortLSH (the operator runs on row-permuted copies)
   int lsh_bits;
+  int lsh_levels; // causal sortLSH: recursion levels run on sorted rows (log2(n_t) - 1; the deepest
+                  // level and the leaves run in the base pass)
   float scale, lam, eps, tau;
 };
 

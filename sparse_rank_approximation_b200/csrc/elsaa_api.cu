@@ -91,17 +91,29 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
     return false;
   }
   const bool lsh = p->selector == ELSAA_SEL_SORTLSH;
+  int lsh_levels = 0;
   if (lsh) {
-    if (p->causal) {
-      *st = fail(ELSAA_ERR_UNSUPPORTED, "the sortLSH selector is non-causal (the causal recursion is not built)");
-      return false;
-    }
     if (T == 1) { *st = fail(ELSAA_ERR_UNSUPPORTED, "sortLSH needs block_size 64 or 128"); return false; }
     if (p->lsh_bits < 1 || p->lsh_bits > 16) {
       *st = fail(ELSAA_ERR_INVALID_ARG, "lsh_bits %d outside [1, 16]", p->lsh_bits);
       return false;
     }
-    if (p->N > 16384) { *st = fail(ELSAA_ERR_UNSUPPORTED, "sortLSH sorts in shared memory: N <= 16384"); return false; }
+    if (p->causal) {
+      // the recursion runs on the tensor-core kernels, halving down to single blocks
+      if (!bf16 || p->d != 128 || T != 128) {
+        *st = fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH needs bf16, d = 128, block_size 128");
+        return false;
+      }
+      if (p->N % T || (n_t & (n_t - 1))) {
+        *st = fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH needs N = block_size * 2^L (got N = %d)", p->N);
+        return false;
+      }
+      if (p->N > 32768) { *st = fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH sorts halves in shared memory: N <= 32768"); return false; }
+      while ((2 << lsh_levels) < n_t) ++lsh_levels;               // log2(n_t) - 1 sorted levels
+    } else if (p->N > 16384) {
+      *st = fail(ELSAA_ERR_UNSUPPORTED, "sortLSH sorts in shared memory: N <= 16384");
+      return false;
+    }
     if ((long)p->B * p->H > 32767) { *st = fail(ELSAA_ERR_UNSUPPORTED, "sortLSH: B * H <= 32767"); return false; }
   }
   if (!lsh && (p->topk < 0 || p->topk > n_t)) {
@@ -113,7 +125,9 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
   g->d = p->d;
   g->T = T;
   g->n_t = n_t;
-  g->k = lsh ? 1 : p->topk;     // sortLSH: tile t selects block t of the sorted orders
+  // sortLSH: tile t selects block t of the sorted orders; causal: the base pass takes the
+  // tile's own block and, for odd t, block t - 1
+  g->k = lsh ? (p->causal ? 2 : 1) : p->topk;
   g->r = p->rank_r;
   g->L = p->rank_r >> kHashBits;
   g->C = bf16 ? T : 64;
@@ -126,6 +140,7 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
   g->fixed_m = p->fixed_m != 0;
   g->selector = p->selector;
   g->lsh_bits = lsh ? p->lsh_bits : 0;
+  g->lsh_levels = lsh_levels;
   g->scale = p->scale;
   g->lam = p->lambda;
   g->eps = p->eps;
@@ -142,7 +157,7 @@ struct Saved {
   float *Ast, *Bst;
   void* Psplit;
   float* Pmass;
-  int* lsh_order;          // sortLSH: sorted query and key orders [BH][2][N]
+  int* lsh_order;          // sortLSH: sorted query and key orders [BH][2][N] (causal: one per level)
 };
 
 Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
@@ -167,7 +182,8 @@ Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
   const bool split = esz == 2 && g.r > 0 && race_bwd_tc_supported(g);
   s.Psplit = split ? c.take<char>((size_t)g.BH * g.n_c * 2 * g.r * g.d * 2) : nullptr;
   s.Pmass = split ? c.take<float>((size_t)g.BH * g.n_c * g.r) : nullptr;
-  s.lsh_order = g.selector == ELSAA_SEL_SORTLSH ? c.take<int>((size_t)g.BH * 2 * g.N) : nullptr;
+  const size_t orders = g.selector != ELSAA_SEL_SORTLSH ? 0 : g.causal ? (size_t)g.lsh_levels : 1;
+  s.lsh_order = orders ? c.take<int>(orders * g.BH * 2 * g.N) : nullptr;
   *bytes = align_up(c.off);
   return s;
 }
@@ -176,6 +192,13 @@ Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
 struct PermBufs {
   void *Q, *K, *V, *X, *dQ, *dK, *dV;     // X: O (forward) or dO (backward)
   float *lam, *gs, *glr;
+  // causal recursion: a level's O_s and log d_s (sorted order), the running fp32 sparse
+  // result (caller's order, log-denominators double-buffered), a level's selection, the
+  // Gray positions and the sorted rows' packed backward scalars
+  void* Os;
+  float *accO, *logd, *m, *accL[2];
+  int *idx, *pos;
+  float4* packed;
 };
 
 PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
@@ -191,9 +214,24 @@ PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
     b.dK = c.take<char>(mat);
     b.dV = c.take<char>(mat);
   }
-  b.lam = c.take<float>(rows);
-  b.gs = c.take<float>(rows);
-  b.glr = c.take<float>(rows);
+  if (!g.causal) {
+    b.lam = c.take<float>(rows);
+    b.gs = c.take<float>(rows);
+    b.glr = c.take<float>(rows);
+    return b;
+  }
+  b.idx = c.take<int>((size_t)g.BH * g.n_t);
+  if (backward) {
+    b.packed = c.take<float4>(rows);
+    return b;
+  }
+  b.Os = c.take<char>(mat);
+  b.accO = c.take<float>(rows * g.d);
+  b.logd = c.take<float>(rows);
+  b.m = c.take<float>(rows);
+  b.accL[0] = c.take<float>(rows);
+  b.accL[1] = c.take<float>(rows);
+  b.pos = c.take<int>(rows * 2);
   return b;
 }
 
@@ -246,7 +284,8 @@ BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
   w.offs = c.take<int>((size_t)g.BH * (g.n_t + 1));
   w.tiles = c.take<int>((size_t)g.BH * g.n_t * std::max(g.k, 1));
   w.order = c.take<int>((size_t)g.BH * g.n_t);
-  const size_t acc = bf16 && g.r > 0 ? rows * g.d : 0;
+  const bool causal_lsh = g.selector == ELSAA_SEL_SORTLSH && g.causal;
+  const size_t acc = bf16 && (g.r > 0 || causal_lsh) ? rows * g.d : 0;
   w.dQacc = c.take<float>(acc);
   w.dKacc = c.take<float>(acc);
   w.dVacc = c.take<float>(acc);
@@ -351,6 +390,146 @@ elsaa_status lsh_gather(const elsaa_params* p, const Geom& g, bool bf16, const i
   return ELSAA_OK;
 }
 
+// ---- causal sortLSH: the recursion of the paper's §3.2 on the tensor-core kernels ----
+//
+// Level l (1 .. lsh_levels) cuts the rows into half-segments of h = N >> l rows; the
+// future half's sorted query blocks meet the past half's sorted key blocks.  Each level
+// gathers its sorted rows, runs the sparse kernel alone (no low-rank branch, m held at 1,
+// so its O_s and log d_s are the level's exact partial softmax) and merges that into the
+// running result by log-sum-exp.  The deepest level (halves of one block) needs no sort:
+// it joins the leaves in the base pass, tile t taking block t under the mask j <= i and,
+// for odd t, block t - 1.  The fusion then runs on the merged sparse branch.  In the
+// backward every level's sparse gradient uses the merged log d_s and Delta, so the levels
+// are independent: each one's dQ, dK, dV (sorted order) are added to the fp32
+// accumulators that the base pass folds into its single bf16 rounding.
+
+Geom sparse_only(const Geom& g, bool causal, int k) {
+  Geom s = g;
+  s.r = 0;
+  s.L = 0;
+  s.fixed_m = 1;
+  s.causal = causal ? 1 : 0;
+  s.k = k;
+  return s;
+}
+
+elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void* Q, const void* K, const void* V,
+                                const float* W, const float* lam, const float* gs, const float* glr, void* O,
+                                const Saved& s, const FwdWs& w, cudaStream_t st) {
+  const PermBufs& b = w.pm;
+  const size_t rows = (size_t)g.BH * g.N;
+  const int rb = g.d * 2, stride = 2 * g.N;
+  ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st), "flag reset"));
+  // the low-rank branch, causal, in the caller's row order
+  if (g.r > 0) {
+    ELSAA_TRY(cuda_status(launch_race_features(Q, K, W, w.wsplit, true, s.phiQ, s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, st),
+                          "race features"));
+    ELSAA_TRY(cuda_status(launch_race_state_fwd(s.phiK, V, true, s.Ast, s.Bst, g, st), "race summaries"));
+    FwdArgs ra{Q, K, V, s.idx, s.phiQ, s.phiK, s.Ast, s.Bst, lam, gs, glr, O, s.Os, s.logd, s.dlr, s.m, s.Olr,
+               s.Psplit, s.Pmass};
+    if (s.Psplit) {
+      ELSAA_TRY(cuda_status(launch_race_state_split(s.Ast, s.Bst, false, s.Psplit, s.Pmass, g, st),
+                            "race statistics split"));
+      ELSAA_TRY(cuda_status(launch_race_readout_tc(ra, g, w.flag, st), "tcgen05 race read-out"));
+    } else {
+      ELSAA_TRY(cuda_status(launch_race_readout_bf16(ra, g, st), "race read-out"));
+    }
+  } else {
+    ELSAA_TRY(cuda_status(cudaMemsetAsync(s.Olr, 0, rows * rb, st), "O_lr"));
+    ELSAA_TRY(cuda_status(cudaMemsetAsync(s.dlr, 0, rows * 4, st), "d_lr"));
+  }
+  // sparse-only passes write O_s and log d_s into the level buffers; their fused output
+  // and m are not used (the low-rank input they read is scratch)
+  FwdArgs sa{};
+  sa.idx = s.idx;
+  sa.O = b.X;
+  sa.Olr = b.X;
+  sa.Os = b.Os;
+  sa.logd = b.logd;
+  sa.dlr = b.logd;
+  sa.m = b.m;
+  // base pass: the leaves and the deepest level, in the caller's order
+  const Geom gb = sparse_only(g, true, 2);
+  ELSAA_TRY(cuda_status(launch_causal_lsh_select(s.idx, 0, g, st), "causal sortLSH base selection"));
+  sa.Q = Q; sa.K = K; sa.V = V;
+  ELSAA_TRY(cuda_status(launch_attn_fwd_tc(sa, gb, w.flag, st), "causal sortLSH base pass"));
+  ELSAA_TRY(cuda_status(launch_lsh_merge(b.Os, b.logd, nullptr, 0, b.accO, nullptr, b.accL[0], g, st), "merge"));
+  int cur = 0;
+  if (g.lsh_levels > 0)
+    ELSAA_TRY(cuda_status(launch_sortlsh_hash(Q, K, true, p->lsh_planes, p->lsh_bits, b.pos, nullptr, g, st),
+                          "sortLSH hash"));
+  const Geom gl = sparse_only(g, false, 1);
+  for (int lev = 0; lev < g.lsh_levels; ++lev) {
+    const int h = g.N >> (lev + 1);
+    int* ord = s.lsh_order + (size_t)lev * g.BH * stride;
+    ELSAA_TRY(cuda_status(launch_sortlsh_level_sort(b.pos, ord, h, p->lsh_bits, g, st), "sortLSH level sort"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(Q, b.Q, ord, rb, g, stride, false, st), "sortLSH gather Q"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(K, b.K, ord + g.N, rb, g, stride, false, st), "sortLSH gather K"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(V, b.V, ord + g.N, rb, g, stride, false, st), "sortLSH gather V"));
+    ELSAA_TRY(cuda_status(launch_causal_lsh_select(b.idx, h / g.T, gl, st), "sortLSH level selection"));
+    sa.Q = b.Q; sa.K = b.K; sa.V = b.V; sa.idx = b.idx;
+    ELSAA_TRY(cuda_status(launch_attn_fwd_tc(sa, gl, w.flag, st), "sortLSH level pass"));
+    ELSAA_TRY(cuda_status(launch_lsh_merge(b.Os, b.logd, ord, h, b.accO, b.accL[cur], b.accL[cur ^ 1], g, st),
+                          "merge"));
+    cur ^= 1;
+  }
+  return cuda_status(launch_lsh_fuse(b.accO, b.accL[cur], s.Olr, s.dlr, lam, gs, glr, O, s.Os, s.logd, s.m, g, st),
+                     "fusion");
+}
+
+elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const BwdWs& w, cudaStream_t st) {
+  const PermBufs& b = w.pm;
+  const size_t rows = (size_t)g.BH * g.N;
+  const int rb = g.d * 2, stride = 2 * g.N;
+  ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st), "flag reset"));
+  ELSAA_TRY(cuda_status(launch_row_scalars(a, true, g, st), "row scalars"));
+  if (g.r > 0) {
+    ELSAA_TRY(cuda_status(launch_race_state_bwd(a, true, g, st), "race suffix summaries"));
+    if (race_bwd_tc_supported(g)) {
+      ELSAA_TRY(cuda_status(launch_race_state_split(w.RA, w.RB, true, w.Rsplit, w.Rmass, g, st),
+                            "race statistics split"));
+      ELSAA_TRY(cuda_status(launch_race_w_split(a.W, w.Wsplit, g, st), "W split"));
+      ELSAA_TRY(cuda_status(launch_race_bwd_tc(a, g, w.flag, st), "tcgen05 race backward"));
+    } else {
+      ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, 1, st), "race backward"));
+    }
+  } else {
+    ELSAA_TRY(cuda_status(cudaMemsetAsync(w.dQacc, 0, rows * g.d * 4, st), "dQ accumulator"));
+    ELSAA_TRY(cuda_status(cudaMemsetAsync(w.dKacc, 0, rows * g.d * 4, st), "dK accumulator"));
+    ELSAA_TRY(cuda_status(cudaMemsetAsync(w.dVacc, 0, rows * g.d * 4, st), "dV accumulator"));
+  }
+  const Geom gl = sparse_only(g, false, 1);
+  for (int lev = 0; lev < g.lsh_levels; ++lev) {
+    const int h = g.N >> (lev + 1);
+    const int* ord = s.lsh_order + (size_t)lev * g.BH * stride;
+    ELSAA_TRY(cuda_status(launch_permute_rows(a.Q, b.Q, ord, rb, g, stride, false, st), "sortLSH gather Q"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(a.K, b.K, ord + g.N, rb, g, stride, false, st), "sortLSH gather K"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(a.V, b.V, ord + g.N, rb, g, stride, false, st), "sortLSH gather V"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(a.dO, b.X, ord, rb, g, stride, false, st), "sortLSH gather dO"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(w.rs.packed, b.packed, ord, 16, g, stride, false, st),
+                          "sortLSH gather row scalars"));
+    ELSAA_TRY(cuda_status(launch_causal_lsh_select(b.idx, h / g.T, gl, st), "sortLSH level selection"));
+    ELSAA_TRY(cuda_status(launch_invert_selection(b.idx, w.offs, w.tiles, w.order, gl, st), "selection inverse"));
+    BwdArgs la{};
+    la.Q = b.Q; la.K = b.K; la.V = b.V; la.dO = b.X;
+    la.idx = b.idx; la.offs = w.offs; la.tiles = w.tiles; la.kv_order = w.order;
+    la.rs.packed = b.packed;
+    la.dQ = b.dQ; la.dK = b.dK; la.dV = b.dV;
+    ELSAA_TRY(cuda_status(launch_dq_tc(la, gl, w.flag, st), "sortLSH level dq"));
+    ELSAA_TRY(cuda_status(launch_dkdv_tc(la, gl, w.flag, st), "sortLSH level dkdv"));
+    ELSAA_TRY(cuda_status(launch_lsh_add_rows(b.dQ, w.dQacc, ord, h, true, g, st), "sortLSH dQ"));
+    ELSAA_TRY(cuda_status(launch_lsh_add_rows(b.dK, w.dKacc, ord + g.N, h, false, g, st), "sortLSH dK"));
+    ELSAA_TRY(cuda_status(launch_lsh_add_rows(b.dV, w.dVacc, ord + g.N, h, false, g, st), "sortLSH dV"));
+  }
+  // base pass in the caller's order: adds the accumulators before the single rounding
+  const Geom gb = sparse_only(g, true, 2);
+  ELSAA_TRY(cuda_status(launch_invert_selection(s.idx, w.offs, w.tiles, w.order, gb, st), "selection inverse"));
+  a.idx = s.idx; a.offs = w.offs; a.tiles = w.tiles; a.kv_order = w.order;
+  a.dQacc = w.dQacc; a.dKacc = w.dKacc; a.dVacc = w.dVacc;
+  ELSAA_TRY(cuda_status(launch_dq_tc(a, gb, w.flag, st), "causal sortLSH base dq"));
+  return cuda_status(launch_dkdv_tc(a, gb, w.flag, st), "causal sortLSH base dkdv");
+}
+
 extern "C" {
 
 elsaa_status elsaa_profile_begin(void) {
@@ -440,6 +619,11 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
   Saved s = carve_saved(saved, g, bf16 ? 2 : 4, &sb);
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
   const bool lsh = g.selector == ELSAA_SEL_SORTLSH;
+  if (lsh && g.causal) {
+    ELSAA_TRY(check_ptr(p->lsh_planes, "lsh_planes"));
+    if (tcgen05_disabled()) return fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH runs on the tcgen05 kernels only");
+    return causal_lsh_forward(p, g, Q, K, V, W, lam, gs, glr, O, s, w, st_);
+  }
   void* O_out = O;
   if (lsh) {
     // the operator runs on the sorted rows (non-causal RACE, the fusion and diagonal-block
@@ -511,6 +695,22 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   Saved s = carve_saved(const_cast<void*>(saved), g, bf16 ? 2 : 4, &sb);
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
   const bool lsh = g.selector == ELSAA_SEL_SORTLSH;
+  if (lsh && g.causal) {
+    if (tcgen05_disabled()) return fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH runs on the tcgen05 kernels only");
+    BwdArgs a{};
+    a.Q = Q; a.K = K; a.V = V; a.dO = dO; a.W = W;
+    a.lam = lam; a.gs = gs; a.glr = glr;
+    a.logd = s.logd; a.dlr = s.dlr; a.m = s.m;
+    a.Os = s.Os; a.Olr = s.Olr; a.phiQ = s.phiQ; a.phiK = s.phiK;
+    a.hQ = s.hQ; a.hK = s.hK; a.nQ = s.nQ; a.nK = s.nK;
+    a.Ast = s.Ast; a.Bst = s.Bst; a.RA = w.RA; a.RB = w.RB;
+    a.rs = w.rs;
+    a.dQacc = w.dQacc; a.dKacc = w.dKacc; a.dVacc = w.dVacc;
+    a.dOcl = g.r > 0 ? w.dOcl : nullptr;
+    a.Psplit = s.Psplit; a.Pmass = s.Pmass; a.Rsplit = w.Rsplit; a.Rmass = w.Rmass; a.Wsplit = w.Wsplit;
+    a.dQ = dQ; a.dK = dK; a.dV = dV;
+    return causal_lsh_backward(g, a, s, w, st_);
+  }
   void *dQ_out = dQ, *dK_out = dK, *dV_out = dV;
   if (lsh) {
     // the forward ran on the sorted rows and saved its state in that order; so does this,
@@ -589,7 +789,9 @@ elsaa_status elsaa_fusion_grads(const elsaa_params* p, const float* lam, const f
   Saved s = carve_saved(const_cast<void*>(saved), g, bf16 ? 2 : 4, &sb);
   if (!dlam && !dgs && !dglr) return ELSAA_OK;
   // sortLSH: the saved state is in the sorted query order; each row maps back through it
-  return cuda_status(launch_fusion_grads(dO, s.Os, s.Olr, s.logd, s.dlr, lam, gs, glr, dlam, dgs, dglr, s.lsh_order,
+  // (the causal recursion fuses in the caller's order)
+  const int* perm = g.selector == ELSAA_SEL_SORTLSH && !g.causal ? s.lsh_order : nullptr;
+  return cuda_status(launch_fusion_grads(dO, s.Os, s.Olr, s.logd, s.dlr, lam, gs, glr, dlam, dgs, dglr, perm,
                                          2 * g.N, bf16, g, static_cast<cudaStream_t>(stream)),
                      "fusion gradients");
 }

@@ -66,6 +66,21 @@ struct BwdArgs {
 cudaError_t launch_sortlsh_order(const void* Q, const void* K, bool bf16, const float* planes, int bits,
                                  int* order, int* codes, const Geom& g, cudaStream_t st);
 size_t sortlsh_smem_bytes(const Geom& g, int bits);
+// Hash only: Gray positions (and, if not null, codes) [BH][2][N].
+cudaError_t launch_sortlsh_hash(const void* Q, const void* K, bool bf16, const float* planes, int bits, int* pos,
+                                int* codes, const Geom& g, cudaStream_t st);
+// Causal recursion: one level's orders [BH][2][N] (queries sorted in the future halves,
+// keys in the past halves of h rows; identity elsewhere); the base / level selections;
+// the log-sum-exp merge of sparse partials; the final fusion; fp32 row scatter-add.
+cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int h, int bits, const Geom& g, cudaStream_t st);
+cudaError_t launch_causal_lsh_select(int* idx, int hb, const Geom& g, cudaStream_t st);
+cudaError_t launch_lsh_merge(const void* Os, const float* logd, const int* perm, int h, float* accO,
+                             const float* accL_in, float* accL_out, const Geom& g, cudaStream_t st);
+cudaError_t launch_lsh_fuse(const float* accO, const float* accL, const void* Olr, const float* dlr, const float* lam,
+                            const float* gs, const float* glr, void* O, void* Os, float* logd, float* m, const Geom& g,
+                            cudaStream_t st);
+cudaError_t launch_lsh_add_rows(const void* src, float* acc, const int* perm, int h, bool future, const Geom& g,
+                                cudaStream_t st);
 // Row permutation of [BH][N] rows of row_bytes (a multiple of 16): gather dst[r] = src[perm[r]]
 // or scatter dst[perm[r]] = src[r]; perm advances by perm_stride per head.
 cudaError_t launch_permute_rows(const void* src, void* dst, const int* perm, int row_bytes, const Geom& g,

@@ -107,24 +107,17 @@ __global__ void __launch_bounds__(256) sortlsh_hash_kernel(const E* __restrict__
   }
 }
 
-// Stable sort of one (head, side) by Gray position, in shared memory: least-significant
-// digit first, 8 bits per pass, each pass a counting sort.  Items are packed
-// (position << 14 | row), so rows need N <= 16384.  Warp w owns the rows of the w-th
-// contiguous slice; counts are kept per (digit, warp) and scanned digit-major, warp-minor,
-// and within a warp equal digits are ranked by lane (match_any), which keeps every pass
-// stable.  Reads its `order` segment (the positions) whole before writing the sorted rows
-// over it.
-__global__ void __launch_bounds__(kSortThreads) sortlsh_sort_kernel(int* __restrict__ order, int bits, Geom g) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  int* cnt = reinterpret_cast<int*>(smem);                          // [256 digits][32 warps]
-  uint32_t* bufA = reinterpret_cast<uint32_t*>(cnt + 256 * 32);
-  uint32_t* bufB = bufA + g.N;
-  __shared__ int wsum[32];
-  int* seg = order + ((size_t)blockIdx.x * 2 + blockIdx.y) * g.N;
+// Stable sort of n items by Gray position, in shared memory: least-significant digit
+// first, 8 bits per pass, each pass a counting sort.  Items are packed
+// (position << 14 | local row), so n <= 16384.  Warp w owns the rows of the w-th
+// contiguous slice; counts are kept per (digit, warp) and scanned digit-major,
+// warp-minor, and within a warp equal digits are ranked by lane (match_any), which
+// keeps every pass stable.  `bufA` holds the items on entry; returns the buffer that
+// holds them sorted.  Called by all kSortThreads threads.
+__device__ uint32_t* block_counting_sort(uint32_t* bufA, uint32_t* bufB, int* cnt, int* wsum, int n, int bits) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < g.N; i += kSortThreads) bufA[i] = ((uint32_t)seg[i] << 14) | (uint32_t)i;
-  const int slice = (g.N + 31) / 32;
-  const int r0 = warp * slice, r1 = min(g.N, r0 + slice);
+  const int slice = (n + 31) / 32;
+  const int r0 = warp * slice, r1 = min(n, r0 + slice);
   uint32_t* src = bufA;
   uint32_t* dst = bufB;
   for (int shift = 0; shift < bits; shift += 8) {
@@ -194,7 +187,177 @@ __global__ void __launch_bounds__(kSortThreads) sortlsh_sort_kernel(int* __restr
     src = dst;
     dst = t;
   }
-  for (int i = tid; i < g.N; i += kSortThreads) seg[i] = (int)(src[i] & 0x3fffu);
+  return src;
+}
+
+// One (head, side) per CTA, grid (BH, 2): reads its `order` segment (the Gray
+// positions) whole, then writes the sorted rows over it.
+__global__ void __launch_bounds__(kSortThreads) sortlsh_sort_kernel(int* __restrict__ order, int bits, Geom g) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  int* cnt = reinterpret_cast<int*>(smem);                          // [256 digits][32 warps]
+  uint32_t* bufA = reinterpret_cast<uint32_t*>(cnt + 256 * 32);
+  uint32_t* bufB = bufA + g.N;
+  __shared__ int wsum[32];
+  int* seg = order + ((size_t)blockIdx.x * 2 + blockIdx.y) * g.N;
+  for (int i = threadIdx.x; i < g.N; i += kSortThreads) bufA[i] = ((uint32_t)seg[i] << 14) | (uint32_t)i;
+  const uint32_t* out = block_counting_sort(bufA, bufB, cnt, wsum, g.N, bits);
+  for (int i = threadIdx.x; i < g.N; i += kSortThreads) seg[i] = (int)(out[i] & 0x3fffu);
+}
+
+// Causal recursion, one level: rows are cut into half-segments of h rows (a past half
+// 2s and a future half 2s + 1 per segment).  grid (BH, 2, N / 2h): side 0 sorts the
+// queries of future half 2s + 1, side 1 the keys of past half 2s, by Gray position
+// (stable); the other half of each side's order is the identity.  pos and order are
+// [BH][2][N]; order holds row indices.
+__global__ void __launch_bounds__(kSortThreads) sortlsh_level_sort_kernel(const int* __restrict__ pos,
+                                                                          int* __restrict__ order, int h, int bits,
+                                                                          Geom g) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  int* cnt = reinterpret_cast<int*>(smem);
+  uint32_t* bufA = reinterpret_cast<uint32_t*>(cnt + 256 * 32);
+  uint32_t* bufB = bufA + h;
+  __shared__ int wsum[32];
+  const int side = blockIdx.y, s = blockIdx.z;
+  const size_t off = ((size_t)blockIdx.x * 2 + side) * g.N;
+  const int sorted0 = (2 * s + (side == 0 ? 1 : 0)) * h;       // first row of the half this CTA sorts
+  const int ident0 = (2 * s + (side == 0 ? 0 : 1)) * h;
+  for (int i = threadIdx.x; i < h; i += kSortThreads) {
+    bufA[i] = ((uint32_t)pos[off + sorted0 + i] << 14) | (uint32_t)i;
+    order[off + ident0 + i] = ident0 + i;
+  }
+  const uint32_t* out = block_counting_sort(bufA, bufB, cnt, wsum, h, bits);
+  for (int i = threadIdx.x; i < h; i += kSortThreads) order[off + sorted0 + i] = sorted0 + (int)(out[i] & 0x3fffu);
+}
+
+// Selections of the causal recursion.  Base pass (the caller's row order, causal): tile
+// t takes its own block and, when t is odd, block t - 1 (the deepest level, whose halves
+// are single blocks and need no sort); ascending, -1 padded, k = 2.  Level with halves
+// of hb blocks (sorted rows): a tile in a future half takes the block hb before it, a
+// tile in a past half takes none; k = 1.
+__global__ void causal_lsh_select_kernel(int* __restrict__ idx, int hb, Geom g) {
+  const size_t total = (size_t)g.BH * g.n_t;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const int t = (int)(e % g.n_t);
+    if (hb == 0) {
+      idx[2 * e] = (t & 1) ? t - 1 : t;
+      idx[2 * e + 1] = (t & 1) ? t : -1;
+    } else {
+      idx[e] = ((t / hb) & 1) ? t - hb : -1;
+    }
+  }
+}
+
+// Sparse partial results into the running fp32 (O_s, log d_s) of the caller's rows.
+// src: bf16 normalised O_s and its log d_s, in sorted order (perm = query order) or in
+// row order (perm null).  h = 0 initialises every row; h > 0 merges the rows at
+// future-half positions of that level by log-sum-exp and carries the others' log d_s
+// over.  The log-denominators are double-buffered (accL_in -> accL_out) so every thread
+// of a row reads the old value.  One thread per 8 columns.
+__global__ void lsh_merge_kernel(const __nv_bfloat16* __restrict__ Os, const float* __restrict__ logd,
+                                 const int* __restrict__ perm, int h, float* __restrict__ accO,
+                                 const float* __restrict__ accL_in, float* __restrict__ accL_out, Geom g) {
+  const int units = g.d / 8;
+  const size_t total = (size_t)g.BH * g.N * units;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t p = e / units;
+    const int u = (int)(e % units);
+    const int bh = (int)(p / g.N), pr = (int)(p % g.N);
+    const size_t row = (size_t)bh * g.N + (perm ? perm[(size_t)bh * 2 * g.N + pr] : pr);
+    const float l = logd[p];
+    const float a = h > 0 ? accL_in[row] : -INFINITY;
+    if (h > 0 && (((pr / h) & 1) == 0 || l == -INFINITY)) {      // nothing from this level
+      if (u == 0) accL_out[row] = a;
+      continue;
+    }
+    const uint4 w = *reinterpret_cast<const uint4*>(Os + p * g.d + 8 * u);
+    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
+    float4* acc = reinterpret_cast<float4*>(accO + row * g.d + 8 * u);
+    float x[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(hv[j]);
+      x[2 * j] = f.x;
+      x[2 * j + 1] = f.y;
+    }
+    if (h == 0) {
+      if (u == 0) accL_out[row] = l;
+      acc[0] = make_float4(x[0], x[1], x[2], x[3]);
+      acc[1] = make_float4(x[4], x[5], x[6], x[7]);
+      continue;
+    }
+    const float L = a == -INFINITY ? l : fmaxf(a, l) + log1pf(__expf(-fabsf(a - l)));
+    const float wa = a == -INFINITY ? 0.f : __expf(a - L), wl = __expf(l - L);
+    const float4 a0 = acc[0], a1 = acc[1];
+    acc[0] = make_float4(wa * a0.x + wl * x[0], wa * a0.y + wl * x[1], wa * a0.z + wl * x[2], wa * a0.w + wl * x[3]);
+    acc[1] = make_float4(wa * a1.x + wl * x[4], wa * a1.y + wl * x[5], wa * a1.z + wl * x[6], wa * a1.w + wl * x[7]);
+    if (u == 0) accL_out[row] = L;
+  }
+}
+
+// Fusion (Eq. 5 weight, Eq. 4 output) of the merged sparse branch with the low-rank
+// branch, per row: m = 1 / (1 + (lambda d_lr + eps) e^{-log d_s}) (1 when m is held),
+// O = g_s m O_s + g_lr O_lr with g_lr = 1 - m by default (1 when m is held).  Writes O,
+// the saved bf16 O_s, log d_s and m.  One thread per 8 columns.
+__global__ void lsh_fuse_kernel(const float* __restrict__ accO, const float* __restrict__ accL,
+                                const __nv_bfloat16* __restrict__ Olr, const float* __restrict__ dlr,
+                                const float* lamv, const float* gsv, const float* glrv, __nv_bfloat16* __restrict__ O,
+                                __nv_bfloat16* __restrict__ Os, float* __restrict__ logd_out, float* __restrict__ m_out,
+                                Geom g) {
+  const int units = g.d / 8;
+  const size_t total = (size_t)g.BH * g.N * units;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t row = e / units;
+    const int u = (int)(e % units);
+    const float l = accL[row];
+    const float lam = lamv ? lamv[row] : g.lam;
+    const float gs = gsv ? gsv[row] : 1.f;
+    const float mf = g.fixed_m ? 1.f : l == -INFINITY ? 0.f : 1.f / (1.f + (lam * dlr[row] + g.eps) * __expf(-l));
+    const float gl = glrv ? glrv[row] : g.fixed_m ? 1.f : 1.f - mf;
+    const float cs = gs * mf;
+    const float4 a0 = reinterpret_cast<const float4*>(accO + row * g.d + 8 * u)[0];
+    const float4 a1 = reinterpret_cast<const float4*>(accO + row * g.d + 8 * u)[1];
+    const float s[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const uint4 w = *reinterpret_cast<const uint4*>(Olr + row * g.d + 8 * u);
+    const __nv_bfloat162* lv = reinterpret_cast<const __nv_bfloat162*>(&w);
+    uint32_t wo[4], ws[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(lv[j]);
+      const __nv_bfloat162 o = __floats2bfloat162_rn(cs * s[2 * j] + gl * f.x, cs * s[2 * j + 1] + gl * f.y);
+      const __nv_bfloat162 q = __floats2bfloat162_rn(s[2 * j], s[2 * j + 1]);
+      wo[j] = *reinterpret_cast<const uint32_t*>(&o);
+      ws[j] = *reinterpret_cast<const uint32_t*>(&q);
+    }
+    *reinterpret_cast<uint4*>(O + row * g.d + 8 * u) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
+    *reinterpret_cast<uint4*>(Os + row * g.d + 8 * u) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+    if (u == 0) {
+      logd_out[row] = l;
+      m_out[row] = mf;
+    }
+  }
+}
+
+// acc[perm[p]] += src[p] (bf16 rows into fp32 rows) for the positions p in the future
+// halves (future = 1) or the past halves (future = 0) of a level with halves of h rows.
+__global__ void lsh_add_rows_kernel(const __nv_bfloat16* __restrict__ src, float* __restrict__ acc,
+                                    const int* __restrict__ perm, int h, int future, Geom g) {
+  const int units = g.d / 8;
+  const size_t total = (size_t)g.BH * g.N * units;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t p = e / units;
+    const int u = (int)(e % units);
+    const int bh = (int)(p / g.N), pr = (int)(p % g.N);
+    if (((pr / h) & 1) != future) continue;
+    const size_t row = (size_t)bh * g.N + perm[(size_t)bh * 2 * g.N + pr];
+    const uint4 w = *reinterpret_cast<const uint4*>(src + p * g.d + 8 * u);
+    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
+    float4* a = reinterpret_cast<float4*>(acc + row * g.d + 8 * u);
+    const float2 f0 = __bfloat1622float2(hv[0]), f1 = __bfloat1622float2(hv[1]);
+    const float2 f2 = __bfloat1622float2(hv[2]), f3 = __bfloat1622float2(hv[3]);
+    const float4 a0 = a[0], a1 = a[1];
+    a[0] = make_float4(a0.x + f0.x, a0.y + f0.y, a0.z + f1.x, a0.w + f1.y);
+    a[1] = make_float4(a1.x + f2.x, a1.y + f2.y, a1.z + f3.x, a1.w + f3.y);
+  }
 }
 
 // Rows of 16-byte units: dst[r] = src[perm[r]] (gather) or dst[perm[r]] = src[r]
@@ -240,29 +403,73 @@ size_t sortlsh_smem_bytes(const Geom& g, int bits) {
   return (size_t)256 * 32 * 4 + (size_t)2 * g.N * 4;
 }
 
-cudaError_t launch_sortlsh_order(const void* Q, const void* K, bool bf16, const float* planes, int bits,
-                                 int* order, int* codes, const Geom& g, cudaStream_t st) {
+cudaError_t launch_sortlsh_hash(const void* Q, const void* K, bool bf16, const float* planes, int bits, int* pos,
+                                int* codes, const Geom& g, cudaStream_t st) {
   const size_t hsmem = (size_t)bits * g.d * 4;
-  // about eight blocks of 256 threads per SM over all segments
   const int per_seg_max = (g.N + 8 * 4 * kHashRows - 1) / (8 * 4 * kHashRows);   // one iteration each
   const int per_seg = std::max(1, std::min(per_seg_max, (148 * 8 + 2 * g.BH - 1) / (2 * g.BH)));
   const dim3 hgrid(per_seg, 2 * g.BH);
-  {
-    ProfScope ps("sortlsh_hash", st);
-    auto run = [&](auto kern, const auto* q, const auto* k) {
-      kern<<<hgrid, 256, hsmem, st>>>(q, k, planes, bits, order, codes, g);
-    };
-    const auto* q16 = (const __nv_bfloat16*)Q;
-    const auto* k16 = (const __nv_bfloat16*)K;
-    const auto* q32 = (const float*)Q;
-    const auto* k32 = (const float*)K;
-    if (bf16 && g.d == 128) run(sortlsh_hash_kernel<__nv_bfloat16, 16>, q16, k16);
-    else if (bf16) run(sortlsh_hash_kernel<__nv_bfloat16, 8>, q16, k16);
-    else if (g.d == 128) run(sortlsh_hash_kernel<float, 16>, q32, k32);
-    else run(sortlsh_hash_kernel<float, 8>, q32, k32);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
+  ProfScope ps("sortlsh_hash", st);
+  auto run = [&](auto kern, const auto* q, const auto* k) {
+    kern<<<hgrid, 256, hsmem, st>>>(q, k, planes, bits, pos, codes, g);
+  };
+  const auto* q16 = (const __nv_bfloat16*)Q;
+  const auto* k16 = (const __nv_bfloat16*)K;
+  const auto* q32 = (const float*)Q;
+  const auto* k32 = (const float*)K;
+  if (bf16 && g.d == 128) run(sortlsh_hash_kernel<__nv_bfloat16, 16>, q16, k16);
+  else if (bf16) run(sortlsh_hash_kernel<__nv_bfloat16, 8>, q16, k16);
+  else if (g.d == 128) run(sortlsh_hash_kernel<float, 16>, q32, k32);
+  else run(sortlsh_hash_kernel<float, 8>, q32, k32);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int h, int bits, const Geom& g, cudaStream_t st) {
+  const size_t smem = (size_t)256 * 32 * 4 + (size_t)2 * h * 4;
+  cudaError_t e = cudaFuncSetAttribute(sortlsh_level_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  ProfScope ps("sortlsh_level_sort", st);
+  sortlsh_level_sort_kernel<<<dim3(g.BH, 2, g.N / (2 * h)), kSortThreads, smem, st>>>(pos, order, h, bits, g);
+  return cudaGetLastError();
+}
+
+static int elementwise_blocks(size_t total) { return (int)std::min<size_t>((total + 255) / 256, 148 * 16); }
+
+cudaError_t launch_causal_lsh_select(int* idx, int hb, const Geom& g, cudaStream_t st) {
+  causal_lsh_select_kernel<<<elementwise_blocks((size_t)g.BH * g.n_t), 256, 0, st>>>(idx, hb, g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lsh_merge(const void* Os, const float* logd, const int* perm, int h, float* accO,
+                             const float* accL_in, float* accL_out, const Geom& g, cudaStream_t st) {
+  ProfScope ps("lsh_merge", st);
+  lsh_merge_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
+      (const __nv_bfloat16*)Os, logd, perm, h, accO, accL_in, accL_out, g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lsh_fuse(const float* accO, const float* accL, const void* Olr, const float* dlr, const float* lam,
+                            const float* gs, const float* glr, void* O, void* Os, float* logd, float* m, const Geom& g,
+                            cudaStream_t st) {
+  ProfScope ps("lsh_fuse", st);
+  lsh_fuse_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
+      accO, accL, (const __nv_bfloat16*)Olr, dlr, lam, gs, glr, (__nv_bfloat16*)O, (__nv_bfloat16*)Os, logd, m, g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lsh_add_rows(const void* src, float* acc, const int* perm, int h, bool future, const Geom& g,
+                                cudaStream_t st) {
+  ProfScope ps("lsh_add_rows", st);
+  lsh_add_rows_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
+      (const __nv_bfloat16*)src, acc, perm, h, future ? 1 : 0, g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sortlsh_order(const void* Q, const void* K, bool bf16, const float* planes, int bits,
+                                 int* order, int* codes, const Geom& g, cudaStream_t st) {
+  const cudaError_t eh = launch_sortlsh_hash(Q, K, bf16, planes, bits, order, codes, g, st);
+  if (eh != cudaSuccess) return eh;
   const size_t smem = sortlsh_smem_bytes(g, bits);
   cudaError_t e = cudaFuncSetAttribute(sortlsh_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

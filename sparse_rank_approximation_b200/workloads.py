@@ -81,6 +81,9 @@ WORKLOADS = {
     # 128 blocks of 128 rows
     "n16k_d128_sortlsh": Workload("n16k_d128_sortlsh", 1, 32, 16384, 128, "bf16", False, 128, 128, 1,
                                   n_centroids=256, sigma=0.5, selector="sortlsh", lsh_bits=7),
+    # the headline shape with the causal sortLSH recursion (halves down to single blocks)
+    "n16k_d128_sortlsh_causal": Workload("n16k_d128_sortlsh_causal", 1, 32, 16384, 128, "bf16", True, 128, 128, 2,
+                                         n_centroids=256, sigma=0.5, selector="sortlsh", lsh_bits=7),
     "n64k_d128": Workload("n64k_d128", 1, 8, 65536, 128, "bf16", True, 256, 128, 32,
                           n_centroids=512, sigma=0.3),
 }

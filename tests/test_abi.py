@@ -85,3 +85,25 @@ def test_status_strings():
     for s in range(6):
         assert L.elsaa_status_string(s)
     assert L.elsaa_status_string(99) == b"unknown status"
+
+
+def test_sortlsh_shape_limits():
+    """sortLSH: non-causal up to N = 16384 on every path; the causal recursion needs the
+    tensor-core shape (bf16, d = 128, block 128), a power-of-two block count and N <= 32768."""
+    L = bd.lib()
+    ok = dict(selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=6, topk=1)
+    assert L.elsaa_saved_bytes(ctypes.byref(bd.make_params(1, 2, 16384, 64, block_size=64, rank_r=16, causal=False,
+                                                           **ok))) > 0
+    assert L.elsaa_saved_bytes(ctypes.byref(bd.make_params(1, 2, 16384, 128, block_size=128, rank_r=128, causal=True,
+                                                           **ok))) > 0
+    bad = [dict(N=32768, d=64, block_size=64, causal=False),
+           dict(N=512, d=64, block_size=64, causal=True),
+           dict(N=128 * 6, d=128, block_size=128, causal=True),
+           dict(N=1024, d=128, block_size=128, causal=True, dtype=bd.ELSAA_DTYPE_F32),
+           dict(N=65536, d=128, block_size=128, causal=True)]
+    for kw in bad:
+        p = bd.make_params(1, 1, kw.pop("N"), kw.pop("d"), rank_r=128 if kw["block_size"] == 128 else 16, **kw, **ok)
+        assert L.elsaa_saved_bytes(ctypes.byref(p)) == 0, kw
+    p = bd.make_params(1, 1, 1024, 128, block_size=128, rank_r=128, causal=True, selector=bd.ELSAA_SEL_SORTLSH,
+                       lsh_bits=17, topk=1)
+    assert L.elsaa_saved_bytes(ctypes.byref(p)) == 0

@@ -102,17 +102,6 @@ def test_forward_backward(geom, gates, fixed_m):
         check_fusion_grads(w, h, p, fw, ex, get("dO"), (dl, dgs, dgl), ref)
 
 
-def test_rejects_causal_and_oversize():
-    L = bd.lib()
-    import ctypes
-    p = bd.make_params(1, 1, 512, 64, block_size=64, topk=1, rank_r=16, causal=True,
-                       selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=8)
-    assert L.elsaa_saved_bytes(ctypes.byref(p)) == 0
-    p = bd.make_params(1, 1, 32768, 64, block_size=64, topk=1, rank_r=16, causal=False,
-                       selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=8)
-    assert L.elsaa_saved_bytes(ctypes.byref(p)) == 0
-
-
 def _sparse_rounding_scales(q, k, v, dO, fw, p):
     """Per-element scales of the bf16 rounding inside the sparse backward, from the oracle's
     own quantities: dS is rounded before dS K and dS^T Q, P before P^T dO_s, and Delta is a
@@ -123,7 +112,7 @@ def _sparse_rounding_scales(q, k, v, dO, fw, p):
     Delta = (dOs * fw["O_s"]).sum(axis=1) - dds_ds
     eD = (np.abs(dOs) * np.abs(fw["O_s"])).sum(axis=1)
     Bq, Bk, Bv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
-    for i, keys in enumerate(orc.sortlsh_support(q, k, p)):
+    for i, keys in enumerate(orc.lsh_support(q, k, p)):
         P = np.exp(p.scale * (k[keys] @ q[i]) - fw["logd_s"][i])
         dz = np.abs(P * (v[keys] @ dOs[i] - Delta[i])) + P * eD[i]
         Bq[i] += p.scale * dz @ np.abs(k[keys])
@@ -154,6 +143,92 @@ def test_full_size():
         # the gradients: the usual bf16 bound plus the rounding inside the sparse backward
         # (twice its half-ulp scale); at this length sorted blocks put most of a row's
         # mass on a few keys, where the Delta term dominates
+        scales = _sparse_rounding_scales(get("Q"), get("K"), get("V"), get("dO"), fw, p)
+        for name, got, ref, B in zip(("dQ", "dK", "dV"), (dQ, dK, dV), (dq, dk, dv), scales):
+            err = np.abs(np64(got[0, h]) - ref)
+            excess = (err - BF16_STORE_REL * np.abs(ref) - 2.0 ** -8 * B).max()
+            assert excess <= BF16_ABS_TOL, f"{name}[{h}]: max err {err.max():.3e}, beyond the bound {excess:.3e}"
+
+
+# ---- the causal recursion (bf16, d = 128, block 128 on the tensor-core kernels) ----
+
+def _causal_setup(N, r, seed, fixed_m=False, bits=6, H=2):
+    w = small_workload(N=N, d=128, block_size=128, topk=2, rank_r=r, causal=True, dtype="bf16", H=H)
+    inp = make_inputs(w, seed)
+    dev = device_inputs(w, inp)
+    g = torch.Generator().manual_seed(seed + 7)
+    R = torch.randn(w.d, bits, generator=g)
+    op = gpu_op(w, fixed_m=fixed_m, selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=bits, lsh_planes=R.cuda())
+    return w, inp, dev, R, op
+
+
+def _causal_oracle_params(w, R, codes, h, fixed_m=False):
+    p = oracle_params(w, fixed_m=fixed_m)
+    p.selector = "sortlsh"
+    p.lsh_planes = R.double().numpy()
+    p.lsh_codes = (codes[0, h, 0].cpu().numpy(), codes[0, h, 1].cpu().numpy())
+    return p
+
+
+@pytest.mark.parametrize("N,r,gates,fixed_m", [(1024, 128, False, False), (1024, 128, True, False),
+                                               (2048, 64, False, False), (1024, 0, False, False),
+                                               (1024, 128, True, True), (128, 128, False, False),
+                                               (256, 128, False, False)])
+def test_causal_forward_backward(N, r, gates, fixed_m):
+    """O, dQ, dK, dV and the fusion gradients against the oracle's recursion run on the GPU's
+    hash codes (every level's sorted order follows from them); N = 128 and 256 are the
+    single-block and two-block cases (exact causal attention)."""
+    w, inp, dev, R, op = _causal_setup(N, r, seed=3, fixed_m=fixed_m)
+    BH = (w.B, w.H, w.N)
+    g = torch.Generator().manual_seed(13)
+    extra = {}
+    if gates:
+        extra = {"lam": torch.rand(BH, generator=g) * 2.0, "g_s": torch.rand(BH, generator=g),
+                 "g_lr": torch.rand(BH, generator=g)}
+    ex_dev = {k: v.cuda() for k, v in extra.items()}
+    O = op.forward(dev["Q"], dev["K"], dev["V"], dev["W"], ex_dev.get("lam"), ex_dev.get("g_s"), ex_dev.get("g_lr"))
+    dQ, dK, dV = op.backward(dev["Q"], dev["K"], dev["V"], dev["W"], dev["dO"], ex_dev.get("lam"),
+                             ex_dev.get("g_s"), ex_dev.get("g_lr"))
+    dl, dgs, dgl = op.fusion_grads(dev["dO"], ex_dev.get("lam"), ex_dev.get("g_s"), ex_dev.get("g_lr"))
+    codes, _ = op.debug_sortlsh(dev["Q"], dev["K"])
+    op.check_device_flags()
+    torch.cuda.synchronize()
+    W = inp["W"].double().numpy()
+    for h in range(w.H):
+        p = _causal_oracle_params(w, R, codes, h, fixed_m)
+        get = lambda n: inp[n][0, h].double().numpy()
+        ex = {k: v[0, h].double().numpy() for k, v in extra.items()}
+        fw = orc.forward_head(get("Q"), get("K"), get("V"), W, p, ex.get("lam"), ex.get("g_s"), ex.get("g_lr"))
+        dq, dk, dv = orc.backward_head(get("Q"), get("K"), get("V"), W, get("dO"), fw, p, ex.get("lam"),
+                                       ex.get("g_s"), ex.get("g_lr"))
+        check(w, f"O[{h}]", np64(O[0, h]), fw["O"])
+        check(w, f"dQ[{h}]", np64(dQ[0, h]), dq)
+        check(w, f"dK[{h}]", np64(dK[0, h]), dk)
+        check(w, f"dV[{h}]", np64(dV[0, h]), dv)
+        ref = orc.fusion_param_grads(get("dO"), fw, p, ex.get("lam"), ex.get("g_s"), ex.get("g_lr"))
+        check_fusion_grads(w, h, p, fw, ex, get("dO"), (dl, dgs, dgl), ref)
+
+
+def test_causal_full_size():
+    """The full-length causal sortLSH workload (B1 H32 N16384 d128, 7-bit codes, six sorted
+    levels), launched as the benchmark launches it; every row of two heads."""
+    w = WORKLOADS["n16k_d128_sortlsh_causal"]
+    inp = make_inputs(w, 0)
+    dev = device_inputs(w, inp)
+    R = inp["R"]
+    op = gpu_op(w, selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=w.lsh_bits, lsh_planes=R.cuda())
+    O = op.forward(dev["Q"], dev["K"], dev["V"], dev["W"])
+    dQ, dK, dV = op.backward(dev["Q"], dev["K"], dev["V"], dev["W"], dev["dO"])
+    codes, _ = op.debug_sortlsh(dev["Q"], dev["K"])
+    op.check_device_flags()
+    torch.cuda.synchronize()
+    W = inp["W"].double().numpy()
+    for h in (0, w.H - 1):
+        get = lambda n: inp[n][0, h].double().numpy()
+        p = _causal_oracle_params(w, R, codes, h)
+        fw = orc.forward_head(get("Q"), get("K"), get("V"), W, p)
+        dq, dk, dv = orc.backward_head(get("Q"), get("K"), get("V"), W, get("dO"), fw, p)
+        check(w, f"O[{h}]", np64(O[0, h]), fw["O"])
         scales = _sparse_rounding_scales(get("Q"), get("K"), get("V"), get("dO"), fw, p)
         for name, got, ref, B in zip(("dQ", "dK", "dV"), (dQ, dK, dV), (dq, dk, dv), scales):
             err = np.abs(np64(got[0, h]) - ref)
