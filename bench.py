@@ -206,10 +206,19 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(use), "in_window": bool(inside)}
 
 
-def kernel_sources_hash():
+# the sources each profiled kernel is compiled from (its file and the headers it includes)
+KERNEL_SOURCES = {
+    "dkdv_tc": ("bwd_tc.cu", "tc_common.cuh", "common.cuh", "kernels.h"),
+    "dq_tc": ("bwd_tc.cu", "tc_common.cuh", "common.cuh", "kernels.h"),
+    "attn_fwd_tc": ("attn_fwd_tc.cu", "tc_common.cuh", "common.cuh", "kernels.h"),
+    "race_k_bwd_tc": ("race_tc.cu", "tc_common.cuh", "common.cuh", "kernels.h"),
+}
+
+
+def kernel_sources_hash(kernel: str):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_rank_approximation_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in KERNEL_SOURCES.get(kernel, sorted(os.listdir(csrc))):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -221,7 +230,7 @@ def dram_traffic(kernel: str, workload: str):
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
-    src = kernel_sources_hash()
+    src = kernel_sources_hash(kernel)
     for line in open(path):
         parts = line.split()
         if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload \

@@ -192,12 +192,14 @@ Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
 struct PermBufs {
   void *Q, *K, *V, *X, *dQ, *dK, *dV;     // X: O (forward) or dO (backward)
   float *lam, *gs, *glr;
-  // causal recursion: a level's O_s and log d_s (sorted order), the running fp32 sparse
-  // result (caller's order, log-denominators double-buffered), a level's selection, the
-  // Gray positions and the sorted rows' packed backward scalars
-  void* Os;
-  float *accO, *logd, *m, *accL[2];
-  int *idx, *pos;
+  // causal recursion.  Forward: the base pass's O_s, log d_s (and a scratch m), every
+  // level's partial O_s and log d_s in its sorted order ([levels][BH][N][d], [levels][BH][N])
+  // with the future-half rows' positions ([levels][BH][N]), the Gray positions.
+  // Backward: dQ, dK, dV hold every level's gradients ([levels][BH][N][d]), inv the
+  // orders' inverses ([levels][BH][2][N]), packed the sorted rows' backward scalars.
+  void *Os, *Os_lv;
+  float *logd, *m, *logd_lv;
+  int *idx, *pos, *inv;
   float4* packed;
 };
 
@@ -205,14 +207,15 @@ PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
   PermBufs b{};
   if (g.selector != ELSAA_SEL_SORTLSH) return b;
   const size_t rows = (size_t)g.BH * g.N, mat = rows * g.d * esz;
+  const size_t lv = g.causal ? (size_t)g.lsh_levels : 1;
   b.Q = c.take<char>(mat);
   b.K = c.take<char>(mat);
   b.V = c.take<char>(mat);
   b.X = c.take<char>(mat);
   if (backward) {
-    b.dQ = c.take<char>(mat);
-    b.dK = c.take<char>(mat);
-    b.dV = c.take<char>(mat);
+    b.dQ = c.take<char>(lv * mat);
+    b.dK = c.take<char>(lv * mat);
+    b.dV = c.take<char>(lv * mat);
   }
   if (!g.causal) {
     b.lam = c.take<float>(rows);
@@ -223,14 +226,15 @@ PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
   b.idx = c.take<int>((size_t)g.BH * g.n_t);
   if (backward) {
     b.packed = c.take<float4>(rows);
+    b.inv = c.take<int>(lv * rows * 2);
     return b;
   }
   b.Os = c.take<char>(mat);
-  b.accO = c.take<float>(rows * g.d);
   b.logd = c.take<float>(rows);
   b.m = c.take<float>(rows);
-  b.accL[0] = c.take<float>(rows);
-  b.accL[1] = c.take<float>(rows);
+  b.Os_lv = c.take<char>(lv * mat);
+  b.logd_lv = c.take<float>(lv * rows);
+  b.inv = c.take<int>(lv * rows);
   b.pos = c.take<int>(rows * 2);
   return b;
 }
@@ -453,8 +457,6 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
   ELSAA_TRY(cuda_status(launch_causal_lsh_select(s.idx, 0, g, st), "causal sortLSH base selection"));
   sa.Q = Q; sa.K = K; sa.V = V;
   ELSAA_TRY(cuda_status(launch_attn_fwd_tc(sa, gb, w.flag, st), "causal sortLSH base pass"));
-  ELSAA_TRY(cuda_status(launch_lsh_merge(b.Os, b.logd, nullptr, 0, b.accO, nullptr, b.accL[0], g, st), "merge"));
-  int cur = 0;
   if (g.lsh_levels > 0)
     ELSAA_TRY(cuda_status(launch_sortlsh_hash(Q, K, true, p->lsh_planes, p->lsh_bits, b.pos, nullptr, g, st),
                           "sortLSH hash"));
@@ -462,19 +464,24 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
   for (int lev = 0; lev < g.lsh_levels; ++lev) {
     const int h = g.N >> (lev + 1);
     int* ord = s.lsh_order + (size_t)lev * g.BH * stride;
-    ELSAA_TRY(cuda_status(launch_sortlsh_level_sort(b.pos, ord, h, p->lsh_bits, g, st), "sortLSH level sort"));
-    ELSAA_TRY(cuda_status(launch_permute_rows(Q, b.Q, ord, rb, g, stride, false, st), "sortLSH gather Q"));
-    ELSAA_TRY(cuda_status(launch_permute_rows(K, b.K, ord + g.N, rb, g, stride, false, st), "sortLSH gather K"));
-    ELSAA_TRY(cuda_status(launch_permute_rows(V, b.V, ord + g.N, rb, g, stride, false, st), "sortLSH gather V"));
+    ELSAA_TRY(cuda_status(launch_sortlsh_level_sort(b.pos, ord, b.inv + lev * rows, h, p->lsh_bits, g, st),
+                          "sortLSH level sort"));
+    // only the future halves' queries and the past halves' keys and values are read
+    const void* qs[1] = {Q};
+    void* qd[1] = {b.Q};
+    const void* kvs[2] = {K, V};
+    void* kvd[2] = {b.K, b.V};
+    ELSAA_TRY(cuda_status(launch_gather_rows(qs, qd, 1, ord, rb, stride, h, 1, g, st), "sortLSH gather Q"));
+    ELSAA_TRY(cuda_status(launch_gather_rows(kvs, kvd, 2, ord + g.N, rb, stride, h, 0, g, st), "sortLSH gather K, V"));
     ELSAA_TRY(cuda_status(launch_causal_lsh_select(b.idx, h / g.T, gl, st), "sortLSH level selection"));
     sa.Q = b.Q; sa.K = b.K; sa.V = b.V; sa.idx = b.idx;
+    sa.Os = static_cast<char*>(b.Os_lv) + lev * rows * rb;
+    sa.logd = sa.dlr = b.logd_lv + lev * rows;
     ELSAA_TRY(cuda_status(launch_attn_fwd_tc(sa, gl, w.flag, st), "sortLSH level pass"));
-    ELSAA_TRY(cuda_status(launch_lsh_merge(b.Os, b.logd, ord, h, b.accO, b.accL[cur], b.accL[cur ^ 1], g, st),
-                          "merge"));
-    cur ^= 1;
   }
-  return cuda_status(launch_lsh_fuse(b.accO, b.accL[cur], s.Olr, s.dlr, lam, gs, glr, O, s.Os, s.logd, s.m, g, st),
-                     "fusion");
+  return cuda_status(launch_lsh_fuse(b.Os, b.logd, b.Os_lv, b.logd_lv, b.inv, g.lsh_levels, s.Olr, s.dlr, lam, gs,
+                                     glr, O, s.Os, s.logd, s.m, g, st),
+                     "merge and fusion");
 }
 
 elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const BwdWs& w, cudaStream_t st) {
@@ -502,24 +509,33 @@ elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const
   for (int lev = 0; lev < g.lsh_levels; ++lev) {
     const int h = g.N >> (lev + 1);
     const int* ord = s.lsh_order + (size_t)lev * g.BH * stride;
-    ELSAA_TRY(cuda_status(launch_permute_rows(a.Q, b.Q, ord, rb, g, stride, false, st), "sortLSH gather Q"));
-    ELSAA_TRY(cuda_status(launch_permute_rows(a.K, b.K, ord + g.N, rb, g, stride, false, st), "sortLSH gather K"));
-    ELSAA_TRY(cuda_status(launch_permute_rows(a.V, b.V, ord + g.N, rb, g, stride, false, st), "sortLSH gather V"));
-    ELSAA_TRY(cuda_status(launch_permute_rows(a.dO, b.X, ord, rb, g, stride, false, st), "sortLSH gather dO"));
-    ELSAA_TRY(cuda_status(launch_permute_rows(w.rs.packed, b.packed, ord, 16, g, stride, false, st),
-                          "sortLSH gather row scalars"));
+    const void* qs[2] = {a.Q, a.dO};
+    void* qd[2] = {b.Q, b.X};
+    const void* kvs[2] = {a.K, a.V};
+    void* kvd[2] = {b.K, b.V};
+    const void* ps[1] = {w.rs.packed};
+    void* pd[1] = {b.packed};
+    ELSAA_TRY(cuda_status(launch_gather_rows(qs, qd, 2, ord, rb, stride, h, 1, g, st), "sortLSH gather Q, dO"));
+    ELSAA_TRY(cuda_status(launch_gather_rows(kvs, kvd, 2, ord + g.N, rb, stride, h, 0, g, st), "sortLSH gather K, V"));
+    ELSAA_TRY(cuda_status(launch_gather_rows(ps, pd, 1, ord, 16, stride, h, 1, g, st), "sortLSH gather row scalars"));
     ELSAA_TRY(cuda_status(launch_causal_lsh_select(b.idx, h / g.T, gl, st), "sortLSH level selection"));
     ELSAA_TRY(cuda_status(launch_invert_selection(b.idx, w.offs, w.tiles, w.order, gl, st), "selection inverse"));
     BwdArgs la{};
     la.Q = b.Q; la.K = b.K; la.V = b.V; la.dO = b.X;
     la.idx = b.idx; la.offs = w.offs; la.tiles = w.tiles; la.kv_order = w.order;
     la.rs.packed = b.packed;
-    la.dQ = b.dQ; la.dK = b.dK; la.dV = b.dV;
+    la.dQ = static_cast<char*>(b.dQ) + lev * rows * rb;
+    la.dK = static_cast<char*>(b.dK) + lev * rows * rb;
+    la.dV = static_cast<char*>(b.dV) + lev * rows * rb;
     ELSAA_TRY(cuda_status(launch_dq_tc(la, gl, w.flag, st), "sortLSH level dq"));
     ELSAA_TRY(cuda_status(launch_dkdv_tc(la, gl, w.flag, st), "sortLSH level dkdv"));
-    ELSAA_TRY(cuda_status(launch_lsh_add_rows(b.dQ, w.dQacc, ord, h, true, g, st), "sortLSH dQ"));
-    ELSAA_TRY(cuda_status(launch_lsh_add_rows(b.dK, w.dKacc, ord + g.N, h, false, g, st), "sortLSH dK"));
-    ELSAA_TRY(cuda_status(launch_lsh_add_rows(b.dV, w.dVacc, ord + g.N, h, false, g, st), "sortLSH dV"));
+  }
+  if (g.lsh_levels > 0) {
+    ELSAA_TRY(cuda_status(launch_lsh_invert_orders(s.lsh_order, b.inv, g.lsh_levels, g, st), "order inverses"));
+    ELSAA_TRY(cuda_status(launch_lsh_collect(b.dQ, w.dQacc, nullptr, nullptr, b.inv, g.lsh_levels, false, g, st),
+                          "sortLSH dQ"));
+    ELSAA_TRY(cuda_status(launch_lsh_collect(b.dK, w.dKacc, b.dV, w.dVacc, b.inv, g.lsh_levels, true, g, st),
+                          "sortLSH dK, dV"));
   }
   // base pass in the caller's order: adds the accumulators before the single rounding
   const Geom gb = sparse_only(g, true, 2);

@@ -70,17 +70,22 @@ size_t sortlsh_smem_bytes(const Geom& g, int bits);
 cudaError_t launch_sortlsh_hash(const void* Q, const void* K, bool bf16, const float* planes, int bits, int* pos,
                                 int* codes, const Geom& g, cudaStream_t st);
 // Causal recursion: one level's orders [BH][2][N] (queries sorted in the future halves,
-// keys in the past halves of h rows; identity elsewhere); the base / level selections;
-// the log-sum-exp merge of sparse partials; the final fusion; fp32 row scatter-add.
-cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int h, int bits, const Geom& g, cudaStream_t st);
+// keys in the past halves of h rows; identity elsewhere) and, if inv is not null, the
+// future-half rows' positions [BH][N]; the base / level selections; the final
+// log-sum-exp merge of the partials with the fusion; the orders' inverses; the level
+// gradients collected into the fp32 accumulators; multi-tensor half-row gathers.
+cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int* inv, int h, int bits, const Geom& g,
+                                      cudaStream_t st);
 cudaError_t launch_causal_lsh_select(int* idx, int hb, const Geom& g, cudaStream_t st);
-cudaError_t launch_lsh_merge(const void* Os, const float* logd, const int* perm, int h, float* accO,
-                             const float* accL_in, float* accL_out, const Geom& g, cudaStream_t st);
-cudaError_t launch_lsh_fuse(const float* accO, const float* accL, const void* Olr, const float* dlr, const float* lam,
+cudaError_t launch_lsh_fuse(const void* Os0, const float* logd0, const void* Os_lv, const float* logd_lv,
+                            const int* inv_lv, int levels, const void* Olr, const float* dlr, const float* lam,
                             const float* gs, const float* glr, void* O, void* Os, float* logd, float* m, const Geom& g,
                             cudaStream_t st);
-cudaError_t launch_lsh_add_rows(const void* src, float* acc, const int* perm, int h, bool future, const Geom& g,
-                                cudaStream_t st);
+cudaError_t launch_lsh_invert_orders(const int* order, int* inv, int levels, const Geom& g, cudaStream_t st);
+cudaError_t launch_lsh_collect(const void* src0, float* acc0, const void* src1, float* acc1, const int* inv,
+                               int levels, bool keys, const Geom& g, cudaStream_t st);
+cudaError_t launch_gather_rows(const void* const* src, void* const* dst, int n, const int* perm, int row_bytes,
+                               int perm_stride, int h, int half, const Geom& g, cudaStream_t st);
 // Row permutation of [BH][N] rows of row_bytes (a multiple of 16): gather dst[r] = src[perm[r]]
 // or scatter dst[perm[r]] = src[r]; perm advances by perm_stride per head.
 cudaError_t launch_permute_rows(const void* src, void* dst, const int* perm, int row_bytes, const Geom& g,

@@ -208,9 +208,11 @@ __global__ void __launch_bounds__(kSortThreads) sortlsh_sort_kernel(int* __restr
 // 2s and a future half 2s + 1 per segment).  grid (BH, 2, N / 2h): side 0 sorts the
 // queries of future half 2s + 1, side 1 the keys of past half 2s, by Gray position
 // (stable); the other half of each side's order is the identity.  pos and order are
-// [BH][2][N]; order holds row indices.
+// [BH][2][N]; order holds row indices.  inv, if not null, receives for every row of a
+// future half its position in the sorted query order ([BH][N]).
 __global__ void __launch_bounds__(kSortThreads) sortlsh_level_sort_kernel(const int* __restrict__ pos,
-                                                                          int* __restrict__ order, int h, int bits,
+                                                                          int* __restrict__ order,
+                                                                          int* __restrict__ inv, int h, int bits,
                                                                           Geom g) {
   extern __shared__ __align__(16) unsigned char smem[];
   int* cnt = reinterpret_cast<int*>(smem);
@@ -226,7 +228,12 @@ __global__ void __launch_bounds__(kSortThreads) sortlsh_level_sort_kernel(const 
     order[off + ident0 + i] = ident0 + i;
   }
   const uint32_t* out = block_counting_sort(bufA, bufB, cnt, wsum, h, bits);
-  for (int i = threadIdx.x; i < h; i += kSortThreads) order[off + sorted0 + i] = sorted0 + (int)(out[i] & 0x3fffu);
+  for (int i = threadIdx.x; i < h; i += kSortThreads) {
+    const int r = sorted0 + (int)(out[i] & 0x3fffu);
+    order[off + sorted0 + i] = r;
+    // queries: where each future-half row sits in the sorted order ([BH][N])
+    if (inv && side == 0) inv[(size_t)blockIdx.x * g.N + r] = sorted0 + i;
+  }
 }
 
 // Selections of the causal recursion.  Base pass (the caller's row order, causal): tile
@@ -247,76 +254,73 @@ __global__ void causal_lsh_select_kernel(int* __restrict__ idx, int hb, Geom g) 
   }
 }
 
-// Sparse partial results into the running fp32 (O_s, log d_s) of the caller's rows.
-// src: bf16 normalised O_s and its log d_s, in sorted order (perm = query order) or in
-// row order (perm null).  h = 0 initialises every row; h > 0 merges the rows at
-// future-half positions of that level by log-sum-exp and carries the others' log d_s
-// over.  The log-denominators are double-buffered (accL_in -> accL_out) so every thread
-// of a row reads the old value.  One thread per 8 columns.
-__global__ void lsh_merge_kernel(const __nv_bfloat16* __restrict__ Os, const float* __restrict__ logd,
-                                 const int* __restrict__ perm, int h, float* __restrict__ accO,
-                                 const float* __restrict__ accL_in, float* __restrict__ accL_out, Geom g) {
-  const int units = g.d / 8;
-  const size_t total = (size_t)g.BH * g.N * units;
-  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
-    const size_t p = e / units;
-    const int u = (int)(e % units);
-    const int bh = (int)(p / g.N), pr = (int)(p % g.N);
-    const size_t row = (size_t)bh * g.N + (perm ? perm[(size_t)bh * 2 * g.N + pr] : pr);
-    const float l = logd[p];
-    const float a = h > 0 ? accL_in[row] : -INFINITY;
-    if (h > 0 && (((pr / h) & 1) == 0 || l == -INFINITY)) {      // nothing from this level
-      if (u == 0) accL_out[row] = a;
-      continue;
-    }
-    const uint4 w = *reinterpret_cast<const uint4*>(Os + p * g.d + 8 * u);
-    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
-    float4* acc = reinterpret_cast<float4*>(accO + row * g.d + 8 * u);
-    float x[8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = __bfloat1622float2(hv[j]);
-      x[2 * j] = f.x;
-      x[2 * j + 1] = f.y;
-    }
-    if (h == 0) {
-      if (u == 0) accL_out[row] = l;
-      acc[0] = make_float4(x[0], x[1], x[2], x[3]);
-      acc[1] = make_float4(x[4], x[5], x[6], x[7]);
-      continue;
-    }
-    const float L = a == -INFINITY ? l : fmaxf(a, l) + log1pf(__expf(-fabsf(a - l)));
-    const float wa = a == -INFINITY ? 0.f : __expf(a - L), wl = __expf(l - L);
-    const float4 a0 = acc[0], a1 = acc[1];
-    acc[0] = make_float4(wa * a0.x + wl * x[0], wa * a0.y + wl * x[1], wa * a0.z + wl * x[2], wa * a0.w + wl * x[3]);
-    acc[1] = make_float4(wa * a1.x + wl * x[4], wa * a1.y + wl * x[5], wa * a1.z + wl * x[6], wa * a1.w + wl * x[7]);
-    if (u == 0) accL_out[row] = L;
-  }
-}
+// Log-sum-exp merge of the recursion's sparse partials, then the fusion (Eq. 5 weight,
+// Eq. 4 output) with the low-rank branch, per row.  The base pass's partial (O_s, log d_s)
+// is in row order; level l's is in its sorted query order, at position inv_l[row], and
+// exists for the rows of its future halves (halves of h_l = N >> (l + 1) rows).  Then
+// m = 1 / (1 + (lambda d_lr + eps) e^{-log d_s}) (1 when m is held), O = g_s m O_s + g_lr O_lr
+// with g_lr = 1 - m by default (1 when m is held).  Writes O, the saved bf16 O_s, log d_s
+// and m.  One thread per 8 columns; partials are bf16, the merge is fp32.
+constexpr int kMaxLevels = 8;             // N <= 32768 rows of 128: at most 7 sorted levels
 
-// Fusion (Eq. 5 weight, Eq. 4 output) of the merged sparse branch with the low-rank
-// branch, per row: m = 1 / (1 + (lambda d_lr + eps) e^{-log d_s}) (1 when m is held),
-// O = g_s m O_s + g_lr O_lr with g_lr = 1 - m by default (1 when m is held).  Writes O,
-// the saved bf16 O_s, log d_s and m.  One thread per 8 columns.
-__global__ void lsh_fuse_kernel(const float* __restrict__ accO, const float* __restrict__ accL,
-                                const __nv_bfloat16* __restrict__ Olr, const float* __restrict__ dlr,
-                                const float* lamv, const float* gsv, const float* glrv, __nv_bfloat16* __restrict__ O,
-                                __nv_bfloat16* __restrict__ Os, float* __restrict__ logd_out, float* __restrict__ m_out,
-                                Geom g) {
+__global__ void lsh_fuse_kernel(const __nv_bfloat16* __restrict__ Os0, const float* __restrict__ logd0,
+                                const __nv_bfloat16* __restrict__ Os_lv, const float* __restrict__ logd_lv,
+                                const int* __restrict__ inv_lv, int levels, const __nv_bfloat16* __restrict__ Olr,
+                                const float* __restrict__ dlr, const float* lamv, const float* gsv, const float* glrv,
+                                __nv_bfloat16* __restrict__ O, __nv_bfloat16* __restrict__ Os,
+                                float* __restrict__ logd_out, float* __restrict__ m_out, Geom g) {
   const int units = g.d / 8;
-  const size_t total = (size_t)g.BH * g.N * units;
+  const size_t rows = (size_t)g.BH * g.N;
+  const size_t total = rows * units;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
     const size_t row = e / units;
     const int u = (int)(e % units);
-    const float l = accL[row];
+    const int bh = (int)(row / g.N), r = (int)(row % g.N);
+    // the partials this row has: base (slot 0), then one per level where it is in a
+    // future half; every level's loads are issued before any is used
+    const __nv_bfloat16* src[kMaxLevels + 1];
+    float lg[kMaxLevels + 1];
+    src[0] = Os0 + row * g.d + 8 * u;
+    lg[0] = logd0[row];
+#pragma unroll
+    for (int l = 0; l < kMaxLevels; ++l) {
+      lg[l + 1] = -INFINITY;
+      src[l + 1] = nullptr;
+      if (l < levels && ((r / (g.N >> (l + 1))) & 1)) {
+        const size_t p = (size_t)l * rows + (size_t)bh * g.N + inv_lv[(size_t)l * rows + row];
+        src[l + 1] = Os_lv + p * g.d + 8 * u;
+        lg[l + 1] = logd_lv[p];
+      }
+    }
+    float L = -INFINITY;
+#pragma unroll
+    for (int j = 0; j <= kMaxLevels; ++j) L = fmaxf(L, lg[j]);
+    float sum = 0.f, s[8] = {};
+    if (L > -INFINITY) {
+#pragma unroll
+      for (int j = 0; j <= kMaxLevels; ++j) {
+        if (lg[j] == -INFINITY) continue;
+        const float wj = __expf(lg[j] - L);
+        sum += wj;
+        const uint4 w = *reinterpret_cast<const uint4*>(src[j]);
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(hv[k]);
+          s[2 * k] = fmaf(wj, f.x, s[2 * k]);
+          s[2 * k + 1] = fmaf(wj, f.y, s[2 * k + 1]);
+        }
+      }
+      const float inv_sum = 1.f / sum;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) s[k] *= inv_sum;
+      L += __logf(sum);
+    }
     const float lam = lamv ? lamv[row] : g.lam;
     const float gs = gsv ? gsv[row] : 1.f;
-    const float mf = g.fixed_m ? 1.f : l == -INFINITY ? 0.f : 1.f / (1.f + (lam * dlr[row] + g.eps) * __expf(-l));
+    const float mf = g.fixed_m ? 1.f : L == -INFINITY ? 0.f : 1.f / (1.f + (lam * dlr[row] + g.eps) * __expf(-L));
     const float gl = glrv ? glrv[row] : g.fixed_m ? 1.f : 1.f - mf;
     const float cs = gs * mf;
-    const float4 a0 = reinterpret_cast<const float4*>(accO + row * g.d + 8 * u)[0];
-    const float4 a1 = reinterpret_cast<const float4*>(accO + row * g.d + 8 * u)[1];
-    const float s[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
     const uint4 w = *reinterpret_cast<const uint4*>(Olr + row * g.d + 8 * u);
     const __nv_bfloat162* lv = reinterpret_cast<const __nv_bfloat162*>(&w);
     uint32_t wo[4], ws[4];
@@ -331,32 +335,87 @@ __global__ void lsh_fuse_kernel(const float* __restrict__ accO, const float* __r
     *reinterpret_cast<uint4*>(O + row * g.d + 8 * u) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
     *reinterpret_cast<uint4*>(Os + row * g.d + 8 * u) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
     if (u == 0) {
-      logd_out[row] = l;
+      logd_out[row] = L;
       m_out[row] = mf;
     }
   }
 }
 
-// acc[perm[p]] += src[p] (bf16 rows into fp32 rows) for the positions p in the future
-// halves (future = 1) or the past halves (future = 0) of a level with halves of h rows.
-__global__ void lsh_add_rows_kernel(const __nv_bfloat16* __restrict__ src, float* __restrict__ acc,
-                                    const int* __restrict__ perm, int h, int future, Geom g) {
+// Inverse of every level's two orders: inv[l][bh][side][order[l][bh][side][p]] = p.
+__global__ void lsh_invert_orders_kernel(const int* __restrict__ order, int* __restrict__ inv, size_t total, int N) {
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t seg = e / N;
+    inv[seg * N + order[e]] = (int)(e % N);
+  }
+}
+
+// The recursion's sparse gradient parts, per row of the caller's order: acc[row] += the
+// sum over the levels where the row is in a future half (queries: want = 1) or a past
+// half (keys: want = 0) of src_l at the row's sorted position.  Up to two tensors (dK
+// and dV) share the key side's positions.  src slots are bf16 [levels][BH][N][d]; inv
+// [levels][BH][2][N].
+__global__ void lsh_collect_kernel(const __nv_bfloat16* __restrict__ src0, float* __restrict__ acc0,
+                                   const __nv_bfloat16* __restrict__ src1, float* __restrict__ acc1,
+                                   const int* __restrict__ inv, int levels, int side, int want, Geom g) {
   const int units = g.d / 8;
+  const size_t rows = (size_t)g.BH * g.N;
+  const size_t total = rows * units;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t row = e / units;
+    const int u = (int)(e % units);
+    const int bh = (int)(row / g.N), r = (int)(row % g.N);
+    float s0[8] = {}, s1[8] = {};
+    bool any = false;
+    for (int l = 0; l < levels; ++l) {
+      const int h = g.N >> (l + 1);
+      if (((r / h) & 1) != want) continue;
+      any = true;
+      const size_t p = (size_t)l * rows + (size_t)bh * g.N +
+                       inv[(((size_t)l * g.BH + bh) * 2 + side) * g.N + r];
+      for (int t = 0; t < (src1 ? 2 : 1); ++t) {
+        const uint4 w = *reinterpret_cast<const uint4*>((t ? src1 : src0) + p * g.d + 8 * u);
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
+        float* sv = t ? s1 : s0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(hv[k]);
+          sv[2 * k] += f.x;
+          sv[2 * k + 1] += f.y;
+        }
+      }
+    }
+    if (!any) continue;
+    for (int t = 0; t < (src1 ? 2 : 1); ++t) {
+      float4* a = reinterpret_cast<float4*>((t ? acc1 : acc0) + row * g.d + 8 * u);
+      const float* sv = t ? s1 : s0;
+      const float4 a0 = a[0], a1 = a[1];
+      a[0] = make_float4(a0.x + sv[0], a0.y + sv[1], a0.z + sv[2], a0.w + sv[3]);
+      a[1] = make_float4(a1.x + sv[4], a1.y + sv[5], a1.z + sv[6], a1.w + sv[7]);
+    }
+  }
+}
+
+// Several row-major tensors with the same rows gathered by one order: dst_t[p] =
+// src_t[perm[p]] for up to four tensors, 16-byte units; half >= 0 moves only the
+// positions in the past (0) or future (1) halves of h rows.
+struct RowMoves {
+  const uint4* src[4];
+  uint4* dst[4];
+  int n;
+};
+
+__global__ void gather_rows_kernel(RowMoves mv, const int* __restrict__ perm, int units, int perm_stride, int h,
+                                   int half, Geom g) {
   const size_t total = (size_t)g.BH * g.N * units;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
-    const size_t p = e / units;
+    const size_t row = e / units;
     const int u = (int)(e % units);
-    const int bh = (int)(p / g.N), pr = (int)(p % g.N);
-    if (((pr / h) & 1) != future) continue;
-    const size_t row = (size_t)bh * g.N + perm[(size_t)bh * 2 * g.N + pr];
-    const uint4 w = *reinterpret_cast<const uint4*>(src + p * g.d + 8 * u);
-    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
-    float4* a = reinterpret_cast<float4*>(acc + row * g.d + 8 * u);
-    const float2 f0 = __bfloat1622float2(hv[0]), f1 = __bfloat1622float2(hv[1]);
-    const float2 f2 = __bfloat1622float2(hv[2]), f3 = __bfloat1622float2(hv[3]);
-    const float4 a0 = a[0], a1 = a[1];
-    a[0] = make_float4(a0.x + f0.x, a0.y + f0.y, a0.z + f1.x, a0.w + f1.y);
-    a[1] = make_float4(a1.x + f2.x, a1.y + f2.y, a1.z + f3.x, a1.w + f3.y);
+    const int bh = (int)(row / g.N), r = (int)(row % g.N);
+    if (half >= 0 && ((r / h) & 1) != half) continue;
+    const size_t pr = (size_t)bh * g.N + perm[(size_t)bh * perm_stride + r];
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if (t < mv.n) mv.dst[t][row * units + u] = mv.src[t][pr * units + u];
   }
 }
 
@@ -424,13 +483,14 @@ cudaError_t launch_sortlsh_hash(const void* Q, const void* K, bool bf16, const f
   return cudaGetLastError();
 }
 
-cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int h, int bits, const Geom& g, cudaStream_t st) {
+cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int* inv, int h, int bits, const Geom& g,
+                                      cudaStream_t st) {
   const size_t smem = (size_t)256 * 32 * 4 + (size_t)2 * h * 4;
   cudaError_t e = cudaFuncSetAttribute(sortlsh_level_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("sortlsh_level_sort", st);
-  sortlsh_level_sort_kernel<<<dim3(g.BH, 2, g.N / (2 * h)), kSortThreads, smem, st>>>(pos, order, h, bits, g);
+  sortlsh_level_sort_kernel<<<dim3(g.BH, 2, g.N / (2 * h)), kSortThreads, smem, st>>>(pos, order, inv, h, bits, g);
   return cudaGetLastError();
 }
 
@@ -441,28 +501,46 @@ cudaError_t launch_causal_lsh_select(int* idx, int hb, const Geom& g, cudaStream
   return cudaGetLastError();
 }
 
-cudaError_t launch_lsh_merge(const void* Os, const float* logd, const int* perm, int h, float* accO,
-                             const float* accL_in, float* accL_out, const Geom& g, cudaStream_t st) {
-  ProfScope ps("lsh_merge", st);
-  lsh_merge_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
-      (const __nv_bfloat16*)Os, logd, perm, h, accO, accL_in, accL_out, g);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_lsh_fuse(const float* accO, const float* accL, const void* Olr, const float* dlr, const float* lam,
+cudaError_t launch_lsh_fuse(const void* Os0, const float* logd0, const void* Os_lv, const float* logd_lv,
+                            const int* inv_lv, int levels, const void* Olr, const float* dlr, const float* lam,
                             const float* gs, const float* glr, void* O, void* Os, float* logd, float* m, const Geom& g,
                             cudaStream_t st) {
+  if (levels > kMaxLevels) return cudaErrorInvalidValue;
   ProfScope ps("lsh_fuse", st);
   lsh_fuse_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
-      accO, accL, (const __nv_bfloat16*)Olr, dlr, lam, gs, glr, (__nv_bfloat16*)O, (__nv_bfloat16*)Os, logd, m, g);
+      (const __nv_bfloat16*)Os0, logd0, (const __nv_bfloat16*)Os_lv, logd_lv, inv_lv, levels,
+      (const __nv_bfloat16*)Olr, dlr, lam, gs, glr, (__nv_bfloat16*)O, (__nv_bfloat16*)Os, logd, m, g);
   return cudaGetLastError();
 }
 
-cudaError_t launch_lsh_add_rows(const void* src, float* acc, const int* perm, int h, bool future, const Geom& g,
-                                cudaStream_t st) {
-  ProfScope ps("lsh_add_rows", st);
-  lsh_add_rows_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
-      (const __nv_bfloat16*)src, acc, perm, h, future ? 1 : 0, g);
+cudaError_t launch_lsh_invert_orders(const int* order, int* inv, int levels, const Geom& g, cudaStream_t st) {
+  const size_t total = (size_t)levels * g.BH * 2 * g.N;
+  lsh_invert_orders_kernel<<<elementwise_blocks(total), 256, 0, st>>>(order, inv, total, g.N);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lsh_collect(const void* src0, float* acc0, const void* src1, float* acc1, const int* inv,
+                               int levels, bool keys, const Geom& g, cudaStream_t st) {
+  ProfScope ps("lsh_collect", st);
+  lsh_collect_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
+      (const __nv_bfloat16*)src0, acc0, (const __nv_bfloat16*)src1, acc1, inv, levels, keys ? 1 : 0, keys ? 0 : 1,
+      g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* const* src, void* const* dst, int n, const int* perm, int row_bytes,
+                               int perm_stride, int h, int half, const Geom& g, cudaStream_t st) {
+  if (n < 1 || n > 4) return cudaErrorInvalidValue;
+  RowMoves mv{};
+  for (int t = 0; t < n; ++t) {
+    mv.src[t] = (const uint4*)src[t];
+    mv.dst[t] = (uint4*)dst[t];
+  }
+  mv.n = n;
+  const int units = row_bytes / 16;
+  ProfScope ps("sortlsh_gather", st);
+  gather_rows_kernel<<<elementwise_blocks((size_t)g.BH * g.N * units), 256, 0, st>>>(mv, perm, units, perm_stride, h,
+                                                                                     half, g);
   return cudaGetLastError();
 }
 
