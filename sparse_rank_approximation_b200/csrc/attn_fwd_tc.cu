@@ -92,8 +92,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem[];
   Misc* ms = reinterpret_cast<Misc*>(smem + OFF_MISC);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = g.n_t - 1 - blockIdx.x;
   const int bh = blockIdx.y;
+  const int t = a.tile_list ? a.tile_list[(size_t)bh * a.n_list + blockIdx.x] : g.n_t - 1 - (int)blockIdx.x;
   const size_t head = (size_t)bh * g.N;
   if (smem_u32(smem) & 1023u) {            // the swizzled layouts need 1024-byte aligned tiles
     if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
@@ -443,7 +443,8 @@ cudaError_t launch_attn_fwd_tc(const FwdArgs& a, const Geom& g, uint32_t* err, c
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   ProfScope ps("attn_fwd_tc", st);
-  attn_fwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, kSmemBytes, st>>>(mq, mk, mv, mlr, mo, ms, a, g, err);
+  attn_fwd_tc_kernel<<<dim3(a.tile_list ? a.n_list : g.n_t, g.BH), kThreads, kSmemBytes, st>>>(mq, mk, mv, mlr, mo,
+                                                                                               ms, a, g, err);
   return cudaGetLastError();
 }
 

@@ -101,8 +101,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem[];
   DqMisc* ms = reinterpret_cast<DqMisc*>(smem + DQ_MISC);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = g.n_t - 1 - blockIdx.x;
   const int bh = blockIdx.y;
+  const int t = a.tile_list ? a.tile_list[(size_t)bh * a.n_list + blockIdx.x] : g.n_t - 1 - (int)blockIdx.x;
   const size_t head = (size_t)bh * g.N;
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
@@ -630,7 +630,7 @@ cudaError_t launch_dq_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStr
   cudaError_t e = cudaFuncSetAttribute(dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("dq_tc", st);
-  dq_tc_kernel<<<dim3(g.n_t, g.BH), kDqThreads, smem, st>>>(mq, mk, mv, mdo, mdq, a, g, err);
+  dq_tc_kernel<<<dim3(a.tile_list ? a.n_list : g.n_t, g.BH), kDqThreads, smem, st>>>(mq, mk, mv, mdo, mdq, a, g, err);
   return cudaGetLastError();
 }
 
@@ -648,7 +648,8 @@ static bool map_scalars(CUtensorMap* m, const void* base, int N, int BH) {
 }
 
 cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
-  if (!bwd_tc_supported(g) || !a.rs.packed || g.n_t > kMaxUnits) return cudaErrorInvalidValue;
+  if (!bwd_tc_supported(g) || !a.rs.packed || g.n_t > kMaxUnits || (a.n_kv && !a.kv_order) || a.n_kv > g.n_t)
+    return cudaErrorInvalidValue;
   CUtensorMap mk, mv, mq, mdo, msc, mdk, mdv;
   if (!tc::map_rows_bf16(&mk, a.K, g.N, g.BH, kT) || !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kT) ||
       !tc::map_rows_bf16(&mq, a.Q, g.N, g.BH, kT) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, kT) ||
@@ -660,7 +661,9 @@ cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaS
   cudaError_t e = cudaFuncSetAttribute(dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("dkdv_tc", st);
-  dkdv_tc_kernel<<<dim3(g.BH, g.n_t), kKvThreads, smem, st>>>(mk, mv, mq, mdo, msc, mdk, mdv, a, g, err);
+  // with n_kv, only the first n_kv key blocks of kv_order (the ones with query tiles) run
+  dkdv_tc_kernel<<<dim3(g.BH, a.n_kv ? a.n_kv : g.n_t), kKvThreads, smem, st>>>(mk, mv, mq, mdo, msc, mdk, mdv, a, g,
+                                                                               err);
   return cudaGetLastError();
 }
 

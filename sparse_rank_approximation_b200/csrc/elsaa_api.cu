@@ -192,14 +192,16 @@ Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
 struct PermBufs {
   void *Q, *K, *V, *X, *dQ, *dK, *dV;     // X: O (forward) or dO (backward)
   float *lam, *gs, *glr;
-  // causal recursion.  Forward: the base pass's O_s, log d_s (and a scratch m), every
-  // level's partial O_s and log d_s in its sorted order ([levels][BH][N][d], [levels][BH][N])
-  // with the future-half rows' positions ([levels][BH][N]), the Gray positions.
-  // Backward: dQ, dK, dV hold every level's gradients ([levels][BH][N][d]), inv the
-  // orders' inverses ([levels][BH][2][N]), packed the sorted rows' backward scalars.
+  // causal recursion: every sorted level is one more block of heads ("level slots",
+  // [levels][BH][N][d]).  Q, K, V (and dO, dQ, dK, dV in the backward) are slotted; idx
+  // and tile_list hold every level's selection and future tiles; offs, tiles, order the
+  // selection inverse over the level heads.  Forward: the base pass's O_s, log d_s (X is
+  // its scratch output), the levels' partial O_s and log d_s, the future rows' positions
+  // inv ([levels][BH][N]), the Gray positions.  Backward: the orders' inverses inv
+  // ([levels][BH][2][N]) and the sorted rows' packed backward scalars.
   void *Os, *Os_lv;
   float *logd, *m, *logd_lv;
-  int *idx, *pos, *inv;
+  int *idx, *tile_list, *offs, *tiles, *order, *pos, *inv;
   float4* packed;
 };
 
@@ -207,31 +209,43 @@ PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
   PermBufs b{};
   if (g.selector != ELSAA_SEL_SORTLSH) return b;
   const size_t rows = (size_t)g.BH * g.N, mat = rows * g.d * esz;
-  const size_t lv = g.causal ? (size_t)g.lsh_levels : 1;
-  b.Q = c.take<char>(mat);
-  b.K = c.take<char>(mat);
-  b.V = c.take<char>(mat);
-  b.X = c.take<char>(mat);
-  if (backward) {
-    b.dQ = c.take<char>(lv * mat);
-    b.dK = c.take<char>(lv * mat);
-    b.dV = c.take<char>(lv * mat);
-  }
   if (!g.causal) {
+    b.Q = c.take<char>(mat);
+    b.K = c.take<char>(mat);
+    b.V = c.take<char>(mat);
+    b.X = c.take<char>(mat);
+    if (backward) {
+      b.dQ = c.take<char>(mat);
+      b.dK = c.take<char>(mat);
+      b.dV = c.take<char>(mat);
+    }
     b.lam = c.take<float>(rows);
     b.gs = c.take<float>(rows);
     b.glr = c.take<float>(rows);
     return b;
   }
-  b.idx = c.take<int>((size_t)g.BH * g.n_t);
+  const size_t lv = (size_t)g.lsh_levels, vheads = lv * g.BH;
+  b.Q = c.take<char>(lv * mat);
+  b.K = c.take<char>(lv * mat);
+  b.V = c.take<char>(lv * mat);
+  b.idx = c.take<int>(vheads * g.n_t);
+  b.tile_list = c.take<int>(vheads * (g.n_t / 2));
   if (backward) {
-    b.packed = c.take<float4>(rows);
+    b.X = c.take<char>(lv * mat);
+    b.dQ = c.take<char>(lv * mat);
+    b.dK = c.take<char>(lv * mat);
+    b.dV = c.take<char>(lv * mat);
+    b.packed = c.take<float4>(lv * rows);
+    b.offs = c.take<int>(vheads * (g.n_t + 1));
+    b.tiles = c.take<int>(vheads * g.n_t);
+    b.order = c.take<int>(vheads * g.n_t);
     b.inv = c.take<int>(lv * rows * 2);
     return b;
   }
+  b.X = c.take<char>(mat);
   b.Os = c.take<char>(mat);
   b.logd = c.take<float>(rows);
-  b.m = c.take<float>(rows);
+  b.m = c.take<float>(std::max<size_t>(lv, 1) * rows);
   b.Os_lv = c.take<char>(lv * mat);
   b.logd_lv = c.take<float>(lv * rows);
   b.inv = c.take<int>(lv * rows);
@@ -457,27 +471,35 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
   ELSAA_TRY(cuda_status(launch_causal_lsh_select(s.idx, 0, g, st), "causal sortLSH base selection"));
   sa.Q = Q; sa.K = K; sa.V = V;
   ELSAA_TRY(cuda_status(launch_attn_fwd_tc(sa, gb, w.flag, st), "causal sortLSH base pass"));
-  if (g.lsh_levels > 0)
+  if (g.lsh_levels > 0) {
+    const int lv = g.lsh_levels;
     ELSAA_TRY(cuda_status(launch_sortlsh_hash(Q, K, true, p->lsh_planes, p->lsh_bits, b.pos, nullptr, g, st),
                           "sortLSH hash"));
-  const Geom gl = sparse_only(g, false, 1);
-  for (int lev = 0; lev < g.lsh_levels; ++lev) {
-    const int h = g.N >> (lev + 1);
-    int* ord = s.lsh_order + (size_t)lev * g.BH * stride;
-    ELSAA_TRY(cuda_status(launch_sortlsh_level_sort(b.pos, ord, b.inv + lev * rows, h, p->lsh_bits, g, st),
-                          "sortLSH level sort"));
+    for (int lev = 0; lev < lv; ++lev)
+      ELSAA_TRY(cuda_status(launch_sortlsh_level_sort(b.pos, s.lsh_order + (size_t)lev * g.BH * stride,
+                                                      b.inv + lev * rows, g.N >> (lev + 1), p->lsh_bits, g, st),
+                            "sortLSH level sort"));
     // only the future halves' queries and the past halves' keys and values are read
     const void* qs[1] = {Q};
     void* qd[1] = {b.Q};
     const void* kvs[2] = {K, V};
     void* kvd[2] = {b.K, b.V};
-    ELSAA_TRY(cuda_status(launch_gather_rows(qs, qd, 1, ord, rb, stride, h, 1, g, st), "sortLSH gather Q"));
-    ELSAA_TRY(cuda_status(launch_gather_rows(kvs, kvd, 2, ord + g.N, rb, stride, h, 0, g, st), "sortLSH gather K, V"));
-    ELSAA_TRY(cuda_status(launch_causal_lsh_select(b.idx, h / g.T, gl, st), "sortLSH level selection"));
+    ELSAA_TRY(cuda_status(launch_gather_rows(qs, qd, 1, s.lsh_order, rb, lv, 1, g, st), "sortLSH gather Q"));
+    ELSAA_TRY(cuda_status(launch_gather_rows(kvs, kvd, 2, s.lsh_order + g.N, rb, lv, 0, g, st),
+                          "sortLSH gather K, V"));
+    ELSAA_TRY(cuda_status(launch_causal_lsh_select_levels(b.idx, b.tile_list, lv, g, st), "sortLSH level selection"));
+    // all levels in one launch, as lv * BH heads, over their future tiles only.  The fused
+    // output goes over each tile's own gathered queries (read before it is written), the
+    // low-rank input it does not use is read from the values
+    Geom gv = sparse_only(g, false, 1);
+    gv.BH = lv * g.BH;
     sa.Q = b.Q; sa.K = b.K; sa.V = b.V; sa.idx = b.idx;
-    sa.Os = static_cast<char*>(b.Os_lv) + lev * rows * rb;
-    sa.logd = sa.dlr = b.logd_lv + lev * rows;
-    ELSAA_TRY(cuda_status(launch_attn_fwd_tc(sa, gl, w.flag, st), "sortLSH level pass"));
+    sa.O = b.Q; sa.Olr = b.V;
+    sa.Os = b.Os_lv;
+    sa.logd = sa.dlr = b.logd_lv;
+    sa.tile_list = b.tile_list;
+    sa.n_list = g.n_t / 2;
+    ELSAA_TRY(cuda_status(launch_attn_fwd_tc(sa, gv, w.flag, st), "sortLSH level pass"));
   }
   return cuda_status(launch_lsh_fuse(b.Os, b.logd, b.Os_lv, b.logd_lv, b.inv, g.lsh_levels, s.Olr, s.dlr, lam, gs,
                                      glr, O, s.Os, s.logd, s.m, g, st),
@@ -505,36 +527,37 @@ elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const
     ELSAA_TRY(cuda_status(cudaMemsetAsync(w.dKacc, 0, rows * g.d * 4, st), "dK accumulator"));
     ELSAA_TRY(cuda_status(cudaMemsetAsync(w.dVacc, 0, rows * g.d * 4, st), "dV accumulator"));
   }
-  const Geom gl = sparse_only(g, false, 1);
-  for (int lev = 0; lev < g.lsh_levels; ++lev) {
-    const int h = g.N >> (lev + 1);
-    const int* ord = s.lsh_order + (size_t)lev * g.BH * stride;
+  if (g.lsh_levels > 0) {
+    const int lv = g.lsh_levels;
     const void* qs[2] = {a.Q, a.dO};
     void* qd[2] = {b.Q, b.X};
     const void* kvs[2] = {a.K, a.V};
     void* kvd[2] = {b.K, b.V};
     const void* ps[1] = {w.rs.packed};
     void* pd[1] = {b.packed};
-    ELSAA_TRY(cuda_status(launch_gather_rows(qs, qd, 2, ord, rb, stride, h, 1, g, st), "sortLSH gather Q, dO"));
-    ELSAA_TRY(cuda_status(launch_gather_rows(kvs, kvd, 2, ord + g.N, rb, stride, h, 0, g, st), "sortLSH gather K, V"));
-    ELSAA_TRY(cuda_status(launch_gather_rows(ps, pd, 1, ord, 16, stride, h, 1, g, st), "sortLSH gather row scalars"));
-    ELSAA_TRY(cuda_status(launch_causal_lsh_select(b.idx, h / g.T, gl, st), "sortLSH level selection"));
-    ELSAA_TRY(cuda_status(launch_invert_selection(b.idx, w.offs, w.tiles, w.order, gl, st), "selection inverse"));
+    ELSAA_TRY(cuda_status(launch_gather_rows(qs, qd, 2, s.lsh_order, rb, lv, 1, g, st), "sortLSH gather Q, dO"));
+    ELSAA_TRY(cuda_status(launch_gather_rows(kvs, kvd, 2, s.lsh_order + g.N, rb, lv, 0, g, st),
+                          "sortLSH gather K, V"));
+    ELSAA_TRY(cuda_status(launch_gather_rows(ps, pd, 1, s.lsh_order, 16, lv, 1, g, st), "sortLSH gather row scalars"));
+    ELSAA_TRY(cuda_status(launch_causal_lsh_select_levels(b.idx, b.tile_list, lv, g, st), "sortLSH level selection"));
+    Geom gv = sparse_only(g, false, 1);
+    gv.BH = lv * g.BH;
+    ELSAA_TRY(cuda_status(launch_invert_selection(b.idx, b.offs, b.tiles, b.order, gv, st), "selection inverse"));
+    // all levels in one launch each: dQ over the future tiles, dK/dV over the key blocks
+    // that have a tile (the past halves, first in the longest-first order)
     BwdArgs la{};
     la.Q = b.Q; la.K = b.K; la.V = b.V; la.dO = b.X;
-    la.idx = b.idx; la.offs = w.offs; la.tiles = w.tiles; la.kv_order = w.order;
+    la.idx = b.idx; la.offs = b.offs; la.tiles = b.tiles; la.kv_order = b.order;
     la.rs.packed = b.packed;
-    la.dQ = static_cast<char*>(b.dQ) + lev * rows * rb;
-    la.dK = static_cast<char*>(b.dK) + lev * rows * rb;
-    la.dV = static_cast<char*>(b.dV) + lev * rows * rb;
-    ELSAA_TRY(cuda_status(launch_dq_tc(la, gl, w.flag, st), "sortLSH level dq"));
-    ELSAA_TRY(cuda_status(launch_dkdv_tc(la, gl, w.flag, st), "sortLSH level dkdv"));
-  }
-  if (g.lsh_levels > 0) {
-    ELSAA_TRY(cuda_status(launch_lsh_invert_orders(s.lsh_order, b.inv, g.lsh_levels, g, st), "order inverses"));
-    ELSAA_TRY(cuda_status(launch_lsh_collect(b.dQ, w.dQacc, nullptr, nullptr, b.inv, g.lsh_levels, false, g, st),
-                          "sortLSH dQ"));
-    ELSAA_TRY(cuda_status(launch_lsh_collect(b.dK, w.dKacc, b.dV, w.dVacc, b.inv, g.lsh_levels, true, g, st),
+    la.dQ = b.dQ; la.dK = b.dK; la.dV = b.dV;
+    la.tile_list = b.tile_list;
+    la.n_list = g.n_t / 2;
+    la.n_kv = g.n_t / 2;
+    ELSAA_TRY(cuda_status(launch_dq_tc(la, gv, w.flag, st), "sortLSH level dq"));
+    ELSAA_TRY(cuda_status(launch_dkdv_tc(la, gv, w.flag, st), "sortLSH level dkdv"));
+    ELSAA_TRY(cuda_status(launch_lsh_invert_orders(s.lsh_order, b.inv, lv, g, st), "order inverses"));
+    ELSAA_TRY(cuda_status(launch_lsh_collect(b.dQ, w.dQacc, nullptr, nullptr, b.inv, lv, false, g, st), "sortLSH dQ"));
+    ELSAA_TRY(cuda_status(launch_lsh_collect(b.dK, w.dKacc, b.dV, w.dVacc, b.inv, lv, true, g, st),
                           "sortLSH dK, dV"));
   }
   // base pass in the caller's order: adds the accumulators before the single rounding

@@ -26,6 +26,9 @@ struct FwdArgs {
   void* Olr;      // O_lr saved for the backward
   const void* Psplit;  // prefix statistics per chunk as bf16 hi/lo [BH][n_c][2][r][d] (tensor-core RACE path)
   const float* Pmass;  // their key-mass column [BH][n_c][r]
+  // optional: the query tiles to run, n_list per head ([BH][n_list]); null runs all tiles
+  const int* tile_list;
+  int n_list;
 };
 
 // Per-row adjoint scalars of the fusion (Eq. 4 / Eq. 5), float32 [BH, N] each.
@@ -59,6 +62,11 @@ struct BwdArgs {
   const float* Rmass;
   const void* Wsplit;            // W as bf16 hi/lo rows n = 4 l + b, [2][NW][d]
   void *dQ, *dK, *dV;
+  // optional (tensor-core sparse kernels): the query tiles dQ runs, n_list per head
+  // ([BH][n_list], null: all), and how many key blocks dK/dV runs in kv_order (0: all)
+  const int* tile_list;
+  int n_list;
+  int n_kv;
 };
 
 // sortLSH selector: per head the sorted query and key orders, int32 [BH][2][N]
@@ -85,7 +93,9 @@ cudaError_t launch_lsh_invert_orders(const int* order, int* inv, int levels, con
 cudaError_t launch_lsh_collect(const void* src0, float* acc0, const void* src1, float* acc1, const int* inv,
                                int levels, bool keys, const Geom& g, cudaStream_t st);
 cudaError_t launch_gather_rows(const void* const* src, void* const* dst, int n, const int* perm, int row_bytes,
-                               int perm_stride, int h, int half, const Geom& g, cudaStream_t st);
+                               int levels, int half, const Geom& g, cudaStream_t st);
+// Every level's selection ([levels][BH][n_t], k = 1) and its future tiles ([levels][BH][n_t / 2]).
+cudaError_t launch_causal_lsh_select_levels(int* idx, int* tile_list, int levels, const Geom& g, cudaStream_t st);
 // Row permutation of [BH][N] rows of row_bytes (a multiple of 16): gather dst[r] = src[perm[r]]
 // or scatter dst[perm[r]] = src[r]; perm advances by perm_stride per head.
 cudaError_t launch_permute_rows(const void* src, void* dst, const int* perm, int row_bytes, const Geom& g,

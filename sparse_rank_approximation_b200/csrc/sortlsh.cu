@@ -395,27 +395,47 @@ __global__ void lsh_collect_kernel(const __nv_bfloat16* __restrict__ src0, float
   }
 }
 
-// Several row-major tensors with the same rows gathered by one order: dst_t[p] =
-// src_t[perm[p]] for up to four tensors, 16-byte units; half >= 0 moves only the
-// positions in the past (0) or future (1) halves of h rows.
+// Every level's sorted rows, gathered into level slots: for level l (halves of
+// h_l = N >> (l + 1) rows, orders at perm + l BH perm_stride), dst_t[l][bh][p] =
+// src_t[bh][perm_l[p]] for up to four tensors, 16-byte units; half >= 0 moves only the
+// positions in the past (0) or future (1) halves.
 struct RowMoves {
   const uint4* src[4];
   uint4* dst[4];
   int n;
 };
 
-__global__ void gather_rows_kernel(RowMoves mv, const int* __restrict__ perm, int units, int perm_stride, int h,
-                                   int half, Geom g) {
-  const size_t total = (size_t)g.BH * g.N * units;
+__global__ void gather_rows_kernel(RowMoves mv, const int* __restrict__ perm, int units, int levels, int half,
+                                   Geom g) {
+  const size_t rows = (size_t)g.BH * g.N;
+  const size_t total = (size_t)levels * rows * units;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
-    const size_t row = e / units;
+    const size_t row = e / units;                     // slot row: [levels][BH][N]
     const int u = (int)(e % units);
-    const int bh = (int)(row / g.N), r = (int)(row % g.N);
-    if (half >= 0 && ((r / h) & 1) != half) continue;
-    const size_t pr = (size_t)bh * g.N + perm[(size_t)bh * perm_stride + r];
+    const int l = (int)(row / rows);
+    const size_t hr = row % rows;
+    const int bh = (int)(hr / g.N), r = (int)(hr % g.N);
+    if (half >= 0 && ((r >> (31 - __clz(g.N >> (l + 1)))) & 1) != half) continue;
+    const size_t pr = (size_t)bh * g.N + perm[((size_t)l * g.BH + bh) * 2 * g.N + r];
 #pragma unroll
     for (int t = 0; t < 4; ++t)
       if (t < mv.n) mv.dst[t][row * units + u] = mv.src[t][pr * units + u];
+  }
+}
+
+// Every level's selection and future tiles (halves of hb_l = n_t >> (l + 1) blocks): idx
+// [levels][BH][n_t] (a future tile takes the block hb_l before it, a past tile none) and
+// tile_list [levels][BH][n_t / 2] (the future tiles, in block order).
+__global__ void causal_lsh_select_levels_kernel(int* __restrict__ idx, int* __restrict__ tile_list, int levels,
+                                                Geom g) {
+  const size_t total = (size_t)levels * g.BH * g.n_t;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t vh = e / g.n_t;                      // level-major virtual head
+    const int l = (int)(vh / g.BH), t = (int)(e % g.n_t);
+    const int hb = g.n_t >> (l + 1);
+    const bool future = (t / hb) & 1;
+    idx[e] = future ? t - hb : -1;
+    if (future) tile_list[vh * (g.n_t / 2) + (t / (2 * hb)) * hb + (t % hb)] = t;
   }
 }
 
@@ -529,7 +549,7 @@ cudaError_t launch_lsh_collect(const void* src0, float* acc0, const void* src1, 
 }
 
 cudaError_t launch_gather_rows(const void* const* src, void* const* dst, int n, const int* perm, int row_bytes,
-                               int perm_stride, int h, int half, const Geom& g, cudaStream_t st) {
+                               int levels, int half, const Geom& g, cudaStream_t st) {
   if (n < 1 || n > 4) return cudaErrorInvalidValue;
   RowMoves mv{};
   for (int t = 0; t < n; ++t) {
@@ -539,8 +559,14 @@ cudaError_t launch_gather_rows(const void* const* src, void* const* dst, int n, 
   mv.n = n;
   const int units = row_bytes / 16;
   ProfScope ps("sortlsh_gather", st);
-  gather_rows_kernel<<<elementwise_blocks((size_t)g.BH * g.N * units), 256, 0, st>>>(mv, perm, units, perm_stride, h,
-                                                                                     half, g);
+  gather_rows_kernel<<<elementwise_blocks((size_t)levels * g.BH * g.N * units), 256, 0, st>>>(mv, perm, units, levels,
+                                                                                              half, g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_causal_lsh_select_levels(int* idx, int* tile_list, int levels, const Geom& g, cudaStream_t st) {
+  causal_lsh_select_levels_kernel<<<elementwise_blocks((size_t)levels * g.BH * g.n_t), 256, 0, st>>>(idx, tile_list,
+                                                                                                     levels, g);
   return cudaGetLastError();
 }
 
