@@ -398,42 +398,68 @@ def main():
     value = tokens_step / (ms_step * 1e-3)
     launches = sum(c for _, c in prof.values())
 
-    # end to end: pinned host inputs in, results (O and the three gradients) out, every step
+    # end to end: pinned host inputs in, results (O and the three gradients) out, every step.
+    # Two sets of device inputs and outputs: step i copies its inputs in on an H2D stream,
+    # computes on the compute stream and copies its results out on a D2H stream, so step
+    # i+1's inputs and step i-1's results cross PCIe (full duplex) while step i computes.
+    # A set is rewritten only after the step that last used it is done with it.
     e2e = None
     if not args.no_e2e:
-        host = {n: inp[n + key].pin_memory() for n in ("Q", "K", "V", "dO")}
+        names = ("Q", "K", "V", "dO")
+        host = {n: inp[n + key].pin_memory() for n in names}
         host_W = inp["W"].pin_memory()
         host_R = inp["R"].pin_memory() if lsh else None
-        outs = [torch.empty(O.shape, dtype=O.dtype).pin_memory() for _ in range(4)]
+        outs = [[torch.empty(O.shape, dtype=O.dtype).pin_memory() for _ in range(4)] for _ in range(2)]
         h2d = (sum(x.numel() * x.element_size() for x in host.values()) + host_W.numel() * 4
                + (host_R.numel() * 4 if lsh else 0))
-        d2h = sum(x.numel() * x.element_size() for x in outs)
+        d2h = sum(x.numel() * x.element_size() for x in outs[0])
+        dsets = [dict(Q=q, K=k, V=v, dO=dO, W=W),
+                 {n: torch.empty_like(t) for n, t in dict(Q=q, K=k, V=v, dO=dO, W=W).items()}]
+        osets = [(O,) + grads, tuple(torch.empty_like(O) for _ in range(4))]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        comp_done = [torch.cuda.Event() for _ in range(2)]
+        out_done = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            q.copy_(host["Q"], non_blocking=True)
-            k.copy_(host["K"], non_blocking=True)
-            v.copy_(host["V"], non_blocking=True)
-            dO.copy_(host["dO"], non_blocking=True)
-            W.copy_(host_W, non_blocking=True)
-            if lsh:
+        def e2e_step(i):
+            j = i % 2
+            d, o = dsets[j], osets[j]
+            s_in.wait_event(comp_done[j])             # step i-2 has finished reading set j
+            with torch.cuda.stream(s_in):
+                for n in names:
+                    d[n].copy_(host[n], non_blocking=True)
+                d["W"].copy_(host_W, non_blocking=True)
+                in_ready[j].record(s_in)
+            stream.wait_event(in_ready[j])
+            stream.wait_event(out_done[j])            # step i-2's results have left set j
+            if lsh:                                   # the planes live at one address, in stream order
                 R.copy_(host_R, non_blocking=True)
-            step()
-            for hsrc, dsrc in zip(outs, (O,) + grads):
-                hsrc.copy_(dsrc, non_blocking=True)
+            op.forward(d["Q"], d["K"], d["V"], d["W"], out=o[0], stream=stream)
+            op.backward(d["Q"], d["K"], d["V"], d["W"], d["dO"], grads=o[1:], stream=stream)
+            comp_done[j].record(stream)
+            s_out.wait_event(comp_done[j])
+            with torch.cuda.stream(s_out):
+                for hdst, dsrc in zip(outs[j], o):
+                    hdst.copy_(dsrc, non_blocking=True)
+                out_done[j].record(s_out)
 
-        for _ in range(2):
-            e2e_step()
+        for i in range(4):
+            e2e_step(i)
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_e2e = max(3, args.steps // 4)
+        n_e2e = max(4, args.steps // 4)
         e0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
+        s_in.wait_event(e0)
+        for i in range(n_e2e):
+            e2e_step(i)
+        stream.wait_event(out_done[(n_e2e - 1) % 2])
+        stream.wait_event(out_done[n_e2e % 2])
         e1.record(stream)
         barrier()
         te = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dev)
         e2e = {"value": tokens_step / (te * 1e-3), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": te}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": te,
+               "pipelined": "double-buffered: step i+1's H2D and step i-1's D2H overlap step i's compute"}
 
     if world > 1:
         dist.destroy_process_group()
