@@ -82,3 +82,25 @@ def check_fusion_grads(w: Workload, h: int, p: orc.Params, fw: dict, ex: dict, d
     for name, g, want, bnd in zip(("dlambda", "dg_s", "dg_lr"), got, ref, bounds):
         err = np.abs(np64(g[0, h]) - want)
         assert np.all(err <= BF16_ABS_TOL + 2.0 ** -8 * bnd), f"{name}[{h}]: max err {err.max():.3e}"
+
+
+def sparse_rounding_scales(q, k, v, dO, fw, p, lam=None, g_s=None, g_lr=None):
+    """Per-element scales of the bf16 rounding inside the sparse backward, from the oracle's
+    own quantities: dS is rounded before dS K and dS^T Q, P before P^T dO_s, and Delta is a
+    row sum over the bf16-saved O_s, so it is off by up to 2^-9 sum_c |dO_s,ic O_s,ic|, which
+    every dS_ij = P_ij (dP_ij - Delta_i) inherits times P_ij.  When one key dominates a row,
+    dP_ij and Delta_i nearly cancel and that last term is the whole of dS_ij's error."""
+    dOs, _, dds_ds, _ = orc._fusion_adjoints(dO, fw, p, lam, g_s, g_lr)
+    Delta = (dOs * fw["O_s"]).sum(axis=1) - dds_ds
+    eD = (np.abs(dOs) * np.abs(fw["O_s"])).sum(axis=1)
+    Bq, Bk, Bv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    sup = orc.lsh_support(q, k, p) if p.selector == "sortlsh" else orc.support(fw["idx"], p)
+    for i, keys in enumerate(sup):
+        if keys.size == 0:
+            continue
+        P = np.exp(p.scale * (k[keys] @ q[i]) - fw["logd_s"][i])
+        dz = np.abs(P * (v[keys] @ dOs[i] - Delta[i])) + P * eD[i]
+        Bq[i] += p.scale * dz @ np.abs(k[keys])
+        Bk[keys] += p.scale * np.outer(dz, np.abs(q[i]))
+        Bv[keys] += np.outer(P, np.abs(dOs[i]))
+    return Bq, Bk, Bv

@@ -11,7 +11,8 @@ import torch
 from oracle import elsaa_oracle as orc
 from sparse_rank_approximation_b200 import binding as bd
 from sparse_rank_approximation_b200.workloads import WORKLOADS, make_inputs, small_workload
-from tests.harness import BF16_ABS_TOL, BF16_STORE_REL, check, check_fusion_grads, device_inputs, gpu_op, np64, oracle_params
+from tests.harness import (BF16_ABS_TOL, BF16_STORE_REL, check, check_fusion_grads, device_inputs, gpu_op, np64,
+                           oracle_params, sparse_rounding_scales)
 
 pytestmark = pytest.mark.gpu
 
@@ -102,25 +103,6 @@ def test_forward_backward(geom, gates, fixed_m):
         check_fusion_grads(w, h, p, fw, ex, get("dO"), (dl, dgs, dgl), ref)
 
 
-def _sparse_rounding_scales(q, k, v, dO, fw, p):
-    """Per-element scales of the bf16 rounding inside the sparse backward, from the oracle's
-    own quantities: dS is rounded before dS K and dS^T Q, P before P^T dO_s, and Delta is a
-    row sum over the bf16-saved O_s, so it is off by up to 2^-9 sum_c |dO_s,ic O_s,ic|, which
-    every dS_ij = P_ij (dP_ij - Delta_i) inherits times P_ij.  When one key dominates a row,
-    dP_ij and Delta_i nearly cancel and that last term is the whole of dS_ij's error."""
-    dOs, _, dds_ds, _ = orc._fusion_adjoints(dO, fw, p, None, None, None)
-    Delta = (dOs * fw["O_s"]).sum(axis=1) - dds_ds
-    eD = (np.abs(dOs) * np.abs(fw["O_s"])).sum(axis=1)
-    Bq, Bk, Bv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
-    for i, keys in enumerate(orc.lsh_support(q, k, p)):
-        P = np.exp(p.scale * (k[keys] @ q[i]) - fw["logd_s"][i])
-        dz = np.abs(P * (v[keys] @ dOs[i] - Delta[i])) + P * eD[i]
-        Bq[i] += p.scale * dz @ np.abs(k[keys])
-        Bk[keys] += p.scale * np.outer(dz, np.abs(q[i]))
-        Bv[keys] += np.outer(P, np.abs(dOs[i]))
-    return Bq, Bk, Bv
-
-
 def test_full_size():
     """The full-length sortLSH workload (B1 H32 N16384 d128, 7-bit codes), launched as the
     benchmark launches it; every row of two heads against the oracle on the GPU's orders."""
@@ -143,7 +125,7 @@ def test_full_size():
         # the gradients: the usual bf16 bound plus the rounding inside the sparse backward
         # (twice its half-ulp scale); at this length sorted blocks put most of a row's
         # mass on a few keys, where the Delta term dominates
-        scales = _sparse_rounding_scales(get("Q"), get("K"), get("V"), get("dO"), fw, p)
+        scales = sparse_rounding_scales(get("Q"), get("K"), get("V"), get("dO"), fw, p)
         for name, got, ref, B in zip(("dQ", "dK", "dV"), (dQ, dK, dV), (dq, dk, dv), scales):
             err = np.abs(np64(got[0, h]) - ref)
             excess = (err - BF16_STORE_REL * np.abs(ref) - 2.0 ** -8 * B).max()
@@ -191,7 +173,7 @@ def test_causal_forward_backward(N, r, gates, fixed_m):
                              ex_dev.get("g_s"), ex_dev.get("g_lr"))
     dl, dgs, dgl = op.fusion_grads(dev["dO"], ex_dev.get("lam"), ex_dev.get("g_s"), ex_dev.get("g_lr"))
     codes, _ = op.debug_sortlsh(dev["Q"], dev["K"])
-    op.check_device_flags()
+    assert op.check_device_flags() == 0
     torch.cuda.synchronize()
     W = inp["W"].double().numpy()
     for h in range(w.H):
@@ -220,7 +202,7 @@ def test_causal_full_size():
     O = op.forward(dev["Q"], dev["K"], dev["V"], dev["W"])
     dQ, dK, dV = op.backward(dev["Q"], dev["K"], dev["V"], dev["W"], dev["dO"])
     codes, _ = op.debug_sortlsh(dev["Q"], dev["K"])
-    op.check_device_flags()
+    assert op.check_device_flags() == 0
     torch.cuda.synchronize()
     W = inp["W"].double().numpy()
     for h in (0, w.H - 1):
@@ -229,7 +211,7 @@ def test_causal_full_size():
         fw = orc.forward_head(get("Q"), get("K"), get("V"), W, p)
         dq, dk, dv = orc.backward_head(get("Q"), get("K"), get("V"), W, get("dO"), fw, p)
         check(w, f"O[{h}]", np64(O[0, h]), fw["O"])
-        scales = _sparse_rounding_scales(get("Q"), get("K"), get("V"), get("dO"), fw, p)
+        scales = sparse_rounding_scales(get("Q"), get("K"), get("V"), get("dO"), fw, p)
         for name, got, ref, B in zip(("dQ", "dK", "dV"), (dQ, dK, dV), (dq, dk, dv), scales):
             err = np.abs(np64(got[0, h]) - ref)
             excess = (err - BF16_STORE_REL * np.abs(ref) - 2.0 ** -8 * B).max()
