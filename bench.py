@@ -326,6 +326,7 @@ def main():
     ap.add_argument("--impl", default="elsaa", choices=["elsaa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads (a smaller case for ncu captures)")
     args = ap.parse_args()
@@ -397,6 +398,31 @@ def main():
     tokens_step = w.B * w.N * world
     value = tokens_step / (ms_step * 1e-3)
     launches = sum(c for _, c in prof.values())
+
+    # the same step captured once in a CUDA graph and replayed K times: what is left when
+    # the host launch path is taken out (reported beside the eager `value`)
+    graph_line = None
+    if not args.no_graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(3):
+            graph.replay()
+        barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        g1.record(stream)
+        barrier()
+        tg = max_over_ranks(g0.elapsed_time(g1) / args.steps, dev)
+        graph_line = {"ms_per_step": tg, "value": tokens_step / (tg * 1e-3), "unit": UNIT}
+        del graph
 
     # end to end: pinned host inputs in, results (O and the three gradients) out, every step.
     # Two sets of device inputs and outputs: step i copies its inputs in on an H2D stream,
@@ -508,7 +534,7 @@ def main():
             "config": {"workload": w.name, "shape": w.describe(), "global_batch": w.B * world,
                        "seq_len": w.N, "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (Q, K, V, dO: 4 x %.0f MB)" % (q.numel() * 2 / 1e6)},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "graph": graph_line,
             "clocks": clk.summary(),
             "north_star_roofline": north_star_roofline(w, peaks, ms_step),
             "kernels": kernels}
