@@ -541,35 +541,39 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     // every product has completed: stage dK in the stage-0 Q buffer and dV in the stage-0 dO buffer
 #pragma unroll 1
     for (int which = 0; which < 2; ++which) {
-      float o[64];
+      const float mul = which == 0 ? g.scale : 1.f;
+      const float* accp = which == 0 ? a.dKacc : a.dVacc;
+      const float4* ak = accp && alive && key_ok
+                             ? reinterpret_cast<const float4*>(accp + (head + (size_t)b * kT + row) * kD + 64 * hq)
+                             : nullptr;
+      unsigned char* orow = smem + (which == 0 ? kv_q(0) : kv_do(0)) + hq * kSlab + row * 128;
+      // 32 columns at a time: TMEM -> scale -> + low-rank part -> bf16 -> swizzled row
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float o[32];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) o[c] = 0.f;
-      if (have) {
-        const float mul = which == 0 ? g.scale : 1.f;
-        float tmp[32];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tc::tmem_ld32(tmem + lane_base + (which == 0 ? TM_DK : TM_DV) + 64 * hq + 32 * c, tmp);
+        for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        if (have) {
+          tc::tmem_ld32(tmem + lane_base + (which == 0 ? TM_DK : TM_DV) + 64 * hq + 32 * c, o);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[32 * c + i] = tmp[i] * mul;
+          for (int i = 0; i < 32; ++i) o[i] *= mul;
+        }
+        if (ak) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 x = ak[8 * c + q];
+            o[4 * q] += x.x; o[4 * q + 1] += x.y; o[4 * q + 2] += x.z; o[4 * q + 3] += x.w;
+          }
+        }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int ch = 4 * c + cc;
+          *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) =
+              make_uint4(pack_bf16(o[8 * cc], o[8 * cc + 1]), pack_bf16(o[8 * cc + 2], o[8 * cc + 3]),
+                         pack_bf16(o[8 * cc + 4], o[8 * cc + 5]), pack_bf16(o[8 * cc + 6], o[8 * cc + 7]));
         }
       }
-      const float* accp = which == 0 ? a.dKacc : a.dVacc;
-      if (alive && key_ok && accp) {
-        const float4* ak = reinterpret_cast<const float4*>(accp + (head + (size_t)b * kT + row) * kD + 64 * hq);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float4 x = ak[c];
-          o[4 * c] += x.x; o[4 * c + 1] += x.y; o[4 * c + 2] += x.z; o[4 * c + 3] += x.w;
-        }
-      }
-      unsigned char* orow = smem + (which == 0 ? kv_q(0) : kv_do(0)) + hq * kSlab + row * 128;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) =
-            make_uint4(pack_bf16(o[8 * ch], o[8 * ch + 1]), pack_bf16(o[8 * ch + 2], o[8 * ch + 3]),
-                       pack_bf16(o[8 * ch + 4], o[8 * ch + 5]), pack_bf16(o[8 * ch + 6], o[8 * ch + 7]));
     }
     tc::fence_proxy_async_smem();
     softmax_bar();
