@@ -264,41 +264,42 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       tc::mbar_arrive(&ms->ds_full[j & 1]);
     }
     // ---------------- epilogue: dQ = scale dQ_sparse + dQ_lowrank, bf16 TMA store ----------------
-    float o[64];
-#pragma unroll
-    for (int c = 0; c < 64; ++c) o[c] = 0.f;
+    bool have = false;
     if (alive && n_sel > 0) {
       alive = __all_sync(0xffffffffu, wait_or_abort(&ms->done, 0, ms, err, 256u));
-      if (alive) {
-        tc::tc_fence_after();
-        float tmp[32];
+      have = alive;
+      if (have) tc::tc_fence_after();
+    }
+    const float4* acc =
+        alive && row_ok && a.dQacc ? reinterpret_cast<const float4*>(a.dQacc + (head + qrow) * kD + 64 * half) : nullptr;
+    // every product has completed: stage the bf16 tile in the Q buffer, 32 columns at a time
+    unsigned char* orow = smem + DQ_Q + half * kSlab + row * 128;
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      float o[32];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tc::tmem_ld32(tmem + lane_base + TM_DQ + 64 * half + 32 * c, tmp);
-          tc::tmem_wait_ld();
+      for (int i = 0; i < 32; ++i) o[i] = 0.f;
+      if (have) {
+        tc::tmem_ld32(tmem + lane_base + TM_DQ + 64 * half + 32 * c, o);
+        tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[32 * c + i] = tmp[i] * g.scale;
+        for (int i = 0; i < 32; ++i) o[i] *= g.scale;
+      }
+      if (acc) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 v = acc[8 * c + q];
+          o[4 * q] += v.x; o[4 * q + 1] += v.y; o[4 * q + 2] += v.z; o[4 * q + 3] += v.w;
         }
       }
-    }
-    if (alive && row_ok && a.dQacc) {
-      const float4* acc = reinterpret_cast<const float4*>(a.dQacc + (head + qrow) * kD + 64 * half);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float4 v = acc[c];
-        o[4 * c] += v.x;
-        o[4 * c + 1] += v.y;
-        o[4 * c + 2] += v.z;
-        o[4 * c + 3] += v.w;
+      for (int cc = 0; cc < 4; ++cc) {
+        const int ch = 4 * c + cc;
+        *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) =
+            make_uint4(pack_bf16(o[8 * cc], o[8 * cc + 1]), pack_bf16(o[8 * cc + 2], o[8 * cc + 3]),
+                       pack_bf16(o[8 * cc + 4], o[8 * cc + 5]), pack_bf16(o[8 * cc + 6], o[8 * cc + 7]));
       }
     }
-    // every product has completed: stage the bf16 tile in the Q buffer
-    unsigned char* orow = smem + DQ_Q + half * kSlab + row * 128;
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch)
-      *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) =
-          make_uint4(pack_bf16(o[8 * ch], o[8 * ch + 1]), pack_bf16(o[8 * ch + 2], o[8 * ch + 3]),
-                     pack_bf16(o[8 * ch + 4], o[8 * ch + 5]), pack_bf16(o[8 * ch + 6], o[8 * ch + 7]));
     tc::fence_proxy_async_smem();
     softmax_bar();
     if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {

@@ -277,18 +277,19 @@ __global__ void lsh_fuse_kernel(const __nv_bfloat16* __restrict__ Os0, const flo
     const int u = (int)(e % units);
     const int bh = (int)(row / g.N), r = (int)(row % g.N);
     // the partials this row has: base (slot 0), then one per level where it is in a
-    // future half; every level's loads are issued before any is used
-    const __nv_bfloat16* src[kMaxLevels + 1];
+    // future half.  Every partial's log-denominator and row are loaded as soon as its
+    // position is known (predicated loads, no branch on the values)
+    uint4 w[kMaxLevels + 1];
     float lg[kMaxLevels + 1];
-    src[0] = Os0 + row * g.d + 8 * u;
+    w[0] = *reinterpret_cast<const uint4*>(Os0 + row * g.d + 8 * u);
     lg[0] = logd0[row];
 #pragma unroll
     for (int l = 0; l < kMaxLevels; ++l) {
       lg[l + 1] = -INFINITY;
-      src[l + 1] = nullptr;
+      w[l + 1] = make_uint4(0u, 0u, 0u, 0u);
       if (l < levels && ((r / (g.N >> (l + 1))) & 1)) {
         const size_t p = (size_t)l * rows + (size_t)bh * g.N + inv_lv[(size_t)l * rows + row];
-        src[l + 1] = Os_lv + p * g.d + 8 * u;
+        w[l + 1] = *reinterpret_cast<const uint4*>(Os_lv + p * g.d + 8 * u);
         lg[l + 1] = logd_lv[p];
       }
     }
@@ -299,11 +300,9 @@ __global__ void lsh_fuse_kernel(const __nv_bfloat16* __restrict__ Os0, const flo
     if (L > -INFINITY) {
 #pragma unroll
       for (int j = 0; j <= kMaxLevels; ++j) {
-        if (lg[j] == -INFINITY) continue;
-        const float wj = __expf(lg[j] - L);
+        const float wj = lg[j] == -INFINITY ? 0.f : __expf(lg[j] - L);
         sum += wj;
-        const uint4 w = *reinterpret_cast<const uint4*>(src[j]);
-        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w[j]);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float2 f = __bfloat1622float2(hv[k]);
@@ -321,8 +320,8 @@ __global__ void lsh_fuse_kernel(const __nv_bfloat16* __restrict__ Os0, const flo
     const float mf = g.fixed_m ? 1.f : L == -INFINITY ? 0.f : 1.f / (1.f + (lam * dlr[row] + g.eps) * __expf(-L));
     const float gl = glrv ? glrv[row] : g.fixed_m ? 1.f : 1.f - mf;
     const float cs = gs * mf;
-    const uint4 w = *reinterpret_cast<const uint4*>(Olr + row * g.d + 8 * u);
-    const __nv_bfloat162* lv = reinterpret_cast<const __nv_bfloat162*>(&w);
+    const uint4 wl = *reinterpret_cast<const uint4*>(Olr + row * g.d + 8 * u);
+    const __nv_bfloat162* lv = reinterpret_cast<const __nv_bfloat162*>(&wl);
     uint32_t wo[4], ws[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -541,6 +540,7 @@ cudaError_t launch_lsh_invert_orders(const int* order, int* inv, int levels, con
 
 cudaError_t launch_lsh_collect(const void* src0, float* acc0, const void* src1, float* acc1, const int* inv,
                                int levels, bool keys, const Geom& g, cudaStream_t st) {
+  if (levels > kMaxLevels) return cudaErrorInvalidValue;
   ProfScope ps("lsh_collect", st);
   lsh_collect_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
       (const __nv_bfloat16*)src0, acc0, (const __nv_bfloat16*)src1, acc1, inv, levels, keys ? 1 : 0, keys ? 0 : 1,
