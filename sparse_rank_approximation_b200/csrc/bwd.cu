@@ -37,14 +37,19 @@ __device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
   v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
 }
 
-// Row scalars (see the header comment).  grid (ceil(N / rows_per_block), BH), block 256;
-// d/8 threads per row, 8 elements each.  The scalar algebra runs in float64.
+// Row scalars (see the header comment).  grid (ceil(N / rows_per_block), BH), block 256.
+// d/8 threads per row reduce the row's <dO, O_s> and <dO, O_lr> (8 elements each); then
+// one thread per row (the block's first rows_per_block threads, so a warp covers 16 or 32
+// consecutive rows) runs the scalar algebra in float64 and writes the per-row outputs;
+// cl comes back through shared memory for the cl dO rows.
 template <typename E>
 __global__ void __launch_bounds__(256) row_scalars_kernel(BwdArgs a, Geom g) {
+  __shared__ float sA[32], sB[32], sCl[32];
   const int tpr = g.d / 8;
   const int rpb = 256 / tpr;
   const int sub = threadIdx.x % tpr;
-  const int row = blockIdx.x * rpb + threadIdx.x / tpr;
+  const int lr = threadIdx.x / tpr;
+  const int row = blockIdx.x * rpb + lr;
   const size_t i = (size_t)blockIdx.y * g.N + min(row, g.N - 1);
   float dO[8], os[8], ol[8];
   load8<E>((const E*)a.dO + i * g.d + sub * 8, dO);
@@ -60,20 +65,46 @@ __global__ void __launch_bounds__(256) row_scalars_kernel(BwdArgs a, Geom g) {
     A += __shfl_xor_sync(0xffffffffu, A, o);
     Bv += __shfl_xor_sync(0xffffffffu, Bv, o);
   }
-  // cl = g_lr / d_lr, broadcast from the row's first lane: the rows cl dO (bf16) feed the
-  // RACE suffix statistics
-  if (a.dOcl) {
-    double cl_row = 0.0;
-    if (sub == 0 && row < g.N) {
-      const double logd0 = a.logd[i], dl0 = a.dlr[i];
-      const double lam0 = a.lam ? a.lam[i] : g.lam;
-      const double c0 = lam0 * dl0 + (double)g.eps;
-      const double D0 = exp(logd0) + c0;
-      const double gl0 = a.glr ? (double)a.glr[i] : g.fixed_m ? 1.0 : (D0 > 0.0 ? c0 / D0 : 1.0);
-      cl_row = dl0 > 0.0 ? gl0 / dl0 : 0.0;
+  if (sub == 0) {
+    sA[lr] = A;
+    sB[lr] = Bv;
+  }
+  __syncthreads();
+  if ((int)threadIdx.x < rpb) {
+    const int r = blockIdx.x * rpb + threadIdx.x;
+    float clv = 0.f;
+    if (r < g.N) {
+      const size_t k = (size_t)blockIdx.y * g.N + r;
+      const double Ar = sA[threadIdx.x], Br = sB[threadIdx.x];
+      const double logd = a.logd[k], dl = a.dlr[k];
+      const double lam = a.lam ? a.lam[k] : g.lam;
+      const double gs = a.gs ? a.gs[k] : 1.0;
+      const double ds = exp(logd);
+      const double c = lam * dl + (double)g.eps;
+      const double D = ds + c;
+      // fixed_m: the ablation without denominator-aware fusion (m = 1, default g_lr = 1, no dm)
+      const double m = g.fixed_m ? 1.0 : D > 0.0 ? ds / D : 0.0;
+      const double one_m = g.fixed_m ? 0.0 : D > 0.0 ? c / D : 1.0;
+      const double gl = a.glr ? (double)a.glr[k] : g.fixed_m ? 1.0 : one_m;
+      const double dm = g.fixed_m ? 0.0 : gs * Ar - (a.glr ? 0.0 : Br);
+      const double cs = gs * m;
+      const double cl = dl > 0.0 ? gl / dl : 0.0;
+      const double ddlr = D > 0.0 ? -dm * lam * ds / (D * D) : 0.0;
+      const double Dl = cs * Ar - dm * m * one_m;
+      a.rs.cs[k] = (float)cs;
+      a.rs.Delta[k] = (float)Dl;
+      if (a.rs.packed) a.rs.packed[k] = make_float4((float)(logd * 1.4426950408889634), (float)cs, (float)Dl, 0.f);
+      a.rs.cl[k] = (float)cl;
+      a.rs.delta[k] = (float)(ddlr - cl * Br);
+      clv = (float)cl;
     }
-    const float clf = __shfl_sync(0xffffffffu, (float)cl_row, (threadIdx.x & 31) - sub);
+    sCl[threadIdx.x] = clv;
+  }
+  // the rows cl dO (bf16) feed the RACE suffix statistics
+  if (a.dOcl) {
+    __syncthreads();
     if (row < g.N) {
+      const float clf = sCl[lr];
       uint4 w;
       w.x = pack_bf16(clf * dO[0], clf * dO[1]);
       w.y = pack_bf16(clf * dO[2], clf * dO[3]);
@@ -82,27 +113,6 @@ __global__ void __launch_bounds__(256) row_scalars_kernel(BwdArgs a, Geom g) {
       *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dOcl) + i * g.d + sub * 8) = w;
     }
   }
-  if (sub != 0 || row >= g.N) return;
-  const double logd = a.logd[i], dl = a.dlr[i];
-  const double lam = a.lam ? a.lam[i] : g.lam;
-  const double gs = a.gs ? a.gs[i] : 1.0;
-  const double ds = exp(logd);
-  const double c = lam * dl + (double)g.eps;
-  const double D = ds + c;
-  // fixed_m: the ablation without denominator-aware fusion (m = 1, default g_lr = 1, no dm)
-  const double m = g.fixed_m ? 1.0 : D > 0.0 ? ds / D : 0.0;
-  const double one_m = g.fixed_m ? 0.0 : D > 0.0 ? c / D : 1.0;
-  const double gl = a.glr ? (double)a.glr[i] : g.fixed_m ? 1.0 : one_m;
-  const double dm = g.fixed_m ? 0.0 : gs * A - (a.glr ? 0.0 : (double)Bv);
-  const double cs = gs * m;
-  const double cl = dl > 0.0 ? gl / dl : 0.0;
-  const double ddlr = D > 0.0 ? -dm * lam * ds / (D * D) : 0.0;
-  a.rs.cs[i] = (float)cs;
-  a.rs.Delta[i] = (float)(cs * A - dm * m * one_m);
-  if (a.rs.packed)
-    a.rs.packed[i] = make_float4((float)(logd * 1.4426950408889634), (float)cs, (float)(cs * A - dm * m * one_m), 0.f);
-  a.rs.cl[i] = (float)cl;
-  a.rs.delta[i] = (float)(ddlr - cl * Bv);
 }
 
 // Per-row gradients of sum(dO * O) with respect to lambda, g_s and g_lr (Eq. 5 / Eq. 4):
