@@ -88,7 +88,7 @@ typedef enum { ELSAA_DTYPE_F32 = 0, ELSAA_DTYPE_BF16 = 1 } elsaa_dtype;
  *     gives the extra block to the past); each half recurses; the future queries
  *     attend the past keys by non-causal sortLSH on the two halves; the future
  *     half's results merge by log-sum-exp; a single block is attended exactly under
- *     j <= i.  Needs bf16, d = 128, block_size 128 and N = 128 * 2^L <= 32768. */
+ *     j <= i.  Needs bf16 and N = block_size * 2^L <= 32768. */
 typedef enum { ELSAA_SEL_TOPK_BLOCKS = 0, ELSAA_SEL_SORTLSH = 1 } elsaa_selector;
 
 typedef struct {

@@ -232,9 +232,16 @@ __global__ void __launch_bounds__(2 * T) sparse_dq_bf16_kernel(BwdArgs a, Geom g
   for (int h = 0; h < 2; ++h) {
     const int row = t * T + rl[h];
     const bool ok = row < g.N;
-    lg2[h] = ok ? a.logd[head + row] * kLog2e : INFINITY;
-    cs[h] = ok ? a.rs.cs[head + row] : 0.f;
-    Dl[h] = ok ? a.rs.Delta[head + row] : 0.f;
+    if (a.rs.packed) {                // (log2 d_s, cs, Delta) in one row (also the gathered rows of sortLSH)
+      const float4 p = ok ? a.rs.packed[head + row] : make_float4(INFINITY, 0.f, 0.f, 0.f);
+      lg2[h] = p.x;
+      cs[h] = p.y;
+      Dl[h] = p.z;
+    } else {
+      lg2[h] = ok ? a.logd[head + row] * kLog2e : INFINITY;
+      cs[h] = ok ? a.rs.cs[head + row] : 0.f;
+      Dl[h] = ok ? a.rs.Delta[head + row] : 0.f;
+    }
   }
   if (n_sel > 0) {
     load_kv(0, my_idx[0]);
@@ -388,9 +395,16 @@ __global__ void __launch_bounds__(2 * T) sparse_dkdv_bf16_kernel(BwdArgs a, Geom
     for (int r = tid; r < T; r += NT) {
       const int row = t * T + r;
       const bool ok = row < g.N;
-      sc[r] = ok ? a.logd[head + row] * kLog2e : INFINITY;
-      sc[T + r] = ok ? a.rs.cs[head + row] : 0.f;
-      sc[2 * T + r] = ok ? a.rs.Delta[head + row] : 0.f;
+      if (a.rs.packed) {
+        const float4 p = ok ? a.rs.packed[head + row] : make_float4(INFINITY, 0.f, 0.f, 0.f);
+        sc[r] = p.x;
+        sc[T + r] = p.y;
+        sc[2 * T + r] = p.z;
+      } else {
+        sc[r] = ok ? a.logd[head + row] * kLog2e : INFINITY;
+        sc[T + r] = ok ? a.rs.cs[head + row] : 0.f;
+        sc[2 * T + r] = ok ? a.rs.Delta[head + row] : 0.f;
+      }
     }
   };
   if (n_list > 0) {
@@ -531,13 +545,10 @@ template <int D, int T>
 static cudaError_t bwd_t(const BwdArgs& a0, const Geom& g, int parts, cudaStream_t st) {
   BwdArgs a = a0;
   cudaError_t e;
-  if (g.r > 0) {
-    if (parts & 1) {
-      e = launch_race_bwd_bf16(a, g, st);
-      if (e != cudaSuccess) return e;
-    }
-  } else {
-    a.dQacc = a.dKacc = a.dVacc = nullptr;
+  // the sparse kernels add the fp32 accumulators when they are given (null: nothing to add)
+  if (g.r > 0 && (parts & 1)) {
+    e = launch_race_bwd_bf16(a, g, st);
+    if (e != cudaSuccess) return e;
   }
   const size_t lds = (size_t)(D + 8) * 2;
   if (parts & 2) {

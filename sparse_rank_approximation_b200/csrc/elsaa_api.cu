@@ -99,9 +99,10 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
       return false;
     }
     if (p->causal) {
-      // the recursion runs on the tensor-core kernels, halving down to single blocks
-      if (!bf16 || p->d != 128 || T != 128) {
-        *st = fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH needs bf16, d = 128, block_size 128");
+      // the recursion runs on the bf16 sparse kernels (tcgen05 or mma.sync), halving down
+      // to single blocks
+      if (!bf16) {
+        *st = fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH needs bf16");
         return false;
       }
       if (p->N % T || (n_t & (n_t - 1))) {
@@ -203,6 +204,10 @@ struct PermBufs {
   float *logd, *m, *logd_lv;
   int *idx, *tile_list, *offs, *tiles, *order, *pos, *inv;
   float4* packed;
+  // the sparse-only passes' low-rank outputs: the mma.sync forward writes O_lr and d_lr
+  // (zero without a low-rank branch), the tcgen05 one reads them; neither is used
+  void* Olr;
+  float* dlr;
 };
 
 PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
@@ -246,6 +251,8 @@ PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
   b.Os = c.take<char>(mat);
   b.logd = c.take<float>(rows);
   b.m = c.take<float>(std::max<size_t>(lv, 1) * rows);
+  b.Olr = c.take<char>(std::max<size_t>(lv, 1) * mat);
+  b.dlr = c.take<float>(std::max<size_t>(lv, 1) * rows);
   b.Os_lv = c.take<char>(lv * mat);
   b.logd_lv = c.take<float>(lv * rows);
   b.inv = c.take<int>(lv * rows);
@@ -304,9 +311,9 @@ BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
   w.order = c.take<int>((size_t)g.BH * g.n_t);
   const bool causal_lsh = g.selector == ELSAA_SEL_SORTLSH && g.causal;
   const size_t acc = bf16 && (g.r > 0 || causal_lsh) ? rows * g.d : 0;
-  w.dQacc = c.take<float>(acc);
-  w.dKacc = c.take<float>(acc);
-  w.dVacc = c.take<float>(acc);
+  w.dQacc = acc ? c.take<float>(acc) : nullptr;
+  w.dKacc = acc ? c.take<float>(acc) : nullptr;
+  w.dVacc = acc ? c.take<float>(acc) : nullptr;
   w.dOcl = c.take<char>(bf16 && g.r > 0 ? rows * g.d * 2 : 0);
   const bool split = bf16 && g.r > 0 && race_bwd_tc_supported(g);
   w.Rsplit = split ? c.take<char>((size_t)g.BH * g.n_c * 2 * g.r * g.d * 2) : nullptr;
@@ -435,6 +442,8 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
                                 const float* W, const float* lam, const float* gs, const float* glr, void* O,
                                 const Saved& s, const FwdWs& w, cudaStream_t st) {
   const PermBufs& b = w.pm;
+  // tcgen05 kernels for d = 128, block 128; mma.sync kernels for the other shapes
+  const bool tc = attn_fwd_tc_supported(g) && !tcgen05_disabled();
   const size_t rows = (size_t)g.BH * g.N;
   const int rb = g.d * 2, stride = 2 * g.N;
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st), "flag reset"));
@@ -445,7 +454,7 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
     ELSAA_TRY(cuda_status(launch_race_state_fwd(s.phiK, V, true, s.Ast, s.Bst, g, st), "race summaries"));
     FwdArgs ra{Q, K, V, s.idx, s.phiQ, s.phiK, s.Ast, s.Bst, lam, gs, glr, O, s.Os, s.logd, s.dlr, s.m, s.Olr,
                s.Psplit, s.Pmass};
-    if (s.Psplit) {
+    if (s.Psplit && tc) {
       ELSAA_TRY(cuda_status(launch_race_state_split(s.Ast, s.Bst, false, s.Psplit, s.Pmass, g, st),
                             "race statistics split"));
       ELSAA_TRY(cuda_status(launch_race_readout_tc(ra, g, w.flag, st), "tcgen05 race read-out"));
@@ -461,16 +470,19 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
   FwdArgs sa{};
   sa.idx = s.idx;
   sa.O = b.X;
-  sa.Olr = b.X;
+  sa.Olr = b.Olr;
   sa.Os = b.Os;
   sa.logd = b.logd;
-  sa.dlr = b.logd;
+  sa.dlr = b.dlr;
   sa.m = b.m;
   // base pass: the leaves and the deepest level, in the caller's order
   const Geom gb = sparse_only(g, true, 2);
+  auto sparse_pass = [&](const FwdArgs& fa, const Geom& fg) {
+    return tc ? launch_attn_fwd_tc(fa, fg, w.flag, st) : launch_attn_fwd_bf16(fa, fg, st);
+  };
   ELSAA_TRY(cuda_status(launch_causal_lsh_select(s.idx, 0, g, st), "causal sortLSH base selection"));
   sa.Q = Q; sa.K = K; sa.V = V;
-  ELSAA_TRY(cuda_status(launch_attn_fwd_tc(sa, gb, w.flag, st), "causal sortLSH base pass"));
+  ELSAA_TRY(cuda_status(sparse_pass(sa, gb), "causal sortLSH base pass"));
   if (g.lsh_levels > 0) {
     const int lv = g.lsh_levels;
     ELSAA_TRY(cuda_status(launch_sortlsh_hash(Q, K, true, p->lsh_planes, p->lsh_bits, b.pos, nullptr, g, st),
@@ -488,18 +500,18 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
     ELSAA_TRY(cuda_status(launch_gather_rows(kvs, kvd, 2, s.lsh_order + g.N, rb, lv, 0, g, st),
                           "sortLSH gather K, V"));
     ELSAA_TRY(cuda_status(launch_causal_lsh_select_levels(b.idx, b.tile_list, lv, g, st), "sortLSH level selection"));
-    // all levels in one launch, as lv * BH heads, over their future tiles only.  The fused
-    // output goes over each tile's own gathered queries (read before it is written), the
-    // low-rank input it does not use is read from the values
+    // all levels in one launch, as lv * BH heads (the tcgen05 kernel over their future
+    // tiles only).  The fused output, not used, goes over each tile's own gathered queries,
+    // which only that tile reads and reads before it is written
     Geom gv = sparse_only(g, false, 1);
     gv.BH = lv * g.BH;
     sa.Q = b.Q; sa.K = b.K; sa.V = b.V; sa.idx = b.idx;
-    sa.O = b.Q; sa.Olr = b.V;
+    sa.O = b.Q;
     sa.Os = b.Os_lv;
-    sa.logd = sa.dlr = b.logd_lv;
+    sa.logd = b.logd_lv;
     sa.tile_list = b.tile_list;
     sa.n_list = g.n_t / 2;
-    ELSAA_TRY(cuda_status(launch_attn_fwd_tc(sa, gv, w.flag, st), "sortLSH level pass"));
+    ELSAA_TRY(cuda_status(sparse_pass(sa, gv), "sortLSH level pass"));
   }
   return cuda_status(launch_lsh_fuse(b.Os, b.logd, b.Os_lv, b.logd_lv, b.inv, g.lsh_levels, s.Olr, s.dlr, lam, gs,
                                      glr, O, s.Os, s.logd, s.m, g, st),
@@ -508,13 +520,14 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
 
 elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const BwdWs& w, cudaStream_t st) {
   const PermBufs& b = w.pm;
+  const bool tc = bwd_tc_supported(g) && !tcgen05_disabled();
   const size_t rows = (size_t)g.BH * g.N;
   const int rb = g.d * 2, stride = 2 * g.N;
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st), "flag reset"));
   ELSAA_TRY(cuda_status(launch_row_scalars(a, true, g, st), "row scalars"));
   if (g.r > 0) {
     ELSAA_TRY(cuda_status(launch_race_state_bwd(a, true, g, st), "race suffix summaries"));
-    if (race_bwd_tc_supported(g)) {
+    if (tc && race_bwd_tc_supported(g)) {
       ELSAA_TRY(cuda_status(launch_race_state_split(w.RA, w.RB, true, w.Rsplit, w.Rmass, g, st),
                             "race statistics split"));
       ELSAA_TRY(cuda_status(launch_race_w_split(a.W, w.Wsplit, g, st), "W split"));
@@ -553,8 +566,12 @@ elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const
     la.tile_list = b.tile_list;
     la.n_list = g.n_t / 2;
     la.n_kv = g.n_t / 2;
-    ELSAA_TRY(cuda_status(launch_dq_tc(la, gv, w.flag, st), "sortLSH level dq"));
-    ELSAA_TRY(cuda_status(launch_dkdv_tc(la, gv, w.flag, st), "sortLSH level dkdv"));
+    if (tc) {
+      ELSAA_TRY(cuda_status(launch_dq_tc(la, gv, w.flag, st), "sortLSH level dq"));
+      ELSAA_TRY(cuda_status(launch_dkdv_tc(la, gv, w.flag, st), "sortLSH level dkdv"));
+    } else {                          // mma.sync: every tile and block (the empty ones are cheap)
+      ELSAA_TRY(cuda_status(launch_bwd_bf16(la, gv, 6, st), "sortLSH level sparse backward"));
+    }
     ELSAA_TRY(cuda_status(launch_lsh_invert_orders(s.lsh_order, b.inv, lv, g, st), "order inverses"));
     ELSAA_TRY(cuda_status(launch_lsh_collect(b.dQ, w.dQacc, nullptr, nullptr, b.inv, lv, false, g, st), "sortLSH dQ"));
     ELSAA_TRY(cuda_status(launch_lsh_collect(b.dK, w.dKacc, b.dV, w.dVacc, b.inv, lv, true, g, st),
@@ -565,6 +582,7 @@ elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const
   ELSAA_TRY(cuda_status(launch_invert_selection(s.idx, w.offs, w.tiles, w.order, gb, st), "selection inverse"));
   a.idx = s.idx; a.offs = w.offs; a.tiles = w.tiles; a.kv_order = w.order;
   a.dQacc = w.dQacc; a.dKacc = w.dKacc; a.dVacc = w.dVacc;
+  if (!tc) return cuda_status(launch_bwd_bf16(a, gb, 6, st), "causal sortLSH base sparse backward");
   ELSAA_TRY(cuda_status(launch_dq_tc(a, gb, w.flag, st), "causal sortLSH base dq"));
   return cuda_status(launch_dkdv_tc(a, gb, w.flag, st), "causal sortLSH base dkdv");
 }
@@ -660,7 +678,6 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
   const bool lsh = g.selector == ELSAA_SEL_SORTLSH;
   if (lsh && g.causal) {
     ELSAA_TRY(check_ptr(p->lsh_planes, "lsh_planes"));
-    if (tcgen05_disabled()) return fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH runs on the tcgen05 kernels only");
     return causal_lsh_forward(p, g, Q, K, V, W, lam, gs, glr, O, s, w, st_);
   }
   void* O_out = O;
@@ -735,7 +752,6 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
   const bool lsh = g.selector == ELSAA_SEL_SORTLSH;
   if (lsh && g.causal) {
-    if (tcgen05_disabled()) return fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH runs on the tcgen05 kernels only");
     BwdArgs a{};
     a.Q = Q; a.K = K; a.V = V; a.dO = dO; a.W = W;
     a.lam = lam; a.gs = gs; a.glr = glr;

@@ -88,16 +88,18 @@ def test_status_strings():
 
 
 def test_sortlsh_shape_limits():
-    """sortLSH: non-causal up to N = 16384 on every path; the causal recursion needs the
-    tensor-core shape (bf16, d = 128, block 128), a power-of-two block count and N <= 32768."""
+    """sortLSH: non-causal up to N = 16384 on every path; the causal recursion needs bf16,
+    a power-of-two block count and N <= 32768."""
     L = bd.lib()
     ok = dict(selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=6, topk=1)
     assert L.elsaa_saved_bytes(ctypes.byref(bd.make_params(1, 2, 16384, 64, block_size=64, rank_r=16, causal=False,
                                                            **ok))) > 0
     assert L.elsaa_saved_bytes(ctypes.byref(bd.make_params(1, 2, 16384, 128, block_size=128, rank_r=128, causal=True,
                                                            **ok))) > 0
+    assert L.elsaa_saved_bytes(ctypes.byref(bd.make_params(1, 2, 32768, 64, block_size=64, rank_r=16, causal=True,
+                                                           **ok))) > 0
     bad = [dict(N=32768, d=64, block_size=64, causal=False),
-           dict(N=512, d=64, block_size=64, causal=True),
+           dict(N=64 * 6, d=64, block_size=64, causal=True),
            dict(N=128 * 6, d=128, block_size=128, causal=True),
            dict(N=1024, d=128, block_size=128, causal=True, dtype=bd.ELSAA_DTYPE_F32),
            dict(N=65536, d=128, block_size=128, causal=True)]

@@ -134,8 +134,8 @@ def test_full_size():
 
 # ---- the causal recursion (bf16, d = 128, block 128 on the tensor-core kernels) ----
 
-def _causal_setup(N, r, seed, fixed_m=False, bits=6, H=2):
-    w = small_workload(N=N, d=128, block_size=128, topk=2, rank_r=r, causal=True, dtype="bf16", H=H)
+def _causal_setup(N, r, seed, fixed_m=False, bits=6, H=2, d=128, T=128):
+    w = small_workload(N=N, d=d, block_size=T, topk=2, rank_r=r, causal=True, dtype="bf16", H=H)
     inp = make_inputs(w, seed)
     dev = device_inputs(w, inp)
     g = torch.Generator().manual_seed(seed + 7)
@@ -152,15 +152,24 @@ def _causal_oracle_params(w, R, codes, h, fixed_m=False):
     return p
 
 
-@pytest.mark.parametrize("N,r,gates,fixed_m", [(1024, 128, False, False), (1024, 128, True, False),
-                                               (2048, 64, False, False), (1024, 0, False, False),
-                                               (1024, 128, True, True), (128, 128, False, False),
-                                               (256, 128, False, False)])
-def test_causal_forward_backward(N, r, gates, fixed_m):
+@pytest.mark.parametrize("N,r,gates,fixed_m,d,T", [(1024, 128, False, False, 128, 128),
+                                                   (1024, 128, True, False, 128, 128),
+                                                   (2048, 64, False, False, 128, 128),
+                                                   (1024, 0, False, False, 128, 128),
+                                                   (1024, 128, True, True, 128, 128),
+                                                   (128, 128, False, False, 128, 128),
+                                                   (256, 128, False, False, 128, 128),
+                                                   (1024, 32, False, False, 64, 64),
+                                                   (512, 64, True, False, 64, 64),
+                                                   (1024, 0, False, True, 64, 64),
+                                                   (1024, 64, False, False, 64, 128),
+                                                   (512, 64, True, False, 128, 64)])
+def test_causal_forward_backward(N, r, gates, fixed_m, d, T):
     """O, dQ, dK, dV and the fusion gradients against the oracle's recursion run on the GPU's
-    hash codes (every level's sorted order follows from them); N = 128 and 256 are the
-    single-block and two-block cases (exact causal attention)."""
-    w, inp, dev, R, op = _causal_setup(N, r, seed=3, fixed_m=fixed_m)
+    hash codes (every level's sorted order follows from them), on the tcgen05 shape (d = 128,
+    block 128) and the mma.sync shapes; N = 128 and 256 at block 128 are the single-block and
+    two-block cases (exact causal attention)."""
+    w, inp, dev, R, op = _causal_setup(N, r, seed=3, fixed_m=fixed_m, d=d, T=T)
     BH = (w.B, w.H, w.N)
     g = torch.Generator().manual_seed(13)
     extra = {}
