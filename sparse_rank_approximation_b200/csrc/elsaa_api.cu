@@ -480,7 +480,7 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
   auto sparse_pass = [&](const FwdArgs& fa, const Geom& fg) {
     return tc ? launch_attn_fwd_tc(fa, fg, w.flag, st) : launch_attn_fwd_bf16(fa, fg, st);
   };
-  ELSAA_TRY(cuda_status(launch_causal_lsh_select(s.idx, 0, g, st), "causal sortLSH base selection"));
+  ELSAA_TRY(cuda_status(launch_causal_lsh_select(s.idx, g, st), "causal sortLSH base selection"));
   sa.Q = Q; sa.K = K; sa.V = V;
   ELSAA_TRY(cuda_status(sparse_pass(sa, gb), "causal sortLSH base pass"));
   if (g.lsh_levels > 0) {

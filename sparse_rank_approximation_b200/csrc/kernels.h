@@ -79,12 +79,12 @@ cudaError_t launch_sortlsh_hash(const void* Q, const void* K, bool bf16, const f
                                 int* codes, const Geom& g, cudaStream_t st);
 // Causal recursion: one level's orders [BH][2][N] (queries sorted in the future halves,
 // keys in the past halves of h rows; identity elsewhere) and, if inv is not null, the
-// future-half rows' positions [BH][N]; the base / level selections; the final
+// future-half rows' positions [BH][N]; the base-pass selection; the final
 // log-sum-exp merge of the partials with the fusion; the orders' inverses; the level
 // gradients collected into the fp32 accumulators; multi-tensor half-row gathers.
 cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int* inv, int h, int bits, const Geom& g,
                                       cudaStream_t st);
-cudaError_t launch_causal_lsh_select(int* idx, int hb, const Geom& g, cudaStream_t st);
+cudaError_t launch_causal_lsh_select(int* idx, const Geom& g, cudaStream_t st);
 cudaError_t launch_lsh_fuse(const void* Os0, const float* logd0, const void* Os_lv, const float* logd_lv,
                             const int* inv_lv, int levels, const void* Olr, const float* dlr, const float* lam,
                             const float* gs, const float* glr, void* O, void* Os, float* logd, float* m, const Geom& g,

@@ -236,21 +236,15 @@ __global__ void __launch_bounds__(kSortThreads) sortlsh_level_sort_kernel(const 
   }
 }
 
-// Selections of the causal recursion.  Base pass (the caller's row order, causal): tile
-// t takes its own block and, when t is odd, block t - 1 (the deepest level, whose halves
-// are single blocks and need no sort); ascending, -1 padded, k = 2.  Level with halves
-// of hb blocks (sorted rows): a tile in a future half takes the block hb before it, a
-// tile in a past half takes none; k = 1.
-__global__ void causal_lsh_select_kernel(int* __restrict__ idx, int hb, Geom g) {
+// Base-pass selection of the causal recursion (the caller's row order, causal): tile t
+// takes its own block and, when t is odd, block t - 1 (the deepest level, whose halves
+// are single blocks and need no sort); ascending, -1 padded, k = 2.
+__global__ void causal_lsh_select_kernel(int* __restrict__ idx, Geom g) {
   const size_t total = (size_t)g.BH * g.n_t;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
     const int t = (int)(e % g.n_t);
-    if (hb == 0) {
-      idx[2 * e] = (t & 1) ? t - 1 : t;
-      idx[2 * e + 1] = (t & 1) ? t : -1;
-    } else {
-      idx[e] = ((t / hb) & 1) ? t - hb : -1;
-    }
+    idx[2 * e] = (t & 1) ? t - 1 : t;
+    idx[2 * e + 1] = (t & 1) ? t : -1;
   }
 }
 
@@ -515,8 +509,8 @@ cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int* inv, int 
 
 static int elementwise_blocks(size_t total) { return (int)std::min<size_t>((total + 255) / 256, 148 * 16); }
 
-cudaError_t launch_causal_lsh_select(int* idx, int hb, const Geom& g, cudaStream_t st) {
-  causal_lsh_select_kernel<<<elementwise_blocks((size_t)g.BH * g.n_t), 256, 0, st>>>(idx, hb, g);
+cudaError_t launch_causal_lsh_select(int* idx, const Geom& g, cudaStream_t st) {
+  causal_lsh_select_kernel<<<elementwise_blocks((size_t)g.BH * g.n_t), 256, 0, st>>>(idx, g);
   return cudaGetLastError();
 }
 
