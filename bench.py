@@ -99,6 +99,9 @@ def work_model(w):
     m["race_k_bwd_tc"] = dict(flops=tiles * 2 * T * (2 * cz * T * r + 2 * cz * T * d + 2 * r * d + NH * d),
                               bytes=tiles * (T * r * 2 * (1 + cz) + T * d * 2 * (2 + cz) + state_b + T * NH * 4
                                              + T * 12 + 2 * T * d * 4))
+    # the mma.sync RACE backward kernels do the same algorithmic work as the tcgen05 ones
+    m["race_q_bwd"] = m["race_q_bwd_tc"]
+    m["race_k_bwd"] = m["race_k_bwd_tc"]
     f_state = tiles * 2 * T * r * (d + 8)
     m["race_state_fwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)
     m["race_state_bwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)
