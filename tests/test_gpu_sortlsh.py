@@ -45,7 +45,7 @@ def _oracle_params(w, R, orders, fixed_m=False):
 
 
 @pytest.mark.parametrize("geom", list(GEOMS))
-@pytest.mark.parametrize("bits", [4, 9])
+@pytest.mark.parametrize("bits", [1, 4, 9, 16])
 def test_codes_and_orders(geom, bits):
     w, inp, dev, R, op = _setup(geom, bits)
     codes, order = op.debug_sortlsh(dev["Q"], dev["K"])
@@ -150,6 +150,28 @@ def _causal_oracle_params(w, R, codes, h, fixed_m=False):
     p.lsh_planes = R.double().numpy()
     p.lsh_codes = (codes[0, h, 0].cpu().numpy(), codes[0, h, 1].cpu().numpy())
     return p
+
+
+@pytest.mark.parametrize("bits", [1, 12])
+def test_causal_hash_widths(bits):
+    """The causal recursion with 1-bit codes (one sort pass, two buckets) and 12-bit codes
+    (two 8-bit passes in every level sort)."""
+    w, inp, dev, R, op = _causal_setup(1024, 128, seed=4, bits=bits)
+    O = op.forward(dev["Q"], dev["K"], dev["V"], dev["W"])
+    dQ, dK, dV = op.backward(dev["Q"], dev["K"], dev["V"], dev["W"], dev["dO"])
+    codes, _ = op.debug_sortlsh(dev["Q"], dev["K"])
+    assert op.check_device_flags() == 0
+    torch.cuda.synchronize()
+    W = inp["W"].double().numpy()
+    for h in range(w.H):
+        p = _causal_oracle_params(w, R, codes, h)
+        get = lambda n: inp[n][0, h].double().numpy()
+        fw = orc.forward_head(get("Q"), get("K"), get("V"), W, p)
+        dq, dk, dv = orc.backward_head(get("Q"), get("K"), get("V"), W, get("dO"), fw, p)
+        check(w, f"O[{h}]", np64(O[0, h]), fw["O"])
+        check(w, f"dQ[{h}]", np64(dQ[0, h]), dq)
+        check(w, f"dK[{h}]", np64(dK[0, h]), dk)
+        check(w, f"dV[{h}]", np64(dV[0, h]), dv)
 
 
 @pytest.mark.parametrize("N,r,gates,fixed_m,d,T", [(1024, 128, False, False, 128, 128),
