@@ -1,14 +1,18 @@
-// sortLSH selector (ELSAA paper §3.2), non-causal: queries and keys are hashed with
-// angular LSH, sorted by hash value and grouped into equal-size blocks; query block t
-// attends exactly key block t.  Rows carry a b-bit code (bit c set when x . R_c > 0),
-// are ordered by the position of the code in the reflected Gray sequence (neighbouring
-// buckets differ in one bit) and then by row index.
+// sortLSH selector (ELSAA paper §3.2): queries and keys are hashed with angular LSH,
+// sorted by hash value and grouped into equal-size blocks; query block t attends exactly
+// key block t.  Rows carry a b-bit code (bit c set when x . R_c > 0), are ordered by the
+// position of the code in the reflected Gray sequence (neighbouring buckets differ in one
+// bit) and then by row index.
 //
-// Non-causal RACE, the fusion and diagonal-block attention all commute with row
+// Non-causal: RACE, the fusion and diagonal-block attention all commute with row
 // permutations, so the selector runs the rest of the operator on row-permuted copies
 // (queries by the query order, keys and values by the key order) with tile t selecting
-// block t, and scatters the outputs back.  This file holds the hashing and sorting,
-// the row gather / scatter and the diagonal selection.
+// block t, and scatters the outputs back.
+// Causal: the paper's recursion.  Every level's future-half queries meet its past-half
+// keys by sorted blocks; the levels run as extra heads of the sparse kernels on gathered
+// rows, and their partial softmaxes are merged by log-sum-exp before the fusion.
+// This file holds the hashing and sorting, the row gathers and scatters, the selections
+// and the recursion's merge and gradient collection.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -255,7 +259,7 @@ __global__ void causal_lsh_select_kernel(int* __restrict__ idx, Geom g) {
 // m = 1 / (1 + (lambda d_lr + eps) e^{-log d_s}) (1 when m is held), O = g_s m O_s + g_lr O_lr
 // with g_lr = 1 - m by default (1 when m is held).  Writes O, the saved bf16 O_s, log d_s
 // and m.  One thread per 8 columns; partials are bf16, the merge is fp32.
-constexpr int kMaxLevels = 8;             // N <= 32768 rows of 128: at most 7 sorted levels
+constexpr int kMaxLevels = 8;             // N <= 32768 in blocks of >= 64 rows: at most 8 sorted levels
 
 __global__ void lsh_fuse_kernel(const __nv_bfloat16* __restrict__ Os0, const float* __restrict__ logd0,
                                 const __nv_bfloat16* __restrict__ Os_lv, const float* __restrict__ logd_lv,
@@ -389,9 +393,9 @@ __global__ void lsh_collect_kernel(const __nv_bfloat16* __restrict__ src0, float
 }
 
 // Every level's sorted rows, gathered into level slots: for level l (halves of
-// h_l = N >> (l + 1) rows, orders at perm + l BH perm_stride), dst_t[l][bh][p] =
-// src_t[bh][perm_l[p]] for up to four tensors, 16-byte units; half >= 0 moves only the
-// positions in the past (0) or future (1) halves.
+// h_l = N >> (l + 1) rows; its orders at perm + l BH 2N, one side of [BH][2][N]),
+// dst_t[l][bh][p] = src_t[bh][perm_l[p]] for up to four tensors, 16-byte units; half >= 0
+// moves only the positions in the past (0) or future (1) halves.
 struct RowMoves {
   const uint4* src[4];
   uint4* dst[4];
