@@ -363,6 +363,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float cs = gs * mf;
       const unsigned char* lrow = smem + off_k(0) + half * kSlab + row * 128;
       unsigned char* orow = smem + off_v(0) + half * kSlab + row * 128;
+      // with a row map, O goes straight to the caller's row (8 bf16 per 16-byte unit)
+      uint4* grow = a.q_rows && qrow < g.N
+                        ? reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) +
+                                                   (head + a.q_rows[(size_t)bh * a.rows_stride + qrow]) * kD + 64 * half)
+                        : nullptr;
       unsigned char* srow = smem + off_v(1) + half * kSlab + row * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
@@ -376,7 +381,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           ws[e] = pack_bf16(s0, s1);
           wo[e] = pack_bf16(cs * s0 + gl * __bfloat162float(lv[2 * e]), cs * s1 + gl * __bfloat162float(lv[2 * e + 1]));
         }
-        *reinterpret_cast<uint4*>(orow + sw) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
+        if (a.q_rows) {
+          if (grow) grow[ch] = make_uint4(wo[0], wo[1], wo[2], wo[3]);
+        } else {
+          *reinterpret_cast<uint4*>(orow + sw) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
+        }
         *reinterpret_cast<uint4*>(srow + sw) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
       }
       if (half == 0 && qrow < g.N) {
@@ -387,8 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_proxy_async_smem();
     softmax_bar();
     if (threadIdx.x == 96 && !*(volatile int*)&ms->abort_flag) {
-      tma_store_3d(&tmO, smem + off_v(0), 0, t * kT, bh);
-      tma_store_3d(&tmO, smem + off_v(0) + kSlab, 64, t * kT, bh);
+      if (!a.q_rows) {
+        tma_store_3d(&tmO, smem + off_v(0), 0, t * kT, bh);
+        tma_store_3d(&tmO, smem + off_v(0) + kSlab, 64, t * kT, bh);
+      }
       tma_store_3d(&tmS, smem + off_v(1), 0, t * kT, bh);
       tma_store_3d(&tmS, smem + off_v(1) + kSlab, 64, t * kT, bh);
       asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");

@@ -273,7 +273,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const float4* acc =
         alive && row_ok && a.dQacc ? reinterpret_cast<const float4*>(a.dQacc + (head + qrow) * kD + 64 * half) : nullptr;
     // every product has completed: stage the bf16 tile in the Q buffer, 32 columns at a time
+    // (with a row map, write each row straight to the caller's row instead)
     unsigned char* orow = smem + DQ_Q + half * kSlab + row * 128;
+    uint4* grow = a.q_rows && row_ok && alive
+                      ? reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dQ) +
+                                                 (head + a.q_rows[(size_t)bh * a.rows_stride + qrow]) * kD + 64 * half)
+                      : nullptr;
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
       float o[32];
@@ -295,17 +300,23 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int ch = 4 * c + cc;
-        *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) =
-            make_uint4(pack_bf16(o[8 * cc], o[8 * cc + 1]), pack_bf16(o[8 * cc + 2], o[8 * cc + 3]),
-                       pack_bf16(o[8 * cc + 4], o[8 * cc + 5]), pack_bf16(o[8 * cc + 6], o[8 * cc + 7]));
+        const uint4 val = make_uint4(pack_bf16(o[8 * cc], o[8 * cc + 1]), pack_bf16(o[8 * cc + 2], o[8 * cc + 3]),
+                                     pack_bf16(o[8 * cc + 4], o[8 * cc + 5]), pack_bf16(o[8 * cc + 6], o[8 * cc + 7]));
+        if (a.q_rows) {
+          if (grow) grow[ch] = val;
+        } else {
+          *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) = val;
+        }
       }
     }
-    tc::fence_proxy_async_smem();
-    softmax_bar();
-    if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
-      tma_store_3d(&tmdQ, smem + DQ_Q, 0, t * kT, bh);
-      tma_store_3d(&tmdQ, smem + DQ_Q + kSlab, 64, t * kT, bh);
-      tma_store_wait();
+    if (!a.q_rows) {
+      tc::fence_proxy_async_smem();
+      softmax_bar();
+      if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
+        tma_store_3d(&tmdQ, smem + DQ_Q, 0, t * kT, bh);
+        tma_store_3d(&tmdQ, smem + DQ_Q + kSlab, 64, t * kT, bh);
+        tma_store_wait();
+      }
     }
   }
   __syncthreads();
@@ -548,6 +559,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                              ? reinterpret_cast<const float4*>(accp + (head + (size_t)b * kT + row) * kD + 64 * hq)
                              : nullptr;
       unsigned char* orow = smem + (which == 0 ? kv_q(0) : kv_do(0)) + hq * kSlab + row * 128;
+      // with a row map, write each key row straight to the caller's row instead
+      uint4* grow = a.k_rows && key_ok && alive
+                        ? reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(which == 0 ? a.dK : a.dV) +
+                                                   (head + a.k_rows[(size_t)bh * a.rows_stride + b * kT + row]) * kD +
+                                                   64 * hq)
+                        : nullptr;
       // 32 columns at a time: TMEM -> scale -> + low-rank part -> bf16 -> swizzled row
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
@@ -570,20 +587,27 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           const int ch = 4 * c + cc;
-          *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) =
+          const uint4 val =
               make_uint4(pack_bf16(o[8 * cc], o[8 * cc + 1]), pack_bf16(o[8 * cc + 2], o[8 * cc + 3]),
                          pack_bf16(o[8 * cc + 4], o[8 * cc + 5]), pack_bf16(o[8 * cc + 6], o[8 * cc + 7]));
+          if (a.k_rows) {
+            if (grow) grow[ch] = val;
+          } else {
+            *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) = val;
+          }
         }
       }
     }
-    tc::fence_proxy_async_smem();
-    softmax_bar();
-    if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
-      tma_store_3d(&tmdK, smem + kv_q(0), 0, b * kT, bh);
-      tma_store_3d(&tmdK, smem + kv_q(0) + kSlab, 64, b * kT, bh);
-      tma_store_3d(&tmdV, smem + kv_do(0), 0, b * kT, bh);
-      tma_store_3d(&tmdV, smem + kv_do(0) + kSlab, 64, b * kT, bh);
-      tma_store_wait();
+    if (!a.k_rows) {
+      tc::fence_proxy_async_smem();
+      softmax_bar();
+      if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
+        tma_store_3d(&tmdK, smem + kv_q(0), 0, b * kT, bh);
+        tma_store_3d(&tmdK, smem + kv_q(0) + kSlab, 64, b * kT, bh);
+        tma_store_3d(&tmdV, smem + kv_do(0), 0, b * kT, bh);
+        tma_store_3d(&tmdV, smem + kv_do(0) + kSlab, 64, b * kT, bh);
+        tma_store_wait();
+      }
     }
   }
   __syncthreads();

@@ -706,17 +706,25 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
                           "race statistics split"));
   FwdArgs a{Q, K, V, s.idx, s.phiQ, s.phiK, s.Ast, s.Bst, lam, gs, glr, O, s.Os, s.logd, s.dlr, s.m, s.Olr,
             s.Psplit, s.Pmass};
+  bool scattered = false;
   if (bf16 && attn_fwd_tc_supported(g) && !tcgen05_disabled()) {
     if (s.Psplit) ELSAA_TRY(cuda_status(launch_race_readout_tc(a, g, w.flag, st_), "tcgen05 race read-out"));
     else
       ELSAA_TRY(cuda_status(launch_race_readout_bf16(a, g, st_), "race read-out"));
-    ELSAA_TRY(cuda_status(launch_attn_fwd_tc(a, g, w.flag, st_), "tcgen05 forward"));
+    FwdArgs at = a;
+    if (lsh) {                        // the epilogue writes O straight into the caller's row order
+      at.O = O_out;
+      at.q_rows = s.lsh_order;
+      at.rows_stride = 2 * g.N;
+      scattered = true;
+    }
+    ELSAA_TRY(cuda_status(launch_attn_fwd_tc(at, g, w.flag, st_), "tcgen05 forward"));
   } else if (bf16) {
     ELSAA_TRY(cuda_status(launch_attn_fwd_bf16(a, g, st_), "fused forward"));
   } else {
     ELSAA_TRY(cuda_status(launch_attn_fwd_f32(a, g, st_), "fused forward"));
   }
-  if (lsh)
+  if (lsh && !scattered)
     ELSAA_TRY(cuda_status(launch_permute_rows(O, O_out, s.lsh_order, g.d * (bf16 ? 2 : 4), g, 2 * g.N, true, st_),
                           "sortLSH scatter O"));
   return ELSAA_OK;
@@ -790,6 +798,7 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   a.Psplit = s.Psplit; a.Pmass = s.Pmass; a.Rsplit = w.Rsplit; a.Rmass = w.Rmass; a.Wsplit = w.Wsplit;
   a.dQ = dQ; a.dK = dK; a.dV = dV;
 
+  bool scattered = false;
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st_), "flag reset"));
   ELSAA_TRY(cuda_status(launch_row_scalars(a, bf16, g, st_), "row scalars"));
   ELSAA_TRY(cuda_status(launch_race_state_bwd(a, bf16, g, st_), "race suffix summaries"));
@@ -807,13 +816,22 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
     }
     ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, tc ? (race_tc ? 0 : 1) : 7, st_), "backward"));
     if (tc) {
+      if (lsh) {                      // the epilogues write straight into the caller's row orders
+        at.dQ = dQ_out;
+        at.dK = dK_out;
+        at.dV = dV_out;
+        at.q_rows = s.lsh_order;
+        at.k_rows = s.lsh_order + g.N;
+        at.rows_stride = 2 * g.N;
+        scattered = true;
+      }
       ELSAA_TRY(cuda_status(launch_dq_tc(at, g, w.flag, st_), "tcgen05 dq"));
       ELSAA_TRY(cuda_status(launch_dkdv_tc(at, g, w.flag, st_), "tcgen05 dkdv"));
     }
   } else {
     ELSAA_TRY(cuda_status(launch_bwd_f32(a, g, st_), "backward"));
   }
-  if (lsh) {
+  if (lsh && !scattered) {
     const int rb = g.d * (bf16 ? 2 : 4);
     ELSAA_TRY(cuda_status(launch_permute_rows(dQ, dQ_out, s.lsh_order, rb, g, 2 * g.N, true, st_), "sortLSH dQ"));
     ELSAA_TRY(cuda_status(launch_permute_rows(dK, dK_out, s.lsh_order + g.N, rb, g, 2 * g.N, true, st_),

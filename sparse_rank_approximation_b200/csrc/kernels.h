@@ -29,6 +29,10 @@ struct FwdArgs {
   // optional: the query tiles to run, n_list per head ([BH][n_list]); null runs all tiles
   const int* tile_list;
   int n_list;
+  // optional (tensor-core kernel): O row r of head bh goes to row q_rows[bh * rows_stride + r]
+  // of the caller's O instead of row r (the sortLSH orders); O_s stays in row order
+  const int* q_rows;
+  int rows_stride;
 };
 
 // Per-row adjoint scalars of the fusion (Eq. 4 / Eq. 5), float32 [BH, N] each.
@@ -67,6 +71,10 @@ struct BwdArgs {
   const int* tile_list;
   int n_list;
   int n_kv;
+  // optional (tensor-core kernels): dQ row r goes to row q_rows[bh * rows_stride + r], dK and
+  // dV row r to row k_rows[bh * rows_stride + r] of the caller's outputs (the sortLSH orders)
+  const int *q_rows, *k_rows;
+  int rows_stride;
 };
 
 // sortLSH selector: per head the sorted query and key orders, int32 [BH][2][N]
