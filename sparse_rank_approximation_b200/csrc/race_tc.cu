@@ -171,13 +171,29 @@ __device__ __forceinline__ void issue_du(uint32_t tmem, uint32_t d_col, uint32_t
   }
 }
 
+// fp32 gradient rows leave through shared memory: each thread writes its row there (pitch
+// kD + 4 floats, so the 16-byte stores of 8 consecutive rows hit 8 different bank groups),
+// then all compute threads copy the [128][kD] tile out with coalesced 16-byte stores.  The
+// staging area reuses operand tiles that no product reads any more.
+constexpr int kStagePitch = kD + 4;
+constexpr uint32_t kStageBytes = (uint32_t)kC * kStagePitch * 4;
+
+__device__ __forceinline__ void copy_staged(const float* stage, float* __restrict__ out, int rows, int ct) {
+  for (int idx = ct; idx < kC * (kD / 4); idx += kComputeThreads) {
+    const int r = idx / (kD / 4), c4 = idx % (kD / 4);
+    if (r < rows)
+      reinterpret_cast<float4*>(out + (size_t)r * kD)[c4] =
+          *reinterpret_cast<const float4*>(stage + r * kStagePitch + 4 * c4);
+  }
+}
+
 // dx = (du - x <x, du> / n^2) / n for one row, this thread's 64 columns; the two
 // column halves of a row meet through `xch`.  Stores fp32 into out (row pointer).
 // Every compute thread calls this (the exchange barrier); `alive` false skips the
 // tensor-memory reads and the stores.
 __device__ __forceinline__ void chain_pass(uint32_t tmem, uint32_t lane_base, int hc, int row_in_chunk,
                                            uint32_t du_col, const uint4 (&xr)[8], float n, float* xch,
-                                           float* __restrict__ out, bool valid, bool alive) {
+                                           float* stage, bool valid, bool alive) {
   float du[64];
   if (alive) {
     tc::tc_fence_after();
@@ -206,7 +222,7 @@ __device__ __forceinline__ void chain_pass(uint32_t tmem, uint32_t lane_base, in
   if (!valid) return;
   const float proj = n <= kNormFloor ? 0.f : xd / (n * n);
   const float inv = 1.f / n;
-  float4* o = reinterpret_cast<float4*>(out + 64 * hc);
+  float4* o = reinterpret_cast<float4*>(stage + row_in_chunk * kStagePitch + 64 * hc);
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&xr[q]);
@@ -226,6 +242,9 @@ constexpr uint32_t K_CL = K_WL + 2 * kWSlab;            // cl [128], delta [128]
 constexpr uint32_t K_BARS = K_CL + (3 * 128 + 256) * 4;
 // TMEM columns
 constexpr uint32_t TK_KAP = 0, TK_X = 128, TK_DV = 256, TK_DPHI = 384, TK_DU = 128;
+// staged dV and dK rows, over the operand tiles once every product that reads them is done
+constexpr uint32_t K_STAGE_V = 0, K_STAGE_K = (kStageBytes + 1023u) & ~1023u;
+static_assert(K_STAGE_K + kStageBytes <= K_WH, "the staged rows overlap only the chunk tiles");
 
 }  // namespace
 
@@ -343,6 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
     const int row = c * kC + j;
     const bool valid = row < g.N;
+    float* stage_v = reinterpret_cast<float*>(smem + K_STAGE_V);
+    float* stage_k = reinterpret_cast<float*>(smem + K_STAGE_K);
     // row data for the corner and chain passes, fetched up front
     float h16[16];
     load_h(valid ? a.hK + (head + row) * kNH : nullptr, hc, h16);
@@ -399,11 +420,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float v[32];
         tc::tmem_ld32(tmem + lane_base + TK_DV + 64 * hc + 32 * h2, v);
         tc::tmem_wait_ld();
-        if (valid) {
-          float4* o = reinterpret_cast<float4*>(a.dVacc + (head + row) * kD + 64 * hc + 32 * h2);
+        // every product has read the operand tiles: dV rows are staged over them
+        float4* o = reinterpret_cast<float4*>(stage_v + j * kStagePitch + 64 * hc + 32 * h2);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        }
+        for (int q = 0; q < 8; ++q) o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
       }
       corner_pass(tmem, lane_base, hc, TK_DPHI, true, 0u, 0.f, valid ? 1.f : 0.f, sR1, h16, rsqrtf((float)g.L),
                   1.f / g.tau);
@@ -414,7 +434,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint4 xr[8];
     load_x((const __nv_bfloat16*)a.K + (head + row) * kD, hc, valid && alive, xr);
     if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->du_full, 0, ms, err, 0x4000u));
-    chain_pass(tmem, lane_base, hc, j, TK_DU, xr, nrm, sX, a.dKacc + (head + row) * kD, valid, alive);
+    chain_pass(tmem, lane_base, hc, j, TK_DU, xr, nrm, sX, stage_k, valid, alive);
+    compute_bar();
+    if (!*(volatile int*)&ms->abort_flag) {
+      const int rows = min(kC, g.N - c * kC);
+      copy_staged(stage_v, a.dVacc + (head + (size_t)c * kC) * kD, rows, ct);
+      copy_staged(stage_k, a.dKacc + (head + (size_t)c * kC) * kD, rows, ct);
+    }
   }
   __syncthreads();
   if (warp == 1) {
@@ -429,6 +455,7 @@ constexpr uint32_t Q_DO = 0, Q_V = kTile, Q_PK = 2 * kTile, Q_PH = 3 * kTile, Q_
 constexpr uint32_t Q_WH = 5 * kTile, Q_WL = Q_WH + 2 * kWSlab;
 constexpr uint32_t Q_P1 = Q_WL + 2 * kWSlab;            // p1 [128], exchange [256]
 constexpr uint32_t Q_BARS = Q_P1 + (128 + 256) * 4;
+static_assert(Q_DO + kStageBytes <= Q_WH, "the staged dQ rows overlap only the chunk tiles");
 constexpr uint32_t TQ_X = 0, TQ_INTRA = 128, TQ_G = 256, TQ_DU = 384;
 }  // namespace
 
@@ -577,7 +604,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint4 xr[8];
     load_x((const __nv_bfloat16*)a.Q + (head + row) * kD, hc, valid && alive, xr);
     if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->du_full, 0, ms, err, 0x4000u));
-    chain_pass(tmem, lane_base, hc, i, TQ_DU, xr, nrm, sX, a.dQacc + (head + row) * kD, valid, alive);
+    // every product is done: dQ rows are staged over the operand tiles
+    float* stage_q = reinterpret_cast<float*>(smem + Q_DO);
+    chain_pass(tmem, lane_base, hc, i, TQ_DU, xr, nrm, sX, stage_q, valid, alive);
+    compute_bar();
+    if (!*(volatile int*)&ms->abort_flag)
+      copy_staged(stage_q, a.dQacc + (head + (size_t)t * kC) * kD, min(kC, g.N - t * kC), ct);
   }
   __syncthreads();
   if (warp == 1) {
