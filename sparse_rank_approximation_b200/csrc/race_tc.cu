@@ -64,7 +64,7 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t base, int kk, uint32_t slab
 __device__ __forceinline__ uint32_t packed_col(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
 
 struct Bars {
-  uint64_t in_main, s_full, p_full, acc_full, dh_full, du_full;
+  uint64_t in_main, s_full, p_full, acc_full, dh_full, du_full, x_full;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -120,10 +120,14 @@ __device__ __forceinline__ void load_h(const float* __restrict__ hrow, int hc, f
     h16[4 * q] = v.x; h16[4 * q + 1] = v.y; h16[4 * q + 2] = v.z; h16[4 * q + 3] = v.w;
   }
 }
-__device__ __forceinline__ void load_x(const __nv_bfloat16* __restrict__ xrow, int hc, bool valid, uint4 (&xr)[8]) {
+// Row `row` of a [128][128] bf16 tile that TMA wrote as two 64-column slabs with the
+// 128-byte swizzle: this thread's half (columns 64 hc .. 64 hc + 63) as 8 x 16 bytes.  Eight
+// consecutive rows read eight different 16-byte positions, so a warp's reads do not conflict.
+__device__ __forceinline__ void load_x(const unsigned char* tile, int row, int hc, bool valid, uint4 (&xr)[8]) {
+  const unsigned char* base = tile + (uint32_t)hc * kSlab + (uint32_t)row * 128u;
 #pragma unroll
   for (int q = 0; q < 8; ++q)
-    xr[q] = valid ? __ldg(reinterpret_cast<const uint4*>(xrow + 64 * hc) + q) : make_uint4(0u, 0u, 0u, 0u);
+    xr[q] = valid ? *reinterpret_cast<const uint4*>(base + ((q ^ (row & 7)) << 4)) : make_uint4(0u, 0u, 0u, 0u);
 }
 
 __device__ __forceinline__ void corner_pass(uint32_t tmem, uint32_t lane_base, int hc, uint32_t dphi_col,
@@ -244,7 +248,9 @@ constexpr uint32_t K_BARS = K_CL + (3 * 128 + 256) * 4;
 constexpr uint32_t TK_KAP = 0, TK_X = 128, TK_DV = 256, TK_DPHI = 384, TK_DU = 128;
 // staged dV and dK rows, over the operand tiles once every product that reads them is done
 constexpr uint32_t K_STAGE_V = 0, K_STAGE_K = (kStageBytes + 1023u) & ~1023u;
-static_assert(K_STAGE_K + kStageBytes <= K_WH, "the staged rows overlap only the chunk tiles");
+// the K rows of the chunk for dx, over the statistics tiles once their products are done
+constexpr uint32_t K_XS = (K_STAGE_K + kStageBytes + 1023u) & ~1023u;
+static_assert(K_XS + kTile <= K_WH, "the staged rows and the K tile overlap only the chunk tiles");
 
 }  // namespace
 
@@ -252,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     race_k_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmPQ,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                          const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmW,
-                         BwdArgs a, Geom g, uint32_t* err) {
+                         const __grid_constant__ CUtensorMap tmX, BwdArgs a, Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   Bars* ms = reinterpret_cast<Bars*>(smem + K_BARS);
   float* sCl = reinterpret_cast<float*>(smem + K_CL);
@@ -274,6 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&ms->acc_full, 1);
     tc::mbar_init(&ms->dh_full, kComputeThreads);
     tc::mbar_init(&ms->du_full, 1);
+    tc::mbar_init(&ms->x_full, 1);
     ms->abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -303,6 +310,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_load_3d(smem + K_WL + s * kWSlab, &tmW, &ms->in_main, 64 * s, 0, 1);
       }
       tc::mbar_wait(&ms->in_main, 0);
+      // the K rows for dx, once every product but du has read the chunk tiles; waited for
+      // here too, so no copy is in flight when the CTA exits
+      if (wait_or_abort(&ms->acc_full, 0, ms, err, 0x10000u)) {
+        tc::mbar_arrive_expect_tx(&ms->x_full, kTile);
+        tc::tma_load_3d(smem + K_XS, &tmX, &ms->x_full, 0, c * kC, bh);
+        tc::tma_load_3d(smem + K_XS + kSlab, &tmX, &ms->x_full, 64, c * kC, bh);
+        wait_or_abort(&ms->x_full, 0, ms, err, 0x20000u);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -432,7 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive(&ms->dh_full);
     }
     uint4 xr[8];
-    load_x((const __nv_bfloat16*)a.K + (head + row) * kD, hc, valid && alive, xr);
+    if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->x_full, 0, ms, err, 0x40000u));
+    load_x(smem + K_XS, j, hc, valid && alive, xr);
     if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->du_full, 0, ms, err, 0x4000u));
     chain_pass(tmem, lane_base, hc, j, TK_DU, xr, nrm, sX, stage_k, valid, alive);
     compute_bar();
@@ -455,14 +471,17 @@ constexpr uint32_t Q_DO = 0, Q_V = kTile, Q_PK = 2 * kTile, Q_PH = 3 * kTile, Q_
 constexpr uint32_t Q_WH = 5 * kTile, Q_WL = Q_WH + 2 * kWSlab;
 constexpr uint32_t Q_P1 = Q_WL + 2 * kWSlab;            // p1 [128], exchange [256]
 constexpr uint32_t Q_BARS = Q_P1 + (128 + 256) * 4;
-static_assert(Q_DO + kStageBytes <= Q_WH, "the staged dQ rows overlap only the chunk tiles");
+// the Q rows of the chunk for dx, after the staged dQ rows
+constexpr uint32_t Q_XS = (Q_DO + kStageBytes + 1023u) & ~1023u;
+static_assert(Q_XS + kTile <= Q_WH, "the staged dQ rows and the Q tile overlap only the chunk tiles");
 constexpr uint32_t TQ_X = 0, TQ_INTRA = 128, TQ_G = 256, TQ_DU = 384;
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1)
     race_q_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmdO, const __grid_constant__ CUtensorMap tmV,
                          const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmP,
-                         const __grid_constant__ CUtensorMap tmW, BwdArgs a, Geom g, uint32_t* err) {
+                         const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                         BwdArgs a, Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   Bars* ms = reinterpret_cast<Bars*>(smem + Q_BARS);
   float* sP1 = reinterpret_cast<float*>(smem + Q_P1);
@@ -482,6 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&ms->acc_full, 1);
     tc::mbar_init(&ms->dh_full, kComputeThreads);
     tc::mbar_init(&ms->du_full, 1);
+    tc::mbar_init(&ms->x_full, 1);
     ms->abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -510,6 +530,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_load_3d(smem + Q_WL + s * kWSlab, &tmW, &ms->in_main, 64 * s, 0, 1);
       }
       tc::mbar_wait(&ms->in_main, 0);
+      // the Q rows for dx, once every product but du has read the chunk tiles; waited for
+      // here too, so no copy is in flight when the CTA exits
+      if (wait_or_abort(&ms->acc_full, 0, ms, err, 0x10000u)) {
+        tc::mbar_arrive_expect_tx(&ms->x_full, kTile);
+        tc::tma_load_3d(smem + Q_XS, &tmX, &ms->x_full, 0, t * kC, bh);
+        tc::tma_load_3d(smem + Q_XS + kSlab, &tmX, &ms->x_full, 64, t * kC, bh);
+        wait_or_abort(&ms->x_full, 0, ms, err, 0x20000u);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -602,7 +630,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive(&ms->dh_full);
     }
     uint4 xr[8];
-    load_x((const __nv_bfloat16*)a.Q + (head + row) * kD, hc, valid && alive, xr);
+    if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->x_full, 0, ms, err, 0x40000u));
+    load_x(smem + Q_XS, i, hc, valid && alive, xr);
     if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->du_full, 0, ms, err, 0x4000u));
     // every product is done: dQ rows are staged over the operand tiles
     float* stage_q = reinterpret_cast<float*>(smem + Q_DO);
@@ -829,8 +858,9 @@ cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, c
   if (!race_bwd_tc_supported(g) || !a.hQ || !a.hK || !a.nQ || !a.nK || !a.Psplit || !a.Pmass || !a.Rsplit ||
       !a.Rmass || !a.Wsplit)
     return cudaErrorInvalidValue;
-  CUtensorMap mpk, mpq, mv, mdo, mp, mr, mw;
-  if (!tc::map_rows_bf16(&mpk, a.phiK, g.N, g.BH, kC) || !tc::map_rows_bf16(&mpq, a.phiQ, g.N, g.BH, kC) ||
+  CUtensorMap mpk, mpq, mv, mdo, mp, mr, mw, mq, mk;
+  if (!tc::map_rows_bf16(&mq, a.Q, g.N, g.BH, kC) || !tc::map_rows_bf16(&mk, a.K, g.N, g.BH, kC) ||
+      !tc::map_rows_bf16(&mpk, a.phiK, g.N, g.BH, kC) || !tc::map_rows_bf16(&mpq, a.phiQ, g.N, g.BH, kC) ||
       !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kC) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, kC) ||
       !tc::map_rows_bf16(&mp, a.Psplit, kR, g.BH * g.n_c * 2, kR) ||
       !tc::map_rows_bf16(&mr, a.Rsplit, kR, g.BH * g.n_c * 2, kR) || !tc::map_rows_bf16(&mw, a.Wsplit, kNH, 2, kNH))
@@ -841,7 +871,7 @@ cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, c
     cudaError_t e = cudaFuncSetAttribute(race_q_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     ProfScope ps("race_q_bwd_tc", st);
-    race_q_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mdo, mv, mpk, mp, mw, a, g, err);
+    race_q_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mdo, mv, mpk, mp, mw, mq, a, g, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -850,7 +880,7 @@ cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, c
   cudaError_t e = cudaFuncSetAttribute(race_k_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("race_k_bwd_tc", st);
-  race_k_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mpk, mpq, mv, mdo, mr, mw, a, g, err);
+  race_k_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mpk, mpq, mv, mdo, mr, mw, mk, a, g, err);
   return cudaGetLastError();
 }
 
