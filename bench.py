@@ -117,7 +117,7 @@ def work_model(w):
                    gathered_fwd=sel * 2 * T * d * 2, unique_fwd=unique_fwd)
 
 
-def north_star_roofline(w, peaks, t_step_ms):
+def whole_step_roofline(w, peaks, t_step_ms):
     """T_roof = max(F / P_bf16, gathered bytes / BW), forward + backward, counted as
     sparse F_bwd = 2.5 F_fwd, low-rank F_bwd = 2 F_fwd, backward bytes = 2x gathered
     plus 8 N d bf16 rows per head."""
@@ -539,7 +539,7 @@ def main():
                        "l2": "inputs larger than L2 (Q, K, V, dO: 4 x %.0f MB)" % (q.numel() * 2 / 1e6)},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "graph": graph_line,
             "clocks": clk.summary(),
-            "north_star_roofline": north_star_roofline(w, peaks, ms_step),
+            "whole_step_roofline": whole_step_roofline(w, peaks, ms_step),
             "kernels": kernels}
     print(json.dumps(line), flush=True)
     return 0

@@ -10,7 +10,7 @@ Approximation for Training Transformers" (arXiv 2607.20214), cited below as
 [ELSAA <section>, <equation>].  Everything is float64; bf16 inputs enter as
 their exact values.
 
-Readings taken where the page is silent (each is listed in the design doc):
+Readings taken where the page is silent:
   * selector: the page allows "any efficient important-key selector that
     returns an exact sparse output and a denominator" [ELSAA §3.3, Practical
     notes]; this operator uses top-k key blocks per query tile, scored by the
