@@ -647,3 +647,32 @@ def test_row_sampled_forms_match_full(causal):
     np.testing.assert_allclose(sq, dq[rows], atol=1e-11)
     np.testing.assert_allclose(sk, dk[rows], atol=1e-11)
     np.testing.assert_allclose(sv, dv[rows], atol=1e-11)
+
+
+def test_sortlsh_external_orders_and_codes_change_nothing_when_they_agree():
+    """The GPU parity tests hand the oracle the GPU's sorted orders (non-causal) or hash codes
+    (causal); given the oracle's own, the results are identical."""
+    N, d, T = 72, 6, 8
+    q, k, v = _rand((N, d), 140), _rand((N, d), 141), _rand((N, d), 142)
+    dO = _rand((N, d), 143)
+    W = np.zeros((0, d, 4))
+    for causal in (False, True):
+        if causal:
+            N2 = 64                       # the causal recursion in the GPU's form: 2^L blocks
+            q2, k2, v2, dO2 = q[:N2], k[:N2], v[:N2], dO[:N2]
+            p = _causal_lsh_params(N2, d, T, 4, 144)
+        else:
+            q2, k2, v2, dO2 = q, k, v, dO
+            p = _sortlsh_params(N, d, T, 4, 144)
+        fw = orc.forward_head(q2, k2, v2, W, p)
+        g = orc.backward_head(q2, k2, v2, W, dO2, fw, p)
+        if causal:
+            p.lsh_codes = (orc.simhash_codes(q2, p.lsh_planes), orc.simhash_codes(k2, p.lsh_planes))
+        else:
+            p.lsh_orders = (orc.sortlsh_order(q2, p.lsh_planes), orc.sortlsh_order(k2, p.lsh_planes))
+        p.lsh_planes = np.full_like(p.lsh_planes, np.nan)    # the overrides alone must decide
+        fw2 = orc.forward_head(q2, k2, v2, W, p)
+        g2 = orc.backward_head(q2, k2, v2, W, dO2, fw2, p)
+        np.testing.assert_array_equal(fw2["O"], fw["O"])
+        for a, b in zip(g2, g):
+            np.testing.assert_array_equal(a, b)
