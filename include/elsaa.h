@@ -113,11 +113,15 @@ typedef struct {
 
 /* Bytes of the caller-owned `saved` buffer the forward fills and the backward
  * reads (selection, per-row denominators, the fusion weight, O_sparse, RACE
- * features and prefix summaries).  Returns 0 when params are invalid. */
+ * features and prefix summaries; with SORTLSH also the sorted orders, one pair per
+ * recursion level when causal).  Returns 0 when params are invalid. */
 ELSAA_API size_t elsaa_saved_bytes(const elsaa_params* params);
 
 /* Bytes of scratch device memory a forward (for_backward = 0) or backward
- * (for_backward = 1) call needs.  Returns 0 when params are invalid. */
+ * (for_backward = 1) call needs.  With SORTLSH this includes the row-permuted copies
+ * of the inputs and, when causal, every recursion level's gathered rows, partial
+ * results and gradients at once (about 11 and 18 times Q, K and V together for a forward and a backward
+ * at N = 16384, block 128).  Returns 0 when params are invalid. */
 ELSAA_API size_t elsaa_workspace_bytes(const elsaa_params* params, int for_backward);
 
 /* Forward: O = g_s m O_s + g_lr O_lr for every (b, h) [Eq. 4, Eq. 5, §3.1, §3.2].
