@@ -31,7 +31,8 @@ def test_sizes_for_valid_and_invalid_params():
     assert L.elsaa_workspace_bytes(ctypes.byref(p), 0) > 0
     assert L.elsaa_workspace_bytes(ctypes.byref(p), 1) > L.elsaa_workspace_bytes(ctypes.byref(p), 0)
     bad = [dict(d=96), dict(rank_r=24), dict(rank_r=512), dict(block_size=32), dict(topk=200),
-           dict(hash_bits=3), dict(tau=0.0), dict(eps=-1.0)]
+           dict(hash_bits=3), dict(tau=0.0), dict(eps=-1.0),
+           dict(N=0), dict(B=0), dict(H=0), dict(N=-5)]      # empty or negative problems are rejected
     for kw in bad:
         args = dict(B=1, H=2, N=1024, d=64, rank_r=64, block_size=64, topk=4)
         hb = kw.pop("hash_bits", 4)
@@ -40,6 +41,9 @@ def test_sizes_for_valid_and_invalid_params():
         assert L.elsaa_saved_bytes(ctypes.byref(q)) == 0, kw
         assert L.elsaa_workspace_bytes(ctypes.byref(q), 1) == 0, kw
     assert L.elsaa_saved_bytes(None) == 0
+    # the smallest problem (one row, one partial tile) is valid
+    one = bd.make_params(1, 1, 1, 64, rank_r=16, block_size=64, topk=1)
+    assert L.elsaa_saved_bytes(ctypes.byref(one)) > 0
 
 
 def test_block_size_one_is_f32_only():
