@@ -3,9 +3,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl elsaa|reference]
 
 A step is one forward and one backward pass of the whole operator (selection,
-RACE features and summaries, fused sparse + low-rank forward, row scalars,
-suffix summaries, selection inverse, and the four backward kernels) over one
-batch of synthetic input that is resident in HBM.  Default workload: B=1, H=32,
+RACE features and chunk statistics, RACE read-out, sparse forward with the fusion,
+row scalars, suffix statistics, selection inverse, the RACE backward and the
+sparse dQ and dK/dV kernels) over one batch of synthetic input that is resident
+in HBM.  Default workload: B=1, H=32,
 N=16384, d=128, bf16, causal, r=128, 128-key blocks, top-16 blocks per tile.
 Each rank runs its own batch (independent problems, no collective on the data
 path), so multi-GPU runs scale weakly; rank 0 prints one JSON line.
@@ -67,45 +68,42 @@ def work_model(w):
     pair_mma = 2 * T * T * d                        # one T x T x d product
     L = w.n_tables
     m = {}
-    # sparse branch forward: QK^T and PV per selected (tile, block) pair
+    # sparse branch forward: QK^T and PV per selected (tile, block) pair (the useful work; with
+    # blocks of 64 keys the kernels stage two tiles' blocks side by side and mask half of it)
     f_sparse = 2 * pair_mma * sel
-    # RACE read-out in the fused kernel: Phi_Q P (T x r x (d+1)) per tile, plus the
-    # diagonal-chunk kappa (T x T x r) and kappa [V|1] (T x T x (d+1)) when causal
     tiles = w.n_tiles * BH
-    f_read = tiles * 2 * T * r * (d + 1) + (tiles * 2 * T * T * (r + d + 1) if w.causal else 0)
-    m["attn_fwd"] = dict(flops=f_sparse + f_read,
-                         bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 5)   # gathered K,V + Q, O, O_s, O_lr
-    m["attn_fwd_tc"] = dict(flops=f_sparse, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 4)
-    m["race_readout"] = dict(flops=f_read, bytes=tiles * T * (r + d) * 2 * 2 + tiles * r * (d + 8) * 4 * 2)
-    m["sparse_dq"] = dict(flops=3 * pair_mma * sel, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 3)
-    m["dq_tc"] = m["sparse_dq"]
-    m["sparse_dkdv"] = dict(flops=4 * pair_mma * sel, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 4)
-    m["dkdv_tc"] = m["sparse_dkdv"]
-    # RACE read-out and backward on the tensor cores, per chunk of T rows (C = T):
-    # read-out  Phi_Q Phi_K^T, kappa V, Phi_Q P;
-    # query side  dO V^T, dO P^T, dkappa Phi_K, dh W^T;
-    # key side  Phi_K Phi_Q^T, V dO^T, Phi_K R, V R^T, kappa^T dO, dkappa^T Phi_Q, dh W^T.
-    NH = 4 * L
+    m["attn_fwd_tc"] = dict(flops=f_sparse, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 5)   # K,V + Q,O,O_lr + O_s fp32
+    m["dq_tc"] = dict(flops=3 * pair_mma * sel, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 3)
+    m["dkdv_tc"] = dict(flops=4 * pair_mma * sel, bytes=sel * 2 * T * d * 2 + tiles * T * d * 2 * 4)
+    # RACE on the tensor cores, per launch: chunks of C = 128 rows, one launch per group of 128
+    # features (8 tables; G = ceil(r / 128) groups, the last zero-padded)
+    C, R = 128, 128
+    chunks = -(-N // C) * BH
+    G = max(1, -(-r // R))
+    NH = 4 * min(L, 8)                                          # projections of one group
     cz = 1 if w.causal else 0
-    state_b = r * d * 2 * 2 + r * 4                            # per-chunk statistics (bf16 hi + lo, key mass)
-    split_b = r * (d + 8) * 4 * (2 if w.causal else 1) + state_b   # split kernel: fp32 parts in, bf16 out
-    m["race_split_fwd"] = dict(flops=0, bytes=tiles * split_b)
-    m["race_split_bwd"] = dict(flops=0, bytes=tiles * split_b)
-    m["race_readout_tc"] = dict(flops=tiles * 2 * T * (cz * T * r + cz * T * d + r * d),
-                                bytes=tiles * (T * r * 2 * (1 + cz) + cz * T * d * 2 + state_b + T * d * 2 + T * 4))
-    m["race_q_bwd_tc"] = dict(flops=tiles * 2 * T * (cz * T * d + d * r + cz * T * r + NH * d),
-                              bytes=tiles * (T * d * 2 * (2 + cz) + cz * T * r * 2 + state_b + T * NH * 4 + T * 12
-                                             + T * d * 4))
-    m["race_k_bwd_tc"] = dict(flops=tiles * 2 * T * (2 * cz * T * r + 2 * cz * T * d + 2 * r * d + NH * d),
-                              bytes=tiles * (T * r * 2 * (1 + cz) + T * d * 2 * (2 + cz) + state_b + T * NH * 4
-                                             + T * 12 + 2 * T * d * 4))
-    # the mma.sync RACE backward kernels do the same algorithmic work as the tcgen05 ones
-    m["race_q_bwd"] = m["race_q_bwd_tc"]
-    m["race_k_bwd"] = m["race_k_bwd_tc"]
-    f_state = tiles * 2 * T * r * (d + 8)
-    m["race_state_fwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)
-    m["race_state_bwd"] = dict(flops=f_state, bytes=tiles * T * (r + d) * 2 + tiles * r * (d + 8) * 4)
-    m["race_features"] = dict(flops=2 * 2 * BH * N * d * 4 * L * 2, bytes=2 * BH * N * (d + r) * 2)
+    state_b = R * d * 2 * 2 + R * 4                             # per-chunk statistics (bf16 hi + lo, mass)
+    # read-out: Phi_Q Phi_K^T, kappa V, Phi_Q P
+    m["race_readout_tc"] = dict(flops=chunks * 2 * C * (cz * C * R + cz * C * d + R * d),
+                                bytes=chunks * (C * R * 2 * (1 + cz) + cz * C * d * 2 + state_b + C * d * 2 + C * 4))
+    # query side: dO V^T, dO P^T, dkappa Phi_K, dh W^T;  key side: Phi_K Phi_Q^T, V dO^T, Phi_K R,
+    # V R^T, kappa^T dO, dkappa^T Phi_Q, dh W^T
+    m["race_q_bwd_tc"] = dict(flops=chunks * 2 * C * (cz * C * d + d * R + cz * C * R + NH * d),
+                              bytes=chunks * (C * d * 2 * (2 + cz) + cz * C * R * 2 + state_b + C * NH * 4 + C * 12
+                                              + C * d * 4))
+    m["race_k_bwd_tc"] = dict(flops=chunks * 2 * C * (2 * cz * C * R + 2 * cz * C * d + 2 * R * d + NH * d),
+                              bytes=chunks * (C * R * 2 * (1 + cz) + C * d * 2 * (2 + cz) + state_b + C * NH * 4
+                                              + C * 12 + 2 * C * d * 4))
+    # statistics of one group: the totals pass reads Phi and Y once; the emit pass reads them
+    # again (causal) and writes every chunk's statistics
+    f_stats = chunks * 2 * C * R * d
+    rd = chunks * C * (R + d) * 2
+    for side in ("fwd", "bwd"):
+        m[f"race_stats_{side}_totals"] = dict(flops=f_stats, bytes=rd)
+        m[f"race_stats_{side}_emit"] = dict(flops=f_stats * cz, bytes=rd * cz + chunks * state_b)
+    rp = 128 * G
+    m["race_features_tc"] = dict(flops=2 * 2 * BH * N * d * 4 * L * 2,
+                                 bytes=2 * BH * N * (d * 2 + rp * 2 + 4 * L * 4 + 4))
     if w.selector == "sortlsh":
         esz = 2 if w.dtype == "bf16" else 4
         mat = BH * N * d * esz
@@ -113,7 +111,8 @@ def work_model(w):
         m["sortlsh_gather"] = dict(flops=0, bytes=2 * mat)                   # per launch: one matrix in, one out
         m["sortlsh_scatter"] = dict(flops=0, bytes=2 * mat)
     unique_fwd = 4 * BH * N * d * 2                # Q, K, V read, O written
-    return m, dict(sel_pairs=sel, tiles=tiles, f_sparse_fwd=f_sparse, f_lr_fwd=f_read + f_state,
+    f_read = G * m["race_readout_tc"]["flops"]
+    return m, dict(sel_pairs=sel, tiles=tiles, f_sparse_fwd=f_sparse, f_lr_fwd=f_read + G * f_stats,
                    gathered_fwd=sel * 2 * T * d * 2, unique_fwd=unique_fwd)
 
 
@@ -152,6 +151,74 @@ def rank_seed(rank: int) -> int:
 
 
 # --------------------------------------------------------------------------
+
+class NvmlClockSampler:
+    """SM clock and throttle reasons read through NVML every 5 ms on a host thread while the
+    timed region runs (reading only; a short timed region still gets dozens of samples)."""
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, dev):
+        import threading
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(dev)
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        self.bits = [pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                     pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap]
+        self.rows, self.on = [], False
+        self.stop = threading.Event()
+        self.thread = threading.Thread(target=self._loop, daemon=True)
+
+    def _loop(self):
+        nv = self.nv
+        while not self.stop.is_set():
+            if self.on:
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.rows.append((mhz, [n for n, b in zip(self.REASONS, self.bits) if rs & b]))
+                except nv.NVMLError:
+                    pass
+            self.stop.wait(0.005)
+
+    def __enter__(self):
+        self.thread.start()
+        return self
+
+    def mark(self, begin: bool):
+        self.on = begin
+
+    def __exit__(self, *exc):
+        self.stop.set()
+        self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "source": "nvml"}
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted({n for r in self.rows for n in r[1]}), "samples": len(self.rows),
+                "in_window": True, "source": "nvml, every 5 ms"}
+
+
+def clock_sampler(dev, index):
+    try:
+        return NvmlClockSampler(dev)
+    except Exception:
+        return ClockSampler(index)
+
+
+def bf16_peak(peaks, clocks):
+    """The measured bf16 rate that matches the run's clocks: the burst figure (measured at
+    full clock) when the timed region's median SM clock is within 5 % of its maximum, else
+    the sustained one (measured under the power cap)."""
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if "bf16_tflops_sustained" in peaks and not (mhz and mx and mhz >= 0.95 * mx):
+        return peaks["bf16_tflops_sustained"], "sustained"
+    return peaks["bf16_tflops"], "burst"
+
 
 class ClockSampler:
     """nvidia-smi sampling (every 100 ms) while the timed region runs."""
@@ -384,7 +451,7 @@ def main():
         step()
     barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with clock_sampler(dev, local) as clk:
         time.sleep(0.3)
         barrier()
         bd.profile_begin()
@@ -393,6 +460,9 @@ def main():
         for _ in range(args.steps):
             step()
         ev1.record(stream)
+        # wait without holding the interpreter lock, so the clock sampler keeps sampling
+        while not ev1.query():
+            time.sleep(0.0005)
         barrier()
         clk.mark(False)
         prof = bd.profile_end()
@@ -496,24 +566,27 @@ def main():
         return 0
 
     model, _ = work_model(w)
+    clocks = clk.summary()
+    peak_f, peak_f_kind = bf16_peak(peaks, clocks)
     dom = max(prof.items(), key=lambda kv: kv[1][0])[0]
     dom_ms = prof[dom][0] / prof[dom][1]
     wm = model.get(dom)
     roof = None
     if wm is not None:
         # the bound is whichever of the kernel's flops and algorithmic bytes takes longer at peak
-        peak_f = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         tensor_kernel = wm["flops"] / (peak_f * 1e12) >= wm["bytes"] / (peaks["hbm_gbs"] * 1e9)
         if tensor_kernel:
             ach = wm["flops"] / (dom_ms * 1e-3) / 1e12
-            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-            roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak}
+            roof = {"bound": "tensor", "achieved": ach, "peak": peak_f, "unit": "TFLOP/s", "frac": ach / peak_f}
+            src = f"bf16 {peak_f_kind}"
         else:
             ach = wm["bytes"] / (dom_ms * 1e-3) / 1e9
-            peak = peaks["hbm_gbs"]
-            roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak}
-        roof.update({"kernel": dom, "ms_per_launch": dom_ms, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"
-                     if peak_kind == "measured" else "fallback",
+            roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm_gbs"]}
+            src = "copy bandwidth"
+        roof.update({"kernel": dom, "ms_per_launch": dom_ms,
+                     "peak_source": f"{src}, of measured (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                     else f"{src}, of fallback",
                      "traffic": dram_traffic(dom, w.name)})
     kernels = {n: {"ms_per_launch": ms / c, "launches": c, "share": ms / sum(x for x, _ in prof.values())}
                for n, (ms, c) in sorted(prof.items(), key=lambda kv: -kv[1][0])}
@@ -538,8 +611,8 @@ def main():
                        "seq_len": w.N, "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (Q, K, V, dO: 4 x %.0f MB)" % (q.numel() * 2 / 1e6)},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "graph": graph_line,
-            "clocks": clk.summary(),
-            "whole_step_roofline": whole_step_roofline(w, peaks, ms_step),
+            "clocks": clocks,
+            "whole_step_roofline": whole_step_roofline(w, dict(peaks, bf16_tflops=peak_f), ms_step),
             "kernels": kernels}
     print(json.dumps(line), flush=True)
     return 0

@@ -114,7 +114,10 @@ typedef struct {
 /* Bytes of the caller-owned `saved` buffer the forward fills and the backward
  * reads (selection, per-row denominators, the fusion weight, O_sparse, RACE
  * features and prefix summaries; with SORTLSH also the sorted orders, one pair per
- * recursion level when causal).  Returns 0 when params are invalid. */
+ * recursion level when causal).  O_sparse is kept in float32 for every dtype: the
+ * backward forms the softmax delta <dO_s, O_s> from it, and a bf16 copy would put
+ * the rounding of O_s into every dS of a row whose mass sits on a few keys.
+ * Returns 0 when params are invalid. */
 ELSAA_API size_t elsaa_saved_bytes(const elsaa_params* params);
 
 /* Bytes of scratch device memory a forward (for_backward = 0) or backward
@@ -212,6 +215,20 @@ ELSAA_API elsaa_status elsaa_select_noalloc(const elsaa_params* params, const vo
  * the start of `workspace`.  Returns ELSAA_ERR_TIMEOUT if a kernel gave up a
  * bounded wait since the last check, else ELSAA_OK (or ELSAA_ERR_CUDA). */
 ELSAA_API elsaa_status elsaa_check_device_flags(void* workspace, void* stream);
+
+/* Test hook for the bounded device waits (failure detection without a GPU fault).
+ * Every pipeline wait of the tensor-core kernels gives up after a time limit,
+ * records a code in the error word at the start of the call's workspace, drains
+ * the copies and products its block has in flight, frees its tensor memory and
+ * returns; elsaa_check_device_flags then reports ELSAA_ERR_TIMEOUT.
+ *   wait_ns  the limit for calls made from now on; 0 restores the default (2 s)
+ *   stall    1: the tensor-core sparse forward's softmax warps first wait on a
+ *            barrier that nothing completes, so every such launch takes the
+ *            give-up path once the limit has passed (code 0x40000 in the error
+ *            word); 0: normal operation
+ * Process-wide, read when a call starts; not for concurrent use with other
+ * calls.  Returns ELSAA_ERR_INVALID_ARG for stall outside {0, 1}. */
+ELSAA_API elsaa_status elsaa_debug_set_wait_limit(unsigned long long wait_ns, int stall);
 
 /* Opt-in kernel timing.  After elsaa_profile_begin() every kernel the library
  * launches (from any thread, on any stream) is bracketed by two CUDA events

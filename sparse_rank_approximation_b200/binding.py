@@ -31,7 +31,7 @@ ELSAA_SEL_SORTLSH = 1
 EXPORTED = ("elsaa_saved_bytes", "elsaa_workspace_bytes", "elsaa_forward", "elsaa_backward",
             "elsaa_debug_select", "elsaa_check_device_flags", "elsaa_status_string",
             "elsaa_last_error_message", "elsaa_profile_begin", "elsaa_profile_end", "elsaa_select_noalloc",
-            "elsaa_fusion_grads", "elsaa_debug_sortlsh")
+            "elsaa_fusion_grads", "elsaa_debug_sortlsh", "elsaa_debug_set_wait_limit")
 
 
 class Params(ctypes.Structure):
@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
     L.elsaa_fusion_grads.restype = i32
     L.elsaa_debug_sortlsh.argtypes = [P, vp, vp, vp, vp, vp]
     L.elsaa_debug_sortlsh.restype = i32
+    L.elsaa_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong, i32]
+    L.elsaa_debug_set_wait_limit.restype = i32
     _lib = L
     return L
 
@@ -205,6 +207,13 @@ class Elsaa:
 
     def check_device_flags(self, stream=None) -> int:
         return lib().elsaa_check_device_flags(_ptr(self.ws), _stream(stream))
+
+
+def set_wait_limit(wait_ns: int = 0, stall: bool = False) -> None:
+    """Test hook: limit of the tensor-core kernels' bounded waits for calls made from now on
+    (0: the default 2 s); with ``stall`` the sparse forward first waits on a barrier that
+    nothing completes, so its give-up path runs."""
+    _check(lib().elsaa_debug_set_wait_limit(int(wait_ns), int(bool(stall))), "elsaa_debug_set_wait_limit")
 
 
 def profile_begin() -> None:

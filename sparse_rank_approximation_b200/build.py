@@ -16,7 +16,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJDIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libelsaa.so")
-SOURCES = ["elsaa_api.cu", "select.cu", "race.cu", "attn_fwd.cu", "bwd.cu", "f32_path.cu", "noalloc.cu", "race_bwd.cu", "race_readout.cu", "attn_fwd_tc.cu", "bwd_tc.cu", "race_tc.cu", "sortlsh.cu"]
+SOURCES = ["elsaa_api.cu", "select.cu", "race.cu", "bwd.cu", "f32_path.cu", "noalloc.cu", "attn_fwd_tc.cu", "bwd_tc.cu",
+           "race_tc.cu", "race_stats_tc.cu", "race_features_tc.cu", "sortlsh.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr"]

@@ -1,8 +1,12 @@
-// Sparse-branch forward on the 5th-generation tensor cores (tcgen05 + TMEM), for
-// 128-query tiles, 128-key blocks and head dimension 128, fused with the
-// denominator-aware fusion epilogue (ELSAA paper §3.2, §3.3 Eq. 5, §1 Eq. 4).
+// Sparse-branch forward on the 5th-generation tensor cores (tcgen05 + TMEM), fused
+// with the denominator-aware fusion epilogue (ELSAA paper §3.2, §3.3 Eq. 5, §1 Eq. 4).
+// Head dimension D = 64 or 128.  A CTA works on 128 query rows: one tile of 128 queries
+// with 128-key blocks, or (PAIR, blocks of 64) the two adjacent 64-query tiles 2u and
+// 2u + 1, whose selected blocks are staged side by side: the K and V stage of step j
+// holds tile 2u's j-th block in rows 0-63 and tile 2u + 1's in rows 64-127, so every
+// product stays M = N = 128 and each query row masks the other tile's 64 keys.
 //
-// One CTA per (head, query tile), 11 warps:
+// One CTA per (head, 128 query rows), 11 warps:
 //   warp 0      TMA producer of Q and of the K ring (3 stages); once the last
 //               score MMA is done it prefetches the tile's low-rank output O_lr
 //               into a K stage for the epilogue;
@@ -30,8 +34,7 @@ namespace elsaa {
 
 namespace {
 
-constexpr int kT = 128;                  // tile rows = keys per block
-constexpr int kD = 128;                  // head dimension
+constexpr int kT = 128;                  // query rows of a CTA = keys of a K/V stage
 constexpr uint32_t kSlab = kT * 128;     // one [128 rows][64 bf16] swizzled slab
 constexpr uint32_t kTile = 2 * kSlab;    // 128 x 128 bf16
 constexpr uint32_t OFF_Q = 0;
@@ -51,10 +54,11 @@ constexpr int kSoftmaxThreads = 256;
 struct Misc {
   uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full[2], p_full[2],
       pv_done[2];
-  uint64_t olr_full, drain;
+  uint64_t olr_full, drain, never;
+  unsigned long long limit_ns;
   uint32_t tmem_base;
   int abort_flag;
-  int idx[32];
+  int idx[2][32];         // selected blocks of the CTA's tile (PAIR: of its two tiles)
   float red[2][256];      // partial row maxima / sums exchanged by the two halves of a row
 };
 constexpr size_t kSmemBytes = OFF_MISC + sizeof(Misc);
@@ -69,7 +73,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Misc* ms, uint32_t* err,
                                               uint32_t code) {
   if (*(volatile int*)&ms->abort_flag) return false;
-  if (tc::mbar_wait(bar, parity)) return true;
+  if (tc::mbar_wait(bar, parity, ms->limit_ns)) return true;
   *(volatile int*)&ms->abort_flag = 1;
   if (err) atomicOr(err, code);
   return false;
@@ -84,6 +88,7 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
 
 }  // namespace
 
+template <int D, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmLr,
@@ -93,7 +98,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   Misc* ms = reinterpret_cast<Misc*>(smem + OFF_MISC);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
-  const int t = a.tile_list ? a.tile_list[(size_t)bh * a.n_list + blockIdx.x] : g.n_t - 1 - (int)blockIdx.x;
+  constexpr int TB = PAIR ? 64 : 128;       // keys per block = queries per tile
+  constexpr int H = D / 2;                  // output columns per thread (half a row)
+  // the CTA's rows: tile t (128 rows), or tiles ta = 2u, tb = 2u + 1 (PAIR; tb may be past the end)
+  const int n_units = PAIR ? (g.n_t + 1) / 2 : g.n_t;
+  const int unit = a.tile_list ? (PAIR ? a.tile_list[(size_t)bh * a.n_list + 2 * blockIdx.x] / 2
+                                       : a.tile_list[(size_t)bh * a.n_list + blockIdx.x])
+                               : n_units - 1 - (int)blockIdx.x;
+  const int ta = PAIR ? 2 * unit : unit, tb = PAIR ? 2 * unit + 1 : unit;
+  const int row0 = kT * unit;
   const size_t head = (size_t)bh * g.N;
   if (smem_u32(smem) & 1023u) {            // the swizzled layouts need 1024-byte aligned tiles
     if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
@@ -101,7 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---- set-up: barriers, selected blocks, TMEM
-  const int* my_idx = a.idx + ((size_t)bh * g.n_t + t) * g.k;
+  const int* idx_a = a.idx + ((size_t)bh * g.n_t + ta) * g.k;
+  const int* idx_b = a.idx + ((size_t)bh * g.n_t + tb) * g.k;
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->q_full, 1);
     for (int s = 0; s < kStages; ++s) {
@@ -117,10 +131,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc::mbar_init(&ms->olr_full, 1);
     tc::mbar_init(&ms->drain, 1);
+    tc::mbar_init(&ms->never, 1);
+    ms->limit_ns = g.wait_ns;
     ms->abort_flag = 0;
     tc::fence_barrier_init();
   }
-  if (threadIdx.x < 32) ms->idx[threadIdx.x] = threadIdx.x < g.k ? my_idx[threadIdx.x] : -1;
+  if (threadIdx.x < 32) {
+    ms->idx[0][threadIdx.x] = threadIdx.x < g.k ? idx_a[threadIdx.x] : -1;
+    ms->idx[1][threadIdx.x] = PAIR && tb < g.n_t && threadIdx.x < g.k ? idx_b[threadIdx.x] : -1;
+  }
   if (warp == 1) {
     tc::tmem_alloc(&ms->tmem_base, kTmemCols);
     tc::tmem_relinquish();
@@ -129,8 +148,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
-  int n_sel = 0;
-  while (n_sel < g.k && n_sel < 32 && ms->idx[n_sel] >= 0) ++n_sel;
+  // block j of tile half h: the first 32 from shared memory, any further ones from global memory
+  auto sel = [&](int h, int j) -> int { return j < 32 ? ms->idx[h][j] : (h ? idx_b : idx_a)[j]; };
+  int n_sel_t[2] = {0, 0};
+  for (int h = 0; h < (PAIR ? 2 : 1); ++h)
+    while (n_sel_t[h] < g.k && (h == 0 || tb < g.n_t) && sel(h, n_sel_t[h]) >= 0) ++n_sel_t[h];
+  const int n_sel = max(n_sel_t[0], n_sel_t[1]);          // steps
 
   if (warp == 0 || warp == 2) {
     // ================= TMA producers: warp 0 Q, K ring, O_lr; warp 2 the V ring =================
@@ -140,10 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t* empty = is_k ? ms->k_empty : ms->v_empty;
       const CUtensorMap* map = is_k ? &tmK : &tmV;
       int issued = 0;
+      constexpr uint32_t kTD = 128u * D * 2;      // bytes of a [128][D] tile
       if (is_k) {
-        tc::mbar_arrive_expect_tx(&ms->q_full, kTile);
-        tc::tma_load_3d(smem + OFF_Q, &tmQ, &ms->q_full, 0, t * kT, bh);
-        tc::tma_load_3d(smem + OFF_Q + kSlab, &tmQ, &ms->q_full, 64, t * kT, bh);
+        tc::mbar_arrive_expect_tx(&ms->q_full, kTD);
+        for (int sl = 0; sl < D / 64; ++sl) tc::tma_load_3d(smem + OFF_Q + sl * kSlab, &tmQ, &ms->q_full, 64 * sl, row0, bh);
       }
       bool alive = true;
       for (int j = 0; j < n_sel; ++j) {
@@ -152,11 +175,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           alive = false;
           break;
         }
-        const int b = ms->idx[j];
         unsigned char* dst = smem + (is_k ? off_k(s) : off_v(s));
-        tc::mbar_arrive_expect_tx(&full[s], kTile);
-        tc::tma_load_3d(dst, map, &full[s], 0, b * kT, bh);
-        tc::tma_load_3d(dst + kSlab, map, &full[s], 64, b * kT, bh);
+        tc::mbar_arrive_expect_tx(&full[s], kTD);
+        for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
+          // PAIR: a tile with fewer blocks stages block 0 in its half (every score of it is masked)
+          const int b = j < (h ? n_sel_t[1] : n_sel_t[0]) ? sel(h, j) : 0;
+          for (int sl = 0; sl < D / 64; ++sl)
+            tc::tma_load_3d(dst + sl * kSlab + h * 64 * 128, map, &full[s], 64 * sl, b * TB, bh);
+        }
         issued = j + 1;
       }
       bool lr_issued = false;
@@ -165,9 +191,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = (n_sel > kStages ? n_sel - kStages : 0); alive && j < n_sel; ++j)
           alive = wait_or_abort(&ms->k_empty[j % kStages], (j / kStages) & 1, ms, err, 2048u);
         if (alive) {
-          tc::mbar_arrive_expect_tx(&ms->olr_full, kTile);
-          tc::tma_load_3d(smem + off_k(0), &tmLr, &ms->olr_full, 0, t * kT, bh);
-          tc::tma_load_3d(smem + off_k(0) + kSlab, &tmLr, &ms->olr_full, 64, t * kT, bh);
+          tc::mbar_arrive_expect_tx(&ms->olr_full, kTD);
+          for (int sl = 0; sl < D / 64; ++sl)
+            tc::tma_load_3d(smem + off_k(0) + sl * kSlab, &tmLr, &ms->olr_full, 64 * sl, row0, bh);
           lr_issued = true;
         }
       }
@@ -181,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================= MMA issuer =================
     if (lane == 0) {
       const uint32_t idS = tc::idesc_bf16(128, 128, false, false);   // Q (K-major) x K (K-major)
-      const uint32_t idPV = tc::idesc_bf16(128, kD, false, true);    // P (TMEM) x V (MN-major)
+      const uint32_t idPV = tc::idesc_bf16(128, D, false, true);     // P (TMEM) x V (MN-major)
       const uint32_t sbase = smem_u32(smem);
       bool ok = wait_or_abort(&ms->q_full, 0, ms, err, 2u);
       int pv_issued = 0;
@@ -208,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tc_fence_after();
         const uint32_t kb = sbase + off_k(sk);
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = tc::sw128_desc(sbase + OFF_Q + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = tc::sw128_desc(kb + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
           tc::mma_bf16(tmem + tm_s(s), ad, bd, idS, kk > 0 ? 1u : 0u);
@@ -225,12 +251,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ================= softmax / epilogue: half a query row per thread =================
     const int q4 = warp & 3;
-    const int half = (warp - 3) >> 2;                // score / output columns [64 half, 64 half + 64)
+    const int half = (warp - 3) >> 2;                // score columns [64 half, +64), output [H half, +H)
     const int row = 32 * q4 + lane;
     const int sid = half * 128 + row;                // slot in the exchange arrays
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
     const float sl2 = g.scale * kLog2e;
-    const int qrow = t * kT + row;
+    const int qrow = row0 + row;
+    // PAIR: rows 0-63 belong to tile ta and score columns 0-63, rows 64-127 to tile tb and
+    // columns 64-127; a thread whose half holds the other tile's keys masks all of them
+    const int mine = PAIR ? (row >= 64) : 0;
+    const int my_tile = PAIR ? (mine ? tb : ta) : ta;
+    const int my_n = mine ? n_sel_t[1] : n_sel_t[0];
+    const bool dead_half = PAIR && half != mine;
+    const int qpos = PAIR ? (row & 63) : row;        // query position within its tile
     const size_t ri = head + min(qrow, g.N - 1);
     // per-row fusion inputs, fetched now so their latency hides behind the main loop
     const float dl = a.dlr[ri];
@@ -239,6 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float glr_in = a.glr ? a.glr[ri] : -1.f;
     float m_used = -INFINITY, lp = 0.f;              // running max (scaled log2 units), partial row sum
     bool alive = true;                               // warp-uniform; every barrier below is still taken
+    // test hook: a wait on a barrier nothing completes, so the give-up path runs
+    if (g.debug_stall) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->never, 0, ms, err, 0x40000u));
     for (int j = 0; j < n_sel; ++j) {
       const int s = j & 1;
       float sv[64];
@@ -255,10 +290,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) sv[32 + i] = tmp[i];
         tc::tmem_wait_ld();
-        const int b = ms->idx[j];
-        const int kvalid = g.N - b * kT;
-        if ((g.causal && b == t) || kvalid < kT) {   // block-uniform: only the diagonal / ragged block masks
-          const int lim = min(kvalid - 1, (g.causal && b == t) ? row : kT - 1) - 64 * half;
+        // key k of this half's 64 columns is key c0 + k of block b (no block: all masked)
+        const bool none = dead_half || j >= my_n;
+        const int b = none ? 0 : sel(PAIR ? half : 0, j);
+        const int c0 = PAIR ? 0 : 64 * half;
+        const int kvalid = g.N - b * TB;
+        const bool diag = g.causal && b == my_tile;
+        if (none) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) sv[c] = -INFINITY;
+        } else if (diag || kvalid < TB) {            // only the diagonal / ragged block masks
+          const int lim = min(kvalid - 1, diag ? qpos : TB - 1) - c0;
 #pragma unroll
           for (int c = 0; c < 64; ++c) sv[c] = c > lim ? -INFINITY : sv[c];
         }
@@ -313,13 +355,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (alive) {
             tc::tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < H / 32; ++c) {
               float tmp[32];
-              tc::tmem_ld32(tmem + lane_base + TM_O + 64 * half + 32 * c, tmp);
+              tc::tmem_ld32(tmem + lane_base + TM_O + H * half + 32 * c, tmp);
               tc::tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 32; ++i) tmp[i] *= alpha;
-              tc::tmem_st32(tmem + lane_base + TM_O + 64 * half + 32 * c, tmp);
+              tc::tmem_st32(tmem + lane_base + TM_O + H * half + 32 * c, tmp);
             }
             tc::tmem_wait_st();
           }
@@ -331,22 +373,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // ---- epilogue: O_s = O / l, log d_s, fusion (Eq. 5, Eq. 4), TMA stores from shared memory
-    float o[64];
+    float o[H];
 #pragma unroll
-    for (int c = 0; c < 64; ++c) o[c] = 0.f;
+    for (int c = 0; c < H; ++c) o[c] = 0.f;
     if (alive && n_sel > 0) {
       alive = __all_sync(0xffffffffu,
                          wait_or_abort(&ms->pv_done[(n_sel - 1) & 1], ((n_sel - 1) >> 1) & 1, ms, err, 128u));
       if (alive) {
         tc::tc_fence_after();
-        float tmp[32];
-        tc::tmem_ld32(tmem + lane_base + TM_O + 64 * half, tmp);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = tmp[i];
-        tc::tmem_ld32(tmem + lane_base + TM_O + 64 * half + 32, tmp);
+        for (int c2 = 0; c2 < H / 32; ++c2) {
+          float tmp[32];
+          tc::tmem_ld32(tmem + lane_base + TM_O + H * half + 32 * c2, tmp);
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[32 + i] = tmp[i];
-        tc::tmem_wait_ld();
+          for (int i = 0; i < 32; ++i) o[32 * c2 + i] = tmp[i];
+        }
       }
     }
     const int rb = n_sel & 1;                         // exchange buffer not read in the last loop step
@@ -354,31 +396,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->olr_full, 0, ms, err, 4096u));
     softmax_bar();
     const float l = ms->red[rb][row] + ms->red[rb][128 + row];
-    // every PV product is done: V stages 0 and 1 hold the outgoing O and O_s
+    // every PV product is done: V stage 0 holds the outgoing O, V stages 1 (and 2) the fp32 O_s
     if (alive) {
       const float logd = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const float mf = g.fixed_m ? 1.f : logd == -INFINITY ? 0.f : 1.f / (1.f + (lam * dl + g.eps) * expf(-logd));
       const float gl = a.glr ? glr_in : g.fixed_m ? 1.f : 1.f - mf;
       const float cs = gs * mf;
-      const unsigned char* lrow = smem + off_k(0) + half * kSlab + row * 128;
-      unsigned char* orow = smem + off_v(0) + half * kSlab + row * 128;
+      // this thread's output columns [col0, col0 + H), 16-byte chunks of 8 bf16 from chunk ch0
+      // of their 64-column slab
+      const int col0 = H * half, ch0 = (col0 & 63) >> 3;
+      const unsigned char* lrow = smem + off_k(0) + (col0 >> 6) * kSlab + row * 128;
+      unsigned char* orow = smem + off_v(0) + (col0 >> 6) * kSlab + row * 128;
       // with a row map, O goes straight to the caller's row (8 bf16 per 16-byte unit)
       uint4* grow = a.q_rows && qrow < g.N
                         ? reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) +
-                                                   (head + a.q_rows[(size_t)bh * a.rows_stride + qrow]) * kD + 64 * half)
+                                                   (head + a.q_rows[(size_t)bh * a.rows_stride + qrow]) * D + col0)
                         : nullptr;
-      unsigned char* srow = smem + off_v(1) + half * kSlab + row * 128;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const int sw = (ch ^ (row & 7)) << 4;
+      for (int ch = 0; ch < H / 8; ++ch) {
+        const int sw = ((ch0 + ch) ^ (row & 7)) << 4;
         const uint4 lr = *reinterpret_cast<const uint4*>(lrow + sw);
         const __nv_bfloat16* lv = reinterpret_cast<const __nv_bfloat16*>(&lr);
-        uint32_t wo[4], ws[4];
+        uint32_t wo[4];
+        float sv[8];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float s0 = o[8 * ch + 2 * e] * inv_l, s1 = o[8 * ch + 2 * e + 1] * inv_l;
-          ws[e] = pack_bf16(s0, s1);
+          sv[2 * e] = s0;
+          sv[2 * e + 1] = s1;
           wo[e] = pack_bf16(cs * s0 + gl * __bfloat162float(lv[2 * e]), cs * s1 + gl * __bfloat162float(lv[2 * e + 1]));
         }
         if (a.q_rows) {
@@ -386,7 +432,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           *reinterpret_cast<uint4*>(orow + sw) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
         }
-        *reinterpret_cast<uint4*>(srow + sw) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+        // O_s in fp32 (the backward's softmax delta is formed from it): boxes of [128 rows][32
+        // floats] with the 128-byte swizzle over the V stages after the first; column fc sits
+        // in box fc / 32, 16-byte chunk (fc % 32) / 4
+        const int fc = col0 + 8 * ch;
+        unsigned char* sbox = smem + off_v(1) + (fc >> 5) * kSlab + row * 128;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int cc = ((fc & 31) >> 2) + e;
+          *reinterpret_cast<float4*>(sbox + ((cc ^ (row & 7)) << 4)) =
+              make_float4(sv[4 * e], sv[4 * e + 1], sv[4 * e + 2], sv[4 * e + 3]);
+        }
       }
       if (half == 0 && qrow < g.N) {
         a.logd[head + qrow] = logd;
@@ -396,12 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_proxy_async_smem();
     softmax_bar();
     if (threadIdx.x == 96 && !*(volatile int*)&ms->abort_flag) {
-      if (!a.q_rows) {
-        tma_store_3d(&tmO, smem + off_v(0), 0, t * kT, bh);
-        tma_store_3d(&tmO, smem + off_v(0) + kSlab, 64, t * kT, bh);
-      }
-      tma_store_3d(&tmS, smem + off_v(1), 0, t * kT, bh);
-      tma_store_3d(&tmS, smem + off_v(1) + kSlab, 64, t * kT, bh);
+      if (!a.q_rows)
+        for (int sl = 0; sl < D / 64; ++sl) tma_store_3d(&tmO, smem + off_v(0) + sl * kSlab, 64 * sl, row0, bh);
+      for (int b = 0; b < D / 32; ++b) tma_store_3d(&tmS, smem + off_v(1) + b * kSlab, 32 * b, row0, bh);
       asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
       asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
     }
@@ -428,35 +481,58 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [BH][N][128] bf16 viewed as a 3-D tensor (d, row, head); boxes of 64 x 128 x 1,
-// 128-byte swizzle; loads past row N read zeros, stores past row N are dropped.
-static bool make_map(CUtensorMap* m, const void* base, int N, int BH) {
+// [BH][N][d] bf16 viewed as a 3-D tensor (column, row, head); boxes of 64 columns x `rows`
+// rows, 128-byte swizzle; loads past row N read zeros, stores past row N are dropped.
+static bool make_map(CUtensorMap* m, const void* base, int d, int N, int BH, int rows) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)N, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)N * kD * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)kT, 1};
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool attn_fwd_tc_supported(const Geom& g) { return g.d == kD && g.T == kT && g.k <= 32; }
+// [BH][N][d] fp32 viewed as (column, row, head); boxes of 32 x 128 x 1 (128-byte rows),
+// 128-byte swizzle; stores past row N are dropped.
+static bool make_map_f32(CUtensorMap* m, void* base, int d, int N, int BH) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)N * d * 4};
+  cuuint32_t box[3] = {32, (cuuint32_t)kT, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool attn_fwd_tc_supported(const Geom& g) { return (g.d == 64 || g.d == 128) && (g.T == 64 || g.T == 128); }
+
+template <int D, bool PAIR>
+static cudaError_t fwd_t(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
+  constexpr int TB = PAIR ? 64 : 128;
+  if (PAIR && a.tile_list && (a.n_list & 1)) return cudaErrorInvalidValue;   // tile pairs
+  CUtensorMap mq, mk, mv, mlr, mo, ms;
+  if (!make_map(&mq, a.Q, D, g.N, g.BH, kT) || !make_map(&mk, a.K, D, g.N, g.BH, TB) ||
+      !make_map(&mv, a.V, D, g.N, g.BH, TB) || !make_map(&mlr, a.Olr, D, g.N, g.BH, kT) ||
+      !make_map(&mo, a.O, D, g.N, g.BH, kT) || !make_map_f32(&ms, a.Os, D, g.N, g.BH))
+    return cudaErrorInvalidValue;
+  auto kern = attn_fwd_tc_kernel<D, PAIR>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int units = a.tile_list ? (PAIR ? a.n_list / 2 : a.n_list) : (PAIR ? (g.n_t + 1) / 2 : g.n_t);
+  ProfScope ps("attn_fwd_tc", st);
+  kern<<<dim3(units, g.BH), kThreads, kSmemBytes, st>>>(mq, mk, mv, mlr, mo, ms, a, g, err);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_attn_fwd_tc(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
   if (!attn_fwd_tc_supported(g)) return cudaErrorInvalidValue;
-  CUtensorMap mq, mk, mv, mlr, mo, ms;
-  if (!make_map(&mq, a.Q, g.N, g.BH) || !make_map(&mk, a.K, g.N, g.BH) || !make_map(&mv, a.V, g.N, g.BH) ||
-      !make_map(&mlr, a.Olr, g.N, g.BH) || !make_map(&mo, a.O, g.N, g.BH) || !make_map(&ms, a.Os, g.N, g.BH))
-    return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
-  ProfScope ps("attn_fwd_tc", st);
-  attn_fwd_tc_kernel<<<dim3(a.tile_list ? a.n_list : g.n_t, g.BH), kThreads, kSmemBytes, st>>>(mq, mk, mv, mlr, mo,
-                                                                                               ms, a, g, err);
-  return cudaGetLastError();
+  if (g.d == 64) return g.T == 64 ? fwd_t<64, true>(a, g, err, st) : fwd_t<64, false>(a, g, err, st);
+  return g.T == 64 ? fwd_t<128, true>(a, g, err, st) : fwd_t<128, false>(a, g, err, st);
 }
 
 }  // namespace elsaa

@@ -63,7 +63,7 @@ struct DqMisc {
       st_free, ds_full[2], done;
   uint32_t tmem_base;
   int abort_flag;
-  int idx[32];
+  int idx[2][32];         // selected blocks of the CTA's tile (PAIR: of its two tiles)
 };
 
 template <typename M>
@@ -94,6 +94,10 @@ __device__ __forceinline__ void dq_softmax_cols(const float (&sv)[64], const flo
 
 }  // namespace
 
+// D = 64 or 128.  PAIR (blocks of 64): the CTA's 128 query rows are the tiles 2u and 2u + 1,
+// and the K / V stage of step j holds tile 2u's j-th block in rows 0-63 and tile 2u + 1's in
+// rows 64-127; each query row masks the other tile's 64 keys (dS = 0 there).
+template <int D, bool PAIR>
 __global__ void __launch_bounds__(kDqThreads, 1)
     dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -102,13 +106,21 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   DqMisc* ms = reinterpret_cast<DqMisc*>(smem + DQ_MISC);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
-  const int t = a.tile_list ? a.tile_list[(size_t)bh * a.n_list + blockIdx.x] : g.n_t - 1 - (int)blockIdx.x;
+  constexpr int TB = PAIR ? 64 : 128;       // keys per block = queries per tile
+  constexpr int H = D / 2;                  // dQ columns per thread (half a row)
+  const int n_units = PAIR ? (g.n_t + 1) / 2 : g.n_t;
+  const int unit = a.tile_list ? (PAIR ? a.tile_list[(size_t)bh * a.n_list + 2 * blockIdx.x] / 2
+                                       : a.tile_list[(size_t)bh * a.n_list + blockIdx.x])
+                               : n_units - 1 - (int)blockIdx.x;
+  const int ta = PAIR ? 2 * unit : unit, tb = PAIR ? 2 * unit + 1 : unit;
+  const int row0 = kT * unit;
   const size_t head = (size_t)bh * g.N;
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
     return;
   }
-  const int* my_idx = a.idx + ((size_t)bh * g.n_t + t) * g.k;
+  const int* idx_a = a.idx + ((size_t)bh * g.n_t + ta) * g.k;
+  const int* idx_b = a.idx + ((size_t)bh * g.n_t + tb) * g.k;
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->qd_full, 1);
     for (int s = 0; s < kDqKStages; ++s) {
@@ -127,7 +139,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     ms->abort_flag = 0;
     tc::fence_barrier_init();
   }
-  if (threadIdx.x < 32) ms->idx[threadIdx.x] = threadIdx.x < g.k ? my_idx[threadIdx.x] : -1;
+  if (threadIdx.x < 32) {
+    ms->idx[0][threadIdx.x] = threadIdx.x < g.k ? idx_a[threadIdx.x] : -1;
+    ms->idx[1][threadIdx.x] = PAIR && tb < g.n_t && threadIdx.x < g.k ? idx_b[threadIdx.x] : -1;
+  }
   if (warp == 1) {
     tc::tmem_alloc(&ms->tmem_base, 512);
     tc::tmem_relinquish();
@@ -136,8 +151,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
-  int n_sel = 0;
-  while (n_sel < g.k && n_sel < 32 && ms->idx[n_sel] >= 0) ++n_sel;
+  // block j of tile half h: the first 32 from shared memory, any further ones from global memory
+  auto sel = [&](int h, int j) -> int { return j < 32 ? ms->idx[h][j] : (h ? idx_b : idx_a)[j]; };
+  int n_sel_a = 0, n_sel_b = 0;
+  while (n_sel_a < g.k && sel(0, n_sel_a) >= 0) ++n_sel_a;
+  while (PAIR && tb < g.n_t && n_sel_b < g.k && sel(1, n_sel_b) >= 0) ++n_sel_b;
+  const int n_sel = max(n_sel_a, n_sel_b);          // steps
 
   if (warp == 0 || warp == 10) {
     // ---------------- TMA producers: warp 0 Q, dO and the K ring; warp 10 the V ring ----------------
@@ -146,22 +165,26 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       const int NS = kside ? kDqKStages : kDqVStages;
       uint64_t* full = kside ? ms->k_full : ms->v_full;
       uint64_t* empty = kside ? ms->k_empty : ms->v_empty;
+      constexpr uint32_t kTD = 128u * D * 2;      // bytes of a [128][D] tile
       if (kside) {
-        tc::mbar_arrive_expect_tx(&ms->qd_full, 2 * kTile);
-        tc::tma_load_3d(smem + DQ_Q, &tmQ, &ms->qd_full, 0, t * kT, bh);
-        tc::tma_load_3d(smem + DQ_Q + kSlab, &tmQ, &ms->qd_full, 64, t * kT, bh);
-        tc::tma_load_3d(smem + DQ_DO, &tmdO, &ms->qd_full, 0, t * kT, bh);
-        tc::tma_load_3d(smem + DQ_DO + kSlab, &tmdO, &ms->qd_full, 64, t * kT, bh);
+        tc::mbar_arrive_expect_tx(&ms->qd_full, 2 * kTD);
+        for (int sl = 0; sl < D / 64; ++sl) {
+          tc::tma_load_3d(smem + DQ_Q + sl * kSlab, &tmQ, &ms->qd_full, 64 * sl, row0, bh);
+          tc::tma_load_3d(smem + DQ_DO + sl * kSlab, &tmdO, &ms->qd_full, 64 * sl, row0, bh);
+        }
       }
       int issued = 0;
       for (int j = 0; j < n_sel; ++j) {
         const int s = j % NS;
         if (j >= NS && !wait_or_abort(&empty[s], ((j / NS) - 1) & 1, ms, err, kside ? 1u : 2u)) break;
-        const int b = ms->idx[j];
         unsigned char* dst = smem + (kside ? dq_k(s) : dq_v(s));
-        tc::mbar_arrive_expect_tx(&full[s], kTile);
-        tc::tma_load_3d(dst, kside ? &tmK : &tmV, &full[s], 0, b * kT, bh);
-        tc::tma_load_3d(dst + kSlab, kside ? &tmK : &tmV, &full[s], 64, b * kT, bh);
+        tc::mbar_arrive_expect_tx(&full[s], kTD);
+        for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
+          // PAIR: a tile with fewer blocks stages block 0 in its half (every score of it is masked)
+          const int b = j < (h ? n_sel_b : n_sel_a) ? sel(h, j) : 0;
+          for (int sl = 0; sl < D / 64; ++sl)
+            tc::tma_load_3d(dst + sl * kSlab + h * 64 * 128, kside ? &tmK : &tmV, &full[s], 64 * sl, b * TB, bh);
+        }
         issued = j + 1;
       }
       if (kside) tc::mbar_wait(&ms->qd_full, 0);
@@ -171,7 +194,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);   // both operands K-major
-      const uint32_t idNM = tc::idesc_bf16(128, kD, false, true);     // B MN-major
+      const uint32_t idNM = tc::idesc_bf16(128, D, false, true);      // B MN-major, N = D
       const uint32_t sb = smem_u32(smem);
       bool ok = wait_or_abort(&ms->qd_full, 0, ms, err, 4u);
       int dq_issued = 0;
@@ -194,7 +217,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         if (j >= 1 && !wait_or_abort(&ms->st_free, (j - 1) & 1, ms, err, 32u)) break;
         tc::tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
           tc::mma_bf16(tmem + TM_DP, tc::sw128_desc(sb + DQ_DO + off, 16, 1024),
                        tc::sw128_desc(sb + dq_v(sv) + off, 16, 1024), idNN, kk > 0 ? 1u : 0u);
@@ -203,7 +226,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         if (!wait_or_abort(&ms->k_full[sk], (j / kDqKStages) & 1, ms, err, 64u)) break;
         tc::tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
           tc::mma_bf16(tmem + TM_S, tc::sw128_desc(sb + DQ_Q + off, 16, 1024),
                        tc::sw128_desc(sb + dq_k(sk) + off, 16, 1024), idNN, kk > 0 ? 1u : 0u);
@@ -221,8 +244,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const int half = (warp - 2) >> 2;
     const int row = 32 * q4 + lane;
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-    const int qrow = t * kT + row;
+    const int qrow = row0 + row;
     const bool row_ok = qrow < g.N;
+    // PAIR: rows 0-63 belong to tile ta and key columns 0-63, rows 64-127 to tile tb and
+    // columns 64-127; a thread whose half holds the other tile's keys masks all of them
+    const int mine = PAIR ? (row >= 64) : 0;
+    const int my_tile = PAIR ? (mine ? tb : ta) : ta;
+    const int my_n = mine ? n_sel_b : n_sel_a;
+    const bool dead_half = PAIR && half != mine;
+    const int qpos = PAIR ? (row & 63) : row;        // query position within its tile
     const float4 sc = row_ok ? a.rs.packed[head + qrow] : make_float4(INFINITY, 0.f, 0.f, 0.f);
     const float lg2 = sc.x, cs = sc.y, Dl = sc.z;
     const float sl2 = g.scale * kLog2e;
@@ -239,10 +269,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       tc::tmem_wait_ld();
       tc::tc_fence_before();
       tc::mbar_arrive(&ms->st_free);
-      const int b = ms->idx[j];
-      const int kvalid = g.N - b * kT;
-      const bool mask = (g.causal && b == t) || kvalid < kT;
-      const int lim = min(kvalid - 1, (g.causal && b == t) ? row : kT - 1) - 64 * half;
+      // key k of this half's 64 columns is key c0 + k of block b (no block: all masked)
+      const bool none = dead_half || j >= my_n;
+      const int b = none ? 0 : sel(PAIR ? half : 0, j);
+      const int c0 = PAIR ? 0 : 64 * half;
+      const int kvalid = g.N - b * TB;
+      const bool diag = g.causal && b == my_tile;
+      const bool mask = none || diag || kvalid < TB;
+      const int lim = none ? -1 : min(kvalid - 1, diag ? qpos : TB - 1) - c0;
       uint32_t w[32];
       // block-uniform: only the diagonal block and a ragged last block need the mask
       if (mask)
@@ -270,22 +304,24 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       have = alive;
       if (have) tc::tc_fence_after();
     }
+    const int col0 = H * half;                       // this thread's dQ columns [col0, col0 + H)
     const float4* acc =
-        alive && row_ok && a.dQacc ? reinterpret_cast<const float4*>(a.dQacc + (head + qrow) * kD + 64 * half) : nullptr;
+        alive && row_ok && a.dQacc ? reinterpret_cast<const float4*>(a.dQacc + (head + qrow) * D + col0) : nullptr;
     // every product has completed: stage the bf16 tile in the Q buffer, 32 columns at a time
     // (with a row map, write each row straight to the caller's row instead)
-    unsigned char* orow = smem + DQ_Q + half * kSlab + row * 128;
+    unsigned char* orow = smem + DQ_Q + (col0 >> 6) * kSlab + row * 128;
+    const int ch0 = (col0 & 63) >> 3;
     uint4* grow = a.q_rows && row_ok && alive
                       ? reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dQ) +
-                                                 (head + a.q_rows[(size_t)bh * a.rows_stride + qrow]) * kD + 64 * half)
+                                                 (head + a.q_rows[(size_t)bh * a.rows_stride + qrow]) * D + col0)
                       : nullptr;
 #pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < H / 32; ++c) {
       float o[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) o[i] = 0.f;
       if (have) {
-        tc::tmem_ld32(tmem + lane_base + TM_DQ + 64 * half + 32 * c, o);
+        tc::tmem_ld32(tmem + lane_base + TM_DQ + col0 + 32 * c, o);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] *= g.scale;
@@ -297,6 +333,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           o[4 * q] += v.x; o[4 * q + 1] += v.y; o[4 * q + 2] += v.z; o[4 * q + 3] += v.w;
         }
       }
+      if (a.out_f32) {                                   // fp32 rows (level slots), no staging
+        if (alive && row_ok) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.dQ) + (head + qrow) * D + col0 + 32 * c);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        }
+        continue;
+      }
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int ch = 4 * c + cc;
@@ -305,16 +349,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         if (a.q_rows) {
           if (grow) grow[ch] = val;
         } else {
-          *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) = val;
+          *reinterpret_cast<uint4*>(orow + (((ch0 + ch) ^ (row & 7)) << 4)) = val;
         }
       }
     }
-    if (!a.q_rows) {
+    if (!a.q_rows && !a.out_f32) {
       tc::fence_proxy_async_smem();
       softmax_bar();
       if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
-        tma_store_3d(&tmdQ, smem + DQ_Q, 0, t * kT, bh);
-        tma_store_3d(&tmdQ, smem + DQ_Q + kSlab, 64, t * kT, bh);
+        for (int sl = 0; sl < D / 64; ++sl) tma_store_3d(&tmdQ, smem + DQ_Q + sl * kSlab, 64 * sl, row0, bh);
         tma_store_wait();
       }
     }
@@ -335,8 +378,8 @@ __host__ __device__ constexpr uint32_t kv_q(int s) { return 2 * kTile + s * 2 * 
 __host__ __device__ constexpr uint32_t kv_do(int s) { return kv_q(s) + kTile; }            // dO tile, stage s
 constexpr uint32_t KV_SC = 2 * kTile + kStages * 2 * kTile;                   // scalars [stage][128] float4
 constexpr int kMaxUnits = 1024;
-constexpr uint32_t KV_UNITS = KV_SC + kStages * 128 * 16;                     // query tiles of this block
-constexpr uint32_t KV_MISC = KV_UNITS + kMaxUnits * 4;
+constexpr uint32_t KV_UNITS = KV_SC + kStages * 128 * 16;                     // query tiles of the block(s)
+constexpr uint32_t KV_MISC = KV_UNITS + 2 * kMaxUnits * 4;
 // TMEM columns: S^T [keys][queries] and dP^T (fp32); once read, (P^T cs) and dS^T (bf16 pairs)
 // overwrite the first 8 of every 16 columns and feed dV / dK as the tensor-memory A operand.
 constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_DV = 256, TM_DK = 384;
@@ -387,6 +430,10 @@ __device__ __forceinline__ void dkdv_softmax_cols(uint32_t tmem, uint32_t st_col
 // softmax warps turn them into (P^T cs) and dS^T in two passes of 64 queries; after each
 // pass dV += (P^T cs) dO and dK += dS^T Q over those 64 queries run on the tensor cores
 // while the other pass is computed.
+// D = 64 or 128.  PAIR (blocks of 64): the CTA's 128 key rows are blocks 2c (rows 0-63) and
+// 2c + 1 (rows 64-127); unit u stages the u-th query tile of block 2c in query rows 0-63 and
+// the u-th of block 2c + 1 in rows 64-127, and each key row masks the other block's queries.
+template <int D, bool PAIR>
 __global__ void __launch_bounds__(kKvThreads, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
@@ -394,24 +441,35 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                    const __grid_constant__ CUtensorMap tmdV, BwdArgs a, Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   KvMisc* ms = reinterpret_cast<KvMisc*>(smem + KV_MISC);
-  int* units = reinterpret_cast<int*>(smem + KV_UNITS);
+  int* units = reinterpret_cast<int*>(smem + KV_UNITS);       // [2][kMaxUnits] query tiles of the block(s)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x;
-  // heaviest key blocks of every head first (order from the selection inverse)
-  const int b = a.kv_order ? a.kv_order[(size_t)bh * g.n_t + blockIdx.y] : (int)blockIdx.y;
+  constexpr int TB = PAIR ? 64 : 128;       // keys per block = queries per tile
+  constexpr int H = D / 2;                  // dK / dV columns per thread (half a row)
+  // heaviest key blocks of every head first (order from the selection inverse); PAIR: the
+  // pairs in order
+  const int b = PAIR ? 2 * (int)blockIdx.y
+                     : (a.kv_order ? a.kv_order[(size_t)bh * g.n_t + blockIdx.y] : (int)blockIdx.y);
+  const int key0 = PAIR ? 64 * b : kT * b;   // first key row of the CTA
   const size_t head = (size_t)bh * g.N;
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
     return;
   }
-  int n_u = 0;
+  int n_ut[2] = {0, 0};
   if (g.k > 0) {
     const int* of = a.offs + (size_t)bh * (g.n_t + 1);
     const int* list = a.tiles + (size_t)bh * g.n_t * g.k;
-    const int e0 = of[b];
-    n_u = min(of[b + 1] - e0, kMaxUnits);
-    for (int i = threadIdx.x; i < n_u; i += kKvThreads) units[i] = list[e0 + i];
+    for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
+      const int bb = b + h;
+      if (bb >= g.n_t) break;
+      const int e0 = of[bb];
+      n_ut[h] = min(of[bb + 1] - e0, kMaxUnits);
+      for (int i = threadIdx.x; i < n_ut[h]; i += kKvThreads) units[h * kMaxUnits + i] = list[e0 + i];
+    }
   }
+  const int n_ua = n_ut[0], n_ub = n_ut[1];
+  const int n_u = max(n_ua, n_ub);
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->kv_full, 1);
     for (int s = 0; s < kStages; ++s) {
@@ -437,22 +495,27 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&ms->kv_full, 2 * kTile);
-      tc::tma_load_3d(smem + KV_K, &tmK, &ms->kv_full, 0, b * kT, bh);
-      tc::tma_load_3d(smem + KV_K + kSlab, &tmK, &ms->kv_full, 64, b * kT, bh);
-      tc::tma_load_3d(smem + KV_V, &tmV, &ms->kv_full, 0, b * kT, bh);
-      tc::tma_load_3d(smem + KV_V + kSlab, &tmV, &ms->kv_full, 64, b * kT, bh);
+      constexpr uint32_t kTD = 128u * D * 2;      // bytes of a [128][D] tile
+      tc::mbar_arrive_expect_tx(&ms->kv_full, 2 * kTD);
+      for (int sl = 0; sl < D / 64; ++sl) {
+        tc::tma_load_3d(smem + KV_K + sl * kSlab, &tmK, &ms->kv_full, 64 * sl, key0, bh);
+        tc::tma_load_3d(smem + KV_V + sl * kSlab, &tmV, &ms->kv_full, 64 * sl, key0, bh);
+      }
       int issued = 0;
       for (int u = 0; u < n_u; ++u) {
         const int s = u % kStages;
         if (u >= kStages && !wait_or_abort(&ms->qd_empty[s], ((u / kStages) - 1) & 1, ms, err, 1u)) break;
-        const int row0 = units[u] * kT;
-        tc::mbar_arrive_expect_tx(&ms->qd_full[s], 2 * kTile + 128 * 16);
-        tc::tma_load_3d(smem + kv_q(s), &tmQ, &ms->qd_full[s], 0, row0, bh);
-        tc::tma_load_3d(smem + kv_q(s) + kSlab, &tmQ, &ms->qd_full[s], 64, row0, bh);
-        tc::tma_load_3d(smem + kv_do(s), &tmdO, &ms->qd_full[s], 0, row0, bh);
-        tc::tma_load_3d(smem + kv_do(s) + kSlab, &tmdO, &ms->qd_full[s], 64, row0, bh);
-        tc::tma_load_3d(smem + KV_SC + s * 128 * 16, &tmSc, &ms->qd_full[s], 0, row0, bh);
+        tc::mbar_arrive_expect_tx(&ms->qd_full[s], 2 * kTD + 128 * 16);
+        for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
+          // PAIR: a block with fewer query tiles stages tile 0 in its half (all of it is masked)
+          const int t = u < (h ? n_ub : n_ua) ? units[h * kMaxUnits + u] : 0;
+          const int qr = t * TB;
+          for (int sl = 0; sl < D / 64; ++sl) {
+            tc::tma_load_3d(smem + kv_q(s) + sl * kSlab + h * 64 * 128, &tmQ, &ms->qd_full[s], 64 * sl, qr, bh);
+            tc::tma_load_3d(smem + kv_do(s) + sl * kSlab + h * 64 * 128, &tmdO, &ms->qd_full[s], 64 * sl, qr, bh);
+          }
+          tc::tma_load_3d(smem + KV_SC + s * 128 * 16 + h * 64 * 16, &tmSc, &ms->qd_full[s], 0, qr, bh);
+        }
         issued = u + 1;
       }
       tc::mbar_wait(&ms->kv_full, 0);
@@ -463,7 +526,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idS = tc::idesc_bf16(128, 128, false, false);    // K (keys x d) x Q (queries x d)
-      const uint32_t idG = tc::idesc_bf16(128, kD, false, true);      // P^T / dS^T (TMEM) x (dO / Q, MN-major)
+      const uint32_t idG = tc::idesc_bf16(128, D, false, true);       // P^T / dS^T (TMEM) x (dO / Q, MN-major)
       const uint32_t sb = smem_u32(smem);
       bool ok = wait_or_abort(&ms->kv_full, 0, ms, err, 2u);
       for (int u = 0; ok && u < n_u; ++u) {
@@ -473,13 +536,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         // S^T and dP^T overwrite the columns that held the previous unit's P^T / dS^T:
         // the products that read those were issued earlier and tcgen05 MMAs run in order
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
           tc::mma_bf16(tmem + TM_ST, tc::sw128_desc(sb + KV_K + off, 16, 1024),
                        tc::sw128_desc(sb + kv_q(s) + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
           tc::mma_bf16(tmem + TM_DPT, tc::sw128_desc(sb + KV_V + off, 16, 1024),
                        tc::sw128_desc(sb + kv_do(s) + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
@@ -512,25 +575,35 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     // ---------------- softmax: one key row; two passes of 32 queries per thread ----------------
     const int q4 = warp & 3;
     const int grp = (warp - 2) >> 2;                // queries 32 grp + 64 pass .. + 31
-    const int row = 32 * q4 + lane;                 // key row within the block
+    const int row = 32 * q4 + lane;                 // key row within the CTA's 128
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-    const bool key_ok = b * kT + row < g.N;
+    const bool key_ok = key0 + row < g.N;
     const float sl2 = g.scale * kLog2e;
+    // PAIR: key rows 0-63 are block b and see query rows 0-63 of a unit (pass 0), rows 64-127
+    // block b + 1 and query rows 64-127 (pass 1)
+    const int mine = PAIR ? (row >= 64) : 0;
+    const int my_block = b + mine;
+    const int kpos = PAIR ? (row & 63) : row;       // key position within its block
     bool alive = true;
     for (int u = 0; u < n_u && alive; ++u) {
       const int s = u % kStages;
-      const int t = units[u];
       alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full, u & 1, ms, err, 32u));
       if (!alive) break;
       tc::tc_fence_after();
-      const bool diag = g.causal && t == b;
 #pragma unroll 1
       for (int pass = 0; pass < 2; ++pass) {
-        const int q0 = 64 * pass + 32 * grp;        // first query (within tile t) of this thread
-        const int qvalid = g.N - t * kT - q0;       // queries of this thread inside the sequence
-        const bool masked = !key_ok || qvalid < 32 || (diag && row > q0);
-        const int lo = diag ? row - q0 : 0;
-        const int hi = key_ok ? qvalid : 0;
+        const int q0 = 64 * pass + 32 * grp;        // first query (column of the unit) of this thread
+        // the query tile of these columns and the first one's position in it
+        const int h = PAIR ? pass : 0;
+        const bool present = u < (h ? n_ub : n_ua);
+        const int t = present ? units[h * kMaxUnits + u] : 0;
+        const int qp0 = PAIR ? q0 - 64 * pass : q0;
+        const bool dead = PAIR && (pass != mine || !present);
+        const bool diag = g.causal && t == my_block;
+        const int qvalid = g.N - t * TB - qp0;      // queries of this thread inside the sequence
+        const bool masked = dead || !key_ok || qvalid < 32 || (diag && kpos > qp0);
+        const int lo = diag ? kpos - qp0 : 0;
+        const int hi = dead ? 0 : key_ok ? qvalid : 0;
         const float4* sc = reinterpret_cast<const float4*>(smem + KV_SC + s * 128 * 16) + q0;
         // masking only on the causal diagonal, at the end of the sequence and for padding keys
         if (__any_sync(0xffffffffu, masked))
@@ -544,6 +617,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     }
     // ---------------- epilogue: dK = scale dK_sparse + dK_lowrank, dV likewise; TMA stores ----------------
     const int hq = grp;
+    const int col0 = H * hq;                         // this thread's columns [col0, col0 + H)
+    const int ch0 = (col0 & 63) >> 3;
     bool have = false;
     if (alive && n_u > 0) {
       alive = __all_sync(0xffffffffu, wait_or_abort(&ms->done, 0, ms, err, 512u));
@@ -556,23 +631,23 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const float mul = which == 0 ? g.scale : 1.f;
       const float* accp = which == 0 ? a.dKacc : a.dVacc;
       const float4* ak = accp && alive && key_ok
-                             ? reinterpret_cast<const float4*>(accp + (head + (size_t)b * kT + row) * kD + 64 * hq)
+                             ? reinterpret_cast<const float4*>(accp + (head + (size_t)key0 + row) * D + col0)
                              : nullptr;
-      unsigned char* orow = smem + (which == 0 ? kv_q(0) : kv_do(0)) + hq * kSlab + row * 128;
+      unsigned char* orow = smem + (which == 0 ? kv_q(0) : kv_do(0)) + (col0 >> 6) * kSlab + row * 128;
       // with a row map, write each key row straight to the caller's row instead
       uint4* grow = a.k_rows && key_ok && alive
                         ? reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(which == 0 ? a.dK : a.dV) +
-                                                   (head + a.k_rows[(size_t)bh * a.rows_stride + b * kT + row]) * kD +
-                                                   64 * hq)
+                                                   (head + a.k_rows[(size_t)bh * a.rows_stride + key0 + row]) * D +
+                                                   col0)
                         : nullptr;
       // 32 columns at a time: TMEM -> scale -> + low-rank part -> bf16 -> swizzled row
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < H / 32; ++c) {
         float o[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0.f;
         if (have) {
-          tc::tmem_ld32(tmem + lane_base + (which == 0 ? TM_DK : TM_DV) + 64 * hq + 32 * c, o);
+          tc::tmem_ld32(tmem + lane_base + (which == 0 ? TM_DK : TM_DV) + col0 + 32 * c, o);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= mul;
@@ -584,6 +659,15 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             o[4 * q] += x.x; o[4 * q + 1] += x.y; o[4 * q + 2] += x.z; o[4 * q + 3] += x.w;
           }
         }
+        if (a.out_f32) {                                 // fp32 rows (level slots), no staging
+          if (alive && key_ok) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(which == 0 ? a.dK : a.dV) +
+                                                    (head + (size_t)key0 + row) * D + col0 + 32 * c);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+          }
+          continue;
+        }
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           const int ch = 4 * c + cc;
@@ -593,19 +677,19 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           if (a.k_rows) {
             if (grow) grow[ch] = val;
           } else {
-            *reinterpret_cast<uint4*>(orow + ((ch ^ (row & 7)) << 4)) = val;
+            *reinterpret_cast<uint4*>(orow + (((ch0 + ch) ^ (row & 7)) << 4)) = val;
           }
         }
       }
     }
-    if (!a.k_rows) {
+    if (!a.k_rows && !a.out_f32) {
       tc::fence_proxy_async_smem();
       softmax_bar();
       if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
-        tma_store_3d(&tmdK, smem + kv_q(0), 0, b * kT, bh);
-        tma_store_3d(&tmdK, smem + kv_q(0) + kSlab, 64, b * kT, bh);
-        tma_store_3d(&tmdV, smem + kv_do(0), 0, b * kT, bh);
-        tma_store_3d(&tmdV, smem + kv_do(0) + kSlab, 64, b * kT, bh);
+        for (int sl = 0; sl < D / 64; ++sl) {
+          tma_store_3d(&tmdK, smem + kv_q(0) + sl * kSlab, 64 * sl, key0, bh);
+          tma_store_3d(&tmdV, smem + kv_do(0) + sl * kSlab, 64 * sl, key0, bh);
+        }
         tma_store_wait();
       }
     }
@@ -634,10 +718,16 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // [BH][N][128] bf16 as a 3-D tensor (d, row, head), boxes of 64 x rows x 1, 128-byte swizzle.
 bool tc::map_rows_bf16(CUtensorMap* m, const void* base, int N, int BH, int rows) {
+  return map_rows_bf16_pitch(m, base, kD, kD, N, BH, rows);
+}
+
+// `cols` columns of [BH][N][pitch] bf16 rows starting at `base` (all of them, or a column
+// block of wider rows), in boxes of 64 columns.
+bool tc::map_rows_bf16_pitch(CUtensorMap* m, const void* base, int cols, int pitch, int N, int BH, int rows) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)N, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)N * kD * 2};
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)pitch * 2, (cuuint64_t)N * pitch * 2};
   cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -645,55 +735,76 @@ bool tc::map_rows_bf16(CUtensorMap* m, const void* base, int N, int BH, int rows
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool bwd_tc_supported(const Geom& g) { return g.d == kD && g.T == kT && g.k <= 32; }
+bool bwd_tc_supported(const Geom& g) { return (g.d == 64 || g.d == 128) && (g.T == 64 || g.T == 128); }
 
-cudaError_t launch_dq_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
-  if (!bwd_tc_supported(g) || !a.rs.packed) return cudaErrorInvalidValue;
+// [BH][N][d] bf16 rows in boxes of 64 columns x `rows` rows
+static bool map_d(CUtensorMap* m, const void* base, const Geom& g, int rows) {
+  return tc::map_rows_bf16_pitch(m, base, g.d, g.d, g.N, g.BH, rows);
+}
+
+template <int D, bool PAIR>
+static cudaError_t dq_t(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
+  constexpr int TB = PAIR ? 64 : 128;
+  if (PAIR && a.tile_list && (a.n_list & 1)) return cudaErrorInvalidValue;   // tile pairs
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if (!tc::map_rows_bf16(&mq, a.Q, g.N, g.BH, kT) || !tc::map_rows_bf16(&mk, a.K, g.N, g.BH, kT) ||
-      !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kT) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, kT) ||
-      !tc::map_rows_bf16(&mdq, a.dQ, g.N, g.BH, kT))
+  if (!map_d(&mq, a.Q, g, kT) || !map_d(&mk, a.K, g, TB) || !map_d(&mv, a.V, g, TB) || !map_d(&mdo, a.dO, g, kT) ||
+      !map_d(&mdq, a.dQ, g, kT))
     return cudaErrorInvalidValue;
   const size_t smem = DQ_MISC + sizeof(DqMisc);
   static_assert(DQ_MISC + sizeof(DqMisc) <= 232448, "shared memory per CTA");
-  cudaError_t e = cudaFuncSetAttribute(dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = dq_tc_kernel<D, PAIR>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  const int units = a.tile_list ? (PAIR ? a.n_list / 2 : a.n_list) : (PAIR ? (g.n_t + 1) / 2 : g.n_t);
   ProfScope ps("dq_tc", st);
-  dq_tc_kernel<<<dim3(a.tile_list ? a.n_list : g.n_t, g.BH), kDqThreads, smem, st>>>(mq, mk, mv, mdo, mdq, a, g, err);
+  kern<<<dim3(units, g.BH), kDqThreads, smem, st>>>(mq, mk, mv, mdo, mdq, a, g, err);
   return cudaGetLastError();
 }
 
-// Per-row scalars (log2 d_s, cs, Delta, 0) as float32 [BH][N][4]; boxes of 4 x 128 x 1.
-static bool map_scalars(CUtensorMap* m, const void* base, int N, int BH) {
+cudaError_t launch_dq_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
+  if (!bwd_tc_supported(g) || !a.rs.packed) return cudaErrorInvalidValue;
+  if (g.d == 64) return g.T == 64 ? dq_t<64, true>(a, g, err, st) : dq_t<64, false>(a, g, err, st);
+  return g.T == 64 ? dq_t<128, true>(a, g, err, st) : dq_t<128, false>(a, g, err, st);
+}
+
+// Per-row scalars (log2 d_s, cs, Delta, 0) as float32 [BH][N][4]; boxes of 4 x rows x 1.
+static bool map_scalars(CUtensorMap* m, const void* base, int N, int BH, int rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {4, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {16, (cuuint64_t)N * 16};
-  cuuint32_t box[3] = {4, 128, 1};
+  cuuint32_t box[3] = {4, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
-  if (!bwd_tc_supported(g) || !a.rs.packed || g.n_t > kMaxUnits || (a.n_kv && !a.kv_order) || a.n_kv > g.n_t)
-    return cudaErrorInvalidValue;
+template <int D, bool PAIR>
+static cudaError_t dkdv_t(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
+  constexpr int TB = PAIR ? 64 : 128;
   CUtensorMap mk, mv, mq, mdo, msc, mdk, mdv;
-  if (!tc::map_rows_bf16(&mk, a.K, g.N, g.BH, kT) || !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kT) ||
-      !tc::map_rows_bf16(&mq, a.Q, g.N, g.BH, kT) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, kT) ||
-      !map_scalars(&msc, a.rs.packed, g.N, g.BH) || !tc::map_rows_bf16(&mdk, a.dK, g.N, g.BH, kT) ||
-      !tc::map_rows_bf16(&mdv, a.dV, g.N, g.BH, kT))
+  if (!map_d(&mk, a.K, g, kT) || !map_d(&mv, a.V, g, kT) || !map_d(&mq, a.Q, g, TB) || !map_d(&mdo, a.dO, g, TB) ||
+      !map_scalars(&msc, a.rs.packed, g.N, g.BH, TB) || !map_d(&mdk, a.dK, g, kT) || !map_d(&mdv, a.dV, g, kT))
     return cudaErrorInvalidValue;
   const size_t smem = KV_MISC + sizeof(KvMisc);
   static_assert(KV_MISC + sizeof(KvMisc) <= 232448, "shared memory per CTA");
-  cudaError_t e = cudaFuncSetAttribute(dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = dkdv_tc_kernel<D, PAIR>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("dkdv_tc", st);
-  // with n_kv, only the first n_kv key blocks of kv_order (the ones with query tiles) run
-  dkdv_tc_kernel<<<dim3(g.BH, a.n_kv ? a.n_kv : g.n_t), kKvThreads, smem, st>>>(mk, mv, mq, mdo, msc, mdk, mdv, a, g,
-                                                                               err);
+  // with n_kv, only the first n_kv key blocks of kv_order (the ones with query tiles) run; pairs
+  // of blocks run in order (the empty ones write zeros)
+  const int ctas = PAIR ? (g.n_t + 1) / 2 : (a.n_kv ? a.n_kv : g.n_t);
+  kern<<<dim3(g.BH, ctas), kKvThreads, smem, st>>>(mk, mv, mq, mdo, msc, mdk, mdv, a, g, err);
   return cudaGetLastError();
+}
+
+cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
+  if (!bwd_tc_supported(g) || !a.rs.packed || g.n_t > kMaxUnits || (a.n_kv && !a.kv_order) || a.n_kv > g.n_t)
+    return cudaErrorInvalidValue;
+  if (g.d == 64) return g.T == 64 ? dkdv_t<64, true>(a, g, err, st) : dkdv_t<64, false>(a, g, err, st);
+  return g.T == 64 ? dkdv_t<128, true>(a, g, err, st) : dkdv_t<128, false>(a, g, err, st);
 }
 
 }  // namespace elsaa

@@ -2,6 +2,7 @@
 // `saved` and `workspace` buffers, and the launch sequence of the forward and
 // backward passes.  The operator is defined in include/elsaa.h.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -19,6 +20,11 @@ using namespace elsaa;
 namespace {
 
 thread_local std::string g_last_error;
+
+// test hook (elsaa_debug_set_wait_limit): pipeline-wait limit and the forward stall
+std::atomic<unsigned long long> g_wait_ns{0};
+std::atomic<int> g_debug_stall{0};
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
 
 elsaa_status fail(elsaa_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 elsaa_status fail(elsaa_status s, const char* fmt, ...) {
@@ -47,6 +53,8 @@ struct Carver {
     return p;
   }
 };
+
+bool tc_race(const Geom& g, bool bf16);
 
 bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
   *st = ELSAA_OK;
@@ -99,7 +107,7 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
       return false;
     }
     if (p->causal) {
-      // the recursion runs on the bf16 sparse kernels (tcgen05 or mma.sync), halving down
+      // the recursion runs on the bf16 tensor-core sparse kernels, halving down
       // to single blocks
       if (!bf16) {
         *st = fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH needs bf16");
@@ -131,7 +139,9 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
   g->k = lsh ? (p->causal ? 2 : 1) : p->topk;
   g->r = p->rank_r;
   g->L = p->rank_r >> kHashBits;
-  g->C = bf16 ? T : 64;
+  // RACE chunk length: 128 rows on the bf16 (tensor-core) path whatever the block size, 64 on the
+  // fp32 path (the result does not depend on it)
+  g->C = bf16 ? 128 : 64;
   g->n_c = (p->N + g->C - 1) / g->C;
   long want = ((long)g->BH * g->n_c + 295) / 296;   // about two segments per SM
   g->seg = (int)std::max(1L, std::min(16L, want));
@@ -146,8 +156,28 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
   g->lam = p->lambda;
   g->eps = p->eps;
   g->tau = p->tau;
+  g->rp = g->r;
+  g->G = 1;
+  if (tc_race(*g, bf16)) {          // decided by dtype and r alone: the shape checks above admit
+                                     // only shapes the tensor-core RACE kernels take
+    // the tensor-core RACE kernels take the features in groups of 128 (8 tables), zero-padded
+    g->G = (g->r + 127) / 128;
+    g->rp = 128 * g->G;
+    // the tensor-core statistics walk a segment per CTA, one CTA per SM: about one wave
+    const int per_head = std::max(1, 148 / g->BH);
+    g->seg = std::max(1, (g->n_c + per_head - 1) / per_head);
+    g->n_seg = (g->n_c + g->seg - 1) / g->seg;
+  }
+  const unsigned long long wn = g_wait_ns.load();
+  g->wait_ns = wn ? wn : kDefaultWaitNs;
+  g->debug_stall = g_debug_stall.load();
   return true;
 }
+
+// The tensor-core RACE path (statistics, read-out, backward): every bf16 problem with a low-rank
+// branch (d = 64 or 128, chunks of 128 rows, r up to 256 in groups of 128 features).  The
+// launchers check the geometry (race_bwd_tc_supported) and refuse anything else.
+bool tc_race(const Geom& g, bool bf16) { return bf16 && g.r > 0; }
 
 struct Saved {
   int* idx;
@@ -165,24 +195,27 @@ Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
   Carver c(base);
   Saved s;
   const size_t rows = (size_t)g.BH * g.N;
-  const size_t state = (size_t)g.r * g.dp;
+  const bool split = tc_race(g, esz == 2);
+  // a state holds the statistics of r features, or on the tensor-core path of one group of 128
+  // (the groups run one after another and reuse it)
+  const size_t state = (size_t)(split ? 128 : g.r) * g.dp;
   s.idx = c.take<int>((size_t)g.BH * g.n_t * std::max(g.k, 1));
   s.logd = c.take<float>(rows);
   s.dlr = c.take<float>(rows);
   s.m = c.take<float>(rows);
-  s.Os = c.take<char>(rows * g.d * esz);
+  s.Os = c.take<float>(rows * g.d);          // fp32 on every path: the backward's softmax delta reads it
   s.Olr = c.take<char>(rows * g.d * esz);
-  s.phiQ = c.take<char>(rows * g.r * esz);
-  s.phiK = c.take<char>(rows * g.r * esz);
+  s.phiQ = c.take<char>(rows * g.rp * esz);
+  s.phiK = c.take<char>(rows * g.rp * esz);
   s.hQ = c.take<float>(rows * g.L * kHashBits);
   s.hK = c.take<float>(rows * g.L * kHashBits);
   s.nQ = c.take<float>(rows);
   s.nK = c.take<float>(rows);
   s.Ast = c.take<float>((size_t)g.BH * (g.n_seg + 1) * state);
-  s.Bst = c.take<float>(g.causal ? (size_t)g.BH * g.n_c * state : 0);
-  const bool split = esz == 2 && g.r > 0 && race_bwd_tc_supported(g);
-  s.Psplit = split ? c.take<char>((size_t)g.BH * g.n_c * 2 * g.r * g.d * 2) : nullptr;
-  s.Pmass = split ? c.take<float>((size_t)g.BH * g.n_c * g.r) : nullptr;
+  // the in-segment prefix is kept only by the fp32 statistics
+  s.Bst = c.take<float>(g.causal && !split ? (size_t)g.BH * g.n_c * state : 0);
+  s.Psplit = split ? c.take<char>((size_t)g.BH * g.n_c * 2 * g.rp * g.d * 2) : nullptr;
+  s.Pmass = split ? c.take<float>((size_t)g.BH * g.n_c * g.rp) : nullptr;
   const size_t orders = g.selector != ELSAA_SEL_SORTLSH ? 0 : g.causal ? (size_t)g.lsh_levels : 1;
   s.lsh_order = orders ? c.take<int>(orders * g.BH * 2 * g.N) : nullptr;
   *bytes = align_up(c.off);
@@ -204,8 +237,8 @@ struct PermBufs {
   float *logd, *m, *logd_lv;
   int *idx, *tile_list, *offs, *tiles, *order, *pos, *inv;
   float4* packed;
-  // the sparse-only passes' low-rank outputs: the mma.sync forward writes O_lr and d_lr
-  // (zero without a low-rank branch), the tcgen05 one reads them; neither is used
+  // the sparse-only passes' low-rank inputs: the forward kernel reads O_lr and d_lr, whose
+  // contents do not matter there (m is held at 1 and the fused output is not used)
   void* Olr;
   float* dlr;
 };
@@ -237,9 +270,10 @@ PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
   b.tile_list = c.take<int>(vheads * (g.n_t / 2));
   if (backward) {
     b.X = c.take<char>(lv * mat);
-    b.dQ = c.take<char>(lv * mat);
-    b.dK = c.take<char>(lv * mat);
-    b.dV = c.take<char>(lv * mat);
+    // the level gradients stay fp32 until the base pass's single bf16 rounding
+    b.dQ = c.take<float>(lv * rows * g.d);
+    b.dK = c.take<float>(lv * rows * g.d);
+    b.dV = c.take<float>(lv * rows * g.d);
     b.packed = c.take<float4>(lv * rows);
     b.offs = c.take<int>(vheads * (g.n_t + 1));
     b.tiles = c.take<int>(vheads * g.n_t);
@@ -248,12 +282,12 @@ PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
     return b;
   }
   b.X = c.take<char>(mat);
-  b.Os = c.take<char>(mat);
+  b.Os = c.take<float>(rows * g.d);
   b.logd = c.take<float>(rows);
   b.m = c.take<float>(std::max<size_t>(lv, 1) * rows);
   b.Olr = c.take<char>(std::max<size_t>(lv, 1) * mat);
   b.dlr = c.take<float>(std::max<size_t>(lv, 1) * rows);
-  b.Os_lv = c.take<char>(lv * mat);
+  b.Os_lv = c.take<float>(lv * rows * g.d);
   b.logd_lv = c.take<float>(lv * rows);
   b.inv = c.take<int>(lv * rows);
   b.pos = c.take<int>(rows * 2);
@@ -265,6 +299,7 @@ struct FwdWs {
   double *qbar, *kbar;
   float* scores;
   void* wsplit;
+  float *lr_num, *lr_den;
   PermBufs pm;
 };
 
@@ -275,7 +310,11 @@ FwdWs carve_fwd_ws(void* base, const Geom& g, size_t esz, size_t* bytes) {
   w.qbar = c.take<double>((size_t)g.BH * g.n_t * g.d);
   w.kbar = c.take<double>((size_t)g.BH * g.n_t * g.d);
   w.scores = c.take<float>((size_t)g.BH * g.n_t * g.n_t);
-  w.wsplit = c.take<char>((size_t)2 * ((g.L * kHashBits + 15) & ~15) * g.d * 2);
+  w.wsplit = c.take<char>((size_t)2 * ((g.L * kHashBits + 31) & ~31) * g.d * 2);
+  // tensor-core read-out over several feature groups: the running numerator and denominator
+  const bool groups = g.G > 1 && tc_race(g, esz == 2);
+  w.lr_num = groups ? c.take<float>((size_t)g.BH * g.N * g.d) : nullptr;
+  w.lr_den = groups ? c.take<float>((size_t)g.BH * g.N) : nullptr;
   w.pm = carve_perm(c, g, esz, false);
   *bytes = align_up(c.off);
   return w;
@@ -297,7 +336,7 @@ BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
   Carver c(base);
   BwdWs w;
   const size_t rows = (size_t)g.BH * g.N;
-  const size_t state = (size_t)g.r * g.dp;
+  const size_t state = (size_t)(tc_race(g, bf16) ? 128 : g.r) * g.dp;
   w.flag = c.take<uint32_t>(64);
   w.rs.cs = c.take<float>(rows);
   w.rs.Delta = c.take<float>(rows);
@@ -305,7 +344,7 @@ BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
   w.rs.delta = c.take<float>(rows);
   w.rs.packed = bf16 ? c.take<float4>(rows) : nullptr;
   w.RA = c.take<float>((size_t)g.BH * (g.n_seg + 1) * state);
-  w.RB = c.take<float>(g.causal ? (size_t)g.BH * g.n_c * state : 0);
+  w.RB = c.take<float>(g.causal && !tc_race(g, bf16) ? (size_t)g.BH * g.n_c * state : 0);
   w.offs = c.take<int>((size_t)g.BH * (g.n_t + 1));
   w.tiles = c.take<int>((size_t)g.BH * g.n_t * std::max(g.k, 1));
   w.order = c.take<int>((size_t)g.BH * g.n_t);
@@ -315,19 +354,13 @@ BwdWs carve_bwd_ws(void* base, const Geom& g, bool bf16, size_t* bytes) {
   w.dKacc = acc ? c.take<float>(acc) : nullptr;
   w.dVacc = acc ? c.take<float>(acc) : nullptr;
   w.dOcl = c.take<char>(bf16 && g.r > 0 ? rows * g.d * 2 : 0);
-  const bool split = bf16 && g.r > 0 && race_bwd_tc_supported(g);
-  w.Rsplit = split ? c.take<char>((size_t)g.BH * g.n_c * 2 * g.r * g.d * 2) : nullptr;
-  w.Rmass = split ? c.take<float>((size_t)g.BH * g.n_c * g.r) : nullptr;
-  w.Wsplit = split ? c.take<char>((size_t)2 * ((g.L * kHashBits + 15) & ~15) * g.d * 2) : nullptr;
+  const bool split = tc_race(g, bf16);
+  w.Rsplit = split ? c.take<char>((size_t)g.BH * g.n_c * 2 * g.rp * g.d * 2) : nullptr;
+  w.Rmass = split ? c.take<float>((size_t)g.BH * g.n_c * g.rp) : nullptr;
+  w.Wsplit = split ? c.take<char>((size_t)2 * ((g.L * kHashBits + 31) & ~31) * g.d * 2) : nullptr;
   w.pm = carve_perm(c, g, bf16 ? 2 : 4, true);
   *bytes = align_up(c.off);
   return w;
-}
-
-// ELSAA_DISABLE_TCGEN05=1 selects the mma.sync kernels everywhere (for A/B checks).
-bool tcgen05_disabled() {
-  const char* v = getenv("ELSAA_DISABLE_TCGEN05");
-  return v && v[0] == '1';
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -348,6 +381,56 @@ elsaa_status cuda_status(cudaError_t e, const char* where) {
     elsaa_status _s = (expr);             \
     if (_s != ELSAA_OK) return _s;        \
   } while (0)
+
+// ---- a second stream for the block selection --------------------------------
+// The selection does not depend on the RACE branch, so a forward runs it on a second stream
+// (one per host thread and device, created on first use) while the features, statistics and
+// read-out run on the caller's stream; one event pair forks and joins them before the sparse
+// forward.  Both are stream-ordered, so a CUDA-graph capture of the caller's stream takes the
+// forked work in as well.  If the stream cannot be created, the selection stays on the caller's.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool failed = false;
+};
+constexpr int kMaxSideDevices = 64;
+SideStream* side_stream() {
+  thread_local SideStream per_dev[kMaxSideDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) return nullptr;
+  SideStream& x = per_dev[dev];
+  if (!x.s && !x.failed) {
+    if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess) {
+      x.failed = true;
+      x.s = nullptr;
+      cudaGetLastError();
+    }
+  }
+  return x.s ? &x : nullptr;
+}
+
+// Makes the caller's stream wait for the selection stream once, on the normal path or, if a
+// launch fails after the fork, when the forward returns (work already queued on the second
+// stream then never outlives the caller's view of the call).  A failure to record the join
+// event leaves the wait on its previous record, which precedes the fork.
+struct JoinGuard {
+  SideStream* side = nullptr;
+  cudaStream_t st = nullptr;
+  bool done = true;
+  cudaError_t join() {
+    if (done || !side) return cudaSuccess;
+    done = true;
+    return cudaStreamWaitEvent(st, side->join, 0);
+  }
+  JoinGuard() = default;
+  JoinGuard(SideStream* s, cudaStream_t t, bool d) : side(s), st(t), done(d) {}
+  JoinGuard& operator=(const JoinGuard&) = default;
+  ~JoinGuard() {
+    if (join() != cudaSuccess) cudaGetLastError();
+  }
+};
 
 // ---- opt-in per-kernel profiler ------------------------------------------
 struct ProfRec {
@@ -442,25 +525,22 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
                                 const float* W, const float* lam, const float* gs, const float* glr, void* O,
                                 const Saved& s, const FwdWs& w, cudaStream_t st) {
   const PermBufs& b = w.pm;
-  // tcgen05 kernels for d = 128, block 128; mma.sync kernels for the other shapes
-  const bool tc = attn_fwd_tc_supported(g) && !tcgen05_disabled();
   const size_t rows = (size_t)g.BH * g.N;
   const int rb = g.d * 2, stride = 2 * g.N;
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st), "flag reset"));
   // the low-rank branch, causal, in the caller's row order
   if (g.r > 0) {
-    ELSAA_TRY(cuda_status(launch_race_features(Q, K, W, w.wsplit, true, s.phiQ, s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, st),
-                          "race features"));
-    ELSAA_TRY(cuda_status(launch_race_state_fwd(s.phiK, V, true, s.Ast, s.Bst, g, st), "race summaries"));
+    ELSAA_TRY(cuda_status(launch_race_w_split(W, w.wsplit, g, st), "W split"));
+    ELSAA_TRY(cuda_status(launch_race_features_tc(Q, K, w.wsplit, s.phiQ, s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, w.flag,
+                                                  st),
+                          "tcgen05 race features"));
     FwdArgs ra{Q, K, V, s.idx, s.phiQ, s.phiK, s.Ast, s.Bst, lam, gs, glr, O, s.Os, s.logd, s.dlr, s.m, s.Olr,
                s.Psplit, s.Pmass};
-    if (s.Psplit && tc) {
-      ELSAA_TRY(cuda_status(launch_race_state_split(s.Ast, s.Bst, false, s.Psplit, s.Pmass, g, st),
-                            "race statistics split"));
-      ELSAA_TRY(cuda_status(launch_race_readout_tc(ra, g, w.flag, st), "tcgen05 race read-out"));
-    } else {
-      ELSAA_TRY(cuda_status(launch_race_readout_bf16(ra, g, st), "race read-out"));
-    }
+    ra.lr_num = w.lr_num;
+    ra.lr_den = w.lr_den;
+    ELSAA_TRY(cuda_status(launch_race_stats_tc(s.phiK, V, nullptr, false, s.Ast, s.Psplit, s.Pmass, g, w.flag, st),
+                          "tcgen05 race statistics"));
+    ELSAA_TRY(cuda_status(launch_race_readout_tc(ra, g, w.flag, st), "tcgen05 race read-out"));
   } else {
     ELSAA_TRY(cuda_status(cudaMemsetAsync(s.Olr, 0, rows * rb, st), "O_lr"));
     ELSAA_TRY(cuda_status(cudaMemsetAsync(s.dlr, 0, rows * 4, st), "d_lr"));
@@ -477,9 +557,7 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
   sa.m = b.m;
   // base pass: the leaves and the deepest level, in the caller's order
   const Geom gb = sparse_only(g, true, 2);
-  auto sparse_pass = [&](const FwdArgs& fa, const Geom& fg) {
-    return tc ? launch_attn_fwd_tc(fa, fg, w.flag, st) : launch_attn_fwd_bf16(fa, fg, st);
-  };
+  auto sparse_pass = [&](const FwdArgs& fa, const Geom& fg) { return launch_attn_fwd_tc(fa, fg, w.flag, st); };
   ELSAA_TRY(cuda_status(launch_causal_lsh_select(s.idx, g, st), "causal sortLSH base selection"));
   sa.Q = Q; sa.K = K; sa.V = V;
   ELSAA_TRY(cuda_status(sparse_pass(sa, gb), "causal sortLSH base pass"));
@@ -520,21 +598,16 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
 
 elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const BwdWs& w, cudaStream_t st) {
   const PermBufs& b = w.pm;
-  const bool tc = bwd_tc_supported(g) && !tcgen05_disabled();
   const size_t rows = (size_t)g.BH * g.N;
   const int rb = g.d * 2, stride = 2 * g.N;
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st), "flag reset"));
   ELSAA_TRY(cuda_status(launch_row_scalars(a, true, g, st), "row scalars"));
   if (g.r > 0) {
-    ELSAA_TRY(cuda_status(launch_race_state_bwd(a, true, g, st), "race suffix summaries"));
-    if (tc && race_bwd_tc_supported(g)) {
-      ELSAA_TRY(cuda_status(launch_race_state_split(w.RA, w.RB, true, w.Rsplit, w.Rmass, g, st),
-                            "race statistics split"));
-      ELSAA_TRY(cuda_status(launch_race_w_split(a.W, w.Wsplit, g, st), "W split"));
-      ELSAA_TRY(cuda_status(launch_race_bwd_tc(a, g, w.flag, st), "tcgen05 race backward"));
-    } else {
-      ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, 1, st), "race backward"));
-    }
+    ELSAA_TRY(cuda_status(launch_race_stats_tc(a.phiQ, a.dOcl, w.rs.delta, true, w.RA, w.Rsplit, w.Rmass, g,
+                                               w.flag, st),
+                          "tcgen05 race statistics"));
+    ELSAA_TRY(cuda_status(launch_race_w_split(a.W, w.Wsplit, g, st), "W split"));
+    ELSAA_TRY(cuda_status(launch_race_bwd_tc(a, g, w.flag, st), "tcgen05 race backward"));
   } else {
     ELSAA_TRY(cuda_status(cudaMemsetAsync(w.dQacc, 0, rows * g.d * 4, st), "dQ accumulator"));
     ELSAA_TRY(cuda_status(cudaMemsetAsync(w.dKacc, 0, rows * g.d * 4, st), "dK accumulator"));
@@ -563,15 +636,12 @@ elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const
     la.idx = b.idx; la.offs = b.offs; la.tiles = b.tiles; la.kv_order = b.order;
     la.rs.packed = b.packed;
     la.dQ = b.dQ; la.dK = b.dK; la.dV = b.dV;
+    la.out_f32 = 1;
     la.tile_list = b.tile_list;
     la.n_list = g.n_t / 2;
     la.n_kv = g.n_t / 2;
-    if (tc) {
-      ELSAA_TRY(cuda_status(launch_dq_tc(la, gv, w.flag, st), "sortLSH level dq"));
-      ELSAA_TRY(cuda_status(launch_dkdv_tc(la, gv, w.flag, st), "sortLSH level dkdv"));
-    } else {                          // mma.sync: every tile and block (the empty ones are cheap)
-      ELSAA_TRY(cuda_status(launch_bwd_bf16(la, gv, 6, st), "sortLSH level sparse backward"));
-    }
+    ELSAA_TRY(cuda_status(launch_dq_tc(la, gv, w.flag, st), "sortLSH level dq"));
+    ELSAA_TRY(cuda_status(launch_dkdv_tc(la, gv, w.flag, st), "sortLSH level dkdv"));
     ELSAA_TRY(cuda_status(launch_lsh_invert_orders(s.lsh_order, b.inv, lv, g, st), "order inverses"));
     ELSAA_TRY(cuda_status(launch_lsh_collect(b.dQ, w.dQacc, nullptr, nullptr, b.inv, lv, false, g, st), "sortLSH dQ"));
     ELSAA_TRY(cuda_status(launch_lsh_collect(b.dK, w.dKacc, b.dV, w.dVacc, b.inv, lv, true, g, st),
@@ -582,7 +652,6 @@ elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const
   ELSAA_TRY(cuda_status(launch_invert_selection(s.idx, w.offs, w.tiles, w.order, gb, st), "selection inverse"));
   a.idx = s.idx; a.offs = w.offs; a.tiles = w.tiles; a.kv_order = w.order;
   a.dQacc = w.dQacc; a.dKacc = w.dKacc; a.dVacc = w.dVacc;
-  if (!tc) return cuda_status(launch_bwd_bf16(a, gb, 6, st), "causal sortLSH base sparse backward");
   ELSAA_TRY(cuda_status(launch_dq_tc(a, gb, w.flag, st), "causal sortLSH base dq"));
   return cuda_status(launch_dkdv_tc(a, gb, w.flag, st), "causal sortLSH base dkdv");
 }
@@ -693,24 +762,52 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
   }
 
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st_), "flag reset"));
+  // the selection on the second stream, joined before the sparse forward
+  SideStream* side = bf16 ? side_stream() : nullptr;
+  cudaStream_t sel_st = st_;
+  JoinGuard joined;                   // an early return still makes the caller's stream wait
+  if (side) {
+    ELSAA_TRY(cuda_status(cudaEventRecord(side->fork, st_), "selection fork"));
+    ELSAA_TRY(cuda_status(cudaStreamWaitEvent(side->s, side->fork, 0), "selection fork"));
+    sel_st = side->s;
+    joined = JoinGuard{side, st_, false};
+  }
   if (lsh)
-    ELSAA_TRY(cuda_status(launch_diag_select(s.idx, g, st_), "selection"));
+    ELSAA_TRY(cuda_status(launch_diag_select(s.idx, g, sel_st), "selection"));
   else
-    ELSAA_TRY(cuda_status(launch_select(Q, K, bf16, w.qbar, w.kbar, w.scores, s.idx, g, st_), "selection"));
-  ELSAA_TRY(cuda_status(launch_race_features(Q, K, W, w.wsplit, bf16, s.phiQ, s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, st_),
-                        "race features"));
-  ELSAA_TRY(cuda_status(launch_race_state_fwd(s.phiK, V, bf16, s.Ast, s.Bst, g, st_), "race summaries"));
-  // per-chunk bf16 hi/lo statistics for the tensor-core read-out and query-side backward
-  if (s.Psplit)
-    ELSAA_TRY(cuda_status(launch_race_state_split(s.Ast, s.Bst, false, s.Psplit, s.Pmass, g, st_),
-                          "race statistics split"));
+    ELSAA_TRY(cuda_status(launch_select(Q, K, bf16, w.qbar, w.kbar, w.scores, s.idx, g, sel_st), "selection"));
+  if (side) ELSAA_TRY(cuda_status(cudaEventRecord(side->join, sel_st), "selection join"));
+  if (g.r > 0 && bf16) {
+    ELSAA_TRY(cuda_status(launch_race_w_split(W, w.wsplit, g, st_), "W split"));
+    ELSAA_TRY(cuda_status(launch_race_features_tc(Q, K, w.wsplit, s.phiQ, s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, w.flag,
+                                                  st_),
+                          "tcgen05 race features"));
+  } else if (g.r > 0) {
+    ELSAA_TRY(cuda_status(launch_race_features_f32((const float*)Q, (const float*)K, W, (float*)s.phiQ,
+                                                   (float*)s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, st_),
+                          "race features"));
+  }
+  // per-chunk bf16 hi/lo statistics for the tensor-core read-out and query-side backward (bf16),
+  // or the segment and in-segment prefixes the fp32 read-out combines
+  if (g.r > 0 && bf16)
+    ELSAA_TRY(cuda_status(launch_race_stats_tc(s.phiK, V, nullptr, false, s.Ast, s.Psplit, s.Pmass, g, w.flag, st_),
+                          "tcgen05 race statistics"));
+  else if (g.r > 0)
+    ELSAA_TRY(cuda_status(launch_race_state_fwd_f32((const float*)s.phiK, (const float*)V, s.Ast, s.Bst, g, st_),
+                          "race summaries"));
   FwdArgs a{Q, K, V, s.idx, s.phiQ, s.phiK, s.Ast, s.Bst, lam, gs, glr, O, s.Os, s.logd, s.dlr, s.m, s.Olr,
             s.Psplit, s.Pmass};
+  a.lr_num = w.lr_num;
+  a.lr_den = w.lr_den;
   bool scattered = false;
-  if (bf16 && attn_fwd_tc_supported(g) && !tcgen05_disabled()) {
-    if (s.Psplit) ELSAA_TRY(cuda_status(launch_race_readout_tc(a, g, w.flag, st_), "tcgen05 race read-out"));
-    else
-      ELSAA_TRY(cuda_status(launch_race_readout_bf16(a, g, st_), "race read-out"));
+  if (bf16) {
+    if (g.r > 0) {
+      ELSAA_TRY(cuda_status(launch_race_readout_tc(a, g, w.flag, st_), "tcgen05 race read-out"));
+    } else {                          // no low-rank branch: the fusion reads O_lr = 0, d_lr = 0
+      ELSAA_TRY(cuda_status(cudaMemsetAsync(s.Olr, 0, (size_t)g.BH * g.N * g.d * 2, st_), "O_lr"));
+      ELSAA_TRY(cuda_status(cudaMemsetAsync(s.dlr, 0, (size_t)g.BH * g.N * 4, st_), "d_lr"));
+    }
+    if (side) ELSAA_TRY(cuda_status(joined.join(), "selection join"));
     FwdArgs at = a;
     if (lsh) {                        // the epilogue writes O straight into the caller's row order
       at.O = O_out;
@@ -719,8 +816,6 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
       scattered = true;
     }
     ELSAA_TRY(cuda_status(launch_attn_fwd_tc(at, g, w.flag, st_), "tcgen05 forward"));
-  } else if (bf16) {
-    ELSAA_TRY(cuda_status(launch_attn_fwd_bf16(a, g, st_), "fused forward"));
   } else {
     ELSAA_TRY(cuda_status(launch_attn_fwd_f32(a, g, st_), "fused forward"));
   }
@@ -801,33 +896,32 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   bool scattered = false;
   ELSAA_TRY(cuda_status(cudaMemsetAsync(w.flag, 0, 4, st_), "flag reset"));
   ELSAA_TRY(cuda_status(launch_row_scalars(a, bf16, g, st_), "row scalars"));
-  ELSAA_TRY(cuda_status(launch_race_state_bwd(a, bf16, g, st_), "race suffix summaries"));
+  const bool race_tc = tc_race(g, bf16);
+  if (race_tc)
+    ELSAA_TRY(cuda_status(launch_race_stats_tc(a.phiQ, a.dOcl, w.rs.delta, true, w.RA, w.Rsplit, w.Rmass, g, w.flag,
+                                               st_),
+                          "tcgen05 race statistics"));
+  else if (!bf16)
+    ELSAA_TRY(cuda_status(launch_race_state_bwd_f32(a, g, st_), "race suffix summaries"));
   if (g.k > 0) ELSAA_TRY(cuda_status(launch_invert_selection(s.idx, w.offs, w.tiles, w.order, g, st_), "selection inverse"));
   if (bf16) {
-    const bool tc = bwd_tc_supported(g) && !tcgen05_disabled();
-    const bool race_tc = tc && g.r > 0 && race_bwd_tc_supported(g);
     BwdArgs at = a;
     if (g.r == 0) at.dQacc = at.dKacc = at.dVacc = nullptr;
     if (race_tc) {
-      ELSAA_TRY(cuda_status(launch_race_state_split(w.RA, w.RB, true, w.Rsplit, w.Rmass, g, st_),
-                            "race statistics split"));
       ELSAA_TRY(cuda_status(launch_race_w_split(W, w.Wsplit, g, st_), "W split"));
       ELSAA_TRY(cuda_status(launch_race_bwd_tc(a, g, w.flag, st_), "tcgen05 race backward"));
     }
-    ELSAA_TRY(cuda_status(launch_bwd_bf16(a, g, tc ? (race_tc ? 0 : 1) : 7, st_), "backward"));
-    if (tc) {
-      if (lsh) {                      // the epilogues write straight into the caller's row orders
-        at.dQ = dQ_out;
-        at.dK = dK_out;
-        at.dV = dV_out;
-        at.q_rows = s.lsh_order;
-        at.k_rows = s.lsh_order + g.N;
-        at.rows_stride = 2 * g.N;
-        scattered = true;
-      }
-      ELSAA_TRY(cuda_status(launch_dq_tc(at, g, w.flag, st_), "tcgen05 dq"));
-      ELSAA_TRY(cuda_status(launch_dkdv_tc(at, g, w.flag, st_), "tcgen05 dkdv"));
+    if (lsh) {                        // the epilogues write straight into the caller's row orders
+      at.dQ = dQ_out;
+      at.dK = dK_out;
+      at.dV = dV_out;
+      at.q_rows = s.lsh_order;
+      at.k_rows = s.lsh_order + g.N;
+      at.rows_stride = 2 * g.N;
+      scattered = true;
     }
+    ELSAA_TRY(cuda_status(launch_dq_tc(at, g, w.flag, st_), "tcgen05 dq"));
+    ELSAA_TRY(cuda_status(launch_dkdv_tc(at, g, w.flag, st_), "tcgen05 dkdv"));
   } else {
     ELSAA_TRY(cuda_status(launch_bwd_f32(a, g, st_), "backward"));
   }
@@ -905,6 +999,14 @@ elsaa_status elsaa_debug_sortlsh(const elsaa_params* p, const void* Q, const voi
   return cuda_status(launch_sortlsh_order(Q, K, p->dtype == ELSAA_DTYPE_BF16, p->lsh_planes, p->lsh_bits, order,
                                           codes, g, static_cast<cudaStream_t>(stream)),
                      "sortLSH order");
+}
+
+elsaa_status elsaa_debug_set_wait_limit(unsigned long long wait_ns, int stall) {
+  g_last_error.clear();
+  if (stall != 0 && stall != 1) return fail(ELSAA_ERR_INVALID_ARG, "stall must be 0 or 1");
+  g_wait_ns.store(wait_ns);
+  g_debug_stall.store(stall);
+  return ELSAA_OK;
 }
 
 elsaa_status elsaa_check_device_flags(void* workspace, void* stream) {

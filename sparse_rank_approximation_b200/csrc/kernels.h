@@ -24,8 +24,9 @@ struct FwdArgs {
   void *O, *Os;
   float *logd, *dlr, *m;
   void* Olr;      // O_lr saved for the backward
-  const void* Psplit;  // prefix statistics per chunk as bf16 hi/lo [BH][n_c][2][r][d] (tensor-core RACE path)
-  const float* Pmass;  // their key-mass column [BH][n_c][r]
+  const void* Psplit;  // prefix statistics per chunk as bf16 hi/lo [G][BH][n_c][2][128][d] (tensor-core RACE
+                       // path; one block per group of 128 features)
+  const float* Pmass;  // their key-mass column [G][BH][n_c][128]
   // optional: the query tiles to run, n_list per head ([BH][n_list]); null runs all tiles
   const int* tile_list;
   int n_list;
@@ -33,6 +34,9 @@ struct FwdArgs {
   // of the caller's O instead of row r (the sortLSH orders); O_s stays in row order
   const int* q_rows;
   int rows_stride;
+  // tensor-core read-out over several feature groups: the running numerator (fp32 [BH][N][d])
+  // and denominator ([BH][N]) between the groups' launches
+  float *lr_num, *lr_den;
 };
 
 // Per-row adjoint scalars of the fusion (Eq. 4 / Eq. 5), float32 [BH, N] each.
@@ -60,8 +64,8 @@ struct BwdArgs {
   RowScalars rs;
   float *dQacc, *dKacc, *dVacc;  // fp32 low-rank gradient parts (bf16 path)
   void* dOcl;                    // cl dO rows (bf16 path), written by the row scalars
-  const void* Psplit;            // prefix statistics per chunk, bf16 hi/lo [BH][n_c][2][r][d] (tensor-core RACE)
-  const float* Pmass;            //   key-mass column [BH][n_c][r]
+  const void* Psplit;            // prefix statistics per chunk, bf16 hi/lo [G][BH][n_c][2][128][d] (tensor-core RACE)
+  const float* Pmass;            //   key-mass column [G][BH][n_c][128]
   const void* Rsplit;            // suffix statistics per chunk, same layout
   const float* Rmass;
   const void* Wsplit;            // W as bf16 hi/lo rows n = 4 l + b, [2][NW][d]
@@ -75,6 +79,9 @@ struct BwdArgs {
   // dV row r to row k_rows[bh * rows_stride + r] of the caller's outputs (the sortLSH orders)
   const int *q_rows, *k_rows;
   int rows_stride;
+  // optional (sparse kernels, no row maps): write dQ, dK, dV as fp32 rows instead of bf16 (the
+  // causal sortLSH recursion's level slots, summed before the single bf16 rounding)
+  int out_f32;
 };
 
 // sortLSH selector: per head the sorted query and key orders, int32 [BH][2][N]
@@ -120,27 +127,37 @@ cudaError_t launch_select(const void* Q, const void* K, bool bf16, double* qbar,
                           int* idx, const Geom& g, cudaStream_t st);
 cudaError_t launch_invert_selection(const int* idx, int* offs, int* tiles, int* order, const Geom& g,
                                     cudaStream_t st);
-// wsplit: scratch bf16 [2][NW][d] (NW = 4L rounded up to 16) that receives W split into hi and lo halves.
-cudaError_t launch_race_features(const void* Q, const void* K, const float* W, void* wsplit, bool bf16, void* phiQ,
-                                 void* phiK, float* hQ, float* hK, float* nQ, float* nK, const Geom& g,
-                                 cudaStream_t st);
-// Forward prefix statistics (Ast: per-segment exclusive prefix, Bst: in-segment prefix).
-cudaError_t launch_race_state_fwd(const void* phiK, const void* V, bool bf16, float* Ast, float* Bst,
-                                  const Geom& g, cudaStream_t st);
-// Per-chunk statistics A[slot] + B[c] as bf16 hi/lo [BH][n_c][2][r][d] plus the key-mass column
-// [BH][n_c][r] (forward prefix when !bwd, backward suffix when bwd).
-cudaError_t launch_race_state_split(const float* A, const float* B, bool bwd, void* out, float* mass, const Geom& g,
-                                    cudaStream_t st);
-// W[l][d][4] -> bf16 hi/lo rows n = 4 l + b, [2][NW][d] with NW = 4L rounded up to 16.
+// fp32 path: RACE features and the chunked prefix / suffix summaries (SIMT).
+cudaError_t launch_race_features_f32(const float* Q, const float* K, const float* W, float* phiQ, float* phiK,
+                                     float* hQ, float* hK, float* nQ, float* nK, const Geom& g, cudaStream_t st);
+cudaError_t launch_race_state_fwd_f32(const float* phiK, const float* V, float* Ast, float* Bst, const Geom& g,
+                                      cudaStream_t st);
+cudaError_t launch_race_state_bwd_f32(const BwdArgs& a, const Geom& g, cudaStream_t st);
+// In place over the segment totals [BH][n_seg + 1][rows][dp] (total of segment s in slot s + 1):
+// forward, slot s becomes the exclusive prefix of the segments before s and slot n_seg the
+// grand total; backward, slot s + 1 the exclusive suffix of the segments after s and slot 0
+// the grand total.
+cudaError_t launch_race_scan(float* Atot, int rows, bool bwd, const Geom& g, cudaStream_t st);
+// RACE chunk statistics on the tensor cores (d = 64 or 128, chunks of 128 rows, features in groups
+// of 128): segment totals in tensor memory, the scan, then every chunk's exclusive prefix
+// (forward: Phi = Phi(K), Y = V, w = null for 1) or suffix (backward: Phi = Phi(Q), Y = cl dO,
+// w = delta) written as bf16 hi/lo [G][BH][n_c][2][128][d] with its fp32 mass [G][BH][n_c][128].
+// Atot is fp32 scratch [BH][n_seg + 1][128][dp], reused by the groups.
+bool race_stats_tc_supported(const Geom& g);
+cudaError_t launch_race_stats_tc(const void* phi, const void* Y, const float* w, bool bwd, float* Atot, void* out,
+                                 float* mass, const Geom& g, uint32_t* err, cudaStream_t st);
+// W[l][d][4] -> bf16 hi/lo rows n = 4 l + b, [2][NW][d] with NW = 4L rounded up to 32.
 cudaError_t launch_race_w_split(const float* W, void* out, const Geom& g, cudaStream_t st);
-// Backward suffix statistics of Phi(q_i) [cl_i dO_i ; delta_i]^T.
-cudaError_t launch_race_state_bwd(const BwdArgs& a, bool bf16, const Geom& g, cudaStream_t st);
-cudaError_t launch_attn_fwd_bf16(const FwdArgs& a, const Geom& g, cudaStream_t st);
-// tcgen05 sparse-branch forward + fusion epilogue (d = 128, block 128); reads the
-// low-rank output written by launch_race_readout_bf16.
+// RACE features on the tensor cores (bf16, d = 64 or 128, L <= 16): Phi (bf16 [BH][N][rp], zero
+// padded), the normalised projections h (fp32 [BH][N][4L]) and the row norms; wsplit is the W
+// split written by launch_race_w_split.
+cudaError_t launch_race_features_tc(const void* Q, const void* K, const void* wsplit, void* phiQ, void* phiK,
+                                    float* hQ, float* hK, float* nQ, float* nK, const Geom& g, uint32_t* err,
+                                    cudaStream_t st);
+// tcgen05 sparse-branch forward + fusion epilogue (d = 64 or 128, blocks of 64 or 128 keys);
+// reads the low-rank output written by launch_race_readout_tc (zeros without a low-rank branch).
 bool attn_fwd_tc_supported(const Geom& g);
 cudaError_t launch_attn_fwd_tc(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
-cudaError_t launch_race_readout_bf16(const FwdArgs& a, const Geom& g, cudaStream_t st);
 // tcgen05 RACE read-out (same shapes as race_bwd_tc_supported): O_lr (bf16) and d_lr.
 cudaError_t launch_race_readout_tc(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
 cudaError_t launch_attn_fwd_f32(const FwdArgs& a, const Geom& g, cudaStream_t st);
@@ -152,19 +169,16 @@ cudaError_t launch_fusion_grads(const void* dO, const void* Os, const void* Olr,
                                 const float* lam, const float* gs, const float* glr, float* dlam, float* dgs,
                                 float* dglr, const int* perm, int perm_stride, bool bf16, const Geom& g,
                                 cudaStream_t st);
-// RACE backward (bf16): low-rank parts of dQ, dK, dV into the fp32 accumulators.
-cudaError_t launch_race_bwd_bf16(const BwdArgs& a, const Geom& g, cudaStream_t st);
-// tcgen05 sparse-branch backward (d = 128, block 128): dQ (query-major) and dK/dV
-// (key-major through the selection inverse), adding the low-rank accumulators.
+// tcgen05 sparse-branch backward (d = 64 or 128, blocks of 64 or 128 keys): dQ (query-major) and
+// dK/dV (key-major through the selection inverse), adding the low-rank accumulators.
 bool bwd_tc_supported(const Geom& g);
-// tcgen05 RACE backward (d = 128, chunk 128, r = 128): low-rank parts of dQ, dK, dV
-// into the fp32 accumulators; needs the saved projections and row norms.
+// tcgen05 RACE backward (d = 64 or 128, chunks of 128 rows, r <= 256 in groups of 128 features):
+// low-rank parts of dQ, dK, dV into the fp32 accumulators; needs the saved projections and
+// row norms.
 bool race_bwd_tc_supported(const Geom& g);
 cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
 cudaError_t launch_dq_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
 cudaError_t launch_dkdv_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st);
-// parts: bit 0 RACE backward, bit 1 sparse dQ, bit 2 sparse dK/dV (mma.sync kernels).
-cudaError_t launch_bwd_bf16(const BwdArgs& a, const Geom& g, int parts, cudaStream_t st);
 cudaError_t launch_bwd_f32(const BwdArgs& a, const Geom& g, cudaStream_t st);
 
 }  // namespace elsaa

@@ -14,6 +14,8 @@
 // so calls whose work overlaps on the GPU (different streams, or different host
 // threads on the same device) race; serialise them.  Nothing in it needs to
 // start at zero: the kernels write every entry they later read.
+#include <cuda.h>
+
 #include <mutex>
 #include <string>
 
@@ -29,6 +31,25 @@ static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchB
 
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};   // the context each cached address belongs to
+
+// The current driver context, or null when it cannot be read.  A device reset or a
+// different (non-primary) context on the same ordinal loads the module again, at a
+// new address, so the cached address is only reused under the context it came from.
+CUcontext current_context() {
+  using Fn = CUresult (*)(CUcontext*);
+  static Fn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<Fn>(p);
+  }
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
 
 elsaa_status noalloc_fail(elsaa_status s, const std::string& msg) {
   elsaa::record_error(msg.c_str());   // read back with elsaa_last_error_message()
@@ -71,20 +92,23 @@ elsaa_status elsaa_select_noalloc(const elsaa_params* p, const void* Q, const vo
                         "selection needs " + std::to_string(need) + " bytes of scratch; the static scratch holds " +
                             std::to_string(kNoAllocScratchBytes) + " (B*H*ceil(N/block)*(16*d + 4*ceil(N/block)))");
 
-  // One-time set-up per device (with that device current): the host-side name of
-  // the array is not a device address, so resolve the address once and cache it.
+  // One-time set-up per device and context (with that device current): the host-side
+  // name of the array is not a device address, so resolve the address and cache it.
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return noalloc_fail(ELSAA_ERR_CUDA, "cudaGetDevice failed or device ordinal out of range");
+  const CUcontext ctx = current_context();
   char* base = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
+    if (!g_scratch_ptr[dev] || !ctx || g_scratch_ctx[dev] != ctx) {
       void* ptr = nullptr;
       const cudaError_t e = cudaGetSymbolAddress(&ptr, g_select_scratch);
       if (e != cudaSuccess || !ptr)
         return noalloc_fail(ELSAA_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
       g_scratch_ptr[dev] = ptr;
+      // with the context unknown the address is resolved again on every call
+      g_scratch_ctx[dev] = ctx;
     }
     base = static_cast<char*>(g_scratch_ptr[dev]);
   }

@@ -1,5 +1,8 @@
 // RACE low-rank branch (ELSAA paper §3.1) read-out and backward on the 5th-generation
-// tensor cores, for d = 128, chunk C = 128 and r = 128 (L = 8 tables of 16 corners).
+// tensor cores, for d = 128 and chunk C = 128, over the features in groups of 128 (8 tables of
+// 16 corners; r up to 256, zero-padded to whole groups).  Each group is one launch; the read-out
+// carries its running numerator and denominator from the first group to the last, the backward
+// kernels add the later groups' parts to the fp32 accumulators.
 // One CTA per (head, chunk of 128 rows); every accumulator lives in tensor memory.
 //
 // Read-out, chunk t (query rows i):
@@ -34,7 +37,7 @@ namespace elsaa {
 namespace {
 
 constexpr int kC = 128;
-constexpr int kD = 128;
+constexpr int kD = 128;                          // widest head dimension: operand slots are sized for it
 constexpr int kR = 128;
 constexpr int kNH = 32;                          // projection columns 4 L
 constexpr uint32_t kSlab = 128 * 128;            // [128 rows][64 bf16], 128-byte swizzle
@@ -113,21 +116,28 @@ __device__ __forceinline__ void corner_bwd(const float (&h)[4], const float (&dp
 // (fp32, 64 TMEM columns from `dphi_col`, plus the optional `cl * G + de * m1`
 // terms), projections h (global, fp32), then dh as bf16 hi / lo into TMEM columns
 // 8 hc (hi) and 16 + 8 hc (lo).
-__device__ __forceinline__ void load_h(const float* __restrict__ hrow, int hc, float (&h16)[16]) {
+// The projections of this thread's 4 tables (tables 8 grp + 4 hc .. + 3 of a row whose 4 L
+// projections start at hrow); tables past the last one (padding of the group) read as zero.
+__device__ __forceinline__ void load_h(const float* __restrict__ hrow, int grp, int hc, int L, float (&h16)[16]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const float4 v = hrow ? __ldg(reinterpret_cast<const float4*>(hrow + 16 * hc) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int table = 8 * grp + 4 * hc + q;
+    const float4 v = hrow && table < L ? __ldg(reinterpret_cast<const float4*>(hrow) + table)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
     h16[4 * q] = v.x; h16[4 * q + 1] = v.y; h16[4 * q + 2] = v.z; h16[4 * q + 3] = v.w;
   }
 }
-// Row `row` of a [128][128] bf16 tile that TMA wrote as two 64-column slabs with the
-// 128-byte swizzle: this thread's half (columns 64 hc .. 64 hc + 63) as 8 x 16 bytes.  Eight
+// Row `row` of a [128][D] bf16 tile that TMA wrote as 64-column slabs with the 128-byte
+// swizzle: this thread's half (columns D/2 hc .. D/2 hc + D/2 - 1) as D/16 x 16 bytes.  Eight
 // consecutive rows read eight different 16-byte positions, so a warp's reads do not conflict.
-__device__ __forceinline__ void load_x(const unsigned char* tile, int row, int hc, bool valid, uint4 (&xr)[8]) {
-  const unsigned char* base = tile + (uint32_t)hc * kSlab + (uint32_t)row * 128u;
+template <int D>
+__device__ __forceinline__ void load_x(const unsigned char* tile, int row, int hc, bool valid, uint4 (&xr)[D / 16]) {
+  const int c0 = (D / 2) * hc;                      // first column of this half
+  const unsigned char* base = tile + (uint32_t)(c0 >> 6) * kSlab + (uint32_t)row * 128u;
 #pragma unroll
-  for (int q = 0; q < 8; ++q)
-    xr[q] = valid ? *reinterpret_cast<const uint4*>(base + ((q ^ (row & 7)) << 4)) : make_uint4(0u, 0u, 0u, 0u);
+  for (int q = 0; q < D / 16; ++q)
+    xr[q] = valid ? *reinterpret_cast<const uint4*>(base + (((((c0 & 63) >> 3) + q) ^ (row & 7)) << 4))
+                  : make_uint4(0u, 0u, 0u, 0u);
 }
 
 __device__ __forceinline__ void corner_pass(uint32_t tmem, uint32_t lane_base, int hc, uint32_t dphi_col,
@@ -161,9 +171,10 @@ __device__ __forceinline__ void corner_pass(uint32_t tmem, uint32_t lane_base, i
   tc::tmem_st8(tmem + lane_base + 16u + 8u * hc, lo);
 }
 
-// du = dh W^T: three products (hi hi, hi lo, lo hi), K = 32 (two steps each).
+// du = dh W^T: three products (hi hi, hi lo, lo hi), K = 32 (two steps each), N = D.
+template <int D>
 __device__ __forceinline__ void issue_du(uint32_t tmem, uint32_t d_col, uint32_t sb, uint32_t w_hi, uint32_t w_lo) {
-  const uint32_t idG = tc::idesc_bf16(128, kD, false, true);
+  const uint32_t idG = tc::idesc_bf16(128, D, false, true);
 #pragma unroll
   for (int part = 0; part < 3; ++part) {
     const uint32_t a_col = part == 2 ? 16u : 0u;
@@ -179,15 +190,23 @@ __device__ __forceinline__ void issue_du(uint32_t tmem, uint32_t d_col, uint32_t
 // kD + 4 floats, so the 16-byte stores of 8 consecutive rows hit 8 different bank groups),
 // then all compute threads copy the [128][kD] tile out with coalesced 16-byte stores.  The
 // staging area reuses operand tiles that no product reads any more.
-constexpr int kStagePitch = kD + 4;
-constexpr uint32_t kStageBytes = (uint32_t)kC * kStagePitch * 4;
+template <int D> constexpr int stage_pitch() { return D + 4; }
+template <int D> constexpr uint32_t stage_bytes() { return (uint32_t)kC * stage_pitch<D>() * 4; }
 
-__device__ __forceinline__ void copy_staged(const float* stage, float* __restrict__ out, int rows, int ct) {
-  for (int idx = ct; idx < kC * (kD / 4); idx += kComputeThreads) {
-    const int r = idx / (kD / 4), c4 = idx % (kD / 4);
-    if (r < rows)
-      reinterpret_cast<float4*>(out + (size_t)r * kD)[c4] =
-          *reinterpret_cast<const float4*>(stage + r * kStagePitch + 4 * c4);
+// `add`: the feature groups after the first add their part to what the earlier ones wrote.
+template <int D>
+__device__ __forceinline__ void copy_staged(const float* stage, float* __restrict__ out, int rows, int ct, bool add) {
+  for (int idx = ct; idx < kC * (D / 4); idx += kComputeThreads) {
+    const int r = idx / (D / 4), c4 = idx % (D / 4);
+    if (r < rows) {
+      float4 v = *reinterpret_cast<const float4*>(stage + r * stage_pitch<D>() + 4 * c4);
+      float4* o = reinterpret_cast<float4*>(out + (size_t)r * D) + c4;
+      if (add) {
+        const float4 p = *o;
+        v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
+      }
+      *o = v;
+    }
   }
 }
 
@@ -195,23 +214,26 @@ __device__ __forceinline__ void copy_staged(const float* stage, float* __restric
 // column halves of a row meet through `xch`.  Stores fp32 into out (row pointer).
 // Every compute thread calls this (the exchange barrier); `alive` false skips the
 // tensor-memory reads and the stores.
+template <int D>
 __device__ __forceinline__ void chain_pass(uint32_t tmem, uint32_t lane_base, int hc, int row_in_chunk,
-                                           uint32_t du_col, const uint4 (&xr)[8], float n, float* xch,
+                                           uint32_t du_col, const uint4 (&xr)[D / 16], float n, float* xch,
                                            float* stage, bool valid, bool alive) {
-  float du[64];
+  constexpr int H = D / 2;                          // this thread's columns
+  float du[H];
   if (alive) {
     tc::tc_fence_after();
-    tc::tmem_ld32(tmem + lane_base + du_col + 64u * hc, *reinterpret_cast<float(*)[32]>(du));
-    tc::tmem_ld32(tmem + lane_base + du_col + 64u * hc + 32u, *reinterpret_cast<float(*)[32]>(du + 32));
+#pragma unroll
+    for (int h2 = 0; h2 < H / 32; ++h2)
+      tc::tmem_ld32(tmem + lane_base + du_col + H * hc + 32u * h2, *reinterpret_cast<float(*)[32]>(du + 32 * h2));
   } else {
 #pragma unroll
-    for (int q = 0; q < 64; ++q) du[q] = 0.f;
+    for (int q = 0; q < H; ++q) du[q] = 0.f;
   }
   valid = valid && alive;
   if (alive) tc::tmem_wait_ld();
   float xd = 0.f;
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
+  for (int q = 0; q < D / 16; ++q) {
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&xr[q]);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -226,9 +248,9 @@ __device__ __forceinline__ void chain_pass(uint32_t tmem, uint32_t lane_base, in
   if (!valid) return;
   const float proj = n <= kNormFloor ? 0.f : xd / (n * n);
   const float inv = 1.f / n;
-  float4* o = reinterpret_cast<float4*>(stage + row_in_chunk * kStagePitch + 64 * hc);
+  float4* o = reinterpret_cast<float4*>(stage + row_in_chunk * stage_pitch<D>() + H * hc);
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
+  for (int q = 0; q < D / 16; ++q) {
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&xr[q]);
     const float2 x0 = __bfloat1622float2(p[0]), x1 = __bfloat1622float2(p[1]);
     const float2 x2 = __bfloat1622float2(p[2]), x3 = __bfloat1622float2(p[3]);
@@ -247,18 +269,21 @@ constexpr uint32_t K_BARS = K_CL + (3 * 128 + 256) * 4;
 // TMEM columns
 constexpr uint32_t TK_KAP = 0, TK_X = 128, TK_DV = 256, TK_DPHI = 384, TK_DU = 128;
 // staged dV and dK rows, over the operand tiles once every product that reads them is done
-constexpr uint32_t K_STAGE_V = 0, K_STAGE_K = (kStageBytes + 1023u) & ~1023u;
+constexpr uint32_t K_STAGE_V = 0;
+template <int D> constexpr uint32_t k_stage_k() { return (stage_bytes<D>() + 1023u) & ~1023u; }
 // the K rows of the chunk for dx, over the statistics tiles once their products are done
-constexpr uint32_t K_XS = (K_STAGE_K + kStageBytes + 1023u) & ~1023u;
-static_assert(K_XS + kTile <= K_WH, "the staged rows and the K tile overlap only the chunk tiles");
+template <int D> constexpr uint32_t k_xs() { return (k_stage_k<D>() + stage_bytes<D>() + 1023u) & ~1023u; }
+static_assert(k_xs<128>() + kTile <= K_WH && k_xs<64>() + kTile <= K_WH,
+              "the staged rows and the K tile overlap only the chunk tiles");
 
 }  // namespace
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     race_k_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmPQ,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                          const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmW,
-                         const __grid_constant__ CUtensorMap tmX, BwdArgs a, Geom g, uint32_t* err) {
+                         const __grid_constant__ CUtensorMap tmX, BwdArgs a, Geom g, int grp, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   Bars* ms = reinterpret_cast<Bars*>(smem + K_BARS);
   float* sCl = reinterpret_cast<float*>(smem + K_CL);
@@ -295,27 +320,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 6 : 4) * kTile + 4 * kWSlab);
+      // Phi tiles are [128][128]; V, dO, the statistics and W are D columns wide
+      constexpr uint32_t kTD = 128u * D * 2, kWD = (uint32_t)kNH * D * 2;
+      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 2 : 1) * kTile + (causal ? 2 : 1) * kTD + 2 * kTD + 2 * kWD);
       const int z = (bh * g.n_c + c) * 2;
       for (int s = 0; s < 2; ++s) {
         tc::tma_load_3d(smem + K_PK + s * kSlab, &tmPK, &ms->in_main, 64 * s, c * kC, bh);
+        if (causal) tc::tma_load_3d(smem + K_PQ + s * kSlab, &tmPQ, &ms->in_main, 64 * s, c * kC, bh);
+      }
+      for (int s = 0; s < D / 64; ++s) {
         tc::tma_load_3d(smem + K_V + s * kSlab, &tmV, &ms->in_main, 64 * s, c * kC, bh);
-        if (causal) {
-          tc::tma_load_3d(smem + K_PQ + s * kSlab, &tmPQ, &ms->in_main, 64 * s, c * kC, bh);
-          tc::tma_load_3d(smem + K_DO + s * kSlab, &tmdO, &ms->in_main, 64 * s, c * kC, bh);
-        }
+        if (causal) tc::tma_load_3d(smem + K_DO + s * kSlab, &tmdO, &ms->in_main, 64 * s, c * kC, bh);
         tc::tma_load_3d(smem + K_RH + s * kSlab, &tmR, &ms->in_main, 64 * s, 0, z);
         tc::tma_load_3d(smem + K_RL + s * kSlab, &tmR, &ms->in_main, 64 * s, 0, z + 1);
-        tc::tma_load_3d(smem + K_WH + s * kWSlab, &tmW, &ms->in_main, 64 * s, 0, 0);
-        tc::tma_load_3d(smem + K_WL + s * kWSlab, &tmW, &ms->in_main, 64 * s, 0, 1);
+        tc::tma_load_3d(smem + K_WH + s * kWSlab, &tmW, &ms->in_main, 64 * s, kNH * grp, 0);
+        tc::tma_load_3d(smem + K_WL + s * kWSlab, &tmW, &ms->in_main, 64 * s, kNH * grp, 1);
       }
       tc::mbar_wait(&ms->in_main, 0);
       // the K rows for dx, once every product but du has read the chunk tiles; waited for
       // here too, so no copy is in flight when the CTA exits
       if (wait_or_abort(&ms->acc_full, 0, ms, err, 0x10000u)) {
-        tc::mbar_arrive_expect_tx(&ms->x_full, kTile);
-        tc::tma_load_3d(smem + K_XS, &tmX, &ms->x_full, 0, c * kC, bh);
-        tc::tma_load_3d(smem + K_XS + kSlab, &tmX, &ms->x_full, 64, c * kC, bh);
+        tc::mbar_arrive_expect_tx(&ms->x_full, kTD);
+        for (int s = 0; s < D / 64; ++s)
+          tc::tma_load_3d(smem + k_xs<D>() + s * kSlab, &tmX, &ms->x_full, 64 * s, c * kC, bh);
         wait_or_abort(&ms->x_full, 0, ms, err, 0x20000u);
       }
     }
@@ -323,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);
       const uint32_t idNM = tc::idesc_bf16(128, 128, false, true);
+      const uint32_t idDM = tc::idesc_bf16(128, D, false, true);     // N = D, B MN-major
       const uint32_t sb = smem_u32(smem);
       bool ok = wait_or_abort(&ms->in_main, 0, ms, err, 0x100u);
       if (ok && causal) {
@@ -330,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 8; ++kk)
           tc::mma_bf16(tmem + TK_KAP, desc_k(sb + K_PK, kk), desc_k(sb + K_PQ, kk), idNN, kk > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < D / 16; ++kk)
           tc::mma_bf16(tmem + TK_X, desc_k(sb + K_V, kk), desc_k(sb + K_DO, kk), idNN, kk > 0 ? 1u : 0u);
         tc::mma_commit(&ms->s_full);
       }
@@ -341,10 +369,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t rb = sb + (part ? K_RL : K_RH);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_bf16(tmem + TK_DV, desc_k(sb + K_PK, kk), desc_mn(rb, kk, kSlab), idNM,
+            tc::mma_bf16(tmem + TK_DV, desc_k(sb + K_PK, kk), desc_mn(rb, kk, kSlab), idDM,
                          (part > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
+          for (int kk = 0; kk < D / 16; ++kk)
             tc::mma_bf16(tmem + TK_DPHI, desc_k(sb + K_V, kk), desc_k(rb, kk), idNN, (part > 0 || kk > 0) ? 1u : 0u);
         }
       }
@@ -355,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // intra-chunk parts, A operands from tensor memory
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_bf16_ts(tmem + TK_DV, tmem + TK_KAP + packed_col(kk), desc_mn(sb + K_DO, kk, kSlab), idNM, 1u);
+            tc::mma_bf16_ts(tmem + TK_DV, tmem + TK_KAP + packed_col(kk), desc_mn(sb + K_DO, kk, kSlab), idDM, 1u);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             tc::mma_bf16_ts(tmem + TK_DPHI, tmem + TK_X + packed_col(kk), desc_mn(sb + K_PQ, kk, kSlab), idNM, 1u);
@@ -365,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = ok && wait_or_abort(&ms->dh_full, 0, ms, err, 0x800u);
       if (ok) {
         tc::tc_fence_after();
-        issue_du(tmem, TK_DU, sb, K_WH, K_WL);
+        issue_du<D>(tmem, TK_DU, sb, K_WH, K_WL);
       }
       tc::mma_commit(&ms->du_full);
       tc::mbar_wait(&ms->du_full, 0);
@@ -378,17 +406,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = c * kC + j;
     const bool valid = row < g.N;
     float* stage_v = reinterpret_cast<float*>(smem + K_STAGE_V);
-    float* stage_k = reinterpret_cast<float*>(smem + K_STAGE_K);
+    float* stage_k = reinterpret_cast<float*>(smem + k_stage_k<D>());
     // row data for the corner and chain passes, fetched up front
     float h16[16];
-    load_h(valid ? a.hK + (head + row) * kNH : nullptr, hc, h16);
+    load_h(valid ? a.hK + (head + row) * 4 * g.L : nullptr, grp, hc, g.L, h16);
     const float nrm = valid ? a.nK[head + row] : 1.f;
     // ---- per-row scalars of the chunk and the key-mass column of the suffix statistics ----
     if (ct < kC) {
       const int r = c * kC + ct;
       sCl[ct] = r < g.N ? a.rs.cl[head + r] : 0.f;
       sDl[ct] = r < g.N ? a.rs.delta[head + r] : 0.f;
-      sR1[ct] = a.Rmass[((size_t)bh * g.n_c + c) * kR + ct];
+      sR1[ct] = a.Rmass[(((size_t)grp * g.BH + bh) * g.n_c + c) * kR + ct];
     }
     compute_bar();
     bool alive = true;
@@ -431,12 +459,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (alive) {
       tc::tc_fence_after();
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      for (int h2 = 0; h2 < D / 64; ++h2) {
         float v[32];
-        tc::tmem_ld32(tmem + lane_base + TK_DV + 64 * hc + 32 * h2, v);
+        tc::tmem_ld32(tmem + lane_base + TK_DV + (D / 2) * hc + 32 * h2, v);
         tc::tmem_wait_ld();
         // every product has read the operand tiles: dV rows are staged over them
-        float4* o = reinterpret_cast<float4*>(stage_v + j * kStagePitch + 64 * hc + 32 * h2);
+        float4* o = reinterpret_cast<float4*>(stage_v + j * stage_pitch<D>() + (D / 2) * hc + 32 * h2);
 #pragma unroll
         for (int q = 0; q < 8; ++q) o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
       }
@@ -446,16 +474,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_before();
       tc::mbar_arrive(&ms->dh_full);
     }
-    uint4 xr[8];
+    uint4 xr[D / 16];
     if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->x_full, 0, ms, err, 0x40000u));
-    load_x(smem + K_XS, j, hc, valid && alive, xr);
+    load_x<D>(smem + k_xs<D>(), j, hc, valid && alive, xr);
     if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->du_full, 0, ms, err, 0x4000u));
-    chain_pass(tmem, lane_base, hc, j, TK_DU, xr, nrm, sX, stage_k, valid, alive);
+    chain_pass<D>(tmem, lane_base, hc, j, TK_DU, xr, nrm, sX, stage_k, valid, alive);
     compute_bar();
     if (!*(volatile int*)&ms->abort_flag) {
       const int rows = min(kC, g.N - c * kC);
-      copy_staged(stage_v, a.dVacc + (head + (size_t)c * kC) * kD, rows, ct);
-      copy_staged(stage_k, a.dKacc + (head + (size_t)c * kC) * kD, rows, ct);
+      copy_staged<D>(stage_v, a.dVacc + (head + (size_t)c * kC) * D, rows, ct, grp > 0);
+      copy_staged<D>(stage_k, a.dKacc + (head + (size_t)c * kC) * D, rows, ct, grp > 0);
     }
   }
   __syncthreads();
@@ -472,16 +500,18 @@ constexpr uint32_t Q_WH = 5 * kTile, Q_WL = Q_WH + 2 * kWSlab;
 constexpr uint32_t Q_P1 = Q_WL + 2 * kWSlab;            // p1 [128], exchange [256]
 constexpr uint32_t Q_BARS = Q_P1 + (128 + 256) * 4;
 // the Q rows of the chunk for dx, after the staged dQ rows
-constexpr uint32_t Q_XS = (Q_DO + kStageBytes + 1023u) & ~1023u;
-static_assert(Q_XS + kTile <= Q_WH, "the staged dQ rows and the Q tile overlap only the chunk tiles");
+template <int D> constexpr uint32_t q_xs() { return (Q_DO + stage_bytes<D>() + 1023u) & ~1023u; }
+static_assert(q_xs<128>() + kTile <= Q_WH && q_xs<64>() + kTile <= Q_WH,
+              "the staged dQ rows and the Q tile overlap only the chunk tiles");
 constexpr uint32_t TQ_X = 0, TQ_INTRA = 128, TQ_G = 256, TQ_DU = 384;
 }  // namespace
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     race_q_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmdO, const __grid_constant__ CUtensorMap tmV,
                          const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmP,
                          const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                         BwdArgs a, Geom g, uint32_t* err) {
+                         BwdArgs a, Geom g, int grp, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   Bars* ms = reinterpret_cast<Bars*>(smem + Q_BARS);
   float* sP1 = reinterpret_cast<float*>(smem + Q_P1);
@@ -516,26 +546,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 5 : 3) * kTile + 4 * kWSlab);
+      // Phi(K) is [128][128]; dO, V, the statistics and W are D columns wide
+      constexpr uint32_t kTD = 128u * D * 2, kWD = (uint32_t)kNH * D * 2;
+      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? kTile + 2 * kTD : kTD) + 2 * kTD + 2 * kWD);
       const int z = (bh * g.n_c + t) * 2;
-      for (int s = 0; s < 2; ++s) {
+      if (causal)
+        for (int s = 0; s < 2; ++s) tc::tma_load_3d(smem + Q_PK + s * kSlab, &tmPK, &ms->in_main, 64 * s, t * kC, bh);
+      for (int s = 0; s < D / 64; ++s) {
         tc::tma_load_3d(smem + Q_DO + s * kSlab, &tmdO, &ms->in_main, 64 * s, t * kC, bh);
-        if (causal) {
-          tc::tma_load_3d(smem + Q_V + s * kSlab, &tmV, &ms->in_main, 64 * s, t * kC, bh);
-          tc::tma_load_3d(smem + Q_PK + s * kSlab, &tmPK, &ms->in_main, 64 * s, t * kC, bh);
-        }
+        if (causal) tc::tma_load_3d(smem + Q_V + s * kSlab, &tmV, &ms->in_main, 64 * s, t * kC, bh);
         tc::tma_load_3d(smem + Q_PH + s * kSlab, &tmP, &ms->in_main, 64 * s, 0, z);
         tc::tma_load_3d(smem + Q_PL + s * kSlab, &tmP, &ms->in_main, 64 * s, 0, z + 1);
-        tc::tma_load_3d(smem + Q_WH + s * kWSlab, &tmW, &ms->in_main, 64 * s, 0, 0);
-        tc::tma_load_3d(smem + Q_WL + s * kWSlab, &tmW, &ms->in_main, 64 * s, 0, 1);
+        tc::tma_load_3d(smem + Q_WH + s * kWSlab, &tmW, &ms->in_main, 64 * s, kNH * grp, 0);
+        tc::tma_load_3d(smem + Q_WL + s * kWSlab, &tmW, &ms->in_main, 64 * s, kNH * grp, 1);
       }
       tc::mbar_wait(&ms->in_main, 0);
       // the Q rows for dx, once every product but du has read the chunk tiles; waited for
       // here too, so no copy is in flight when the CTA exits
       if (wait_or_abort(&ms->acc_full, 0, ms, err, 0x10000u)) {
-        tc::mbar_arrive_expect_tx(&ms->x_full, kTile);
-        tc::tma_load_3d(smem + Q_XS, &tmX, &ms->x_full, 0, t * kC, bh);
-        tc::tma_load_3d(smem + Q_XS + kSlab, &tmX, &ms->x_full, 64, t * kC, bh);
+        tc::mbar_arrive_expect_tx(&ms->x_full, kTD);
+        for (int s = 0; s < D / 64; ++s)
+          tc::tma_load_3d(smem + q_xs<D>() + s * kSlab, &tmX, &ms->x_full, 64 * s, t * kC, bh);
         wait_or_abort(&ms->x_full, 0, ms, err, 0x20000u);
       }
     }
@@ -547,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = wait_or_abort(&ms->in_main, 0, ms, err, 0x100u);
       if (ok && causal) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < D / 16; ++kk)
           tc::mma_bf16(tmem + TQ_X, desc_k(sb + Q_DO, kk), desc_k(sb + Q_V, kk), idNN, kk > 0 ? 1u : 0u);
         tc::mma_commit(&ms->s_full);
       }
@@ -557,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int part = 0; part < 2; ++part) {
           const uint32_t pb = sb + (part ? Q_PL : Q_PH);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
+          for (int kk = 0; kk < D / 16; ++kk)
             tc::mma_bf16(tmem + TQ_G, desc_k(sb + Q_DO, kk), desc_k(pb, kk), idNN, (part > 0 || kk > 0) ? 1u : 0u);
         }
       }
@@ -575,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = ok && wait_or_abort(&ms->dh_full, 0, ms, err, 0x800u);
       if (ok) {
         tc::tc_fence_after();
-        issue_du(tmem, TQ_DU, sb, Q_WH, Q_WL);
+        issue_du<D>(tmem, TQ_DU, sb, Q_WH, Q_WL);
       }
       tc::mma_commit(&ms->du_full);
       tc::mbar_wait(&ms->du_full, 0);
@@ -590,9 +621,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float cl = valid ? a.rs.cl[head + row] : 0.f;
     const float de = valid ? a.rs.delta[head + row] : 0.f;
     float h16[16];
-    load_h(valid ? a.hQ + (head + row) * kNH : nullptr, hc, h16);
+    load_h(valid ? a.hQ + (head + row) * 4 * g.L : nullptr, grp, hc, g.L, h16);
     const float nrm = valid ? a.nQ[head + row] : 1.f;
-    if (ct < kR) sP1[ct] = a.Pmass[((size_t)bh * g.n_c + t) * kR + ct];
+    if (ct < kR) sP1[ct] = a.Pmass[(((size_t)grp * g.BH + bh) * g.n_c + t) * kR + ct];
     compute_bar();
     bool alive = true;
     // ---- intra-chunk element-wise pass: dkappa_ij = cl_i X_ij + delta_i, j <= i ----
@@ -629,16 +660,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_before();
       tc::mbar_arrive(&ms->dh_full);
     }
-    uint4 xr[8];
+    uint4 xr[D / 16];
     if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->x_full, 0, ms, err, 0x40000u));
-    load_x(smem + Q_XS, i, hc, valid && alive, xr);
+    load_x<D>(smem + q_xs<D>(), i, hc, valid && alive, xr);
     if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->du_full, 0, ms, err, 0x4000u));
     // every product is done: dQ rows are staged over the operand tiles
     float* stage_q = reinterpret_cast<float*>(smem + Q_DO);
-    chain_pass(tmem, lane_base, hc, i, TQ_DU, xr, nrm, sX, stage_q, valid, alive);
+    chain_pass<D>(tmem, lane_base, hc, i, TQ_DU, xr, nrm, sX, stage_q, valid, alive);
     compute_bar();
     if (!*(volatile int*)&ms->abort_flag)
-      copy_staged(stage_q, a.dQacc + (head + (size_t)t * kC) * kD, min(kC, g.N - t * kC), ct);
+      copy_staged<D>(stage_q, a.dQacc + (head + (size_t)t * kC) * D, min(kC, g.N - t * kC), ct, grp > 0);
   }
   __syncthreads();
   if (warp == 1) {
@@ -655,16 +686,18 @@ constexpr uint32_t R_BARS = R_P1 + (128 + 256) * 4;
 constexpr uint32_t TR_KAP = 0, TR_N = 128;
 }  // namespace
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     race_readout_tc_kernel(const __grid_constant__ CUtensorMap tmPQ, const __grid_constant__ CUtensorMap tmPK,
                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmOlr,
-                           const __grid_constant__ CUtensorMap tmP, FwdArgs a, Geom g, uint32_t* err) {
+                           const __grid_constant__ CUtensorMap tmP, FwdArgs a, Geom g, int grp, int mode,
+                           uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   Bars* ms = reinterpret_cast<Bars*>(smem + R_BARS);
   float* sP1 = reinterpret_cast<float*>(smem + R_P1);
   float* sX = sP1 + 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = g.n_t - 1 - blockIdx.x, bh = blockIdx.y;
+  const int t = g.n_c - 1 - blockIdx.x, bh = blockIdx.y;
   const size_t head = (size_t)bh * g.N;
   const bool causal = g.causal;
   if (smem_u32(smem) & 1023u) {
@@ -690,14 +723,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 5 : 3) * kTile);
+      // Phi tiles are [128][128]; V and the statistics are D columns wide
+      constexpr uint32_t kTD = 128u * D * 2;
+      tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 2 * kTile + kTD : kTile) + 2 * kTD);
       const int z = (bh * g.n_c + t) * 2;
       for (int s = 0; s < 2; ++s) {
         tc::tma_load_3d(smem + R_PQ + s * kSlab, &tmPQ, &ms->in_main, 64 * s, t * kC, bh);
-        if (causal) {
-          tc::tma_load_3d(smem + R_PK + s * kSlab, &tmPK, &ms->in_main, 64 * s, t * kC, bh);
-          tc::tma_load_3d(smem + R_V + s * kSlab, &tmV, &ms->in_main, 64 * s, t * kC, bh);
-        }
+        if (causal) tc::tma_load_3d(smem + R_PK + s * kSlab, &tmPK, &ms->in_main, 64 * s, t * kC, bh);
+      }
+      for (int s = 0; s < D / 64; ++s) {
+        if (causal) tc::tma_load_3d(smem + R_V + s * kSlab, &tmV, &ms->in_main, 64 * s, t * kC, bh);
         tc::tma_load_3d(smem + R_PH + s * kSlab, &tmP, &ms->in_main, 64 * s, 0, z);
         tc::tma_load_3d(smem + R_PL + s * kSlab, &tmP, &ms->in_main, 64 * s, 0, z + 1);
       }
@@ -706,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);
-      const uint32_t idNM = tc::idesc_bf16(128, 128, false, true);
+      const uint32_t idNM = tc::idesc_bf16(128, D, false, true);       // N = D, B MN-major
       const uint32_t sb = smem_u32(smem);
       bool ok = wait_or_abort(&ms->in_main, 0, ms, err, 0x100u);
       if (ok && causal) {
@@ -745,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
     const int row = t * kC + i;
     const bool valid = row < g.N;
-    if (ct < kR) sP1[ct] = a.Pmass[((size_t)bh * g.n_c + t) * kR + ct];
+    if (ct < kR) sP1[ct] = a.Pmass[(((size_t)grp * g.BH + bh) * g.n_c + t) * kR + ct];
     compute_bar();
     bool alive = true;
     float mass = 0.f;                                  // this thread's share of d_lr
@@ -791,19 +826,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     sX[2 * i + hc] = mass;
     if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->acc_full, 0, ms, err, 0x2000u));
     compute_bar();
-    const float dl = sX[2 * i] + sX[2 * i + 1];
+    // several feature groups (mode 1: the first, 2: the last) carry N and d_lr between launches
+    float* num = a.lr_num ? a.lr_num + (head + min(row, g.N - 1)) * D + (D / 2) * hc : nullptr;
+    float dl = sX[2 * i] + sX[2 * i + 1];
+    if (mode == 2 && valid) dl += a.lr_den[head + row];
     const float il = dl > 0.f ? 1.f / dl : 0.f;
-    if (alive) {
+    if (alive && mode == 1) {
+      tc::tc_fence_after();
+#pragma unroll
+      for (int h2 = 0; h2 < D / 64; ++h2) {
+        float v[32];
+        tc::tmem_ld32(tmem + lane_base + TR_N + (D / 2) * hc + 32 * h2, v);
+        tc::tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            reinterpret_cast<float4*>(num + 32 * h2)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+      }
+      if (hc == 0 && valid) a.lr_den[head + row] = dl;
+    } else if (alive) {
       tc::tc_fence_after();
       // O_lr = N / d_lr as bf16, staged (swizzled) over the Phi(K) tile, then one TMA store
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      for (int h2 = 0; h2 < D / 64; ++h2) {
         float v[32];
-        tc::tmem_ld32(tmem + lane_base + TR_N + 64 * hc + 32 * h2, v);
+        tc::tmem_ld32(tmem + lane_base + TR_N + (D / 2) * hc + 32 * h2, v);
         tc::tmem_wait_ld();
+        if (mode == 2 && valid) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 p = reinterpret_cast<const float4*>(num + 32 * h2)[q];
+            v[4 * q] += p.x; v[4 * q + 1] += p.y; v[4 * q + 2] += p.z; v[4 * q + 3] += p.w;
+          }
+        }
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
-          const int col = 64 * hc + 32 * h2 + 8 * ch;
+          const int col = (D / 2) * hc + 32 * h2 + 8 * ch;
           *reinterpret_cast<uint4*>(smem + R_PK + sw_off(i, col, kSlab)) =
               make_uint4(pack_bf16(v[8 * ch] * il, v[8 * ch + 1] * il), pack_bf16(v[8 * ch + 2] * il, v[8 * ch + 3] * il),
                          pack_bf16(v[8 * ch + 4] * il, v[8 * ch + 5] * il), pack_bf16(v[8 * ch + 6] * il, v[8 * ch + 7] * il));
@@ -813,13 +872,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc::fence_proxy_async_smem();
     compute_bar();
-    if (ct == 0 && !*(volatile int*)&ms->abort_flag) {
+    if (ct == 0 && mode != 1 && !*(volatile int*)&ms->abort_flag) {
       asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];\n"
                    :: "l"(reinterpret_cast<uint64_t>(&tmOlr)), "r"(smem_u32(smem + R_PK)), "r"(0), "r"(t * kC),
                       "r"(bh) : "memory");
-      asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];\n"
-                   :: "l"(reinterpret_cast<uint64_t>(&tmOlr)), "r"(smem_u32(smem + R_PK + kSlab)), "r"(64),
-                      "r"(t * kC), "r"(bh) : "memory");
+      if (D == 128)
+        asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];\n"
+                     :: "l"(reinterpret_cast<uint64_t>(&tmOlr)), "r"(smem_u32(smem + R_PK + kSlab)), "r"(64),
+                        "r"(t * kC), "r"(bh) : "memory");
       asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
       asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
     }
@@ -834,54 +894,97 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-cudaError_t launch_race_readout_tc(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
-  if (!race_bwd_tc_supported(g) || !a.Psplit || !a.Pmass) return cudaErrorInvalidValue;
-  CUtensorMap mpq, mpk, mv, mo, mp;
-  if (!tc::map_rows_bf16(&mpq, a.phiQ, g.N, g.BH, kC) || !tc::map_rows_bf16(&mpk, a.phiK, g.N, g.BH, kC) ||
-      !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kC) || !tc::map_rows_bf16(&mo, a.Olr, g.N, g.BH, kC) ||
-      !tc::map_rows_bf16(&mp, a.Psplit, kR, g.BH * g.n_c * 2, kR))
-    return cudaErrorInvalidValue;
+// Feature group grp's 128 columns of Phi ([BH][N][rp]) and its per-chunk statistics
+// ([G][BH][n_c][2][128][d]).
+static const void* phi_group(const void* phi, int grp) {
+  return static_cast<const __nv_bfloat16*>(phi) + (size_t)grp * kR;
+}
+static const void* split_group(const void* split, const Geom& g, int grp) {
+  return static_cast<const __nv_bfloat16*>(split) + (size_t)grp * g.BH * g.n_c * 2 * kR * g.d;
+}
+// [BH][N][d] rows (d = D) in boxes of 64 columns x 128 rows
+static bool map_d(CUtensorMap* m, const void* base, const Geom& g) {
+  return tc::map_rows_bf16_pitch(m, base, g.d, g.d, g.N, g.BH, kC);
+}
+
+template <int D>
+static cudaError_t readout_t(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
   const size_t smem = R_BARS + sizeof(Bars);
   static_assert(R_BARS + sizeof(Bars) <= 232448, "shared memory per CTA");
-  cudaError_t e = cudaFuncSetAttribute(race_readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(race_readout_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
-  ProfScope ps("race_readout_tc", st);
-  race_readout_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mpq, mpk, mv, mo, mp, a, g, err);
-  return cudaGetLastError();
+  for (int grp = 0; grp < g.G; ++grp) {
+    CUtensorMap mpq, mpk, mv, mo, mp;
+    if (!tc::map_rows_bf16_pitch(&mpq, phi_group(a.phiQ, grp), kR, g.rp, g.N, g.BH, kC) ||
+        !tc::map_rows_bf16_pitch(&mpk, phi_group(a.phiK, grp), kR, g.rp, g.N, g.BH, kC) || !map_d(&mv, a.V, g) ||
+        !map_d(&mo, a.Olr, g) ||
+        !tc::map_rows_bf16_pitch(&mp, split_group(a.Psplit, g, grp), D, D, kR, g.BH * g.n_c * 2, kR))
+      return cudaErrorInvalidValue;
+    // modes: 0 the only group; 1 the first of two (keeps N and d_lr); 2 the last (adds them)
+    const int mode = g.G == 1 ? 0 : grp == 0 ? 1 : 2;
+    ProfScope ps("race_readout_tc", st);
+    race_readout_tc_kernel<D><<<dim3(g.n_c, g.BH), kThreads, smem, st>>>(mpq, mpk, mv, mo, mp, a, g, grp, mode, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_race_readout_tc(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
+  if (!race_bwd_tc_supported(g) || !a.Psplit || !a.Pmass || (g.G > 1 && (!a.lr_num || !a.lr_den)))
+    return cudaErrorInvalidValue;
+  return g.d == 64 ? readout_t<64>(a, g, err, st) : readout_t<128>(a, g, err, st);
 }
 
 bool race_bwd_tc_supported(const Geom& g) {
-  return g.d == kD && g.T == kC && g.C == kC && g.r == kR && g.dp == kD + 8;
+  return (g.d == 64 || g.d == 128) && g.C == kC && g.r > 0 && g.r <= 2 * kR && g.r % 16 == 0 && g.rp == kR * g.G &&
+         g.dp == g.d + 8;
+}
+
+template <int D>
+static cudaError_t race_bwd_t(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
+  const int NW = (4 * g.L + 31) & ~31;                 // rows of each W half (4 L padded to 32)
+  CUtensorMap mv, mdo, mw, mq, mk;
+  if (!map_d(&mq, a.Q, g) || !map_d(&mk, a.K, g) || !map_d(&mv, a.V, g) || !map_d(&mdo, a.dO, g) ||
+      !tc::map_rows_bf16_pitch(&mw, a.Wsplit, D, D, NW, 2, kNH))
+    return cudaErrorInvalidValue;
+  const size_t smem_q = Q_BARS + sizeof(Bars), smem_k = K_BARS + sizeof(Bars);
+  static_assert(Q_BARS + sizeof(Bars) <= 232448, "shared memory per CTA");
+  static_assert(K_BARS + sizeof(Bars) <= 232448, "shared memory per CTA");
+  cudaError_t e = cudaFuncSetAttribute(race_q_bwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem_q);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(race_k_bwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k);
+  if (e != cudaSuccess) return e;
+  // one launch per group of 128 features (8 tables); the later groups add their parts
+  for (int grp = 0; grp < g.G; ++grp) {
+    CUtensorMap mpk, mpq, mp, mr;
+    if (!tc::map_rows_bf16_pitch(&mpk, phi_group(a.phiK, grp), kR, g.rp, g.N, g.BH, kC) ||
+        !tc::map_rows_bf16_pitch(&mpq, phi_group(a.phiQ, grp), kR, g.rp, g.N, g.BH, kC) ||
+        !tc::map_rows_bf16_pitch(&mp, split_group(a.Psplit, g, grp), D, D, kR, g.BH * g.n_c * 2, kR) ||
+        !tc::map_rows_bf16_pitch(&mr, split_group(a.Rsplit, g, grp), D, D, kR, g.BH * g.n_c * 2, kR))
+      return cudaErrorInvalidValue;
+    {
+      ProfScope ps("race_q_bwd_tc", st);
+      race_q_bwd_tc_kernel<D><<<dim3(g.n_c, g.BH), kThreads, smem_q, st>>>(mdo, mv, mpk, mp, mw, mq, a, g, grp, err);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    ProfScope ps("race_k_bwd_tc", st);
+    race_k_bwd_tc_kernel<D><<<dim3(g.n_c, g.BH), kThreads, smem_k, st>>>(mpk, mpq, mv, mdo, mr, mw, mk, a, g, grp,
+                                                                         err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_race_bwd_tc(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
   if (!race_bwd_tc_supported(g) || !a.hQ || !a.hK || !a.nQ || !a.nK || !a.Psplit || !a.Pmass || !a.Rsplit ||
       !a.Rmass || !a.Wsplit)
     return cudaErrorInvalidValue;
-  CUtensorMap mpk, mpq, mv, mdo, mp, mr, mw, mq, mk;
-  if (!tc::map_rows_bf16(&mq, a.Q, g.N, g.BH, kC) || !tc::map_rows_bf16(&mk, a.K, g.N, g.BH, kC) ||
-      !tc::map_rows_bf16(&mpk, a.phiK, g.N, g.BH, kC) || !tc::map_rows_bf16(&mpq, a.phiQ, g.N, g.BH, kC) ||
-      !tc::map_rows_bf16(&mv, a.V, g.N, g.BH, kC) || !tc::map_rows_bf16(&mdo, a.dO, g.N, g.BH, kC) ||
-      !tc::map_rows_bf16(&mp, a.Psplit, kR, g.BH * g.n_c * 2, kR) ||
-      !tc::map_rows_bf16(&mr, a.Rsplit, kR, g.BH * g.n_c * 2, kR) || !tc::map_rows_bf16(&mw, a.Wsplit, kNH, 2, kNH))
-    return cudaErrorInvalidValue;
-  {
-    const size_t smem = Q_BARS + sizeof(Bars);
-  static_assert(Q_BARS + sizeof(Bars) <= 232448, "shared memory per CTA");
-    cudaError_t e = cudaFuncSetAttribute(race_q_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    ProfScope ps("race_q_bwd_tc", st);
-    race_q_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mdo, mv, mpk, mp, mw, mq, a, g, err);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  const size_t smem = K_BARS + sizeof(Bars);
-  static_assert(K_BARS + sizeof(Bars) <= 232448, "shared memory per CTA");
-  cudaError_t e = cudaFuncSetAttribute(race_k_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  ProfScope ps("race_k_bwd_tc", st);
-  race_k_bwd_tc_kernel<<<dim3(g.n_t, g.BH), kThreads, smem, st>>>(mpk, mpq, mv, mdo, mr, mw, mk, a, g, err);
-  return cudaGetLastError();
+  return g.d == 64 ? race_bwd_t<64>(a, g, err, st) : race_bwd_t<128>(a, g, err, st);
 }
 
 }  // namespace elsaa

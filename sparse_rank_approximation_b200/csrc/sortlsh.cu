@@ -257,15 +257,15 @@ __global__ void causal_lsh_select_kernel(int* __restrict__ idx, Geom g) {
 // is in row order; level l's is in its sorted query order, at position inv_l[row], and
 // exists for the rows of its future halves (halves of h_l = N >> (l + 1) rows).  Then
 // m = 1 / (1 + (lambda d_lr + eps) e^{-log d_s}) (1 when m is held), O = g_s m O_s + g_lr O_lr
-// with g_lr = 1 - m by default (1 when m is held).  Writes O, the saved bf16 O_s, log d_s
-// and m.  One thread per 8 columns; partials are bf16, the merge is fp32.
+// with g_lr = 1 - m by default (1 when m is held).  Writes O, the saved fp32 O_s, log d_s
+// and m.  One thread per 8 columns; partials and the merge are fp32.
 constexpr int kMaxLevels = 8;             // N <= 32768 in blocks of >= 64 rows: at most 8 sorted levels
 
-__global__ void lsh_fuse_kernel(const __nv_bfloat16* __restrict__ Os0, const float* __restrict__ logd0,
-                                const __nv_bfloat16* __restrict__ Os_lv, const float* __restrict__ logd_lv,
+__global__ void lsh_fuse_kernel(const float* __restrict__ Os0, const float* __restrict__ logd0,
+                                const float* __restrict__ Os_lv, const float* __restrict__ logd_lv,
                                 const int* __restrict__ inv_lv, int levels, const __nv_bfloat16* __restrict__ Olr,
                                 const float* __restrict__ dlr, const float* lamv, const float* gsv, const float* glrv,
-                                __nv_bfloat16* __restrict__ O, __nv_bfloat16* __restrict__ Os,
+                                __nv_bfloat16* __restrict__ O, float* __restrict__ Os,
                                 float* __restrict__ logd_out, float* __restrict__ m_out, Geom g) {
   const int units = g.d / 8;
   const size_t rows = (size_t)g.BH * g.N;
@@ -277,17 +277,19 @@ __global__ void lsh_fuse_kernel(const __nv_bfloat16* __restrict__ Os0, const flo
     // the partials this row has: base (slot 0), then one per level where it is in a
     // future half.  Every partial's log-denominator and row are loaded as soon as its
     // position is known (predicated loads, no branch on the values)
-    uint4 w[kMaxLevels + 1];
+    float4 w[kMaxLevels + 1][2];
     float lg[kMaxLevels + 1];
-    w[0] = *reinterpret_cast<const uint4*>(Os0 + row * g.d + 8 * u);
+    w[0][0] = reinterpret_cast<const float4*>(Os0 + row * g.d + 8 * u)[0];
+    w[0][1] = reinterpret_cast<const float4*>(Os0 + row * g.d + 8 * u)[1];
     lg[0] = logd0[row];
 #pragma unroll
     for (int l = 0; l < kMaxLevels; ++l) {
       lg[l + 1] = -INFINITY;
-      w[l + 1] = make_uint4(0u, 0u, 0u, 0u);
+      w[l + 1][0] = w[l + 1][1] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (l < levels && ((r / (g.N >> (l + 1))) & 1)) {
         const size_t p = (size_t)l * rows + (size_t)bh * g.N + inv_lv[(size_t)l * rows + row];
-        w[l + 1] = *reinterpret_cast<const uint4*>(Os_lv + p * g.d + 8 * u);
+        w[l + 1][0] = reinterpret_cast<const float4*>(Os_lv + p * g.d + 8 * u)[0];
+        w[l + 1][1] = reinterpret_cast<const float4*>(Os_lv + p * g.d + 8 * u)[1];
         lg[l + 1] = logd_lv[p];
       }
     }
@@ -300,13 +302,9 @@ __global__ void lsh_fuse_kernel(const __nv_bfloat16* __restrict__ Os0, const flo
       for (int j = 0; j <= kMaxLevels; ++j) {
         const float wj = lg[j] == -INFINITY ? 0.f : __expf(lg[j] - L);
         sum += wj;
-        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w[j]);
+        const float* f = reinterpret_cast<const float*>(&w[j][0]);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f = __bfloat1622float2(hv[k]);
-          s[2 * k] = fmaf(wj, f.x, s[2 * k]);
-          s[2 * k + 1] = fmaf(wj, f.y, s[2 * k + 1]);
-        }
+        for (int k = 0; k < 8; ++k) s[k] = fmaf(wj, f[k], s[k]);
       }
       const float inv_sum = 1.f / sum;
 #pragma unroll
@@ -320,17 +318,16 @@ __global__ void lsh_fuse_kernel(const __nv_bfloat16* __restrict__ Os0, const flo
     const float cs = gs * mf;
     const uint4 wl = *reinterpret_cast<const uint4*>(Olr + row * g.d + 8 * u);
     const __nv_bfloat162* lv = reinterpret_cast<const __nv_bfloat162*>(&wl);
-    uint32_t wo[4], ws[4];
+    uint32_t wo[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float2 f = __bfloat1622float2(lv[j]);
       const __nv_bfloat162 o = __floats2bfloat162_rn(cs * s[2 * j] + gl * f.x, cs * s[2 * j + 1] + gl * f.y);
-      const __nv_bfloat162 q = __floats2bfloat162_rn(s[2 * j], s[2 * j + 1]);
       wo[j] = *reinterpret_cast<const uint32_t*>(&o);
-      ws[j] = *reinterpret_cast<const uint32_t*>(&q);
     }
     *reinterpret_cast<uint4*>(O + row * g.d + 8 * u) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
-    *reinterpret_cast<uint4*>(Os + row * g.d + 8 * u) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+    reinterpret_cast<float4*>(Os + row * g.d + 8 * u)[0] = make_float4(s[0], s[1], s[2], s[3]);
+    reinterpret_cast<float4*>(Os + row * g.d + 8 * u)[1] = make_float4(s[4], s[5], s[6], s[7]);
     if (u == 0) {
       logd_out[row] = L;
       m_out[row] = mf;
@@ -349,10 +346,10 @@ __global__ void lsh_invert_orders_kernel(const int* __restrict__ order, int* __r
 // The recursion's sparse gradient parts, per row of the caller's order: acc[row] += the
 // sum over the levels where the row is in a future half (queries: want = 1) or a past
 // half (keys: want = 0) of src_l at the row's sorted position.  Up to two tensors (dK
-// and dV) share the key side's positions.  src slots are bf16 [levels][BH][N][d]; inv
+// and dV) share the key side's positions.  src slots are fp32 [levels][BH][N][d]; inv
 // [levels][BH][2][N].
-__global__ void lsh_collect_kernel(const __nv_bfloat16* __restrict__ src0, float* __restrict__ acc0,
-                                   const __nv_bfloat16* __restrict__ src1, float* __restrict__ acc1,
+__global__ void lsh_collect_kernel(const float* __restrict__ src0, float* __restrict__ acc0,
+                                   const float* __restrict__ src1, float* __restrict__ acc1,
                                    const int* __restrict__ inv, int levels, int side, int want, Geom g) {
   const int units = g.d / 8;
   const size_t rows = (size_t)g.BH * g.N;
@@ -370,15 +367,11 @@ __global__ void lsh_collect_kernel(const __nv_bfloat16* __restrict__ src0, float
       const size_t p = (size_t)l * rows + (size_t)bh * g.N +
                        inv[(((size_t)l * g.BH + bh) * 2 + side) * g.N + r];
       for (int t = 0; t < (src1 ? 2 : 1); ++t) {
-        const uint4 w = *reinterpret_cast<const uint4*>((t ? src1 : src0) + p * g.d + 8 * u);
-        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
+        const float4* w = reinterpret_cast<const float4*>((t ? src1 : src0) + p * g.d + 8 * u);
+        const float4 w0 = w[0], w1 = w[1];
         float* sv = t ? s1 : s0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f = __bfloat1622float2(hv[k]);
-          sv[2 * k] += f.x;
-          sv[2 * k + 1] += f.y;
-        }
+        sv[0] += w0.x; sv[1] += w0.y; sv[2] += w0.z; sv[3] += w0.w;
+        sv[4] += w1.x; sv[5] += w1.y; sv[6] += w1.z; sv[7] += w1.w;
       }
     }
     if (!any) continue;
@@ -525,8 +518,8 @@ cudaError_t launch_lsh_fuse(const void* Os0, const float* logd0, const void* Os_
   if (levels > kMaxLevels) return cudaErrorInvalidValue;
   ProfScope ps("lsh_fuse", st);
   lsh_fuse_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
-      (const __nv_bfloat16*)Os0, logd0, (const __nv_bfloat16*)Os_lv, logd_lv, inv_lv, levels,
-      (const __nv_bfloat16*)Olr, dlr, lam, gs, glr, (__nv_bfloat16*)O, (__nv_bfloat16*)Os, logd, m, g);
+      (const float*)Os0, logd0, (const float*)Os_lv, logd_lv, inv_lv, levels,
+      (const __nv_bfloat16*)Olr, dlr, lam, gs, glr, (__nv_bfloat16*)O, (float*)Os, logd, m, g);
   return cudaGetLastError();
 }
 
@@ -541,7 +534,7 @@ cudaError_t launch_lsh_collect(const void* src0, float* acc0, const void* src1, 
   if (levels > kMaxLevels) return cudaErrorInvalidValue;
   ProfScope ps("lsh_collect", st);
   lsh_collect_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
-      (const __nv_bfloat16*)src0, acc0, (const __nv_bfloat16*)src1, acc1, inv, levels, keys ? 1 : 0, keys ? 0 : 1,
+      (const float*)src0, acc0, (const float*)src1, acc1, inv, levels, keys ? 1 : 0, keys ? 0 : 1,
       g);
   return cudaGetLastError();
 }

@@ -180,6 +180,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
 // Host: tensor map of a [BH][N][128] bf16 array as (column, row, head) with boxes
 // of 64 columns x `rows` rows, 128-byte swizzle (one 64-column slab per load).
 bool map_rows_bf16(CUtensorMap* m, const void* base, int N, int BH, int rows);
+// The same over `cols` (a multiple of 64) columns of rows `pitch` elements apart (pitch a
+// multiple of 8): a whole row, or a column block of wider rows.
+bool map_rows_bf16_pitch(CUtensorMap* m, const void* base, int cols, int pitch, int N, int BH, int rows);
 
 }  // namespace tc
 }  // namespace elsaa

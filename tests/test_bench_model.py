@@ -26,8 +26,8 @@ def test_every_dominant_kernel_has_a_work_model_entry():
     tensor-core ones positive flops too)."""
     for name, w in WORKLOADS.items():
         m, tot = bench.work_model(w)
-        for k in ("attn_fwd_tc", "dq_tc", "dkdv_tc", "race_k_bwd_tc", "race_q_bwd_tc", "race_k_bwd",
-                  "race_q_bwd", "sparse_dq", "sparse_dkdv", "attn_fwd"):
+        for k in ("attn_fwd_tc", "dq_tc", "dkdv_tc", "race_k_bwd_tc", "race_q_bwd_tc", "race_readout_tc",
+                  "race_features_tc", "race_stats_fwd_totals", "race_stats_bwd_totals"):
             assert m[k]["bytes"] > 0, (name, k)
         for k in ("attn_fwd_tc", "dq_tc", "dkdv_tc"):
             assert m[k]["flops"] > 0 or w.topk == 0, (name, k)

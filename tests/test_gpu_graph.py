@@ -13,7 +13,7 @@ pytestmark = pytest.mark.gpu
 
 CASES = {
     "topk_tcgen05": (dict(N=128 * 4 + 37, d=128, block_size=128, topk=2, rank_r=128), {}),
-    "topk_mma": (dict(N=64 * 5 + 11, d=64, block_size=64, topk=2, rank_r=32), {}),
+    "topk_d64_pairs": (dict(N=64 * 5 + 11, d=64, block_size=64, topk=2, rank_r=32), {}),
     "sortlsh": (dict(N=128 * 4 + 37, d=128, block_size=128, topk=1, rank_r=128, causal=False),
                 dict(selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=5)),
     "sortlsh_causal": (dict(N=128 * 8, d=128, block_size=128, topk=2, rank_r=128),

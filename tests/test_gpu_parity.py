@@ -24,6 +24,13 @@ SMALL = {
     "bf16_d128_T128_r128_noncausal": small_workload(N=128 * 3 + 50, d=128, block_size=128, topk=2, rank_r=128,
                                                     causal=False),
     "bf16_d128_T64_r256": small_workload(N=64 * 6, d=128, block_size=64, topk=4, rank_r=256, B=2, H=1),
+    # feature counts that are not one group of 128 on the tensor-core RACE path: two groups,
+    # a padded second group, and a single padded group
+    "bf16_d128_T128_r256_causal_ragged": small_workload(N=128 * 5 + 9, d=128, block_size=128, topk=2, rank_r=256,
+                                                        H=2),
+    "bf16_d128_T128_r192_noncausal": small_workload(N=128 * 3 + 50, d=128, block_size=128, topk=2, rank_r=192,
+                                                    causal=False),
+    "bf16_d128_T128_r48_causal": small_workload(N=128 * 4, d=128, block_size=128, topk=3, rank_r=48, H=2),
     "bf16_all_blocks": small_workload(N=64 * 4, d=64, block_size=64, topk=4, rank_r=16, causal=False),
     "f32_config_tiny": WORKLOADS["tiny_f32"],
     "f32_T64_causal_ragged": small_workload(N=64 * 3 + 11, d=64, block_size=64, topk=2, rank_r=32, dtype="f32"),
@@ -211,3 +218,19 @@ def test_forward_backward_full_size_sampled(name):
         check(w, "dQ rows", np64(dQ[b, h][rows]), dq)
         check(w, "dK rows", np64(dK[b, h][krows]), dk)
         check(w, "dV rows", np64(dV[b, h][krows]), dv)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_race_statistics_in_multi_chunk_segments(causal):
+    """Enough heads that the tensor-core RACE statistics walk segments of several chunks
+    (40 heads: 3 segments per head, of 3, 3 and 1 chunks, the last one ragged), so the
+    carried prefix inside a segment and the scanned carry between segments both matter;
+    three heads against the oracle."""
+    w = small_workload(N=128 * 6 + 5, d=128, block_size=128, topk=2, rank_r=128, H=40, causal=causal)
+    inp, extra, O, scores, idx, grads = _run(w)
+    for h in (0, 17, w.H - 1):
+        fw, (dq, dk, dv) = _oracle_head(w, inp, extra, scores, 0, h)
+        check(w, f"O[{h}]", np64(O[0, h]), fw["O"])
+        check(w, f"dQ[{h}]", np64(grads[0][0, h]), dq)
+        check(w, f"dK[{h}]", np64(grads[1][0, h]), dk)
+        check(w, f"dV[{h}]", np64(grads[2][0, h]), dv)

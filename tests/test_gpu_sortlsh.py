@@ -2,7 +2,7 @@
 
 The hash codes are compared bit for bit (a mismatch is allowed only where a projection
 is within float32 rounding of zero); the outputs and gradients are compared with the
-oracle run on the same sorted orders, for the tensor-core, mma.sync and float32 paths.
+oracle run on the same sorted orders, for the tensor-core (every bf16 shape) and float32 paths.
 """
 import numpy as np
 import pytest
@@ -11,8 +11,7 @@ import torch
 from oracle import elsaa_oracle as orc
 from sparse_rank_approximation_b200 import binding as bd
 from sparse_rank_approximation_b200.workloads import WORKLOADS, make_inputs, small_workload
-from tests.harness import (BF16_ABS_TOL, BF16_STORE_REL, check, check_fusion_grads, device_inputs, gpu_op, np64,
-                           oracle_params, sparse_rounding_scales)
+from tests.harness import check, check_fusion_grads, device_inputs, gpu_op, np64, oracle_params
 
 pytestmark = pytest.mark.gpu
 
@@ -122,14 +121,11 @@ def test_full_size():
         fw = orc.forward_head(get("Q"), get("K"), get("V"), W, p)
         dq, dk, dv = orc.backward_head(get("Q"), get("K"), get("V"), W, get("dO"), fw, p)
         check(w, f"O[{h}]", np64(O[0, h]), fw["O"])
-        # the gradients: the usual bf16 bound plus the rounding inside the sparse backward
-        # (twice its half-ulp scale); at this length sorted blocks put most of a row's
-        # mass on a few keys, where the Delta term dominates
-        scales = sparse_rounding_scales(get("Q"), get("K"), get("V"), get("dO"), fw, p)
-        for name, got, ref, B in zip(("dQ", "dK", "dV"), (dQ, dK, dV), (dq, dk, dv), scales):
-            err = np.abs(np64(got[0, h]) - ref)
-            excess = (err - BF16_STORE_REL * np.abs(ref) - 2.0 ** -8 * B).max()
-            assert excess <= BF16_ABS_TOL, f"{name}[{h}]: max err {err.max():.3e}, beyond the bound {excess:.3e}"
+        # at this length sorted blocks put most of a row's mass on a few keys, where
+        # dP_ij and Delta_i nearly cancel: Delta comes from the fp32 O_s
+        check(w, f"dQ[{h}]", np64(dQ[0, h]), dq)
+        check(w, f"dK[{h}]", np64(dK[0, h]), dk)
+        check(w, f"dV[{h}]", np64(dV[0, h]), dv)
 
 
 # ---- the causal recursion (bf16, d = 128, block 128 on the tensor-core kernels) ----
@@ -188,8 +184,8 @@ def test_causal_hash_widths(bits):
                                                    (512, 64, True, False, 128, 64)])
 def test_causal_forward_backward(N, r, gates, fixed_m, d, T):
     """O, dQ, dK, dV and the fusion gradients against the oracle's recursion run on the GPU's
-    hash codes (every level's sorted order follows from them), on the tcgen05 shape (d = 128,
-    block 128) and the mma.sync shapes; N = 128 and 256 at block 128 are the single-block and
+    hash codes (every level's sorted order follows from them), for d = 64 and 128 and blocks of 64
+    and 128 keys (pair mode at 64); N = 128 and 256 at block 128 are the single-block and
     two-block cases (exact causal attention)."""
     w, inp, dev, R, op = _causal_setup(N, r, seed=3, fixed_m=fixed_m, d=d, T=T)
     BH = (w.B, w.H, w.N)
@@ -242,8 +238,6 @@ def test_causal_full_size():
         fw = orc.forward_head(get("Q"), get("K"), get("V"), W, p)
         dq, dk, dv = orc.backward_head(get("Q"), get("K"), get("V"), W, get("dO"), fw, p)
         check(w, f"O[{h}]", np64(O[0, h]), fw["O"])
-        scales = sparse_rounding_scales(get("Q"), get("K"), get("V"), get("dO"), fw, p)
-        for name, got, ref, B in zip(("dQ", "dK", "dV"), (dQ, dK, dV), (dq, dk, dv), scales):
-            err = np.abs(np64(got[0, h]) - ref)
-            excess = (err - BF16_STORE_REL * np.abs(ref) - 2.0 ** -8 * B).max()
-            assert excess <= BF16_ABS_TOL, f"{name}[{h}]: max err {err.max():.3e}, beyond the bound {excess:.3e}"
+        check(w, f"dQ[{h}]", np64(dQ[0, h]), dq)
+        check(w, f"dK[{h}]", np64(dK[0, h]), dk)
+        check(w, f"dV[{h}]", np64(dV[0, h]), dv)

@@ -5,9 +5,11 @@ the library; the test checks, through the C ABI, that two calls in a row give
 exactly the indices of elsaa_debug_select (which uses caller scratch)."""
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+from oracle import elsaa_oracle as orc
 from sparse_rank_approximation_b200 import binding as bd
 from sparse_rank_approximation_b200.workloads import WORKLOADS, make_inputs, small_workload
 from tests.harness import device_inputs, gpu_op
@@ -33,9 +35,39 @@ def test_noalloc_selection_matches_workspace_selection_twice(w):
     for seed in (0, 1):                      # two calls in a row, different inputs
         dev = device_inputs(w, make_inputs(w, seed))
         _, ref = op.debug_select(dev["Q"], dev["K"])
+        scores, _ = op.debug_select(dev["Q"], dev["K"])
         got = _noalloc(op, dev["Q"], dev["K"])
         torch.cuda.synchronize()
         assert torch.equal(got, ref), f"seed {seed}: selection differs"
+        # and the oracle's selection rule fed the same float32 scores picks the same blocks
+        sc, ix = scores.cpu().numpy(), got.cpu().numpy()
+        for b in range(w.B):
+            for h in range(w.H):
+                assert np.array_equal(orc.select_from_scores(sc[b, h], w.topk, w.causal), ix[b, h]), (b, h)
+
+
+def test_noalloc_selection_replays_from_a_cuda_graph():
+    """The reason for the entry point: it can be captured, since it allocates nothing.
+    One eager call first (it resolves the array's address), then a capture on a side
+    stream; new inputs copied into the captured buffers give the new selection."""
+    w = small_workload(N=128 * 6 + 21, d=128, block_size=128, topk=3, rank_r=16, H=2)
+    op = gpu_op(w)
+    a = device_inputs(w, make_inputs(w, 0))
+    q, k = a["Q"].clone(), a["K"].clone()
+    _noalloc(op, q, k)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        out = _noalloc(op, q, k)
+    for seed in (3, 4):
+        b = device_inputs(w, make_inputs(w, seed))
+        q.copy_(b["Q"])
+        k.copy_(b["K"])
+        g.replay()
+        _, ref = op.debug_select(b["Q"], b["K"])
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref), f"seed {seed}: replayed selection differs"
+    del g
 
 
 def test_noalloc_rejects_problems_beyond_its_static_scratch():
