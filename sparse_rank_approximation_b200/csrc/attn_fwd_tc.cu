@@ -14,13 +14,17 @@
 //               score buffers, then O += P_{j-1} V_{j-1} into the TMEM output
 //               with P_{j-1} read from tensor memory;
 //   warp 2      TMA producer of the V ring (3 stages);
-//   warps 3-10  softmax: each query row is split over two warps (64 score
-//               columns each) that exchange their partial row max; online
-//               softmax in fp32 with lazy rescaling (O and l are rescaled only
-//               when the running max grows by more than 2^16, after P_j is
-//               written and just before it is released); P_j (bf16 pairs)
-//               overwrites the score columns it came from and is the A operand
-//               of the PV product; the epilogue normalises O, applies the
+//   warps 3-10  softmax: each query row is split over two warps, one per half
+//               of the key columns; each half keeps its own running max, row
+//               sum and output accumulator O_h = sum over its keys of P V (the
+//               PV product of a block is two products of 64 keys, one per
+//               half), so the halves never wait on each other inside the loop;
+//               online softmax in fp32 with lazy rescaling (O_h and l_h are
+//               rescaled only when the half's running max grows by more than
+//               2^16, after P_j is written and just before it is released);
+//               P_j (bf16 pairs) overwrites the score columns it came from and
+//               is the A operand of the PV product; the epilogue merges the two
+//               halves (one exchange of max and sum), normalises O, applies the
 //               fusion and writes O and O_s through shared memory with TMA stores.
 // Operand tiles are 64-column slabs with 128-byte swizzle, as TMA writes them.
 // Every mbarrier wait is bounded; a timeout sets a bit in the caller's error
@@ -42,24 +46,26 @@ constexpr int kStages = 3;                 // K and V ring depth
 __host__ __device__ constexpr uint32_t off_k(int s) { return kTile * (1 + s); }              // K stage s
 __host__ __device__ constexpr uint32_t off_v(int s) { return kTile * (1 + kStages + s); }    // V stage s
 constexpr uint32_t OFF_MISC = (1 + 2 * kStages) * kTile;
-// column of the K = 16 step kk of P (key 64 h + m of a row sits at column 64 h + m / 2)
+// column of the K = 16 step kk of P_hi (key 64 h + m of a row sits at column 64 h + m / 2);
+// P_lo = bf16(P - P_hi) sits 32 columns further, over score columns already read
 __host__ __device__ constexpr uint32_t p_col(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
+constexpr uint32_t kPLo = 32;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t TM_O = 0;
+constexpr uint32_t TM_O0 = 0, TM_O1 = 384;                 // output accumulators of the two key halves
 __host__ __device__ constexpr uint32_t tm_s(int s) { return 128u + 128u * s; }         // score buffer s
 constexpr float kRescaleThreshold = 16.f;                // log2 units: P stays below 2^16
 constexpr int kThreads = 352;
 constexpr int kSoftmaxThreads = 256;
 
 struct Misc {
-  uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full[2], p_full[2],
-      pv_done[2];
+  uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full[2],
+      p_full[2][2], pv_done[2][2];       // [score buffer][key half]
   uint64_t olr_full, drain, never;
   unsigned long long limit_ns;
   uint32_t tmem_base;
   int abort_flag;
   int idx[2][32];         // selected blocks of the CTA's tile (PAIR: of its two tiles)
-  float red[2][256];      // partial row maxima / sums exchanged by the two halves of a row
+  float mx_half[256], l_half[256];   // each half's reference max and row sum, for the merge
 };
 constexpr size_t kSmemBytes = OFF_MISC + sizeof(Misc);
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -126,8 +132,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&ms->s_full[s], 1);
-      tc::mbar_init(&ms->p_full[s], kSoftmaxThreads);
-      tc::mbar_init(&ms->pv_done[s], 1);
+      for (int h = 0; h < 2; ++h) {
+        tc::mbar_init(&ms->p_full[s][h], kSoftmaxThreads / 2);
+        tc::mbar_init(&ms->pv_done[s][h], 1);
+      }
     }
     tc::mbar_init(&ms->olr_full, 1);
     tc::mbar_init(&ms->drain, 1);
@@ -211,18 +219,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sbase = smem_u32(smem);
       bool ok = wait_or_abort(&ms->q_full, 0, ms, err, 2u);
       int pv_issued = 0;
+      // O_h += P_jj[:, keys of half h] V_jj[keys of half h, :], each half as soon as its P is
+      // written
       auto issue_pv = [&](int jj) -> bool {
-        if (!wait_or_abort(&ms->p_full[jj & 1], (jj >> 1) & 1, ms, err, 4u)) return false;
-        if (!wait_or_abort(&ms->v_full[jj % kStages], (jj / kStages) & 1, ms, err, 1024u)) return false;
-        tc::tc_fence_after();
         const uint32_t vb = sbase + off_v(jj % kStages);
+        for (int h = 0; h < 2; ++h) {
+          if (!wait_or_abort(&ms->p_full[jj & 1][h], (jj >> 1) & 1, ms, err, 4u)) return false;
+          if (h == 0 && !wait_or_abort(&ms->v_full[jj % kStages], (jj / kStages) & 1, ms, err, 1024u)) return false;
+          tc::tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kT / 16; ++kk) {
-          const uint64_t bd = tc::sw128_desc(vb + kk * 2048, kSlab, 1024);
-          tc::mma_bf16_ts(tmem + TM_O, tmem + tm_s(jj & 1) + p_col(kk), bd, idPV, (jj > 0 || kk > 0) ? 1u : 0u);
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kk = 4 * h + k4;                  // keys 16 kk .. 16 kk + 15
+            const uint64_t bd = tc::sw128_desc(vb + kk * 2048, kSlab, 1024);
+            const uint32_t pa = tmem + tm_s(jj & 1) + p_col(kk);
+            tc::mma_bf16_ts(tmem + (h ? TM_O1 : TM_O0), pa, bd, idPV, (jj > 0 || k4 > 0) ? 1u : 0u);
+            tc::mma_bf16_ts(tmem + (h ? TM_O1 : TM_O0), pa + kPLo, bd, idPV, 1u);
+          }
+          tc::mma_commit(&ms->pv_done[jj & 1][h]);
         }
         tc::mma_commit(&ms->v_empty[jj % kStages]);
-        tc::mma_commit(&ms->pv_done[jj & 1]);
         pv_issued = jj + 1;
         return true;
       };
@@ -253,7 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q4 = warp & 3;
     const int half = (warp - 3) >> 2;                // score columns [64 half, +64), output [H half, +H)
     const int row = 32 * q4 + lane;
-    const int sid = half * 128 + row;                // slot in the exchange arrays
+    const int sid = half * 128 + row;                // slot in the merge arrays
+    const uint32_t o_mine = half ? TM_O1 : TM_O0;    // this half's output accumulator
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
     const float sl2 = g.scale * kLog2e;
     const int qrow = row0 + row;
@@ -270,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float lam = a.lam ? a.lam[ri] : g.lam;
     const float gs = a.gs ? a.gs[ri] : 1.f;
     const float glr_in = a.glr ? a.glr[ri] : -1.f;
-    float m_used = -INFINITY, lp = 0.f;              // running max (scaled log2 units), partial row sum
+    float m_used = -INFINITY, lp = 0.f;              // this half's reference max (scaled log2 units), row sum
     bool alive = true;                               // warp-uniform; every barrier below is still taken
     // test hook: a wait on a barrier nothing completes, so the give-up path runs
     if (g.debug_stall) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->never, 0, ms, err, 0x40000u));
@@ -312,12 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           m4[2] = fmaxf(m4[2], sv[c + 2]);
           m4[3] = fmaxf(m4[3], sv[c + 3]);
         }
-        ms->red[s][sid] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      }
-      softmax_bar();
-      if (alive) {
-        const float mx = fmaxf(ms->red[s][row], ms->red[s][128 + row]) * sl2;
-        // lazy rescaling: move the reference max only when the row max grew by > 2^8
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+        // lazy rescaling: move the reference max only when this half's max grew by > 2^16
         const float m_new = fmaxf(m_used, mx);
         const bool resc = m_new > m_used + kRescaleThreshold;     // false while both are -inf
         float alpha = 1.f;
@@ -326,79 +338,91 @@ __global__ void __launch_bounds__(kThreads, 1)
           lp *= alpha;
           m_used = m_new;
         }
-        // P_j (bf16 pairs) over the first half of this thread's score columns: the
-        // PV product of block j-2 read that buffer before S_j was written into it
-        if (alive) {
-          const float msub = m_used == -INFINITY ? 0.f : m_used;
-          float rs0 = 0.f, rs1 = 0.f;
+        // P_j as bf16 hi + lo pairs (16 significant bits, so O_s and the backward's softmax delta
+        // formed from it carry no bf16 rounding of the weights) over this thread's score
+        // columns: the PV product of block j-2 read that buffer before S_j was written into it
+        const float msub = m_used == -INFINITY ? 0.f : m_used;
+        float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t w[8];
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t w[8], wl[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float p0 = ex2_approx(fmaf(sv[16 * ch + 2 * e], sl2, -msub));
-              const float p1 = ex2_approx(fmaf(sv[16 * ch + 2 * e + 1], sl2, -msub));
-              rs0 += p0;
-              rs1 += p1;
-              w[e] = pack_bf16(p0, p1);
-            }
-            tc::tmem_st8(tmem + lane_base + tm_s(s) + 64 * half + 8 * ch, w);
+          for (int e = 0; e < 8; ++e) {
+            const float p0 = ex2_approx(fmaf(sv[16 * ch + 2 * e], sl2, -msub));
+            const float p1 = ex2_approx(fmaf(sv[16 * ch + 2 * e + 1], sl2, -msub));
+            rs0 += p0;
+            rs1 += p1;
+            w[e] = pack_bf16(p0, p1);
+            wl[e] = pack_bf16(p0 - __uint_as_float(w[e] << 16), p1 - __uint_as_float(w[e] & 0xffff0000u));
           }
-          lp += rs0 + rs1;
-          tc::tmem_wait_st();
+          tc::tmem_st8(tmem + lane_base + tm_s(s) + 64 * half + 8 * ch, w);
+          tc::tmem_st8(tmem + lane_base + tm_s(s) + 64 * half + kPLo + 8 * ch, wl);
         }
-        // O holds the products through block j-1; a moved reference max rescales it (this half
-        // of the columns) once that product is done, before P_j is released to the MMA warp.
-        if (alive && j > 0 && __any_sync(0xffffffffu, resc)) {
-          alive = __all_sync(0xffffffffu,
-                             wait_or_abort(&ms->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ms, err, 64u));
+        lp += rs0 + rs1;
+        tc::tmem_wait_st();
+        // O_h holds this half's products through block j-1; a moved reference max rescales it
+        // once that product is done, before P_j is released to the MMA warp
+        if (j > 0 && __any_sync(0xffffffffu, resc)) {
+          alive = __all_sync(0xffffffffu, wait_or_abort(&ms->pv_done[(j - 1) & 1][half], ((j - 1) >> 1) & 1, ms,
+                                                        err, 64u));
           if (alive) {
             tc::tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < H / 32; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
               float tmp[32];
-              tc::tmem_ld32(tmem + lane_base + TM_O + H * half + 32 * c, tmp);
+              tc::tmem_ld32(tmem + lane_base + o_mine + 32 * c, tmp);
               tc::tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 32; ++i) tmp[i] *= alpha;
-              tc::tmem_st32(tmem + lane_base + TM_O + H * half + 32 * c, tmp);
+              tc::tmem_st32(tmem + lane_base + o_mine + 32 * c, tmp);
             }
             tc::tmem_wait_st();
           }
         }
         if (alive) {
           tc::tc_fence_before();
-          tc::mbar_arrive(&ms->p_full[s]);
+          tc::mbar_arrive(&ms->p_full[s][half]);
         }
       }
     }
-    // ---- epilogue: O_s = O / l, log d_s, fusion (Eq. 5, Eq. 4), TMA stores from shared memory
+    // ---- epilogue: merge the two halves (O = f0 O_0 + f1 O_1, l = f0 l_0 + f1 l_1 with
+    // f_h = 2^(m_h - max(m_0, m_1))), O_s = O / l, log d_s, fusion (Eq. 5, Eq. 4), TMA stores
+    // from shared memory
+    ms->mx_half[sid] = m_used;
+    ms->l_half[sid] = lp;
+    bool have = false;
+    if (alive && n_sel > 0) {
+      const int jl = n_sel - 1;
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->pv_done[jl & 1][0], (jl >> 1) & 1, ms, err, 128u));
+      if (alive)
+        alive = __all_sync(0xffffffffu, wait_or_abort(&ms->pv_done[jl & 1][1], (jl >> 1) & 1, ms, err, 128u));
+      have = alive;
+    }
+    if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->olr_full, 0, ms, err, 4096u));
+    softmax_bar();
+    const float m0 = ms->mx_half[row], m1 = ms->mx_half[128 + row];
+    const float mm = fmaxf(m0, m1);
+    const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - mm);
+    const float f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - mm);
+    const float l = f0 * ms->l_half[row] + f1 * ms->l_half[128 + row];
     float o[H];
 #pragma unroll
     for (int c = 0; c < H; ++c) o[c] = 0.f;
-    if (alive && n_sel > 0) {
-      alive = __all_sync(0xffffffffu,
-                         wait_or_abort(&ms->pv_done[(n_sel - 1) & 1], ((n_sel - 1) >> 1) & 1, ms, err, 128u));
-      if (alive) {
-        tc::tc_fence_after();
+    if (have && alive) {
+      tc::tc_fence_after();
 #pragma unroll
-        for (int c2 = 0; c2 < H / 32; ++c2) {
-          float tmp[32];
-          tc::tmem_ld32(tmem + lane_base + TM_O + H * half + 32 * c2, tmp);
-          tc::tmem_wait_ld();
+      for (int c2 = 0; c2 < H / 32; ++c2) {
+        float t0[32], t1[32];
+        tc::tmem_ld32(tmem + lane_base + TM_O0 + H * half + 32 * c2, t0);
+        tc::tmem_ld32(tmem + lane_base + TM_O1 + H * half + 32 * c2, t1);
+        tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[32 * c2 + i] = tmp[i];
-        }
+        for (int i = 0; i < 32; ++i) o[32 * c2 + i] = f0 * t0[i] + f1 * t1[i];
       }
     }
-    const int rb = n_sel & 1;                         // exchange buffer not read in the last loop step
-    ms->red[rb][sid] = lp;
-    if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->olr_full, 0, ms, err, 4096u));
-    softmax_bar();
-    const float l = ms->red[rb][row] + ms->red[rb][128 + row];
     // every PV product is done: V stage 0 holds the outgoing O, V stages 1 (and 2) the fp32 O_s
     if (alive) {
-      const float logd = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+      const float logd = l > 0.f ? (mm + log2f(l)) * kLn2 : -INFINITY;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const float mf = g.fixed_m ? 1.f : logd == -INFINITY ? 0.f : 1.f / (1.f + (lam * dl + g.eps) * expf(-logd));
       const float gl = a.glr ? glr_in : g.fixed_m ? 1.f : 1.f - mf;

@@ -447,10 +447,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   constexpr int TB = PAIR ? 64 : 128;       // keys per block = queries per tile
   constexpr int H = D / 2;                  // dK / dV columns per thread (half a row)
   // heaviest key blocks of every head first (order from the selection inverse); PAIR: the
-  // pairs in order
-  const int b = PAIR ? 2 * (int)blockIdx.y
-                     : (a.kv_order ? a.kv_order[(size_t)bh * g.n_t + blockIdx.y] : (int)blockIdx.y);
-  const int key0 = PAIR ? 64 * b : kT * b;   // first key row of the CTA
+  // CTA takes entries 2y and 2y + 1 of that order, two blocks with about as many query tiles
+  // (pb[1] = -1 past the last block)
+  const int nb = a.n_kv ? a.n_kv : g.n_t;
+  const int* kvo = a.kv_order ? a.kv_order + (size_t)bh * g.n_t : nullptr;
+  const int y = blockIdx.y;
+  const int b = PAIR ? (kvo ? kvo[2 * y] : 2 * y) : (kvo ? kvo[y] : y);
+  const int pb[2] = {b, PAIR ? (2 * y + 1 < nb ? (kvo ? kvo[2 * y + 1] : 2 * y + 1) : -1) : b};
+  const int key0 = kT * b;                   // first key row of the CTA (not PAIR)
   const size_t head = (size_t)bh * g.N;
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
@@ -461,8 +465,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     const int* of = a.offs + (size_t)bh * (g.n_t + 1);
     const int* list = a.tiles + (size_t)bh * g.n_t * g.k;
     for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
-      const int bb = b + h;
-      if (bb >= g.n_t) break;
+      const int bb = pb[h];
+      if (bb < 0) break;
       const int e0 = of[bb];
       n_ut[h] = min(of[bb + 1] - e0, kMaxUnits);
       for (int i = threadIdx.x; i < n_ut[h]; i += kKvThreads) units[h * kMaxUnits + i] = list[e0 + i];
@@ -497,9 +501,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kTD = 128u * D * 2;      // bytes of a [128][D] tile
       tc::mbar_arrive_expect_tx(&ms->kv_full, 2 * kTD);
-      for (int sl = 0; sl < D / 64; ++sl) {
-        tc::tma_load_3d(smem + KV_K + sl * kSlab, &tmK, &ms->kv_full, 64 * sl, key0, bh);
-        tc::tma_load_3d(smem + KV_V + sl * kSlab, &tmV, &ms->kv_full, 64 * sl, key0, bh);
+      // PAIR: block pb[0] in key rows 0-63, pb[1] in rows 64-127 (a missing one stages pb[0])
+      for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
+        const int kr = PAIR ? 64 * (pb[h] >= 0 ? pb[h] : pb[0]) : key0;
+        for (int sl = 0; sl < D / 64; ++sl) {
+          tc::tma_load_3d(smem + KV_K + sl * kSlab + h * 64 * 128, &tmK, &ms->kv_full, 64 * sl, kr, bh);
+          tc::tma_load_3d(smem + KV_V + sl * kSlab + h * 64 * 128, &tmV, &ms->kv_full, 64 * sl, kr, bh);
+        }
       }
       int issued = 0;
       for (int u = 0; u < n_u; ++u) {
@@ -577,12 +585,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     const int grp = (warp - 2) >> 2;                // queries 32 grp + 64 pass .. + 31
     const int row = 32 * q4 + lane;                 // key row within the CTA's 128
     const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-    const bool key_ok = key0 + row < g.N;
-    const float sl2 = g.scale * kLog2e;
-    // PAIR: key rows 0-63 are block b and see query rows 0-63 of a unit (pass 0), rows 64-127
-    // block b + 1 and query rows 64-127 (pass 1)
+    // PAIR: key rows 0-63 are block pb[0], rows 64-127 block pb[1]
     const int mine = PAIR ? (row >= 64) : 0;
-    const int my_block = b + mine;
+    const int my_block = pb[mine];
+    const int krow = PAIR ? 64 * my_block + (row & 63) : key0 + row;      // key row in the head
+    const bool key_ok = my_block >= 0 && krow < g.N;
+    const float sl2 = g.scale * kLog2e;
+    // PAIR: key rows 0-63 see query rows 0-63 of a unit (pass 0), rows 64-127 query rows
+    // 64-127 (pass 1)
     const int kpos = PAIR ? (row & 63) : row;       // key position within its block
     bool alive = true;
     for (int u = 0; u < n_u && alive; ++u) {
@@ -631,13 +641,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const float mul = which == 0 ? g.scale : 1.f;
       const float* accp = which == 0 ? a.dKacc : a.dVacc;
       const float4* ak = accp && alive && key_ok
-                             ? reinterpret_cast<const float4*>(accp + (head + (size_t)key0 + row) * D + col0)
+                             ? reinterpret_cast<const float4*>(accp + (head + (size_t)krow) * D + col0)
                              : nullptr;
       unsigned char* orow = smem + (which == 0 ? kv_q(0) : kv_do(0)) + (col0 >> 6) * kSlab + row * 128;
       // with a row map, write each key row straight to the caller's row instead
       uint4* grow = a.k_rows && key_ok && alive
                         ? reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(which == 0 ? a.dK : a.dV) +
-                                                   (head + a.k_rows[(size_t)bh * a.rows_stride + key0 + row]) * D +
+                                                   (head + a.k_rows[(size_t)bh * a.rows_stride + krow]) * D +
                                                    col0)
                         : nullptr;
       // 32 columns at a time: TMEM -> scale -> + low-rank part -> bf16 -> swizzled row
@@ -662,7 +672,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         if (a.out_f32) {                                 // fp32 rows (level slots), no staging
           if (alive && key_ok) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(which == 0 ? a.dK : a.dV) +
-                                                    (head + (size_t)key0 + row) * D + col0 + 32 * c);
+                                                    (head + (size_t)krow) * D + col0 + 32 * c);
 #pragma unroll
             for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
           }
@@ -686,9 +696,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       tc::fence_proxy_async_smem();
       softmax_bar();
       if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
-        for (int sl = 0; sl < D / 64; ++sl) {
-          tma_store_3d(&tmdK, smem + kv_q(0) + sl * kSlab, 64 * sl, key0, bh);
-          tma_store_3d(&tmdV, smem + kv_do(0) + sl * kSlab, 64 * sl, key0, bh);
+        for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
+          if (pb[h] < 0) continue;
+          const int kr = PAIR ? 64 * pb[h] : key0;
+          for (int sl = 0; sl < D / 64; ++sl) {
+            tma_store_3d(&tmdK, smem + kv_q(0) + sl * kSlab + h * 64 * 128, 64 * sl, kr, bh);
+            tma_store_3d(&tmdV, smem + kv_do(0) + sl * kSlab + h * 64 * 128, 64 * sl, kr, bh);
+          }
         }
         tma_store_wait();
       }
@@ -784,8 +798,8 @@ template <int D, bool PAIR>
 static cudaError_t dkdv_t(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
   constexpr int TB = PAIR ? 64 : 128;
   CUtensorMap mk, mv, mq, mdo, msc, mdk, mdv;
-  if (!map_d(&mk, a.K, g, kT) || !map_d(&mv, a.V, g, kT) || !map_d(&mq, a.Q, g, TB) || !map_d(&mdo, a.dO, g, TB) ||
-      !map_scalars(&msc, a.rs.packed, g.N, g.BH, TB) || !map_d(&mdk, a.dK, g, kT) || !map_d(&mdv, a.dV, g, kT))
+  if (!map_d(&mk, a.K, g, TB) || !map_d(&mv, a.V, g, TB) || !map_d(&mq, a.Q, g, TB) || !map_d(&mdo, a.dO, g, TB) ||
+      !map_scalars(&msc, a.rs.packed, g.N, g.BH, TB) || !map_d(&mdk, a.dK, g, TB) || !map_d(&mdv, a.dV, g, TB))
     return cudaErrorInvalidValue;
   const size_t smem = KV_MISC + sizeof(KvMisc);
   static_assert(KV_MISC + sizeof(KvMisc) <= 232448, "shared memory per CTA");
@@ -793,9 +807,10 @@ static cudaError_t dkdv_t(const BwdArgs& a, const Geom& g, uint32_t* err, cudaSt
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("dkdv_tc", st);
-  // with n_kv, only the first n_kv key blocks of kv_order (the ones with query tiles) run; pairs
-  // of blocks run in order (the empty ones write zeros)
-  const int ctas = PAIR ? (g.n_t + 1) / 2 : (a.n_kv ? a.n_kv : g.n_t);
+  // with n_kv, only the first n_kv key blocks of kv_order (the ones with query tiles) run;
+  // PAIR: two consecutive entries of that order per CTA
+  const int nb = a.n_kv ? a.n_kv : g.n_t;
+  const int ctas = PAIR ? (nb + 1) / 2 : nb;
   kern<<<dim3(g.BH, ctas), kKvThreads, smem, st>>>(mk, mv, mq, mdo, msc, mdk, mdv, a, g, err);
   return cudaGetLastError();
 }

@@ -411,22 +411,35 @@ SideStream* side_stream() {
   return x.s ? &x : nullptr;
 }
 
-// Makes the caller's stream wait for the selection stream once, on the normal path or, if a
-// launch fails after the fork, when the forward returns (work already queued on the second
-// stream then never outlives the caller's view of the call).  A failure to record the join
-// event leaves the wait on its previous record, which precedes the fork.
+// Joins the selection stream back into the caller's stream exactly once: on the normal path
+// before the sparse forward, or, if a launch fails after the fork, when the forward returns,
+// so no work queued on the second stream outlives the call.  The join event is recorded on
+// the second stream by this guard (never a record left over from an earlier call: inside a
+// graph capture, a wait on an event recorded outside the capture would invalidate it).
 struct JoinGuard {
   SideStream* side = nullptr;
-  cudaStream_t st = nullptr;
-  bool done = true;
-  cudaError_t join() {
-    if (done || !side) return cudaSuccess;
-    done = true;
-    return cudaStreamWaitEvent(st, side->join, 0);
-  }
+  cudaStream_t caller = nullptr;
+  bool recorded = false, done = true;
   JoinGuard() = default;
-  JoinGuard(SideStream* s, cudaStream_t t, bool d) : side(s), st(t), done(d) {}
-  JoinGuard& operator=(const JoinGuard&) = default;
+  JoinGuard(const JoinGuard&) = delete;
+  JoinGuard& operator=(const JoinGuard&) = delete;
+  void arm(SideStream* s, cudaStream_t c) {
+    side = s;
+    caller = c;
+    recorded = false;
+    done = false;
+  }
+  cudaError_t record() {
+    if (done || recorded) return cudaSuccess;
+    recorded = true;
+    return cudaEventRecord(side->join, side->s);
+  }
+  cudaError_t join() {
+    if (done) return cudaSuccess;
+    cudaError_t e = record();
+    done = true;
+    return e != cudaSuccess ? e : cudaStreamWaitEvent(caller, side->join, 0);
+  }
   ~JoinGuard() {
     if (join() != cudaSuccess) cudaGetLastError();
   }
@@ -770,13 +783,13 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
     ELSAA_TRY(cuda_status(cudaEventRecord(side->fork, st_), "selection fork"));
     ELSAA_TRY(cuda_status(cudaStreamWaitEvent(side->s, side->fork, 0), "selection fork"));
     sel_st = side->s;
-    joined = JoinGuard{side, st_, false};
+    joined.arm(side, st_);
   }
   if (lsh)
     ELSAA_TRY(cuda_status(launch_diag_select(s.idx, g, sel_st), "selection"));
   else
     ELSAA_TRY(cuda_status(launch_select(Q, K, bf16, w.qbar, w.kbar, w.scores, s.idx, g, sel_st), "selection"));
-  if (side) ELSAA_TRY(cuda_status(cudaEventRecord(side->join, sel_st), "selection join"));
+  ELSAA_TRY(cuda_status(joined.record(), "selection join"));
   if (g.r > 0 && bf16) {
     ELSAA_TRY(cuda_status(launch_race_w_split(W, w.wsplit, g, st_), "W split"));
     ELSAA_TRY(cuda_status(launch_race_features_tc(Q, K, w.wsplit, s.phiQ, s.phiK, s.hQ, s.hK, s.nQ, s.nK, g, w.flag,
@@ -807,7 +820,7 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
       ELSAA_TRY(cuda_status(cudaMemsetAsync(s.Olr, 0, (size_t)g.BH * g.N * g.d * 2, st_), "O_lr"));
       ELSAA_TRY(cuda_status(cudaMemsetAsync(s.dlr, 0, (size_t)g.BH * g.N * 4, st_), "d_lr"));
     }
-    if (side) ELSAA_TRY(cuda_status(joined.join(), "selection join"));
+    ELSAA_TRY(cuda_status(joined.join(), "selection join"));
     FwdArgs at = a;
     if (lsh) {                        // the epilogue writes O straight into the caller's row order
       at.O = O_out;

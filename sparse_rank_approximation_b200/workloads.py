@@ -84,7 +84,7 @@ WORKLOADS = {
     # the headline shape with the causal sortLSH recursion (halves down to single blocks)
     "n16k_d128_sortlsh_causal": Workload("n16k_d128_sortlsh_causal", 1, 32, 16384, 128, "bf16", True, 128, 128, 2,
                                          n_centroids=256, sigma=0.5, selector="sortlsh", lsh_bits=7),
-    # config 3's shape (d = 64, block 64: the mma.sync kernels) with the causal sortLSH recursion
+    # config 3's shape (d = 64, blocks of 64) with the causal sortLSH recursion
     "n8k_d64_sortlsh_causal": Workload("n8k_d64_sortlsh_causal", 4, 16, 8192, 64, "bf16", True, 128, 64, 2,
                                        n_centroids=128, sigma=0.3, selector="sortlsh", lsh_bits=7),
     "n64k_d128": Workload("n64k_d128", 1, 8, 65536, 128, "bf16", True, 256, 128, 32,
