@@ -18,8 +18,8 @@
 //               that exchange their partial row max; online softmax in fp32 with lazy
 //               rescaling (O and l move only when the running max grows by more than
 //               2^16); P_j goes back over the score columns it came from as bf16 hi + lo
-//               pairs (16 significant bits, so O_s, and the backward's softmax delta formed
-//               from it, carry no bf16 rounding of the weights) and is the A operand of the
+//               pairs (hi + lo within 2^-15 of P, so O_s, and the backward's softmax delta
+//               formed from it, carry no bf16 rounding of the weights) and is the A operand of the
 //               two PV products; the epilogue normalises O, applies the fusion and writes O
 //               (TMA store from shared memory) and the fp32 O_s (row stores).
 // Operand tiles are 64-column slabs with 128-byte swizzle, as TMA writes them.
@@ -75,6 +75,17 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
+}
+
+// A pair (a, b) of non-negative floats as bf16 hi + lo pairs by truncation, with integer and
+// FMA instructions only: hi keeps the top 16 bits of each float (sign, exponent, 7 mantissa
+// bits), lo the top 16 bits of the exact remainder, so hi + lo is within 2^-15 of each value.
+// a sits in the low half of each word, b in the high half.
+__device__ __forceinline__ void split_trunc(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+  hi = __byte_perm(ua, ub, 0x7632);
+  const float ra = a - __uint_as_float(ua & 0xffff0000u), rb = b - __uint_as_float(ub & 0xffff0000u);
+  lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
 }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Misc* ms, uint32_t* err,
@@ -331,12 +342,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             uint32_t w[8], wl[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float p0 = ex2_approx(fmaf(sv[16 * q + 2 * e], sl2, -msub));
-              const float p1 = ex2_approx(fmaf(sv[16 * q + 2 * e + 1], sl2, -msub));
+              const float x0 = fmaf(sv[16 * q + 2 * e], sl2, -msub), x1 = fmaf(sv[16 * q + 2 * e + 1], sl2, -msub);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
               rs0 += p0;
               rs1 += p1;
-              w[e] = pack_bf16(p0, p1);
-              wl[e] = pack_bf16(p0 - __uint_as_float(w[e] << 16), p1 - __uint_as_float(w[e] & 0xffff0000u));
+              split_trunc(p0, p1, w[e], wl[e]);
             }
             const uint32_t col = tmem + lane_base + TM_S + 64 * half + 32 * part + 16 * q;
             tc::tmem_st8(col, w);
