@@ -11,8 +11,10 @@
 // bf16 hi + lo halves (two accumulating products: X is exact in bf16, W nearly exact).  Warp 0
 // issues the TMA loads, warp 1 owns TMEM and issues the products, warps 2-5 (one row per
 // thread, TMEM lane quarter = warp % 4) divide by the row norm (from the staged bf16 row), run
-// the corner probabilities and write Phi (bf16), the normalised projections h (fp32) and the
-// norm.  Every mbarrier wait is bounded; a timeout sets a bit in the caller's error word.
+// the corner probabilities, stage Phi (bf16, zero-padded to rp columns) over the operand tiles
+// the products no longer need and write it with TMA stores; the normalised projections h (fp32)
+// and the norm go out as row stores.  Every mbarrier wait is bounded; a timeout sets a bit in
+// the caller's error word.
 #include <cudaTypedefs.h>
 
 #include "kernels.h"
@@ -31,6 +33,7 @@ constexpr uint32_t F_WH = 2 * kSlab;              // W hi [NW][d], up to 2 slabs
 constexpr uint32_t kWSlab = kMaxNW * 128;
 constexpr uint32_t F_WL = F_WH + 2 * kWSlab;
 constexpr uint32_t F_BARS = F_WL + 2 * kWSlab;
+static_assert(F_BARS >= 4 * kSlab, "Phi staging: up to 256 columns over the X and W tiles");
 
 struct FeatBars {
   uint64_t in_full, acc_full;
@@ -53,13 +56,15 @@ __device__ __forceinline__ uint64_t desc_k(uint32_t base, int kk, uint32_t slab)
   return tc::sw128_desc(base + (uint32_t)(kk >> 2) * slab + (uint32_t)(kk & 3) * 32u, 16, 1024);
 }
 
+__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 128;\n" ::: "memory"); }
+
 }  // namespace
 
 template <int D, int NW>
 __global__ void __launch_bounds__(kThreads, 1)
     race_features_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                            const __grid_constant__ CUtensorMap tmW, __nv_bfloat16* __restrict__ phiQ,
-                            __nv_bfloat16* __restrict__ phiK, float* __restrict__ hQ, float* __restrict__ hK,
+                            const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPQ,
+                            const __grid_constant__ CUtensorMap tmPK, float* __restrict__ hQ, float* __restrict__ hK,
                             float* __restrict__ nQ, float* __restrict__ nK, Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   FeatBars* ms = reinterpret_cast<FeatBars*>(smem + F_BARS);
@@ -148,33 +153,49 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) hp[32 * q + e] = tmp[e];
       }
-      if (valid) {
-        __nv_bfloat16* phi = (side ? phiK : phiQ) + grow * g.rp;
-        float* hout = (side ? hK : hQ) + grow * (size_t)(4 * g.L);
-        const float inv_n = 1.f / n, inv_sqrt_L = rsqrtf((float)g.L), two_over_tau = 2.f / g.tau;
+      // Phi of this row into the staging tile (64-column slabs, 128-byte swizzle): the products
+      // have read X and W, and this thread alone has read X row i
+      float* hout = (side ? hK : hQ) + grow * (size_t)(4 * g.L);
+      const float inv_n = 1.f / n, inv_sqrt_L = rsqrtf((float)g.L), two_over_tau = 2.f / g.tau;
+      auto stage16 = [&](int col, const uint32_t (&w)[8]) {      // 16 bf16 at column col (multiple of 16)
+        unsigned char* base = smem + F_X + (uint32_t)(col >> 6) * kSlab + (uint32_t)i * 128u;
+        const int ch = (col & 63) >> 3;
+        *reinterpret_cast<uint4*>(base + ((ch ^ (i & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(base + (((ch + 1) ^ (i & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+      };
 #pragma unroll
-        for (int l = 0; l < NW / 4; ++l) {
-          if (l >= g.L) break;
-          float sp[kHashBits], sm[kHashBits], hv[kHashBits];
+      for (int l = 0; l < NW / 4; ++l) {
+        if (l >= g.L) break;
+        float sp[kHashBits], sm[kHashBits], hv[kHashBits];
 #pragma unroll
-          for (int b = 0; b < kHashBits; ++b) {
-            hv[b] = hp[4 * l + b] * inv_n;
-            sigmoid_pair(two_over_tau * hv[b], sp[b], sm[b]);   // P(c_b = +1), P(c_b = -1)
-          }
-          reinterpret_cast<float4*>(hout)[l] = make_float4(hv[0], hv[1], hv[2], hv[3]);
-          float pc[kCorners];
-          corner_probs(sp, sm, inv_sqrt_L, pc);
-          uint32_t w[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) w[e] = pack_bf16(pc[2 * e], pc[2 * e + 1]);
-          reinterpret_cast<uint4*>(phi + 16 * l)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          reinterpret_cast<uint4*>(phi + 16 * l)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        for (int b = 0; b < kHashBits; ++b) {
+          hv[b] = hp[4 * l + b] * inv_n;
+          sigmoid_pair(two_over_tau * hv[b], sp[b], sm[b]);   // P(c_b = +1), P(c_b = -1)
         }
-        // stored rows are padded to rp columns with zeros
-        for (int col = g.r; col < g.rp; col += 8)
-          *reinterpret_cast<uint4*>(phi + col) = make_uint4(0u, 0u, 0u, 0u);
-        (side ? nK : nQ)[grow] = n;
+        if (valid) reinterpret_cast<float4*>(hout)[l] = make_float4(hv[0], hv[1], hv[2], hv[3]);
+        float pc[kCorners];
+        corner_probs(sp, sm, inv_sqrt_L, pc);
+        uint32_t w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = pack_bf16(pc[2 * e], pc[2 * e + 1]);
+        stage16(16 * l, w);
       }
+      // stored rows are padded to rp columns with zeros
+      const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      for (int col = 16 * g.L; col < g.rp; col += 16) stage16(col, z);
+      if (valid) (side ? nK : nQ)[grow] = n;
+    }
+    // every row staged: one thread writes the tile (rows past N are dropped by the store)
+    tc::fence_proxy_async_smem();
+    compute_bar();
+    if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag) {
+      const CUtensorMap* map = side ? &tmPK : &tmPQ;
+      for (int sl = 0; sl < g.rp / 64; ++sl)
+        asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];\n"
+                     :: "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(smem + F_X + sl * kSlab)), "r"(64 * sl),
+                        "r"(c * kC), "r"(bh) : "memory");
+      asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+      asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
     }
   }
   __syncthreads();
@@ -187,9 +208,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, int NW>
 static cudaError_t features_t(const void* Q, const void* K, const void* wsplit, void* phiQ, void* phiK, float* hQ,
                               float* hK, float* nQ, float* nK, const Geom& g, uint32_t* err, cudaStream_t st) {
-  CUtensorMap mq, mk, mw;
+  CUtensorMap mq, mk, mw, mpq, mpk;
   if (!tc::map_rows_bf16_pitch(&mq, Q, D, D, g.N, g.BH, kC) || !tc::map_rows_bf16_pitch(&mk, K, D, D, g.N, g.BH, kC) ||
-      !tc::map_rows_bf16_pitch(&mw, wsplit, D, D, NW, 2, NW))
+      !tc::map_rows_bf16_pitch(&mw, wsplit, D, D, NW, 2, NW) ||
+      !tc::map_rows_bf16_pitch(&mpq, phiQ, g.rp, g.rp, g.N, g.BH, kC) ||
+      !tc::map_rows_bf16_pitch(&mpk, phiK, g.rp, g.rp, g.N, g.BH, kC))
     return cudaErrorInvalidValue;
   const size_t smem = F_BARS + sizeof(FeatBars);
   static_assert(F_BARS + sizeof(FeatBars) <= 232448, "shared memory per CTA");
@@ -197,8 +220,7 @@ static cudaError_t features_t(const void* Q, const void* K, const void* wsplit, 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps("race_features_tc", st);
-  kern<<<dim3(g.n_c, g.BH, 2), kThreads, smem, st>>>(mq, mk, mw, (__nv_bfloat16*)phiQ, (__nv_bfloat16*)phiK, hQ, hK,
-                                                     nQ, nK, g, err);
+  kern<<<dim3(g.n_c, g.BH, 2), kThreads, smem, st>>>(mq, mk, mw, mpq, mpk, hQ, hK, nQ, nK, g, err);
   return cudaGetLastError();
 }
 
@@ -207,7 +229,10 @@ cudaError_t launch_race_features_tc(const void* Q, const void* K, const void* ws
                                     float* hQ, float* hK, float* nQ, float* nK, const Geom& g, uint32_t* err,
                                     cudaStream_t st) {
   const int NW = (4 * g.L + 31) & ~31;
-  if ((g.d != 64 && g.d != 128) || NW > kMaxNW || g.C != kC || g.rp < g.r || g.rp % 8) return cudaErrorInvalidValue;
+  // Phi is staged as rp / 64 slabs over the 64 KB of operand tiles: rp = 128 (r <= 128) or 256
+  if ((g.d != 64 && g.d != 128) || NW > kMaxNW || g.C != kC || g.rp < g.r || (g.rp != 128 && g.rp != 256) ||
+      (g.rp == 256) != (NW == 64))
+    return cudaErrorInvalidValue;
   if (g.d == 64)
     return NW == 32 ? features_t<64, 32>(Q, K, wsplit, phiQ, phiK, hQ, hK, nQ, nK, g, err, st)
                     : features_t<64, 64>(Q, K, wsplit, phiQ, phiK, hQ, hK, nQ, nK, g, err, st);
