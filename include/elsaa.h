@@ -82,13 +82,15 @@ typedef enum { ELSAA_DTYPE_F32 = 0, ELSAA_DTYPE_BF16 = 1 } elsaa_dtype;
  * angular LSH (lsh_bits hyperplanes, bit c set when x . R_c > 0) and ordered by the
  * code's position in the reflected Gray sequence, then by row.
  *   causal = 0: the sorted queries and keys are cut into blocks of block_size and
- *     query block t attends key block t exactly.  N <= 16384, block_size 64 or 128.
+ *     query block t attends key block t exactly.  block_size 64 or 128.
  *   causal = 1: the paper's recursion ("For the causal setting", §3.2).  A segment
  *     splits on a block boundary into past and future halves (an odd block count
  *     gives the extra block to the past); each half recurses; the future queries
  *     attend the past keys by non-causal sortLSH on the two halves; the future
  *     half's results merge by log-sum-exp; a single block is attended exactly under
- *     j <= i.  Needs bf16 and N = block_size * 2^L <= 32768. */
+ *     j <= i.  Needs bf16 and N = block_size * 2^L.
+ *   Heads of up to 16384 rows (halves of up to 16384 rows in the recursion) are sorted
+ *   in shared memory, longer ones through global memory in the workspace. */
 typedef enum { ELSAA_SEL_TOPK_BLOCKS = 0, ELSAA_SEL_SORTLSH = 1 } elsaa_selector;
 
 typedef struct {
@@ -176,7 +178,9 @@ ELSAA_API elsaa_status elsaa_fusion_grads(const elsaa_params* params, const floa
  * inspection.  codes and order are int32 [B,H,2,N] (index 0: queries, 1: keys): codes
  * hold the lsh_bits-bit hash, order[.., s, p] the row at sorted position p of the whole
  * sequence (the causal recursion sorts each half-segment by the same key, so its orders
- * follow from the codes).  Needs no workspace; asynchronous on `stream`. */
+ * follow from the codes).  Needs no workspace; asynchronous on `stream`.  For N > 16384
+ * the sort goes through global memory: its scratch (2 B H 2 N int32) is allocated and
+ * freed on `stream` (stream-ordered; not for use inside a graph capture). */
 ELSAA_API elsaa_status elsaa_debug_sortlsh(const elsaa_params* params, const void* Q, const void* K,
                                            int32_t* codes, int32_t* order, void* stream);
 

@@ -117,11 +117,7 @@ bool make_geom(const elsaa_params* p, Geom* g, elsaa_status* st) {
         *st = fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH needs N = block_size * 2^L (got N = %d)", p->N);
         return false;
       }
-      if (p->N > 32768) { *st = fail(ELSAA_ERR_UNSUPPORTED, "causal sortLSH sorts halves in shared memory: N <= 32768"); return false; }
       while ((2 << lsh_levels) < n_t) ++lsh_levels;               // log2(n_t) - 1 sorted levels
-    } else if (p->N > 16384) {
-      *st = fail(ELSAA_ERR_UNSUPPORTED, "sortLSH sorts in shared memory: N <= 16384");
-      return false;
     }
     if ((long)p->B * p->H > 32767) { *st = fail(ELSAA_ERR_UNSUPPORTED, "sortLSH: B * H <= 32767"); return false; }
   }
@@ -300,6 +296,7 @@ struct FwdWs {
   float* scores;
   void* wsplit;
   float *lr_num, *lr_den;
+  int* lsh_scratch;        // sortLSH sorts longer than shared memory takes (else null)
   PermBufs pm;
 };
 
@@ -316,6 +313,8 @@ FwdWs carve_fwd_ws(void* base, const Geom& g, size_t esz, size_t* bytes) {
   w.lr_num = groups ? c.take<float>((size_t)g.BH * g.N * g.d) : nullptr;
   w.lr_den = groups ? c.take<float>((size_t)g.BH * g.N) : nullptr;
   w.pm = carve_perm(c, g, esz, false);
+  const size_t scr = sortlsh_scratch_ints(g);
+  w.lsh_scratch = scr ? c.take<int>(scr) : nullptr;
   *bytes = align_up(c.off);
   return w;
 }
@@ -492,7 +491,7 @@ ProfScope::~ProfScope() {
 
 // sortLSH: sort the rows, then gather the inputs into the sorted orders (queries by the
 // query order, keys and values by the key order, per-row vectors by the query order).
-elsaa_status lsh_gather(const elsaa_params* p, const Geom& g, bool bf16, const int* order, bool sort_first,
+elsaa_status lsh_gather(const elsaa_params* p, const Geom& g, bool bf16, const int* order, bool sort_first, int* scratch,
                         const void* Q, const void* K, const void* V, const void* X, const float* lam,
                         const float* gs, const float* glr, const PermBufs& b, cudaStream_t st) {
   const int row_bytes = g.d * (bf16 ? 2 : 4), stride = 2 * g.N;
@@ -500,7 +499,7 @@ elsaa_status lsh_gather(const elsaa_params* p, const Geom& g, bool bf16, const i
   const int* ok = order + g.N;
   if (sort_first)
     ELSAA_TRY(cuda_status(launch_sortlsh_order(Q, K, bf16, p->lsh_planes, p->lsh_bits, const_cast<int*>(order),
-                                               nullptr, g, st), "sortLSH order"));
+                                               nullptr, scratch, g, st), "sortLSH order"));
   ELSAA_TRY(cuda_status(launch_permute_rows(Q, b.Q, oq, row_bytes, g, stride, false, st), "sortLSH gather Q"));
   ELSAA_TRY(cuda_status(launch_permute_rows(K, b.K, ok, row_bytes, g, stride, false, st), "sortLSH gather K"));
   ELSAA_TRY(cuda_status(launch_permute_rows(V, b.V, ok, row_bytes, g, stride, false, st), "sortLSH gather V"));
@@ -580,7 +579,8 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
                           "sortLSH hash"));
     for (int lev = 0; lev < lv; ++lev)
       ELSAA_TRY(cuda_status(launch_sortlsh_level_sort(b.pos, s.lsh_order + (size_t)lev * g.BH * stride,
-                                                      b.inv + lev * rows, g.N >> (lev + 1), p->lsh_bits, g, st),
+                                                      b.inv + lev * rows, g.N >> (lev + 1), p->lsh_bits,
+                                                      w.lsh_scratch, g, st),
                             "sortLSH level sort"));
     // only the future halves' queries and the past halves' keys and values are read
     const void* qs[1] = {Q};
@@ -767,7 +767,7 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
     // the operator runs on the sorted rows (non-causal RACE, the fusion and diagonal-block
     // attention commute with row permutations); O is scattered back at the end
     ELSAA_TRY(check_ptr(p->lsh_planes, "lsh_planes"));
-    ELSAA_TRY(lsh_gather(p, g, bf16, s.lsh_order, true, Q, K, V, nullptr, lam, gs, glr, w.pm, st_));
+    ELSAA_TRY(lsh_gather(p, g, bf16, s.lsh_order, true, w.lsh_scratch, Q, K, V, nullptr, lam, gs, glr, w.pm, st_));
     Q = w.pm.Q; K = w.pm.K; V = w.pm.V; O = w.pm.X;
     if (lam) lam = w.pm.lam;
     if (gs) gs = w.pm.gs;
@@ -886,7 +886,7 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   if (lsh) {
     // the forward ran on the sorted rows and saved its state in that order; so does this,
     // and the gradients are scattered back at the end
-    ELSAA_TRY(lsh_gather(p, g, bf16, s.lsh_order, false, Q, K, V, dO, lam, gs, glr, w.pm, st_));
+    ELSAA_TRY(lsh_gather(p, g, bf16, s.lsh_order, false, nullptr, Q, K, V, dO, lam, gs, glr, w.pm, st_));
     Q = w.pm.Q; K = w.pm.K; V = w.pm.V; dO = w.pm.X;
     dQ = w.pm.dQ; dK = w.pm.dK; dV = w.pm.dV;
     if (lam) lam = w.pm.lam;
@@ -1009,9 +1009,18 @@ elsaa_status elsaa_debug_sortlsh(const elsaa_params* p, const void* Q, const voi
   ELSAA_TRY(check_ptr(p->lsh_planes, "lsh_planes"));
   ELSAA_TRY(check_ptr(order, "order"));
   ELSAA_TRY(check_ptr(codes, "codes", false));
-  return cuda_status(launch_sortlsh_order(Q, K, p->dtype == ELSAA_DTYPE_BF16, p->lsh_planes, p->lsh_bits, order,
-                                          codes, g, static_cast<cudaStream_t>(stream)),
-                     "sortLSH order");
+  // long heads sort through global memory: scratch allocated and freed on the stream
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  Geom gs = g;
+  gs.causal = 0;                       // the whole-sequence orders, as for the non-causal selector
+  const size_t scr_n = sortlsh_scratch_ints(gs);
+  int* scratch = nullptr;
+  if (scr_n) ELSAA_TRY(cuda_status(cudaMallocAsync(reinterpret_cast<void**>(&scratch), scr_n * 4, st_), "sortLSH scratch"));
+  const elsaa_status r = cuda_status(launch_sortlsh_order(Q, K, p->dtype == ELSAA_DTYPE_BF16, p->lsh_planes,
+                                                          p->lsh_bits, order, codes, scratch, gs, st_),
+                                     "sortLSH order");
+  if (scratch) cudaFreeAsync(scratch, st_);
+  return r;
 }
 
 elsaa_status elsaa_debug_set_wait_limit(unsigned long long wait_ns, int stall) {

@@ -85,10 +85,13 @@ struct BwdArgs {
 };
 
 // sortLSH selector: per head the sorted query and key orders, int32 [BH][2][N]
-// (codes, if not null, receive the hash codes in the same layout).
+// (codes, if not null, receive the hash codes in the same layout).  Heads longer than a
+// shared-memory sort takes (N > 16384) sort through global memory in `scratch`
+// (sortlsh_scratch_ints ints; null is refused there).
 cudaError_t launch_sortlsh_order(const void* Q, const void* K, bool bf16, const float* planes, int bits,
-                                 int* order, int* codes, const Geom& g, cudaStream_t st);
+                                 int* order, int* codes, int* scratch, const Geom& g, cudaStream_t st);
 size_t sortlsh_smem_bytes(const Geom& g, int bits);
+size_t sortlsh_scratch_ints(const Geom& g);
 // Hash only: Gray positions (and, if not null, codes) [BH][2][N].
 cudaError_t launch_sortlsh_hash(const void* Q, const void* K, bool bf16, const float* planes, int bits, int* pos,
                                 int* codes, const Geom& g, cudaStream_t st);
@@ -97,8 +100,8 @@ cudaError_t launch_sortlsh_hash(const void* Q, const void* K, bool bf16, const f
 // future-half rows' positions [BH][N]; the base-pass selection; the final
 // log-sum-exp merge of the partials with the fusion; the orders' inverses; the level
 // gradients collected into the fp32 accumulators; multi-tensor half-row gathers.
-cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int* inv, int h, int bits, const Geom& g,
-                                      cudaStream_t st);
+cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int* inv, int h, int bits, int* scratch,
+                                      const Geom& g, cudaStream_t st);
 cudaError_t launch_causal_lsh_select(int* idx, const Geom& g, cudaStream_t st);
 cudaError_t launch_lsh_fuse(const void* Os0, const float* logd0, const void* Os_lv, const float* logd_lv,
                             const int* inv_lv, int levels, const void* Olr, const float* dlr, const float* lam,

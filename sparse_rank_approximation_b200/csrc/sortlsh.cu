@@ -21,6 +21,7 @@ namespace elsaa {
 namespace {
 
 constexpr int kSortThreads = 1024;
+constexpr int kSmemSortRows = 16384;     // shared-memory sort: items packed (position << 14 | row)
 
 __device__ __forceinline__ uint32_t gray_position(uint32_t code) {
   uint32_t n = code;
@@ -194,6 +195,103 @@ __device__ uint32_t* block_counting_sort(uint32_t* bufA, uint32_t* bufB, int* cn
   return src;
 }
 
+// The same stable LSD counting sort for segments longer than shared memory holds
+// (n > kSmemSortRows): the rows move between two global buffers, 8 bits per pass; the
+// per-(digit, warp) counts stay in shared memory, scanned digit-major, warp-minor, and
+// equal digits within a warp are ranked by lane, so every pass is stable.  pos holds the
+// positions of the segment's rows (indexed from 0); the last pass writes first + row to
+// out and, if inv is not null, the sorted position first + at of every row to
+// inv[first + row].  tmp holds n ints.  Called by all kSortThreads threads.
+__device__ void global_counting_sort(const int* __restrict__ pos, int* __restrict__ tmp, int* __restrict__ out,
+                                     int* __restrict__ inv, int first, int n, int bits, int* cnt, int* wsum) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int slice = (n + 31) / 32;
+  const int r0 = warp * slice, r1 = min(n, r0 + slice);
+  const int passes = (bits + 7) / 8;
+  for (int p = 0; p < passes; ++p) {
+    const int shift = 8 * p;
+    const bool last = p == passes - 1;
+    const int* src = p == 0 ? nullptr : tmp;          // pass 0 reads the rows in order
+    int* dst = last ? nullptr : tmp;                  // (2 passes: rows -> tmp -> out)
+    for (int i = tid; i < 256 * 32; i += kSortThreads) cnt[i] = 0;
+    __syncthreads();
+    for (int base = r0; base < r1; base += 32) {
+      const int i = base + lane;
+      const bool live = i < r1;
+      const int r = live ? (src ? src[i] : i) : 0;
+      const uint32_t dig = live ? ((uint32_t)pos[r] >> shift) & 255u : 256u + lane;
+      const unsigned peers = __match_any_sync(0xffffffffu, dig);
+      if (live && lane == __ffs(peers) - 1) cnt[dig * 32 + warp] += __popc(peers);
+      __syncwarp();
+    }
+    __syncthreads();
+    {
+      int loc[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        loc[j] = cnt[8 * tid + j];
+        sum += loc[j];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      if (lane == 31) wsum[warp] = incl;
+      __syncthreads();
+      if (warp == 0) {
+        int w = wsum[lane], wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, wi, o);
+          if (lane >= o) wi += t;
+        }
+        wsum[lane] = wi - w;
+      }
+      __syncthreads();
+      int run = wsum[warp] + incl - sum;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[8 * tid + j] = run;
+        run += loc[j];
+      }
+    }
+    __syncthreads();
+    for (int base = r0; base < r1; base += 32) {
+      const int i = base + lane;
+      const bool live = i < r1;
+      const int r = live ? (src ? src[i] : i) : 0;
+      const uint32_t dig = live ? ((uint32_t)pos[r] >> shift) & 255u : 256u + lane;
+      const unsigned peers = __match_any_sync(0xffffffffu, dig);
+      if (live) {
+        const int at = cnt[dig * 32 + warp] + __popc(peers & ((1u << lane) - 1u));
+        if (last) {
+          out[at] = first + r;
+          if (inv) inv[first + r] = first + at;
+        } else {
+          dst[at] = r;
+        }
+      }
+      __syncwarp();
+      if (live && lane == __ffs(peers) - 1) cnt[dig * 32 + warp] += __popc(peers);
+      __syncwarp();
+    }
+    __syncthreads();
+  }
+}
+
+// Long heads (N > kSmemSortRows), grid (BH, 2): positions from `pos` ([BH][2][N]), the sorted
+// rows into `order`; tmp ([BH][2][N]) holds the pass in between.
+__global__ void __launch_bounds__(kSortThreads) sortlsh_sort_global_kernel(const int* __restrict__ pos,
+                                                                           int* __restrict__ order,
+                                                                           int* __restrict__ tmp, int bits, Geom g) {
+  __shared__ int cnt[256 * 32];
+  __shared__ int wsum[32];
+  const size_t off = ((size_t)blockIdx.x * 2 + blockIdx.y) * g.N;
+  global_counting_sort(pos + off, tmp + off, order + off, nullptr, 0, g.N, bits, cnt, wsum);
+}
+
 // One (head, side) per CTA, grid (BH, 2): reads its `order` segment (the Gray
 // positions) whole, then writes the sorted rows over it.
 __global__ void __launch_bounds__(kSortThreads) sortlsh_sort_kernel(int* __restrict__ order, int bits, Geom g) {
@@ -240,6 +338,24 @@ __global__ void __launch_bounds__(kSortThreads) sortlsh_level_sort_kernel(const 
   }
 }
 
+// The level sort for halves longer than shared memory holds (h > kSmemSortRows); tmp is
+// [BH][2][N] (each CTA uses its own half's range).
+__global__ void __launch_bounds__(kSortThreads) sortlsh_level_sort_global_kernel(const int* __restrict__ pos,
+                                                                                 int* __restrict__ order,
+                                                                                 int* __restrict__ inv,
+                                                                                 int* __restrict__ tmp, int h,
+                                                                                 int bits, Geom g) {
+  __shared__ int cnt[256 * 32];
+  __shared__ int wsum[32];
+  const int side = blockIdx.y, s = blockIdx.z;
+  const size_t off = ((size_t)blockIdx.x * 2 + side) * g.N;
+  const int sorted0 = (2 * s + (side == 0 ? 1 : 0)) * h;
+  const int ident0 = (2 * s + (side == 0 ? 0 : 1)) * h;
+  for (int i = threadIdx.x; i < h; i += kSortThreads) order[off + ident0 + i] = ident0 + i;
+  global_counting_sort(pos + off + sorted0, tmp + off + sorted0, order + off + sorted0,
+                       inv && side == 0 ? inv + (size_t)blockIdx.x * g.N : nullptr, sorted0, h, bits, cnt, wsum);
+}
+
 // Base-pass selection of the causal recursion (the caller's row order, causal): tile t
 // takes its own block and, when t is odd, block t - 1 (the deepest level, whose halves
 // are single blocks and need no sort); ascending, -1 padded, k = 2.
@@ -259,7 +375,7 @@ __global__ void causal_lsh_select_kernel(int* __restrict__ idx, Geom g) {
 // m = 1 / (1 + (lambda d_lr + eps) e^{-log d_s}) (1 when m is held), O = g_s m O_s + g_lr O_lr
 // with g_lr = 1 - m by default (1 when m is held).  Writes O, the saved fp32 O_s, log d_s
 // and m.  One thread per 8 columns; partials and the merge are fp32.
-constexpr int kMaxLevels = 8;             // N <= 32768 in blocks of >= 64 rows: at most 8 sorted levels
+constexpr int kMaxLevels = 10;            // n_t <= 1024 tiles: at most 9 sorted levels
 
 __global__ void lsh_fuse_kernel(const float* __restrict__ Os0, const float* __restrict__ logd0,
                                 const float* __restrict__ Os_lv, const float* __restrict__ logd_lv,
@@ -472,6 +588,14 @@ size_t sortlsh_smem_bytes(const Geom& g, int bits) {
   return (size_t)256 * 32 * 4 + (size_t)2 * g.N * 4;
 }
 
+size_t sortlsh_scratch_ints(const Geom& g) {
+  if (g.lsh_bits == 0) return 0;                  // not the sortLSH selector
+  // non-causal: positions and the pass buffer of the whole heads; causal: the pass buffer of
+  // the level sorts (their positions are computed once into the workspace)
+  if (!g.causal) return g.N > kSmemSortRows ? (size_t)2 * g.BH * 2 * g.N : 0;
+  return g.N / 2 > kSmemSortRows ? (size_t)g.BH * 2 * g.N : 0;
+}
+
 cudaError_t launch_sortlsh_hash(const void* Q, const void* K, bool bf16, const float* planes, int bits, int* pos,
                                 int* codes, const Geom& g, cudaStream_t st) {
   const size_t hsmem = (size_t)bits * g.d * 4;
@@ -493,8 +617,15 @@ cudaError_t launch_sortlsh_hash(const void* Q, const void* K, bool bf16, const f
   return cudaGetLastError();
 }
 
-cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int* inv, int h, int bits, const Geom& g,
-                                      cudaStream_t st) {
+cudaError_t launch_sortlsh_level_sort(const int* pos, int* order, int* inv, int h, int bits, int* scratch,
+                                      const Geom& g, cudaStream_t st) {
+  if (h > kSmemSortRows) {
+    if (!scratch) return cudaErrorInvalidValue;
+    ProfScope ps("sortlsh_level_sort", st);
+    sortlsh_level_sort_global_kernel<<<dim3(g.BH, 2, g.N / (2 * h)), kSortThreads, 0, st>>>(pos, order, inv, scratch,
+                                                                                            h, bits, g);
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)256 * 32 * 4 + (size_t)2 * h * 4;
   cudaError_t e = cudaFuncSetAttribute(sortlsh_level_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
@@ -562,7 +693,18 @@ cudaError_t launch_causal_lsh_select_levels(int* idx, int* tile_list, int levels
 }
 
 cudaError_t launch_sortlsh_order(const void* Q, const void* K, bool bf16, const float* planes, int bits,
-                                 int* order, int* codes, const Geom& g, cudaStream_t st) {
+                                 int* order, int* codes, int* scratch, const Geom& g, cudaStream_t st) {
+  if (g.N > kSmemSortRows) {
+    // long heads: positions into scratch, the sort through global memory
+    if (!scratch) return cudaErrorInvalidValue;
+    int* pos = scratch;
+    int* tmp = scratch + (size_t)g.BH * 2 * g.N;
+    const cudaError_t eh = launch_sortlsh_hash(Q, K, bf16, planes, bits, pos, codes, g, st);
+    if (eh != cudaSuccess) return eh;
+    ProfScope ps("sortlsh_sort", st);
+    sortlsh_sort_global_kernel<<<dim3(g.BH, 2), kSortThreads, 0, st>>>(pos, order, tmp, bits, g);
+    return cudaGetLastError();
+  }
   const cudaError_t eh = launch_sortlsh_hash(Q, K, bf16, planes, bits, order, codes, g, st);
   if (eh != cudaSuccess) return eh;
   const size_t smem = sortlsh_smem_bytes(g, bits);

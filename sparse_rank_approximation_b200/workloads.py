@@ -89,6 +89,10 @@ WORKLOADS = {
                                        n_centroids=128, sigma=0.3, selector="sortlsh", lsh_bits=7),
     "n64k_d128": Workload("n64k_d128", 1, 8, 65536, 128, "bf16", True, 256, 128, 32,
                           n_centroids=512, sigma=0.3),
+    # config 5's shape with the causal sortLSH recursion (eight sorted levels; the first
+    # level's halves of 32768 rows sort through global memory): 2^9 buckets for 512 blocks
+    "n64k_d128_sortlsh_causal": Workload("n64k_d128_sortlsh_causal", 1, 8, 65536, 128, "bf16", True, 256, 128, 2,
+                                         n_centroids=512, sigma=0.3, selector="sortlsh", lsh_bits=9),
 }
 HEADLINE = "n16k_d128"
 

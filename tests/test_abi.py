@@ -92,21 +92,19 @@ def test_status_strings():
 
 
 def test_sortlsh_shape_limits():
-    """sortLSH: non-causal up to N = 16384 on every path; the causal recursion needs bf16,
-    a power-of-two block count and N <= 32768."""
+    """sortLSH: any length up to 1024 tiles (heads or halves past 16384 rows sort through
+    global memory); the causal recursion needs bf16 and a power-of-two block count."""
     L = bd.lib()
     ok = dict(selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=6, topk=1)
-    assert L.elsaa_saved_bytes(ctypes.byref(bd.make_params(1, 2, 16384, 64, block_size=64, rank_r=16, causal=False,
-                                                           **ok))) > 0
-    assert L.elsaa_saved_bytes(ctypes.byref(bd.make_params(1, 2, 16384, 128, block_size=128, rank_r=128, causal=True,
-                                                           **ok))) > 0
-    assert L.elsaa_saved_bytes(ctypes.byref(bd.make_params(1, 2, 32768, 64, block_size=64, rank_r=16, causal=True,
-                                                           **ok))) > 0
-    bad = [dict(N=32768, d=64, block_size=64, causal=False),
+    for n, d, t, causal in ((16384, 64, 64, False), (65536, 64, 64, False), (16384, 128, 128, True),
+                            (32768, 64, 64, True), (65536, 128, 128, True), (131072, 128, 128, True)):
+        p = bd.make_params(1, 2, n, d, block_size=t, rank_r=128 if t == 128 else 16, causal=causal, **ok)
+        assert L.elsaa_saved_bytes(ctypes.byref(p)) > 0, (n, d, t, causal)
+    bad = [dict(N=64 * 1025, d=64, block_size=64, causal=False),
            dict(N=64 * 6, d=64, block_size=64, causal=True),
            dict(N=128 * 6, d=128, block_size=128, causal=True),
            dict(N=1024, d=128, block_size=128, causal=True, dtype=bd.ELSAA_DTYPE_F32),
-           dict(N=65536, d=128, block_size=128, causal=True)]
+           dict(N=128 * 2048, d=128, block_size=128, causal=True)]
     for kw in bad:
         p = bd.make_params(1, 1, kw.pop("N"), kw.pop("d"), rank_r=128 if kw["block_size"] == 128 else 16, **kw, **ok)
         assert L.elsaa_saved_bytes(ctypes.byref(p)) == 0, kw

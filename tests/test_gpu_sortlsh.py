@@ -128,6 +128,58 @@ def test_full_size():
         check(w, f"dV[{h}]", np64(dV[0, h]), dv)
 
 
+@pytest.mark.parametrize("N", [20000, 65536])
+def test_long_heads_sort_through_global_memory(N):
+    """Heads longer than a shared-memory sort takes (N > 16384) are sorted through global
+    memory, one 8-bit pass after another: the orders are permutations sorted by the Gray
+    position of the GPU's own codes, ties by row, and equal the oracle's where the codes agree."""
+    w = small_workload(N=N, d=64, block_size=64, topk=1, rank_r=16, causal=False, dtype="bf16", H=1)
+    inp = make_inputs(w, 5)
+    dev = device_inputs(w, inp)
+    R = torch.randn(w.d, 12, generator=torch.Generator().manual_seed(12))
+    op = gpu_op(w, selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=12, lsh_planes=R.cuda())
+    codes, order = op.debug_sortlsh(dev["Q"], dev["K"])
+    torch.cuda.synchronize()
+    Rn = R.double().numpy()
+    for side, name in ((0, "Q"), (1, "K")):
+        got = codes[0, 0, side].cpu().numpy()
+        o = order[0, 0, side].cpu().numpy()
+        assert np.array_equal(np.sort(o), np.arange(w.N))
+        pos = orc.gray_rank(got)[o]
+        assert np.all(np.diff(pos) >= 0) and np.all(np.diff(o)[np.diff(pos) == 0] > 0)
+        X = inp[name][0, 0].double().numpy()
+        if np.array_equal(got, orc.simhash_codes(X, Rn)):
+            assert np.array_equal(o, orc.sortlsh_order(X, Rn))
+
+
+def test_long_forward_backward():
+    """Non-causal sortLSH at N = 32768 (its sort goes through global memory): every row of one
+    head's O, and dQ on every 16th sorted query block, against the oracle on the GPU's orders (sparse
+    branch only: the low-rank branch does not depend on the length of the sort, and the oracle's
+    at this length takes minutes)."""
+    w = small_workload(N=32768, d=128, block_size=128, topk=1, rank_r=0, causal=False, dtype="bf16", H=1)
+    inp = make_inputs(w, 2)
+    dev = device_inputs(w, inp)
+    R = torch.randn(w.d, 8, generator=torch.Generator().manual_seed(3))
+    op = gpu_op(w, selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=8, lsh_planes=R.cuda())
+    O = op.forward(dev["Q"], dev["K"], dev["V"], dev["W"])
+    dQ, dK, dV = op.backward(dev["Q"], dev["K"], dev["V"], dev["W"], dev["dO"])
+    _, order = op.debug_sortlsh(dev["Q"], dev["K"])
+    assert op.check_device_flags() == 0
+    torch.cuda.synchronize()
+    W = inp["W"].double().numpy()
+    get = lambda n: inp[n][0, 0].double().numpy()
+    p = _oracle_params(w, R, (order[0, 0, 0].cpu().numpy(), order[0, 0, 1].cpu().numpy()))
+    fw = orc.forward_head(get("Q"), get("K"), get("V"), W, p)
+    check(w, "O", np64(O[0, 0]), fw["O"])
+    # dQ of a row comes from that row's support alone: every 16th sorted query block, all its rows
+    tiles = list(range(0, w.n_tiles, 16))
+    dq, _, _ = orc.backward_head(get("Q"), get("K"), get("V"), W, get("dO"), fw, p, tiles=tiles)
+    oq = p.lsh_orders[0]
+    rows = np.concatenate([oq[t * w.block_size:(t + 1) * w.block_size] for t in tiles])
+    check(w, "dQ", np64(dQ[0, 0])[rows], dq[rows])
+
+
 # ---- the causal recursion (bf16, d = 128, block 128 on the tensor-core kernels) ----
 
 def _causal_setup(N, r, seed, fixed_m=False, bits=6, H=2, d=128, T=128):
@@ -216,6 +268,28 @@ def test_causal_forward_backward(N, r, gates, fixed_m, d, T):
         check(w, f"dV[{h}]", np64(dV[0, h]), dv)
         ref = orc.fusion_param_grads(get("dO"), fw, p, ex.get("lam"), ex.get("g_s"), ex.get("g_lr"))
         check_fusion_grads(w, h, p, fw, ex, get("dO"), (dl, dgs, dgl), ref)
+
+
+def test_causal_long_halves_sort_through_global_memory():
+    """The causal recursion at N = 65536 (8 sorted levels; the first level's halves of 32768
+    rows sort through global memory): one head's O, and dQ on every 16th query tile, against the
+    oracle on the GPU's codes (sparse branch only, as in the long non-causal test)."""
+    w, inp, dev, R, op = _causal_setup(65536, 0, seed=6, bits=7, H=1)
+    O = op.forward(dev["Q"], dev["K"], dev["V"], dev["W"])
+    dQ, dK, dV = op.backward(dev["Q"], dev["K"], dev["V"], dev["W"], dev["dO"])
+    codes, _ = op.debug_sortlsh(dev["Q"], dev["K"])
+    assert op.check_device_flags() == 0
+    torch.cuda.synchronize()
+    W = inp["W"].double().numpy()
+    get = lambda n: inp[n][0, 0].double().numpy()
+    p = _causal_oracle_params(w, R, codes, 0)
+    fw = orc.forward_head(get("Q"), get("K"), get("V"), W, p)
+    check(w, "O", np64(O[0, 0]), fw["O"])
+    # dQ of a row comes from that row's support alone: every 16th query tile, all its rows
+    tiles = list(range(0, w.n_tiles, 16))
+    dq, _, _ = orc.backward_head(get("Q"), get("K"), get("V"), W, get("dO"), fw, p, tiles=tiles)
+    rows = np.concatenate([np.arange(t * w.block_size, min(w.N, (t + 1) * w.block_size)) for t in tiles])
+    check(w, "dQ", np64(dQ[0, 0])[rows], dq[rows])
 
 
 def test_causal_full_size():
