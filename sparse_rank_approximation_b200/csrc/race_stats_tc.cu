@@ -18,9 +18,12 @@
 //            running value goes out as that chunk's bf16 hi + lo tiles (TMA stores) and
 //            mass.  No per-chunk fp32 prefix is ever written.
 // S_c = Phi_c^T Y_c is one M = r, N = d, K = C product with both operands MN-major, as
-// TMA writes the [C rows][r] and [C rows][d] tiles.
+// TMA writes the [C rows][r] and [C rows][d] tiles; the mass Phi_c^T w_c is a second, N = 16
+// product against a K-major tile whose rows 0 and 1 hold w as bf16 hi and lo (the rest zero),
+// so the mass carries w to 16 significant bits.
 // Warps: 0 TMA producer, 1 TMEM owner and MMA issuer, 2-9 (256 threads) compute: TMEM
-// lane quarter = warp % 4 (bucket row f of the statistics), column half = (warp - 2) / 4.
+// lane quarter = warp % 4 (bucket row f of the statistics), column half = (warp - 2) / 4;
+// the first 128 of them write the chunk's weight tile.
 // Every mbarrier wait is bounded; a timeout sets a bit in the caller's error word, the CTA
 // drains its copies and products, frees its tensor memory and exits.
 #include <cudaTypedefs.h>
@@ -33,7 +36,6 @@ namespace elsaa {
 namespace {
 
 constexpr int kC = 128;                           // chunk rows
-constexpr int kD = 128;                           // widest head dimension (slot sizes)
 constexpr int kR = 128;                           // buckets (r = 16 L)
 constexpr uint32_t kSlab = 128 * 128;             // [128 rows][64 bf16], 128-byte swizzle
 constexpr uint32_t kTile = 2 * kSlab;             // [128 rows][128 bf16]
@@ -41,6 +43,7 @@ constexpr int kThreads = 320;
 constexpr int kComputeThreads = 256;
 constexpr int kMaxStages = 3;
 
+constexpr uint32_t kWTile = 2 * 16 * 128;         // weight tile: [16 rows][128 rows of the chunk], K-major
 template <bool EMIT>
 struct StatsLayout {
   static constexpr int stages = EMIT ? 2 : 3;     // emit keeps 64 KB of staging for the stores
@@ -48,12 +51,16 @@ struct StatsLayout {
   static constexpr uint32_t y(int s) { return phi(s) + kTile; }
   static constexpr uint32_t hi = (uint32_t)stages * 2 * kTile;       // staging of the outgoing tiles
   static constexpr uint32_t lo = hi + kTile;
-  static constexpr uint32_t wts = EMIT ? lo + kTile : hi;            // row weights [stages][128] and
-  static constexpr uint32_t bars = wts + (kMaxStages * 128 + 256) * 4;   // mass partials [2][128]
+  static constexpr uint32_t wt0 = EMIT ? lo + kTile : hi;            // weight tiles [stages]
+  static constexpr uint32_t wt(int s) { return wt0 + (uint32_t)s * kWTile; }
+  static constexpr uint32_t bars = wt0 + (uint32_t)kMaxStages * kWTile;
+  // TMEM: the S accumulator(s) at 0 (and 128), the mass accumulator(s) after them
+  static constexpr uint32_t tmem_cols = EMIT ? 512 : 256;
+  static constexpr uint32_t mass_col(int b) { return (EMIT ? 256u : 128u) + 16u * b; }
 };
 
 struct StatBars {
-  uint64_t full[kMaxStages], empty[kMaxStages], x_full[2], x_free[2], drain;
+  uint64_t full[kMaxStages], empty[kMaxStages], w_full[kMaxStages], x_full[2], x_free[2], drain;
   unsigned long long limit_ns;
   uint32_t tmem_base;
   int abort_flag;
@@ -73,6 +80,11 @@ __device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 256;\n
 // MN-major operand: K = 16 rows per step, 64-element M (or N) atoms `slab` bytes apart.
 __device__ __forceinline__ uint64_t desc_mn(uint32_t base, int kk) {
   return tc::sw128_desc(base + (uint32_t)kk * 2048u, kSlab, 1024);
+}
+
+// K-major operand, K = 16 step kk of a tile of 128-byte rows kept as 64-column slabs.
+__device__ __forceinline__ uint64_t desc_k(uint32_t base, int kk, uint32_t slab) {
+  return tc::sw128_desc(base + (uint32_t)(kk >> 2) * slab + (uint32_t)(kk & 3) * 32u, 16, 1024);
 }
 
 // bf16 element (row, col) of a [128][128] tile kept as two 64-column slabs with the 128-byte swizzle.
@@ -108,8 +120,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NS = Lay::stages;
   extern __shared__ __align__(1024) unsigned char smem[];
   StatBars* ms = reinterpret_cast<StatBars*>(smem + Lay::bars);
-  float* sW = reinterpret_cast<float*>(smem + Lay::wts);          // [NS][128]
-  float* sM = sW + kMaxStages * 128;                                // [2][128]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int seg = blockIdx.x, bh = blockIdx.y;
   const int c_begin = seg * g.seg, c_end = min(g.n_c, c_begin + g.seg);
@@ -125,7 +135,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       tc::mbar_init(&ms->full[s], 1);
-      tc::mbar_init(&ms->empty[s], 1 + kComputeThreads);   // the products' commit and every mass reader
+      tc::mbar_init(&ms->empty[s], 1);                     // the products' commit
+      tc::mbar_init(&ms->w_full[s], 128);                  // the weight tile's 128 writers
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&ms->x_full[b], 1);
@@ -136,8 +147,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ms->abort_flag = 0;
     tc::fence_barrier_init();
   }
+  // weight tiles: rows 2-15 stay zero (rows 0 and 1 are rewritten for every chunk)
+  for (int i = threadIdx.x; i < (int)(NS * kWTile / 16); i += kThreads)
+    reinterpret_cast<uint4*>(smem + Lay::wt0)[i] = make_uint4(0u, 0u, 0u, 0u);
   if (warp == 1) {
-    tc::tmem_alloc(&ms->tmem_base, 256);
+    tc::tmem_alloc(&ms->tmem_base, Lay::tmem_cols);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
@@ -167,16 +181,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- MMA issuer: S_c = Phi_c^T Y_c ----------------
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(128, D, true, true);    // A = Phi^T and B = Y, both MN-major
+      const uint32_t idm = tc::idesc_bf16(128, 16, true, false);    // A = Phi^T, B = the weight tile (K-major)
       const uint32_t sb = smem_u32(smem);
       for (int s = 0; s < n_load; ++s) {
         const int st = s % NS, buf = EMIT ? (s & 1) : 0;
         if (!wait_or_abort(&ms->full[st], (s / NS) & 1, ms, err, 0x200000u)) break;
+        if (!wait_or_abort(&ms->w_full[st], (s / NS) & 1, ms, err, 0x200000u)) break;
         if (EMIT && s >= 2 && !wait_or_abort(&ms->x_free[buf], ((s >> 1) - 1) & 1, ms, err, 0x400000u)) break;
         tc::tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kC / 16; ++kk)
-          tc::mma_bf16(tmem + 128u * buf, desc_mn(sb + Lay::phi(st), kk), desc_mn(sb + Lay::y(st), kk), idesc,
-                       (EMIT ? kk > 0 : (s > 0 || kk > 0)) ? 1u : 0u);
+        for (int kk = 0; kk < kC / 16; ++kk) {
+          const uint32_t acc = (EMIT ? kk > 0 : (s > 0 || kk > 0)) ? 1u : 0u;
+          tc::mma_bf16(tmem + 128u * buf, desc_mn(sb + Lay::phi(st), kk), desc_mn(sb + Lay::y(st), kk), idesc, acc);
+          tc::mma_bf16(tmem + Lay::mass_col(buf), desc_mn(sb + Lay::phi(st), kk), desc_k(sb + Lay::wt(st), kk, 2048u),
+                       idm, acc);
+        }
         tc::mma_commit(&ms->empty[st]);
         if (EMIT) tc::mma_commit(&ms->x_full[buf]);
       }
@@ -239,25 +258,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!accumulate) continue;
       const int st = s % NS;
-      // the chunk's row weights (zero past the last row)
+      // the chunk's weight tile (rows 0 and 1: w as bf16 hi and lo, zero past the last row),
+      // once the products that read this stage's previous tile are done
       if (ct < kC) {
+        if (s >= NS && alive)
+          alive = wait_or_abort(&ms->empty[st], ((s / NS) - 1) & 1, ms, err, 0x800000u);
         const int row = c * kC + ct;
-        sW[st * 128 + ct] = row < g.N ? (w ? w[head + row] : 1.f) : 0.f;
+        const float wv = row < g.N ? (w ? w[head + row] : 1.f) : 0.f;
+        const __nv_bfloat16 whi = __float2bfloat16_rn(wv);
+        const __nv_bfloat16 wlo = __float2bfloat16_rn(wv - __bfloat162float(whi));
+        unsigned char* t = smem + Lay::wt(st) + (uint32_t)(ct >> 6) * 2048u;
+        const uint32_t cb = (uint32_t)(((ct & 63) >> 3) << 4) + (uint32_t)(ct & 7) * 2u;
+        *reinterpret_cast<__nv_bfloat16*>(t + 0 * 128 + (cb ^ (0u << 4))) = whi;
+        *reinterpret_cast<__nv_bfloat16*>(t + 1 * 128 + (cb ^ (1u << 4))) = wlo;
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(&ms->w_full[st]);
       }
-      compute_bar();
-      if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->full[st], (s / NS) & 1, ms, err, 0x800000u));
-      // mass of bucket f over this thread's 64 rows of the chunk (Phi read from the staged tile)
-      float part = 0.f;
-      if (alive) {
-        const unsigned char* tile = smem + Lay::phi(st);
-#pragma unroll 8
-        for (int j = 64 * hc; j < 64 * hc + 64; ++j) {
-          const __nv_bfloat16 p = *reinterpret_cast<const __nv_bfloat16*>(tile + sw_off(j, f));
-          part = fmaf(__bfloat162float(p), sW[st * 128 + j], part);
-        }
-        tc::mbar_arrive(&ms->empty[st]);
-      }
-      sM[hc * 128 + f] = part;
       if (EMIT && alive) {
         const int buf = s & 1;
         alive = __all_sync(0xffffffffu, wait_or_abort(&ms->x_full[buf], (s >> 1) & 1, ms, err, 0x1000000u));
@@ -271,12 +287,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) run[32 * h2 + i] += x[i];
           }
+          float m2[16];
+          tc::tmem_ld16(tmem + lane_base + Lay::mass_col(buf), m2);
+          tc::tmem_wait_ld();
+          run_mass += m2[0] + m2[1];
           tc::tc_fence_before();
           tc::mbar_arrive(&ms->x_free[buf]);
         }
       }
-      compute_bar();
-      run_mass += sM[f] + sM[128 + f];
     }
     if (!EMIT) {
       // the segment's total: S from tensor memory, the mass from the CUDA cores
@@ -300,7 +318,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
         }
         if (hc == 0) {
-          o[D] = run_mass;
+          float m2[16];
+          if (n_here > 0) {
+            tc::tmem_ld16(tmem + lane_base + Lay::mass_col(0), m2);
+            tc::tmem_wait_ld();
+          } else {
+            m2[0] = m2[1] = 0.f;
+          }
+          o[D] = m2[0] + m2[1];
           for (int e = D + 1; e < g.dp; ++e) o[e] = 0.f;
         }
       }
@@ -311,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, 256);
+    tc::tmem_dealloc(tmem, Lay::tmem_cols);
   }
 }
 
