@@ -7,15 +7,16 @@
 // plus the low-rank gradient parts accumulated in fp32 by the RACE backward.
 //
 // dq kernel: one CTA per (head, query tile); Q and dO stay in shared memory, the
-// selected K/V blocks stream through a 2-stage TMA ring; S = Q K^T and dP = dO V^T
-// land in TMEM, 8 softmax warps form dS (bf16, swizzled K-major) in shared memory,
-// and dQ += dS K accumulates in TMEM.
+// selected K and V blocks stream through TMA rings (3 and 2 stages); S = Q K^T and
+// dP = dO V^T land in TMEM, 8 softmax warps write dS as bf16 pairs into one of two
+// TMEM buffers, and dQ += dS K (dS as the tensor-memory operand) accumulates in TMEM.
 // dkdv kernel: one CTA per (head, key block); K and V stay in shared memory, the
-// query tiles that selected the block (ascending, from the selection inverse)
-// stream in halves of 64 queries through a 3-stage ring together with their
-// per-row scalars; S^T = K Q^T and dP^T = V dO^T land in double-buffered TMEM,
-// the softmax warps form (P^T cs) and dS^T, and dV += (P^T cs) dO, dK += dS^T Q
-// accumulate in TMEM.  No atomics: the results are deterministic.
+// query tiles that selected the block (from the selection inverse) stream through a
+// 2-stage ring together with their per-row scalars; S^T = K Q^T and dP^T = V dO^T
+// land in TMEM, the softmax warps write (P^T cs) and dS^T back over them as bf16 in
+// two passes of 64 queries, and dV += (P^T cs) dO, dK += dS^T Q accumulate in TMEM
+// after each pass.  The low-rank parts are brought into L2 once every load is issued
+// and read while the last products run.  No atomics: the results are deterministic.
 // Every mbarrier wait is bounded; a timeout sets a bit in the caller's error word,
 // the CTA drains its copies and MMAs, frees TMEM and exits.
 #include <cudaTypedefs.h>
@@ -187,6 +188,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
         issued = j + 1;
       }
+      // every load is issued: bring the tile's low-rank dQ rows into L2 for the epilogue
+      if (kside && a.dQacc && row0 < g.N)
+        tc::prefetch_l2(a.dQacc + (head + row0) * D, (uint32_t)min(kT, g.N - row0) * D * 4u);
       if (kside) tc::mbar_wait(&ms->qd_full, 0);
       for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j) tc::mbar_wait(&full[j % NS], (j / NS) & 1);
     }
@@ -298,15 +302,21 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       tc::mbar_arrive(&ms->ds_full[j & 1]);
     }
     // ---------------- epilogue: dQ = scale dQ_sparse + dQ_lowrank, bf16 TMA store ----------------
+    const int col0 = H * half;                       // this thread's dQ columns [col0, col0 + H)
+    // the low-rank part is read while the last products run
+    const bool use_acc = alive && row_ok && a.dQacc;
+    float4 av[H / 4];
+    if (use_acc) {
+      const float4* acc = reinterpret_cast<const float4*>(a.dQacc + (head + qrow) * D + col0);
+#pragma unroll
+      for (int i = 0; i < H / 4; ++i) av[i] = acc[i];
+    }
     bool have = false;
     if (alive && n_sel > 0) {
       alive = __all_sync(0xffffffffu, wait_or_abort(&ms->done, 0, ms, err, 256u));
       have = alive;
       if (have) tc::tc_fence_after();
     }
-    const int col0 = H * half;                       // this thread's dQ columns [col0, col0 + H)
-    const float4* acc =
-        alive && row_ok && a.dQacc ? reinterpret_cast<const float4*>(a.dQacc + (head + qrow) * D + col0) : nullptr;
     // every product has completed: stage the bf16 tile in the Q buffer, 32 columns at a time
     // (with a row map, write each row straight to the caller's row instead)
     unsigned char* orow = smem + DQ_Q + (col0 >> 6) * kSlab + row * 128;
@@ -315,7 +325,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                       ? reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dQ) +
                                                  (head + a.q_rows[(size_t)bh * a.rows_stride + qrow]) * D + col0)
                       : nullptr;
-#pragma unroll 1
+#pragma unroll
     for (int c = 0; c < H / 32; ++c) {
       float o[32];
 #pragma unroll
@@ -326,10 +336,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] *= g.scale;
       }
-      if (acc) {
+      if (use_acc && alive) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const float4 v = acc[8 * c + q];
+          const float4 v = av[8 * c + q];
           o[4 * q] += v.x; o[4 * q + 1] += v.y; o[4 * q + 2] += v.z; o[4 * q + 3] += v.w;
         }
       }
@@ -526,6 +536,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         }
         issued = u + 1;
       }
+      // every load is issued: bring the block's low-rank dK and dV rows into L2 for the epilogue
+      for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
+        const int kr = PAIR ? 64 * pb[h] : key0;
+        if ((PAIR && pb[h] < 0) || kr >= g.N) continue;
+        const uint32_t bytes = (uint32_t)min(TB, g.N - kr) * D * 4u;
+        if (a.dKacc) tc::prefetch_l2(a.dKacc + (head + kr) * D, bytes);
+        if (a.dVacc) tc::prefetch_l2(a.dVacc + (head + kr) * D, bytes);
+      }
       tc::mbar_wait(&ms->kv_full, 0);
       for (int u = (issued > kStages ? issued - kStages : 0); u < issued; ++u)
         tc::mbar_wait(&ms->qd_full[u % kStages], (u / kStages) & 1);
@@ -629,6 +647,16 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     const int hq = grp;
     const int col0 = H * hq;                         // this thread's columns [col0, col0 + H)
     const int ch0 = (col0 & 63) >> 3;
+    // the low-rank dK part is read while the last products run, dV's (from L2) once dK is staged
+    float4 av[H / 4];
+    auto load_acc = [&](const float* accp) {
+      if (accp && alive && key_ok) {
+        const float4* p = reinterpret_cast<const float4*>(accp + (head + (size_t)krow) * D + col0);
+#pragma unroll
+        for (int i = 0; i < H / 4; ++i) av[i] = p[i];
+      }
+    };
+    load_acc(a.dKacc);
     bool have = false;
     if (alive && n_u > 0) {
       alive = __all_sync(0xffffffffu, wait_or_abort(&ms->done, 0, ms, err, 512u));
@@ -636,13 +664,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       if (have) tc::tc_fence_after();
     }
     // every product has completed: stage dK in the stage-0 Q buffer and dV in the stage-0 dO buffer
-#pragma unroll 1
+#pragma unroll
     for (int which = 0; which < 2; ++which) {
       const float mul = which == 0 ? g.scale : 1.f;
-      const float* accp = which == 0 ? a.dKacc : a.dVacc;
-      const float4* ak = accp && alive && key_ok
-                             ? reinterpret_cast<const float4*>(accp + (head + (size_t)krow) * D + col0)
-                             : nullptr;
+      const bool use_acc = (which == 0 ? a.dKacc : a.dVacc) && alive && key_ok;
+      if (which == 1) load_acc(a.dVacc);
       unsigned char* orow = smem + (which == 0 ? kv_q(0) : kv_do(0)) + (col0 >> 6) * kSlab + row * 128;
       // with a row map, write each key row straight to the caller's row instead
       uint4* grow = a.k_rows && key_ok && alive
@@ -651,7 +677,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                                                    col0)
                         : nullptr;
       // 32 columns at a time: TMEM -> scale -> + low-rank part -> bf16 -> swizzled row
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < H / 32; ++c) {
         float o[32];
 #pragma unroll
@@ -662,10 +688,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= mul;
         }
-        if (ak) {
+        if (use_acc) {
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const float4 x = ak[8 * c + q];
+            const float4 x = av[8 * c + q];
             o[4 * q] += x.x; o[4 * q + 1] += x.y; o[4 * q + 2] += x.z; o[4 * q + 3] += x.w;
           }
         }
