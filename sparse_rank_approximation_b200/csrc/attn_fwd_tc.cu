@@ -225,6 +225,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t idS = tc::idesc_bf16(128, 128, false, false);   // Q (K-major) x K (K-major)
       const uint32_t idPV = tc::idesc_bf16(128, D, false, true);     // P (TMEM) x V (MN-major)
       const uint32_t sbase = smem_u32(smem);
+      // operand descriptors built once; a K step or a ring stage only moves the start address
+      const uint64_t q_desc = tc::sw128_desc(sbase + L::kQ, 16, 1024);
+      const uint64_t k_desc = tc::sw128_desc(sbase + L::k(0), 16, 1024);
+      const uint64_t v_desc = tc::sw128_desc(sbase + L::v(0), kSlab, 1024);   // V as the MN-major B of P V
       bool ok = wait_or_abort(&ms->q_full, 0, ms, err, 2u);
       // S_j overwrites P_{j-1}: the PV product that reads it was issued earlier, and tcgen05
       // MMAs of one thread run in issue order
@@ -232,12 +236,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int s = j % KS;
         if (!wait_or_abort(&ms->k_full[s], (j / KS) & 1, ms, err, 8u)) break;
         tc::tc_fence_after();
-        const uint32_t kb = sbase + L::k(s);
+        const uint64_t kb = tc::desc_adv(k_desc, L::k(s) - L::k(0));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = tc::sw128_desc(sbase + L::kQ + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::sw128_desc(kb + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
-          tc::mma_bf16(tmem + TM_S, ad, bd, idS, kk > 0 ? 1u : 0u);
+          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+          tc::mma_bf16(tmem + TM_S, tc::desc_adv(q_desc, off), tc::desc_adv(kb, off), idS, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(&ms->s_full);
         tc::mma_commit(&ms->k_empty[s]);
@@ -245,10 +248,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!wait_or_abort(&ms->p_full, j & 1, ms, err, 4u)) break;
         if (!wait_or_abort(&ms->v_full[s], (j / KS) & 1, ms, err, 1024u)) break;
         tc::tc_fence_after();
-        const uint32_t vb = sbase + L::v(s);
+        const uint64_t vb = tc::desc_adv(v_desc, L::v(s) - L::v(0));
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk) {
-          const uint64_t bd = tc::sw128_desc(vb + kk * 2048, kSlab, 1024);
+          const uint64_t bd = tc::desc_adv(vb, kk * 2048);
           const uint32_t pa = tmem + TM_S + p_col(kk);
           tc::mma_bf16_ts(tmem + TM_O, pa, bd, idPV, (j > 0 || kk > 0) ? 1u : 0u);
           tc::mma_bf16_ts(tmem + TM_O, pa + kPLo, bd, idPV, 1u);

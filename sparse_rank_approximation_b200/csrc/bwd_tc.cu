@@ -200,18 +200,23 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);   // both operands K-major
       const uint32_t idNM = tc::idesc_bf16(128, D, false, true);      // B MN-major, N = D
       const uint32_t sb = smem_u32(smem);
+      // operand descriptors built once; a K step or a ring stage only moves the start address
+      const uint64_t q_desc = tc::sw128_desc(sb + DQ_Q, 16, 1024), do_desc = tc::sw128_desc(sb + DQ_DO, 16, 1024);
+      const uint64_t k_desc = tc::sw128_desc(sb + dq_k(0), 16, 1024), v_desc = tc::sw128_desc(sb + dq_v(0), 16, 1024);
+      const uint64_t kmn_desc = tc::sw128_desc(sb + dq_k(0), kSlab, 1024);    // K as the MN-major B of dS K
       bool ok = wait_or_abort(&ms->qd_full, 0, ms, err, 4u);
       int dq_issued = 0;
       // dQ += dS K: dS (bf16 pairs, TMEM buffer jj & 1) is the A operand
       auto issue_dq = [&](int jj) -> bool {
         if (!wait_or_abort(&ms->ds_full[jj & 1], (jj >> 1) & 1, ms, err, 8u)) return false;
         tc::tc_fence_after();
-        const uint32_t kb = sb + dq_k(jj % kDqKStages);
+        const int st = jj % kDqKStages;
+        const uint64_t kb = tc::desc_adv(kmn_desc, (uint32_t)st * kTile);
+        const uint32_t ds = tmem + TM_DS + 64u * (jj & 1);
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
-          tc::mma_bf16_ts(tmem + TM_DQ, tmem + TM_DS + 64u * (jj & 1) + 8u * kk,
-                          tc::sw128_desc(kb + kk * 2048, kSlab, 1024), idNM, (jj > 0 || kk > 0) ? 1u : 0u);
-        tc::mma_commit(&ms->k_empty[jj % kDqKStages]);
+          tc::mma_bf16_ts(tmem + TM_DQ, ds + 8u * kk, tc::desc_adv(kb, kk * 2048), idNM, (jj > 0 || kk > 0) ? 1u : 0u);
+        tc::mma_commit(&ms->k_empty[st]);
         dq_issued = jj + 1;
         return true;
       };
@@ -220,20 +225,20 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         if (!wait_or_abort(&ms->v_full[sv], (j / kDqVStages) & 1, ms, err, 16u)) break;
         if (j >= 1 && !wait_or_abort(&ms->st_free, (j - 1) & 1, ms, err, 32u)) break;
         tc::tc_fence_after();
+        const uint64_t vb = tc::desc_adv(v_desc, (uint32_t)sv * kTile);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
-          tc::mma_bf16(tmem + TM_DP, tc::sw128_desc(sb + DQ_DO + off, 16, 1024),
-                       tc::sw128_desc(sb + dq_v(sv) + off, 16, 1024), idNN, kk > 0 ? 1u : 0u);
+          tc::mma_bf16(tmem + TM_DP, tc::desc_adv(do_desc, off), tc::desc_adv(vb, off), idNN, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(&ms->v_empty[sv]);              // V slot free once dP is done
         if (!wait_or_abort(&ms->k_full[sk], (j / kDqKStages) & 1, ms, err, 64u)) break;
         tc::tc_fence_after();
+        const uint64_t kb = tc::desc_adv(k_desc, (uint32_t)sk * kTile);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
-          tc::mma_bf16(tmem + TM_S, tc::sw128_desc(sb + DQ_Q + off, 16, 1024),
-                       tc::sw128_desc(sb + dq_k(sk) + off, 16, 1024), idNN, kk > 0 ? 1u : 0u);
+          tc::mma_bf16(tmem + TM_S, tc::desc_adv(q_desc, off), tc::desc_adv(kb, off), idNN, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(&ms->s_full);
         if (j >= 1 && !issue_dq(j - 1)) break;
@@ -554,26 +559,32 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const uint32_t idS = tc::idesc_bf16(128, 128, false, false);    // K (keys x d) x Q (queries x d)
       const uint32_t idG = tc::idesc_bf16(128, D, false, true);       // P^T / dS^T (TMEM) x (dO / Q, MN-major)
       const uint32_t sb = smem_u32(smem);
+      // operand descriptors built once; a K step or a ring stage only moves the start address
+      const uint64_t k_desc = tc::sw128_desc(sb + KV_K, 16, 1024), v_desc = tc::sw128_desc(sb + KV_V, 16, 1024);
+      const uint64_t q_desc = tc::sw128_desc(sb + kv_q(0), 16, 1024), do_desc = tc::sw128_desc(sb + kv_do(0), 16, 1024);
+      const uint64_t qmn_desc = tc::sw128_desc(sb + kv_q(0), kSlab, 1024);     // Q, dO as MN-major B
+      const uint64_t domn_desc = tc::sw128_desc(sb + kv_do(0), kSlab, 1024);
       bool ok = wait_or_abort(&ms->kv_full, 0, ms, err, 2u);
       for (int u = 0; ok && u < n_u; ++u) {
         const int s = u % kStages;
         if (!wait_or_abort(&ms->qd_full[s], (u / kStages) & 1, ms, err, 8u)) break;
         tc::tc_fence_after();
+        const uint32_t so = (uint32_t)s * 2 * kTile;             // stage offset of Q and dO
+        const uint64_t qb = tc::desc_adv(q_desc, so), dob = tc::desc_adv(do_desc, so);
         // S^T and dP^T overwrite the columns that held the previous unit's P^T / dS^T:
         // the products that read those were issued earlier and tcgen05 MMAs run in order
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
-          tc::mma_bf16(tmem + TM_ST, tc::sw128_desc(sb + KV_K + off, 16, 1024),
-                       tc::sw128_desc(sb + kv_q(s) + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          tc::mma_bf16(tmem + TM_ST, tc::desc_adv(k_desc, off), tc::desc_adv(qb, off), idS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
-          tc::mma_bf16(tmem + TM_DPT, tc::sw128_desc(sb + KV_V + off, 16, 1024),
-                       tc::sw128_desc(sb + kv_do(s) + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          tc::mma_bf16(tmem + TM_DPT, tc::desc_adv(v_desc, off), tc::desc_adv(dob, off), idS, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(&ms->s_full);
+        const uint64_t domb = tc::desc_adv(domn_desc, so), qmb = tc::desc_adv(qmn_desc, so);
         // gradient products over each pass of 64 queries as soon as it is written
         for (int h = 0; ok && h < 2; ++h) {
           ok = wait_or_abort(&ms->p_half[h], u & 1, ms, err, 4u);
@@ -582,14 +593,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4) {
             const int kk = 4 * h + k4;               // queries 16 kk .. 16 kk + 15
-            tc::mma_bf16_ts(tmem + TM_DV, tmem + TM_ST + 16 * kk, tc::sw128_desc(sb + kv_do(s) + kk * 2048, kSlab, 1024),
-                            idG, (u > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_bf16_ts(tmem + TM_DV, tmem + TM_ST + 16 * kk, tc::desc_adv(domb, kk * 2048), idG,
+                            (u > 0 || kk > 0) ? 1u : 0u);
           }
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4) {
             const int kk = 4 * h + k4;
-            tc::mma_bf16_ts(tmem + TM_DK, tmem + TM_DPT + 16 * kk, tc::sw128_desc(sb + kv_q(s) + kk * 2048, kSlab, 1024),
-                            idG, (u > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_bf16_ts(tmem + TM_DK, tmem + TM_DPT + 16 * kk, tc::desc_adv(qmb, kk * 2048), idG,
+                            (u > 0 || kk > 0) ? 1u : 0u);
           }
         }
         if (ok) tc::mma_commit(&ms->qd_empty[s]);

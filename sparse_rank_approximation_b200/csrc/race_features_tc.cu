@@ -51,9 +51,10 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Fe
   return false;
 }
 
-// K-major operand, K = 16 step kk of a tile of 128-byte rows kept as 64-column slabs.
-__device__ __forceinline__ uint64_t desc_k(uint32_t base, int kk, uint32_t slab) {
-  return tc::sw128_desc(base + (uint32_t)(kk >> 2) * slab + (uint32_t)(kk & 3) * 32u, 16, 1024);
+// K-major operand at byte offset `off`, K = 16 step kk of a tile of 128-byte rows kept as
+// 64-column slabs; `d0` is the descriptor of offset 0, built once by the issuing thread.
+__device__ __forceinline__ uint64_t desc_k(uint64_t d0, uint32_t off, int kk, uint32_t slab) {
+  return tc::desc_adv(d0, off + (uint32_t)(kk >> 2) * slab + (uint32_t)(kk & 3) * 32u);
 }
 
 __device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 128;\n" ::: "memory"); }
@@ -104,14 +105,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(128, NW, false, false);   // X (K-major) x W (K-major)
-      const uint32_t sb = smem_u32(smem);
+      const uint64_t d0 = tc::sw128_desc(smem_u32(smem), 16, 1024);
       if (wait_or_abort(&ms->in_full, 0, ms, err, 0x4000000u)) {
         tc::tc_fence_after();
 #pragma unroll
         for (int part = 0; part < 2; ++part)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            tc::mma_bf16(tmem, desc_k(sb + F_X, kk, kSlab), desc_k(sb + (part ? F_WL : F_WH), kk, kWSlab), idesc,
+            tc::mma_bf16(tmem, desc_k(d0, F_X, kk, kSlab), desc_k(d0, part ? F_WL : F_WH, kk, kWSlab), idesc,
                          (part > 0 || kk > 0) ? 1u : 0u);
       }
       tc::mma_commit(&ms->acc_full);

@@ -77,14 +77,17 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, St
 
 __device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
 
-// MN-major operand: K = 16 rows per step, 64-element M (or N) atoms `slab` bytes apart.
-__device__ __forceinline__ uint64_t desc_mn(uint32_t base, int kk) {
-  return tc::sw128_desc(base + (uint32_t)kk * 2048u, kSlab, 1024);
+// Operand descriptors are built once from the shared-memory base (`d0`, with the layout's
+// leading offset); an operand at byte offset `off` and its K = 16 step kk only move the start
+// address.
+// MN-major operand: K = 16 rows per step, 64-element M (or N) atoms kSlab bytes apart.
+__device__ __forceinline__ uint64_t desc_mn(uint64_t d0, uint32_t off, int kk) {
+  return tc::desc_adv(d0, off + (uint32_t)kk * 2048u);
 }
 
 // K-major operand, K = 16 step kk of a tile of 128-byte rows kept as 64-column slabs.
-__device__ __forceinline__ uint64_t desc_k(uint32_t base, int kk, uint32_t slab) {
-  return tc::sw128_desc(base + (uint32_t)(kk >> 2) * slab + (uint32_t)(kk & 3) * 32u, 16, 1024);
+__device__ __forceinline__ uint64_t desc_k(uint64_t d0, uint32_t off, int kk, uint32_t slab) {
+  return tc::desc_adv(d0, off + (uint32_t)(kk >> 2) * slab + (uint32_t)(kk & 3) * 32u);
 }
 
 // bf16 element (row, col) of a [128][128] tile kept as two 64-column slabs with the 128-byte swizzle.
@@ -183,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = tc::idesc_bf16(128, D, true, true);    // A = Phi^T and B = Y, both MN-major
       const uint32_t idm = tc::idesc_bf16(128, 16, true, false);    // A = Phi^T, B = the weight tile (K-major)
       const uint32_t sb = smem_u32(smem);
+      const uint64_t dmn = tc::sw128_desc(sb, kSlab, 1024), dk = tc::sw128_desc(sb, 16, 1024);
       for (int s = 0; s < n_load; ++s) {
         const int st = s % NS, buf = EMIT ? (s & 1) : 0;
         if (!wait_or_abort(&ms->full[st], (s / NS) & 1, ms, err, 0x200000u)) break;
@@ -192,8 +196,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kC / 16; ++kk) {
           const uint32_t acc = (EMIT ? kk > 0 : (s > 0 || kk > 0)) ? 1u : 0u;
-          tc::mma_bf16(tmem + 128u * buf, desc_mn(sb + Lay::phi(st), kk), desc_mn(sb + Lay::y(st), kk), idesc, acc);
-          tc::mma_bf16(tmem + Lay::mass_col(buf), desc_mn(sb + Lay::phi(st), kk), desc_k(sb + Lay::wt(st), kk, 2048u),
+          tc::mma_bf16(tmem + 128u * buf, desc_mn(dmn, Lay::phi(st), kk), desc_mn(dmn, Lay::y(st), kk), idesc, acc);
+          tc::mma_bf16(tmem + Lay::mass_col(buf), desc_mn(dmn, Lay::phi(st), kk), desc_k(dk, Lay::wt(st), kk, 2048u),
                        idm, acc);
         }
         tc::mma_commit(&ms->empty[st]);

@@ -54,14 +54,21 @@ __device__ __forceinline__ uint32_t sw_off(int row, int col, uint32_t slab) {
 }
 __device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
 
-// K-major operand, K = 16 step kk of a [rows][128] tile.
-__device__ __forceinline__ uint64_t desc_k(uint32_t base, int kk) {
-  return tc::sw128_desc(base + (uint32_t)(kk >> 2) * kSlab + (uint32_t)(kk & 3) * 32u, 16, 1024);
-}
-// MN-major operand: rows are K, 128 columns are N; K = 16 step kk.
-__device__ __forceinline__ uint64_t desc_mn(uint32_t base, int kk, uint32_t slab) {
-  return tc::sw128_desc(base + (uint32_t)kk * 2048u, slab, 1024);
-}
+// Operand descriptors, built once from the shared-memory base; an operand at byte offset
+// `off` and its K = 16 step kk only move the start address (one 32-bit add per descriptor).
+struct SDesc {
+  uint64_t k16, mn, mn_w;
+  __device__ explicit SDesc(uint32_t sb)
+      : k16(tc::sw128_desc(sb, 16, 1024)), mn(tc::sw128_desc(sb, kSlab, 1024)), mn_w(tc::sw128_desc(sb, kWSlab, 1024)) {}
+  // K-major operand, K = 16 step kk of a [rows][128] tile
+  __device__ uint64_t k(uint32_t off, int kk) const {
+    return tc::desc_adv(k16, off + (uint32_t)(kk >> 2) * kSlab + (uint32_t)(kk & 3) * 32u);
+  }
+  // MN-major operand: rows are K, 128 columns are N (64-column slabs kSlab apart)
+  __device__ uint64_t kn(uint32_t off, int kk) const { return tc::desc_adv(mn, off + (uint32_t)kk * 2048u); }
+  // MN-major with slabs kWSlab apart (the hash-projection weights)
+  __device__ uint64_t kn_w(uint32_t off, int kk) const { return tc::desc_adv(mn_w, off + (uint32_t)kk * 2048u); }
+};
 // TMEM column of the K = 16 step kk of a packed bf16 operand whose K index
 // 64 h + m (h = column half of the thread that wrote it) sits at column 64 h + m / 2.
 __device__ __forceinline__ uint32_t packed_col(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
@@ -173,15 +180,15 @@ __device__ __forceinline__ void corner_pass(uint32_t tmem, uint32_t lane_base, i
 
 // du = dh W^T: three products (hi hi, hi lo, lo hi), K = 32 (two steps each), N = D.
 template <int D>
-__device__ __forceinline__ void issue_du(uint32_t tmem, uint32_t d_col, uint32_t sb, uint32_t w_hi, uint32_t w_lo) {
+__device__ __forceinline__ void issue_du(uint32_t tmem, uint32_t d_col, const SDesc& sd, uint32_t w_hi, uint32_t w_lo) {
   const uint32_t idG = tc::idesc_bf16(128, D, false, true);
 #pragma unroll
   for (int part = 0; part < 3; ++part) {
     const uint32_t a_col = part == 2 ? 16u : 0u;
-    const uint32_t wb = sb + (part == 1 ? w_lo : w_hi);
+    const uint32_t wb = part == 1 ? w_lo : w_hi;
 #pragma unroll
     for (int kk = 0; kk < 2; ++kk)
-      tc::mma_bf16_ts(tmem + d_col, tmem + a_col + 8u * kk, desc_mn(wb, kk, kWSlab), idG,
+      tc::mma_bf16_ts(tmem + d_col, tmem + a_col + 8u * kk, sd.kn_w(wb, kk), idG,
                       (part > 0 || kk > 0) ? 1u : 0u);
   }
 }
@@ -351,29 +358,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);
       const uint32_t idNM = tc::idesc_bf16(128, 128, false, true);
       const uint32_t idDM = tc::idesc_bf16(128, D, false, true);     // N = D, B MN-major
-      const uint32_t sb = smem_u32(smem);
+      const SDesc sd(smem_u32(smem));
       bool ok = wait_or_abort(&ms->in_main, 0, ms, err, 0x100u);
       if (ok && causal) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          tc::mma_bf16(tmem + TK_KAP, desc_k(sb + K_PK, kk), desc_k(sb + K_PQ, kk), idNN, kk > 0 ? 1u : 0u);
+          tc::mma_bf16(tmem + TK_KAP, sd.k(K_PK, kk), sd.k(K_PQ, kk), idNN, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          tc::mma_bf16(tmem + TK_X, desc_k(sb + K_V, kk), desc_k(sb + K_DO, kk), idNN, kk > 0 ? 1u : 0u);
+          tc::mma_bf16(tmem + TK_X, sd.k(K_V, kk), sd.k(K_DO, kk), idNN, kk > 0 ? 1u : 0u);
         tc::mma_commit(&ms->s_full);
       }
       if (ok) {
         // inter-chunk parts: dv = Phi_K R^V, dPhi = V R^V^T (R as bf16 hi + lo)
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
-          const uint32_t rb = sb + (part ? K_RL : K_RH);
+          const uint32_t rb = part ? K_RL : K_RH;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_bf16(tmem + TK_DV, desc_k(sb + K_PK, kk), desc_mn(rb, kk, kSlab), idDM,
+            tc::mma_bf16(tmem + TK_DV, sd.k(K_PK, kk), sd.kn(rb, kk), idDM,
                          (part > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            tc::mma_bf16(tmem + TK_DPHI, desc_k(sb + K_V, kk), desc_k(rb, kk), idNN, (part > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_bf16(tmem + TK_DPHI, sd.k(K_V, kk), sd.k(rb, kk), idNN, (part > 0 || kk > 0) ? 1u : 0u);
         }
       }
       if (ok && causal) {
@@ -383,17 +390,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           // intra-chunk parts, A operands from tensor memory
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_bf16_ts(tmem + TK_DV, tmem + TK_KAP + packed_col(kk), desc_mn(sb + K_DO, kk, kSlab), idDM, 1u);
+            tc::mma_bf16_ts(tmem + TK_DV, tmem + TK_KAP + packed_col(kk), sd.kn(K_DO, kk), idDM, 1u);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_bf16_ts(tmem + TK_DPHI, tmem + TK_X + packed_col(kk), desc_mn(sb + K_PQ, kk, kSlab), idNM, 1u);
+            tc::mma_bf16_ts(tmem + TK_DPHI, tmem + TK_X + packed_col(kk), sd.kn(K_PQ, kk), idNM, 1u);
         }
       }
       tc::mma_commit(&ms->acc_full);
       ok = ok && wait_or_abort(&ms->dh_full, 0, ms, err, 0x800u);
       if (ok) {
         tc::tc_fence_after();
-        issue_du<D>(tmem, TK_DU, sb, K_WH, K_WL);
+        issue_du<D>(tmem, TK_DU, sd, K_WH, K_WL);
       }
       tc::mma_commit(&ms->du_full);
       tc::mbar_wait(&ms->du_full, 0);
@@ -574,22 +581,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);
       const uint32_t idNM = tc::idesc_bf16(128, 128, false, true);
-      const uint32_t sb = smem_u32(smem);
+      const SDesc sd(smem_u32(smem));
       bool ok = wait_or_abort(&ms->in_main, 0, ms, err, 0x100u);
       if (ok && causal) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          tc::mma_bf16(tmem + TQ_X, desc_k(sb + Q_DO, kk), desc_k(sb + Q_V, kk), idNN, kk > 0 ? 1u : 0u);
+          tc::mma_bf16(tmem + TQ_X, sd.k(Q_DO, kk), sd.k(Q_V, kk), idNN, kk > 0 ? 1u : 0u);
         tc::mma_commit(&ms->s_full);
       }
       if (ok) {
         // inter-chunk part: G = dO P^V^T (P as bf16 hi + lo)
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
-          const uint32_t pb = sb + (part ? Q_PL : Q_PH);
+          const uint32_t pb = part ? Q_PL : Q_PH;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            tc::mma_bf16(tmem + TQ_G, desc_k(sb + Q_DO, kk), desc_k(pb, kk), idNN, (part > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_bf16(tmem + TQ_G, sd.k(Q_DO, kk), sd.k(pb, kk), idNN, (part > 0 || kk > 0) ? 1u : 0u);
         }
       }
       if (ok && causal) {
@@ -598,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_bf16_ts(tmem + TQ_INTRA, tmem + TQ_X + packed_col(kk), desc_mn(sb + Q_PK, kk, kSlab), idNM,
+            tc::mma_bf16_ts(tmem + TQ_INTRA, tmem + TQ_X + packed_col(kk), sd.kn(Q_PK, kk), idNM,
                             kk > 0 ? 1u : 0u);
         }
       }
@@ -606,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = ok && wait_or_abort(&ms->dh_full, 0, ms, err, 0x800u);
       if (ok) {
         tc::tc_fence_after();
-        issue_du<D>(tmem, TQ_DU, sb, Q_WH, Q_WL);
+        issue_du<D>(tmem, TQ_DU, sd, Q_WH, Q_WL);
       }
       tc::mma_commit(&ms->du_full);
       tc::mbar_wait(&ms->du_full, 0);
@@ -742,22 +749,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idNN = tc::idesc_bf16(128, 128, false, false);
       const uint32_t idNM = tc::idesc_bf16(128, D, false, true);       // N = D, B MN-major
-      const uint32_t sb = smem_u32(smem);
+      const SDesc sd(smem_u32(smem));
       bool ok = wait_or_abort(&ms->in_main, 0, ms, err, 0x100u);
       if (ok && causal) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          tc::mma_bf16(tmem + TR_KAP, desc_k(sb + R_PQ, kk), desc_k(sb + R_PK, kk), idNN, kk > 0 ? 1u : 0u);
+          tc::mma_bf16(tmem + TR_KAP, sd.k(R_PQ, kk), sd.k(R_PK, kk), idNN, kk > 0 ? 1u : 0u);
         tc::mma_commit(&ms->s_full);
       }
       if (ok) {
         // inter-chunk part: N = Phi_Q P^V (P as bf16 hi + lo)
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
-          const uint32_t pb = sb + (part ? R_PL : R_PH);
+          const uint32_t pb = part ? R_PL : R_PH;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_bf16(tmem + TR_N, desc_k(sb + R_PQ, kk), desc_mn(pb, kk, kSlab), idNM,
+            tc::mma_bf16(tmem + TR_N, sd.k(R_PQ, kk), sd.kn(pb, kk), idNM,
                          (part > 0 || kk > 0) ? 1u : 0u);
         }
       }
@@ -767,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_bf16_ts(tmem + TR_N, tmem + TR_KAP + packed_col(kk), desc_mn(sb + R_V, kk, kSlab), idNM, 1u);
+            tc::mma_bf16_ts(tmem + TR_N, tmem + TR_KAP + packed_col(kk), sd.kn(R_V, kk), idNM, 1u);
         }
       }
       tc::mma_commit(&ms->acc_full);

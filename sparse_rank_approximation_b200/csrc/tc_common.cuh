@@ -180,6 +180,14 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo_
   return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
+// The same descriptor with its start address `bytes` (a multiple of 16) further on.
+// Shared-memory addresses stay below 256 KB, so the sum never leaves the 14-bit address
+// field of the low word: one 32-bit add, where rebuilding the descriptor costs a chain
+// of 64-bit operations in the issuing thread between two MMAs.
+__device__ __forceinline__ uint64_t desc_adv(uint64_t desc, uint32_t bytes) {
+  const uint32_t lo = (uint32_t)desc + (bytes >> 4), hi = (uint32_t)(desc >> 32);
+  return ((uint64_t)hi << 32) | lo;
+}
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, dense, M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
