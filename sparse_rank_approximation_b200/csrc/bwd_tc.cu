@@ -13,9 +13,9 @@
 // dkdv kernel: one CTA per (head, key block); K and V stay in shared memory, the
 // query tiles that selected the block (from the selection inverse) stream through a
 // 2-stage ring together with their per-row scalars; S^T = K Q^T and dP^T = V dO^T
-// land in TMEM, the softmax warps write (P^T cs) and dS^T back over them as bf16 in
-// two passes of 64 queries, and dV += (P^T cs) dO, dK += dS^T Q accumulate in TMEM
-// after each pass.  The low-rank parts are brought into L2 once every load is issued
+// land in TMEM, the softmax warps write (P^T cs) and dS^T back over them as bf16 in two
+// passes of 64 queries, and dV += (P^T cs) dO, dK += dS^T Q accumulate in TMEM (with
+// d = 64, in two buffers, the next pass's scores computed while the softmax works).  The low-rank parts are brought into L2 once every load is issued
 // and read while the last products run.  No atomics: the results are deterministic.
 // Every mbarrier wait is bounded; a timeout sets a bit in the caller's error word,
 // the CTA drains its copies and MMAs, frees TMEM and exits.
@@ -395,13 +395,23 @@ constexpr uint32_t KV_SC = 2 * kTile + kStages * 2 * kTile;                   //
 constexpr int kMaxUnits = 1024;
 constexpr uint32_t KV_UNITS = KV_SC + kStages * 128 * 16;                     // query tiles of the block(s)
 constexpr uint32_t KV_MISC = KV_UNITS + 2 * kMaxUnits * 4;
-// TMEM columns: S^T [keys][queries] and dP^T (fp32); once read, (P^T cs) and dS^T (bf16 pairs)
-// overwrite the first 8 of every 16 columns and feed dV / dK as the tensor-memory A operand.
-constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_DV = 256, TM_DK = 384;
+// TMEM columns 0-255 hold S^T [keys][queries] and dP^T (fp32) for the 128 queries of a tile,
+// taken as two passes of 64 queries.  d = 128: S^T in columns 0-127 and dP^T in 128-255, both
+// products at N = 128 once per tile.  d = 64 (products half as long, so the softmax warps
+// dominate): two buffers of one pass each (columns 128 h: S^T, then dP^T 64 further), the
+// products at N = 64 per pass, so the next pass's scores are computed while the softmax warps
+// work on this one.  Once read, (P^T cs) and dS^T (bf16 pairs) overwrite the first 8 of every
+// 16 columns and feed dV / dK as the tensor-memory A operand.
+constexpr uint32_t TM_DV = 256, TM_DK = 384;
+template <int D> struct KvTmem {
+  static constexpr bool kTwoBuf = D == 64;
+  static constexpr uint32_t kDp = kTwoBuf ? 64 : 128;             // dP^T columns after S^T
+  __host__ __device__ static constexpr uint32_t st(int pass) { return (kTwoBuf ? 128u : 64u) * pass; }
+};
 constexpr int kKvThreads = 320;
 
 struct KvMisc {
-  uint64_t kv_full, qd_full[kStages], qd_empty[kStages], s_full, p_half[2], done;
+  uint64_t kv_full, qd_full[kStages], qd_empty[kStages], s_full[2], p_half[2], done;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -441,10 +451,11 @@ __device__ __forceinline__ void dkdv_softmax_cols(uint32_t tmem, uint32_t st_col
 
 // One CTA per (head, key block b): K_b and V_b stay in shared memory; the query tiles that
 // selected b (ascending, from the selection inverse) stream through a 2-stage ring with
-// their per-row scalars.  Per tile: S^T = K Q^T and dP^T = V dO^T (N = 128) into TMEM; the
-// softmax warps turn them into (P^T cs) and dS^T in two passes of 64 queries; after each
-// pass dV += (P^T cs) dO and dK += dS^T Q over those 64 queries run on the tensor cores
-// while the other pass is computed.
+// their per-row scalars.  Per tile: S^T = K Q^T and dP^T = V dO^T into TMEM; the softmax
+// warps turn them into (P^T cs) and dS^T in two passes of 64 queries, and after each pass
+// dV += (P^T cs) dO and dK += dS^T Q over those 64 queries run on the tensor cores while the
+// other pass is computed.  With d = 64 the scores are computed per pass into two buffers, so
+// the next pass's scores also overlap the softmax work.
 // D = 64 or 128.  PAIR (blocks of 64): the CTA's 128 key rows are blocks 2c (rows 0-63) and
 // 2c + 1 (rows 64-127); unit u stages the u-th query tile of block 2c in query rows 0-63 and
 // the u-th of block 2c + 1 in rows 64-127, and each key row masks the other block's queries.
@@ -495,7 +506,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       tc::mbar_init(&ms->qd_full[s], 1);
       tc::mbar_init(&ms->qd_empty[s], 1);
     }
-    tc::mbar_init(&ms->s_full, 1);
+    tc::mbar_init(&ms->s_full[0], 1);
+    tc::mbar_init(&ms->s_full[1], 1);
     tc::mbar_init(&ms->p_half[0], kSoftmaxThreads);
     tc::mbar_init(&ms->p_half[1], kSoftmaxThreads);
     tc::mbar_init(&ms->done, 1);
@@ -556,7 +568,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t idS = tc::idesc_bf16(128, 128, false, false);    // K (keys x d) x Q (queries x d)
+      using TL = KvTmem<D>;
+      constexpr int NQ = TL::kTwoBuf ? 64 : 128;                       // queries per score product
+      const uint32_t idS = tc::idesc_bf16(128, NQ, false, false);     // K (keys x d) x Q (queries x d)
       const uint32_t idG = tc::idesc_bf16(128, D, false, true);       // P^T / dS^T (TMEM) x (dO / Q, MN-major)
       const uint32_t sb = smem_u32(smem);
       // operand descriptors built once; a K step or a ring stage only moves the start address
@@ -565,45 +579,102 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const uint64_t qmn_desc = tc::sw128_desc(sb + kv_q(0), kSlab, 1024);     // Q, dO as MN-major B
       const uint64_t domn_desc = tc::sw128_desc(sb + kv_do(0), kSlab, 1024);
       bool ok = wait_or_abort(&ms->kv_full, 0, ms, err, 2u);
-      for (int u = 0; ok && u < n_u; ++u) {
-        const int s = u % kStages;
-        if (!wait_or_abort(&ms->qd_full[s], (u / kStages) & 1, ms, err, 8u)) break;
+      // pass i = 2u + h: queries 64 h .. 64 h + 63 of unit u.
+      // dV += (P^T cs) dO and dK += dS^T Q over the 64 queries of pass i
+      auto issue_grads = [&](int i) -> bool {
+        const int u = i >> 1, h = i & 1, s = u % kStages;
+        if (!wait_or_abort(&ms->p_half[h], u & 1, ms, err, 4u)) return false;
         tc::tc_fence_after();
-        const uint32_t so = (uint32_t)s * 2 * kTile;             // stage offset of Q and dO
-        const uint64_t qb = tc::desc_adv(q_desc, so), dob = tc::desc_adv(do_desc, so);
-        // S^T and dP^T overwrite the columns that held the previous unit's P^T / dS^T:
-        // the products that read those were issued earlier and tcgen05 MMAs run in order
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
-          tc::mma_bf16(tmem + TM_ST, tc::desc_adv(k_desc, off), tc::desc_adv(qb, off), idS, kk > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
-          tc::mma_bf16(tmem + TM_DPT, tc::desc_adv(v_desc, off), tc::desc_adv(dob, off), idS, kk > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(&ms->s_full);
+        const uint32_t so = (uint32_t)s * 2 * kTile;
         const uint64_t domb = tc::desc_adv(domn_desc, so), qmb = tc::desc_adv(qmn_desc, so);
-        // gradient products over each pass of 64 queries as soon as it is written
-        for (int h = 0; ok && h < 2; ++h) {
-          ok = wait_or_abort(&ms->p_half[h], u & 1, ms, err, 4u);
-          if (!ok) break;
-          tc::tc_fence_after();
+        const uint32_t pt = tmem + TL::st(h);
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const int kk = 4 * h + k4;               // queries 16 kk .. 16 kk + 15
-            tc::mma_bf16_ts(tmem + TM_DV, tmem + TM_ST + 16 * kk, tc::desc_adv(domb, kk * 2048), idG,
-                            (u > 0 || kk > 0) ? 1u : 0u);
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * h + k4;                 // queries 16 kk .. 16 kk + 15 of the unit
+          tc::mma_bf16_ts(tmem + TM_DV, pt + 16 * k4, tc::desc_adv(domb, kk * 2048), idG, (u > 0 || kk > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * h + k4;
+          tc::mma_bf16_ts(tmem + TM_DK, pt + TL::kDp + 16 * k4, tc::desc_adv(qmb, kk * 2048), idG,
+                          (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (h == 1) tc::mma_commit(&ms->qd_empty[s]);   // the unit's Q / dO stage is read
+        return true;
+      };
+      if constexpr (!TL::kTwoBuf) {
+        // one buffer: per tile, the scores (N = 128), then each pass's products once the softmax
+        // warps have written it; the next tile's scores overwrite this tile's after them
+        // (tcgen05 MMAs of one thread run in issue order)
+        for (int u = 0; ok && u < n_u; ++u) {
+          const int s = u % kStages;
+          if (!wait_or_abort(&ms->qd_full[s], (u / kStages) & 1, ms, err, 8u)) break;
+          tc::tc_fence_after();
+          const uint32_t so = (uint32_t)s * 2 * kTile;             // stage offset of Q and dO
+          const uint64_t qb = tc::desc_adv(q_desc, so), dob = tc::desc_adv(do_desc, so);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+            tc::mma_bf16(tmem, tc::desc_adv(k_desc, off), tc::desc_adv(qb, off), idS, kk > 0 ? 1u : 0u);
           }
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const int kk = 4 * h + k4;
-            tc::mma_bf16_ts(tmem + TM_DK, tmem + TM_DPT + 16 * kk, tc::desc_adv(qmb, kk * 2048), idG,
-                            (u > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+            tc::mma_bf16(tmem + TL::kDp, tc::desc_adv(v_desc, off), tc::desc_adv(dob, off), idS, kk > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&ms->s_full[0]);
+          const uint64_t domb = tc::desc_adv(domn_desc, so), qmb = tc::desc_adv(qmn_desc, so);
+          for (int h = 0; ok && h < 2; ++h) {
+            ok = wait_or_abort(&ms->p_half[h], u & 1, ms, err, 4u);
+            if (!ok) break;
+            tc::tc_fence_after();
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const int kk = 4 * h + k4;             // queries 16 kk .. 16 kk + 15
+              tc::mma_bf16_ts(tmem + TM_DV, tmem + 16 * kk, tc::desc_adv(domb, kk * 2048), idG,
+                              (u > 0 || kk > 0) ? 1u : 0u);
+            }
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const int kk = 4 * h + k4;
+              tc::mma_bf16_ts(tmem + TM_DK, tmem + TL::kDp + 16 * kk, tc::desc_adv(qmb, kk * 2048), idG,
+                              (u > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          if (ok) tc::mma_commit(&ms->qd_empty[s]);
+        }
+      } else {
+        // two buffers: the scores of pass i + 1 run on the tensor cores while the softmax warps
+        // work on pass i
+        int n_grads = 0;                                 // passes whose products are issued
+        for (int i = 0; ok && i < 2 * n_u; ++i) {
+          const int u = i >> 1, h = i & 1, s = u % kStages;
+          if (h == 0 && !wait_or_abort(&ms->qd_full[s], (u / kStages) & 1, ms, err, 8u)) break;
+          tc::tc_fence_after();
+          // buffer h last held pass i - 2, whose products were issued before (in order) and
+          // whose scores the softmax warps had read before they arrived on p_half[h]
+          const uint32_t qo = (uint32_t)s * 2 * kTile + (uint32_t)h * 64 * 128;   // query rows 64 h ..
+          const uint64_t qb = tc::desc_adv(q_desc, qo), dob = tc::desc_adv(do_desc, qo);
+          const uint32_t st = tmem + TL::st(h);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+            tc::mma_bf16(st, tc::desc_adv(k_desc, off), tc::desc_adv(qb, off), idS, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+            tc::mma_bf16(st + TL::kDp, tc::desc_adv(v_desc, off), tc::desc_adv(dob, off), idS, kk > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&ms->s_full[h]);
+          // the previous pass's products, behind this pass's scores
+          if (i >= 1) {
+            ok = issue_grads(i - 1);
+            if (!ok) break;
+            n_grads = i;
           }
         }
-        if (ok) tc::mma_commit(&ms->qd_empty[s]);
+        if (ok && n_u > 0 && n_grads == 2 * n_u - 1) issue_grads(2 * n_u - 1);
       }
       tc::mma_commit(&ms->done);
       tc::mbar_wait(&ms->done, 0);
@@ -626,11 +697,17 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     bool alive = true;
     for (int u = 0; u < n_u && alive; ++u) {
       const int s = u % kStages;
-      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full, u & 1, ms, err, 32u));
+      // one buffer: both passes' scores arrive together; two: each pass's on its own
+      alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full[0], u & 1, ms, err, 32u));
       if (!alive) break;
       tc::tc_fence_after();
 #pragma unroll 1
       for (int pass = 0; pass < 2; ++pass) {
+        if (KvTmem<D>::kTwoBuf && pass == 1) {
+          alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full[1], u & 1, ms, err, 32u));
+          if (!alive) break;
+          tc::tc_fence_after();
+        }
         const int q0 = 64 * pass + 32 * grp;        // first query (column of the unit) of this thread
         // the query tile of these columns and the first one's position in it
         const int h = PAIR ? pass : 0;
@@ -644,11 +721,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         const int lo = diag ? kpos - qp0 : 0;
         const int hi = dead ? 0 : key_ok ? qvalid : 0;
         const float4* sc = reinterpret_cast<const float4*>(smem + KV_SC + s * 128 * 16) + q0;
+        const uint32_t st_col = lane_base + KvTmem<D>::st(pass) + 32 * grp;
         // masking only on the causal diagonal, at the end of the sequence and for padding keys
         if (__any_sync(0xffffffffu, masked))
-          dkdv_softmax_cols<true>(tmem, lane_base + TM_ST + q0, lane_base + TM_DPT + q0, sc, sl2, lo, hi);
+          dkdv_softmax_cols<true>(tmem, st_col, st_col + KvTmem<D>::kDp, sc, sl2, lo, hi);
         else
-          dkdv_softmax_cols<false>(tmem, lane_base + TM_ST + q0, lane_base + TM_DPT + q0, sc, sl2, lo, hi);
+          dkdv_softmax_cols<false>(tmem, st_col, st_col + KvTmem<D>::kDp, sc, sl2, lo, hi);
         tc::tmem_wait_st();
         tc::tc_fence_before();
         tc::mbar_arrive(&ms->p_half[pass]);
