@@ -38,23 +38,26 @@ __device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
 }
 
 // Row scalars (see the header comment).  grid (ceil(N / rows_per_block), BH), block 256.
-// d/8 threads per row reduce the row's <dO, O_s> and <dO, O_lr> (8 elements each); then
-// one thread per row (the block's first rows_per_block threads, so a warp covers 16 or 32
-// consecutive rows) runs the scalar algebra in float64 and writes the per-row outputs;
-// cl comes back through shared memory for the cl dO rows.
+// d/8 threads per row reduce the row's <dO, O_s> and <dO, O_lr> (8 elements each; the
+// butterfly leaves both sums in every one of them); each of those threads then runs the
+// scalar algebra in fp32 (no block barrier, so the memory traffic of other rows keeps
+// flowing), the row's first thread writes the per-row outputs and all of them write
+// their 8 elements of cl dO.
 template <typename E>
 __global__ void __launch_bounds__(256) row_scalars_kernel(BwdArgs a, Geom g) {
-  __shared__ float sA[32], sB[32], sCl[32];
   const int tpr = g.d / 8;
   const int rpb = 256 / tpr;
   const int sub = threadIdx.x % tpr;
-  const int lr = threadIdx.x / tpr;
-  const int row = blockIdx.x * rpb + lr;
+  const int row = blockIdx.x * rpb + threadIdx.x / tpr;
   const size_t i = (size_t)blockIdx.y * g.N + min(row, g.N - 1);
   float dO[8], os[8], ol[8];
   load8<E>((const E*)a.dO + i * g.d + sub * 8, dO);
   load8<float>((const float*)a.Os + i * g.d + sub * 8, os);     // O_s is saved in fp32
   load8<E>((const E*)a.Olr + i * g.d + sub * 8, ol);
+  const float logd = a.logd[i], dl = a.dlr[i];
+  const float lam = a.lam ? a.lam[i] : g.lam;
+  const float gs = a.gs ? a.gs[i] : 1.f;
+  const float glr = a.glr ? a.glr[i] : 0.f;
   float A = 0.f, Bv = 0.f;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -65,53 +68,34 @@ __global__ void __launch_bounds__(256) row_scalars_kernel(BwdArgs a, Geom g) {
     A += __shfl_xor_sync(0xffffffffu, A, o);
     Bv += __shfl_xor_sync(0xffffffffu, Bv, o);
   }
+  if (row >= g.N) return;
+  const float ds = expf(logd);
+  const float c = lam * dl + g.eps;
+  const float D = ds + c;
+  // fixed_m: the ablation without denominator-aware fusion (m = 1, default g_lr = 1, no dm)
+  const float m = g.fixed_m ? 1.f : D > 0.f ? ds / D : 0.f;
+  const float one_m = g.fixed_m ? 0.f : D > 0.f ? c / D : 1.f;
+  const float gl = a.glr ? glr : g.fixed_m ? 1.f : one_m;
+  const float dm = g.fixed_m ? 0.f : gs * A - (a.glr ? 0.f : Bv);
+  const float cs = gs * m;
+  const float cl = dl > 0.f ? gl / dl : 0.f;
+  const float ddlr = D > 0.f ? -dm * lam * ds / (D * D) : 0.f;
+  const float Dl = cs * A - dm * m * one_m;
   if (sub == 0) {
-    sA[lr] = A;
-    sB[lr] = Bv;
-  }
-  __syncthreads();
-  if ((int)threadIdx.x < rpb) {
-    const int r = blockIdx.x * rpb + threadIdx.x;
-    float clv = 0.f;
-    if (r < g.N) {
-      const size_t k = (size_t)blockIdx.y * g.N + r;
-      const double Ar = sA[threadIdx.x], Br = sB[threadIdx.x];
-      const double logd = a.logd[k], dl = a.dlr[k];
-      const double lam = a.lam ? a.lam[k] : g.lam;
-      const double gs = a.gs ? a.gs[k] : 1.0;
-      const double ds = exp(logd);
-      const double c = lam * dl + (double)g.eps;
-      const double D = ds + c;
-      // fixed_m: the ablation without denominator-aware fusion (m = 1, default g_lr = 1, no dm)
-      const double m = g.fixed_m ? 1.0 : D > 0.0 ? ds / D : 0.0;
-      const double one_m = g.fixed_m ? 0.0 : D > 0.0 ? c / D : 1.0;
-      const double gl = a.glr ? (double)a.glr[k] : g.fixed_m ? 1.0 : one_m;
-      const double dm = g.fixed_m ? 0.0 : gs * Ar - (a.glr ? 0.0 : Br);
-      const double cs = gs * m;
-      const double cl = dl > 0.0 ? gl / dl : 0.0;
-      const double ddlr = D > 0.0 ? -dm * lam * ds / (D * D) : 0.0;
-      const double Dl = cs * Ar - dm * m * one_m;
-      a.rs.cs[k] = (float)cs;
-      a.rs.Delta[k] = (float)Dl;
-      if (a.rs.packed) a.rs.packed[k] = make_float4((float)(logd * 1.4426950408889634), (float)cs, (float)Dl, 0.f);
-      a.rs.cl[k] = (float)cl;
-      a.rs.delta[k] = (float)(ddlr - cl * Br);
-      clv = (float)cl;
-    }
-    sCl[threadIdx.x] = clv;
+    a.rs.cs[i] = cs;
+    a.rs.Delta[i] = Dl;
+    if (a.rs.packed) a.rs.packed[i] = make_float4(logd * 1.44269504f, cs, Dl, 0.f);
+    a.rs.cl[i] = cl;
+    a.rs.delta[i] = ddlr - cl * Bv;
   }
   // the rows cl dO (bf16) feed the RACE suffix statistics
   if (a.dOcl) {
-    __syncthreads();
-    if (row < g.N) {
-      const float clf = sCl[lr];
-      uint4 w;
-      w.x = pack_bf16(clf * dO[0], clf * dO[1]);
-      w.y = pack_bf16(clf * dO[2], clf * dO[3]);
-      w.z = pack_bf16(clf * dO[4], clf * dO[5]);
-      w.w = pack_bf16(clf * dO[6], clf * dO[7]);
-      *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dOcl) + i * g.d + sub * 8) = w;
-    }
+    uint4 w;
+    w.x = pack_bf16(cl * dO[0], cl * dO[1]);
+    w.y = pack_bf16(cl * dO[2], cl * dO[3]);
+    w.z = pack_bf16(cl * dO[4], cl * dO[5]);
+    w.w = pack_bf16(cl * dO[6], cl * dO[7]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dOcl) + i * g.d + sub * 8) = w;
   }
 }
 
