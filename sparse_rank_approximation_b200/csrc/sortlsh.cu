@@ -382,72 +382,69 @@ __global__ void lsh_fuse_kernel(const float* __restrict__ Os0, const float* __re
                                 const int* __restrict__ inv_lv, int levels, const __nv_bfloat16* __restrict__ Olr,
                                 const float* __restrict__ dlr, const float* lamv, const float* gsv, const float* glrv,
                                 __nv_bfloat16* __restrict__ O, float* __restrict__ Os,
-                                float* __restrict__ logd_out, float* __restrict__ m_out, Geom g) {
-  const int units = g.d / 8;
+                                float* __restrict__ logd_out, float* __restrict__ m_out, int units_log2, Geom g) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (g.N << units_log2)) return;
+  const int r = e >> units_log2, u = e & ((1 << units_log2) - 1);
   const size_t rows = (size_t)g.BH * g.N;
-  const size_t total = rows * units;
-  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
-    const size_t row = e / units;
-    const int u = (int)(e % units);
-    const int bh = (int)(row / g.N), r = (int)(row % g.N);
-    // the partials this row has: base (slot 0), then one per level where it is in a
-    // future half.  Every partial's log-denominator and row are loaded as soon as its
-    // position is known (predicated loads, no branch on the values)
-    float4 w[kMaxLevels + 1][2];
-    float lg[kMaxLevels + 1];
-    w[0][0] = reinterpret_cast<const float4*>(Os0 + row * g.d + 8 * u)[0];
-    w[0][1] = reinterpret_cast<const float4*>(Os0 + row * g.d + 8 * u)[1];
-    lg[0] = logd0[row];
+  const size_t row = (size_t)bh * g.N + r;
+  // the partials this row has: base (slot 0), then one per level where it is in a future
+  // half; first their log-denominators (and slot rows), for the common maximum
+  size_t pos[kMaxLevels];
+  float lg[kMaxLevels + 1];
+  lg[0] = logd0[row];
 #pragma unroll
-    for (int l = 0; l < kMaxLevels; ++l) {
-      lg[l + 1] = -INFINITY;
-      w[l + 1][0] = w[l + 1][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (l < levels && ((r / (g.N >> (l + 1))) & 1)) {
-        const size_t p = (size_t)l * rows + (size_t)bh * g.N + inv_lv[(size_t)l * rows + row];
-        w[l + 1][0] = reinterpret_cast<const float4*>(Os_lv + p * g.d + 8 * u)[0];
-        w[l + 1][1] = reinterpret_cast<const float4*>(Os_lv + p * g.d + 8 * u)[1];
-        lg[l + 1] = logd_lv[p];
-      }
+  for (int l = 0; l < kMaxLevels; ++l) {
+    lg[l + 1] = -INFINITY;
+    pos[l] = 0;
+    const int hl = 31 - __clz(g.N >> (l + 1));      // log2 of the half length
+    if (l < levels && ((r >> hl) & 1)) {
+      pos[l] = (size_t)l * rows + (size_t)bh * g.N + inv_lv[(size_t)l * rows + row];
+      lg[l + 1] = logd_lv[pos[l]];
     }
-    float L = -INFINITY;
+  }
+  float L = -INFINITY;
 #pragma unroll
-    for (int j = 0; j <= kMaxLevels; ++j) L = fmaxf(L, lg[j]);
-    float sum = 0.f, s[8] = {};
-    if (L > -INFINITY) {
+  for (int j = 0; j <= kMaxLevels; ++j) L = fmaxf(L, lg[j]);
+  float sum = 0.f, s[8] = {};
+  if (L > -INFINITY) {
+    // then the rows, weighted by e^{log d - L} as they arrive
 #pragma unroll
-      for (int j = 0; j <= kMaxLevels; ++j) {
-        const float wj = lg[j] == -INFINITY ? 0.f : __expf(lg[j] - L);
-        sum += wj;
-        const float* f = reinterpret_cast<const float*>(&w[j][0]);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) s[k] = fmaf(wj, f[k], s[k]);
-      }
-      const float inv_sum = 1.f / sum;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) s[k] *= inv_sum;
-      L += __logf(sum);
+    for (int j = 0; j <= kMaxLevels; ++j) {
+      if (lg[j] == -INFINITY) continue;
+      const float wj = __expf(lg[j] - L);
+      sum += wj;
+      const float4* src = reinterpret_cast<const float4*>((j ? Os_lv + pos[j - 1] * g.d : Os0 + row * g.d) + 8 * u);
+      const float4 w0 = src[0], w1 = src[1];
+      s[0] = fmaf(wj, w0.x, s[0]); s[1] = fmaf(wj, w0.y, s[1]); s[2] = fmaf(wj, w0.z, s[2]); s[3] = fmaf(wj, w0.w, s[3]);
+      s[4] = fmaf(wj, w1.x, s[4]); s[5] = fmaf(wj, w1.y, s[5]); s[6] = fmaf(wj, w1.z, s[6]); s[7] = fmaf(wj, w1.w, s[7]);
     }
-    const float lam = lamv ? lamv[row] : g.lam;
-    const float gs = gsv ? gsv[row] : 1.f;
-    const float mf = g.fixed_m ? 1.f : L == -INFINITY ? 0.f : 1.f / (1.f + (lam * dlr[row] + g.eps) * __expf(-L));
-    const float gl = glrv ? glrv[row] : g.fixed_m ? 1.f : 1.f - mf;
-    const float cs = gs * mf;
-    const uint4 wl = *reinterpret_cast<const uint4*>(Olr + row * g.d + 8 * u);
-    const __nv_bfloat162* lv = reinterpret_cast<const __nv_bfloat162*>(&wl);
-    uint32_t wo[4];
+    const float inv_sum = 1.f / sum;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = __bfloat1622float2(lv[j]);
-      const __nv_bfloat162 o = __floats2bfloat162_rn(cs * s[2 * j] + gl * f.x, cs * s[2 * j + 1] + gl * f.y);
-      wo[j] = *reinterpret_cast<const uint32_t*>(&o);
-    }
-    *reinterpret_cast<uint4*>(O + row * g.d + 8 * u) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
-    reinterpret_cast<float4*>(Os + row * g.d + 8 * u)[0] = make_float4(s[0], s[1], s[2], s[3]);
-    reinterpret_cast<float4*>(Os + row * g.d + 8 * u)[1] = make_float4(s[4], s[5], s[6], s[7]);
-    if (u == 0) {
-      logd_out[row] = L;
-      m_out[row] = mf;
-    }
+    for (int k = 0; k < 8; ++k) s[k] *= inv_sum;
+    L += __logf(sum);
+  }
+  const float lam = lamv ? lamv[row] : g.lam;
+  const float gs = gsv ? gsv[row] : 1.f;
+  const float mf = g.fixed_m ? 1.f : L == -INFINITY ? 0.f : 1.f / (1.f + (lam * dlr[row] + g.eps) * __expf(-L));
+  const float gl = glrv ? glrv[row] : g.fixed_m ? 1.f : 1.f - mf;
+  const float cs = gs * mf;
+  const uint4 wl = *reinterpret_cast<const uint4*>(Olr + row * g.d + 8 * u);
+  const __nv_bfloat162* lv = reinterpret_cast<const __nv_bfloat162*>(&wl);
+  uint32_t wo[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(lv[j]);
+    const __nv_bfloat162 o = __floats2bfloat162_rn(cs * s[2 * j] + gl * f.x, cs * s[2 * j + 1] + gl * f.y);
+    wo[j] = *reinterpret_cast<const uint32_t*>(&o);
+  }
+  *reinterpret_cast<uint4*>(O + row * g.d + 8 * u) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
+  reinterpret_cast<float4*>(Os + row * g.d + 8 * u)[0] = make_float4(s[0], s[1], s[2], s[3]);
+  reinterpret_cast<float4*>(Os + row * g.d + 8 * u)[1] = make_float4(s[4], s[5], s[6], s[7]);
+  if (u == 0) {
+    logd_out[row] = L;
+    m_out[row] = mf;
   }
 }
 
@@ -466,23 +463,26 @@ __global__ void lsh_invert_orders_kernel(const int* __restrict__ order, int* __r
 // [levels][BH][2][N].
 __global__ void lsh_collect_kernel(const float* __restrict__ src0, float* __restrict__ acc0,
                                    const float* __restrict__ src1, float* __restrict__ acc1,
-                                   const int* __restrict__ inv, int levels, int side, int want, Geom g) {
-  const int units = g.d / 8;
+                                   const int* __restrict__ inv, int levels, int side, int want, int units_log2,
+                                   Geom g) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (g.N << units_log2)) return;
+  const int r = e >> units_log2, u = e & ((1 << units_log2) - 1);
   const size_t rows = (size_t)g.BH * g.N;
-  const size_t total = rows * units;
-  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
-    const size_t row = e / units;
-    const int u = (int)(e % units);
-    const int bh = (int)(row / g.N), r = (int)(row % g.N);
-    float s0[8] = {}, s1[8] = {};
-    bool any = false;
-    for (int l = 0; l < levels; ++l) {
-      const int h = g.N >> (l + 1);
-      if (((r / h) & 1) != want) continue;
+  const size_t row = (size_t)bh * g.N + r;
+  float s0[8] = {}, s1[8] = {};
+  bool any = false;
+  // every level's slot row is loaded as soon as its position is known (predicated, unrolled)
+#pragma unroll
+  for (int l = 0; l < kMaxLevels; ++l) {
+    const int hl = 31 - __clz(g.N >> (l + 1));      // log2 of the half length
+    if (l < levels && ((r >> hl) & 1) == want) {
       any = true;
-      const size_t p = (size_t)l * rows + (size_t)bh * g.N +
-                       inv[(((size_t)l * g.BH + bh) * 2 + side) * g.N + r];
-      for (int t = 0; t < (src1 ? 2 : 1); ++t) {
+      const size_t p = (size_t)l * rows + (size_t)bh * g.N + inv[(((size_t)l * g.BH + bh) * 2 + side) * g.N + r];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (t == 1 && !src1) break;
         const float4* w = reinterpret_cast<const float4*>((t ? src1 : src0) + p * g.d + 8 * u);
         const float4 w0 = w[0], w1 = w[1];
         float* sv = t ? s1 : s0;
@@ -490,14 +490,16 @@ __global__ void lsh_collect_kernel(const float* __restrict__ src0, float* __rest
         sv[4] += w1.x; sv[5] += w1.y; sv[6] += w1.z; sv[7] += w1.w;
       }
     }
-    if (!any) continue;
-    for (int t = 0; t < (src1 ? 2 : 1); ++t) {
-      float4* a = reinterpret_cast<float4*>((t ? acc1 : acc0) + row * g.d + 8 * u);
-      const float* sv = t ? s1 : s0;
-      const float4 a0 = a[0], a1 = a[1];
-      a[0] = make_float4(a0.x + sv[0], a0.y + sv[1], a0.z + sv[2], a0.w + sv[3]);
-      a[1] = make_float4(a1.x + sv[4], a1.y + sv[5], a1.z + sv[6], a1.w + sv[7]);
-    }
+  }
+  if (!any) return;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    if (t == 1 && !src1) break;
+    float4* a = reinterpret_cast<float4*>((t ? acc1 : acc0) + row * g.d + 8 * u);
+    const float* sv = t ? s1 : s0;
+    const float4 a0 = a[0], a1 = a[1];
+    a[0] = make_float4(a0.x + sv[0], a0.y + sv[1], a0.z + sv[2], a0.w + sv[3]);
+    a[1] = make_float4(a1.x + sv[4], a1.y + sv[5], a1.z + sv[6], a1.w + sv[7]);
   }
 }
 
@@ -511,22 +513,27 @@ struct RowMoves {
   int n;
 };
 
-__global__ void gather_rows_kernel(RowMoves mv, const int* __restrict__ perm, int units, int levels, int half,
-                                   Geom g) {
-  const size_t rows = (size_t)g.BH * g.N;
-  const size_t total = (size_t)levels * rows * units;
-  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
-    const size_t row = e / units;                     // slot row: [levels][BH][N]
-    const int u = (int)(e % units);
-    const int l = (int)(row / rows);
-    const size_t hr = row % rows;
-    const int bh = (int)(hr / g.N), r = (int)(hr % g.N);
-    if (half >= 0 && ((r >> (31 - __clz(g.N >> (l + 1)))) & 1) != half) continue;
-    const size_t pr = (size_t)bh * g.N + perm[((size_t)l * g.BH + bh) * 2 * g.N + r];
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-      if (t < mv.n) mv.dst[t][row * units + u] = mv.src[t][pr * units + u];
+// One level-major virtual head per blockIdx.y (level l, head bh); x covers the rows it moves
+// (with half >= 0 only the rows of that half of each length-(N >> (l + 1)) pair of halves,
+// taken in order) times their 16-byte units.  N and the unit count are powers of two.
+__global__ void gather_rows_kernel(RowMoves mv, const int* __restrict__ perm, int units_log2, int half, Geom g) {
+  const int vh = blockIdx.y;
+  const int l = vh / g.BH, bh = vh - l * g.BH;
+  const int nrows = half >= 0 ? g.N >> 1 : g.N;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (nrows << units_log2)) return;
+  const int c = e >> units_log2, u = e & ((1 << units_log2) - 1);
+  int r = c;
+  if (half >= 0) {
+    const int hl = 31 - __clz(g.N >> (l + 1));      // log2 of the half length
+    r = ((c >> hl) << (hl + 1)) | (half << hl) | (c & ((1 << hl) - 1));
   }
+  const size_t pr = (size_t)bh * g.N + perm[((size_t)l * g.BH + bh) * 2 * g.N + r];
+  const size_t row = (size_t)vh * g.N + r;         // slot row: [levels][BH][N]
+  const size_t units = (size_t)1 << units_log2;
+#pragma unroll
+  for (int t = 0; t < 4; ++t)
+    if (t < mv.n) mv.dst[t][row * units + u] = mv.src[t][pr * units + u];
 }
 
 // Every level's selection and future tiles (halves of hb_l = n_t >> (l + 1) blocks): idx
@@ -647,10 +654,13 @@ cudaError_t launch_lsh_fuse(const void* Os0, const float* logd0, const void* Os_
                             const float* gs, const float* glr, void* O, void* Os, float* logd, float* m, const Geom& g,
                             cudaStream_t st) {
   if (levels > kMaxLevels) return cudaErrorInvalidValue;
+  const int units = g.d / 8;
+  if ((units & (units - 1)) || (g.N & (g.N - 1)) || g.BH > 65535) return cudaErrorInvalidValue;
+  const int units_log2 = 31 - __builtin_clz((unsigned)units);
   ProfScope ps("lsh_fuse", st);
-  lsh_fuse_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
+  lsh_fuse_kernel<<<dim3((unsigned)(((size_t)g.N * units + 255) / 256), g.BH), 256, 0, st>>>(
       (const float*)Os0, logd0, (const float*)Os_lv, logd_lv, inv_lv, levels,
-      (const __nv_bfloat16*)Olr, dlr, lam, gs, glr, (__nv_bfloat16*)O, (float*)Os, logd, m, g);
+      (const __nv_bfloat16*)Olr, dlr, lam, gs, glr, (__nv_bfloat16*)O, (float*)Os, logd, m, units_log2, g);
   return cudaGetLastError();
 }
 
@@ -663,10 +673,12 @@ cudaError_t launch_lsh_invert_orders(const int* order, int* inv, int levels, con
 cudaError_t launch_lsh_collect(const void* src0, float* acc0, const void* src1, float* acc1, const int* inv,
                                int levels, bool keys, const Geom& g, cudaStream_t st) {
   if (levels > kMaxLevels) return cudaErrorInvalidValue;
+  const int units = g.d / 8;
+  if ((units & (units - 1)) || (g.N & (g.N - 1)) || g.BH > 65535) return cudaErrorInvalidValue;
+  const int units_log2 = 31 - __builtin_clz((unsigned)units);
   ProfScope ps("lsh_collect", st);
-  lsh_collect_kernel<<<elementwise_blocks((size_t)g.BH * g.N * (g.d / 8)), 256, 0, st>>>(
-      (const float*)src0, acc0, (const float*)src1, acc1, inv, levels, keys ? 1 : 0, keys ? 0 : 1,
-      g);
+  lsh_collect_kernel<<<dim3((unsigned)(((size_t)g.N * units + 255) / 256), g.BH), 256, 0, st>>>(
+      (const float*)src0, acc0, (const float*)src1, acc1, inv, levels, keys ? 1 : 0, keys ? 0 : 1, units_log2, g);
   return cudaGetLastError();
 }
 
@@ -680,9 +692,13 @@ cudaError_t launch_gather_rows(const void* const* src, void* const* dst, int n, 
   }
   mv.n = n;
   const int units = row_bytes / 16;
+  if (units < 1 || (units & (units - 1)) || (g.N & (g.N - 1)) || levels < 1 || (size_t)levels * g.BH > 65535)
+    return cudaErrorInvalidValue;
+  const int units_log2 = 31 - __builtin_clz((unsigned)units);
+  const int nrows = half >= 0 ? g.N / 2 : g.N;
   ProfScope ps("sortlsh_gather", st);
-  gather_rows_kernel<<<elementwise_blocks((size_t)levels * g.BH * g.N * units), 256, 0, st>>>(mv, perm, units, levels,
-                                                                                              half, g);
+  gather_rows_kernel<<<dim3((unsigned)(((size_t)nrows * units + 255) / 256), levels * g.BH), 256, 0, st>>>(
+      mv, perm, units_log2, half, g);
   return cudaGetLastError();
 }
 
