@@ -58,10 +58,11 @@ constexpr uint32_t DQ_MISC = kTile * (2 + kDqKStages + kDqVStages);
 // TMEM: S and dP (fp32), the dQ accumulator, dS (bf16 pairs) double-buffered
 constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256, TM_DS = 384;
 constexpr int kDqThreads = 352;          // Q/dO + K producer, MMA, 8 softmax warps, V producer
+constexpr uint32_t kAccBox = 128 * 128;  // [128 rows][32 fp32] box of the low-rank dQ tile
 
 struct DqMisc {
   uint64_t qd_full, k_full[kDqKStages], k_empty[kDqKStages], v_full[kDqVStages], v_empty[kDqVStages], s_full,
-      st_free, ds_full[2], done;
+      st_free, ds_full[2], done, acc_full;
   uint32_t tmem_base;
   int abort_flag;
   int idx[2][32];         // selected blocks of the CTA's tile (PAIR: of its two tiles)
@@ -102,7 +103,8 @@ template <int D, bool PAIR>
 __global__ void __launch_bounds__(kDqThreads, 1)
     dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                 const __grid_constant__ CUtensorMap tmdQ, BwdArgs a, Geom g, uint32_t* err) {
+                 const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmAcc, BwdArgs a,
+                 Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   DqMisc* ms = reinterpret_cast<DqMisc*>(smem + DQ_MISC);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -137,6 +139,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     tc::mbar_init(&ms->ds_full[0], kSoftmaxThreads);
     tc::mbar_init(&ms->ds_full[1], kSoftmaxThreads);
     tc::mbar_init(&ms->done, 1);
+    tc::mbar_init(&ms->acc_full, 1);
     ms->abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -188,11 +191,23 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
         issued = j + 1;
       }
-      // every load is issued: bring the tile's low-rank dQ rows into L2 for the epilogue
-      if (kside && a.dQacc && row0 < g.N)
-        tc::prefetch_l2(a.dQacc + (head + row0) * D, (uint32_t)min(kT, g.N - row0) * D * 4u);
+      // the V ring is free once the last dP products are done: the tile's low-rank dQ rows
+      // (fp32, 32-column boxes, 128-byte swizzle) go there for the epilogue
+      bool acc_issued = false;
+      if (!kside && a.dQacc && issued == n_sel) {
+        bool free_ring = true;
+        for (int j = (n_sel > NS ? n_sel - NS : 0); free_ring && j < n_sel; ++j)
+          free_ring = wait_or_abort(&empty[j % NS], (j / NS) & 1, ms, err, 2u);
+        if (free_ring) {
+          tc::mbar_arrive_expect_tx(&ms->acc_full, 128u * D * 4);
+          for (int b = 0; b < D / 32; ++b)
+            tc::tma_load_3d(smem + dq_v(0) + b * kAccBox, &tmAcc, &ms->acc_full, 32 * b, row0, bh);
+          acc_issued = true;
+        }
+      }
       if (kside) tc::mbar_wait(&ms->qd_full, 0);
       for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j) tc::mbar_wait(&full[j % NS], (j / NS) & 1);
+      if (acc_issued) tc::mbar_wait(&ms->acc_full, 0);   // no copy in flight when the CTA exits
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -308,20 +323,20 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     }
     // ---------------- epilogue: dQ = scale dQ_sparse + dQ_lowrank, bf16 TMA store ----------------
     const int col0 = H * half;                       // this thread's dQ columns [col0, col0 + H)
-    // the low-rank part is read while the last products run
-    const bool use_acc = alive && row_ok && a.dQacc;
-    float4 av[H / 4];
-    if (use_acc) {
-      const float4* acc = reinterpret_cast<const float4*>(a.dQacc + (head + qrow) * D + col0);
-#pragma unroll
-      for (int i = 0; i < H / 4; ++i) av[i] = acc[i];
-    }
     bool have = false;
     if (alive && n_sel > 0) {
       alive = __all_sync(0xffffffffu, wait_or_abort(&ms->done, 0, ms, err, 256u));
       have = alive;
       if (have) tc::tc_fence_after();
     }
+    // the low-rank part, brought into the V ring by the V producer
+    if (alive && a.dQacc) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->acc_full, 0, ms, err, 512u));
+    const bool use_acc = alive && row_ok && a.dQacc;
+    // fp32 element (row, c) of the low-rank tile: box c / 32, 16-byte chunk (c % 32) / 4 swizzled by row
+    auto acc4 = [&](int c) -> float4 {
+      return *reinterpret_cast<const float4*>(smem + dq_v(0) + (uint32_t)(c >> 5) * kAccBox + (uint32_t)row * 128u +
+                                              ((uint32_t)(((c & 31) >> 2) ^ (row & 7)) << 4));
+    };
     // every product has completed: stage the bf16 tile in the Q buffer, 32 columns at a time
     // (with a row map, write each row straight to the caller's row instead)
     unsigned char* orow = smem + DQ_Q + (col0 >> 6) * kSlab + row * 128;
@@ -341,10 +356,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] *= g.scale;
       }
-      if (use_acc && alive) {
+      if (use_acc) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const float4 v = av[8 * c + q];
+          const float4 v = acc4(col0 + 32 * c + 4 * q);
           o[4 * q] += v.x; o[4 * q + 1] += v.y; o[4 * q + 2] += v.z; o[4 * q + 3] += v.w;
         }
       }
@@ -871,14 +886,32 @@ static bool map_d(CUtensorMap* m, const void* base, const Geom& g, int rows) {
   return tc::map_rows_bf16_pitch(m, base, g.d, g.d, g.N, g.BH, rows);
 }
 
+// fp32 [BH][N][d] low-rank gradient rows in boxes of 32 columns x 128 rows, 128-byte swizzle.
+static bool map_acc_f32(CUtensorMap* m, const float* base, const Geom& g) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)g.d, (cuuint64_t)g.N, (cuuint64_t)g.BH};
+  cuuint64_t strides[2] = {(cuuint64_t)g.d * 4, (cuuint64_t)g.N * g.d * 4};
+  cuuint32_t box[3] = {32, (cuuint32_t)kT, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, bool PAIR>
 static cudaError_t dq_t(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
   constexpr int TB = PAIR ? 64 : 128;
   if (PAIR && a.tile_list && (a.n_list & 1)) return cudaErrorInvalidValue;   // tile pairs
-  CUtensorMap mq, mk, mv, mdo, mdq;
+  CUtensorMap mq, mk, mv, mdo, mdq, macc;
   if (!map_d(&mq, a.Q, g, kT) || !map_d(&mk, a.K, g, TB) || !map_d(&mv, a.V, g, TB) || !map_d(&mdo, a.dO, g, kT) ||
       !map_d(&mdq, a.dQ, g, kT))
     return cudaErrorInvalidValue;
+  if (a.dQacc) {
+    if (!map_acc_f32(&macc, a.dQacc, g)) return cudaErrorInvalidValue;
+  } else {
+    macc = mdq;                                      // not read without a low-rank part
+  }
   const size_t smem = DQ_MISC + sizeof(DqMisc);
   static_assert(DQ_MISC + sizeof(DqMisc) <= 232448, "shared memory per CTA");
   auto kern = dq_tc_kernel<D, PAIR>;
@@ -886,7 +919,7 @@ static cudaError_t dq_t(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStre
   if (e != cudaSuccess) return e;
   const int units = a.tile_list ? (PAIR ? a.n_list / 2 : a.n_list) : (PAIR ? (g.n_t + 1) / 2 : g.n_t);
   ProfScope ps("dq_tc", st);
-  kern<<<dim3(units, g.BH), kDqThreads, smem, st>>>(mq, mk, mv, mdo, mdq, a, g, err);
+  kern<<<dim3(units, g.BH), kDqThreads, smem, st>>>(mq, mk, mv, mdo, mdq, macc, a, g, err);
   return cudaGetLastError();
 }
 

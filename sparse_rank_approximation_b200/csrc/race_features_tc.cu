@@ -28,12 +28,17 @@ constexpr int kC = 128;                           // rows per CTA
 constexpr uint32_t kSlab = 128 * 128;             // [128 rows][64 bf16], 128-byte swizzle
 constexpr int kThreads = 192;
 constexpr int kMaxNW = 64;                        // projections per row: 4 L <= 64
-constexpr uint32_t F_X = 0;                       // X tile, up to 2 slabs
-constexpr uint32_t F_WH = 2 * kSlab;              // W hi [NW][d], up to 2 slabs of kMaxNW rows
-constexpr uint32_t kWSlab = kMaxNW * 128;
-constexpr uint32_t F_WL = F_WH + 2 * kWSlab;
-constexpr uint32_t F_BARS = F_WL + 2 * kWSlab;
-static_assert(F_BARS >= 4 * kSlab, "Phi staging: up to 256 columns over the X and W tiles");
+// Shared memory for NW projections: the X tile (2 slabs), W hi and W lo ([NW][d], 2 slabs of
+// NW rows each), the barriers after them; Phi (rp / 64 slabs, rp = 2 NW) is staged over X and
+// W once the products have read them.  NW = 32: 48 KB, four CTAs per SM.
+constexpr uint32_t F_X = 0;
+template <int NW> struct FeatLayout {
+  static constexpr uint32_t kWSlab = (uint32_t)NW * 128;
+  static constexpr uint32_t kWH = 2 * kSlab;
+  static constexpr uint32_t kWL = kWH + 2 * kWSlab;
+  static constexpr uint32_t kBars = kWL + 2 * kWSlab;
+  static_assert(kBars >= (uint32_t)(2 * NW / 64) * kSlab, "Phi staging over the X and W tiles");
+};
 
 struct FeatBars {
   uint64_t in_full, acc_full;
@@ -62,13 +67,14 @@ __device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 128;\n
 }  // namespace
 
 template <int D, int NW>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, NW == 32 ? 4 : 1)
     race_features_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPQ,
                             const __grid_constant__ CUtensorMap tmPK, float* __restrict__ hQ, float* __restrict__ hK,
                             float* __restrict__ nQ, float* __restrict__ nK, Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  FeatBars* ms = reinterpret_cast<FeatBars*>(smem + F_BARS);
+  using FL = FeatLayout<NW>;
+  FeatBars* ms = reinterpret_cast<FeatBars*>(smem + FL::kBars);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x, bh = blockIdx.y, side = blockIdx.z;
   if (smem_u32(smem) & 1023u) {
@@ -97,8 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive_expect_tx(&ms->in_full, 128u * D * 2 + 2 * kWD);
       for (int s = 0; s < D / 64; ++s) {
         tc::tma_load_3d(smem + F_X + s * kSlab, side ? &tmK : &tmQ, &ms->in_full, 64 * s, c * kC, bh);
-        tc::tma_load_3d(smem + F_WH + s * kWSlab, &tmW, &ms->in_full, 64 * s, 0, 0);
-        tc::tma_load_3d(smem + F_WL + s * kWSlab, &tmW, &ms->in_full, 64 * s, 0, 1);
+        tc::tma_load_3d(smem + FL::kWH + s * FL::kWSlab, &tmW, &ms->in_full, 64 * s, 0, 0);
+        tc::tma_load_3d(smem + FL::kWL + s * FL::kWSlab, &tmW, &ms->in_full, 64 * s, 0, 1);
       }
       tc::mbar_wait(&ms->in_full, 0);                 // no copy in flight when the CTA exits
     }
@@ -112,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int part = 0; part < 2; ++part)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            tc::mma_bf16(tmem, desc_k(d0, F_X, kk, kSlab), desc_k(d0, part ? F_WL : F_WH, kk, kWSlab), idesc,
+            tc::mma_bf16(tmem, desc_k(d0, F_X, kk, kSlab), desc_k(d0, part ? FL::kWL : FL::kWH, kk, FL::kWSlab), idesc,
                          (part > 0 || kk > 0) ? 1u : 0u);
       }
       tc::mma_commit(&ms->acc_full);
@@ -215,8 +221,8 @@ static cudaError_t features_t(const void* Q, const void* K, const void* wsplit, 
       !tc::map_rows_bf16_pitch(&mpq, phiQ, g.rp, g.rp, g.N, g.BH, kC) ||
       !tc::map_rows_bf16_pitch(&mpk, phiK, g.rp, g.rp, g.N, g.BH, kC))
     return cudaErrorInvalidValue;
-  const size_t smem = F_BARS + sizeof(FeatBars);
-  static_assert(F_BARS + sizeof(FeatBars) <= 232448, "shared memory per CTA");
+  const size_t smem = FeatLayout<NW>::kBars + sizeof(FeatBars);
+  static_assert(FeatLayout<NW>::kBars + sizeof(FeatBars) <= 232448, "shared memory per CTA");
   auto kern = race_features_tc_kernel<D, NW>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
