@@ -427,6 +427,7 @@ constexpr int kKvThreads = 320;
 
 struct KvMisc {
   uint64_t kv_full, qd_full[kStages], qd_empty[kStages], s_full[2], p_half[2], done;
+  uint64_t kv_read, st1_read, acck_full, accv_full;   // K / V and stage 1 free; low-rank rows landed
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -479,7 +480,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                    const __grid_constant__ CUtensorMap tmSc, const __grid_constant__ CUtensorMap tmdK,
-                   const __grid_constant__ CUtensorMap tmdV, BwdArgs a, Geom g, uint32_t* err) {
+                   const __grid_constant__ CUtensorMap tmdV, const __grid_constant__ CUtensorMap tmKacc,
+                   const __grid_constant__ CUtensorMap tmVacc, BwdArgs a, Geom g, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   KvMisc* ms = reinterpret_cast<KvMisc*>(smem + KV_MISC);
   int* units = reinterpret_cast<int*>(smem + KV_UNITS);       // [2][kMaxUnits] query tiles of the block(s)
@@ -515,6 +517,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   }
   const int n_ua = n_ut[0], n_ub = n_ut[1];
   const int n_u = max(n_ua, n_ub);
+  const int last1 = n_u >= 2 ? ((n_u - 1) & 1 ? n_u - 1 : n_u - 2) : -1;   // last tile staged in stage 1
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->kv_full, 1);
     for (int s = 0; s < kStages; ++s) {
@@ -523,6 +526,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     }
     tc::mbar_init(&ms->s_full[0], 1);
     tc::mbar_init(&ms->s_full[1], 1);
+    tc::mbar_init(&ms->kv_read, 1);
+    tc::mbar_init(&ms->st1_read, 1);
+    tc::mbar_init(&ms->acck_full, 1);
+    tc::mbar_init(&ms->accv_full, 1);
     tc::mbar_init(&ms->p_half[0], kSoftmaxThreads);
     tc::mbar_init(&ms->p_half[1], kSoftmaxThreads);
     tc::mbar_init(&ms->done, 1);
@@ -568,17 +575,31 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         }
         issued = u + 1;
       }
-      // every load is issued: bring the block's low-rank dK and dV rows into L2 for the epilogue
-      for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
-        const int kr = PAIR ? 64 * pb[h] : key0;
-        if ((PAIR && pb[h] < 0) || kr >= g.N) continue;
-        const uint32_t bytes = (uint32_t)min(TB, g.N - kr) * D * 4u;
-        if (a.dKacc) tc::prefetch_l2(a.dKacc + (head + kr) * D, bytes);
-        if (a.dVacc) tc::prefetch_l2(a.dVacc + (head + kr) * D, bytes);
+      // the block's fp32 low-rank rows for the epilogue (32-column boxes, 128-byte swizzle): dV's
+      // into stage 1 once no tile reads it, dK's into the K / V tiles once the last scores are done
+      bool accv = false, acck = false;
+      auto load_acc = [&](const CUtensorMap* map, uint64_t* bar, uint32_t dst) {
+        const int nh = PAIR ? (pb[1] >= 0 ? 2 : 1) : 1;
+        tc::mbar_arrive_expect_tx(bar, (uint32_t)(D / 32) * nh * TB * 128u);
+        for (int b = 0; b < D / 32; ++b)
+          for (int h = 0; h < nh; ++h)
+            tc::tma_load_3d(smem + dst + b * kAccBox + h * 64 * 128, map, bar, 32 * b, PAIR ? 64 * pb[h] : key0, bh);
+      };
+      if (issued == n_u && a.dVacc && (last1 < 0 || wait_or_abort(&ms->st1_read, 0, ms, err, 1u))) {
+        load_acc(&tmVacc, &ms->accv_full, kv_q(1));
+        accv = true;
+      }
+      // (with no tile, the K / V copies must have landed before their space is reused)
+      if (issued == n_u && a.dKacc &&
+          (n_u == 0 ? wait_or_abort(&ms->kv_full, 0, ms, err, 1u) : wait_or_abort(&ms->kv_read, 0, ms, err, 1u))) {
+        load_acc(&tmKacc, &ms->acck_full, KV_K);
+        acck = true;
       }
       tc::mbar_wait(&ms->kv_full, 0);
       for (int u = (issued > kStages ? issued - kStages : 0); u < issued; ++u)
         tc::mbar_wait(&ms->qd_full[u % kStages], (u / kStages) & 1);
+      if (accv) tc::mbar_wait(&ms->accv_full, 0);      // no copy in flight when the CTA exits
+      if (acck) tc::mbar_wait(&ms->acck_full, 0);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -615,6 +636,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                           (u > 0 || kk > 0) ? 1u : 0u);
         }
         if (h == 1) tc::mma_commit(&ms->qd_empty[s]);   // the unit's Q / dO stage is read
+        if (h == 1 && u == last1) tc::mma_commit(&ms->st1_read);
         return true;
       };
       if constexpr (!TL::kTwoBuf) {
@@ -638,6 +660,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             tc::mma_bf16(tmem + TL::kDp, tc::desc_adv(v_desc, off), tc::desc_adv(dob, off), idS, kk > 0 ? 1u : 0u);
           }
           tc::mma_commit(&ms->s_full[0]);
+          if (u == n_u - 1) tc::mma_commit(&ms->kv_read);   // every score product has read K and V
           const uint64_t domb = tc::desc_adv(domn_desc, so), qmb = tc::desc_adv(qmn_desc, so);
           for (int h = 0; ok && h < 2; ++h) {
             ok = wait_or_abort(&ms->p_half[h], u & 1, ms, err, 4u);
@@ -657,6 +680,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             }
           }
           if (ok) tc::mma_commit(&ms->qd_empty[s]);
+          if (ok && u == last1) tc::mma_commit(&ms->st1_read);
         }
       } else {
         // two buffers: the scores of pass i + 1 run on the tensor cores while the softmax warps
@@ -682,6 +706,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             tc::mma_bf16(st + TL::kDp, tc::desc_adv(v_desc, off), tc::desc_adv(dob, off), idS, kk > 0 ? 1u : 0u);
           }
           tc::mma_commit(&ms->s_full[h]);
+          if (i == 2 * n_u - 1) tc::mma_commit(&ms->kv_read);   // every score product has read K and V
           // the previous pass's products, behind this pass's scores
           if (i >= 1) {
             ok = issue_grads(i - 1);
@@ -751,16 +776,6 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     const int hq = grp;
     const int col0 = H * hq;                         // this thread's columns [col0, col0 + H)
     const int ch0 = (col0 & 63) >> 3;
-    // the low-rank dK part is read while the last products run, dV's (from L2) once dK is staged
-    float4 av[H / 4];
-    auto load_acc = [&](const float* accp) {
-      if (accp && alive && key_ok) {
-        const float4* p = reinterpret_cast<const float4*>(accp + (head + (size_t)krow) * D + col0);
-#pragma unroll
-        for (int i = 0; i < H / 4; ++i) av[i] = p[i];
-      }
-    };
-    load_acc(a.dKacc);
     bool have = false;
     if (alive && n_u > 0) {
       alive = __all_sync(0xffffffffu, wait_or_abort(&ms->done, 0, ms, err, 512u));
@@ -771,8 +786,17 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
       const float mul = which == 0 ? g.scale : 1.f;
+      // the low-rank part, brought into shared memory by the producer
+      if (alive && (which == 0 ? a.dKacc : a.dVacc))
+        alive = __all_sync(0xffffffffu,
+                           wait_or_abort(which == 0 ? &ms->acck_full : &ms->accv_full, 0, ms, err, 1024u));
       const bool use_acc = (which == 0 ? a.dKacc : a.dVacc) && alive && key_ok;
-      if (which == 1) load_acc(a.dVacc);
+      const uint32_t acc_base = which == 0 ? KV_K : kv_q(1);
+      // fp32 element (row, c): box c / 32, 16-byte chunk (c % 32) / 4 swizzled by the row
+      auto acc4 = [&](int cc) -> float4 {
+        return *reinterpret_cast<const float4*>(smem + acc_base + (uint32_t)(cc >> 5) * kAccBox + (uint32_t)row * 128u +
+                                                ((uint32_t)(((cc & 31) >> 2) ^ (row & 7)) << 4));
+      };
       unsigned char* orow = smem + (which == 0 ? kv_q(0) : kv_do(0)) + (col0 >> 6) * kSlab + row * 128;
       // with a row map, write each key row straight to the caller's row instead
       uint4* grow = a.k_rows && key_ok && alive
@@ -795,7 +819,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         if (use_acc) {
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const float4 x = av[8 * c + q];
+            const float4 x = acc4(col0 + 32 * c + 4 * q);
             o[4 * q] += x.x; o[4 * q + 1] += x.y; o[4 * q + 2] += x.z; o[4 * q + 3] += x.w;
           }
         }
@@ -886,13 +910,13 @@ static bool map_d(CUtensorMap* m, const void* base, const Geom& g, int rows) {
   return tc::map_rows_bf16_pitch(m, base, g.d, g.d, g.N, g.BH, rows);
 }
 
-// fp32 [BH][N][d] low-rank gradient rows in boxes of 32 columns x 128 rows, 128-byte swizzle.
-static bool map_acc_f32(CUtensorMap* m, const float* base, const Geom& g) {
+// fp32 [BH][N][d] low-rank gradient rows in boxes of 32 columns x `rows` rows, 128-byte swizzle.
+static bool map_acc_f32(CUtensorMap* m, const float* base, const Geom& g, int rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)g.d, (cuuint64_t)g.N, (cuuint64_t)g.BH};
   cuuint64_t strides[2] = {(cuuint64_t)g.d * 4, (cuuint64_t)g.N * g.d * 4};
-  cuuint32_t box[3] = {32, (cuuint32_t)kT, 1};
+  cuuint32_t box[3] = {32, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -908,7 +932,7 @@ static cudaError_t dq_t(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStre
       !map_d(&mdq, a.dQ, g, kT))
     return cudaErrorInvalidValue;
   if (a.dQacc) {
-    if (!map_acc_f32(&macc, a.dQacc, g)) return cudaErrorInvalidValue;
+    if (!map_acc_f32(&macc, a.dQacc, g, kT)) return cudaErrorInvalidValue;
   } else {
     macc = mdq;                                      // not read without a low-rank part
   }
@@ -945,10 +969,15 @@ static bool map_scalars(CUtensorMap* m, const void* base, int N, int BH, int row
 template <int D, bool PAIR>
 static cudaError_t dkdv_t(const BwdArgs& a, const Geom& g, uint32_t* err, cudaStream_t st) {
   constexpr int TB = PAIR ? 64 : 128;
-  CUtensorMap mk, mv, mq, mdo, msc, mdk, mdv;
+  CUtensorMap mk, mv, mq, mdo, msc, mdk, mdv, mka, mva;
   if (!map_d(&mk, a.K, g, TB) || !map_d(&mv, a.V, g, TB) || !map_d(&mq, a.Q, g, TB) || !map_d(&mdo, a.dO, g, TB) ||
       !map_scalars(&msc, a.rs.packed, g.N, g.BH, TB) || !map_d(&mdk, a.dK, g, TB) || !map_d(&mdv, a.dV, g, TB))
     return cudaErrorInvalidValue;
+  // maps of the low-rank parts (not read when absent)
+  if ((a.dKacc && !map_acc_f32(&mka, a.dKacc, g, TB)) || (a.dVacc && !map_acc_f32(&mva, a.dVacc, g, TB)))
+    return cudaErrorInvalidValue;
+  if (!a.dKacc) mka = mk;
+  if (!a.dVacc) mva = mv;
   const size_t smem = KV_MISC + sizeof(KvMisc);
   static_assert(KV_MISC + sizeof(KvMisc) <= 232448, "shared memory per CTA");
   auto kern = dkdv_tc_kernel<D, PAIR>;
@@ -959,7 +988,7 @@ static cudaError_t dkdv_t(const BwdArgs& a, const Geom& g, uint32_t* err, cudaSt
   // PAIR: two consecutive entries of that order per CTA
   const int nb = a.n_kv ? a.n_kv : g.n_t;
   const int ctas = PAIR ? (nb + 1) / 2 : nb;
-  kern<<<dim3(g.BH, ctas), kKvThreads, smem, st>>>(mk, mv, mq, mdo, msc, mdk, mdv, a, g, err);
+  kern<<<dim3(g.BH, ctas), kKvThreads, smem, st>>>(mk, mv, mq, mdo, msc, mdk, mdv, mka, mva, a, g, err);
   return cudaGetLastError();
 }
 
