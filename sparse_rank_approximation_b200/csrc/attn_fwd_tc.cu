@@ -81,10 +81,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // FMA instructions only: hi keeps the top 16 bits of each float (sign, exponent, 7 mantissa
 // bits), lo the top 16 bits of the exact remainder, so hi + lo is within 2^-15 of each value.
 // a sits in the low half of each word, b in the high half.
-__device__ __forceinline__ void split_trunc(float a, float b, uint32_t& hi, uint32_t& lo) {
+// ab holds the same pair as packed fp32 lanes, so both remainders take one f32x2 subtraction.
+__device__ __forceinline__ void split_trunc(float a, float b, uint64_t ab, uint32_t& hi, uint32_t& lo) {
   const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
   hi = __byte_perm(ua, ub, 0x7632);
-  const float ra = a - __uint_as_float(ua & 0xffff0000u), rb = b - __uint_as_float(ub & 0xffff0000u);
+  float ra, rb;
+  tc::f2_unpack(tc::f2_sub(ab, tc::f2_pack(__uint_as_float(ua & 0xffff0000u), __uint_as_float(ub & 0xffff0000u))), ra,
+                rb);
   lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
 }
 
@@ -152,6 +155,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     ms->limit_ns = g.wait_ns;
     ms->abort_flag = 0;
     tc::fence_barrier_init();
+    // Q does not depend on the selection: its copy starts before anything else
+    tc::mbar_arrive_expect_tx(&ms->q_full, 128u * D * 2);
+    for (int sl = 0; sl < D / 64; ++sl) tc::tma_load_3d(smem + L::kQ + sl * kSlab, &tmQ, &ms->q_full, 64 * sl, row0, bh);
+    tc::prefetch_tensormap(&tmK);
+    tc::prefetch_tensormap(&tmV);
   }
   if (threadIdx.x < 32) {
     ms->idx[0][threadIdx.x] = threadIdx.x < g.k ? idx_a[threadIdx.x] : -1;
@@ -176,8 +184,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ================= TMA producer: Q, the K and V rings, O_lr =================
     if (lane == 0) {
       constexpr uint32_t kTD = 128u * D * 2;      // bytes of a [128][D] tile
-      tc::mbar_arrive_expect_tx(&ms->q_full, kTD);
-      for (int sl = 0; sl < D / 64; ++sl) tc::tma_load_3d(smem + L::kQ + sl * kSlab, &tmQ, &ms->q_full, 64 * sl, row0, bh);
       bool alive = true;
       int k_issued = 0, v_issued = 0;
       // K_j and V_j in consumption order; a stage is reloaded once the product that read it is done
@@ -336,7 +342,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         // P_j as bf16 hi + lo pairs, part 1 (in registers) and then part 0 (read again)
         const float msub = m_used == -INFINITY ? 0.f : m_used;
-        float rs0 = 0.f, rs1 = 0.f;
+        // pairs of columns in packed fp32 lanes: x = s sl2 - m, the row sum and the lo remainder
+        // each take one f32x2 instruction per pair
+        const uint64_t sl2x2 = tc::f2_pack(sl2, sl2), negm2 = tc::f2_pack(-msub, -msub);
+        uint64_t rs2 = tc::f2_pack(0.f, 0.f);
 #pragma unroll 1
         for (int part = 1; part >= 0; --part) {
           if (part == 0) load_part(0);
@@ -345,17 +354,20 @@ __global__ void __launch_bounds__(kThreads, 2)
             uint32_t w[8], wl[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float x0 = fmaf(sv[16 * q + 2 * e], sl2, -msub), x1 = fmaf(sv[16 * q + 2 * e + 1], sl2, -msub);
+              float x0, x1;
+              tc::f2_unpack(tc::f2_fma(tc::f2_pack(sv[16 * q + 2 * e], sv[16 * q + 2 * e + 1]), sl2x2, negm2), x0, x1);
               const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-              rs0 += p0;
-              rs1 += p1;
-              split_trunc(p0, p1, w[e], wl[e]);
+              const uint64_t p2 = tc::f2_pack(p0, p1);
+              rs2 = tc::f2_add(rs2, p2);
+              split_trunc(p0, p1, p2, w[e], wl[e]);
             }
             const uint32_t col = tmem + lane_base + TM_S + 64 * half + 32 * part + 16 * q;
             tc::tmem_st8(col, w);
             tc::tmem_st8(col + kPLo, wl);
           }
         }
+        float rs0, rs1;
+        tc::f2_unpack(rs2, rs0, rs1);
         lp += rs0 + rs1;
         // O holds the products through block j-1 (complete: S_j was issued after them and its
         // completion was signalled); a moved reference max rescales this half of its columns

@@ -79,18 +79,24 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, M*
 
 // dS = P (cs dP - Delta) for one thread's 64 keys of a query row, as bf16 pairs;
 // MASK: keys after column `lim` get P = 0.
+// Pairs of columns go through packed fp32 lanes (one f32x2 instruction per pair and step).
 template <bool MASK>
 __device__ __forceinline__ void dq_softmax_cols(const float (&sv)[64], const float (&dp)[64], float sl2, float lg2,
                                                 float cs, float Dl, int lim, uint32_t (&w)[32]) {
+  const uint64_t sl2x2 = tc::f2_pack(sl2, sl2), neg_lg2 = tc::f2_pack(-lg2, -lg2);
+  const uint64_t cs2 = tc::f2_pack(cs, cs), neg_dl = tc::f2_pack(-Dl, -Dl);
 #pragma unroll
   for (int c = 0; c < 64; c += 2) {
-    float p0 = ex2_approx(fmaf(sv[c], sl2, -lg2));
-    float p1 = ex2_approx(fmaf(sv[c + 1], sl2, -lg2));
+    float x0, x1;
+    tc::f2_unpack(tc::f2_fma(tc::f2_pack(sv[c], sv[c + 1]), sl2x2, neg_lg2), x0, x1);
+    float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
     if (MASK) {
       p0 = c > lim ? 0.f : p0;
       p1 = c + 1 > lim ? 0.f : p1;
     }
-    w[c >> 1] = pack_bf16(p0 * fmaf(cs, dp[c], -Dl), p1 * fmaf(cs, dp[c + 1], -Dl));
+    float d0, d1;
+    tc::f2_unpack(tc::f2_mul(tc::f2_pack(p0, p1), tc::f2_fma(cs2, tc::f2_pack(dp[c], dp[c + 1]), neg_dl)), d0, d1);
+    w[c >> 1] = pack_bf16(d0, d1);
   }
 }
 
@@ -142,6 +148,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     tc::mbar_init(&ms->acc_full, 1);
     ms->abort_flag = 0;
     tc::fence_barrier_init();
+    // Q and dO do not depend on the selection: their copies start before anything else
+    tc::mbar_arrive_expect_tx(&ms->qd_full, 2 * 128u * D * 2);
+    for (int sl = 0; sl < D / 64; ++sl) {
+      tc::tma_load_3d(smem + DQ_Q + sl * kSlab, &tmQ, &ms->qd_full, 64 * sl, row0, bh);
+      tc::tma_load_3d(smem + DQ_DO + sl * kSlab, &tmdO, &ms->qd_full, 64 * sl, row0, bh);
+    }
+    tc::prefetch_tensormap(&tmK);
+    tc::prefetch_tensormap(&tmV);
   }
   if (threadIdx.x < 32) {
     ms->idx[0][threadIdx.x] = threadIdx.x < g.k ? idx_a[threadIdx.x] : -1;
@@ -170,13 +184,6 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       uint64_t* full = kside ? ms->k_full : ms->v_full;
       uint64_t* empty = kside ? ms->k_empty : ms->v_empty;
       constexpr uint32_t kTD = 128u * D * 2;      // bytes of a [128][D] tile
-      if (kside) {
-        tc::mbar_arrive_expect_tx(&ms->qd_full, 2 * kTD);
-        for (int sl = 0; sl < D / 64; ++sl) {
-          tc::tma_load_3d(smem + DQ_Q + sl * kSlab, &tmQ, &ms->qd_full, 64 * sl, row0, bh);
-          tc::tma_load_3d(smem + DQ_DO + sl * kSlab, &tmdO, &ms->qd_full, 64 * sl, row0, bh);
-        }
-      }
       int issued = 0;
       for (int j = 0; j < n_sel; ++j) {
         const int s = j % NS;
@@ -503,21 +510,6 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     if (threadIdx.x == 0 && err) atomicOr(err, 0x80000000u);
     return;
   }
-  int n_ut[2] = {0, 0};
-  if (g.k > 0) {
-    const int* of = a.offs + (size_t)bh * (g.n_t + 1);
-    const int* list = a.tiles + (size_t)bh * g.n_t * g.k;
-    for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
-      const int bb = pb[h];
-      if (bb < 0) break;
-      const int e0 = of[bb];
-      n_ut[h] = min(of[bb + 1] - e0, kMaxUnits);
-      for (int i = threadIdx.x; i < n_ut[h]; i += kKvThreads) units[h * kMaxUnits + i] = list[e0 + i];
-    }
-  }
-  const int n_ua = n_ut[0], n_ub = n_ut[1];
-  const int n_u = max(n_ua, n_ub);
-  const int last1 = n_u >= 2 ? ((n_u - 1) & 1 ? n_u - 1 : n_u - 2) : -1;   // last tile staged in stage 1
   if (threadIdx.x == 0) {
     tc::mbar_init(&ms->kv_full, 1);
     for (int s = 0; s < kStages; ++s) {
@@ -535,7 +527,37 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     tc::mbar_init(&ms->done, 1);
     ms->abort_flag = 0;
     tc::fence_barrier_init();
+    // K and V of the block(s) do not depend on the query tiles: their copies start first
+    constexpr uint32_t kTD = 128u * D * 2;
+    tc::mbar_arrive_expect_tx(&ms->kv_full, 2 * kTD);
+    // PAIR: block pb[0] in key rows 0-63, pb[1] in rows 64-127 (a missing one stages pb[0])
+    for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
+      const int kr = PAIR ? 64 * (pb[h] >= 0 ? pb[h] : pb[0]) : key0;
+      for (int sl = 0; sl < D / 64; ++sl) {
+        tc::tma_load_3d(smem + KV_K + sl * kSlab + h * 64 * 128, &tmK, &ms->kv_full, 64 * sl, kr, bh);
+        tc::tma_load_3d(smem + KV_V + sl * kSlab + h * 64 * 128, &tmV, &ms->kv_full, 64 * sl, kr, bh);
+      }
+    }
+    tc::prefetch_tensormap(&tmQ);
+    tc::prefetch_tensormap(&tmdO);
+    tc::prefetch_tensormap(&tmSc);
   }
+  int n_ut[2] = {0, 0};
+  if (g.k > 0) {
+    const int* of = a.offs + (size_t)bh * (g.n_t + 1);
+    const int* list = a.tiles + (size_t)bh * g.n_t * g.k;
+    for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
+      const int bb = pb[h];
+      if (bb < 0) break;
+      const int e0 = of[bb];
+      n_ut[h] = min(of[bb + 1] - e0, kMaxUnits);
+      for (int i = threadIdx.x; i < n_ut[h]; i += kKvThreads) units[h * kMaxUnits + i] = list[e0 + i];
+    }
+  }
+  const int n_ua = n_ut[0], n_ub = n_ut[1];
+  const int n_u = max(n_ua, n_ub);
+  const int last1 = n_u >= 2 ? ((n_u - 1) & 1 ? n_u - 1 : n_u - 2) : -1;   // last tile staged in stage 1
+
   if (warp == 1) {
     tc::tmem_alloc(&ms->tmem_base, 512);
     tc::tmem_relinquish();
@@ -549,15 +571,6 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       constexpr uint32_t kTD = 128u * D * 2;      // bytes of a [128][D] tile
-      tc::mbar_arrive_expect_tx(&ms->kv_full, 2 * kTD);
-      // PAIR: block pb[0] in key rows 0-63, pb[1] in rows 64-127 (a missing one stages pb[0])
-      for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
-        const int kr = PAIR ? 64 * (pb[h] >= 0 ? pb[h] : pb[0]) : key0;
-        for (int sl = 0; sl < D / 64; ++sl) {
-          tc::tma_load_3d(smem + KV_K + sl * kSlab + h * 64 * 128, &tmK, &ms->kv_full, 64 * sl, kr, bh);
-          tc::tma_load_3d(smem + KV_V + sl * kSlab + h * 64 * 128, &tmV, &ms->kv_full, 64 * sl, kr, bh);
-        }
-      }
       int issued = 0;
       for (int u = 0; u < n_u; ++u) {
         const int s = u % kStages;
