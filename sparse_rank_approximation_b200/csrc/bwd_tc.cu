@@ -415,7 +415,9 @@ __host__ __device__ constexpr uint32_t kv_q(int s) { return 2 * kTile + s * 2 * 
 __host__ __device__ constexpr uint32_t kv_do(int s) { return kv_q(s) + kTile; }            // dO tile, stage s
 constexpr uint32_t KV_SC = 2 * kTile + kStages * 2 * kTile;                   // scalars [stage][128] float4
 constexpr int kMaxUnits = 1024;
-constexpr uint32_t KV_UNITS = KV_SC + kStages * 128 * 16;                     // query tiles of the block(s)
+// the scalars as three arrays per stage (-log2 d_s, cs, -Delta), for 8-byte column-pair loads
+constexpr uint32_t KV_SOA = KV_SC + kStages * 128 * 16;
+constexpr uint32_t KV_UNITS = KV_SOA + kStages * 3 * 128 * 4;                 // query tiles of the block(s)
 constexpr uint32_t KV_MISC = KV_UNITS + 2 * kMaxUnits * 4;
 // TMEM columns 0-255 hold S^T [keys][queries] and dP^T (fp32) for the 128 queries of a tile,
 // taken as two passes of 64 queries.  d = 128: S^T in columns 0-127 and dP^T in 128-255, both
@@ -430,21 +432,24 @@ template <int D> struct KvTmem {
   static constexpr uint32_t kDp = kTwoBuf ? 64 : 128;             // dP^T columns after S^T
   __host__ __device__ static constexpr uint32_t st(int pass) { return (kTwoBuf ? 128u : 64u) * pass; }
 };
-constexpr int kKvThreads = 320;
+constexpr int kKvThreads = 352;          // TMA producer, MMA, 8 softmax warps, scalar transposer
 
 struct KvMisc {
   uint64_t kv_full, qd_full[kStages], qd_empty[kStages], s_full[2], p_half[2], done;
   uint64_t kv_read, st1_read, acck_full, accv_full;   // K / V and stage 1 free; low-rank rows landed
+  uint64_t sc_ready[kStages];                          // the stage's scalars transposed
   uint32_t tmem_base;
   int abort_flag;
 };
 
 // One thread's 32 queries (columns q0 .. q0 + 31 of the unit) for its key row: S^T and dP^T
 // (fp32, TMEM) -> (P^T cs) and dS^T as bf16 pairs in the first 8 of each 16 columns read.
-// MASK: queries outside [lo, hi) (relative to q0) get P = 0.
+// nx, cs, nd: -log2 d_s, cs and -Delta of those queries; pairs of columns go through packed
+// fp32 lanes.  MASK: queries outside [lo, hi) (relative to q0) get P = 0.
 template <bool MASK>
-__device__ __forceinline__ void dkdv_softmax_cols(uint32_t tmem, uint32_t st_col, uint32_t dp_col, const float4* sc,
-                                                  float sl2, int lo, int hi) {
+__device__ __forceinline__ void dkdv_softmax_cols(uint32_t tmem, uint32_t st_col, uint32_t dp_col, const float* nx,
+                                                  const float* cs, const float* nd, float sl2, int lo, int hi) {
+  const uint64_t sl2x2 = tc::f2_pack(sl2, sl2);
 #pragma unroll
   for (int c0 = 0; c0 < 32; c0 += 16) {
     float sv[16], dp[16];
@@ -454,17 +459,23 @@ __device__ __forceinline__ void dkdv_softmax_cols(uint32_t tmem, uint32_t st_col
     uint32_t wp[8], wd[8];
 #pragma unroll
     for (int c = 0; c < 16; c += 2) {
-      float pv[2], dv[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float4 q = sc[c0 + c + e];          // (log2 d_s, cs, Delta)
-        float p = ex2_approx(fmaf(sv[c + e], sl2, -q.x));
-        if (MASK && (c0 + c + e < lo || c0 + c + e >= hi)) p = 0.f;
-        pv[e] = p * q.y;
-        dv[e] = p * fmaf(q.y, dp[c + e], -q.z);
+      const int q = c0 + c;
+      const uint64_t x2 = *reinterpret_cast<const uint64_t*>(nx + q);
+      const uint64_t y2 = *reinterpret_cast<const uint64_t*>(cs + q);
+      const uint64_t z2 = *reinterpret_cast<const uint64_t*>(nd + q);
+      float e0, e1;
+      tc::f2_unpack(tc::f2_fma(tc::f2_pack(sv[c], sv[c + 1]), sl2x2, x2), e0, e1);
+      float p0 = ex2_approx(e0), p1 = ex2_approx(e1);
+      if (MASK) {
+        if (q < lo || q >= hi) p0 = 0.f;
+        if (q + 1 < lo || q + 1 >= hi) p1 = 0.f;
       }
-      wp[c >> 1] = pack_bf16(pv[0], pv[1]);
-      wd[c >> 1] = pack_bf16(dv[0], dv[1]);
+      const uint64_t p2 = tc::f2_pack(p0, p1);
+      float a0, a1, b0, b1;
+      tc::f2_unpack(tc::f2_mul(p2, y2), a0, a1);
+      tc::f2_unpack(tc::f2_mul(p2, tc::f2_fma(y2, tc::f2_pack(dp[c], dp[c + 1]), z2)), b0, b1);
+      wp[c >> 1] = pack_bf16(a0, a1);
+      wd[c >> 1] = pack_bf16(b0, b1);
     }
     tc::tmem_st8(tmem + st_col + c0, wp);
     tc::tmem_st8(tmem + dp_col + c0, wd);
@@ -522,6 +533,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     tc::mbar_init(&ms->st1_read, 1);
     tc::mbar_init(&ms->acck_full, 1);
     tc::mbar_init(&ms->accv_full, 1);
+    for (int st = 0; st < kStages; ++st) tc::mbar_init(&ms->sc_ready[st], 1);
     tc::mbar_init(&ms->p_half[0], kSoftmaxThreads);
     tc::mbar_init(&ms->p_half[1], kSoftmaxThreads);
     tc::mbar_init(&ms->done, 1);
@@ -732,6 +744,25 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       tc::mma_commit(&ms->done);
       tc::mbar_wait(&ms->done, 0);
     }
+  } else if (warp == 10) {
+    // ---------------- scalar transposer: each stage's per-query (log2 d_s, cs, Delta) as three
+    // arrays (-log2 d_s, cs, -Delta) once the stage has landed.  The stage's previous tile is
+    // done with them: its copy waited for that tile's products, which waited for its softmax.
+    for (int u = 0; u < n_u; ++u) {
+      const int s = u % kStages;
+      if (!__all_sync(0xffffffffu, wait_or_abort(&ms->qd_full[s], (u / kStages) & 1, ms, err, 2048u))) break;
+      const float4* src = reinterpret_cast<const float4*>(smem + KV_SC + s * 128 * 16);
+      float* dst = reinterpret_cast<float*>(smem + KV_SOA + s * 3 * 128 * 4);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 v = src[lane + 32 * k];
+        dst[lane + 32 * k] = -v.x;
+        dst[128 + lane + 32 * k] = v.y;
+        dst[256 + lane + 32 * k] = -v.z;
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&ms->sc_ready[s]);
+    }
   } else {
     // ---------------- softmax: one key row; two passes of 32 queries per thread ----------------
     const int q4 = warp & 3;
@@ -752,6 +783,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const int s = u % kStages;
       // one buffer: both passes' scores arrive together; two: each pass's on its own
       alive = __all_sync(0xffffffffu, wait_or_abort(&ms->s_full[0], u & 1, ms, err, 32u));
+      if (alive) alive = __all_sync(0xffffffffu, wait_or_abort(&ms->sc_ready[s], (u / kStages) & 1, ms, err, 4096u));
       if (!alive) break;
       tc::tc_fence_after();
 #pragma unroll 1
@@ -773,13 +805,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         const bool masked = dead || !key_ok || qvalid < 32 || (diag && kpos > qp0);
         const int lo = diag ? kpos - qp0 : 0;
         const int hi = dead ? 0 : key_ok ? qvalid : 0;
-        const float4* sc = reinterpret_cast<const float4*>(smem + KV_SC + s * 128 * 16) + q0;
+        const float* nx = reinterpret_cast<const float*>(smem + KV_SOA + s * 3 * 128 * 4) + q0;
         const uint32_t st_col = lane_base + KvTmem<D>::st(pass) + 32 * grp;
         // masking only on the causal diagonal, at the end of the sequence and for padding keys
         if (__any_sync(0xffffffffu, masked))
-          dkdv_softmax_cols<true>(tmem, st_col, st_col + KvTmem<D>::kDp, sc, sl2, lo, hi);
+          dkdv_softmax_cols<true>(tmem, st_col, st_col + KvTmem<D>::kDp, nx, nx + 128, nx + 256, sl2, lo, hi);
         else
-          dkdv_softmax_cols<false>(tmem, st_col, st_col + KvTmem<D>::kDp, sc, sl2, lo, hi);
+          dkdv_softmax_cols<false>(tmem, st_col, st_col + KvTmem<D>::kDp, nx, nx + 128, nx + 256, sl2, lo, hi);
         tc::tmem_wait_st();
         tc::tc_fence_before();
         tc::mbar_arrive(&ms->p_half[pass]);
