@@ -87,6 +87,16 @@ __global__ void __launch_bounds__(kThreads, NW == 32 ? 4 : 1)
     ms->limit_ns = g.wait_ns;
     ms->abort_flag = 0;
     tc::fence_barrier_init();
+    // the chunk's tiles do not depend on anything the set-up computes: their copies start first
+    {
+      constexpr uint32_t kWD = (uint32_t)NW * D * 2;
+      tc::mbar_arrive_expect_tx(&ms->in_full, 128u * D * 2 + 2 * kWD);
+      for (int s = 0; s < D / 64; ++s) {
+        tc::tma_load_3d(smem + F_X + s * kSlab, side ? &tmK : &tmQ, &ms->in_full, 64 * s, c * kC, bh);
+        tc::tma_load_3d(smem + FL::kWH + s * FL::kWSlab, &tmW, &ms->in_full, 64 * s, 0, 0);
+        tc::tma_load_3d(smem + FL::kWL + s * FL::kWSlab, &tmW, &ms->in_full, 64 * s, 0, 1);
+      }
+    }
   }
   if (warp == 1) {
     tc::tmem_alloc(&ms->tmem_base, NW < 32 ? 32 : NW);
@@ -99,13 +109,6 @@ __global__ void __launch_bounds__(kThreads, NW == 32 ? 4 : 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      constexpr uint32_t kWD = (uint32_t)NW * D * 2;
-      tc::mbar_arrive_expect_tx(&ms->in_full, 128u * D * 2 + 2 * kWD);
-      for (int s = 0; s < D / 64; ++s) {
-        tc::tma_load_3d(smem + F_X + s * kSlab, side ? &tmK : &tmQ, &ms->in_full, 64 * s, c * kC, bh);
-        tc::tma_load_3d(smem + FL::kWH + s * FL::kWSlab, &tmW, &ms->in_full, 64 * s, 0, 0);
-        tc::tma_load_3d(smem + FL::kWL + s * FL::kWSlab, &tmW, &ms->in_full, 64 * s, 0, 1);
-      }
       tc::mbar_wait(&ms->in_full, 0);                 // no copy in flight when the CTA exits
     }
   } else if (warp == 1) {

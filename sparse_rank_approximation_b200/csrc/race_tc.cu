@@ -37,7 +37,6 @@ namespace elsaa {
 namespace {
 
 constexpr int kC = 128;
-constexpr int kD = 128;                          // widest head dimension: operand slots are sized for it
 constexpr int kR = 128;
 constexpr int kNH = 32;                          // projection columns 4 L
 constexpr uint32_t kSlab = 128 * 128;            // [128 rows][64 bf16], 128-byte swizzle
@@ -194,8 +193,8 @@ __device__ __forceinline__ void issue_du(uint32_t tmem, uint32_t d_col, const SD
 }
 
 // fp32 gradient rows leave through shared memory: each thread writes its row there (pitch
-// kD + 4 floats, so the 16-byte stores of 8 consecutive rows hit 8 different bank groups),
-// then all compute threads copy the [128][kD] tile out with coalesced 16-byte stores.  The
+// D + 4 floats, so the 16-byte stores of 8 consecutive rows hit 8 different bank groups),
+// then all compute threads copy the [128][D] tile out with coalesced 16-byte stores.  The
 // staging area reuses operand tiles that no product reads any more.
 template <int D> constexpr int stage_pitch() { return D + 4; }
 template <int D> constexpr uint32_t stage_bytes() { return (uint32_t)kC * stage_pitch<D>() * 4; }
@@ -315,18 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&ms->x_full, 1);
     ms->abort_flag = 0;
     tc::fence_barrier_init();
-  }
-  if (warp == 1) {
-    tc::tmem_alloc(&ms->tmem_base, 512);
-    tc::tmem_relinquish();
-  }
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
-  const uint32_t tmem = ms->tmem_base;
-
-  if (warp == 0) {
-    if (lane == 0) {
+    // the chunk's tiles do not depend on anything the set-up computes: their copies start first
+    {
       // Phi tiles are [128][128]; V, dO, the statistics and W are D columns wide
       constexpr uint32_t kTD = 128u * D * 2, kWD = (uint32_t)kNH * D * 2;
       tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 2 : 1) * kTile + (causal ? 2 : 1) * kTD + 2 * kTD + 2 * kWD);
@@ -343,6 +332,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_load_3d(smem + K_WH + s * kWSlab, &tmW, &ms->in_main, 64 * s, kNH * grp, 0);
         tc::tma_load_3d(smem + K_WL + s * kWSlab, &tmW, &ms->in_main, 64 * s, kNH * grp, 1);
       }
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&ms->tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      constexpr uint32_t kTD = 128u * D * 2;
       tc::mbar_wait(&ms->in_main, 0);
       // the K rows for dx, once every product but du has read the chunk tiles; waited for
       // here too, so no copy is in flight when the CTA exits
@@ -541,18 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&ms->x_full, 1);
     ms->abort_flag = 0;
     tc::fence_barrier_init();
-  }
-  if (warp == 1) {
-    tc::tmem_alloc(&ms->tmem_base, 512);
-    tc::tmem_relinquish();
-  }
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
-  const uint32_t tmem = ms->tmem_base;
-
-  if (warp == 0) {
-    if (lane == 0) {
+    // the chunk's tiles do not depend on anything the set-up computes: their copies start first
+    {
       // Phi(K) is [128][128]; dO, V, the statistics and W are D columns wide
       constexpr uint32_t kTD = 128u * D * 2, kWD = (uint32_t)kNH * D * 2;
       tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? kTile + 2 * kTD : kTD) + 2 * kTD + 2 * kWD);
@@ -567,6 +560,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_load_3d(smem + Q_WH + s * kWSlab, &tmW, &ms->in_main, 64 * s, kNH * grp, 0);
         tc::tma_load_3d(smem + Q_WL + s * kWSlab, &tmW, &ms->in_main, 64 * s, kNH * grp, 1);
       }
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&ms->tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      constexpr uint32_t kTD = 128u * D * 2;
       tc::mbar_wait(&ms->in_main, 0);
       // the Q rows for dx, once every product but du has read the chunk tiles; waited for
       // here too, so no copy is in flight when the CTA exits
@@ -718,18 +725,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&ms->acc_full, 1);
     ms->abort_flag = 0;
     tc::fence_barrier_init();
-  }
-  if (warp == 1) {
-    tc::tmem_alloc(&ms->tmem_base, 256);
-    tc::tmem_relinquish();
-  }
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
-  const uint32_t tmem = ms->tmem_base;
-
-  if (warp == 0) {
-    if (lane == 0) {
+    // the chunk's tiles do not depend on anything the set-up computes: their copies start first
+    {
       // Phi tiles are [128][128]; V and the statistics are D columns wide
       constexpr uint32_t kTD = 128u * D * 2;
       tc::mbar_arrive_expect_tx(&ms->in_main, (causal ? 2 * kTile + kTD : kTile) + 2 * kTD);
@@ -743,6 +740,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_load_3d(smem + R_PH + s * kSlab, &tmP, &ms->in_main, 64 * s, 0, z);
         tc::tma_load_3d(smem + R_PL + s * kSlab, &tmP, &ms->in_main, 64 * s, 0, z + 1);
       }
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&ms->tmem_base, 256);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
       tc::mbar_wait(&ms->in_main, 0);
     }
   } else if (warp == 1) {
