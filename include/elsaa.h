@@ -116,7 +116,8 @@ typedef struct {
 /* Bytes of the caller-owned `saved` buffer the forward fills and the backward
  * reads (selection, per-row denominators, the fusion weight, O_sparse, RACE
  * features and prefix summaries; with SORTLSH also the sorted orders, one pair per
- * recursion level when causal).  O_sparse is kept in float32 for every dtype: the
+ * recursion level when causal, and then also every level's gathered query, key and
+ * value rows, 3 * levels * B * H * N * d * 2 bytes, which the backward reuses).  O_sparse is kept in float32 for every dtype: the
  * backward forms the softmax delta <dO_s, O_s> from it, and a bf16 copy would put
  * the rounding of O_s into every dS of a row whose mass sits on a few keys.
  * Returns 0 when params are invalid. */

@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     tc::fence_proxy_async_smem();
     softmax_bar();
-    if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag && !a.q_rows) {
+    if (threadIdx.x == 64 && !*(volatile int*)&ms->abort_flag && !a.q_rows && a.O) {
       for (int sl = 0; sl < D / 64; ++sl) tma_store_3d(&tmO, smem + L::v(0) + sl * kSlab, 64 * sl, row0, bh);
       asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
       asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
@@ -519,7 +519,7 @@ static cudaError_t fwd_t(const FwdArgs& a, const Geom& g, uint32_t* err, cudaStr
   CUtensorMap mq, mk, mv, mlr, mo;
   if (!make_map(&mq, a.Q, D, g.N, g.BH, kT) || !make_map(&mk, a.K, D, g.N, g.BH, TB) ||
       !make_map(&mv, a.V, D, g.N, g.BH, TB) || !make_map(&mlr, a.Olr, D, g.N, g.BH, kT) ||
-      !make_map(&mo, a.O, D, g.N, g.BH, kT))
+      !make_map(&mo, a.O ? a.O : a.Q, D, g.N, g.BH, kT))    // without O the map is not used
     return cudaErrorInvalidValue;
   auto kern = attn_fwd_tc_kernel<D, PAIR>;
   constexpr size_t smem = smem_bytes<D>();

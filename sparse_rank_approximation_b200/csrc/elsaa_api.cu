@@ -185,6 +185,9 @@ struct Saved {
   void* Psplit;
   float* Pmass;
   int* lsh_order;          // sortLSH: sorted query and key orders [BH][2][N] (causal: one per level)
+  // causal sortLSH: every level's gathered future-half queries and past-half keys and values
+  // ([levels][BH][N][d]); the forward gathers them once and the backward reads them again
+  void *lvQ, *lvK, *lvV;
 };
 
 Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
@@ -214,6 +217,11 @@ Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
   s.Pmass = split ? c.take<float>((size_t)g.BH * g.n_c * g.rp) : nullptr;
   const size_t orders = g.selector != ELSAA_SEL_SORTLSH ? 0 : g.causal ? (size_t)g.lsh_levels : 1;
   s.lsh_order = orders ? c.take<int>(orders * g.BH * 2 * g.N) : nullptr;
+  const bool lv_rows = g.selector == ELSAA_SEL_SORTLSH && g.causal && g.lsh_levels > 0;
+  const size_t lv_mat = lv_rows ? (size_t)g.lsh_levels * rows * g.d * esz : 0;
+  s.lvQ = lv_rows ? c.take<char>(lv_mat) : nullptr;
+  s.lvK = lv_rows ? c.take<char>(lv_mat) : nullptr;
+  s.lvV = lv_rows ? c.take<char>(lv_mat) : nullptr;
   *bytes = align_up(c.off);
   return s;
 }
@@ -258,10 +266,8 @@ PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
     b.glr = c.take<float>(rows);
     return b;
   }
+  // (the levels' gathered Q, K and V are kept in the saved buffer)
   const size_t lv = (size_t)g.lsh_levels, vheads = lv * g.BH;
-  b.Q = c.take<char>(lv * mat);
-  b.K = c.take<char>(lv * mat);
-  b.V = c.take<char>(lv * mat);
   b.idx = c.take<int>(vheads * g.n_t);
   b.tile_list = c.take<int>(vheads * (g.n_t / 2));
   if (backward) {
@@ -584,20 +590,20 @@ elsaa_status causal_lsh_forward(const elsaa_params* p, const Geom& g, const void
                             "sortLSH level sort"));
     // only the future halves' queries and the past halves' keys and values are read
     const void* qs[1] = {Q};
-    void* qd[1] = {b.Q};
+    void* qd[1] = {s.lvQ};
     const void* kvs[2] = {K, V};
-    void* kvd[2] = {b.K, b.V};
+    void* kvd[2] = {s.lvK, s.lvV};
     ELSAA_TRY(cuda_status(launch_gather_rows(qs, qd, 1, s.lsh_order, rb, lv, 1, g, st), "sortLSH gather Q"));
     ELSAA_TRY(cuda_status(launch_gather_rows(kvs, kvd, 2, s.lsh_order + g.N, rb, lv, 0, g, st),
                           "sortLSH gather K, V"));
     ELSAA_TRY(cuda_status(launch_causal_lsh_select_levels(b.idx, b.tile_list, lv, g, st), "sortLSH level selection"));
     // all levels in one launch, as lv * BH heads (the tcgen05 kernel over their future
-    // tiles only).  The fused output, not used, goes over each tile's own gathered queries,
-    // which only that tile reads and reads before it is written
+    // tiles only); the fused output is not used and not written, so the gathered rows stay
+    // intact for the backward
     Geom gv = sparse_only(g, false, 1);
     gv.BH = lv * g.BH;
-    sa.Q = b.Q; sa.K = b.K; sa.V = b.V; sa.idx = b.idx;
-    sa.O = b.Q;
+    sa.Q = s.lvQ; sa.K = s.lvK; sa.V = s.lvV; sa.idx = b.idx;
+    sa.O = nullptr;
     sa.Os = b.Os_lv;
     sa.logd = b.logd_lv;
     sa.tile_list = b.tile_list;
@@ -628,15 +634,13 @@ elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const
   }
   if (g.lsh_levels > 0) {
     const int lv = g.lsh_levels;
-    const void* qs[2] = {a.Q, a.dO};
-    void* qd[2] = {b.Q, b.X};
-    const void* kvs[2] = {a.K, a.V};
-    void* kvd[2] = {b.K, b.V};
+    // Q, K and V of the levels are the forward's gathered rows (saved); dO and the row scalars
+    // are gathered here
+    const void* qs[1] = {a.dO};
+    void* qd[1] = {b.X};
     const void* ps[1] = {w.rs.packed};
     void* pd[1] = {b.packed};
-    ELSAA_TRY(cuda_status(launch_gather_rows(qs, qd, 2, s.lsh_order, rb, lv, 1, g, st), "sortLSH gather Q, dO"));
-    ELSAA_TRY(cuda_status(launch_gather_rows(kvs, kvd, 2, s.lsh_order + g.N, rb, lv, 0, g, st),
-                          "sortLSH gather K, V"));
+    ELSAA_TRY(cuda_status(launch_gather_rows(qs, qd, 1, s.lsh_order, rb, lv, 1, g, st), "sortLSH gather dO"));
     ELSAA_TRY(cuda_status(launch_gather_rows(ps, pd, 1, s.lsh_order, 16, lv, 1, g, st), "sortLSH gather row scalars"));
     ELSAA_TRY(cuda_status(launch_causal_lsh_select_levels(b.idx, b.tile_list, lv, g, st), "sortLSH level selection"));
     Geom gv = sparse_only(g, false, 1);
@@ -645,7 +649,7 @@ elsaa_status causal_lsh_backward(const Geom& g, BwdArgs a, const Saved& s, const
     // all levels in one launch each: dQ over the future tiles, dK/dV over the key blocks
     // that have a tile (the past halves, first in the longest-first order)
     BwdArgs la{};
-    la.Q = b.Q; la.K = b.K; la.V = b.V; la.dO = b.X;
+    la.Q = s.lvQ; la.K = s.lvK; la.V = s.lvV; la.dO = b.X;
     la.idx = b.idx; la.offs = b.offs; la.tiles = b.tiles; la.kv_order = b.order;
     la.rs.packed = b.packed;
     la.dQ = b.dQ; la.dK = b.dK; la.dV = b.dV;
