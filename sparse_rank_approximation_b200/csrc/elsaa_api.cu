@@ -185,8 +185,9 @@ struct Saved {
   void* Psplit;
   float* Pmass;
   int* lsh_order;          // sortLSH: sorted query and key orders [BH][2][N] (causal: one per level)
-  // causal sortLSH: every level's gathered future-half queries and past-half keys and values
-  // ([levels][BH][N][d]); the forward gathers them once and the backward reads them again
+  // sortLSH: the rows the operator runs on, gathered by the forward and read again by the
+  // backward.  Non-causal: Q by the query order, K and V by the key order ([BH][N][d]).
+  // Causal: every level's future-half queries and past-half keys and values ([levels][BH][N][d]).
   void *lvQ, *lvK, *lvV;
 };
 
@@ -217,8 +218,9 @@ Saved carve_saved(void* base, const Geom& g, size_t esz, size_t* bytes) {
   s.Pmass = split ? c.take<float>((size_t)g.BH * g.n_c * g.rp) : nullptr;
   const size_t orders = g.selector != ELSAA_SEL_SORTLSH ? 0 : g.causal ? (size_t)g.lsh_levels : 1;
   s.lsh_order = orders ? c.take<int>(orders * g.BH * 2 * g.N) : nullptr;
-  const bool lv_rows = g.selector == ELSAA_SEL_SORTLSH && g.causal && g.lsh_levels > 0;
-  const size_t lv_mat = lv_rows ? (size_t)g.lsh_levels * rows * g.d * esz : 0;
+  const size_t lv_count = g.selector != ELSAA_SEL_SORTLSH ? 0 : g.causal ? (size_t)g.lsh_levels : 1;
+  const bool lv_rows = lv_count > 0;
+  const size_t lv_mat = lv_count * rows * g.d * esz;
   s.lvQ = lv_rows ? c.take<char>(lv_mat) : nullptr;
   s.lvK = lv_rows ? c.take<char>(lv_mat) : nullptr;
   s.lvV = lv_rows ? c.take<char>(lv_mat) : nullptr;
@@ -252,9 +254,7 @@ PermBufs carve_perm(Carver& c, const Geom& g, size_t esz, bool backward) {
   if (g.selector != ELSAA_SEL_SORTLSH) return b;
   const size_t rows = (size_t)g.BH * g.N, mat = rows * g.d * esz;
   if (!g.causal) {
-    b.Q = c.take<char>(mat);
-    b.K = c.take<char>(mat);
-    b.V = c.take<char>(mat);
+    // (the sorted Q, K and V are kept in the saved buffer)
     b.X = c.take<char>(mat);
     if (backward) {
       b.dQ = c.take<char>(mat);
@@ -495,20 +495,24 @@ ProfScope::~ProfScope() {
 }
 }  // namespace elsaa
 
-// sortLSH: sort the rows, then gather the inputs into the sorted orders (queries by the
-// query order, keys and values by the key order, per-row vectors by the query order).
-elsaa_status lsh_gather(const elsaa_params* p, const Geom& g, bool bf16, const int* order, bool sort_first, int* scratch,
+// sortLSH: gather the inputs into the sorted orders (queries by the query order, keys and values
+// by the key order, per-row vectors by the query order).  The forward sorts first and gathers Q,
+// K and V into the saved buffer (qkv); the backward reuses those and gathers only dO and the
+// per-row vectors.
+elsaa_status lsh_gather(const elsaa_params* p, const Geom& g, bool bf16, const int* order, bool forward, int* scratch,
                         const void* Q, const void* K, const void* V, const void* X, const float* lam,
-                        const float* gs, const float* glr, const PermBufs& b, cudaStream_t st) {
+                        const float* gs, const float* glr, void* const (&qkv)[3], const PermBufs& b,
+                        cudaStream_t st) {
   const int row_bytes = g.d * (bf16 ? 2 : 4), stride = 2 * g.N;
   const int* oq = order;
   const int* ok = order + g.N;
-  if (sort_first)
+  if (forward) {
     ELSAA_TRY(cuda_status(launch_sortlsh_order(Q, K, bf16, p->lsh_planes, p->lsh_bits, const_cast<int*>(order),
                                                nullptr, scratch, g, st), "sortLSH order"));
-  ELSAA_TRY(cuda_status(launch_permute_rows(Q, b.Q, oq, row_bytes, g, stride, false, st), "sortLSH gather Q"));
-  ELSAA_TRY(cuda_status(launch_permute_rows(K, b.K, ok, row_bytes, g, stride, false, st), "sortLSH gather K"));
-  ELSAA_TRY(cuda_status(launch_permute_rows(V, b.V, ok, row_bytes, g, stride, false, st), "sortLSH gather V"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(Q, qkv[0], oq, row_bytes, g, stride, false, st), "sortLSH gather Q"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(K, qkv[1], ok, row_bytes, g, stride, false, st), "sortLSH gather K"));
+    ELSAA_TRY(cuda_status(launch_permute_rows(V, qkv[2], ok, row_bytes, g, stride, false, st), "sortLSH gather V"));
+  }
   if (X) ELSAA_TRY(cuda_status(launch_permute_rows(X, b.X, oq, row_bytes, g, stride, false, st), "sortLSH gather dO"));
   if (lam) ELSAA_TRY(cuda_status(launch_gather_vec(lam, b.lam, oq, g, stride, st), "sortLSH gather lambda"));
   if (gs) ELSAA_TRY(cuda_status(launch_gather_vec(gs, b.gs, oq, g, stride, st), "sortLSH gather g_sparse"));
@@ -771,8 +775,10 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* Q, const void* K, 
     // the operator runs on the sorted rows (non-causal RACE, the fusion and diagonal-block
     // attention commute with row permutations); O is scattered back at the end
     ELSAA_TRY(check_ptr(p->lsh_planes, "lsh_planes"));
-    ELSAA_TRY(lsh_gather(p, g, bf16, s.lsh_order, true, w.lsh_scratch, Q, K, V, nullptr, lam, gs, glr, w.pm, st_));
-    Q = w.pm.Q; K = w.pm.K; V = w.pm.V; O = w.pm.X;
+    void* const qkv[3] = {s.lvQ, s.lvK, s.lvV};
+    ELSAA_TRY(lsh_gather(p, g, bf16, s.lsh_order, true, w.lsh_scratch, Q, K, V, nullptr, lam, gs, glr, qkv, w.pm,
+                         st_));
+    Q = s.lvQ; K = s.lvK; V = s.lvV; O = w.pm.X;
     if (lam) lam = w.pm.lam;
     if (gs) gs = w.pm.gs;
     if (glr) glr = w.pm.glr;
@@ -890,8 +896,9 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   if (lsh) {
     // the forward ran on the sorted rows and saved its state in that order; so does this,
     // and the gradients are scattered back at the end
-    ELSAA_TRY(lsh_gather(p, g, bf16, s.lsh_order, false, nullptr, Q, K, V, dO, lam, gs, glr, w.pm, st_));
-    Q = w.pm.Q; K = w.pm.K; V = w.pm.V; dO = w.pm.X;
+    void* const qkv[3] = {s.lvQ, s.lvK, s.lvV};
+    ELSAA_TRY(lsh_gather(p, g, bf16, s.lsh_order, false, nullptr, Q, K, V, dO, lam, gs, glr, qkv, w.pm, st_));
+    Q = s.lvQ; K = s.lvK; V = s.lvV; dO = w.pm.X;
     dQ = w.pm.dQ; dK = w.pm.dK; dV = w.pm.dV;
     if (lam) lam = w.pm.lam;
     if (gs) gs = w.pm.gs;
