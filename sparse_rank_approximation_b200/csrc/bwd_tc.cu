@@ -154,8 +154,19 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       tc::tma_load_3d(smem + DQ_Q + sl * kSlab, &tmQ, &ms->qd_full, 64 * sl, row0, bh);
       tc::tma_load_3d(smem + DQ_DO + sl * kSlab, &tmdO, &ms->qd_full, 64 * sl, row0, bh);
     }
-    tc::prefetch_tensormap(&tmK);
-    tc::prefetch_tensormap(&tmV);
+    // so do the first selected block's K and V (its index is the first of the tile's list):
+    // the producers start at the second block
+    const int b0[2] = {g.k > 0 ? idx_a[0] : -1, PAIR && tb < g.n_t && g.k > 0 ? idx_b[0] : -1};
+    if (b0[0] >= 0 || b0[1] >= 0) {
+      for (int kv = 0; kv < 2; ++kv) {
+        uint64_t* full = kv ? &ms->v_full[0] : &ms->k_full[0];
+        tc::mbar_arrive_expect_tx(full, 128u * D * 2);
+        for (int h = 0; h < (PAIR ? 2 : 1); ++h)
+          for (int sl = 0; sl < D / 64; ++sl)
+            tc::tma_load_3d(smem + (kv ? dq_v(0) : dq_k(0)) + sl * kSlab + h * 64 * 128, kv ? &tmV : &tmK, full,
+                            64 * sl, (b0[h] >= 0 ? b0[h] : 0) * TB, bh);
+      }
+    }
   }
   if (threadIdx.x < 32) {
     ms->idx[0][threadIdx.x] = threadIdx.x < g.k ? idx_a[threadIdx.x] : -1;
@@ -184,8 +195,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       uint64_t* full = kside ? ms->k_full : ms->v_full;
       uint64_t* empty = kside ? ms->k_empty : ms->v_empty;
       constexpr uint32_t kTD = 128u * D * 2;      // bytes of a [128][D] tile
-      int issued = 0;
-      for (int j = 0; j < n_sel; ++j) {
+      int issued = n_sel > 0 ? 1 : 0;             // block 0 was issued with the barriers
+      for (int j = issued; j < n_sel; ++j) {
         const int s = j % NS;
         if (j >= NS && !wait_or_abort(&empty[s], ((j / NS) - 1) & 1, ms, err, kside ? 1u : 2u)) break;
         unsigned char* dst = smem + (kside ? dq_k(s) : dq_v(s));
@@ -550,9 +561,29 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         tc::tma_load_3d(smem + KV_V + sl * kSlab + h * 64 * 128, &tmV, &ms->kv_full, 64 * sl, kr, bh);
       }
     }
-    tc::prefetch_tensormap(&tmQ);
-    tc::prefetch_tensormap(&tmdO);
-    tc::prefetch_tensormap(&tmSc);
+    // so do the first query tile's Q, dO and scalars (the first entries of the block(s)' tile
+    // lists): the producer starts at the second tile
+    if (g.k > 0) {
+      const int* of = a.offs + (size_t)bh * (g.n_t + 1);
+      const int* list = a.tiles + (size_t)bh * g.n_t * g.k;
+      int t0[2] = {-1, -1};
+      for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
+        if (pb[h] < 0) break;
+        const int e0 = of[pb[h]];
+        if (of[pb[h] + 1] > e0) t0[h] = list[e0];
+      }
+      if (t0[0] >= 0 || t0[1] >= 0) {
+        tc::mbar_arrive_expect_tx(&ms->qd_full[0], 2 * kTD + 128 * 16);
+        for (int h = 0; h < (PAIR ? 2 : 1); ++h) {
+          const int qr = (t0[h] >= 0 ? t0[h] : 0) * TB;
+          for (int sl = 0; sl < D / 64; ++sl) {
+            tc::tma_load_3d(smem + kv_q(0) + sl * kSlab + h * 64 * 128, &tmQ, &ms->qd_full[0], 64 * sl, qr, bh);
+            tc::tma_load_3d(smem + kv_do(0) + sl * kSlab + h * 64 * 128, &tmdO, &ms->qd_full[0], 64 * sl, qr, bh);
+          }
+          tc::tma_load_3d(smem + KV_SC + h * 64 * 16, &tmSc, &ms->qd_full[0], 0, qr, bh);
+        }
+      }
+    }
   }
   int n_ut[2] = {0, 0};
   if (g.k > 0) {
@@ -583,8 +614,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       constexpr uint32_t kTD = 128u * D * 2;      // bytes of a [128][D] tile
-      int issued = 0;
-      for (int u = 0; u < n_u; ++u) {
+      int issued = n_u > 0 ? 1 : 0;               // tile 0 was issued with the barriers
+      for (int u = issued; u < n_u; ++u) {
         const int s = u % kStages;
         if (u >= kStages && !wait_or_abort(&ms->qd_empty[s], ((u / kStages) - 1) & 1, ms, err, 1u)) break;
         tc::mbar_arrive_expect_tx(&ms->qd_full[s], 2 * kTD + 128 * 16);
