@@ -111,3 +111,22 @@ def test_sortlsh_shape_limits():
     p = bd.make_params(1, 1, 1024, 128, block_size=128, rank_r=128, causal=True, selector=bd.ELSAA_SEL_SORTLSH,
                        lsh_bits=17, topk=1)
     assert L.elsaa_saved_bytes(ctypes.byref(p)) == 0
+
+
+def test_sortlsh_saved_buffer_holds_the_gathered_rows():
+    """With sortLSH the forward keeps the rows it gathered (the sorted Q, K, V; with the causal
+    recursion every level's future-half queries and past-half keys and values) in the saved
+    buffer for the backward, so saved grows by 3 x levels x B H N d x element bytes."""
+    L = bd.lib()
+    B, H, N, d = 1, 2, 4096, 128
+    base = dict(block_size=128, rank_r=128, topk=1)
+    n_t = N // 128                             # 32 tiles: the sorted levels are 1 .. log2(32) - 1
+    lv = n_t.bit_length() - 2
+    for causal, n_levels in ((False, 1), (True, lv)):
+        p = bd.make_params(B, H, N, d, causal=causal, selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=5, **base)
+        q = bd.make_params(B, H, N, d, causal=causal, **base)
+        rows = 3 * n_levels * B * H * N * d * 2
+        orders = (n_levels if causal else 1) * B * H * 2 * N * 4
+        grown = L.elsaa_saved_bytes(ctypes.byref(p)) - L.elsaa_saved_bytes(ctypes.byref(q))
+        assert grown >= rows + orders, (causal, grown, rows, orders)
+        assert grown <= rows + orders + 4096, (causal, grown, rows, orders)
