@@ -1,6 +1,6 @@
 // Sparse-branch backward on the 5th-generation tensor cores (tcgen05 + TMEM),
-// 128-query tiles, 128-key blocks, head dimension 128 (ELSAA paper §3.2 with the
-// Eq. 5 adjoint folded into the softmax delta):
+// 128-query tiles (or pairs of 64-query tiles), head dimension 64 or 128 (ELSAA paper
+// §3.2 with the Eq. 5 adjoint folded into the softmax delta):
 //   P_ij  = exp(z_ij - log d_s,i)            (z = scale q.k, j in the selected blocks)
 //   dz_ij = P_ij (cs_i <dO_i, v_j> - Delta_i)
 //   dq_i  = scale sum_j dz_ij k_j,  dk_j = scale sum_i dz_ij q_i,  dv_j = sum_i P_ij cs_i dO_i
@@ -12,11 +12,15 @@
 // TMEM buffers, and dQ += dS K (dS as the tensor-memory operand) accumulates in TMEM.
 // dkdv kernel: one CTA per (head, key block); K and V stay in shared memory, the
 // query tiles that selected the block (from the selection inverse) stream through a
-// 2-stage ring together with their per-row scalars; S^T = K Q^T and dP^T = V dO^T
-// land in TMEM, the softmax warps write (P^T cs) and dS^T back over them as bf16 in two
-// passes of 64 queries, and dV += (P^T cs) dO, dK += dS^T Q accumulate in TMEM (with
-// d = 64, in two buffers, the next pass's scores computed while the softmax works).  The low-rank parts are brought into L2 once every load is issued
-// and read while the last products run.  No atomics: the results are deterministic.
+// 2-stage ring together with their per-row scalars (a warp rewrites those as three
+// arrays); S^T = K Q^T and dP^T = V dO^T land in TMEM, the softmax warps write
+// (P^T cs) and dS^T back over them as bf16 in two passes of 64 queries, and
+// dV += (P^T cs) dO, dK += dS^T Q accumulate in TMEM (with d = 64 in two buffers, the
+// next pass's scores computed while the softmax works).
+// Both: the tile loads that need no selection data start with the barrier set-up; the
+// softmax arithmetic runs in packed fp32 pairs; the fp32 low-rank rows are TMA-loaded
+// into buffers the products are done with, for the epilogue.  No atomics: the results
+// are deterministic.
 // Every mbarrier wait is bounded; a timeout sets a bit in the caller's error word,
 // the CTA drains its copies and MMAs, frees TMEM and exits.
 #include <cudaTypedefs.h>
