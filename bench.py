@@ -497,11 +497,12 @@ def main():
         graph_line = {"ms_per_step": tg, "value": tokens_step / (tg * 1e-3), "unit": UNIT}
         del graph
 
-    # end to end: pinned host inputs in, results (O and the three gradients) out, every step.
-    # Two sets of device inputs and outputs: step i copies its inputs in on an H2D stream,
-    # computes on the compute stream and copies its results out on a D2H stream, so step
-    # i+1's inputs and step i-1's results cross PCIe (full duplex) while step i computes.
-    # A set is rewritten only after the step that last used it is done with it.
+    # end to end, through the library's host-buffer entry (elsaa_step_host): pinned host
+    # inputs in, results (O and the three gradients) out, every step.  Two sets of device
+    # inputs and outputs: step i copies its inputs in on an H2D stream, computes on the compute
+    # stream and copies its results out on a D2H stream, so step i+1's inputs and step i-1's
+    # results cross PCIe (full duplex) while step i computes.  The library orders each set's
+    # reuse with the set's three events.
     e2e = None
     if not args.no_e2e:
         names = ("Q", "K", "V", "dO")
@@ -519,28 +520,15 @@ def main():
         in_ready = [torch.cuda.Event() for _ in range(2)]
         comp_done = [torch.cuda.Event() for _ in range(2)]
         out_done = [torch.cuda.Event() for _ in range(2)]
+        for e in in_ready + comp_done + out_done:     # create the events before the first wait
+            e.record(stream)
+        host_in = [host[n] for n in names] + [host_W] + ([host_R] if lsh else [])
 
         def e2e_step(i):
             j = i % 2
             d, o = dsets[j], osets[j]
-            s_in.wait_event(comp_done[j])             # step i-2 has finished reading set j
-            with torch.cuda.stream(s_in):
-                for n in names:
-                    d[n].copy_(host[n], non_blocking=True)
-                d["W"].copy_(host_W, non_blocking=True)
-                in_ready[j].record(s_in)
-            stream.wait_event(in_ready[j])
-            stream.wait_event(out_done[j])            # step i-2's results have left set j
-            if lsh:                                   # the planes live at one address, in stream order
-                R.copy_(host_R, non_blocking=True)
-            op.forward(d["Q"], d["K"], d["V"], d["W"], out=o[0], stream=stream)
-            op.backward(d["Q"], d["K"], d["V"], d["W"], d["dO"], grads=o[1:], stream=stream)
-            comp_done[j].record(stream)
-            s_out.wait_event(comp_done[j])
-            with torch.cuda.stream(s_out):
-                for hdst, dsrc in zip(outs[j], o):
-                    hdst.copy_(dsrc, non_blocking=True)
-                out_done[j].record(s_out)
+            op.step_host(host_in, outs[j], [d[n] for n in names] + [d["W"]], list(o),
+                         (in_ready[j], comp_done[j], out_done[j]), stream, s_in, s_out)
 
         for i in range(4):
             e2e_step(i)
@@ -558,6 +546,7 @@ def main():
         te = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dev)
         e2e = {"value": tokens_step / (te * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": te,
+               "api": "elsaa_step_host (pinned host buffers, two device sets)",
                "pipelined": "double-buffered: step i+1's H2D and step i-1's D2H overlap step i's compute"}
 
     if world > 1:

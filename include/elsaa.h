@@ -116,8 +116,9 @@ typedef struct {
 /* Bytes of the caller-owned `saved` buffer the forward fills and the backward
  * reads (selection, per-row denominators, the fusion weight, O_sparse, RACE
  * features and prefix summaries; with SORTLSH also the sorted orders, one pair per
- * recursion level when causal, and then also every level's gathered query, key and
- * value rows, 3 * levels * B * H * N * d * 2 bytes, which the backward reuses).  O_sparse is kept in float32 for every dtype: the
+ * recursion level when causal, and the rows the operator ran on, which the backward
+ * reuses: the sorted Q, K, V, or with the causal recursion every level's gathered
+ * query, key and value rows, 3 * levels * B * H * N * d elements).  O_sparse is kept in float32 for every dtype: the
  * backward forms the softmax delta <dO_s, O_s> from it, and a bf16 copy would put
  * the rounding of O_s into every dS of a row whose mass sits on a few keys.
  * Returns 0 when params are invalid. */
@@ -125,9 +126,8 @@ ELSAA_API size_t elsaa_saved_bytes(const elsaa_params* params);
 
 /* Bytes of scratch device memory a forward (for_backward = 0) or backward
  * (for_backward = 1) call needs.  With SORTLSH this includes the row-permuted copies
- * of the inputs and, when causal, every recursion level's gathered rows, partial
- * results and gradients at once (about 11 and 18 times Q, K and V together for a forward and a backward
- * at N = 16384, block 128).  Returns 0 when params are invalid. */
+ * of O (forward) or dO and the gradients (backward) and, when causal, every recursion
+ * level's partial results and gradients at once.  Returns 0 when params are invalid. */
 ELSAA_API size_t elsaa_workspace_bytes(const elsaa_params* params, int for_backward);
 
 /* Forward: O = g_s m O_s + g_lr O_lr for every (b, h) [Eq. 4, Eq. 5, §3.1, §3.2].
@@ -157,6 +157,32 @@ ELSAA_API elsaa_status elsaa_backward(const elsaa_params* params,
                             const void* dO, const void* saved,
                             void* dQ, void* dK, void* dV,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* One forward + backward step from pinned host memory: the end-to-end path a training
+ * loop takes when its batches live on the host.  Copies the step's inputs host -> device
+ * on `h2d_stream`, runs elsaa_forward and elsaa_backward on `stream` (default lambda and
+ * gates), and copies O, dQ, dK, dV device -> host on `d2h_stream`; everything is
+ * asynchronous and the call allocates nothing.
+ *   host_in   in   pinned host pointers {Q, K, V, dO (each [B,H,N,d] dtype), W_hash (float32
+ *                  [L, d, hash_bits]; may be NULL when rank_r = 0), sortLSH planes (float32
+ *                  [d, lsh_bits], copied into params->lsh_planes in `stream` order; NULL otherwise)}
+ *   host_out  out  pinned host pointers {O, dQ, dK, dV}, [B,H,N,d] dtype
+ *   dev_in, dev_out    one set of caller-owned device buffers of the same shapes {Q, K, V, dO,
+ *                  W_hash} and {O, dQ, dK, dV}; alternate two sets between consecutive calls so
+ *                  that one step's copies overlap the other's compute
+ *   saved, workspace   as elsaa_forward / elsaa_backward (elsaa_saved_bytes(), and the larger of
+ *                  the two elsaa_workspace_bytes() sizes), shared by every call in `stream` order
+ *   events    three caller-owned CUDA events (cudaEvent_t) of this device set: {inputs landed,
+ *                  step computed, results left}.  The input copies first wait for "step computed"
+ *                  of the set's previous use, the step for "inputs landed" and the set's previous
+ *                  "results left", the result copies for "step computed".  The caller waits on
+ *                  "results left" before reading host_out.
+ * NULL arrays, inputs or events return ELSAA_ERR_INVALID_ARG before any copy; otherwise the
+ * status of the copies, the forward and the backward. */
+ELSAA_API elsaa_status elsaa_step_host(const elsaa_params* params, const void* const* host_in,
+                                       void* const* host_out, void* const* dev_in, void* const* dev_out,
+                                       void* saved, void* workspace, size_t workspace_bytes, void* stream,
+                                       void* h2d_stream, void* d2h_stream, void* const* events);
 
 /* Per-row gradients of sum(dO * O) with respect to the fusion parameters of Eq. 5 /
  * Eq. 4 (the paper's optional learnable lambda, §1 contribution 3, and the two gates):

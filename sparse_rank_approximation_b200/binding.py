@@ -31,7 +31,7 @@ ELSAA_SEL_SORTLSH = 1
 EXPORTED = ("elsaa_saved_bytes", "elsaa_workspace_bytes", "elsaa_forward", "elsaa_backward",
             "elsaa_debug_select", "elsaa_check_device_flags", "elsaa_status_string",
             "elsaa_last_error_message", "elsaa_profile_begin", "elsaa_profile_end", "elsaa_select_noalloc",
-            "elsaa_fusion_grads", "elsaa_debug_sortlsh", "elsaa_debug_set_wait_limit")
+            "elsaa_fusion_grads", "elsaa_debug_sortlsh", "elsaa_debug_set_wait_limit", "elsaa_step_host")
 
 
 class Params(ctypes.Structure):
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
     L.elsaa_profile_end.restype = i32
     L.elsaa_select_noalloc.argtypes = [P, vp, vp, vp, vp]
     L.elsaa_select_noalloc.restype = i32
+    L.elsaa_step_host.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp, vp]
+    L.elsaa_step_host.restype = i32
     L.elsaa_fusion_grads.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.elsaa_fusion_grads.restype = i32
     L.elsaa_debug_sortlsh.argtypes = [P, vp, vp, vp, vp, vp]
@@ -117,6 +119,16 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
         return None
     if not t.is_cuda:
         raise ValueError("tensors passed to the ELSAA library must live on the GPU")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the ELSAA library must be contiguous")
+    return t.data_ptr()
+
+
+def _host_ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if t.is_cuda or not t.is_pinned():
+        raise ValueError("host buffers passed to the ELSAA library must be pinned CPU tensors")
     if not t.is_contiguous():
         raise ValueError("tensors passed to the ELSAA library must be contiguous")
     return t.data_ptr()
@@ -175,6 +187,22 @@ class Elsaa:
                                   _ptr(dV), _ptr(self.ws), self.ws.numel(), _stream(stream))
         _check(st, "elsaa_backward")
         return dQ, dK, dV
+
+    def step_host(self, host_in, host_out, dev_in, dev_out, events, stream, h2d_stream, d2h_stream):
+        """One forward + backward step from pinned host memory (``elsaa_step_host``).
+
+        host_in: pinned CPU tensors (Q, K, V, dO, W, planes or None); host_out: (O, dQ, dK, dV);
+        dev_in / dev_out: one device set of the same shapes; events: three recorded
+        ``torch.cuda.Event`` of that set (inputs landed, step computed, results left)."""
+        def arr(ts, conv):
+            return (ctypes.c_void_p * len(ts))(*[conv(t) for t in ts])
+        ins = list(host_in) + [None] * (6 - len(host_in))
+        ev = (ctypes.c_void_p * 3)(*[e.cuda_event for e in events])
+        st = lib().elsaa_step_host(ctypes.byref(self.p), arr(ins, _host_ptr), arr(host_out, _host_ptr),
+                                   arr(dev_in, _ptr), arr(dev_out, _ptr),
+                                   _ptr(self.saved), _ptr(self.ws), self.ws.numel(), stream.cuda_stream,
+                                   h2d_stream.cuda_stream, d2h_stream.cuda_stream, ev)
+        _check(st, "elsaa_step_host")
 
     def fusion_grads(self, dO, lam_vec=None, g_s=None, g_lr=None, stream=None):
         """Per-row gradients (dlambda, dg_sparse, dg_lr), float32 [B, H, N], of sum(dO * O)

@@ -960,6 +960,66 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* Q, const void* K,
   return ELSAA_OK;
 }
 
+elsaa_status elsaa_step_host(const elsaa_params* p, const void* const* host_in, void* const* host_out,
+                             void* const* dev_in, void* const* dev_out, void* saved, void* workspace,
+                             size_t ws_bytes, void* stream, void* h2d_stream, void* d2h_stream,
+                             void* const* events) {
+  g_last_error.clear();
+  Geom g;
+  elsaa_status st;
+  if (!make_geom(p, &g, &st)) return st;
+  if (!host_in || !host_out || !dev_in || !dev_out || !events)
+    return fail(ELSAA_ERR_INVALID_ARG, "host_in, host_out, dev_in, dev_out and events must not be NULL");
+  static const char* in_names[5] = {"host Q", "host K", "host V", "host dO", "host W_hash"};
+  static const char* out_names[4] = {"host O", "host dQ", "host dK", "host dV"};
+  for (int i = 0; i < 5; ++i) {
+    if (i == 4 && g.r == 0) continue;
+    if (!host_in[i]) return fail(ELSAA_ERR_INVALID_ARG, "%s is NULL", in_names[i]);
+    ELSAA_TRY(check_ptr(dev_in[i], "device input"));
+  }
+  for (int i = 0; i < 4; ++i) {
+    if (!host_out[i]) return fail(ELSAA_ERR_INVALID_ARG, "%s is NULL", out_names[i]);
+    ELSAA_TRY(check_ptr(dev_out[i], "device output"));
+  }
+  for (int i = 0; i < 3; ++i)
+    if (!events[i]) return fail(ELSAA_ERR_INVALID_ARG, "event %d is NULL", i);
+  const bool lsh = g.selector == ELSAA_SEL_SORTLSH;
+  if (lsh && (!host_in[5] || !p->lsh_planes))
+    return fail(ELSAA_ERR_INVALID_ARG, "sortLSH: host planes (host_in[5]) and params->lsh_planes are required");
+  const size_t mat = (size_t)g.BH * g.N * g.d * (p->dtype == ELSAA_DTYPE_BF16 ? 2 : 4);
+  const size_t wbytes = (size_t)g.L * g.d * kHashBits * sizeof(float);
+  cudaStream_t sc = static_cast<cudaStream_t>(stream), si = static_cast<cudaStream_t>(h2d_stream),
+               so = static_cast<cudaStream_t>(d2h_stream);
+  cudaEvent_t in_ready = static_cast<cudaEvent_t>(events[0]), computed = static_cast<cudaEvent_t>(events[1]),
+              out_done = static_cast<cudaEvent_t>(events[2]);
+  // inputs in, once this set's previous step has read them
+  ELSAA_TRY(cuda_status(cudaStreamWaitEvent(si, computed, 0), "wait for the set's previous step"));
+  for (int i = 0; i < 5; ++i) {
+    if (i == 4 && g.r == 0) continue;
+    ELSAA_TRY(cuda_status(cudaMemcpyAsync(dev_in[i], host_in[i], i == 4 ? wbytes : mat, cudaMemcpyHostToDevice, si),
+                          "input copy"));
+  }
+  ELSAA_TRY(cuda_status(cudaEventRecord(in_ready, si), "inputs landed"));
+  // the step, once its inputs have landed and the set's previous results have left
+  ELSAA_TRY(cuda_status(cudaStreamWaitEvent(sc, in_ready, 0), "wait for the inputs"));
+  ELSAA_TRY(cuda_status(cudaStreamWaitEvent(sc, out_done, 0), "wait for the previous results"));
+  if (lsh)      // the planes live at one address: copied in stream order with the steps that read them
+    ELSAA_TRY(cuda_status(cudaMemcpyAsync(const_cast<float*>(p->lsh_planes), host_in[5],
+                                          (size_t)g.d * p->lsh_bits * sizeof(float), cudaMemcpyHostToDevice, sc),
+                          "planes copy"));
+  const float* W = g.r > 0 ? static_cast<const float*>(dev_in[4]) : nullptr;
+  ELSAA_TRY(elsaa_forward(p, dev_in[0], dev_in[1], dev_in[2], W, nullptr, nullptr, nullptr, dev_out[0], saved,
+                          workspace, ws_bytes, stream));
+  ELSAA_TRY(elsaa_backward(p, dev_in[0], dev_in[1], dev_in[2], W, nullptr, nullptr, nullptr, dev_in[3], saved,
+                           dev_out[1], dev_out[2], dev_out[3], workspace, ws_bytes, stream));
+  ELSAA_TRY(cuda_status(cudaEventRecord(computed, sc), "step computed"));
+  // results out
+  ELSAA_TRY(cuda_status(cudaStreamWaitEvent(so, computed, 0), "wait for the step"));
+  for (int i = 0; i < 4; ++i)
+    ELSAA_TRY(cuda_status(cudaMemcpyAsync(host_out[i], dev_out[i], mat, cudaMemcpyDeviceToHost, so), "result copy"));
+  return cuda_status(cudaEventRecord(out_done, so), "results left");
+}
+
 elsaa_status elsaa_fusion_grads(const elsaa_params* p, const float* lam, const float* gs, const float* glr,
                                 const void* dO, const void* saved, float* dlam, float* dgs, float* dglr,
                                 void* stream) {

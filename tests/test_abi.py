@@ -130,3 +130,28 @@ def test_sortlsh_saved_buffer_holds_the_gathered_rows():
         grown = L.elsaa_saved_bytes(ctypes.byref(p)) - L.elsaa_saved_bytes(ctypes.byref(q))
         assert grown >= rows + orders, (causal, grown, rows, orders)
         assert grown <= rows + orders + 4096, (causal, grown, rows, orders)
+
+
+def test_step_host_argument_errors_return_before_any_copy():
+    """The host-buffer step entry checks its arrays, inputs and events before it copies."""
+    L = bd.lib()
+    p = bd.make_params(1, 2, 1024, 64, rank_r=64, block_size=64, topk=4)
+    arr = lambda *xs: (ctypes.c_void_p * len(xs))(*xs)
+    hin, hout = arr(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None), arr(0x1000, 0x1000, 0x1000, 0x1000)
+    din, dout = arr(0x1000, 0x1000, 0x1000, 0x1000, 0x1000), arr(0x1000, 0x1000, 0x1000, 0x1000)
+    ev = arr(0x1000, 0x1000, 0x1000)
+    call = lambda *a: L.elsaa_step_host(ctypes.byref(p), *a, 0x1000, 0x1000, 1 << 40, None, None, None, ev)
+    assert call(None, hout, din, dout) == bd.ELSAA_ERR_INVALID_ARG
+    assert call(hin, hout, din, None) == bd.ELSAA_ERR_INVALID_ARG
+    assert call(arr(0x1000, None, 0x1000, 0x1000, 0x1000, None), hout, din, dout) == bd.ELSAA_ERR_INVALID_ARG
+    assert b"host K" in L.elsaa_last_error_message()
+    assert call(hin, arr(0x1000, 0x1000, None, 0x1000), din, dout) == bd.ELSAA_ERR_INVALID_ARG
+    assert b"host dK" in L.elsaa_last_error_message()
+    assert call(hin, hout, arr(0x1000, 0x1008, 0x1000, 0x1000, 0x1000), dout) == bd.ELSAA_ERR_INVALID_ARG
+    assert b"aligned" in L.elsaa_last_error_message()
+    assert L.elsaa_step_host(ctypes.byref(p), hin, hout, din, dout, 0x1000, 0x1000, 1 << 40, None, None, None,
+                             arr(0x1000, None, 0x1000)) == bd.ELSAA_ERR_INVALID_ARG
+    lsh = bd.make_params(1, 2, 1024, 64, rank_r=64, block_size=64, topk=1, selector=bd.ELSAA_SEL_SORTLSH, lsh_bits=4)
+    assert L.elsaa_step_host(ctypes.byref(lsh), hin, hout, din, dout, 0x1000, 0x1000, 1 << 40, None, None, None,
+                             ev) == bd.ELSAA_ERR_INVALID_ARG
+    assert b"planes" in L.elsaa_last_error_message()
