@@ -87,8 +87,9 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const double* __restr
   }
 }
 
-// One warp per tile row: pick the best `need` candidates by (score desc, index asc)
-// with repeated warp arg-max, then emit the set in ascending order.
+// One warp per tile row: the row's scores are read once into registers (lane l holds blocks
+// l, l + 32, ..., n_t <= 1024), the best `need` candidates by (score desc, index asc) come out
+// of repeated warp arg-max passes over them, and the set is emitted in ascending order.
 // grid (ceil(n_t/8), BH), block 256.
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ scores, int* __restrict__ idx,
                                                    Geom g) {
@@ -109,16 +110,27 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
   if (need >= n_cand) {
     for (int b = lane; b < n_cand; b += 32) atomicOr(&sel[warp][b >> 5], 1u << (b & 31));
   } else {
+    const int nj = (n_cand + 31) >> 5;          // register slots in use (warp-uniform)
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (j >= nj) break;
+      const int b = lane + 32 * j;
+      v[j] = b < n_cand ? row[b] : 0.f;
+    }
     float last_s = __int_as_float(0x7f800000);   // +inf: everything ranks below
     int last_b = -1;
     for (int it = 0; it < need; ++it) {
       float bs = -__int_as_float(0x7f800000);
       int bb = 0x7fffffff;
-      for (int b = lane; b < n_cand; b += 32) {
-        const float s = row[b];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j >= nj) break;
+        const int b = lane + 32 * j;
+        const float s = v[j];
         const bool below = (s < last_s) || (s == last_s && b > last_b);
         const bool better = (s > bs) || (s == bs && b < bb);
-        if (below && better) { bs = s; bb = b; }
+        if (b < n_cand && below && better) { bs = s; bb = b; }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
